@@ -1,0 +1,241 @@
+"""fp64 CPU oracle of the Multi-Token Attention (MTA) forward pass.
+
+TEST INFRASTRUCTURE ONLY.  Imported by tests/, by __graft_entry__.smoke() and by
+the CPU-baseline leg of bench.py; the library (token_attention_b200) never
+imports, links or runs anything here, and nothing here imports the library.
+
+It is the plain definition written out: the full L x L logit, convolution and
+attention maps are materialised per head group in float64 and every step is a
+separate array operation, in the order the pages give it.  Sources (page title,
+section):
+
+  [MTA-2]   "Multi-Token Attention | Summary" (greeksharifa), section 2
+            "Background on multi-head attention": per-head Q, K, V; logits
+            A_hat = Q K^T / sqrt(d); causal -inf mask; softmax over keys; A V;
+            concatenation; output projection.
+  [MTA-3.1] same page, section 3.1 "Key-query convolution":
+            A = Softmax(Mask_-inf(Conv2d_theta(Mask_0(A_hat)))), a separate 2-D
+            kernel per head over (query, key) offsets, using only the current and
+            previous queries.
+  [MTA-3.2] same page, section 3.2 "Head mixing convolution": heads split into
+            M/c_h groups; A1_new = w11 A1 + w12 A2, ...; applied to logits
+            (before softmax) or to attention weights (after softmax).
+  [MTA-3.3] same page, section 3.3 "Putting everything together": both on the
+            same side of the softmax = one 3-D convolution; group normalisation
+            of head outputs before concatenation, with a scale.
+  [MTA-B]   same page, appendix B "MTA Architecture": post-softmax mixing acts
+            through the value/output projections.
+  [bycloud] "Multi-Token Attention" (bycloud), "Understanding Multi-Token
+            Attention (MTA) Mechanism", item 3: group normalisation with depth
+            scaling.
+
+Readings where the pages leave a step open (all listed in the design doc):
+  * Mask_0 zeroes logits of future keys (key j > query i) before the
+    convolution; indices outside [0, L) contribute 0 (zero padding).
+  * theta[h][a][t] multiplies Mask_0(A_hat)[i - a][j - (t - c_k//2)]:
+    a = 0..c_q-1 steps back over queries, t over keys centred on j.  No bias.
+  * Pre-softmax head mixing is applied after the key-query convolution.
+  * Post-softmax mixing is a plain linear combination (no renormalisation) and
+    the mixed map of head r multiplies head r's own values.
+  * Group norm: per (token, head) over the d channels, biased variance,
+    eps, affine gamma/beta of length D; then times lambda.
+"""
+from __future__ import annotations
+
+import numpy as np
+
+OFF, PRE, POST = 0, 1, 2
+
+__all__ = ["OFF", "PRE", "POST", "attention_logits", "mask_zero", "key_query_conv",
+           "head_mix", "mask_neg_inf", "softmax_rows", "mta_attention_group",
+           "mta_attention", "mta_attention_rows", "group_norm_scale", "mta_layer",
+           "mta_layer_rows"]
+
+
+# ----------------------------------------------------------------------------
+# the steps, each on arrays of one head group: [c_h, rows, keys]
+# ----------------------------------------------------------------------------
+
+def attention_logits(q_rows: np.ndarray, k: np.ndarray, scale: float) -> np.ndarray:
+    """A_hat[h, r, j] = scale * q[h, r] . k[h, j]   [MTA-2].
+
+    q_rows [c_h, R, d], k [c_h, L, d] -> [c_h, R, L] float64."""
+    return scale * np.matmul(q_rows.astype(np.float64), k.astype(np.float64).transpose(0, 2, 1))
+
+
+def _future(qpos: np.ndarray, L: int) -> np.ndarray:
+    """Boolean [R, L]: True where key j lies in the future of query qpos[r]."""
+    return np.arange(L)[None, :] > qpos[:, None]
+
+
+def mask_zero(a: np.ndarray, qpos: np.ndarray) -> np.ndarray:
+    """Mask_0: entries with key j > query position qpos[r] become 0  [MTA-3.1]."""
+    return np.where(_future(qpos, a.shape[-1])[None], 0.0, a)
+
+
+def key_query_conv(m: np.ndarray, theta: np.ndarray) -> np.ndarray:
+    """Conv2d_theta over (query, key) per head  [MTA-3.1].
+
+    m [c_h, R, L]: rows are consecutive queries (row r-1 is the query before
+    row r); rows before the first and keys outside [0, L) count as 0.
+    theta [c_h, c_q, c_k].
+    out[h, r, j] = sum_a sum_t theta[h, a, t] * m[h, r - a, j - (t - c_k//2)].
+    """
+    ch, R, L = m.shape
+    cq, ck = theta.shape[1], theta.shape[2]
+    c = ck // 2
+    out = np.zeros_like(m, dtype=np.float64)
+    for a in range(cq):                       # a queries back
+        if a >= R:
+            break
+        for t in range(ck):
+            b = t - c                          # key offset: reads key j - b
+            j_lo, j_hi = max(0, b), min(L, L + b)
+            if j_lo >= j_hi:
+                continue
+            coef = theta[:, a, t].astype(np.float64)[:, None, None]
+            out[:, a:, j_lo:j_hi] += coef * m[:, :R - a, j_lo - b:j_hi - b]
+    return out
+
+
+def head_mix(a: np.ndarray, w: np.ndarray) -> np.ndarray:
+    """Within-group linear combination: out[r] = sum_s w[r, s] * a[s]  [MTA-3.2]."""
+    return np.einsum("rs,s...->r...", w.astype(np.float64), a)
+
+
+def mask_neg_inf(c: np.ndarray, qpos: np.ndarray) -> np.ndarray:
+    """Mask_-inf: entries with key j > query qpos[r] become -inf  [MTA-2, MTA-3.1]."""
+    return np.where(_future(qpos, c.shape[-1])[None], -np.inf, c)
+
+
+def softmax_rows(c: np.ndarray) -> np.ndarray:
+    """Softmax over keys (last axis)  [MTA-2]."""
+    mx = np.max(c, axis=-1, keepdims=True)
+    e = np.exp(c - mx)
+    return e / np.sum(e, axis=-1, keepdims=True)
+
+
+def mta_attention_group(q_rows, k, v, theta, w, qpos, scale, kq_place, head_place):
+    """MTA attention of one head group for the query rows `qpos` (consecutive).
+
+    q_rows [c_h, R, d] (queries at positions qpos), k, v [c_h, L, d],
+    theta [c_h, c_q, c_k], w [c_h, c_h].  Returns [c_h, R, d] float64.
+    Steps in the pages' order [MTA-2, MTA-3.1, MTA-3.2, MTA-3.3]."""
+    qpos = np.asarray(qpos)
+    a_hat = attention_logits(q_rows, k, scale)
+    if kq_place == PRE:
+        c = key_query_conv(mask_zero(a_hat, qpos), theta)
+    else:
+        c = a_hat
+    if head_place == PRE:
+        c = head_mix(c, w)
+    attn = softmax_rows(mask_neg_inf(c, qpos))
+    if head_place == POST:
+        attn = head_mix(attn, w)
+    return np.matmul(attn, v.astype(np.float64))        # head r: A_r V_r
+
+
+# ----------------------------------------------------------------------------
+# whole tensors in the library's layout: q, k, v, out [B][L][H][d]
+# ----------------------------------------------------------------------------
+
+def _group(x: np.ndarray, b: int, g: int, ch: int) -> np.ndarray:
+    """[L, H, d] slice of batch b -> heads of group g as [c_h, L, d]."""
+    return np.ascontiguousarray(x[b, :, g * ch:(g + 1) * ch, :].transpose(1, 0, 2))
+
+
+def _default_scale(d: int, scale) -> float:
+    return 1.0 / np.sqrt(d) if not scale else float(scale)
+
+
+def mta_attention(q, k, v, theta, w, c_h, kq_place=PRE, head_place=POST, scale=None):
+    """Full MTA attention.  q, k, v [B][L][H][d]; theta [H][c_q][c_k];
+    w [H/c_h][c_h][c_h].  Returns out [B][L][H][d] float64."""
+    B, L, H, d = q.shape
+    s = _default_scale(d, scale)
+    out = np.zeros((B, L, H, d), np.float64)
+    qpos = np.arange(L)
+    for b in range(B):
+        for g in range(H // c_h):
+            hs = slice(g * c_h, (g + 1) * c_h)
+            og = mta_attention_group(_group(q, b, g, c_h), _group(k, b, g, c_h),
+                                     _group(v, b, g, c_h), theta[hs], w[g], qpos, s,
+                                     kq_place, head_place)
+            out[b, :, hs, :] = og.transpose(1, 0, 2)
+    return out
+
+
+def mta_attention_rows(q, k, v, theta, w, c_h, rows, kq_place=PRE, head_place=POST,
+                       scale=None):
+    """MTA attention output at selected tokens only.
+
+    rows: sequence of (b, i).  Returns [n, H, d] float64.  Each row is computed
+    from the window of the c_q queries ending at i (the only rows the
+    convolution reads), with exactly the same steps as mta_attention."""
+    B, L, H, d = q.shape
+    cq = theta.shape[1]
+    s = _default_scale(d, scale)
+    out = np.zeros((len(rows), H, d), np.float64)
+    for n, (b, i) in enumerate(rows):
+        lo = max(0, i - cq + 1)
+        qpos = np.arange(lo, i + 1)
+        for g in range(H // c_h):
+            hs = slice(g * c_h, (g + 1) * c_h)
+            qg = np.ascontiguousarray(q[b, lo:i + 1, hs, :].transpose(1, 0, 2))
+            og = mta_attention_group(qg, _group(k, b, g, c_h), _group(v, b, g, c_h),
+                                     theta[hs], w[g], qpos, s, kq_place, head_place)
+            out[n, hs, :] = og[:, -1, :]
+    return out
+
+
+def group_norm_scale(o, gamma, beta, eps, lam):
+    """Per-(token, head) normalisation over d, affine, then depth scale
+    [MTA-3.3, bycloud].  o [..., H, d]; gamma, beta [H*d].  Returns float64."""
+    o = o.astype(np.float64)
+    H, d = o.shape[-2], o.shape[-1]
+    mu = np.mean(o, axis=-1, keepdims=True)
+    var = np.mean((o - mu) ** 2, axis=-1, keepdims=True)
+    y = (o - mu) / np.sqrt(var + eps)
+    y = y * gamma.astype(np.float64).reshape(H, d) + beta.astype(np.float64).reshape(H, d)
+    return lam * y
+
+
+def _split_qkv(qkv, H, d):
+    D = H * d
+    shp = qkv.shape[:-1] + (H, d)
+    return (qkv[..., :D].reshape(shp), qkv[..., D:2 * D].reshape(shp),
+            qkv[..., 2 * D:].reshape(shp))
+
+
+def mta_layer(x, wqkv, theta, w, gamma, beta, eps, lam, wo, H, c_h,
+              kq_place=PRE, head_place=POST):
+    """Full MTA attention layer  [MTA-2, MTA-3.x, bycloud].
+    x [B][L][D]; wqkv [3D][D]; wo [D][D].  Returns out [B][L][D] float64."""
+    B, L, D = x.shape
+    d = D // H
+    qkv = np.matmul(x.astype(np.float64), wqkv.astype(np.float64).T)      # x W^T
+    q, k, v = _split_qkv(qkv, H, d)
+    o = mta_attention(q, k, v, theta, w, c_h, kq_place, head_place)
+    y = group_norm_scale(o, gamma, beta, eps, lam).reshape(B, L, D)
+    return np.matmul(y, wo.astype(np.float64).T)
+
+
+def mta_layer_rows(x, wqkv, theta, w, gamma, beta, eps, lam, wo, H, c_h, rows,
+                   kq_place=PRE, head_place=POST):
+    """mta_layer at selected tokens (b, i) only: K, V of the token's batch in
+    full, queries of the convolution window.  Returns [n, D] float64."""
+    B, L, D = x.shape
+    d = D // H
+    wq = wqkv.astype(np.float64)
+    out = np.zeros((len(rows), D), np.float64)
+    cache = {}
+    for n, (b, i) in enumerate(rows):
+        if b not in cache:
+            qkv_b = np.matmul(x[b].astype(np.float64), wq.T)              # [L, 3D]
+            cache = {b: _split_qkv(qkv_b, H, d)}
+        q, k, v = cache[b]
+        o = mta_attention_rows(q[None], k[None], v[None], theta, w, c_h, [(0, i)],
+                               kq_place, head_place)[0]                     # [H, d]
+        y = group_norm_scale(o, gamma, beta, eps, lam).reshape(D)
+        out[n] = y @ wo.astype(np.float64).T
+    return out

@@ -1,0 +1,333 @@
+"""Pins of the fp64 oracle to facts other than itself.
+
+Each test checks the oracle against a library routine, a closed form, an
+invariant stated or implied by the pages, or a brute-force restatement on tiny
+inputs, chosen so that a dropped term, a wrong sign or index or a transposed
+operand anywhere in the oracle fails at least one of them.  Sources:
+"Multi-Token Attention | Summary" (greeksharifa), sections 2, 3.1, 3.2, 3.3,
+4.6 (identity initialisation) and appendix B.
+"""
+import itertools
+
+import numpy as np
+import pytest
+import scipy.signal
+import scipy.special
+import torch
+
+import oracle as O
+
+
+def rand(shape, seed, std=1.0):
+    return np.random.default_rng(seed).standard_normal(shape) * std
+
+
+def sdpa(q, k, v, scale):
+    """Causal softmax attention by torch's library routine, fp64.  q,k,v [H,L,d]."""
+    t = lambda x: torch.from_numpy(np.ascontiguousarray(x, dtype=np.float64))
+    return torch.nn.functional.scaled_dot_product_attention(
+        t(q)[None], t(k)[None], t(v)[None], is_causal=True, scale=scale)[0].numpy()
+
+
+def to_bhld(x):  # [B,L,H,d] -> [B,H,L,d]
+    return np.ascontiguousarray(x.transpose(0, 2, 1, 3))
+
+
+def delta_theta(H, cq, ck, a, t, tau=1.0):
+    th = np.zeros((H, cq, ck))
+    th[:, a, t] = tau
+    return th
+
+
+SHAPE = dict(B=2, L=23, H=4, d=8)
+
+
+@pytest.fixture(scope="module")
+def qkv():
+    B, L, H, d = SHAPE["B"], SHAPE["L"], SHAPE["H"], SHAPE["d"]
+    return rand((B, L, H, d), 1), rand((B, L, H, d), 2), rand((B, L, H, d), 3)
+
+
+@pytest.mark.parametrize("head_place", [O.OFF, O.PRE, O.POST])
+def test_identity_kernels_equal_causal_sdpa(qkv, head_place):
+    """theta = delta at (0,0), w = I reduces MTA to standard causal multi-head
+    attention (identity initialisation keeps the pretrained map, section 4.6)."""
+    q, k, v = qkv
+    B, L, H, d = q.shape
+    cq, ck, ch = 3, 5, 2
+    th = delta_theta(H, cq, ck, 0, ck // 2)
+    w = np.tile(np.eye(ch), (H // ch, 1, 1))
+    out = O.mta_attention(q, k, v, th, w, ch, O.PRE, head_place)
+    ref = sdpa(to_bhld(q).reshape(B * H, L, d), to_bhld(k).reshape(B * H, L, d),
+               to_bhld(v).reshape(B * H, L, d), 1 / np.sqrt(d))
+    np.testing.assert_allclose(to_bhld(out).reshape(B * H, L, d), ref, rtol=0, atol=1e-12)
+
+
+def _closed_form_attention(q, k, v, logit_fn, scale):
+    """Brute force on one head: logits from a closed form, -inf on future keys,
+    softmax by scipy, times V.  q,k,v [L,d]."""
+    L = q.shape[0]
+    lg = np.full((L, L), -np.inf)
+    for i in range(L):
+        for j in range(i + 1):
+            lg[i, j] = logit_fn(i, j)
+    return scipy.special.softmax(lg, axis=1) @ v
+
+
+@pytest.mark.parametrize("a", [1, 2])
+def test_query_shift_delta_closed_form(qkv, a):
+    """theta = delta at (a, 0): C[i,j] = s q[i-a].k[j] if j <= i-a, and 0 for
+    i-a < j <= i (Mask_0 zeroes the future of the shifted query), section 3.1."""
+    q, k, v = qkv
+    B, L, H, d = q.shape
+    cq, ck = 3, 5
+    s = 1 / np.sqrt(d)
+    th = delta_theta(H, cq, ck, a, ck // 2)
+    out = O.mta_attention(q, k, v, th, np.tile(np.eye(1), (H, 1, 1)), 1, O.PRE, O.OFF)
+    for b, h in [(0, 0), (1, 3)]:
+        qq, kk, vv = q[b, :, h], k[b, :, h], v[b, :, h]
+        fn = lambda i, j: s * qq[i - a] @ kk[j] if (i - a >= 0 and j <= i - a) else 0.0
+        np.testing.assert_allclose(out[b, :, h], _closed_form_attention(qq, kk, vv, fn, s),
+                                   rtol=0, atol=1e-12)
+
+
+@pytest.mark.parametrize("boff", [-2, -1, 1, 2])
+def test_key_shift_delta_closed_form(qkv, boff):
+    """theta = delta at (0, b): C[i,j] = s q[i].k[j-b] when 0 <= j-b <= i, else 0
+    inside the causal region (pins the key orientation), section 3.1."""
+    q, k, v = qkv
+    B, L, H, d = q.shape
+    cq, ck = 2, 5
+    s = 1 / np.sqrt(d)
+    th = delta_theta(H, cq, ck, 0, ck // 2 + boff)
+    out = O.mta_attention(q, k, v, th, np.tile(np.eye(1), (H, 1, 1)), 1, O.PRE, O.OFF)
+    for b, h in [(0, 1), (1, 2)]:
+        qq, kk, vv = q[b, :, h], k[b, :, h], v[b, :, h]
+        fn = lambda i, j: s * qq[i] @ kk[j - boff] if 0 <= j - boff <= i else 0.0
+        np.testing.assert_allclose(out[b, :, h], _closed_form_attention(qq, kk, vv, fn, s),
+                                   rtol=0, atol=1e-12)
+
+
+def test_scaled_delta_is_temperature(qkv):
+    """theta = tau * delta(0,0) gives softmax(tau s Q K^T) V (library SDPA with
+    scale tau*s)."""
+    q, k, v = qkv
+    B, L, H, d = q.shape
+    tau = 1.7
+    th = delta_theta(H, 3, 5, 0, 2, tau)
+    out = O.mta_attention(q, k, v, th, np.ones((H, 1, 1)), 1, O.PRE, O.OFF)
+    ref = sdpa(to_bhld(q).reshape(B * H, L, d), to_bhld(k).reshape(B * H, L, d),
+               to_bhld(v).reshape(B * H, L, d), tau / np.sqrt(d))
+    np.testing.assert_allclose(to_bhld(out).reshape(B * H, L, d), ref, rtol=0, atol=1e-12)
+
+
+@pytest.mark.parametrize("head_place", [O.PRE, O.POST])
+def test_causality_bit_exact(qkv, head_place):
+    """Only current and past queries and keys matter (section 3.1, causal mask of
+    section 2): perturbing position t leaves outputs at i < t bit-identical."""
+    q, k, v = qkv
+    H = q.shape[2]
+    th = rand((H, 3, 5), 5, 0.3)
+    w = rand((H // 2, 2, 2), 6, 0.5)
+    base = O.mta_attention(q, k, v, th, w, 2, O.PRE, head_place)
+    t = 14
+    q2, k2, v2 = q.copy(), k.copy(), v.copy()
+    q2[:, t:] += rand(q2[:, t:].shape, 7)
+    k2[:, t:] += rand(k2[:, t:].shape, 8)
+    v2[:, t:] += rand(v2[:, t:].shape, 9)
+    pert = O.mta_attention(q2, k2, v2, th, w, 2, O.PRE, head_place)
+    assert np.array_equal(base[:, :t], pert[:, :t])
+    assert not np.allclose(base[:, t:], pert[:, t:])
+
+
+def test_rows_sum_to_one_and_post_mix_row_sums(qkv):
+    """Softmax rows sum to 1 (section 2); post-softmax mixing is a plain linear
+    combination, so with V = 1 the output of head r is sum_s w[r,s] (section 3.2)."""
+    q, k, _ = qkv
+    B, L, H, d = q.shape
+    ones = np.ones_like(q)
+    th = rand((H, 3, 5), 11, 0.3)
+    out = O.mta_attention(q, k, ones, th, np.ones((H, 1, 1)), 1, O.PRE, O.OFF)
+    np.testing.assert_allclose(out, 1.0, rtol=0, atol=1e-12)
+    w = rand((H // 2, 2, 2), 12)
+    out = O.mta_attention(q, k, ones, th, w, 2, O.PRE, O.POST)
+    rs = w.sum(axis=2).reshape(H)               # head g*2+r -> sum_s w[g,r,s]
+    np.testing.assert_allclose(out, np.broadcast_to(rs[None, None, :, None], out.shape),
+                               rtol=0, atol=1e-12)
+
+
+def test_post_mix_is_linear_in_w(qkv):
+    q, k, v = qkv
+    H = q.shape[2]
+    th = rand((H, 3, 5), 13, 0.3)
+    w1, w2 = rand((H // 2, 2, 2), 14), rand((H // 2, 2, 2), 15)
+    f = lambda w: O.mta_attention(q, k, v, th, w, 2, O.PRE, O.POST)
+    np.testing.assert_allclose(f(w1 + w2), f(w1) + f(w2), rtol=0, atol=1e-12)
+    np.testing.assert_allclose(f(-2.5 * w1), -2.5 * f(w1), rtol=0, atol=1e-12)
+
+
+def test_appendix_b_destination_values(qkv):
+    """Appendix B: post-softmax mixing acts through the value projection, i.e.
+    O^h = sum_h' w[h,h'] softmax-attention(Q^h', K^h', V^h).  With identity
+    theta every term is the library's causal SDPA."""
+    q, k, v = qkv
+    B, L, H, d = q.shape
+    ch = 2
+    w = rand((H // ch, ch, ch), 16)
+    th = delta_theta(H, 3, 5, 0, 2)
+    out = O.mta_attention(q, k, v, th, w, ch, O.PRE, O.POST)
+    s = 1 / np.sqrt(d)
+    for b in range(B):
+        for h in range(H):
+            g, r = divmod(h, ch)
+            ref = sum(w[g, r, sp] * sdpa(q[b, :, g * ch + sp][None], k[b, :, g * ch + sp][None],
+                                         v[b, :, h][None], s)[0] for sp in range(ch))
+            np.testing.assert_allclose(out[b, :, h], ref, rtol=0, atol=1e-12)
+
+
+def test_first_row(qkv):
+    """Query 0 sees only key 0: A[0,0] = 1, so O_0 = (sum_s w[r,s]) v_0 after a
+    post mix and O_0 = v_0 without mixing or with a pre-softmax mix."""
+    q, k, v = qkv
+    B, L, H, d = q.shape
+    th = rand((H, 3, 5), 17, 0.4)
+    w = rand((H // 2, 2, 2), 18)
+    out = O.mta_attention(q, k, v, th, w, 2, O.PRE, O.POST)
+    rs = w.sum(axis=2).reshape(H)
+    np.testing.assert_allclose(out[:, 0], rs[None, :, None] * v[:, 0], rtol=0, atol=1e-12)
+    out = O.mta_attention(q, k, v, th, w, 2, O.PRE, O.PRE)
+    np.testing.assert_allclose(out[:, 0], v[:, 0], rtol=0, atol=1e-12)
+
+
+def test_conv_matches_scipy_convolve2d():
+    """Conv2d_theta over (query, key) is a zero-padded 2-D convolution: scipy's
+    'full' convolve2d of the masked map with theta, shifted by c_k//2 keys."""
+    ch, L, cq, ck = 2, 19, 4, 7
+    m = rand((ch, L, L), 21)
+    th = rand((ch, cq, ck), 22)
+    out = O.key_query_conv(m, th)
+    for h in range(ch):
+        full = scipy.signal.convolve2d(m[h], th[h], mode="full")   # [L+cq-1, L+ck-1]
+        ref = full[:L, ck // 2: ck // 2 + L]
+        np.testing.assert_allclose(out[h], ref, rtol=0, atol=1e-12)
+
+
+def test_pipeline_matches_scipy_restatement(qkv):
+    """Whole attention with random theta and w (pre and post mixing), restated
+    with library pieces: logits by einsum, Mask_0 by np.tril, the convolution by
+    scipy.signal.convolve2d, softmax by scipy.special.softmax."""
+    q, k, v = qkv
+    B, L, H, d = q.shape
+    cq, ck, ch = 3, 5, 2
+    th = rand((H, cq, ck), 23, 0.5)
+    w = rand((H // ch, ch, ch), 24)
+    s = 1 / np.sqrt(d)
+    causal = np.tril(np.ones((L, L), bool))
+    for head_place in (O.PRE, O.POST):
+        out = O.mta_attention(q, k, v, th, w, ch, O.PRE, head_place)
+        for b in range(B):
+            lg = s * np.einsum("lhd,mhd->hlm", q[b], k[b])
+            conv = np.stack([scipy.signal.convolve2d(np.tril(lg[h]), th[h], mode="full")
+                             [:L, ck // 2: ck // 2 + L] for h in range(H)])
+            conv = conv.reshape(H // ch, ch, L, L)
+            if head_place == O.PRE:
+                conv = np.einsum("grs,gslm->grlm", w, conv)
+            p = scipy.special.softmax(np.where(causal, conv, -np.inf), axis=-1)
+            if head_place == O.POST:
+                p = np.einsum("grs,gslm->grlm", w, p)
+            ref = np.einsum("hlm,mhd->lhd", p.reshape(H, L, L), v[b])
+            np.testing.assert_allclose(out[b], ref, rtol=0, atol=1e-12)
+
+
+def test_pre_mix_as_3d_convolution_bruteforce():
+    """Section 3.3: key-query and head mixing on the same side of the softmax form
+    one 3-D convolution over (head, query, key).  Pure-Python loops on a tiny
+    case with theta3[h][h'][a][t] = w[h,h'] theta[h'][a][t]."""
+    B, L, H, d, cq, ck, ch = 1, 7, 2, 3, 2, 3, 2
+    q, k, v = rand((B, L, H, d), 31), rand((B, L, H, d), 32), rand((B, L, H, d), 33)
+    th = rand((H, cq, ck), 34)
+    w = rand((1, ch, ch), 35)
+    out = O.mta_attention(q, k, v, th, w, ch, O.PRE, O.PRE)
+    s = 1 / np.sqrt(d)
+    c = ck // 2
+
+    def m0(h, i, j):
+        if i < 0 or j < 0 or j >= L or j > i:
+            return 0.0
+        return s * sum(q[0, i, h, x] * k[0, j, h, x] for x in range(d))
+
+    for h in range(H):
+        for i in range(L):
+            row = []
+            for j in range(i + 1):
+                acc = 0.0
+                for hp, a, t in itertools.product(range(ch), range(cq), range(ck)):
+                    acc += w[0, h, hp] * th[hp, a, t] * m0(hp, i - a, j - (t - c))
+                row.append(acc)
+            mx = max(row)
+            e = [np.exp(x - mx) for x in row]
+            z = sum(e)
+            ref = [sum(e[j] / z * v[0, j, h, x] for j in range(i + 1)) for x in range(d)]
+            np.testing.assert_allclose(out[0, i, h], ref, rtol=0, atol=1e-12)
+
+
+def test_group_norm_matches_torch():
+    """Per-(token, head) group normalisation = torch group_norm with H groups over
+    the D = H*d channels, affine gamma/beta, then the depth scale."""
+    T, H, d = 9, 4, 6
+    o = rand((T, H, d), 41, 3.0) + 2.0
+    gamma, beta = 1 + rand((H * d,), 42, 0.1), rand((H * d,), 43, 0.1)
+    lam, eps = 0.97814, 1e-5
+    y = O.group_norm_scale(o, gamma, beta, eps, lam).reshape(T, H * d)
+    ref = torch.nn.functional.group_norm(torch.from_numpy(o.reshape(T, H * d)), H,
+                                         torch.from_numpy(gamma), torch.from_numpy(beta),
+                                         eps).numpy() * lam
+    np.testing.assert_allclose(y, ref, rtol=0, atol=1e-12)
+
+
+def test_group_norm_invariants():
+    T, H, d = 5, 3, 16
+    o = rand((T, H, d), 44, 2.0)
+    eps = 1e-5
+    y = O.group_norm_scale(o, np.ones(H * d), np.zeros(H * d), eps, 1.0)
+    np.testing.assert_allclose(y.mean(-1), 0.0, atol=1e-12)
+    var = o.var(-1)
+    np.testing.assert_allclose(y.var(-1), var / (var + eps), rtol=1e-12)
+
+
+def test_rows_match_full(qkv):
+    q, k, v = qkv
+    H = q.shape[2]
+    th = rand((H, 3, 5), 51, 0.3)
+    w = rand((H // 2, 2, 2), 52)
+    rows = [(0, 0), (0, 1), (1, 2), (1, 7), (0, 22)]
+    for hp in (O.PRE, O.POST, O.OFF):
+        full = O.mta_attention(q, k, v, th, w, 2, O.PRE, hp)
+        part = O.mta_attention_rows(q, k, v, th, w, 2, rows, O.PRE, hp)
+        for n, (b, i) in enumerate(rows):
+            np.testing.assert_allclose(part[n], full[b, i], rtol=0, atol=1e-12)
+
+
+def test_layer_matches_library_pipeline():
+    """Layer: x W_qkv^T -> MTA attention -> torch group_norm * lambda -> Y W_o^T
+    (section 2: projections and output projection; section 3.3: group norm)."""
+    B, L, H, d, ch = 2, 11, 4, 4, 2
+    D = H * d
+    x = rand((B, L, D), 61)
+    wqkv, wo = rand((3 * D, D), 62, 0.3), rand((D, D), 63, 0.3)
+    th, w = rand((H, 3, 5), 64, 0.3), rand((H // ch, ch, ch), 65)
+    gamma, beta = 1 + rand((D,), 66, 0.1), rand((D,), 67, 0.1)
+    lam, eps = 0.9, 1e-5
+    out = O.mta_layer(x, wqkv, th, w, gamma, beta, eps, lam, wo, H, ch, O.PRE, O.POST)
+    qkv = np.einsum("bld,ed->ble", x, wqkv)
+    q, k, v = (qkv[..., i * D:(i + 1) * D].reshape(B, L, H, d) for i in range(3))
+    att = O.mta_attention(q, k, v, th, w, ch, O.PRE, O.POST).reshape(B * L, D)
+    y = torch.nn.functional.group_norm(torch.from_numpy(att), H, torch.from_numpy(gamma),
+                                       torch.from_numpy(beta), eps).numpy() * lam
+    ref = (y @ wo.T).reshape(B, L, D)
+    np.testing.assert_allclose(out, ref, rtol=0, atol=1e-11)
+    rows = [(0, 0), (1, 5), (1, 10)]
+    part = O.mta_layer_rows(x, wqkv, th, w, gamma, beta, eps, lam, wo, H, ch, rows,
+                            O.PRE, O.POST)
+    for n, (b, i) in enumerate(rows):
+        np.testing.assert_allclose(part[n], out[b, i], rtol=0, atol=1e-11)
