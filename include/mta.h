@@ -1,0 +1,160 @@
+/*
+ * mta.h -- C ABI of libmta: Multi-Token Attention (MTA) forward on NVIDIA B200
+ * (sm_100a).
+ *
+ * What is computed (sources are the pages' titles and sections):
+ *   "Multi-Token Attention | Summary" (greeksharifa),
+ *     section 2  : per-head logits A_hat = Q K^T / sqrt(d), causal -inf mask,
+ *                  softmax over keys, A V, concatenation, output projection;
+ *     section 3.1: A = Softmax(Mask_-inf(Conv2d_theta(Mask_0(A_hat)))), one
+ *                  c_q x c_k kernel per head over (previous queries, neighbouring
+ *                  keys);
+ *     section 3.2: head mixing inside groups of c_h heads, before or after the
+ *                  softmax (A1_new = w11 A1 + w12 A2, ...);
+ *     section 3.3: group normalisation of each head's output with a scale;
+ *   "Multi-Token Attention" (bycloud), mechanism item 3: group normalisation
+ *     with depth scaling.
+ *
+ * Index conventions (the readings this library implements):
+ *   theta[h][a][t] multiplies Mask_0(A_hat)[i-a][j-(t-c_k/2)], a = 0..c_q-1
+ *   (current and previous queries), t = 0..c_k-1 (keys centred on j); entries
+ *   outside [0,L) and future keys of the shifted query count as 0.  The
+ *   identity kernel is theta[h][0][c_k/2] = 1.
+ *   w_head[g][r][s] weighs source head g*c_h+s in destination head g*c_h+r.
+ *   Post-softmax mixing is not renormalised; the mixed map of head r
+ *   multiplies head r's own values.  Pre-softmax mixing follows the
+ *   key-query convolution.
+ *
+ * Ownership and threading: every pointer is a DEVICE pointer owned by the
+ * caller (theta, w_head, gamma and beta included).  The library allocates no
+ * memory and keeps no state between calls; scratch space comes from
+ * cfg->workspace.  Calls are asynchronous on cfg->stream and re-entrant;
+ * calls that share a workspace must be ordered on one stream.
+ *
+ * Errors: every argument is checked before anything is enqueued; a bad
+ * argument returns MTA_ERR_INVALID / MTA_ERR_UNSUPPORTED / MTA_ERR_WORKSPACE
+ * and enqueues nothing.  A failed launch returns MTA_ERR_CUDA.  Kernels never
+ * wait without a bound: a wait that runs out sets a flag in the workspace and
+ * the kernel returns; mta_sync_status() reports it as MTA_ERR_TIMEOUT.
+ * Outputs must not alias inputs.
+ */
+#ifndef MTA_H
+#define MTA_H
+
+#include <stddef.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define MTA_ABI_VERSION 1
+
+typedef enum {
+  MTA_OK = 0,
+  MTA_ERR_INVALID = 1,      /* null pointer, bad shape or inconsistent configuration */
+  MTA_ERR_UNSUPPORTED = 2,  /* a valid configuration this build has no kernel for */
+  MTA_ERR_WORKSPACE = 3,    /* workspace missing, misaligned or smaller than required */
+  MTA_ERR_CUDA = 4,         /* a CUDA runtime call or a kernel launch failed */
+  MTA_ERR_TIMEOUT = 5       /* a kernel's bounded wait ran out (see mta_sync_status) */
+} mta_status;
+
+typedef enum { MTA_F32 = 0, MTA_BF16 = 1 } mta_dtype;
+
+/* Where a mixing step sits relative to the softmax.  kq_place: OFF or PRE
+ * (pre-softmax key-query convolution, section 3.1).  head_place: OFF, PRE or
+ * POST (section 3.2). */
+typedef enum { MTA_OFF = 0, MTA_PRE = 1, MTA_POST = 2 } mta_place;
+
+typedef struct mta_cfg {
+  int B;                 /* batch size, >= 1                                     */
+  int H;                 /* heads, >= 1, multiple of c_h                         */
+  int L;                 /* sequence length, >= 1                                */
+  int d;                 /* head dimension: 16..128, multiple of 8               */
+  int c_q;               /* query taps of the key-query kernel, 1..8             */
+  int c_k;               /* key taps, odd, 1..15                                 */
+  int c_h;               /* heads per mixing group, 1..16 (1 = no mixing)        */
+  int kq_place;          /* MTA_OFF or MTA_PRE                                   */
+  int head_place;        /* MTA_OFF, MTA_PRE or MTA_POST (OFF when c_h == 1)     */
+  int dtype;             /* mta_dtype of q, k, v and out (x, W and out in a layer) */
+  int path;              /* attention kernel: 0 = choose, 1 = CUDA-core kernel,
+                            2 = tensor-core kernel (MTA_ERR_UNSUPPORTED where it
+                            does not apply)                                       */
+  float scale;           /* logit scale; 0 selects 1/sqrt(d)                     */
+  long long qkv_row_stride; /* elements between consecutive tokens of q, k and v;
+                              0 selects H*d (dense [B][L][H][d]); ignored by
+                              mta_layer_fwd                                       */
+  void *stream;          /* cudaStream_t to enqueue on; NULL = legacy default    */
+  void *workspace;       /* device scratch, 256-byte aligned                      */
+  size_t workspace_bytes;
+} mta_cfg;
+
+/* Depth-scaled group normalisation of head outputs (section 3.3; bycloud item 3):
+ * y = lambda * ((o - mean_d) / sqrt(var_d + eps) * gamma + beta) per (token, head),
+ * biased variance over the d channels of one head. */
+typedef struct mta_gn {
+  const float *gamma;    /* [H*d] device, fp32                                   */
+  const float *beta;     /* [H*d] device, fp32                                   */
+  float eps;             /* <= 0 selects 1e-5                                    */
+  int layer;             /* layer index for the default depth scale             */
+  float depth_scale;     /* lambda; < 0 selects 1 - 0.8*exp(-0.3*layer)         */
+} mta_gn;
+
+/* Bytes of workspace mta_attn_fwd needs for cfg (0 if cfg is invalid). */
+size_t mta_attn_workspace_bytes(const mta_cfg *cfg);
+
+/* MTA attention core, sections 2, 3.1, 3.2 (steps: logits, Mask_0, key-query
+ * convolution, pre-softmax head mix, Mask_-inf, softmax, post-softmax head mix,
+ * A V).  Never materialises an L x L map.
+ *   q, k, v  : [B][L][H][d] with token stride cfg->qkv_row_stride, cfg->dtype
+ *   theta_kq : [H][c_q][c_k] fp32 (ignored when kq_place == MTA_OFF)
+ *   w_head   : [H/c_h][c_h][c_h] fp32 (ignored when head_place == MTA_OFF)
+ *   out      : [B][L][H][d] dense, cfg->dtype
+ * Pointers to bf16 data must be 16-byte aligned and the row stride a multiple
+ * of 8 elements for the tensor-core path; other layouts use the CUDA-core path. */
+mta_status mta_attn_fwd(const void *q, const void *k, const void *v,
+                        const float *theta_kq, const float *w_head,
+                        const mta_cfg *cfg, void *out);
+
+/* Bytes of workspace mta_layer_fwd needs for cfg (0 if cfg is invalid). */
+size_t mta_layer_workspace_bytes(const mta_cfg *cfg);
+
+/* Full MTA attention layer (bf16 only):
+ *   QKV = x Wqkv^T (section 2), attention as mta_attn_fwd, depth-scaled group
+ *   norm (section 3.3), out = Y Wo^T (section 2).
+ *   x    : [B][L][D] bf16, D = H*d
+ *   Wqkv : [3D][D] bf16, rows [Q | K | V], each head-major (row h*d+e)
+ *   Wo   : [D][D] bf16 (out x in)
+ *   out  : [B][L][D] bf16
+ * QKV and Y are kept in the workspace (bf16); no L x L map is stored. */
+mta_status mta_layer_fwd(const void *x, const void *Wqkv, const float *theta,
+                         const float *w_head, const mta_gn *gn, const void *Wo,
+                         const mta_cfg *cfg, void *out);
+
+/* Building blocks of mta_layer_fwd, exposed for testing and timing. */
+
+/* C[M][N] = A[M][K] * Bm[N][K]^T, bf16 in, fp32 accumulate, bf16 out.
+ * M, N, K >= 1; K a multiple of 8 and all pointers 16-byte aligned.
+ * Enqueued on `stream`. */
+mta_status mta_gemm_bf16_nt(const void *A, const void *Bm, void *C, int M, int N, int K,
+                            void *stream);
+
+/* y = depth-scaled group norm of o, both [tokens][H][d] bf16, dense. */
+mta_status mta_group_norm_scale(const void *o, const mta_gn *gn, int tokens, int H, int d,
+                                void *y, void *stream);
+
+/* Waits for cfg->stream and reports whether a kernel of the last call that used
+ * cfg->workspace gave up a bounded wait (MTA_ERR_TIMEOUT), else MTA_OK or
+ * MTA_ERR_CUDA.  Blocking; for tests and diagnostics. */
+mta_status mta_sync_status(const mta_cfg *cfg);
+
+/* Static description of a status code. */
+const char *mta_status_string(mta_status s);
+
+/* MTA_ABI_VERSION of the loaded library. */
+int mta_abi_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MTA_H */

@@ -1,0 +1,127 @@
+"""The C-ABI library: it builds, loads, exports every function include/mta.h
+declares, and rejects bad arguments on the host before any CUDA call (these
+tests need no GPU)."""
+import ctypes
+import os
+import re
+import subprocess
+
+import pytest
+
+from token_attention_b200 import build, mta
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def L():
+    build.build()
+    return mta.lib()
+
+
+def declared_functions():
+    text = open(os.path.join(ROOT, "include", "mta.h")).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(mta_\w+)\s*\(", text)))
+
+
+def test_header_and_binding_agree():
+    assert declared_functions() == sorted(mta.EXPORTS)
+
+
+def test_every_declared_symbol_is_exported(L):
+    out = subprocess.run(["nm", "-D", "--defined-only", mta.LIB_PATH], capture_output=True,
+                         text=True, check=True).stdout
+    exported = set(re.findall(r"\sT\s(\w+)$", out, flags=re.M))
+    missing = [f for f in declared_functions() if f not in exported]
+    assert not missing, missing
+    for f in declared_functions():
+        assert hasattr(L, f)
+
+
+def test_version_and_strings(L):
+    assert L.mta_abi_version() == 1
+    for code in range(6):
+        assert L.mta_status_string(code)
+    assert L.mta_status_string(0) == b"ok"
+
+
+def good_cfg(**kw):
+    base = dict(B=2, H=4, L=64, d=64, c_q=6, c_k=11, c_h=2, kq_place=mta.PRE,
+                head_place=mta.POST, dtype=mta.BF16)
+    base.update(kw)
+    return mta.make_cfg(**base)
+
+
+FAKE = ctypes.c_void_p(0x10000)  # never dereferenced: every case below fails a host check
+
+
+def call_attn(L, cfg, q=FAKE, theta=FAKE, w=FAKE, out=FAKE):
+    return L.mta_attn_fwd(q, FAKE, FAKE, theta, w, ctypes.byref(cfg) if cfg else None, out)
+
+
+def test_workspace_query(L):
+    cfg = good_cfg()
+    assert L.mta_attn_workspace_bytes(ctypes.byref(cfg)) == 256
+    t = 2 * 64
+    D = 4 * 64
+    want = 256 + -(-t * 3 * D * 2 // 256) * 256 + 2 * (-(-t * D * 2 // 256) * 256)
+    assert L.mta_layer_workspace_bytes(ctypes.byref(cfg)) == want
+    assert L.mta_attn_workspace_bytes(ctypes.byref(good_cfg(c_k=4))) == 0
+    assert L.mta_attn_workspace_bytes(None) == 0
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(c_k=4), 1), (dict(c_k=17), 1), (dict(c_q=0), 1), (dict(c_q=9), 1),
+    (dict(H=5), 1), (dict(c_h=0), 1), (dict(B=0), 1), (dict(L=0), 1),
+    (dict(kq_place=2), 1), (dict(head_place=3), 1), (dict(dtype=7), 1), (dict(path=3), 1),
+    (dict(scale=-1.0), 1), (dict(qkv_row_stride=10), 1),
+    (dict(d=200), 2), (dict(d=20), 2), (dict(B=70000), 2),
+])
+def test_bad_config_rejected(L, kw, code):
+    cfg = good_cfg(**kw)
+    cfg.workspace, cfg.workspace_bytes = 0x100000, 1 << 20
+    assert call_attn(L, cfg) == code
+
+
+def test_null_and_workspace_errors(L):
+    assert call_attn(L, None) == 1
+    cfg = good_cfg()
+    cfg.workspace, cfg.workspace_bytes = 0x100000, 1 << 20
+    assert call_attn(L, cfg, q=None) == 1
+    assert call_attn(L, cfg, out=None) == 1
+    assert call_attn(L, cfg, theta=None) == 1           # kq_place PRE needs theta
+    assert call_attn(L, cfg, w=None) == 1               # head mixing needs w
+    nomix = good_cfg(kq_place=mta.OFF, head_place=mta.OFF)
+    nomix.workspace, nomix.workspace_bytes = 0x100000, 1 << 20
+    assert call_attn(L, nomix, q=ctypes.c_void_p(0x10001)) == 1   # misaligned bf16
+    cfg.workspace_bytes = 16
+    assert call_attn(L, cfg) == 3
+    cfg.workspace, cfg.workspace_bytes = 0x100010, 1 << 20   # not 256-byte aligned
+    assert call_attn(L, cfg) == 3
+    cfg.workspace = None
+    assert call_attn(L, cfg) == 3
+
+
+def test_layer_argument_errors(L):
+    cfg = good_cfg()
+    cfg.workspace, cfg.workspace_bytes = 0x100000, 1 << 30
+    gn = mta.MtaGn(0x20000, 0x20000, 1e-5, 12, -1.0)
+    f = lambda c, g=ctypes.byref(gn), x=FAKE: L.mta_layer_fwd(x, FAKE, FAKE, FAKE, g, FAKE,
+                                                              ctypes.byref(c), FAKE)
+    assert f(cfg, g=None) == 1
+    assert f(cfg, x=None) == 1
+    f32 = good_cfg(dtype=mta.F32)
+    f32.workspace, f32.workspace_bytes = 0x100000, 1 << 30
+    assert f(f32) == 2
+    small = good_cfg()
+    small.workspace, small.workspace_bytes = 0x100000, 1024
+    assert f(small) == 3
+
+
+def test_building_block_argument_errors(L):
+    assert L.mta_gemm_bf16_nt(FAKE, FAKE, FAKE, 0, 8, 8, None) == 1
+    assert L.mta_gemm_bf16_nt(FAKE, FAKE, FAKE, 8, 8, 12, None) == 1   # K % 8
+    gn = mta.MtaGn(0x20000, 0x20000, 1e-5, 12, -1.0)
+    assert L.mta_group_norm_scale(FAKE, ctypes.byref(gn), 4, 2, 0, FAKE, None) == 1
+    assert L.mta_group_norm_scale(FAKE, None, 4, 2, 64, FAKE, None) == 1

@@ -1,0 +1,246 @@
+"""GPU parity: the CUDA path through the C ABI against the fp64 oracle.
+
+Tolerances (stated for the MTA forward): bf16 outputs within a relative L2
+error of 1e-2 and a max-abs error of 3e-2 of the oracle; fp32 outputs within a
+relative L2 error of 1e-4.  Small cases compare every element and span several
+tiles plus a ragged tail; full-size workloads, in the launch configuration the
+bench times, compare sampled tokens the oracle computes one by one.
+"""
+import ctypes
+
+import numpy as np
+import pytest
+import torch
+
+import oracle as O
+from token_attention_b200 import build, mta, synth
+
+pytestmark = pytest.mark.gpu
+
+TOL_BF16 = (1e-2, 3e-2)
+TOL_F32 = 1e-4
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _gpu():
+    if not torch.cuda.is_available():
+        pytest.skip("needs a CUDA GPU")
+    build.build()
+    mta.lib()
+
+
+def dev(x, dtype="bf16"):
+    t = torch.from_numpy(np.ascontiguousarray(x)).cuda()
+    return t.to(torch.bfloat16) if dtype == "bf16" else t
+
+
+def errs(gpu, ref):
+    g = gpu.detach().double().cpu().numpy().reshape(ref.shape)
+    diff = g - ref
+    return float(np.linalg.norm(diff) / max(np.linalg.norm(ref), 1e-300)), float(np.abs(diff).max())
+
+
+def assert_close(gpu, ref, dtype):
+    rel, mx = errs(gpu, ref)
+    if dtype == "bf16":
+        assert rel <= TOL_BF16[0] and mx <= TOL_BF16[1], (rel, mx)
+    else:
+        assert rel <= TOL_F32, (rel, mx)
+    return rel, mx
+
+
+def run_attn(wl, inp, path=mta.PATH_AUTO, **kw):
+    q, k, v = (dev(inp[n], wl.dtype) for n in ("q", "k", "v"))
+    th, w = dev(inp["theta"], "f32"), dev(inp["w"], "f32")
+    out = mta.attn_fwd(q, k, v, th, w, wl.c_q, wl.c_k, wl.c_h, wl.kq_place, wl.head_place,
+                       path=path, check=True, **kw)
+    torch.cuda.synchronize()
+    return out
+
+
+def oracle_full(wl, inp):
+    return O.mta_attention(inp["q"], inp["k"], inp["v"], inp["theta"], inp["w"], wl.c_h,
+                           wl.kq_place, wl.head_place)
+
+
+# ---------------------------------------------------------------------------
+# small cases: every element
+# ---------------------------------------------------------------------------
+
+@pytest.mark.parametrize("path", [mta.PATH_AUTO, mta.PATH_SIMT])
+def test_tiny_f32_L256(path):
+    wl = synth.WORKLOADS["tiny_f32_L256"]
+    inp = synth.make_attn_inputs(wl)
+    assert_close(run_attn(wl, inp, path), oracle_full(wl, inp), "f32")
+
+
+SMALL = []
+for d in (64, 128):
+    for hp in (synth.OFF, synth.PRE, synth.POST):
+        for L in (1, 9, 300):
+            SMALL.append((d, hp, L))
+
+
+@pytest.mark.parametrize("d,hp,L", SMALL)
+@pytest.mark.parametrize("path", [mta.PATH_AUTO, mta.PATH_SIMT])
+def test_small_bf16(d, hp, L, path):
+    base = synth.WORKLOADS["pretrain_d128_L2048"]
+    wl = synth.shrink(base, B=2, H=4, L=L, d=d, head_place=hp, seed=77 + L + d + hp)
+    inp = synth.make_attn_inputs(wl)
+    assert_close(run_attn(wl, inp, path), oracle_full(wl, inp), "bf16")
+
+
+@pytest.mark.parametrize("c_q,c_k,c_h,kq", [(1, 1, 1, synth.PRE), (3, 5, 4, synth.PRE),
+                                            (6, 11, 1, synth.OFF), (8, 15, 2, synth.PRE)])
+def test_small_bf16_other_kernels(c_q, c_k, c_h, kq):
+    base = synth.WORKLOADS["pretrain_d128_L2048"]
+    wl = synth.shrink(base, B=1, H=8, L=200, d=64, c_q=c_q, c_k=c_k, c_h=c_h, kq_place=kq,
+                      head_place=synth.POST if c_h > 1 else synth.OFF, seed=91 + c_q)
+    inp = synth.make_attn_inputs(wl)
+    assert_close(run_attn(wl, inp), oracle_full(wl, inp), "bf16")
+
+
+def test_strided_qkv_views():
+    """q, k, v as column blocks of one [B, L, 3*H*d] buffer (the layer's layout)."""
+    base = synth.WORKLOADS["pretrain_d128_L2048"]
+    wl = synth.shrink(base, B=2, H=4, L=260, d=128, seed=5)
+    inp = synth.make_attn_inputs(wl)
+    B, L, H, d = wl.B, wl.L, wl.H, wl.d
+    buf = torch.empty((B, L, 3, H, d), dtype=torch.bfloat16, device="cuda")
+    for i, n in enumerate("qkv"):
+        buf[:, :, i] = dev(inp[n])
+    q, k, v = buf[:, :, 0], buf[:, :, 1], buf[:, :, 2]
+    out = mta.attn_fwd(q, k, v, dev(inp["theta"], "f32"), dev(inp["w"], "f32"), wl.c_q, wl.c_k,
+                       wl.c_h, wl.kq_place, wl.head_place, check=True)
+    assert_close(out, oracle_full(wl, inp), "bf16")
+
+
+def test_causality_on_gpu():
+    """Outputs before position t do not change when q, k, v at >= t change."""
+    base = synth.WORKLOADS["pretrain_d128_L2048"]
+    wl = synth.shrink(base, B=1, H=4, L=400, d=128, seed=8)
+    inp = synth.make_attn_inputs(wl)
+    a = run_attn(wl, inp)
+    t = 201
+    for n, s in (("q", 1), ("k", 2), ("v", 3)):
+        x = inp[n].copy()
+        x[:, t:] = synth.round_bf16(synth.normal(99, s, x[:, t:].shape))
+        inp[n] = x
+    b = run_attn(wl, inp)
+    assert torch.equal(a[:, :t], b[:, :t])
+    assert not torch.equal(a[:, t:], b[:, t:])
+
+
+# ---------------------------------------------------------------------------
+# full-size workloads: sampled tokens
+# ---------------------------------------------------------------------------
+
+def sample_rows(wl, n_extra=6, seed=0):
+    rng = np.random.default_rng(seed)
+    fixed = [0, 1, 4, 5, 6, 122, 123, 127, 128, 129, 245, 246, wl.L // 2, wl.L - 2, wl.L - 1]
+    rows = sorted({(int(rng.integers(wl.B)), i) for i in fixed if i < wl.L})
+    rows += [(int(rng.integers(wl.B)), int(rng.integers(wl.L))) for _ in range(n_extra)]
+    return sorted(set(rows))
+
+
+@pytest.mark.parametrize("name", ["identity_d64_L2048", "pretrain_d128_L2048", "long_d128_L16384"])
+def test_full_size_sampled(name):
+    wl = synth.WORKLOADS[name]
+    inp = synth.make_attn_inputs(wl)
+    out = run_attn(wl, inp)
+    rows = sample_rows(wl)
+    ref = O.mta_attention_rows(inp["q"], inp["k"], inp["v"], inp["theta"], inp["w"], wl.c_h,
+                               rows, wl.kq_place, wl.head_place)
+    got = torch.stack([out[b, i] for b, i in rows])
+    assert_close(got, ref, "bf16")
+
+
+def test_identity_workload_equals_causal_attention():
+    """Identity kernels: the whole output equals causal softmax attention (torch
+    SDPA in fp32 on the same bf16 inputs)."""
+    wl = synth.WORKLOADS["identity_d64_L2048"]
+    inp = synth.make_attn_inputs(wl)
+    out = run_attn(wl, inp)
+    q, k, v = (dev(inp[n], "f32").permute(0, 2, 1, 3) for n in "qkv")
+    ref = torch.nn.functional.scaled_dot_product_attention(q, k, v, is_causal=True)
+    ref = ref.permute(0, 2, 1, 3).double().cpu().numpy()
+    assert_close(out, ref, "bf16")
+
+
+def test_no_LxL_buffer():
+    """Peak device memory of a call stays at inputs + outputs + workspace."""
+    wl = synth.WORKLOADS["pretrain_d128_L2048"]
+    inp = synth.make_attn_inputs(wl)
+    q, k, v = (dev(inp[n]) for n in "qkv")
+    th, w = dev(inp["theta"], "f32"), dev(inp["w"], "f32")
+    out = torch.empty_like(q)
+    ws = mta.workspace(256)
+    torch.cuda.synchronize()
+    torch.cuda.reset_peak_memory_stats()
+    before = torch.cuda.memory_allocated()
+    mta.attn_fwd(q, k, v, th, w, wl.c_q, wl.c_k, wl.c_h, out=out, ws=ws, check=True)
+    torch.cuda.synchronize()
+    assert torch.cuda.max_memory_allocated() == before
+    lxl = wl.B * wl.H * wl.L * wl.L * 4
+    assert before < lxl
+
+
+# ---------------------------------------------------------------------------
+# building blocks and the layer
+# ---------------------------------------------------------------------------
+
+@pytest.mark.parametrize("M,N,K", [(300, 520, 264), (128, 256, 64), (1000, 96, 2048), (7, 9, 8)])
+def test_gemm_bf16_nt(M, N, K):
+    a = synth.round_bf16(synth.normal(3, 1, (M, K)))
+    b = synth.round_bf16(synth.normal(3, 2, (N, K), std=0.05))
+    c = mta.gemm_bf16_nt(dev(a), dev(b))
+    torch.cuda.synchronize()
+    assert_close(c, a.astype(np.float64) @ b.astype(np.float64).T, "bf16")
+
+
+def test_group_norm_scale():
+    o = synth.round_bf16(synth.normal(4, 1, (515, 16, 128), mean=0.3, std=2.0))
+    gamma = synth.normal(4, 2, (16 * 128,), mean=1.0, std=0.1)
+    beta = synth.normal(4, 3, (16 * 128,), std=0.1)
+    y = mta.group_norm_scale(dev(o), dev(gamma, "f32"), dev(beta, "f32"), 1e-5, 0.97814)
+    torch.cuda.synchronize()
+    assert_close(y, O.group_norm_scale(o, gamma, beta, 1e-5, 0.97814), "bf16")
+    o2 = o[:, :, :72].copy()
+    y2 = mta.group_norm_scale(dev(o2), dev(gamma[:16 * 72], "f32"), dev(beta[:16 * 72], "f32"),
+                              1e-5, 0.5)
+    torch.cuda.synchronize()
+    assert_close(y2, O.group_norm_scale(o2, gamma[:16 * 72], beta[:16 * 72], 1e-5, 0.5), "bf16")
+
+
+def run_layer(wl, inp, path=mta.PATH_AUTO):
+    x, wqkv, wo = dev(inp["x"]), dev(inp["wqkv"]), dev(inp["wo"])
+    out = mta.layer_fwd(x, wqkv, dev(inp["theta"], "f32"), dev(inp["w"], "f32"),
+                        dev(inp["gamma"], "f32"), dev(inp["beta"], "f32"), wo, wl.H, wl.c_q,
+                        wl.c_k, wl.c_h, wl.kq_place, wl.head_place, eps=inp["eps"],
+                        layer=wl.depth, path=path, check=True)
+    torch.cuda.synchronize()
+    return out
+
+
+@pytest.mark.parametrize("name", ["layer_pre_D2048_L4096", "layer_post_D2048_L4096"])
+@pytest.mark.parametrize("path", [mta.PATH_AUTO, mta.PATH_SIMT])
+def test_layer_small(name, path):
+    wl = synth.shrink(synth.WORKLOADS[name], B=2, L=300, D=256, H=2, d=128, seed=123)
+    inp = synth.make_layer_inputs(wl)
+    out = run_layer(wl, inp, path)
+    ref = O.mta_layer(inp["x"], inp["wqkv"], inp["theta"], inp["w"], inp["gamma"], inp["beta"],
+                      inp["eps"], inp["lam"], inp["wo"], wl.H, wl.c_h, wl.kq_place, wl.head_place)
+    assert_close(out, ref, "bf16")
+
+
+@pytest.mark.parametrize("name", ["layer_pre_D2048_L4096", "layer_post_D2048_L4096"])
+def test_layer_full_size_sampled(name):
+    wl = synth.WORKLOADS[name]
+    inp = synth.make_layer_inputs(wl)
+    out = run_layer(wl, inp)
+    rows = [(0, 0), (0, 5), (0, 123), (0, 2048), (0, 4095), (1, 1), (1, 700), (1, 4094)]
+    ref = O.mta_layer_rows(inp["x"], inp["wqkv"], inp["theta"], inp["w"], inp["gamma"],
+                           inp["beta"], inp["eps"], inp["lam"], inp["wo"], wl.H, wl.c_h, rows,
+                           wl.kq_place, wl.head_place)
+    got = torch.stack([out[b, i] for b, i in rows])
+    assert_close(got, ref, "bf16")

@@ -1,0 +1,54 @@
+// internal.h -- host-side launchers shared by the C-ABI layer (mta_api.cu).
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+
+namespace mta {
+
+// Bits of the error word kept at the start of the caller's workspace.
+enum : unsigned { ERRBIT_TIMEOUT = 1u };
+
+// Arguments of one attention call, already validated by the C-ABI layer.
+struct AttnArgs {
+  const void *q, *k, *v;  // [B][L][H][d], token stride rs elements
+  long long rs;
+  const float *theta;     // [H][c_q][c_k]
+  const float *w;         // [H/c_h][c_h][c_h]
+  void *out;              // [B][L][H][d] dense
+  int B, H, L, d, cq, ck, ch, kq, hp, dtype;
+  float scale;
+  unsigned *err;          // error word in the workspace
+  cudaStream_t stream;
+};
+
+// Depth-scaled group norm fused into an attention epilogue (optional).
+struct GnArgs {
+  const float *gamma, *beta;  // [H*d]
+  float eps, lam;
+};
+
+// Generic CUDA-core kernel: every supported configuration, fp32 arithmetic.
+size_t attn_simt_smem_bytes(const AttnArgs &a, int BR, int BC);
+int attn_simt_pick_rows(const AttnArgs &a, int BC);  // 0 if nothing fits
+cudaError_t launch_attn_simt(const AttnArgs &a);
+
+// tcgen05 kernel (bf16, fused); attn_tc_supported() says whether it applies.
+bool attn_tc_supported(const AttnArgs &a);
+cudaError_t launch_attn_tc(const AttnArgs &a, const GnArgs *gn);
+
+// tcgen05 GEMM: C[M][N] = A[M][K] * B[N][K]^T (bf16 -> fp32 -> bf16).
+cudaError_t launch_gemm_bf16_nt(const void *A, const void *B, void *C, int M, int N, int K,
+                                unsigned *err, cudaStream_t stream);
+
+// Depth-scaled group norm over [tokens][H][d] bf16.
+cudaError_t launch_group_norm(const void *o, const GnArgs &gn, int tokens, int H, int d, void *y,
+                              cudaStream_t stream);
+
+// cuTensorMapEncodeTiled through the runtime's driver entry point.
+// dims/strides innermost first; strides in bytes for dims 1..rank-1.
+bool encode_tmap_bf16(void *map_out, const void *base, int rank, const unsigned long long *dims,
+                      const unsigned long long *strides_bytes, const unsigned *box,
+                      bool swizzle128);
+
+}  // namespace mta

@@ -1,0 +1,264 @@
+// mta_api.cu -- the C ABI declared in include/mta.h: argument checks, workspace
+// layout, kernel selection.  Every check runs before anything is enqueued, and
+// nothing here calls CUDA before the arguments have passed.
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cudaTypedefs.h>
+#include <math.h>
+#include <stdint.h>
+
+#include "internal.h"
+#include "mta.h"
+
+namespace mta {
+namespace {
+
+constexpr size_t kAlign = 256;
+constexpr size_t kStatusBytes = 256;  // error word + padding at the workspace start
+
+size_t align_up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
+
+bool aligned(const void *p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+// Shape and option checks shared by the attention and the layer.
+mta_status check_cfg(const mta_cfg *c) {
+  if (!c) return MTA_ERR_INVALID;
+  if (c->B < 1 || c->H < 1 || c->L < 1) return MTA_ERR_INVALID;
+  if (c->B > 65535) return MTA_ERR_UNSUPPORTED;
+  if (c->d < 16 || c->d > 128 || c->d % 8 != 0) return MTA_ERR_UNSUPPORTED;
+  if (c->c_q < 1 || c->c_q > 8) return MTA_ERR_INVALID;
+  if (c->c_k < 1 || c->c_k > 15 || c->c_k % 2 == 0) return MTA_ERR_INVALID;
+  if (c->c_h < 1 || c->c_h > 16 || c->H % c->c_h != 0) return MTA_ERR_INVALID;
+  if (c->kq_place != MTA_OFF && c->kq_place != MTA_PRE) return MTA_ERR_INVALID;
+  if (c->head_place != MTA_OFF && c->head_place != MTA_PRE && c->head_place != MTA_POST)
+    return MTA_ERR_INVALID;
+  if (c->dtype != MTA_F32 && c->dtype != MTA_BF16) return MTA_ERR_INVALID;
+  if (c->path < 0 || c->path > 2) return MTA_ERR_INVALID;
+  if (!isfinite(c->scale) || c->scale < 0.f) return MTA_ERR_INVALID;
+  const long long hd = static_cast<long long>(c->H) * c->d;
+  if (c->qkv_row_stride != 0 && c->qkv_row_stride < hd) return MTA_ERR_INVALID;
+  return MTA_OK;
+}
+
+AttnArgs make_args(const void *q, const void *k, const void *v, const float *theta,
+                   const float *w, const mta_cfg *c, void *out) {
+  AttnArgs a;
+  a.q = q; a.k = k; a.v = v; a.theta = theta; a.w = w; a.out = out;
+  a.rs = c->qkv_row_stride ? c->qkv_row_stride : static_cast<long long>(c->H) * c->d;
+  a.B = c->B; a.H = c->H; a.L = c->L; a.d = c->d;
+  a.cq = c->c_q; a.ck = c->c_k; a.ch = c->c_h;
+  a.kq = c->kq_place; a.hp = c->head_place; a.dtype = c->dtype;
+  a.scale = c->scale > 0.f ? c->scale : 1.0f / sqrtf(static_cast<float>(c->d));
+  a.err = static_cast<unsigned *>(c->workspace);
+  a.stream = static_cast<cudaStream_t>(c->stream);
+  return a;
+}
+
+// Which attention kernel serves `a` under cfg->path (0: the tensor-core kernel
+// where it applies, else the CUDA-core kernel; 1: CUDA-core; 2: tensor-core).
+mta_status select_kernel(const AttnArgs &a, int path, bool *use_tc) {
+  const bool tc_ok = attn_tc_supported(a);
+  if (path == 2 && !tc_ok) return MTA_ERR_UNSUPPORTED;
+  *use_tc = tc_ok && path != 1;
+  if (!*use_tc && attn_simt_pick_rows(a, 32) == 0) return MTA_ERR_UNSUPPORTED;
+  return MTA_OK;
+}
+
+mta_status check_attn_pointers(const void *q, const void *k, const void *v, const float *theta,
+                               const float *w, const mta_cfg *c, const void *out) {
+  if (!q || !k || !v || !out) return MTA_ERR_INVALID;
+  if (c->kq_place == MTA_PRE && !theta) return MTA_ERR_INVALID;
+  if (c->head_place != MTA_OFF && !w) return MTA_ERR_INVALID;
+  const size_t es = c->dtype == MTA_F32 ? 4 : 2;
+  if (!aligned(q, es) || !aligned(k, es) || !aligned(v, es) || !aligned(out, es))
+    return MTA_ERR_INVALID;
+  if ((theta && !aligned(theta, 4)) || (w && !aligned(w, 4))) return MTA_ERR_INVALID;
+  return MTA_OK;
+}
+
+mta_status check_workspace(const mta_cfg *c, size_t need) {
+  if (!c->workspace || c->workspace_bytes < need || !aligned(c->workspace, kAlign))
+    return MTA_ERR_WORKSPACE;
+  return MTA_OK;
+}
+
+mta_status clear_status(const mta_cfg *c) {
+  return cudaMemsetAsync(c->workspace, 0, sizeof(unsigned), static_cast<cudaStream_t>(c->stream)) ==
+                 cudaSuccess
+             ? MTA_OK
+             : MTA_ERR_CUDA;
+}
+
+size_t layer_tokens(const mta_cfg *c) { return static_cast<size_t>(c->B) * c->L; }
+
+GnArgs make_gn(const mta_gn *gn) {
+  GnArgs g;
+  g.gamma = gn->gamma;
+  g.beta = gn->beta;
+  g.eps = gn->eps > 0.f ? gn->eps : 1e-5f;
+  g.lam = gn->depth_scale >= 0.f ? gn->depth_scale
+                                 : static_cast<float>(1.0 - 0.8 * exp(-0.3 * gn->layer));
+  return g;
+}
+
+}  // namespace
+
+bool encode_tmap_bf16(void *map_out, const void *base, int rank, const unsigned long long *dims,
+                      const unsigned long long *strides_bytes, const unsigned *box, bool swizzle128) {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = [] {
+    void *p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) != cudaSuccess ||
+        q != cudaDriverEntryPointSuccess)
+      p = nullptr;
+    return reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  }();
+  if (!fn) return false;
+  cuuint64_t gdim[5], gstr[4];
+  cuuint32_t bdim[5], estr[5];
+  for (int i = 0; i < rank; ++i) {
+    gdim[i] = dims[i];
+    bdim[i] = box[i];
+    estr[i] = 1;
+    if (i > 0) gstr[i - 1] = strides_bytes[i - 1];
+  }
+  CUresult r = fn(static_cast<CUtensorMap *>(map_out), CU_TENSOR_MAP_DATA_TYPE_BFLOAT16,
+                  static_cast<cuuint32_t>(rank), const_cast<void *>(base), gdim, gstr, bdim, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE,
+                  swizzle128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+}  // namespace mta
+
+using namespace mta;
+
+extern "C" {
+
+int mta_abi_version(void) { return MTA_ABI_VERSION; }
+
+const char *mta_status_string(mta_status s) {
+  switch (s) {
+    case MTA_OK: return "ok";
+    case MTA_ERR_INVALID: return "invalid argument";
+    case MTA_ERR_UNSUPPORTED: return "unsupported configuration";
+    case MTA_ERR_WORKSPACE: return "workspace missing, misaligned or too small";
+    case MTA_ERR_CUDA: return "CUDA error";
+    case MTA_ERR_TIMEOUT: return "a kernel gave up a bounded wait";
+  }
+  return "unknown status";
+}
+
+size_t mta_attn_workspace_bytes(const mta_cfg *cfg) {
+  if (check_cfg(cfg) != MTA_OK) return 0;
+  return kStatusBytes;
+}
+
+mta_status mta_attn_fwd(const void *q, const void *k, const void *v, const float *theta_kq,
+                        const float *w_head, const mta_cfg *cfg, void *out) {
+  mta_status s = check_cfg(cfg);
+  if (s != MTA_OK) return s;
+  if ((s = check_attn_pointers(q, k, v, theta_kq, w_head, cfg, out)) != MTA_OK) return s;
+  if ((s = check_workspace(cfg, kStatusBytes)) != MTA_OK) return s;
+  AttnArgs a = make_args(q, k, v, theta_kq, w_head, cfg, out);
+  bool use_tc = false;
+  if ((s = select_kernel(a, cfg->path, &use_tc)) != MTA_OK) return s;
+  if ((s = clear_status(cfg)) != MTA_OK) return s;
+  const cudaError_t e = use_tc ? launch_attn_tc(a, nullptr) : launch_attn_simt(a);
+  return e == cudaSuccess ? MTA_OK : MTA_ERR_CUDA;
+}
+
+size_t mta_layer_workspace_bytes(const mta_cfg *cfg) {
+  if (check_cfg(cfg) != MTA_OK) return 0;
+  const size_t T = layer_tokens(cfg), D = static_cast<size_t>(cfg->H) * cfg->d;
+  return kStatusBytes + align_up(T * 3 * D * 2) + 2 * align_up(T * D * 2);
+}
+
+mta_status mta_layer_fwd(const void *x, const void *Wqkv, const float *theta, const float *w_head,
+                         const mta_gn *gn, const void *Wo, const mta_cfg *cfg, void *out) {
+  mta_status s = check_cfg(cfg);
+  if (s != MTA_OK) return s;
+  if (cfg->dtype != MTA_BF16) return MTA_ERR_UNSUPPORTED;
+  if (!x || !Wqkv || !Wo || !out || !gn || !gn->gamma || !gn->beta) return MTA_ERR_INVALID;
+  if (cfg->kq_place == MTA_PRE && !theta) return MTA_ERR_INVALID;
+  if (cfg->head_place != MTA_OFF && !w_head) return MTA_ERR_INVALID;
+  if (!aligned(x, 16) || !aligned(Wqkv, 16) || !aligned(Wo, 16) || !aligned(out, 16) ||
+      !aligned(gn->gamma, 4) || !aligned(gn->beta, 4))
+    return MTA_ERR_INVALID;
+  const size_t T = layer_tokens(cfg), D = static_cast<size_t>(cfg->H) * cfg->d;
+  if (T > static_cast<size_t>(65535) * 128 || 3 * D > static_cast<size_t>(1) << 30)
+    return MTA_ERR_UNSUPPORTED;
+  if ((s = check_workspace(cfg, mta_layer_workspace_bytes(cfg))) != MTA_OK) return s;
+
+  char *ws = static_cast<char *>(cfg->workspace);
+  void *qkv = ws + kStatusBytes;
+  void *obuf = ws + kStatusBytes + align_up(T * 3 * D * 2);
+  void *ybuf = static_cast<char *>(obuf) + align_up(T * D * 2);
+  const uint16_t *qkvb = static_cast<const uint16_t *>(qkv);  // bf16 elements
+
+  mta_cfg acfg = *cfg;
+  acfg.qkv_row_stride = static_cast<long long>(3 * D);
+  AttnArgs a = make_args(qkvb, qkvb + D, qkvb + 2 * D, theta, w_head, &acfg, obuf);
+  bool use_tc = false;
+  if ((s = select_kernel(a, cfg->path, &use_tc)) != MTA_OK) return s;
+
+  const GnArgs g = make_gn(gn);
+  cudaStream_t st = static_cast<cudaStream_t>(cfg->stream);
+  unsigned *err = static_cast<unsigned *>(cfg->workspace);
+  if ((s = clear_status(cfg)) != MTA_OK) return s;
+  // QKV = x Wqkv^T
+  if (launch_gemm_bf16_nt(x, Wqkv, qkv, static_cast<int>(T), static_cast<int>(3 * D),
+                          static_cast<int>(D), err, st) != cudaSuccess)
+    return MTA_ERR_CUDA;
+  if (use_tc) {
+    // attention with the group norm and depth scale fused into its epilogue: Y
+    a.out = ybuf;
+    if (launch_attn_tc(a, &g) != cudaSuccess) return MTA_ERR_CUDA;
+  } else {
+    // attention output O, then the stand-alone group norm O -> Y
+    a.out = obuf;
+    if (launch_attn_simt(a) != cudaSuccess) return MTA_ERR_CUDA;
+    if (launch_group_norm(obuf, g, static_cast<int>(T), cfg->H, cfg->d, ybuf, st) != cudaSuccess)
+      return MTA_ERR_CUDA;
+  }
+  // out = Y Wo^T
+  if (launch_gemm_bf16_nt(ybuf, Wo, out, static_cast<int>(T), static_cast<int>(D),
+                          static_cast<int>(D), err, st) != cudaSuccess)
+    return MTA_ERR_CUDA;
+  return MTA_OK;
+}
+
+mta_status mta_gemm_bf16_nt(const void *A, const void *Bm, void *C, int M, int N, int K, void *stream) {
+  if (!A || !Bm || !C || M < 1 || N < 1 || K < 1) return MTA_ERR_INVALID;
+  if (K % 8 != 0 || !aligned(A, 16) || !aligned(Bm, 16) || !aligned(C, 16)) return MTA_ERR_INVALID;
+  if (M > 65535 * 128) return MTA_ERR_UNSUPPORTED;
+  return launch_gemm_bf16_nt(A, Bm, C, M, N, K, nullptr, static_cast<cudaStream_t>(stream)) ==
+                 cudaSuccess
+             ? MTA_OK
+             : MTA_ERR_CUDA;
+}
+
+mta_status mta_group_norm_scale(const void *o, const mta_gn *gn, int tokens, int H, int d, void *y,
+                                void *stream) {
+  if (!o || !gn || !gn->gamma || !gn->beta || !y || tokens < 0 || H < 1 || d < 1 || d > 128)
+    return MTA_ERR_INVALID;
+  if (!aligned(o, 2) || !aligned(y, 2) || !aligned(gn->gamma, 4) || !aligned(gn->beta, 4))
+    return MTA_ERR_INVALID;
+  return launch_group_norm(o, make_gn(gn), tokens, H, d, y, static_cast<cudaStream_t>(stream)) ==
+                 cudaSuccess
+             ? MTA_OK
+             : MTA_ERR_CUDA;
+}
+
+mta_status mta_sync_status(const mta_cfg *cfg) {
+  if (!cfg || !cfg->workspace) return MTA_ERR_INVALID;
+  cudaStream_t st = static_cast<cudaStream_t>(cfg->stream);
+  if (cudaStreamSynchronize(st) != cudaSuccess) return MTA_ERR_CUDA;
+  unsigned word = 0;
+  if (cudaMemcpy(&word, cfg->workspace, sizeof(word), cudaMemcpyDeviceToHost) != cudaSuccess)
+    return MTA_ERR_CUDA;
+  return (word & ERRBIT_TIMEOUT) ? MTA_ERR_TIMEOUT : MTA_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,211 @@
+"""ctypes binding of libmta.so (include/mta.h).
+
+Argument marshalling only: shapes and pointers are taken from torch tensors and
+handed to the C ABI; every step of the computation runs in the library's CUDA
+kernels.  There is no fallback: if libmta.so is missing or a call fails, this
+module raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(HERE, "libmta.so")
+
+OFF, PRE, POST = 0, 1, 2
+F32, BF16 = 0, 1
+PATH_AUTO, PATH_SIMT, PATH_TC = 0, 1, 2
+
+STATUS = {0: "MTA_OK", 1: "MTA_ERR_INVALID", 2: "MTA_ERR_UNSUPPORTED", 3: "MTA_ERR_WORKSPACE",
+          4: "MTA_ERR_CUDA", 5: "MTA_ERR_TIMEOUT"}
+
+# Every function include/mta.h declares.
+EXPORTS = ["mta_attn_workspace_bytes", "mta_attn_fwd", "mta_layer_workspace_bytes",
+           "mta_layer_fwd", "mta_gemm_bf16_nt", "mta_group_norm_scale", "mta_sync_status",
+           "mta_status_string", "mta_abi_version"]
+
+
+class MtaCfg(ctypes.Structure):
+    _fields_ = [("B", ctypes.c_int), ("H", ctypes.c_int), ("L", ctypes.c_int), ("d", ctypes.c_int),
+                ("c_q", ctypes.c_int), ("c_k", ctypes.c_int), ("c_h", ctypes.c_int),
+                ("kq_place", ctypes.c_int), ("head_place", ctypes.c_int),
+                ("dtype", ctypes.c_int), ("path", ctypes.c_int), ("scale", ctypes.c_float),
+                ("qkv_row_stride", ctypes.c_longlong), ("stream", ctypes.c_void_p),
+                ("workspace", ctypes.c_void_p), ("workspace_bytes", ctypes.c_size_t)]
+
+
+class MtaGn(ctypes.Structure):
+    _fields_ = [("gamma", ctypes.c_void_p), ("beta", ctypes.c_void_p), ("eps", ctypes.c_float),
+                ("layer", ctypes.c_int), ("depth_scale", ctypes.c_float)]
+
+
+class MtaError(RuntimeError):
+    def __init__(self, fn: str, code: int):
+        super().__init__(f"{fn} returned {STATUS.get(code, code)}")
+        self.code = code
+
+
+_lib = None
+
+
+def lib() -> ctypes.CDLL:
+    """The loaded libmta.so (raises if it has not been built)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(f"{LIB_PATH} is missing: build it with "
+                               "`python -m token_attention_b200.build`")
+        L = ctypes.CDLL(LIB_PATH)
+        P, I, S = ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t
+        cfgp = ctypes.POINTER(MtaCfg)
+        L.mta_attn_workspace_bytes.argtypes = [cfgp]
+        L.mta_attn_workspace_bytes.restype = S
+        L.mta_layer_workspace_bytes.argtypes = [cfgp]
+        L.mta_layer_workspace_bytes.restype = S
+        L.mta_attn_fwd.argtypes = [P, P, P, P, P, cfgp, P]
+        L.mta_attn_fwd.restype = I
+        L.mta_layer_fwd.argtypes = [P, P, P, P, ctypes.POINTER(MtaGn), P, cfgp, P]
+        L.mta_layer_fwd.restype = I
+        L.mta_gemm_bf16_nt.argtypes = [P, P, P, I, I, I, P]
+        L.mta_gemm_bf16_nt.restype = I
+        L.mta_group_norm_scale.argtypes = [P, ctypes.POINTER(MtaGn), I, I, I, P, P]
+        L.mta_group_norm_scale.restype = I
+        L.mta_sync_status.argtypes = [cfgp]
+        L.mta_sync_status.restype = I
+        L.mta_status_string.argtypes = [I]
+        L.mta_status_string.restype = ctypes.c_char_p
+        L.mta_abi_version.argtypes = []
+        L.mta_abi_version.restype = I
+        _lib = L
+    return _lib
+
+
+def _check(fn: str, code: int) -> None:
+    if code != 0:
+        raise MtaError(fn, code)
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream_handle(stream):
+    import torch
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def make_cfg(B, H, L, d, c_q, c_k, c_h, kq_place, head_place, dtype, path=PATH_AUTO, scale=0.0,
+             qkv_row_stride=0, stream=None, workspace=None) -> MtaCfg:
+    cfg = MtaCfg()
+    cfg.B, cfg.H, cfg.L, cfg.d = B, H, L, d
+    cfg.c_q, cfg.c_k, cfg.c_h = c_q, c_k, c_h
+    cfg.kq_place, cfg.head_place, cfg.dtype, cfg.path = kq_place, head_place, dtype, path
+    cfg.scale = scale
+    cfg.qkv_row_stride = qkv_row_stride
+    cfg.stream = stream
+    if workspace is not None:
+        cfg.workspace = workspace.data_ptr()
+        cfg.workspace_bytes = workspace.numel() * workspace.element_size()
+    return cfg
+
+
+def _dtype_code(t) -> int:
+    import torch
+    if t.dtype == torch.float32:
+        return F32
+    if t.dtype == torch.bfloat16:
+        return BF16
+    raise TypeError(f"unsupported dtype {t.dtype}")
+
+
+def workspace(nbytes: int, device="cuda"):
+    """A 256-byte aligned device buffer of at least nbytes (torch allocations are)."""
+    import torch
+    return torch.empty(max(int(nbytes), 256), dtype=torch.uint8, device=device)
+
+
+def attn_fwd(q, k, v, theta, w, c_q, c_k, c_h, kq_place=PRE, head_place=POST, *, out=None,
+             ws=None, path=PATH_AUTO, scale=0.0, stream=None, check=False):
+    """MTA attention.  q, k, v: [B, L, H, d] CUDA tensors (fp32 or bf16), dense in
+    (H, d) with a common token stride; theta [H, c_q, c_k] fp32; w [H/c_h, c_h, c_h]
+    fp32.  Returns out [B, L, H, d] (dtype of q)."""
+    import torch
+    B, L, H, d = q.shape
+    for t in (k, v):
+        if t.shape != q.shape or t.stride() != q.stride() or t.dtype != q.dtype:
+            raise ValueError("q, k, v must share shape, strides and dtype")
+    if q.stride(3) != 1 or q.stride(2) != d or q.stride(0) != L * q.stride(1):
+        raise ValueError("q, k, v must be [B, L, H, d] with dense heads and a token stride")
+    if out is None:
+        out = torch.empty((B, L, H, d), dtype=q.dtype, device=q.device)
+    cfg = make_cfg(B, H, L, d, c_q, c_k, c_h, kq_place, head_place, _dtype_code(q), path, scale,
+                   q.stride(1), _stream_handle(stream))
+    if ws is None:
+        ws = workspace(lib().mta_attn_workspace_bytes(ctypes.byref(cfg)), q.device)
+    cfg.workspace, cfg.workspace_bytes = ws.data_ptr(), ws.numel()
+    _check("mta_attn_fwd", lib().mta_attn_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(theta), _ptr(w),
+                                             ctypes.byref(cfg), _ptr(out)))
+    if check:
+        _check("mta_sync_status", lib().mta_sync_status(ctypes.byref(cfg)))
+    return out
+
+
+def depth_scale(layer: int) -> float:
+    return 1.0 - 0.8 * math.exp(-0.3 * layer)
+
+
+def layer_fwd(x, wqkv, theta, w, gamma, beta, wo, H, c_q, c_k, c_h, kq_place=PRE,
+              head_place=POST, *, eps=1e-5, layer=12, lam=-1.0, out=None, ws=None,
+              path=PATH_AUTO, stream=None, check=False):
+    """Full MTA layer, bf16.  x [B, L, D]; wqkv [3D, D]; wo [D, D]; gamma, beta [D]
+    fp32.  Returns out [B, L, D] bf16."""
+    import torch
+    B, L, D = x.shape
+    d = D // H
+    if out is None:
+        out = torch.empty((B, L, D), dtype=x.dtype, device=x.device)
+    cfg = make_cfg(B, H, L, d, c_q, c_k, c_h, kq_place, head_place, _dtype_code(x), path, 0.0, 0,
+                   _stream_handle(stream))
+    if ws is None:
+        ws = workspace(lib().mta_layer_workspace_bytes(ctypes.byref(cfg)), x.device)
+    cfg.workspace, cfg.workspace_bytes = ws.data_ptr(), ws.numel()
+    gn = MtaGn(gamma.data_ptr(), beta.data_ptr(), eps, layer, lam)
+    _check("mta_layer_fwd", lib().mta_layer_fwd(_ptr(x), _ptr(wqkv), _ptr(theta), _ptr(w),
+                                               ctypes.byref(gn), _ptr(wo), ctypes.byref(cfg),
+                                               _ptr(out)))
+    if check:
+        _check("mta_sync_status", lib().mta_sync_status(ctypes.byref(cfg)))
+    return out
+
+
+def layer_workspace_bytes(B, L, H, d, c_q, c_k, c_h, kq_place=PRE, head_place=POST) -> int:
+    cfg = make_cfg(B, H, L, d, c_q, c_k, c_h, kq_place, head_place, BF16)
+    return lib().mta_layer_workspace_bytes(ctypes.byref(cfg))
+
+
+def gemm_bf16_nt(a, b, out=None, stream=None):
+    """C = a b^T for bf16 a [M, K], b [N, K] (contiguous)."""
+    import torch
+    M, K = a.shape
+    N = b.shape[0]
+    if out is None:
+        out = torch.empty((M, N), dtype=torch.bfloat16, device=a.device)
+    _check("mta_gemm_bf16_nt", lib().mta_gemm_bf16_nt(_ptr(a), _ptr(b), _ptr(out), M, N, K,
+                                                     _stream_handle(stream)))
+    return out
+
+
+def group_norm_scale(o, gamma, beta, eps=1e-5, lam=1.0, out=None, stream=None):
+    """Depth-scaled group norm of o [..., H, d] bf16 (dense)."""
+    import torch
+    H, d = o.shape[-2], o.shape[-1]
+    tokens = o.numel() // (H * d)
+    if out is None:
+        out = torch.empty_like(o)
+    gn = MtaGn(gamma.data_ptr(), beta.data_ptr(), eps, 0, lam)
+    _check("mta_group_norm_scale", lib().mta_group_norm_scale(_ptr(o), ctypes.byref(gn), tokens, H,
+                                                             d, _ptr(out), _stream_handle(stream)))
+    return out
