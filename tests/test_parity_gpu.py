@@ -81,10 +81,19 @@ for d in (64, 128):
             SMALL.append((d, hp, L))
 
 
+def tc_applies(wl):
+    """Whether the tensor-core kernel serves this configuration."""
+    return (wl.dtype == "bf16" and wl.d in (64, 128)
+            and (wl.kq_place == synth.OFF or (wl.c_q, wl.c_k) == (6, 11))
+            and (wl.head_place == synth.OFF or (wl.head_place == synth.POST and wl.c_h == 2)))
+
+
 @pytest.mark.parametrize("d,hp,L", SMALL)
-@pytest.mark.parametrize("path", [mta.PATH_AUTO, mta.PATH_SIMT])
+@pytest.mark.parametrize("path", [mta.PATH_AUTO, mta.PATH_SIMT, mta.PATH_TC])
 def test_small_bf16(d, hp, L, path):
     base = synth.WORKLOADS["pretrain_d128_L2048"]
+    if path == mta.PATH_TC and hp == synth.PRE:
+        pytest.skip("pre-softmax head mixing runs on the CUDA-core kernel")
     wl = synth.shrink(base, B=2, H=4, L=L, d=d, head_place=hp, seed=77 + L + d + hp)
     inp = synth.make_attn_inputs(wl)
     assert_close(run_attn(wl, inp, path), oracle_full(wl, inp), "bf16")
@@ -97,7 +106,19 @@ def test_small_bf16_other_kernels(c_q, c_k, c_h, kq):
     wl = synth.shrink(base, B=1, H=8, L=200, d=64, c_q=c_q, c_k=c_k, c_h=c_h, kq_place=kq,
                       head_place=synth.POST if c_h > 1 else synth.OFF, seed=91 + c_q)
     inp = synth.make_attn_inputs(wl)
-    assert_close(run_attn(wl, inp), oracle_full(wl, inp), "bf16")
+    ref = oracle_full(wl, inp)
+    assert_close(run_attn(wl, inp), ref, "bf16")
+    if tc_applies(wl):
+        assert_close(run_attn(wl, inp, mta.PATH_TC), ref, "bf16")
+
+
+def test_tc_path_unsupported_is_reported():
+    base = synth.WORKLOADS["pretrain_d128_L2048"]
+    wl = synth.shrink(base, B=1, H=4, L=64, d=64, head_place=synth.PRE, seed=3)
+    inp = synth.make_attn_inputs(wl)
+    with pytest.raises(mta.MtaError) as e:
+        run_attn(wl, inp, mta.PATH_TC)
+    assert e.value.code == 2
 
 
 def test_strided_qkv_views():
@@ -146,6 +167,7 @@ def sample_rows(wl, n_extra=6, seed=0):
 @pytest.mark.parametrize("name", ["identity_d64_L2048", "pretrain_d128_L2048", "long_d128_L16384"])
 def test_full_size_sampled(name):
     wl = synth.WORKLOADS[name]
+    assert tc_applies(wl)
     inp = synth.make_attn_inputs(wl)
     out = run_attn(wl, inp)
     rows = sample_rows(wl)
