@@ -1,0 +1,518 @@
+"""Benchmark of the MTA forward hot path on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl mine|reference]
+
+One step = one call of the library over one batch of seeded synthetic input
+(mta_attn_fwd for attention workloads, mta_layer_fwd for layer workloads).
+Inputs rotate through three resident sets larger than L2 together, so no step
+reads its inputs from L2 left by the previous one.  Timing: W untimed warm-up
+steps, then K steps bracketed by a barrier and torch.cuda.synchronize(), timed
+with CUDA events on the launch stream; the max over ranks is reported.  Rank 0
+prints one JSON line.
+
+Multi-GPU (torchrun): the (batch, head-group) units of MTA are independent, so
+every rank runs its own copy of the workload (weak scaling, no collective on
+the data path); value = all ranks' tokens / max-over-ranks time.
+
+--impl reference times the fp64 CPU oracle (test infrastructure, oracle/) on a
+bounded sample of the same workload on the host cores; it is a deliberately
+slow baseline, not a target.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from token_attention_b200 import synth  # noqa: E402
+
+METRIC = "MTA fwd tokens/s and TFLOP/s at L=2048 on 1 B200; % of BF16 tensor peak"
+UNIT = "tokens/s"
+DEFAULT_WORKLOAD = "pretrain_d128_L2048"
+N_SETS = 3
+# B200: 148 SMs x 128 fp32 lanes x 2 flop per FMA at the 1965 MHz max SM clock
+FP32_PEAK_TFLOPS = 148 * 128 * 2 * 1.965e9 / 1e12
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+# ---------------------------------------------------------------------------
+# workload arithmetic (algorithmic counts, measurement)
+# ---------------------------------------------------------------------------
+
+def flops(wl: synth.Workload) -> dict:
+    """Algorithmic flops of one step.  Per causal (query, key) pair and head:
+    F_std = 4d (Q K^T and A V), F_mta = F_std + 2 c_q c_k + 2 c_h
+    (the key-query convolution and the head mix).  Layer adds 2 B L D 4D
+    (QKV and output projections)."""
+    P = wl.causal_pairs
+    f_std = 4 * wl.d * P
+    conv = (2 * wl.c_q * wl.c_k if wl.kq_place else 0) * P
+    mix = (2 * wl.c_h if wl.head_place else 0) * P
+    gemm = 2 * wl.B * wl.L * wl.D * 4 * wl.D if wl.layer else 0
+    return {"std": f_std + gemm, "mta": f_std + conv + mix + gemm, "conv": conv, "gemm": gemm,
+            "attn_std": f_std, "attn_mta": f_std + conv + mix}
+
+
+def launches_per_step(wl: synth.Workload) -> int:
+    """Kernels of this library one step launches: the attention kernel; a layer
+    adds the two projection GEMMs, and the stand-alone group norm when the
+    attention runs on the CUDA-core kernel (pre-softmax head mixing)."""
+    if not wl.layer:
+        return 1
+    return 3 if wl.head_place != synth.PRE else 4
+
+
+def read_peaks() -> tuple[dict, str]:
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            return json.load(f), "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def read_traffic(kernel_key: str, workload: str):
+    """dram bytes per launch from a committed ncu summary, if one matches."""
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(p):
+        return None
+    with open(p) as f:
+        t = json.load(f)
+    e = t.get(kernel_key, {}).get(workload)
+    return None if e is None else e.get("bytes_per_launch")
+
+
+# ---------------------------------------------------------------------------
+# clocks during the timed region
+# ---------------------------------------------------------------------------
+
+class ClockSampler:
+    QUERY = ("timestamp,index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+        self.t0 = self.t1 = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.QUERY}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+
+    def mark_begin(self):
+        self.t0 = time.time()
+
+    def mark_end(self):
+        self.t1 = time.time()
+
+    def stop(self) -> dict | None:
+        if self.proc is None:
+            return None
+        time.sleep(0.25)
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+            out, _ = self.proc.communicate()
+        rows = []
+        for line in out.strip().splitlines():
+            f = [x.strip() for x in line.split(",")]
+            if len(f) < 10:
+                continue
+            try:
+                ts = time.mktime(time.strptime(f[0].split(".")[0], "%Y/%m/%d %H:%M:%S"))
+                ts += float("0." + f[0].split(".")[1]) if "." in f[0] else 0.0
+                rows.append((ts, float(f[2]), float(f[3]), f[6:10]))
+            except (ValueError, IndexError):
+                continue
+        if not rows:
+            return None
+        inside = [r for r in rows if self.t0 is not None and self.t0 - 0.15 <= r[0] <= self.t1 + 0.15]
+        use = inside or rows
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in use for i, v in enumerate(r[3]) if v.lower() == "active"})
+        return {"sm_mhz": statistics.median(r[1] for r in use), "sm_max_mhz": max(r[2] for r in use),
+                "reasons": reasons, "samples": len(use), "samples_in_window": len(inside)}
+
+
+# ---------------------------------------------------------------------------
+# the library arm
+# ---------------------------------------------------------------------------
+
+def make_sets(wl, dev, n_sets):
+    import torch
+
+    def to(x, dt):
+        t = torch.from_numpy(np.ascontiguousarray(x)).to(dev)
+        return t.to(torch.bfloat16) if dt == "bf16" else t
+
+    sets = []
+    for s in range(n_sets):
+        w = synth.shrink(wl, seed=wl.seed + 100 * s)
+        if wl.layer:
+            inp = synth.make_layer_inputs(w)
+            sets.append({k: to(inp[k], "bf16" if k in ("x", "wqkv", "wo") else "f32")
+                         for k in ("x", "wqkv", "wo", "theta", "w", "gamma", "beta")})
+        else:
+            inp = synth.make_attn_inputs(w)
+            sets.append({k: to(inp[k], wl.dtype if k in "qkv" else "f32")
+                         for k in ("q", "k", "v", "theta", "w")})
+    return sets
+
+
+def step_fn(wl, mta, sets, ws, outs, stream):
+    """Returns f(i): enqueue step i (input set i % n) on `stream`."""
+    if wl.layer:
+        def f(i):
+            s = sets[i % len(sets)]
+            mta.layer_fwd(s["x"], s["wqkv"], s["theta"], s["w"], s["gamma"], s["beta"], s["wo"],
+                          wl.H, wl.c_q, wl.c_k, wl.c_h, wl.kq_place, wl.head_place, eps=1e-5,
+                          layer=wl.depth, out=outs[i % len(outs)], ws=ws, stream=stream)
+    else:
+        def f(i):
+            s = sets[i % len(sets)]
+            mta.attn_fwd(s["q"], s["k"], s["v"], s["theta"], s["w"], wl.c_q, wl.c_k, wl.c_h,
+                         wl.kq_place, wl.head_place, out=outs[i % len(outs)], ws=ws, stream=stream)
+    return f
+
+
+def run_mine(args, wl, rank, world, local_rank):
+    import torch
+    from token_attention_b200 import mta
+    import ctypes
+
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    mta.lib()
+    stream = torch.cuda.Stream(device=dev)
+    sets = make_sets(wl, dev, N_SETS)
+    out_shape = (wl.B, wl.L, wl.D) if wl.layer else (wl.B, wl.L, wl.H, wl.d)
+    odt = torch.float32 if wl.dtype == "f32" else torch.bfloat16
+    outs = [torch.empty(out_shape, dtype=odt, device=dev) for _ in range(N_SETS)]
+    cfg = mta.make_cfg(wl.B, wl.H, wl.L, wl.d, wl.c_q, wl.c_k, wl.c_h, wl.kq_place, wl.head_place,
+                       mta.F32 if wl.dtype == "f32" else mta.BF16)
+    nbytes = (mta.lib().mta_layer_workspace_bytes if wl.layer else mta.lib().mta_attn_workspace_bytes)(
+        ctypes.byref(cfg))
+    ws = mta.workspace(nbytes, dev)
+    f = step_fn(wl, mta, sets, ws, outs, stream)
+
+    def barrier():
+        if world > 1:
+            import torch.distributed as dist
+            dist.barrier()
+
+    sampler = ClockSampler(local_rank) if not args.no_clocks else None
+    if sampler:
+        sampler.start()
+        time.sleep(0.3)
+    warm = max(3, args.warmup)
+    with torch.cuda.stream(stream):
+        for i in range(warm):
+            f(i)
+    stream.synchronize()
+    # status word of the warm-up calls: no kernel gave up a wait
+    cfg.workspace, cfg.workspace_bytes, cfg.stream = ws.data_ptr(), ws.numel(), stream.cuda_stream
+    st = mta.lib().mta_sync_status(ctypes.byref(cfg))
+    if st != 0:
+        raise RuntimeError(f"warm-up status {mta.STATUS.get(st, st)}")
+
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    barrier()
+    torch.cuda.synchronize()
+    if sampler:
+        sampler.mark_begin()
+    t_begin = torch.cuda.Event(enable_timing=True)
+    t_end = torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(stream):
+        t_begin.record(stream)
+        for i in range(args.steps):
+            starts[i].record(stream)
+            f(warm + i)
+            ends[i].record(stream)
+        t_end.record(stream)
+    stream.synchronize()
+    barrier()
+    torch.cuda.synchronize()
+    if sampler:
+        sampler.mark_end()
+    total_ms = t_begin.elapsed_time(t_end)
+    per_launch = [s.elapsed_time(e) for s, e in zip(starts, ends)]
+    st = mta.lib().mta_sync_status(ctypes.byref(cfg))
+    if st != 0:
+        raise RuntimeError(f"timed-region status {mta.STATUS.get(st, st)}")
+    clocks = sampler.stop() if sampler else None
+
+    # max over ranks
+    t_max = total_ms
+    if world > 1:
+        import torch.distributed as dist
+        t = torch.tensor([total_ms], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        t_max = float(t.item())
+
+    e2e = None
+    if not args.no_e2e:
+        e2e = run_e2e(args, wl, mta, sets, ws, stream, dev, barrier, world)
+    return {"total_ms": t_max, "per_launch_ms": per_launch, "clocks": clocks, "e2e": e2e,
+            "warmup": warm}
+
+
+def run_e2e(args, wl, mta, sets, ws, stream, dev, barrier, world):
+    """Same metric through the public API with host buffers: every step copies
+    its inputs from pinned host memory to the device, runs the call, and reads
+    the result back to pinned host memory."""
+    import torch
+    names = ("x",) if wl.layer else ("q", "k", "v")
+    host_sets = [{n: s[n].cpu().pin_memory() for n in names} for s in sets]
+    dev_in = [{n: torch.empty_like(sets[0][n]) for n in names}]
+    out_shape = (wl.B, wl.L, wl.D) if wl.layer else (wl.B, wl.L, wl.H, wl.d)
+    odt = torch.float32 if wl.dtype == "f32" else torch.bfloat16
+    dout = torch.empty(out_shape, dtype=odt, device=dev)
+    hout = torch.empty(out_shape, dtype=odt).pin_memory()
+    steps = max(3, min(args.steps, args.e2e_steps))
+    h2d = sum(host_sets[0][n].numel() * host_sets[0][n].element_size() for n in names)
+    d2h = hout.numel() * hout.element_size()
+
+    def one(i):
+        hs, s = host_sets[i % len(host_sets)], sets[i % len(sets)]
+        for n in names:
+            dev_in[0][n].copy_(hs[n], non_blocking=True)
+        if wl.layer:
+            mta.layer_fwd(dev_in[0]["x"], s["wqkv"], s["theta"], s["w"], s["gamma"], s["beta"],
+                          s["wo"], wl.H, wl.c_q, wl.c_k, wl.c_h, wl.kq_place, wl.head_place,
+                          layer=wl.depth, out=dout, ws=ws, stream=stream)
+        else:
+            mta.attn_fwd(dev_in[0]["q"], dev_in[0]["k"], dev_in[0]["v"], s["theta"], s["w"],
+                         wl.c_q, wl.c_k, wl.c_h, wl.kq_place, wl.head_place, out=dout, ws=ws,
+                         stream=stream)
+        hout.copy_(dout, non_blocking=True)
+
+    with torch.cuda.stream(stream):
+        for i in range(3):
+            one(i)
+    stream.synchronize()
+    barrier()
+    torch.cuda.synchronize()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(stream):
+        a.record(stream)
+        for i in range(steps):
+            one(i)
+        b.record(stream)
+    stream.synchronize()
+    barrier()
+    ms = a.elapsed_time(b)
+    if world > 1:
+        import torch.distributed as dist
+        t = torch.tensor([ms], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = float(t.item())
+    return {"value": world * wl.tokens * steps / (ms / 1e3), "unit": UNIT,
+            "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h), "steps": steps,
+            "ms_per_step": ms / steps}
+
+
+# ---------------------------------------------------------------------------
+# the oracle on the host cores
+# ---------------------------------------------------------------------------
+
+def blas_threads() -> int:
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i.get("num_threads", 1) for i in threadpool_info() if i.get("user_api") == "blas"]
+        return max(n) if n else 1
+    except Exception:
+        return 1
+
+
+def oracle_sample(wl, budget_s: float, mode: str):
+    """Times the oracle on a bounded sample of the workload.  mode "groups":
+    whole head groups at full length; mode "rows": single query rows of one
+    head group.  Returns (tokens-equivalent/s, seconds, description)."""
+    import oracle as O
+    if wl.layer:
+        inp = synth.make_layer_inputs(wl)
+        rows = [(0, 0)]
+        t = time.perf_counter()
+        O.mta_layer_rows(inp["x"][:1], inp["wqkv"], inp["theta"], inp["w"], inp["gamma"],
+                         inp["beta"], inp["eps"], inp["lam"], inp["wo"], wl.H, wl.c_h, rows,
+                         wl.kq_place, wl.head_place)
+        dt = time.perf_counter() - t
+        return 1 / dt, dt, "1 token of the layer (QKV of its batch, attention window, norm, projection)"
+    inp = synth.make_attn_inputs(wl)
+    q, k, v, th, w = inp["q"], inp["k"], inp["v"], inp["theta"], inp["w"]
+    ch = wl.c_h
+    if mode == "groups":
+        n_units = wl.B * (wl.H // ch)
+        done, t0 = 0, time.perf_counter()
+        for u in range(n_units):
+            b, g = divmod(u, wl.H // ch)
+            hs = slice(g * ch, (g + 1) * ch)
+            O.mta_attention_group(np.ascontiguousarray(q[b, :, hs].transpose(1, 0, 2)),
+                                  np.ascontiguousarray(k[b, :, hs].transpose(1, 0, 2)),
+                                  np.ascontiguousarray(v[b, :, hs].transpose(1, 0, 2)),
+                                  th[hs], w[g], np.arange(wl.L), 1 / math.sqrt(wl.d),
+                                  wl.kq_place, wl.head_place)
+            done += 1
+            if time.perf_counter() - t0 > budget_s:
+                break
+        dt = time.perf_counter() - t0
+        tok = done * ch / wl.H * wl.L
+        return tok / dt, dt, (f"{done} of {n_units} (batch, head-group) units at full length "
+                              f"L={wl.L} ({tok:.0f} token-equivalents)")
+    # rows of one head group, spread over the sequence
+    rng = np.random.default_rng(0)
+    done, t0 = 0, time.perf_counter()
+    g = 0
+    hs = slice(0, ch)
+    while True:
+        i = int(rng.integers(wl.L))
+        O.mta_attention_rows(q[:1, :, hs], k[:1, :, hs], v[:1, :, hs], th[hs], w[g:g + 1], ch,
+                             [(0, i)], wl.kq_place, wl.head_place)
+        done += 1
+        if time.perf_counter() - t0 > budget_s:
+            break
+    dt = time.perf_counter() - t0
+    tok = done * ch / wl.H
+    return tok / dt, dt, f"{done} single query rows of one head group (uniform positions)"
+
+
+def run_reference(args, wl, rank):
+    if rank != 0:
+        return None
+    budget_total = 150.0
+    nsteps = max(1, args.steps) + max(3, args.warmup)
+    per_step = max(0.02, min(2.0, budget_total / nsteps))
+    # warm-up steps (untimed), then timed steps
+    for _ in range(max(3, args.warmup)):
+        oracle_sample(wl, per_step, "rows")
+    vals, secs = [], 0.0
+    desc = ""
+    for _ in range(max(1, args.steps)):
+        v, s, desc = oracle_sample(wl, per_step, "rows")
+        vals.append(v)
+        secs += s
+    value = statistics.mean(vals)
+    return {"value": value, "seconds": secs, "sample": desc, "cores": blas_threads()}
+
+
+# ---------------------------------------------------------------------------
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--warmup", type=int, default=50)
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(synth.WORKLOADS))
+    ap.add_argument("--impl", default="mine", choices=["mine", "reference"])
+    ap.add_argument("--cpu-budget", type=float, default=15.0,
+                    help="seconds of oracle work for the cpu_baseline (rank 0, N=1)")
+    ap.add_argument("--e2e-steps", type=int, default=50)
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu", action="store_true")
+    ap.add_argument("--no-clocks", action="store_true")
+    args = ap.parse_args()
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    wl = synth.WORKLOADS[args.workload]
+    fl = flops(wl)
+    config = {"workload": wl.name, "B": wl.B, "H": wl.H, "L": wl.L, "d": wl.d, "c_q": wl.c_q,
+              "c_k": wl.c_k, "c_h": wl.c_h, "kq_place": ["off", "pre", "post"][wl.kq_place],
+              "head_place": ["off", "pre", "post"][wl.head_place],
+              "parallelism": f"replicas x{max(world, args.gpus)}" if max(world, args.gpus) > 1 else "single",
+              "l2": f"{N_SETS} rotating input sets, each step reads a set not touched by the previous step"}
+    if wl.layer:
+        config["D"] = wl.D
+
+    if args.impl == "reference":
+        r = run_reference(args, wl, rank)
+        if r is None:
+            return 0
+        line = {"impl": "reference", "metric": METRIC, "value": r["value"], "unit": UNIT,
+                "n_gpus": args.gpus, "steps": args.steps, "warmup": max(3, args.warmup),
+                "ms_per_step": 1e3 * r["seconds"] / max(1, args.steps), "higher_is_better": True,
+                "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+                "config": config,
+                "cpu_baseline": {"value": r["value"], "unit": UNIT, "cores": r["cores"],
+                                 "kind": "oracle", "sample": r["sample"]},
+                "e2e": {"value": r["value"], "unit": UNIT, "h2d_bytes_per_step": 0,
+                        "d2h_bytes_per_step": 0}}
+        print(json.dumps(line), flush=True)
+        return 0
+
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    res = run_mine(args, wl, rank, world, local_rank)
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+    if rank != 0:
+        return 0
+
+    ms = res["total_ms"]
+    value = world * wl.tokens * args.steps / (ms / 1e3)
+    launch_ms = statistics.mean(res["per_launch_ms"])
+    peaks, peak_src = read_peaks()
+    s = launch_ms / 1e3
+    if wl.layer:
+        kernel = "mta_layer_fwd"
+        achieved = fl["mta"] / s / 1e12
+        roof = {"bound": "tensor", "achieved": achieved, "peak": peaks["bf16_tflops"],
+                "unit": "TFLOP/s", "frac": achieved / peaks["bf16_tflops"],
+                "traffic": read_traffic("layer", wl.name),
+                "kernel": "layer step (QKV GEMM + fused attention + output GEMM)",
+                "per_unit": "F_mta per causal pair-head + 8 B L D^2 GEMM flops",
+                "peak_source": f"{peak_src} bf16 burst"}
+    else:
+        kernel = "attn_tc_kernel"
+        achieved = fl["conv"] / s / 1e12
+        roof = {"bound": "alu", "achieved": achieved, "peak": FP32_PEAK_TFLOPS, "unit": "TFLOP/s",
+                "frac": achieved / FP32_PEAK_TFLOPS,
+                "traffic": read_traffic("attn_tc_kernel", wl.name),
+                "kernel": kernel,
+                "per_unit": f"2*c_q*c_k = {2 * wl.c_q * wl.c_k} fp32 flop per causal pair-head "
+                            f"(key-query convolution), x {wl.causal_pairs} pair-heads per launch",
+                "peak_source": "148 SMs x 128 FP32 lanes x 2 x 1965 MHz"}
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": res["warmup"], "ms_per_step": ms / args.steps, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16" if wl.dtype == "bf16" else "f32",
+        "data": "synthetic", "config": config,
+        "tflops": {"std": fl["std"] / s / 1e12, "mta": fl["mta"] / s / 1e12},
+        "pct_bf16_peak": {"std": fl["std"] / s / 1e12 / peaks["bf16_tflops"],
+                          "mta": fl["mta"] / s / 1e12 / peaks["bf16_tflops"],
+                          "peak_tflops": peaks["bf16_tflops"], "peak_source": peak_src},
+        "roofline": roof, "gpu_launches": args.steps * launches_per_step(wl),
+        "clocks": res["clocks"], "e2e": res["e2e"],
+    }
+    if world == 1 and not args.no_cpu:
+        v, secs, desc = oracle_sample(wl, args.cpu_budget, "groups" if not wl.layer else "rows")
+        line["cpu_baseline"] = {"value": v, "unit": UNIT, "cores": blas_threads(), "kind": "oracle",
+                                "sample": f"{desc}; {secs:.1f} s"}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

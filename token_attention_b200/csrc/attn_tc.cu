@@ -83,6 +83,8 @@ struct Geo {
   static constexpr int NS = (BN + 2 * C + 15) / 16 * 16;  // S columns (MMA N)
   static constexpr int NDC = D / 64;                  // 64-element (128-byte) d chunks
   static constexpr int WIN = 32 + 2 * C;              // convolution window per 32 keys
+  static constexpr int NP = (WIN + 1) / 2;            // aligned pairs of the window
+  static constexpr int NS2 = (WIN - 1) / 2 > 0 ? (WIN - 1) / 2 : 1;  // shifted pairs
   static constexpr int SSTR0 = (WIN + 3) / 4 * 4;
   static constexpr int SSTR = (SSTR0 % 8 == 0) ? SSTR0 + 4 : SSTR0;  // conflict-free rows
   static constexpr int NV = CH;                       // destination heads (V tiles)
@@ -131,7 +133,14 @@ struct TcParams {
   unsigned *err;
 };
 
-// acc[jj] += sum_t th[t] * X[jj + 2C - t]   (keys j - (t - C) of one query row)
+__device__ __forceinline__ float ex2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+// One query row of the key-query convolution for 32 output keys:
+//   acc[jj] += sum_t th[t] * X[jj + 2C - t]      (key j - (t - C) of the row)
 template <int CK, int WIN>
 __device__ __forceinline__ void conv_row(float (&acc)[32], const float (&X)[WIN], const float *th) {
   constexpr int C = CK / 2;
@@ -155,13 +164,13 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint8_t *Vs = smem + G::OFF_V;
   uint8_t *Ps = smem + G::OFF_P;
   float *Scr = reinterpret_cast<float *>(smem + G::OFF_SCR);
-  float *small = reinterpret_cast<float *>(smem + G::OFF_SMALL);
-  float *th_s = small;                    // [CQ*CK] (scaled)
-  float *w_s = small + 64 + 64;           // [CH*CH] -> offset 128
-  float *redmax = small + 256;            // [2 parity][2 wg][128]
-  float *redsum = small + 256 + 512;      // [2][128]
-  float *redgn = small + 256 + 512 + 256; // [2][128]
-  uint64_t *bars = reinterpret_cast<uint64_t *>(small + 256 + 512 + 512);
+  uint8_t *small = smem + G::OFF_SMALL;
+  float *th_s = reinterpret_cast<float *>(small);             // [CQ*CK], scaled
+  float *w_s = reinterpret_cast<float *>(small + 1024);       // [CH*CH]
+  float *redmax = reinterpret_cast<float *>(small + 1088);    // [2 parity][2 wg][128]
+  float *redsum = reinterpret_cast<float *>(small + 3136);    // [2 wg][128]
+  float *redgn = reinterpret_cast<float *>(small + 4160);     // [2 wg][128]
+  uint64_t *bars = reinterpret_cast<uint64_t *>(small + 5184);
   uint64_t *q_full = bars + 0, *k_full = bars + 1, *k_empty = bars + 2, *v_full = bars + 3;
   uint64_t *v_empty = bars + 4, *s_full = bars + 5, *s_free = bars + 6, *p_full = bars + 7;
   uint64_t *mma_done = bars + 8;
@@ -188,8 +197,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
   if (threadIdx.x >= 64 && threadIdx.x < 64 + CQ * CK) {
     const int i = threadIdx.x - 64;
-    const float th = p.theta ? p.theta[static_cast<long long>(h) * CQ * CK + i] : 1.f;
-    th_s[i] = th * (p.qk_scale * kLog2e);
+    const float th = (p.theta ? p.theta[static_cast<long long>(h) * CQ * CK + i] : 1.f) *
+                     (p.qk_scale * kLog2e);
+    th_s[i] = th;
   }
   if (threadIdx.x >= 192 && threadIdx.x < 192 + CH * CH)
     w_s[threadIdx.x - 192] = p.w[static_cast<long long>(g) * CH * CH + (threadIdx.x - 192)];
@@ -321,9 +331,11 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int k = G::WIN / 4 * 4; k < G::WIN; ++k) my[k] = X[k];
           named_bar_sync(1 + wg, 128);
         }
-        if (out_row) {
+        // a warp whose 32 rows all precede the chunk's first key has nothing to compute
+        const bool live = (j0 + cb) <= (row0 + 32 * q4 + 31);
+        if (out_row && live) {
           conv_row<CK, G::WIN>(acc, X, th_s);
-#pragma unroll
+#pragma unroll 1
           for (int a = 1; a < CQ; ++a) {
             const float *src = scr + (r - a) * G::SSTR;
             float Y[G::WIN];
@@ -391,8 +403,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       uint32_t pk[32];
 #pragma unroll
       for (int jj = 0; jj < 64; jj += 2) {
-        const float p0 = out_row ? exp2f(cv[jj] - m_run) : 0.f;
-        const float p1 = out_row ? exp2f(cv[jj + 1] - m_run) : 0.f;
+        const float p0 = out_row ? ex2(cv[jj] - m_run) : 0.f;
+        const float p1 = out_row ? ex2(cv[jj + 1] - m_run) : 0.f;
         ls += p0 + p1;
         pk[jj >> 1] = pack_bf16x2(p0, p1);
       }

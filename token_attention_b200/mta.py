@@ -12,7 +12,9 @@ import math
 import os
 
 HERE = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(HERE, "libmta.so")
+# MTA_LIB selects another build of the library (for comparing builds); default:
+# the in-tree libmta.so next to this file.
+LIB_PATH = os.environ.get("MTA_LIB") or os.path.join(HERE, "libmta.so")
 
 OFF, PRE, POST = 0, 1, 2
 F32, BF16 = 0, 1
