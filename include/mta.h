@@ -130,6 +130,27 @@ mta_status mta_layer_fwd(const void *x, const void *Wqkv, const float *theta,
                          const float *w_head, const mta_gn *gn, const void *Wo,
                          const mta_cfg *cfg, void *out);
 
+/* mta_layer_fwd without a caller-supplied workspace.  The paper has no
+ * counterpart to this entry point; it exists for callers that cannot allocate
+ * device memory (for example a runtime that is handed device pointers to its
+ * inputs and outputs by another component and has no allocator of its own, or
+ * a loop that must not call cudaMalloc because allocation can synchronise the
+ * device).  The layer's scratch lives in a static device buffer of
+ * MTA_STATIC_SCRATCH_BYTES inside the library, which every GPU that loads the
+ * library holds until the process exits.  cfg->workspace and
+ * cfg->workspace_bytes are ignored; everything else is as for mta_layer_fwd.
+ * Returns MTA_ERR_WORKSPACE, enqueuing nothing, when mta_layer_workspace_bytes(cfg)
+ * exceeds MTA_STATIC_SCRATCH_BYTES.  The first call on a device looks up the
+ * buffer's address on that device (make it before any stream capture).  All
+ * calls on a device share the buffer: calls that overlap on the GPU race, so
+ * order them on one stream.  A bounded wait that runs out is recorded in the
+ * static buffer and is not reported; use mta_layer_fwd with a workspace and
+ * mta_sync_status to observe it.  Allocates no memory. */
+#define MTA_STATIC_SCRATCH_BYTES (16u * 1024u * 1024u)
+mta_status mta_layer_fwd_static(const void *x, const void *Wqkv, const float *theta,
+                                const float *w_head, const mta_gn *gn, const void *Wo,
+                                const mta_cfg *cfg, void *out);
+
 /* Building blocks of mta_layer_fwd, exposed for testing and timing. */
 
 /* C[M][N] = A[M][K] * Bm[N][K]^T, bf16 in, fp32 accumulate, bf16 out.

@@ -26,7 +26,7 @@ STATUS = {0: "MTA_OK", 1: "MTA_ERR_INVALID", 2: "MTA_ERR_UNSUPPORTED", 3: "MTA_E
 # Every function include/mta.h declares.
 EXPORTS = ["mta_attn_workspace_bytes", "mta_attn_fwd", "mta_layer_workspace_bytes",
            "mta_layer_fwd", "mta_gemm_bf16_nt", "mta_group_norm_scale", "mta_sync_status",
-           "mta_status_string", "mta_abi_version"]
+           "mta_status_string", "mta_abi_version", "mta_layer_fwd_static"]
 
 
 class MtaCfg(ctypes.Structure):
