@@ -16,15 +16,17 @@
 //     convolution reads) and, per key tile of 128, the key rows j0-c .. j0+128+c
 //     (c = c_k/2 column halo), 128-byte swizzled.
 //   * One thread issues tcgen05.mma: S = Q K^T (M=128, N=144, fp32 in tensor
-//     memory), then Z_hd += P V^hd for every destination head hd of the group.
-//   * Two warpgroups of 128 threads (one TMEM lane = one query row per thread,
-//     one warpgroup per 64 output keys) read S with tcgen05.ld, apply Mask_0,
-//     share rows through a shared-memory window (the convolution needs the c_q-1
-//     rows above), convolve with theta (fp32 FMA, 1/sqrt(d) and log2(e) folded
-//     into theta), apply Mask_-inf, keep an exact online softmax (the
-//     convolution is local and precedes the row max; the running max is only
-//     moved when it grows by more than 2^8, and the accumulators are rescaled
-//     then), and write P (bf16) into the operand tile of the next MMA.
+//     memory), then Z_hd += P V^hd for every destination head hd of the group,
+//     with P read from tensor memory.
+//   * Four warpgroups of 128 threads (one TMEM lane = one query row per thread,
+//     one warpgroup per 32 output keys) read S with tcgen05.ld, apply Mask_0,
+//     publish their columns to a shared-memory copy of the masked tile (the
+//     convolution needs the c_q-1 rows above and c columns on each side),
+//     convolve with theta (fp32 FMA, 1/sqrt(d) and log2(e) folded into theta),
+//     apply Mask_-inf, keep an exact online softmax (the convolution is local
+//     and precedes the row max; the running max is only moved when it grows by
+//     more than 2^8, and the accumulators are rescaled then), and write P
+//     (bf16, two keys per 32-bit column) into tensor memory for the next MMA.
 //   * Post-softmax mixing (c_h = 2): the two heads of a group run as a 2-CTA
 //     cluster.  CTA s accumulates Z_{s->h} = P^s V^h for both destination heads h
 //     and, at the end, sends Z_{s->peer} / l_s to the peer through distributed
@@ -44,7 +46,14 @@ namespace {
 
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kRescaleLog2 = 8.0f;  // move the running max only when it grows by > 2^8
-constexpr int kThreads = 320;         // warp 0 TMA, warp 1 MMA, warps 2..9 softmax/conv
+constexpr int kConvWarps = 16;        // four warpgroups
+constexpr int kThreads = 64 + 32 * kConvWarps;  // warp 0 TMA, warp 1 MMA, warps 2..17 softmax/conv
+constexpr int kConvThreads = 32 * kConvWarps;
+
+// named barriers (0 is __syncthreads)
+constexpr int kBarScratch = 1;  // masked S tile published to shared memory
+constexpr int kBarMax = 2;      // row maxima exchanged between warpgroups
+constexpr int kBarSum = 3;      // row sums exchanged (end of the key loop)
 
 // ---------------------------------------------------------------------------
 // cluster helpers (distributed shared memory)
@@ -70,6 +79,23 @@ __device__ __forceinline__ void drain_wait(uint64_t *bar, uint32_t parity) {
     if (globaltimer_ns() - t0 > kWaitLimitNs) return;
 }
 
+// D[tmem] (+)= A[tmem] * B[smem], kind::f16 (bf16 A packed two per 32-bit column).
+__device__ __forceinline__ void mma_bf16_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc,
+                                            uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+__device__ __forceinline__ float ex2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
 // ---------------------------------------------------------------------------
 // compile-time geometry
 // ---------------------------------------------------------------------------
@@ -82,43 +108,44 @@ struct Geo {
   static constexpr int BN = 128;                      // output keys per key tile
   static constexpr int NS = (BN + 2 * C + 15) / 16 * 16;  // S columns (MMA N)
   static constexpr int NDC = D / 64;                  // 64-element (128-byte) d chunks
-  static constexpr int WIN = 32 + 2 * C;              // convolution window per 32 keys
-  static constexpr int NP = (WIN + 1) / 2;            // aligned pairs of the window
-  static constexpr int NS2 = (WIN - 1) / 2 > 0 ? (WIN - 1) / 2 : 1;  // shifted pairs
-  static constexpr int SSTR0 = (WIN + 3) / 4 * 4;
+  static constexpr int KW = 32;                       // output keys per warpgroup
+  static constexpr int WIN = KW + 2 * C;              // convolution window of a warpgroup
+  static constexpr int SCOLS = BN + 2 * C;            // columns of the shared masked tile
+  static constexpr int SSTR0 = (SCOLS + 3) / 4 * 4;
   static constexpr int SSTR = (SSTR0 % 8 == 0) ? SSTR0 + 4 : SSTR0;  // conflict-free rows
   static constexpr int NV = CH;                       // destination heads (V tiles)
+  static constexpr int DQ = D / 4;                    // output columns per warpgroup
   // shared memory (bytes)
   static constexpr int Q_BYTES = BM * D * 2;
+  static constexpr int Q_CHUNK = BM * 128;
   static constexpr int K_CHUNK = NS * 128;
   static constexpr int K_BYTES = NS * D * 2;
   static constexpr int V_CHUNK = BN * 128;
   static constexpr int V_HEAD = BN * D * 2;
   static constexpr int V_BYTES = NV * V_HEAD;
-  static constexpr int P_CHUNK = BM * 128;
-  static constexpr int P_BYTES = BM * BN * 2;
-  static constexpr int SCR_BYTES = 2 * BM * SSTR * 4;
+  static constexpr int SCR_BYTES = (CQ > 1 || CH == 2) ? BM * SSTR * 4 : 0;  // also the exchange buffer
   static constexpr int OFF_Q = 0;
   static constexpr int OFF_K = OFF_Q + Q_BYTES;
   static constexpr int OFF_V = OFF_K + K_BYTES;
-  static constexpr int OFF_P = OFF_V + V_BYTES;
-  static constexpr int OFF_SCR = OFF_P + P_BYTES;
-  static constexpr int OFF_SMALL = OFF_SCR + SCR_BYTES;
-  static constexpr int SMALL_BYTES = 8192;
-  static constexpr int SMEM = OFF_SMALL + SMALL_BYTES + 1024;
-  // exchange buffer for the post-softmax mix (reuses V and P after the loop)
+  static constexpr int OFF_SCR = OFF_V + V_BYTES;
+  static constexpr int OFF_SMALL = (OFF_SCR + SCR_BYTES + 1023) / 1024 * 1024;
+  static constexpr int SMALL_BYTES = 10240;
+  static constexpr int SMEM_USED = OFF_SMALL + SMALL_BYTES + 1024;
+  // at least half the SM's shared memory, so that one CTA runs per SM and the
+  // 512-column TMEM allocation never waits for another CTA
+  static constexpr int SMEM = SMEM_USED > 232448 / 2 + 1024 ? SMEM_USED : 232448 / 2 + 1024;
+  // exchange buffer for the post-softmax mix (reuses V and the scratch after the loop)
   static constexpr int XSTR = D + 4;
   // tensor memory columns
   static constexpr uint32_t TMEM_COLS = 512;
   static constexpr uint32_t S_COL = 0;
+  static constexpr uint32_t P_COL = 160;   // 64 columns: 128 keys of bf16, two per column
   static constexpr uint32_t Z_COL0 = 256;
-  static_assert(NS <= 256 && NS % 16 == 0, "S tile");
+  static_assert(NS <= 160 && NS % 16 == 0, "S tile");
   static_assert(Z_COL0 + 128 * (NV - 1) + D <= TMEM_COLS, "tensor memory");
-  static_assert(OFF_K % 1024 == 0 && OFF_V % 1024 == 0 && OFF_P % 1024 == 0, "swizzle alignment");
-  static_assert(CH == 1 || BM * XSTR * 4 <= V_BYTES + P_BYTES, "exchange buffer");
+  static_assert(OFF_K % 1024 == 0 && OFF_V % 1024 == 0, "swizzle alignment");
+  static_assert(CH == 1 || BM * XSTR * 4 <= V_BYTES + SCR_BYTES, "exchange buffer");
   static_assert(SMEM <= 232448, "shared memory");
-  // one CTA per SM, so the 512-column TMEM allocation never waits for another CTA
-  static_assert(SMEM > 232448 / 2, "exclusive residency");
 };
 
 struct TcParams {
@@ -133,12 +160,6 @@ struct TcParams {
   unsigned *err;
 };
 
-__device__ __forceinline__ float ex2(float x) {
-  float y;
-  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
-  return y;
-}
-
 // One query row of the key-query convolution for 32 output keys:
 //   acc[jj] += sum_t th[t] * X[jj + 2C - t]      (key j - (t - C) of the row)
 template <int CK, int WIN>
@@ -152,6 +173,18 @@ __device__ __forceinline__ void conv_row(float (&acc)[32], const float (&X)[WIN]
   }
 }
 
+template <int N>
+__device__ __forceinline__ float tree_max(const float (&x)[N]) {
+  float m[N / 2];
+#pragma unroll
+  for (int i = 0; i < N / 2; ++i) m[i] = fmaxf(x[2 * i], x[2 * i + 1]);
+#pragma unroll
+  for (int s = N / 4; s >= 1; s >>= 1)
+#pragma unroll
+    for (int i = 0; i < s; ++i) m[i] = fmaxf(m[i], m[i + s]);
+  return m[0];
+}
+
 template <int D, int CQ, int CK, int CH>
 __global__ void __launch_bounds__(kThreads, 1)
     attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
@@ -162,15 +195,14 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint8_t *Qs = smem + G::OFF_Q;
   uint8_t *Ks = smem + G::OFF_K;
   uint8_t *Vs = smem + G::OFF_V;
-  uint8_t *Ps = smem + G::OFF_P;
   float *Scr = reinterpret_cast<float *>(smem + G::OFF_SCR);
   uint8_t *small = smem + G::OFF_SMALL;
   float *th_s = reinterpret_cast<float *>(small);             // [CQ*CK], scaled
-  float *w_s = reinterpret_cast<float *>(small + 1024);       // [CH*CH]
-  float *redmax = reinterpret_cast<float *>(small + 1088);    // [2 parity][2 wg][128]
-  float *redsum = reinterpret_cast<float *>(small + 3136);    // [2 wg][128]
-  float *redgn = reinterpret_cast<float *>(small + 4160);     // [2 wg][128]
-  uint64_t *bars = reinterpret_cast<uint64_t *>(small + 5184);
+  float *w_s = reinterpret_cast<float *>(small + 512);        // [CH*CH]
+  float *redmax = reinterpret_cast<float *>(small + 1024);    // [2 parity][4 wg][128]
+  float *redsum = reinterpret_cast<float *>(small + 5120);    // [4 wg][128]
+  float *redgn = reinterpret_cast<float *>(small + 7168);     // [4 wg][128]
+  uint64_t *bars = reinterpret_cast<uint64_t *>(small + 9216);
   uint64_t *q_full = bars + 0, *k_full = bars + 1, *k_empty = bars + 2, *v_full = bars + 3;
   uint64_t *v_empty = bars + 4, *s_full = bars + 5, *s_free = bars + 6, *p_full = bars + 7;
   uint64_t *mma_done = bars + 8;
@@ -190,19 +222,18 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (threadIdx.x == 0) {
     mbar_init(q_full, 1); mbar_init(k_full, 1); mbar_init(k_empty, 1); mbar_init(v_full, 1);
-    mbar_init(v_empty, 1); mbar_init(s_full, 1); mbar_init(s_free, 8); mbar_init(p_full, 8);
-    mbar_init(mma_done, 1);
+    mbar_init(v_empty, 1); mbar_init(s_full, 1); mbar_init(s_free, kConvWarps);
+    mbar_init(p_full, kConvWarps); mbar_init(mma_done, 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
   if (threadIdx.x >= 64 && threadIdx.x < 64 + CQ * CK) {
     const int i = threadIdx.x - 64;
-    const float th = (p.theta ? p.theta[static_cast<long long>(h) * CQ * CK + i] : 1.f) *
-                     (p.qk_scale * kLog2e);
-    th_s[i] = th;
+    th_s[i] = (p.theta ? p.theta[static_cast<long long>(h) * CQ * CK + i] : 1.f) *
+              (p.qk_scale * kLog2e);
   }
-  if (threadIdx.x >= 192 && threadIdx.x < 192 + CH * CH)
-    w_s[threadIdx.x - 192] = p.w[static_cast<long long>(g) * CH * CH + (threadIdx.x - 192)];
+  if (threadIdx.x >= 256 && threadIdx.x < 256 + CH * CH)
+    w_s[threadIdx.x - 256] = p.w[static_cast<long long>(g) * CH * CH + (threadIdx.x - 256)];
   if (warp == 1) { tmem_alloc(tslot, G::TMEM_COLS); tmem_relinquish(); }
   tc_fence_before();
   __syncthreads();
@@ -211,19 +242,29 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (warp == 0) {
     // ------------------------------------------------------------------ TMA
+    // Two independent streams: lane 0 loads Q and the key tiles (a key tile is
+    // requested as soon as the previous QK^T has consumed the buffer), lane 1
+    // loads the value tiles (after the previous P V has consumed theirs).
     if (lane == 0) {
-      prefetch_tmap(&tmQ); prefetch_tmap(&tmK); prefetch_tmap(&tmV);
+      prefetch_tmap(&tmQ); prefetch_tmap(&tmK);
       mbar_arrive_expect_tx(q_full, G::Q_BYTES);
 #pragma unroll
-      for (int dc = 0; dc < G::NDC; ++dc) tma_load_4d(Qs + dc * G::P_CHUNK, &tmQ, q_full, dc * 64, h, row0, b);
-      int nk = 0, nv = 0;
+      for (int dc = 0; dc < G::NDC; ++dc) tma_load_4d(Qs + dc * G::Q_CHUNK, &tmQ, q_full, dc * 64, h, row0, b);
+      int nk = 0;
       for (int t = 0; t < n_kv; ++t) {
-        const int j0 = t * G::BN;
         if (!mbar_wait(k_empty, (t & 1) ^ 1, abort_flag, p.err)) break;
         mbar_arrive_expect_tx(k_full, G::K_BYTES);
 #pragma unroll
-        for (int dc = 0; dc < G::NDC; ++dc) tma_load_4d(Ks + dc * G::K_CHUNK, &tmK, k_full, dc * 64, h, j0 - G::C, b);
+        for (int dc = 0; dc < G::NDC; ++dc)
+          tma_load_4d(Ks + dc * G::K_CHUNK, &tmK, k_full, dc * 64, h, t * G::BN - G::C, b);
         ++nk;
+      }
+      drain_wait(q_full, 0);
+      if (*abort_flag && nk) drain_wait(k_full, (nk - 1) & 1);  // copies in flight land first
+    } else if (lane == 1) {
+      prefetch_tmap(&tmV);
+      int nv = 0;
+      for (int t = 0; t < n_kv; ++t) {
         if (!mbar_wait(v_empty, (t & 1) ^ 1, abort_flag, p.err)) break;
         mbar_arrive_expect_tx(v_full, G::V_BYTES);
 #pragma unroll
@@ -231,22 +272,18 @@ __global__ void __launch_bounds__(kThreads, 1)
           const int hv = (CH == 1) ? h : g * CH + hd;
 #pragma unroll
           for (int dc = 0; dc < G::NDC; ++dc)
-            tma_load_4d(Vs + hd * G::V_HEAD + dc * G::V_CHUNK, &tmV, v_full, dc * 64, hv, j0, b);
+            tma_load_4d(Vs + hd * G::V_HEAD + dc * G::V_CHUNK, &tmV, v_full, dc * 64, hv, t * G::BN, b);
         }
         ++nv;
       }
-      drain_wait(q_full, 0);
-      if (*abort_flag) {  // let copies in flight land before the CTA ends
-        if (nk) drain_wait(k_full, (nk - 1) & 1);
-        if (nv) drain_wait(v_full, (nv - 1) & 1);
-      }
+      if (*abort_flag && nv) drain_wait(v_full, (nv - 1) & 1);
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------------ MMA
     if (lane == 0) {
       const uint32_t idesc_qk = idesc_bf16_f32(128, G::NS, 0, 0);
       const uint32_t idesc_pv = idesc_bf16_f32(128, D, 0, 1);
-      const uint32_t q_base = smem_u32(Qs), k_base = smem_u32(Ks), v_base = smem_u32(Vs), p_base = smem_u32(Ps);
+      const uint32_t q_base = smem_u32(Qs), k_base = smem_u32(Ks), v_base = smem_u32(Vs);
       bool ok = mbar_wait(q_full, 0, abort_flag, p.err);
       auto issue_qk = [&](int t) -> bool {
         if (!mbar_wait(k_full, t & 1, abort_flag, p.err)) return false;
@@ -255,7 +292,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk)
           mma_bf16_ss(tmem + G::S_COL,
-                      sdesc_sw128(q_base + (kk >> 2) * G::P_CHUNK + (kk & 3) * 32, 16, 1024),
+                      sdesc_sw128(q_base + (kk >> 2) * G::Q_CHUNK + (kk & 3) * 32, 16, 1024),
                       sdesc_sw128(k_base + (kk >> 2) * G::K_CHUNK + (kk & 3) * 32, 16, 1024), idesc_qk,
                       kk > 0);
         mma_commit(k_empty);
@@ -272,8 +309,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int hd = 0; hd < G::NV; ++hd)
 #pragma unroll
           for (int kk = 0; kk < G::BN / 16; ++kk)
-            mma_bf16_ss(tmem + G::Z_COL0 + 128 * hd,
-                        sdesc_sw128(p_base + (kk >> 2) * G::P_CHUNK + (kk & 3) * 32, 16, 1024),
+            mma_bf16_ts(tmem + G::Z_COL0 + 128 * hd, tmem + G::P_COL + 8 * kk,
                         sdesc_sw128(v_base + hd * G::V_HEAD + kk * 16 * 128, G::V_CHUNK, 1024),
                         idesc_pv, (t > 0 || kk > 0));
         mma_commit(v_empty);
@@ -283,89 +319,81 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else {
     // ------------------------------------------------------- softmax / conv
-    const int wg = (warp - 2) >> 2;      // 0: keys 0..63 of a tile, 1: keys 64..127
+    const int wg = (warp - 2) >> 2;      // warpgroup: output keys 32*wg .. 32*wg+31 of a tile
     const int q4 = warp & 3;             // TMEM lane quadrant of this warp
     const int r = 32 * q4 + lane;        // S row = TMEM lane
     const int qrow = row0 + r;           // query index of this row
     const bool out_row = r >= G::HALO;   // rows below the halo produce outputs
     const uint32_t tl = tmem + (static_cast<uint32_t>(32 * q4) << 16);
-    float *scr = Scr + wg * G::BM * G::SSTR;
+    const int cb = G::KW * wg;           // first output key (tile-relative) of this warpgroup
     float m_run = -INFINITY, l_part = 0.f;
 
     for (int t = 0; t < n_kv; ++t) {
       const int j0 = t * G::BN;
       mbar_wait(s_full, t & 1, abort_flag, p.err);
       tc_fence_after();
-      float cv[64];
+      uint32_t u0[32], u1[16];
+      tmem_ld32(tl + G::S_COL + cb, u0);
+      if (G::WIN > 32) tmem_ld16(tl + G::S_COL + cb + 32, u1);
+      tmem_wait_ld();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(s_free);
+      float X[G::WIN];
 #pragma unroll
-      for (int ch = 0; ch < 2; ++ch) {
-        const int cb = 64 * wg + 32 * ch;  // first output key (tile-relative) of this chunk
-        uint32_t u0[32], u1[16];
-        tmem_ld32(tl + G::S_COL + cb, u0);
-        if (G::WIN > 32) tmem_ld16(tl + G::S_COL + cb + 32, u1);
-        tmem_wait_ld();
-        if (ch == 1) {
-          tc_fence_before();
-          __syncwarp();
-          if (lane == 0) mbar_arrive(s_free);
-        }
-        float X[G::WIN];
+      for (int k = 0; k < G::WIN; ++k) X[k] = __uint_as_float(k < 32 ? u0[k] : u1[(k - 32) & 15]);
+      // Mask_0: keys after this row's query count as 0 inside the convolution
+      const int key0 = j0 - G::C + cb;  // key of window element 0
+      if (key0 + G::WIN - 1 > qrow) {
 #pragma unroll
-        for (int k = 0; k < G::WIN; ++k) X[k] = __uint_as_float(k < 32 ? u0[k] : u1[(k - 32) & 15]);
-        // Mask_0: keys after this row's query count as 0 inside the convolution
-        const int key0 = j0 - G::C + cb;  // key of window element 0
-        if (key0 + G::WIN - 1 > qrow) {
+        for (int k = 0; k < G::WIN; ++k)
+          if (key0 + k > qrow) X[k] = 0.f;
+      }
+      if (CQ > 1) {  // publish this warpgroup's columns of the masked tile
+        float *my = Scr + r * G::SSTR + cb;
 #pragma unroll
-          for (int k = 0; k < G::WIN; ++k)
-            if (key0 + k > qrow) X[k] = 0.f;
-        }
-        float acc[32];
+        for (int k = 0; k < 32; k += 4)
+          *reinterpret_cast<float4 *>(my + k) = make_float4(X[k], X[k + 1], X[k + 2], X[k + 3]);
+        if (wg == 3) {
 #pragma unroll
-        for (int jj = 0; jj < 32; ++jj) acc[jj] = 0.f;
-        if (CQ > 1) {
-          float *my = scr + r * G::SSTR;
-#pragma unroll
-          for (int k = 0; k + 4 <= G::WIN; k += 4)
+          for (int k = 32; k + 4 <= G::WIN; k += 4)
             *reinterpret_cast<float4 *>(my + k) = make_float4(X[k], X[k + 1], X[k + 2], X[k + 3]);
 #pragma unroll
-          for (int k = G::WIN / 4 * 4; k < G::WIN; ++k) my[k] = X[k];
-          named_bar_sync(1 + wg, 128);
+          for (int k = 32 + (G::WIN - 32) / 4 * 4; k < G::WIN; ++k) my[k] = X[k];
         }
-        // a warp whose 32 rows all precede the chunk's first key has nothing to compute
-        const bool live = (j0 + cb) <= (row0 + 32 * q4 + 31);
-        if (out_row && live) {
-          conv_row<CK, G::WIN>(acc, X, th_s);
+        named_bar_sync(kBarScratch, kConvThreads);
+      }
+      float acc[32];
+#pragma unroll
+      for (int jj = 0; jj < 32; ++jj) acc[jj] = 0.f;
+      // a warp whose 32 rows all precede the chunk's first key has nothing to compute
+      const bool live = (j0 + cb) <= (row0 + 32 * q4 + 31);
+      if (out_row && live) {
+        conv_row<CK, G::WIN>(acc, X, th_s);
 #pragma unroll 1
-          for (int a = 1; a < CQ; ++a) {
-            const float *src = scr + (r - a) * G::SSTR;
-            float Y[G::WIN];
+        for (int a = 1; a < CQ; ++a) {
+          const float *src = Scr + (r - a) * G::SSTR + cb;
+          float Y[G::WIN];
 #pragma unroll
-            for (int k = 0; k + 4 <= G::WIN; k += 4) {
-              const float4 f = *reinterpret_cast<const float4 *>(src + k);
-              Y[k] = f.x; Y[k + 1] = f.y; Y[k + 2] = f.z; Y[k + 3] = f.w;
-            }
-#pragma unroll
-            for (int k = G::WIN / 4 * 4; k < G::WIN; ++k) Y[k] = src[k];
-            conv_row<CK, G::WIN>(acc, Y, th_s + a * CK);
+          for (int k = 0; k + 4 <= G::WIN; k += 4) {
+            const float4 f = *reinterpret_cast<const float4 *>(src + k);
+            Y[k] = f.x; Y[k + 1] = f.y; Y[k + 2] = f.z; Y[k + 3] = f.w;
           }
-        }
-        if (CQ > 1) named_bar_sync(1 + wg, 128);
 #pragma unroll
-        for (int jj = 0; jj < 32; ++jj) cv[32 * ch + jj] = acc[jj];
+          for (int k = G::WIN / 4 * 4; k < G::WIN; ++k) Y[k] = src[k];
+          conv_row<CK, G::WIN>(acc, Y, th_s + a * CK);
+        }
       }
       // Mask_-inf and the tile's row max (log2 units)
-      float mt = -INFINITY;
-      const int kbase = j0 + 64 * wg;
+      const int kbase = j0 + cb;
 #pragma unroll
-      for (int jj = 0; jj < 64; ++jj) {
-        if (kbase + jj > qrow) cv[jj] = -INFINITY;
-        mt = fmaxf(mt, cv[jj]);
-      }
-      if (!out_row) mt = -INFINITY;
-      float *rm = redmax + (t & 1) * 256;
+      for (int jj = 0; jj < 32; ++jj)
+        if (kbase + jj > qrow) acc[jj] = -INFINITY;
+      float mt = out_row ? tree_max<32>(acc) : -INFINITY;
+      float *rm = redmax + (t & 1) * 512;
       rm[wg * 128 + r] = mt;
-      named_bar_sync(3, 256);
-      mt = fmaxf(rm[r], rm[128 + r]);
+      named_bar_sync(kBarMax, kConvThreads);  // also: every read of the shared tile is done
+      mt = fmaxf(fmaxf(rm[r], rm[128 + r]), fmaxf(rm[256 + r], rm[384 + r]));
       const float m_new = fmaxf(m_run, mt);
       bool resc = false;
       float alpha = 1.f;
@@ -373,9 +401,23 @@ __global__ void __launch_bounds__(kThreads, 1)
         m_run = m_new;
       } else if (m_new > m_run + kRescaleLog2) {
         resc = true;
-        alpha = exp2f(m_run - m_new);
+        alpha = ex2(m_run - m_new);
         m_run = m_new;
       }
+      // P = 2^(C - m) (bf16), row sums
+      uint32_t pk[16];
+      float ps[16];
+#pragma unroll
+      for (int jj = 0; jj < 32; jj += 2) {
+        const float p0 = out_row ? ex2(acc[jj] - m_run) : 0.f;
+        const float p1 = out_row ? ex2(acc[jj + 1] - m_run) : 0.f;
+        ps[jj >> 1] = p0 + p1;
+        pk[jj >> 1] = pack_bf16x2(p0, p1);
+      }
+#pragma unroll
+      for (int s = 8; s >= 1; s >>= 1)
+#pragma unroll
+        for (int i = 0; i < s; ++i) ps[i] += ps[i + s];
       if (t > 0) {  // P(t-1) consumed and Z(t-1) complete
         mbar_wait(v_empty, (t - 1) & 1, abort_flag, p.err);
         tc_fence_after();
@@ -387,34 +429,19 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
         for (int hd = 0; hd < G::NV; ++hd)
 #pragma unroll
-          for (int c0 = 0; c0 < D / 2; c0 += 16) {
+          for (int c0 = 0; c0 < G::DQ; c0 += 16) {
             uint32_t z[16];
-            const uint32_t ad = tl + G::Z_COL0 + 128 * hd + wg * (D / 2) + c0;
+            const uint32_t ad = tl + G::Z_COL0 + 128 * hd + wg * G::DQ + c0;
             tmem_ld16(ad, z);
             tmem_wait_ld();
 #pragma unroll
             for (int i = 0; i < 16; ++i) z[i] = __float_as_uint(__uint_as_float(z[i]) * alpha);
             tmem_st16(ad, z);
           }
-        tmem_wait_st();
       }
-      // P = 2^(C - m) in bf16, written row-wise into the 128-byte-swizzled operand tile
-      float ls = 0.f;
-      uint32_t pk[32];
-#pragma unroll
-      for (int jj = 0; jj < 64; jj += 2) {
-        const float p0 = out_row ? ex2(cv[jj] - m_run) : 0.f;
-        const float p1 = out_row ? ex2(cv[jj + 1] - m_run) : 0.f;
-        ls += p0 + p1;
-        pk[jj >> 1] = pack_bf16x2(p0, p1);
-      }
-      l_part += ls;
-      uint8_t *prow = Ps + wg * G::P_CHUNK + (r >> 3) * 1024 + (r & 7) * 128;
-#pragma unroll
-      for (int c = 0; c < 8; ++c)
-        *reinterpret_cast<uint4 *>(prow + ((c ^ (r & 7)) << 4)) =
-            make_uint4(pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
-      fence_proxy_async_smem();
+      l_part += ps[0];
+      tmem_st16(tl + G::P_COL + (cb >> 1), pk);
+      tmem_wait_st();
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(p_full);
@@ -423,7 +450,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     mbar_wait(v_empty, (n_kv - 1) & 1, abort_flag, p.err);
     tc_fence_after();
     redsum[wg * 128 + r] = l_part;
-    named_bar_sync(3, 256);
+    named_bar_sync(kBarSum, kConvThreads);
   }
 
   // ------------------------------------------------------------- epilogue
@@ -433,21 +460,21 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int r = 32 * q4 + lane;
   const int qrow = row0 + r;
   const uint32_t tl = tmem + (static_cast<uint32_t>(32 * q4) << 16);
-  const int cbase = wg * (D / 2);
-  float o[D / 2];
+  const int cbase = wg * G::DQ;
+  float o[G::DQ];
   float inv_l = 0.f;
   if (conv_thread) {
-    inv_l = redsum[r] + redsum[128 + r];
+    inv_l = redsum[r] + redsum[128 + r] + redsum[256 + r] + redsum[384 + r];
     inv_l = (r >= G::HALO && inv_l > 0.f) ? 1.f / inv_l : 0.f;
   }
   if constexpr (CH == 2) {
-    float *xbuf = reinterpret_cast<float *>(Vs);  // [BM][XSTR] fp32, reuses V and P
-    cluster_sync_all();                           // both CTAs are done with V and P
+    float *xbuf = reinterpret_cast<float *>(Vs);  // [BM][XSTR] fp32, reuses V and the scratch
+    cluster_sync_all();                           // both CTAs are done with V and the scratch
     if (conv_thread) {
       const uint32_t peer = static_cast<uint32_t>(hr ^ 1);
       const uint32_t dst = map_peer(smem_u32(xbuf + r * G::XSTR + cbase), peer);
 #pragma unroll
-      for (int c0 = 0; c0 < D / 2; c0 += 16) {
+      for (int c0 = 0; c0 < G::DQ; c0 += 16) {
         uint32_t z[16];
         tmem_ld16(tl + G::Z_COL0 + 128 * (hr ^ 1) + cbase + c0, z);
         tmem_wait_ld();
@@ -462,7 +489,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const float w_own = w_s[hr * CH + hr], w_peer = w_s[hr * CH + (hr ^ 1)];
       const float *xr = xbuf + r * G::XSTR + cbase;
 #pragma unroll
-      for (int c0 = 0; c0 < D / 2; c0 += 16) {
+      for (int c0 = 0; c0 < G::DQ; c0 += 16) {
         uint32_t z[16];
         tmem_ld16(tl + G::Z_COL0 + 128 * hr + cbase + c0, z);
         tmem_wait_ld();
@@ -474,7 +501,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else {
     if (conv_thread) {
 #pragma unroll
-      for (int c0 = 0; c0 < D / 2; c0 += 16) {
+      for (int c0 = 0; c0 < G::DQ; c0 += 16) {
         uint32_t z[16];
         tmem_ld16(tl + G::Z_COL0 + cbase + c0, z);
         tmem_wait_ld();
@@ -487,33 +514,33 @@ __global__ void __launch_bounds__(kThreads, 1)
     float s = 0.f;
     if (conv_thread) {
 #pragma unroll
-      for (int i = 0; i < D / 2; ++i) s += o[i];
+      for (int i = 0; i < G::DQ; ++i) s += o[i];
       redgn[wg * 128 + r] = s;
     }
     __syncthreads();
     float mu = 0.f, rstd = 0.f;
     if (conv_thread) {
-      mu = (redgn[r] + redgn[128 + r]) * (1.f / D);
+      mu = (redgn[r] + redgn[128 + r] + redgn[256 + r] + redgn[384 + r]) * (1.f / D);
       float s2 = 0.f;
 #pragma unroll
-      for (int i = 0; i < D / 2; ++i) { const float x = o[i] - mu; s2 += x * x; }
+      for (int i = 0; i < G::DQ; ++i) { const float x = o[i] - mu; s2 += x * x; }
       s = s2;
     }
     __syncthreads();
     if (conv_thread) redgn[wg * 128 + r] = s;
     __syncthreads();
     if (conv_thread) {
-      rstd = rsqrtf((redgn[r] + redgn[128 + r]) * (1.f / D) + p.eps);
+      rstd = rsqrtf((redgn[r] + redgn[128 + r] + redgn[256 + r] + redgn[384 + r]) * (1.f / D) + p.eps);
       const float *gm = p.gamma + static_cast<long long>(h) * D + cbase;
       const float *bt = p.beta + static_cast<long long>(h) * D + cbase;
 #pragma unroll
-      for (int i = 0; i < D / 2; ++i) o[i] = ((o[i] - mu) * rstd * gm[i] + bt[i]) * p.lam;
+      for (int i = 0; i < G::DQ; ++i) o[i] = ((o[i] - mu) * rstd * gm[i] + bt[i]) * p.lam;
     }
   }
   if (conv_thread && r >= G::HALO && qrow < L) {
     __nv_bfloat16 *dst = p.out + ((static_cast<long long>(b) * L + qrow) * p.H + h) * D + cbase;
 #pragma unroll
-    for (int i = 0; i < D / 2; i += 8) {
+    for (int i = 0; i < G::DQ; i += 8) {
       uint4 v;
       v.x = pack_bf16x2(o[i], o[i + 1]);
       v.y = pack_bf16x2(o[i + 2], o[i + 3]);
