@@ -66,10 +66,12 @@ def flops(wl: synth.Workload) -> dict:
 def launches_per_step(wl: synth.Workload) -> int:
     """Kernels of this library one step launches: the attention kernel; a layer
     adds the two projection GEMMs, and the stand-alone group norm when the
-    attention runs on the CUDA-core kernel (pre-softmax head mixing)."""
+    attention runs on the CUDA-core kernel (shapes the tensor-core kernel does not take)."""
     if not wl.layer:
         return 1
-    return 3 if wl.head_place != synth.PRE else 4
+    tc = (wl.dtype == "bf16" and wl.d in (64, 128) and (wl.c_h == 2 or wl.head_place == synth.OFF)
+          and (wl.kq_place == synth.OFF or (wl.c_q, wl.c_k) == (6, 11)))
+    return 3 if tc else 4
 
 
 def read_peaks() -> tuple[dict, str]:

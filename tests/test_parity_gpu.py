@@ -85,15 +85,13 @@ def tc_applies(wl):
     """Whether the tensor-core kernel serves this configuration."""
     return (wl.dtype == "bf16" and wl.d in (64, 128)
             and (wl.kq_place == synth.OFF or (wl.c_q, wl.c_k) == (6, 11))
-            and (wl.head_place == synth.OFF or (wl.head_place == synth.POST and wl.c_h == 2)))
+            and (wl.head_place == synth.OFF or wl.c_h == 2))
 
 
 @pytest.mark.parametrize("d,hp,L", SMALL)
 @pytest.mark.parametrize("path", [mta.PATH_AUTO, mta.PATH_SIMT, mta.PATH_TC])
 def test_small_bf16(d, hp, L, path):
     base = synth.WORKLOADS["pretrain_d128_L2048"]
-    if path == mta.PATH_TC and hp == synth.PRE:
-        pytest.skip("pre-softmax head mixing runs on the CUDA-core kernel")
     wl = synth.shrink(base, B=2, H=4, L=L, d=d, head_place=hp, seed=77 + L + d + hp)
     inp = synth.make_attn_inputs(wl)
     assert_close(run_attn(wl, inp, path), oracle_full(wl, inp), "bf16")
@@ -114,7 +112,7 @@ def test_small_bf16_other_kernels(c_q, c_k, c_h, kq):
 
 def test_tc_path_unsupported_is_reported():
     base = synth.WORKLOADS["pretrain_d128_L2048"]
-    wl = synth.shrink(base, B=1, H=4, L=64, d=64, head_place=synth.PRE, seed=3)
+    wl = synth.shrink(base, B=1, H=8, L=64, d=64, c_h=4, seed=3)
     inp = synth.make_attn_inputs(wl)
     with pytest.raises(mta.MtaError) as e:
         run_attn(wl, inp, mta.PATH_TC)

@@ -99,8 +99,13 @@ __device__ __forceinline__ float ex2(float x) {
 // ---------------------------------------------------------------------------
 // compile-time geometry
 // ---------------------------------------------------------------------------
-template <int D, int CQ, int CK, int CH>
+// MIX: 0 = no head mixing, 1 = pre-softmax (group of 2), 2 = post-softmax (group of 2)
+template <int D, int CQ, int CK, int MIX>
 struct Geo {
+  static constexpr int CH = MIX ? 2 : 1;              // heads per group
+  static constexpr int NH = MIX == 1 ? 2 : 1;         // source heads whose logits this CTA convolves
+  static constexpr int NV = MIX == 2 ? 2 : 1;         // destination heads (V tiles, Z accumulators)
+  static constexpr int CLUSTER = MIX == 2 ? 2 : 1;
   static constexpr int C = CK / 2;
   static constexpr int HALO = CQ - 1;
   static constexpr int BM = 128;                      // S rows = queries incl. halo
@@ -113,17 +118,17 @@ struct Geo {
   static constexpr int SCOLS = BN + 2 * C;            // columns of the shared masked tile
   static constexpr int SSTR0 = (SCOLS + 3) / 4 * 4;
   static constexpr int SSTR = (SSTR0 % 8 == 0) ? SSTR0 + 4 : SSTR0;  // conflict-free rows
-  static constexpr int NV = CH;                       // destination heads (V tiles)
   static constexpr int DQ = D / 4;                    // output columns per warpgroup
   // shared memory (bytes)
-  static constexpr int Q_BYTES = BM * D * 2;
+  static constexpr int Q_HEAD = BM * D * 2;
+  static constexpr int Q_BYTES = NH * Q_HEAD;
   static constexpr int Q_CHUNK = BM * 128;
   static constexpr int K_CHUNK = NS * 128;
   static constexpr int K_BYTES = NS * D * 2;
   static constexpr int V_CHUNK = BN * 128;
   static constexpr int V_HEAD = BN * D * 2;
   static constexpr int V_BYTES = NV * V_HEAD;
-  static constexpr int SCR_BYTES = (CQ > 1 || CH == 2) ? BM * SSTR * 4 : 0;  // also the exchange buffer
+  static constexpr int SCR_BYTES = (CQ > 1 || MIX == 2) ? BM * SSTR * 4 : 0;  // also the exchange buffer
   static constexpr int OFF_Q = 0;
   static constexpr int OFF_K = OFF_Q + Q_BYTES;
   static constexpr int OFF_V = OFF_K + K_BYTES;
@@ -138,13 +143,15 @@ struct Geo {
   static constexpr int XSTR = D + 4;
   // tensor memory columns
   static constexpr uint32_t TMEM_COLS = 512;
-  static constexpr uint32_t S_COL = 0;
+  static constexpr uint32_t S_COL0 = 0;
+  static constexpr uint32_t S_COL1 = 224;  // second source head (pre-softmax mixing)
   static constexpr uint32_t P_COL = 160;   // 64 columns: 128 keys of bf16, two per column
-  static constexpr uint32_t Z_COL0 = 256;
+  static constexpr uint32_t Z_COL0 = NH == 2 ? 384 : 256;
   static_assert(NS <= 160 && NS % 16 == 0, "S tile");
   static_assert(Z_COL0 + 128 * (NV - 1) + D <= TMEM_COLS, "tensor memory");
+  static_assert(NH == 1 || (S_COL1 + NS <= Z_COL0 && P_COL + 64 <= S_COL1), "tensor memory (two S)");
   static_assert(OFF_K % 1024 == 0 && OFF_V % 1024 == 0, "swizzle alignment");
-  static_assert(CH == 1 || BM * XSTR * 4 <= V_BYTES + SCR_BYTES, "exchange buffer");
+  static_assert(MIX != 2 || BM * XSTR * 4 <= V_BYTES + SCR_BYTES, "exchange buffer");
   static_assert(SMEM <= 232448, "shared memory");
 };
 
@@ -185,11 +192,12 @@ __device__ __forceinline__ float tree_max(const float (&x)[N]) {
   return m[0];
 }
 
-template <int D, int CQ, int CK, int CH>
+template <int D, int CQ, int CK, int MIX>
 __global__ void __launch_bounds__(kThreads, 1)
     attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                    const __grid_constant__ CUtensorMap tmV, const TcParams p) {
-  using G = Geo<D, CQ, CK, CH>;
+  using G = Geo<D, CQ, CK, MIX>;
+  constexpr int CH = G::CH, NH = G::NH;
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t *Qs = smem + G::OFF_Q;
@@ -197,17 +205,17 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint8_t *Vs = smem + G::OFF_V;
   float *Scr = reinterpret_cast<float *>(smem + G::OFF_SCR);
   uint8_t *small = smem + G::OFF_SMALL;
-  float *th_s = reinterpret_cast<float *>(small);             // [CQ*CK], scaled
-  float *w_s = reinterpret_cast<float *>(small + 512);        // [CH*CH]
-  float *redmax = reinterpret_cast<float *>(small + 1024);    // [2 parity][4 wg][128]
-  float *redsum = reinterpret_cast<float *>(small + 5120);    // [4 wg][128]
-  float *redgn = reinterpret_cast<float *>(small + 7168);     // [4 wg][128]
-  uint64_t *bars = reinterpret_cast<uint64_t *>(small + 9216);
+  float *th_s = reinterpret_cast<float *>(small);             // [NH][CQ*CK], scaled
+  float *w_s = reinterpret_cast<float *>(small + 1024);       // [CH*CH]
+  float *redmax = reinterpret_cast<float *>(small + 1088);    // [2 parity][4 wg][128]
+  float *redsum = reinterpret_cast<float *>(small + 5184);    // [4 wg][128]
+  float *redgn = reinterpret_cast<float *>(small + 7232);     // [4 wg][128]
+  uint64_t *bars = reinterpret_cast<uint64_t *>(small + 9280);
   uint64_t *q_full = bars + 0, *k_full = bars + 1, *k_empty = bars + 2, *v_full = bars + 3;
-  uint64_t *v_empty = bars + 4, *s_full = bars + 5, *s_free = bars + 6, *p_full = bars + 7;
-  uint64_t *mma_done = bars + 8;
-  uint32_t *tslot = reinterpret_cast<uint32_t *>(bars + 10);
-  volatile int *abort_flag = reinterpret_cast<volatile int *>(bars + 11);
+  uint64_t *v_empty = bars + 4, *s_full = bars + 5, *s_free = bars + 7, *p_full = bars + 9;
+  uint64_t *mma_done = bars + 10;   // s_full[NH], s_free[NH]: one per source head
+  uint32_t *tslot = reinterpret_cast<uint32_t *>(bars + 11);
+  volatile int *abort_flag = reinterpret_cast<volatile int *>(bars + 12);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int h = blockIdx.x;
@@ -222,15 +230,21 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (threadIdx.x == 0) {
     mbar_init(q_full, 1); mbar_init(k_full, 1); mbar_init(k_empty, 1); mbar_init(v_full, 1);
-    mbar_init(v_empty, 1); mbar_init(s_full, 1); mbar_init(s_free, kConvWarps);
+    mbar_init(v_empty, 1);
+    for (int hh = 0; hh < NH; ++hh) { mbar_init(s_full + hh, 1); mbar_init(s_free + hh, kConvWarps); }
     mbar_init(p_full, kConvWarps); mbar_init(mma_done, 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
-  if (threadIdx.x >= 64 && threadIdx.x < 64 + CQ * CK) {
-    const int i = threadIdx.x - 64;
-    th_s[i] = (p.theta ? p.theta[static_cast<long long>(h) * CQ * CK + i] : 1.f) *
-              (p.qk_scale * kLog2e);
+  if (threadIdx.x >= 64 && threadIdx.x < 64 + NH * CQ * CK) {
+    // key-query kernels, scaled by 1/sqrt(d) and log2(e).  Pre-softmax mixing is
+    // linear after the convolution, so w[h][s] is folded into source head s's
+    // kernel: C'_h = sum_s (w[h][s] theta_s) * Mask_0(A_hat_s).
+    const int i = threadIdx.x - 64, hh = i / (CQ * CK), e = i % (CQ * CK);
+    const int hs = NH == 2 ? g * CH + hh : h;
+    float th = (p.theta ? p.theta[static_cast<long long>(hs) * CQ * CK + e] : 1.f) * (p.qk_scale * kLog2e);
+    if (NH == 2) th *= p.w[(static_cast<long long>(g) * CH + hr) * CH + hh];
+    th_s[i] = th;
   }
   if (threadIdx.x >= 256 && threadIdx.x < 256 + CH * CH)
     w_s[threadIdx.x - 256] = p.w[static_cast<long long>(g) * CH * CH + (threadIdx.x - 256)];
@@ -249,14 +263,20 @@ __global__ void __launch_bounds__(kThreads, 1)
       prefetch_tmap(&tmQ); prefetch_tmap(&tmK);
       mbar_arrive_expect_tx(q_full, G::Q_BYTES);
 #pragma unroll
-      for (int dc = 0; dc < G::NDC; ++dc) tma_load_4d(Qs + dc * G::Q_CHUNK, &tmQ, q_full, dc * 64, h, row0, b);
+      for (int hh = 0; hh < NH; ++hh)
+#pragma unroll
+        for (int dc = 0; dc < G::NDC; ++dc)
+          tma_load_4d(Qs + hh * G::Q_HEAD + dc * G::Q_CHUNK, &tmQ, q_full, dc * 64,
+                      NH == 2 ? g * CH + hh : h, row0, b);
       int nk = 0;
-      for (int t = 0; t < n_kv; ++t) {
-        if (!mbar_wait(k_empty, (t & 1) ^ 1, abort_flag, p.err)) break;
+      for (int u = 0; u < n_kv * NH; ++u) {  // key tiles, source heads alternating
+        const int t = u / NH, hh = u % NH;
+        if (!mbar_wait(k_empty, (u & 1) ^ 1, abort_flag, p.err)) break;
         mbar_arrive_expect_tx(k_full, G::K_BYTES);
 #pragma unroll
         for (int dc = 0; dc < G::NDC; ++dc)
-          tma_load_4d(Ks + dc * G::K_CHUNK, &tmK, k_full, dc * 64, h, t * G::BN - G::C, b);
+          tma_load_4d(Ks + dc * G::K_CHUNK, &tmK, k_full, dc * 64, NH == 2 ? g * CH + hh : h,
+                      t * G::BN - G::C, b);
         ++nk;
       }
       drain_wait(q_full, 0);
@@ -269,7 +289,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         mbar_arrive_expect_tx(v_full, G::V_BYTES);
 #pragma unroll
         for (int hd = 0; hd < G::NV; ++hd) {
-          const int hv = (CH == 1) ? h : g * CH + hd;
+          const int hv = (G::NV == 1) ? h : g * CH + hd;
 #pragma unroll
           for (int dc = 0; dc < G::NDC; ++dc)
             tma_load_4d(Vs + hd * G::V_HEAD + dc * G::V_CHUNK, &tmV, v_full, dc * 64, hv, t * G::BN, b);
@@ -285,23 +305,27 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint32_t idesc_pv = idesc_bf16_f32(128, D, 0, 1);
       const uint32_t q_base = smem_u32(Qs), k_base = smem_u32(Ks), v_base = smem_u32(Vs);
       bool ok = mbar_wait(q_full, 0, abort_flag, p.err);
-      auto issue_qk = [&](int t) -> bool {
-        if (!mbar_wait(k_full, t & 1, abort_flag, p.err)) return false;
-        if (t > 0 && !mbar_wait(s_free, (t - 1) & 1, abort_flag, p.err)) return false;
+      auto issue_qk = [&](int t, int hh) -> bool {
+        const int u = t * NH + hh;
+        if (!mbar_wait(k_full, u & 1, abort_flag, p.err)) return false;
+        if (t > 0 && !mbar_wait(s_free + hh, (t - 1) & 1, abort_flag, p.err)) return false;
         tc_fence_after();
+        const uint32_t qh = q_base + hh * G::Q_HEAD;
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk)
-          mma_bf16_ss(tmem + G::S_COL,
-                      sdesc_sw128(q_base + (kk >> 2) * G::Q_CHUNK + (kk & 3) * 32, 16, 1024),
+          mma_bf16_ss(tmem + (hh ? G::S_COL1 : G::S_COL0),
+                      sdesc_sw128(qh + (kk >> 2) * G::Q_CHUNK + (kk & 3) * 32, 16, 1024),
                       sdesc_sw128(k_base + (kk >> 2) * G::K_CHUNK + (kk & 3) * 32, 16, 1024), idesc_qk,
                       kk > 0);
         mma_commit(k_empty);
-        mma_commit(s_full);
+        mma_commit(s_full + hh);
         return true;
       };
-      if (ok) ok = issue_qk(0);
+      for (int hh = 0; ok && hh < NH; ++hh) ok = issue_qk(0, hh);
       for (int t = 0; ok && t < n_kv; ++t) {
-        if (t + 1 < n_kv && !issue_qk(t + 1)) break;
+        bool next_ok = true;
+        for (int hh = 0; next_ok && hh < NH && t + 1 < n_kv; ++hh) next_ok = issue_qk(t + 1, hh);
+        if (!next_ok) break;
         if (!mbar_wait(p_full, t & 1, abort_flag, p.err)) break;
         if (!mbar_wait(v_full, t & 1, abort_flag, p.err)) break;
         tc_fence_after();
@@ -330,58 +354,64 @@ __global__ void __launch_bounds__(kThreads, 1)
 
     for (int t = 0; t < n_kv; ++t) {
       const int j0 = t * G::BN;
-      mbar_wait(s_full, t & 1, abort_flag, p.err);
-      tc_fence_after();
-      uint32_t u0[32], u1[16];
-      tmem_ld32(tl + G::S_COL + cb, u0);
-      if (G::WIN > 32) tmem_ld16(tl + G::S_COL + cb + 32, u1);
-      tmem_wait_ld();
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(s_free);
-      float X[G::WIN];
-#pragma unroll
-      for (int k = 0; k < G::WIN; ++k) X[k] = __uint_as_float(k < 32 ? u0[k] : u1[(k - 32) & 15]);
-      // Mask_0: keys after this row's query count as 0 inside the convolution
-      const int key0 = j0 - G::C + cb;  // key of window element 0
-      if (key0 + G::WIN - 1 > qrow) {
-#pragma unroll
-        for (int k = 0; k < G::WIN; ++k)
-          if (key0 + k > qrow) X[k] = 0.f;
-      }
-      if (CQ > 1) {  // publish this warpgroup's columns of the masked tile
-        float *my = Scr + r * G::SSTR + cb;
-#pragma unroll
-        for (int k = 0; k < 32; k += 4)
-          *reinterpret_cast<float4 *>(my + k) = make_float4(X[k], X[k + 1], X[k + 2], X[k + 3]);
-        if (wg == 3) {
-#pragma unroll
-          for (int k = 32; k + 4 <= G::WIN; k += 4)
-            *reinterpret_cast<float4 *>(my + k) = make_float4(X[k], X[k + 1], X[k + 2], X[k + 3]);
-#pragma unroll
-          for (int k = 32 + (G::WIN - 32) / 4 * 4; k < G::WIN; ++k) my[k] = X[k];
-        }
-        named_bar_sync(kBarScratch, kConvThreads);
-      }
       float acc[32];
 #pragma unroll
       for (int jj = 0; jj < 32; ++jj) acc[jj] = 0.f;
       // a warp whose 32 rows all precede the chunk's first key has nothing to compute
       const bool live = (j0 + cb) <= (row0 + 32 * q4 + 31);
-      if (out_row && live) {
-        conv_row<CK, G::WIN>(acc, X, th_s);
 #pragma unroll 1
-        for (int a = 1; a < CQ; ++a) {
-          const float *src = Scr + (r - a) * G::SSTR + cb;
-          float Y[G::WIN];
+      for (int hh = 0; hh < NH; ++hh) {  // source heads (two when mixing before the softmax)
+        mbar_wait(s_full + hh, t & 1, abort_flag, p.err);
+        tc_fence_after();
+        const uint32_t scol = hh ? G::S_COL1 : G::S_COL0;
+        uint32_t u0[32], u1[16];
+        tmem_ld32(tl + scol + cb, u0);
+        if (G::WIN > 32) tmem_ld16(tl + scol + cb + 32, u1);
+        tmem_wait_ld();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(s_free + hh);
+        float X[G::WIN];
 #pragma unroll
-          for (int k = 0; k + 4 <= G::WIN; k += 4) {
-            const float4 f = *reinterpret_cast<const float4 *>(src + k);
-            Y[k] = f.x; Y[k + 1] = f.y; Y[k + 2] = f.z; Y[k + 3] = f.w;
+        for (int k = 0; k < G::WIN; ++k) X[k] = __uint_as_float(k < 32 ? u0[k] : u1[(k - 32) & 15]);
+        // Mask_0: keys after this row's query count as 0 inside the convolution
+        const int key0 = j0 - G::C + cb;  // key of window element 0
+        if (key0 + G::WIN - 1 > qrow) {
+#pragma unroll
+          for (int k = 0; k < G::WIN; ++k)
+            if (key0 + k > qrow) X[k] = 0.f;
+        }
+        if (CQ > 1) {  // publish this warpgroup's columns of the masked tile
+          if (hh > 0) named_bar_sync(kBarScratch, kConvThreads);  // previous head's tile fully read
+          float *my = Scr + r * G::SSTR + cb;
+#pragma unroll
+          for (int k = 0; k < 32; k += 4)
+            *reinterpret_cast<float4 *>(my + k) = make_float4(X[k], X[k + 1], X[k + 2], X[k + 3]);
+          if (wg == 3) {
+#pragma unroll
+            for (int k = 32; k + 4 <= G::WIN; k += 4)
+              *reinterpret_cast<float4 *>(my + k) = make_float4(X[k], X[k + 1], X[k + 2], X[k + 3]);
+#pragma unroll
+            for (int k = 32 + (G::WIN - 32) / 4 * 4; k < G::WIN; ++k) my[k] = X[k];
           }
+          named_bar_sync(kBarScratch, kConvThreads);
+        }
+        if (out_row && live) {
+          const float *th = th_s + hh * CQ * CK;
+          conv_row<CK, G::WIN>(acc, X, th);
+#pragma unroll 1
+          for (int a = 1; a < CQ; ++a) {
+            const float *src = Scr + (r - a) * G::SSTR + cb;
+            float Y[G::WIN];
 #pragma unroll
-          for (int k = G::WIN / 4 * 4; k < G::WIN; ++k) Y[k] = src[k];
-          conv_row<CK, G::WIN>(acc, Y, th_s + a * CK);
+            for (int k = 0; k + 4 <= G::WIN; k += 4) {
+              const float4 f = *reinterpret_cast<const float4 *>(src + k);
+              Y[k] = f.x; Y[k + 1] = f.y; Y[k + 2] = f.z; Y[k + 3] = f.w;
+            }
+#pragma unroll
+            for (int k = G::WIN / 4 * 4; k < G::WIN; ++k) Y[k] = src[k];
+            conv_row<CK, G::WIN>(acc, Y, th + a * CK);
+          }
         }
       }
       // Mask_-inf and the tile's row max (log2 units)
@@ -467,7 +497,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     inv_l = redsum[r] + redsum[128 + r] + redsum[256 + r] + redsum[384 + r];
     inv_l = (r >= G::HALO && inv_l > 0.f) ? 1.f / inv_l : 0.f;
   }
-  if constexpr (CH == 2) {
+  if constexpr (MIX == 2) {
     float *xbuf = reinterpret_cast<float *>(Vs);  // [BM][XSTR] fp32, reuses V and the scratch
     cluster_sync_all();                           // both CTAs are done with V and the scratch
     if (conv_thread) {
@@ -557,9 +587,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 }
 
-template <int D, int CQ, int CK, int CH>
+template <int D, int CQ, int CK, int MIX>
 cudaError_t launch_one(const AttnArgs &a, const GnArgs *gn) {
-  using G = Geo<D, CQ, CK, CH>;
+  using G = Geo<D, CQ, CK, MIX>;
   alignas(64) CUtensorMap tq, tk, tv;
   const unsigned long long dims[4] = {static_cast<unsigned long long>(D), static_cast<unsigned long long>(a.H),
                                       static_cast<unsigned long long>(a.L), static_cast<unsigned long long>(a.B)};
@@ -584,7 +614,7 @@ cudaError_t launch_one(const AttnArgs &a, const GnArgs *gn) {
   p.n_qtiles = (a.L + G::BR - 1) / G::BR;
   p.qk_scale = a.scale;
   p.err = a.err;
-  auto kern = attn_tc_kernel<D, CQ, CK, CH>;
+  auto kern = attn_tc_kernel<D, CQ, CK, MIX>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, G::SMEM);
   if (e != cudaSuccess) return e;
   cudaLaunchConfig_t cfg = {};
@@ -594,7 +624,7 @@ cudaError_t launch_one(const AttnArgs &a, const GnArgs *gn) {
   cfg.stream = a.stream;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = CH;
+  attr[0].val.clusterDim.x = G::CLUSTER;
   attr[0].val.clusterDim.y = 1;
   attr[0].val.clusterDim.z = 1;
   cfg.attrs = attr;
@@ -611,8 +641,8 @@ bool attn_tc_supported(const AttnArgs &a) {
   const bool kq_off = a.kq == 0;
   if (!kq_std && !kq_off) return false;
   const bool mix_off = a.hp == 0;
-  const bool mix_post2 = a.hp == 2 && a.ch == 2;
-  if (!mix_off && !mix_post2) return false;
+  const bool mix_group2 = (a.hp == 1 || a.hp == 2) && a.ch == 2;  // pre- or post-softmax
+  if (!mix_off && !mix_group2) return false;
   if (a.B > 65535 || a.H > 65535 || (a.L + 122) / 123 > 65535) return false;
   const uintptr_t al = reinterpret_cast<uintptr_t>(a.q) | reinterpret_cast<uintptr_t>(a.k) |
                        reinterpret_cast<uintptr_t>(a.v) | reinterpret_cast<uintptr_t>(a.out);
@@ -620,16 +650,18 @@ bool attn_tc_supported(const AttnArgs &a) {
   return true;
 }
 
+template <int D, int CQ, int CK>
+cudaError_t launch_mix(const AttnArgs &a, const GnArgs *gn) {
+  if (a.hp == 1) return launch_one<D, CQ, CK, 1>(a, gn);
+  if (a.hp == 2) return launch_one<D, CQ, CK, 2>(a, gn);
+  return launch_one<D, CQ, CK, 0>(a, gn);
+}
+
 cudaError_t launch_attn_tc(const AttnArgs &a0, const GnArgs *gn) {
   AttnArgs a = a0;
-  const bool post = a.hp == 2;
-  if (a.kq == 1) {
-    if (a.d == 128) return post ? launch_one<128, 6, 11, 2>(a, gn) : launch_one<128, 6, 11, 1>(a, gn);
-    return post ? launch_one<64, 6, 11, 2>(a, gn) : launch_one<64, 6, 11, 1>(a, gn);
-  }
+  if (a.kq == 1) return a.d == 128 ? launch_mix<128, 6, 11>(a, gn) : launch_mix<64, 6, 11>(a, gn);
   a.theta = nullptr;  // no key-query convolution: 1 x 1 identity kernel
-  if (a.d == 128) return post ? launch_one<128, 1, 1, 2>(a, gn) : launch_one<128, 1, 1, 1>(a, gn);
-  return post ? launch_one<64, 1, 1, 2>(a, gn) : launch_one<64, 1, 1, 1>(a, gn);
+  return a.d == 128 ? launch_mix<128, 1, 1>(a, gn) : launch_mix<64, 1, 1>(a, gn);
 }
 
 }  // namespace mta
