@@ -63,15 +63,55 @@ def flops(wl: synth.Workload) -> dict:
             "attn_std": f_std, "attn_mta": f_std + conv + mix}
 
 
+def uses_contraction(wl: synth.Workload) -> bool:
+    """Whether the library's default path runs the contraction kernel (with its
+    prepass) for this workload."""
+    return (wl.dtype == "bf16" and wl.d in (64, 128) and wl.kq_place == synth.PRE
+            and (wl.c_q, wl.c_k) == (6, 11)
+            and (wl.head_place == synth.OFF or (wl.head_place == synth.POST and wl.c_h == 2)))
+
+
+def contraction_tensor_flops(wl: synth.Workload) -> float:
+    """Tensor flops the contraction kernel executes per launch: per (batch, head,
+    query tile, key tile at or below the diagonal) a 128x128 tile of the
+    c_q*d-long contraction and, per destination head of the group, a 128x128xd
+    P V product."""
+    nt = -(-wl.L // 128)
+    tiles = wl.B * wl.H * nt * (nt + 1) // 2
+    nv = 2 if wl.head_place == synth.POST else 1
+    return tiles * 2.0 * 128 * 128 * (wl.c_q * wl.d + nv * wl.d)
+
+
 def launches_per_step(wl: synth.Workload) -> int:
-    """Kernels of this library one step launches: the attention kernel; a layer
-    adds the two projection GEMMs, and the stand-alone group norm when the
-    attention runs on the CUDA-core kernel (shapes the tensor-core kernel does not take)."""
-    if not wl.layer:
-        return 1
+    """Kernels of this library one step launches: the attention kernel (and the
+    prepass of the contraction kernel); a layer adds the two projection GEMMs,
+    and the stand-alone group norm when the attention runs on the CUDA-core
+    kernel."""
+    kq = uses_contraction(wl)
     tc = (wl.dtype == "bf16" and wl.d in (64, 128) and (wl.c_h == 2 or wl.head_place == synth.OFF)
           and (wl.kq_place == synth.OFF or (wl.c_q, wl.c_k) == (6, 11)))
-    return 3 if tc else 4
+    attn = 2 if kq else 1  # the contraction kernel runs after its prepass
+    if not wl.layer:
+        return attn
+    return 2 + (attn if (kq or tc) else 2)
+
+
+def max_over_ranks(ms: float, world: int, device) -> float:
+    """The job's time: the largest of the ranks' device-timed milliseconds (an
+    all-reduce MAX over the default process group when there is more than one)."""
+    if world <= 1:
+        return ms
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([ms], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_tokens_per_s(world: int, tokens_per_rank_step: int, steps: int, ms: float) -> float:
+    """Whole-job throughput: every rank processes its own batch each step (weak
+    scaling, replicas), divided by the slowest rank's time."""
+    return world * tokens_per_rank_step * steps / (ms / 1e3)
 
 
 def read_peaks() -> tuple[dict, str]:
@@ -261,13 +301,7 @@ def run_mine(args, wl, rank, world, local_rank):
         raise RuntimeError(f"timed-region status {mta.STATUS.get(st, st)}")
     clocks = sampler.stop() if sampler else None
 
-    # max over ranks
-    t_max = total_ms
-    if world > 1:
-        import torch.distributed as dist
-        t = torch.tensor([total_ms], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        t_max = float(t.item())
+    t_max = max_over_ranks(total_ms, world, dev)
 
     e2e = None
     if not args.no_e2e:
@@ -320,13 +354,8 @@ def run_e2e(args, wl, mta, sets, ws, stream, dev, barrier, world):
         b.record(stream)
     stream.synchronize()
     barrier()
-    ms = a.elapsed_time(b)
-    if world > 1:
-        import torch.distributed as dist
-        t = torch.tensor([ms], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = float(t.item())
-    return {"value": world * wl.tokens * steps / (ms / 1e3), "unit": UNIT,
+    ms = max_over_ranks(a.elapsed_time(b), world, dev)
+    return {"value": job_tokens_per_s(world, wl.tokens, steps, ms), "unit": UNIT,
             "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h), "steps": steps,
             "ms_per_step": ms / steps}
 
@@ -473,7 +502,7 @@ def main():
         return 0
 
     ms = res["total_ms"]
-    value = world * wl.tokens * args.steps / (ms / 1e3)
+    value = job_tokens_per_s(world, wl.tokens, args.steps, ms)
     launch_ms = statistics.mean(res["per_launch_ms"])
     peaks, peak_src = read_peaks()
     s = launch_ms / 1e3
@@ -486,6 +515,22 @@ def main():
                 "kernel": "layer step (QKV GEMM + fused attention + output GEMM)",
                 "per_unit": "F_mta per causal pair-head + 8 B L D^2 GEMM flops",
                 "peak_source": f"{peak_src} bf16 burst"}
+    elif uses_contraction(wl):
+        # the attention call: kq_prep_kernel + attn_kq_kernel (the dominant one);
+        # algorithmic flops F_mta per causal pair-head against the bf16 tensor peak
+        # sustained under the power cap (the timed loop runs for about a second)
+        kernel = "attn_kq_kernel"
+        peak = peaks["bf16_tflops_sustained"]
+        achieved = fl["attn_mta"] / s / 1e12
+        executed = contraction_tensor_flops(wl) / s / 1e12
+        roof = {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+                "frac": achieved / peak,
+                "traffic": read_traffic("attn_kq_kernel", wl.name),
+                "kernel": "mta_attn_fwd call = kq_prep_kernel + attn_kq_kernel",
+                "per_unit": f"F_mta = 4d + 2 c_q c_k + 2 c_h = {fl['attn_mta'] // wl.causal_pairs} flop "
+                            f"per causal pair-head, x {wl.causal_pairs} pair-heads per launch",
+                "executed_tensor_tflops": executed, "executed_frac": executed / peak,
+                "peak_source": f"{peak_src} bf16 sustained"}
     else:
         kernel = "attn_tc_kernel"
         achieved = fl["conv"] / s / 1e12

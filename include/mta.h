@@ -76,9 +76,14 @@ typedef struct mta_cfg {
   int kq_place;          /* MTA_OFF or MTA_PRE                                   */
   int head_place;        /* MTA_OFF, MTA_PRE or MTA_POST (OFF when c_h == 1)     */
   int dtype;             /* mta_dtype of q, k, v and out (x, W and out in a layer) */
-  int path;              /* attention kernel: 0 = choose, 1 = CUDA-core kernel,
-                            2 = tensor-core kernel (MTA_ERR_UNSUPPORTED where it
-                            does not apply)                                       */
+  int path;              /* attention kernel: 0 = choose (the contraction kernel
+                            where it applies and the workspace holds its operands,
+                            else the direct tensor-core kernel where it applies,
+                            else the CUDA-core kernel); 1 = CUDA-core kernel;
+                            2 = tensor-core kernel with the convolution on CUDA
+                            cores; 3 = tensor-core kernel with the convolution as
+                            a contraction of length c_q*d (MTA_ERR_UNSUPPORTED
+                            where the forced kernel does not apply)             */
   float scale;           /* logit scale; 0 selects 1/sqrt(d)                     */
   long long qkv_row_stride; /* elements between consecutive tokens of q, k and v;
                               0 selects H*d (dense [B][L][H][d]); ignored by
@@ -99,7 +104,11 @@ typedef struct mta_gn {
   float depth_scale;     /* lambda; < 0 selects 1 - 0.8*exp(-0.3*layer)         */
 } mta_gn;
 
-/* Bytes of workspace mta_attn_fwd needs for cfg (0 if cfg is invalid). */
+/* Bytes of workspace mta_attn_fwd needs for cfg (0 if cfg is invalid): 256
+ * bytes, plus, where the contraction kernel applies, its per-call operands
+ * (the convolved keys, c_q*B*H*L*d fp16, their B*H*L fp32 scales, and
+ * B*H*L*(c_q-1+2*(c_k/2)) fp32 dot products).  With a smaller workspace path 0
+ * uses another kernel. */
 size_t mta_attn_workspace_bytes(const mta_cfg *cfg);
 
 /* MTA attention core, sections 2, 3.1, 3.2 (steps: logits, Mask_0, key-query
@@ -115,7 +124,11 @@ mta_status mta_attn_fwd(const void *q, const void *k, const void *v,
                         const float *theta_kq, const float *w_head,
                         const mta_cfg *cfg, void *out);
 
-/* Bytes of workspace mta_layer_fwd needs for cfg (0 if cfg is invalid). */
+/* Bytes of workspace mta_layer_fwd uses for cfg (0 if cfg is invalid): the
+ * error word, QKV, the attention output and the normalised output (all bf16),
+ * plus the contraction kernel's operands where it applies (as for
+ * mta_attn_workspace_bytes).  The layer runs with less as long as the first
+ * four fit; path 0 then takes another attention kernel. */
 size_t mta_layer_workspace_bytes(const mta_cfg *cfg);
 
 /* Full MTA attention layer (bf16 only):
@@ -139,8 +152,10 @@ mta_status mta_layer_fwd(const void *x, const void *Wqkv, const float *theta,
  * MTA_STATIC_SCRATCH_BYTES inside the library, which every GPU that loads the
  * library holds until the process exits.  cfg->workspace and
  * cfg->workspace_bytes are ignored; everything else is as for mta_layer_fwd.
- * Returns MTA_ERR_WORKSPACE, enqueuing nothing, when mta_layer_workspace_bytes(cfg)
- * exceeds MTA_STATIC_SCRATCH_BYTES.  The first call on a device looks up the
+ * Returns MTA_ERR_WORKSPACE, enqueuing nothing, when the layer's fixed scratch
+ * (mta_layer_workspace_bytes(cfg) less the contraction kernel's operands)
+ * exceeds MTA_STATIC_SCRATCH_BYTES; the contraction kernel runs where the
+ * whole of mta_layer_workspace_bytes(cfg) fits.  The first call on a device looks up the
  * buffer's address on that device (make it before any stream capture).  All
  * calls on a device share the buffer: calls that overlap on the GPU race, so
  * order them on one stream.  A bounded wait that runs out is recorded in the

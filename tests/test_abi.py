@@ -60,13 +60,22 @@ def call_attn(L, cfg, q=FAKE, theta=FAKE, w=FAKE, out=FAKE):
     return L.mta_attn_fwd(q, FAKE, FAKE, theta, w, ctypes.byref(cfg) if cfg else None, out)
 
 
+def up(x):
+    return -(-x // 256) * 256
+
+
 def test_workspace_query(L):
-    cfg = good_cfg()
-    assert L.mta_attn_workspace_bytes(ctypes.byref(cfg)) == 256
+    cfg = good_cfg()   # the contraction kernel applies: its operands are counted
+    B, H, Ls, d, cq, M = 2, 4, 64, 64, 6, 6 - 1 + 2 * (11 // 2)
+    kq = up(B * H * cq * Ls * d * 2) + up(B * H * Ls * 4) + up(B * H * Ls * M * 4)
+    assert L.mta_attn_workspace_bytes(ctypes.byref(cfg)) == 256 + kq
     t = 2 * 64
     D = 4 * 64
-    want = 256 + -(-t * 3 * D * 2 // 256) * 256 + 2 * (-(-t * D * 2 // 256) * 256)
-    assert L.mta_layer_workspace_bytes(ctypes.byref(cfg)) == want
+    base = 256 + up(t * 3 * D * 2) + 2 * up(t * D * 2)
+    assert L.mta_layer_workspace_bytes(ctypes.byref(cfg)) == base + kq
+    other = good_cfg(c_q=3)   # not a contraction shape: fixed scratch only
+    assert L.mta_attn_workspace_bytes(ctypes.byref(other)) == 256
+    assert L.mta_layer_workspace_bytes(ctypes.byref(other)) == base
     assert L.mta_attn_workspace_bytes(ctypes.byref(good_cfg(c_k=4))) == 0
     assert L.mta_attn_workspace_bytes(None) == 0
 
@@ -74,7 +83,7 @@ def test_workspace_query(L):
 @pytest.mark.parametrize("kw,code", [
     (dict(c_k=4), 1), (dict(c_k=17), 1), (dict(c_q=0), 1), (dict(c_q=9), 1),
     (dict(H=5), 1), (dict(c_h=0), 1), (dict(B=0), 1), (dict(L=0), 1),
-    (dict(kq_place=2), 1), (dict(head_place=3), 1), (dict(dtype=7), 1), (dict(path=3), 1),
+    (dict(kq_place=2), 1), (dict(head_place=3), 1), (dict(dtype=7), 1), (dict(path=4), 1), (dict(path=-1), 1),
     (dict(scale=-1.0), 1), (dict(qkv_row_stride=10), 1),
     (dict(d=200), 2), (dict(d=20), 2), (dict(B=70000), 2),
 ])
@@ -117,6 +126,10 @@ def test_layer_argument_errors(L):
     small = good_cfg()
     small.workspace, small.workspace_bytes = 0x100000, 1024
     assert f(small) == 3
+    forced = good_cfg(path=mta.PATH_KQ)   # the contraction kernel without room for its operands
+    base = L.mta_layer_workspace_bytes(ctypes.byref(good_cfg(c_q=3)))
+    forced.workspace, forced.workspace_bytes = 0x100000, base
+    assert f(forced) == 3
 
 
 def test_building_block_argument_errors(L):

@@ -82,17 +82,26 @@ for d in (64, 128):
 
 
 def tc_applies(wl):
-    """Whether the tensor-core kernel serves this configuration."""
+    """Whether the direct tensor-core kernel serves this configuration."""
     return (wl.dtype == "bf16" and wl.d in (64, 128)
             and (wl.kq_place == synth.OFF or (wl.c_q, wl.c_k) == (6, 11))
             and (wl.head_place == synth.OFF or wl.c_h == 2))
 
 
+def kq_applies(wl):
+    """Whether the contraction kernel serves this configuration."""
+    return (wl.dtype == "bf16" and wl.d in (64, 128) and wl.kq_place == synth.PRE
+            and (wl.c_q, wl.c_k) == (6, 11)
+            and (wl.head_place == synth.OFF or (wl.head_place == synth.POST and wl.c_h == 2)))
+
+
 @pytest.mark.parametrize("d,hp,L", SMALL)
-@pytest.mark.parametrize("path", [mta.PATH_AUTO, mta.PATH_SIMT, mta.PATH_TC])
+@pytest.mark.parametrize("path", [mta.PATH_AUTO, mta.PATH_SIMT, mta.PATH_TC, mta.PATH_KQ])
 def test_small_bf16(d, hp, L, path):
     base = synth.WORKLOADS["pretrain_d128_L2048"]
     wl = synth.shrink(base, B=2, H=4, L=L, d=d, head_place=hp, seed=77 + L + d + hp)
+    if path == mta.PATH_KQ and not kq_applies(wl):
+        pytest.skip("the contraction kernel does not take this configuration")
     inp = synth.make_attn_inputs(wl)
     assert_close(run_attn(wl, inp, path), oracle_full(wl, inp), "bf16")
 
@@ -108,6 +117,8 @@ def test_small_bf16_other_kernels(c_q, c_k, c_h, kq):
     assert_close(run_attn(wl, inp), ref, "bf16")
     if tc_applies(wl):
         assert_close(run_attn(wl, inp, mta.PATH_TC), ref, "bf16")
+    if kq_applies(wl):
+        assert_close(run_attn(wl, inp, mta.PATH_KQ), ref, "bf16")
 
 
 def test_tc_path_unsupported_is_reported():
@@ -134,20 +145,36 @@ def test_strided_qkv_views():
     assert_close(out, oracle_full(wl, inp), "bf16")
 
 
-def test_causality_on_gpu():
+@pytest.mark.parametrize("path", [mta.PATH_TC, mta.PATH_KQ])
+def test_causality_on_gpu(path):
     """Outputs before position t do not change when q, k, v at >= t change."""
     base = synth.WORKLOADS["pretrain_d128_L2048"]
     wl = synth.shrink(base, B=1, H=4, L=400, d=128, seed=8)
     inp = synth.make_attn_inputs(wl)
-    a = run_attn(wl, inp)
+    a = run_attn(wl, inp, path)
     t = 201
     for n, s in (("q", 1), ("k", 2), ("v", 3)):
         x = inp[n].copy()
         x[:, t:] = synth.round_bf16(synth.normal(99, s, x[:, t:].shape))
         inp[n] = x
-    b = run_attn(wl, inp)
+    b = run_attn(wl, inp, path)
     assert torch.equal(a[:, :t], b[:, :t])
     assert not torch.equal(a[:, t:], b[:, t:])
+
+
+@pytest.mark.parametrize("eq,ek", [(15, -15), (-12, 12), (0, -20)])
+def test_kq_operand_scales(eq, ek):
+    """The contraction kernel keeps its fp16 operands in range: queries scaled by
+    2^eq and keys by 2^ek (exact in bf16).  With eq = -ek the logits, and so the
+    oracle's output, are those of the unscaled inputs; (0, -20) makes the keys
+    tiny, so only the per-key-row exponents keep their precision."""
+    base = synth.WORKLOADS["pretrain_d128_L2048"]
+    wl = synth.shrink(base, B=1, H=4, L=300, d=128, seed=12)
+    inp = synth.make_attn_inputs(wl)
+    inp["q"] = (inp["q"] * 2.0 ** eq).astype(np.float32)
+    inp["k"] = (inp["k"] * 2.0 ** ek).astype(np.float32)
+    ref = oracle_full(wl, inp)
+    assert_close(run_attn(wl, inp, mta.PATH_KQ), ref, "bf16")
 
 
 # ---------------------------------------------------------------------------
@@ -163,11 +190,14 @@ def sample_rows(wl, n_extra=6, seed=0):
 
 
 @pytest.mark.parametrize("name", ["identity_d64_L2048", "pretrain_d128_L2048", "long_d128_L16384"])
-def test_full_size_sampled(name):
+@pytest.mark.parametrize("path", [mta.PATH_AUTO, mta.PATH_TC])
+def test_full_size_sampled(name, path):
+    """Full-size workloads: the default path (the bench's launch configuration)
+    and the direct tensor-core kernel."""
     wl = synth.WORKLOADS[name]
-    assert tc_applies(wl)
+    assert tc_applies(wl) and kq_applies(wl)
     inp = synth.make_attn_inputs(wl)
-    out = run_attn(wl, inp)
+    out = run_attn(wl, inp, path)
     rows = sample_rows(wl)
     ref = O.mta_attention_rows(inp["q"], inp["k"], inp["v"], inp["theta"], inp["w"], wl.c_h,
                                rows, wl.kq_place, wl.head_place)

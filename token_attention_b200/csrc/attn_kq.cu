@@ -1,0 +1,598 @@
+// attn_kq.cu -- fused MTA attention with the key-query convolution as a
+// tensor-core contraction (bf16 in/out, fp16 contraction operands).
+//
+// What it computes ("Multi-Token Attention | Summary" (greeksharifa)):
+//   section 2  : logits A_hat = Q K^T / sqrt(d), causal softmax, A V;
+//   section 3.1: A = Softmax(Mask_-inf(Conv2d_theta(Mask_0(A_hat))));
+//   section 3.2: post-softmax head mixing inside groups of 2 heads (appendix B:
+//                through the values, O^h = sum_s w[h][s] A^s V^h);
+//   section 3.3: optional group norm + depth scale (fused epilogue).
+//
+// The convolution is linear in the logits, and the logits are bilinear in q and
+// k, so without the mask
+//   C[i][j] = s * sum_a q[i-a] . Kt_a[j],   Kt_a[j] = sum_t theta[a][t] k[j-(t-c)],
+// a contraction of length c_q*d between the c_q shifted query rows and the
+// per-row-convolved keys (built by the prepass in kq_prep.cu).  Mask_0 zeroes
+// the taps that read a key after the shifted query (key j-(t-c) > i-a); such taps
+// only exist in the band 0 <= i-j < W = (c_q-1)+c, where the kernel replaces the
+// contraction's value by the convolution taken tap by tap over the unmasked taps:
+//   C[i][j] = s * sum_{a,t: m = (i-a) - (j-(t-c)) >= 0} theta[a][t] Vp[i-a][m],
+// with the prepass's past dot products Vp[i][m] = q[i] . k[i-m].  Nothing the
+// kernel reads for query i depends on an input after position i, so outputs are
+// exactly causal (the query tile's fp16 scale only scales down, when |q| > 2^14).
+//
+// Design (one CTA = one (batch, head, tile of 128 queries)):
+//   * TMA loads the query rows i0-(c_q-1) .. i0+127 once, as 8-element strips in
+//     which consecutive rows are 16 bytes apart; the softmax warpgroup converts
+//     them in place to fp16 with a power-of-2 scale.  A row shift by a is then a
+//     16*a-byte offset of the MMA descriptor (SWIZZLE_NONE layout).
+//   * Per key tile of 128: TMA streams the c_q*d/64 chunks of Kt (fp16, 128-byte
+//     swizzle) through a 4-stage ring; one thread issues the 4*c_q*d/64 MMAs
+//     (M=128, N=128, K=16) of C into tensor memory, then P V (P read from tensor
+//     memory) into Z for every destination head of the group.
+//   * One softmax warpgroup (a whole query row per thread, so the row max needs
+//     no exchange) reads C, rescales it, applies the Mask_0 correction near the
+//     diagonal and Mask_-inf, keeps an exact online softmax (the running max
+//     moves only when it grows by more than 2^8, then Z is rescaled) and writes
+//     P (bf16) to tensor memory.
+//   * Post-softmax mixing runs as a 2-CTA cluster with one exchange of
+//     Z_{s->peer}/l_s through distributed shared memory in the epilogue.
+//   * Every mbarrier wait is bounded (error word + early exit).
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+#include <math.h>
+#include <stdint.h>
+
+#include "internal.h"
+#include "ptx.cuh"
+
+namespace mta {
+namespace {
+
+constexpr float kLog2e = 1.4426950408889634f;
+constexpr float kRescaleLog2 = 8.0f;
+constexpr int kThreads = 256;   // warp 0 TMA, warp 1 MMA, warps 2-3 idle, warps 4-7 softmax
+constexpr int kSmWarp0 = 4;
+constexpr int kSmThreads = 128;
+constexpr int kNStage = 4;      // Kt ring stages
+constexpr int kBarSm = 1;       // named barrier of the softmax warpgroup
+
+template <int D, int CQ, int CK, int MIX>
+struct KGeo {
+  static constexpr int C = CK / 2, HALO = CQ - 1, W = HALO + C, M = HALO + 2 * C;
+  static constexpr int BM = 128, BN = 128;
+  static constexpr int QROWS = (BM + HALO + 7) / 8 * 8;  // query rows staged (with halo)
+  static constexpr int NSTRIP = D / 8;
+  static constexpr int STRIP = QROWS * 16;               // bytes of one 8-element strip
+  static constexpr int Q_BYTES = NSTRIP * STRIP;
+  static constexpr int NDC = D / 64;
+  static constexpr int NCH = CQ * NDC;                   // Kt chunks per key tile
+  static constexpr int KCHUNK = BN * 128;                // 128 keys x 64 elements, fp16
+  static constexpr int NV = MIX == 2 ? 2 : 1;
+  static constexpr int CLUSTER = MIX == 2 ? 2 : 1;
+  static constexpr int V_CHUNK = BN * 128;
+  static constexpr int V_HEAD = BN * D * 2;
+  static constexpr int V_BYTES = NV * V_HEAD;
+  static constexpr int UROWS = BM + HALO;
+  static constexpr int OFF_Q = 0;
+  static constexpr int OFF_K = (Q_BYTES + 1023) / 1024 * 1024;
+  static constexpr int OFF_V = OFF_K + kNStage * KCHUNK;
+  static constexpr int OFF_U = OFF_V + V_BYTES;
+  static constexpr int OFF_CORR = (OFF_U + UROWS * M * 4 + 15) / 16 * 16;
+  static constexpr int OFF_FAC = (OFF_CORR + BM * W * 4 + 15) / 16 * 16;   // [2][BN] column scales
+  static constexpr int OFF_SMALL = (OFF_FAC + 2 * BN * 4 + 15) / 16 * 16;
+  static constexpr int SMALL_BYTES = 2048;
+  static constexpr int SMEM_USED = OFF_SMALL + SMALL_BYTES + 1024;
+  // at least half the SM's shared memory: one CTA per SM, so the 512-column TMEM
+  // allocation never waits for another CTA
+  static constexpr int SMEM = SMEM_USED > 232448 / 2 + 1024 ? SMEM_USED : 232448 / 2 + 1024;
+  static constexpr int XSTR = D + 4;  // exchange buffer row (post-softmax mix), reuses ring + V
+  static constexpr uint32_t TMEM_COLS = 512, C_COL = 0, P_COL = 128, Z_COL0 = 256;
+  static_assert(Z_COL0 + 128 * (NV - 1) + D <= TMEM_COLS, "tensor memory");
+  static_assert(OFF_K % 1024 == 0 && OFF_V % 1024 == 0, "swizzle alignment");
+  static_assert(OFF_FAC % 16 == 0, "vector loads of the column scales");
+  static_assert(MIX != 2 || BM * XSTR * 4 <= kNStage * KCHUNK + V_BYTES, "exchange buffer");
+  static_assert(SMEM <= 232448, "shared memory");
+  static_assert(CQ * CK <= 120, "kernel taps");
+};
+
+struct KqParams {
+  const float *theta;   // [H][CQ][CK] (raw; the Mask_0 correction uses it)
+  const float *w;       // [H/2][2][2]
+  __nv_bfloat16 *out;   // [B][L][H][D]
+  const float *gamma, *beta;
+  float eps, lam;
+  int gn;
+  int L, H, n_qtiles;
+  float qk_scale;
+  const float *fac;     // [B][H][L] 2^-e_j of the convolved key rows
+  const float *vp;      // [B][H][L][M] past dot products
+  unsigned *err;
+};
+
+template <int N>
+__device__ __forceinline__ float tree_max(const float (&x)[N]) {
+  float m[N / 2];
+#pragma unroll
+  for (int i = 0; i < N / 2; ++i) m[i] = fmaxf(x[2 * i], x[2 * i + 1]);
+#pragma unroll
+  for (int s = N / 4; s >= 1; s >>= 1)
+#pragma unroll
+    for (int i = 0; i < s; ++i) m[i] = fmaxf(m[i], m[i + s]);
+  return m[0];
+}
+
+template <int D, int CQ, int CK, int MIX>
+__global__ void __launch_bounds__(kThreads, 1)
+    attn_kq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                   const __grid_constant__ CUtensorMap tmV, const KqParams p) {
+  using G = KGeo<D, CQ, CK, MIX>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t *Qs = smem + G::OFF_Q;
+  uint8_t *Ks = smem + G::OFF_K;
+  uint8_t *Vs = smem + G::OFF_V;
+  float *Us = reinterpret_cast<float *>(smem + G::OFF_U);
+  float *Cs = reinterpret_cast<float *>(smem + G::OFF_CORR);
+  float *facs = reinterpret_cast<float *>(smem + G::OFF_FAC);
+  uint8_t *small = smem + G::OFF_SMALL;
+  float *th_s = reinterpret_cast<float *>(small);          // [CQ*CK]
+  float *w_s = reinterpret_cast<float *>(small + 512);     // [4]
+  float *red = reinterpret_cast<float *>(small + 528);     // [4]
+  uint64_t *bars = reinterpret_cast<uint64_t *>(small + 640);
+  uint64_t *q_full = bars + 0, *q_ready = bars + 1, *k_full = bars + 2, *k_empty = bars + 2 + kNStage;
+  uint64_t *v_full = bars + 2 + 2 * kNStage, *v_empty = v_full + 1, *c_full = v_full + 2;
+  uint64_t *c_free = v_full + 3, *p_full = v_full + 4, *mma_done = v_full + 5;
+  uint32_t *tslot = reinterpret_cast<uint32_t *>(small + 640 + 8 * 24);
+  volatile int *abort_flag = reinterpret_cast<volatile int *>(small + 640 + 8 * 24 + 8);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int h = blockIdx.x, b = blockIdx.y;
+  const int qt = p.n_qtiles - 1 - static_cast<int>(blockIdx.z);  // longest tiles first
+  const int hr = h & 1, g = h >> 1;
+  const int L = p.L;
+  const int i0 = qt * G::BM;
+  const int row0 = i0 - G::HALO;  // query index of staged row 0
+  const int last_q = min(L - 1, i0 + G::BM - 1);
+  const int n_kv = last_q / G::BN + 1;
+
+  if (threadIdx.x == 0) {
+    mbar_init(q_full, 1); mbar_init(q_ready, 4);
+    for (int s = 0; s < kNStage; ++s) { mbar_init(k_full + s, 1); mbar_init(k_empty + s, 1); }
+    mbar_init(v_full, 1); mbar_init(v_empty, 1); mbar_init(c_full, 1); mbar_init(c_free, 4);
+    mbar_init(p_full, 4); mbar_init(mma_done, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (threadIdx.x >= 32 && threadIdx.x < 32 + CQ * CK)
+    th_s[threadIdx.x - 32] = p.theta[static_cast<long long>(h) * CQ * CK + (threadIdx.x - 32)];
+  if (MIX == 2 && threadIdx.x >= 192 && threadIdx.x < 196)
+    w_s[threadIdx.x - 192] = p.w[static_cast<long long>(g) * 4 + (threadIdx.x - 192)];
+  if (warp == 1) { tmem_alloc(tslot, G::TMEM_COLS); tmem_relinquish(); }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tslot;
+
+  if (warp == 0) {
+    // -------------------------------------------------------------- TMA
+    if (lane == 0) {
+      prefetch_tmap(&tmQ); prefetch_tmap(&tmK);
+      mbar_arrive_expect_tx(q_full, G::Q_BYTES);
+#pragma unroll 1
+      for (int s = 0; s < G::NSTRIP; ++s) tma_load_4d(Qs + s * G::STRIP, &tmQ, q_full, 8 * s, h, row0, b);
+      int cnt = 0;
+      const int zbase = (b * p.H + h) * CQ;
+      for (int t = 0; t < n_kv && !*abort_flag; ++t)
+        for (int ch = 0; ch < G::NCH; ++ch, ++cnt) {
+          const int st = cnt % kNStage;
+          if (!mbar_wait(k_empty + st, ((cnt / kNStage) & 1) ^ 1, abort_flag, p.err)) break;
+          mbar_arrive_expect_tx(k_full + st, G::KCHUNK);
+          tma_load_3d(Ks + st * G::KCHUNK, &tmK, k_full + st, (ch % G::NDC) * 64, t * G::BN, zbase + ch / G::NDC);
+        }
+      drain_wait(q_full, 0);
+      if (*abort_flag)
+        for (int c2 = (cnt > kNStage ? cnt - kNStage : 0); c2 < cnt; ++c2)
+          drain_wait(k_full + c2 % kNStage, (c2 / kNStage) & 1);
+    } else if (lane == 1) {
+      prefetch_tmap(&tmV);
+      int nv = 0;
+      for (int t = 0; t < n_kv; ++t) {
+        if (!mbar_wait(v_empty, (t & 1) ^ 1, abort_flag, p.err)) break;
+        mbar_arrive_expect_tx(v_full, G::V_BYTES);
+#pragma unroll
+        for (int hd = 0; hd < G::NV; ++hd)
+#pragma unroll
+          for (int dc = 0; dc < G::NDC; ++dc)
+            tma_load_4d(Vs + hd * G::V_HEAD + dc * G::V_CHUNK, &tmV, v_full, dc * 64,
+                        G::NV == 2 ? 2 * g + hd : h, t * G::BN, b);
+        ++nv;
+      }
+      if (*abort_flag && nv) drain_wait(v_full, (nv - 1) & 1);
+    }
+  } else if (warp == 1) {
+    // -------------------------------------------------------------- MMA
+    if (lane == 0) {
+      const uint32_t idesc_c = idesc_f16_f32(128, G::BN);
+      const uint32_t idesc_pv = idesc_bf16_f32(128, D, 0, 1);
+      const uint32_t q_base = smem_u32(Qs), k_base = smem_u32(Ks), v_base = smem_u32(Vs);
+      int cnt = 0;
+      bool ok = mbar_wait(q_ready, 0, abort_flag, p.err);
+      // C(t) = sum over the NCH chunks (a, 64-wide d block) of Q shifted by a rows x Kt_a
+      auto issue_c = [&](int t) -> bool {
+        if (t > 0 && !mbar_wait(c_free, (t - 1) & 1, abort_flag, p.err)) return false;
+        for (int ch = 0; ch < G::NCH; ++ch, ++cnt) {
+          const int st = cnt % kNStage;
+          if (!mbar_wait(k_full + st, (cnt / kNStage) & 1, abort_flag, p.err)) return false;
+          tc_fence_after();
+          const int a = ch / G::NDC, dc = ch % G::NDC;
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk) {
+            const uint32_t qa = q_base + (8 * dc + 2 * kk) * G::STRIP + 16 * (G::HALO - a);
+            mma_bf16_ss(tmem + G::C_COL, sdesc_noswz(qa, G::STRIP, 128),
+                        sdesc_sw128(k_base + st * G::KCHUNK + kk * 32, 16, 1024), idesc_c,
+                        (ch > 0 || kk > 0));
+          }
+          mma_commit(k_empty + st);
+        }
+        mma_commit(c_full);
+        return true;
+      };
+      if (ok) ok = issue_c(0);
+      for (int t = 0; ok && t < n_kv; ++t) {
+        if (t + 1 < n_kv && !issue_c(t + 1)) break;
+        if (!mbar_wait(p_full, t & 1, abort_flag, p.err)) break;
+        if (!mbar_wait(v_full, t & 1, abort_flag, p.err)) break;
+        tc_fence_after();
+#pragma unroll
+        for (int hd = 0; hd < G::NV; ++hd)
+#pragma unroll
+          for (int kk = 0; kk < G::BN / 16; ++kk)
+            mma_f16_ts(tmem + G::Z_COL0 + 128 * hd, tmem + G::P_COL + 8 * kk,
+                       sdesc_sw128(v_base + hd * G::V_HEAD + kk * 16 * 128, G::V_CHUNK, 1024),
+                       idesc_pv, (t > 0 || kk > 0));
+        mma_commit(v_empty);
+      }
+      mma_commit(mma_done);
+      drain_wait(mma_done, 0);
+    }
+  } else if (warp >= kSmWarp0) {
+    // ------------------------------------------------------ softmax group
+    const int q4 = warp & 3;
+    const int r = 32 * q4 + lane;            // query row of this thread = TMEM lane
+    const int qi = i0 + r;
+    const bool out_row = qi < L;
+    const int st_id = threadIdx.x - 32 * kSmWarp0;  // 0..127
+    const uint32_t tl = tmem + (static_cast<uint32_t>(32 * q4) << 16);
+
+    // stage: queries in fp16 with a power-of-2 scale (no overflow), and U rows
+    mbar_wait(q_full, 0, abort_flag, p.err);
+    float qmax = 0.f;
+    for (int c16 = st_id; c16 < G::Q_BYTES / 16; c16 += kSmThreads) {
+      const uint4 raw = *reinterpret_cast<const uint4 *>(Qs + 16 * c16);
+      const __nv_bfloat162 *p2 = reinterpret_cast<const __nv_bfloat162 *>(&raw);
+#pragma unroll
+      for (int u = 0; u < 4; ++u)
+        qmax = fmaxf(qmax, fmaxf(fabsf(__low2float(p2[u])), fabsf(__high2float(p2[u]))));
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) qmax = fmaxf(qmax, __shfl_xor_sync(0xffffffffu, qmax, o));
+    if (lane == 0) red[q4] = qmax;
+    named_bar_sync(kBarSm, kSmThreads);
+    qmax = fmaxf(fmaxf(red[0], red[1]), fmaxf(red[2], red[3]));
+    // scale down only (|q| > 2^14): otherwise the fp16 queries are the bf16 ones
+    int eq = 0;
+    if (qmax > 16384.f) eq = max(-60, static_cast<int>(floorf(log2f(16384.f / qmax))));
+    const float qsc = exp2f(static_cast<float>(eq));
+    for (int c16 = st_id; c16 < G::Q_BYTES / 16; c16 += kSmThreads) {
+      uint4 raw = *reinterpret_cast<const uint4 *>(Qs + 16 * c16);
+      __nv_bfloat162 *p2 = reinterpret_cast<__nv_bfloat162 *>(&raw);
+      uint4 o;
+      uint32_t *ow = reinterpret_cast<uint32_t *>(&o);
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        __half2 hv = __floats2half2_rn(__low2float(p2[u]) * qsc, __high2float(p2[u]) * qsc);
+        ow[u] = *reinterpret_cast<uint32_t *>(&hv);
+      }
+      *reinterpret_cast<uint4 *>(Qs + 16 * c16) = o;
+    }
+    fence_proxy_async_smem();
+    __syncwarp();
+    if (lane == 0) mbar_arrive(q_ready);
+    const long long bh = static_cast<long long>(b) * p.H + h;
+    for (int e = st_id; e < G::UROWS * G::M; e += kSmThreads) {
+      const int rr = e / G::M, k = e % G::M, iq = row0 + rr;
+      Us[e] = (iq >= 0 && iq < L) ? p.vp[(bh * L + iq) * G::M + k] : 0.f;
+    }
+
+    const float sc0 = p.qk_scale * kLog2e;
+    const float sc = sc0 * exp2f(static_cast<float>(-eq));
+    const float *fac = p.fac + bh * L;
+    float m_run = -INFINITY, l_run = 0.f;
+    for (int t = 0; t < n_kv; ++t) {
+      const int j0 = t * G::BN;
+      // column scales of this key tile (double-buffered: the barrier below also
+      // tells every thread that the others are done with tile t-2's buffer)
+      float *fs = facs + (t & 1) * G::BN;
+      fs[st_id] = fac[min(j0 + st_id, L - 1)] * sc;
+      named_bar_sync(kBarSm, kSmThreads);
+      mbar_wait(c_full, t & 1, abort_flag, p.err);
+      tc_fence_after();
+      float cv[G::BN];
+#pragma unroll
+      for (int c0 = 0; c0 < G::BN; c0 += 32) {
+        uint32_t u32[32];
+        tmem_ld32(tl + G::C_COL + c0, u32);
+        tmem_wait_ld();
+#pragma unroll
+        for (int i = 0; i < 32; i += 4) {
+          const float4 f4 = *reinterpret_cast<const float4 *>(fs + c0 + i);
+          cv[c0 + i] = __uint_as_float(u32[i]) * f4.x;
+          cv[c0 + i + 1] = __uint_as_float(u32[i + 1]) * f4.y;
+          cv[c0 + i + 2] = __uint_as_float(u32[i + 2]) * f4.z;
+          cv[c0 + i + 3] = __uint_as_float(u32[i + 3]) * f4.w;
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(c_free);
+      // the band 0 <= i-j < W, where Mask_0 removes taps: the convolution tap by
+      // tap over the unmasked taps, from the past dot products
+      const int dmax = qi - j0;  // i - j for jj = 0
+      if (out_row && dmax >= 0 && dmax - (G::BN - 1) < G::W) {
+        float *crow = Cs + r * G::W;
+#pragma unroll 1
+        for (int dd = 0; dd < G::W; ++dd) {
+          float val = 0.f;
+          const int j = qi - dd;
+          if (j >= j0 && j < j0 + G::BN) {
+#pragma unroll 1
+            for (int a = 0; a < CQ; ++a) {
+              if (qi - a < 0) break;
+              const float *vrow = Us + (r + G::HALO - a) * G::M;
+              // tap t reads key j-(t-c) = (i-a) - m with m = dd - a + (t - c) >= 0
+              for (int t = max(0, a + G::C - dd); t < CK; ++t)
+                val = fmaf(th_s[a * CK + t], vrow[dd - a + t - G::C], val);
+            }
+          }
+          crow[dd] = val * sc0;
+        }
+#pragma unroll
+        for (int jj = 0; jj < G::BN; ++jj) {
+          const int dd = dmax - jj;
+          if (static_cast<unsigned>(dd) < static_cast<unsigned>(G::W)) cv[jj] = crow[dd];
+        }
+      }
+      __syncwarp();  // the warp-collective tensor-memory accesses below need the whole warp
+      // Mask_-inf and the tile's row max (log2 units)
+#pragma unroll
+      for (int jj = 0; jj < G::BN; ++jj)
+        if (j0 + jj > qi) cv[jj] = -INFINITY;
+      const float mt = out_row ? tree_max<G::BN>(cv) : -INFINITY;
+      const float m_new = fmaxf(m_run, mt);
+      bool resc = false;
+      float alpha = 1.f;
+      if (t == 0) {
+        m_run = m_new;
+      } else if (m_new > m_run + kRescaleLog2) {
+        resc = true;
+        alpha = ex2(m_run - m_new);
+        m_run = m_new;
+      }
+      if (t > 0) {  // P(t-1) consumed and Z(t-1) complete
+        mbar_wait(v_empty, (t - 1) & 1, abort_flag, p.err);
+        tc_fence_after();
+      }
+      if (__any_sync(0xffffffffu, resc)) {  // warp-collective tensor-memory access
+        l_run *= alpha;
+#pragma unroll 1
+        for (int c0 = 0; c0 < 128 * (G::NV - 1) + D; c0 += 32) {
+          if (G::NV == 2 && c0 >= D && c0 < 128) continue;
+          uint32_t z[32];
+          tmem_ld32(tl + G::Z_COL0 + c0, z);
+          tmem_wait_ld();
+#pragma unroll
+          for (int i = 0; i < 32; ++i) z[i] = __float_as_uint(__uint_as_float(z[i]) * alpha);
+          tmem_st32(tl + G::Z_COL0 + c0, z);
+        }
+      }
+      float ls = 0.f;
+#pragma unroll
+      for (int half = 0; half < 2; ++half) {
+        uint32_t pk[32];
+#pragma unroll
+        for (int q2 = 0; q2 < 32; ++q2) {
+          const int jj = 64 * half + 2 * q2;
+          const float p0 = out_row ? ex2(cv[jj] - m_run) : 0.f;
+          const float p1 = out_row ? ex2(cv[jj + 1] - m_run) : 0.f;
+          ls += p0 + p1;
+          pk[q2] = pack_bf16x2(p0, p1);
+        }
+        tmem_st32(tl + G::P_COL + 32 * half, pk);
+      }
+      l_run += ls;
+      tmem_wait_st();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(p_full);
+    }
+    mbar_wait(v_empty, (n_kv - 1) & 1, abort_flag, p.err);
+    tc_fence_after();
+    const float inv_l = (out_row && l_run > 0.f) ? 1.f / l_run : 0.f;
+
+    // ---------------------------------------------------------- epilogue
+    float o[D];
+    if constexpr (MIX == 2) {
+      float *xbuf = reinterpret_cast<float *>(Ks);  // [BM][XSTR] fp32, reuses the ring and V
+      __syncwarp();
+      cluster_sync_all();                           // both CTAs are done with their ring and V
+      const uint32_t dst = map_peer(smem_u32(xbuf + r * G::XSTR), static_cast<uint32_t>(hr ^ 1));
+#pragma unroll
+      for (int c0 = 0; c0 < D; c0 += 32) {
+        uint32_t z[32];
+        tmem_ld32(tl + G::Z_COL0 + 128 * (hr ^ 1) + c0, z);
+        tmem_wait_ld();
+#pragma unroll
+        for (int i = 0; i < 32; i += 4)
+          st_cluster_v4(dst + 4 * (c0 + i), __uint_as_float(z[i]) * inv_l, __uint_as_float(z[i + 1]) * inv_l,
+                        __uint_as_float(z[i + 2]) * inv_l, __uint_as_float(z[i + 3]) * inv_l);
+      }
+      cluster_sync_all();  // the peer's Z_{peer->h} / l_peer is in xbuf
+      const float w_own = w_s[hr * 2 + hr], w_peer = w_s[hr * 2 + (hr ^ 1)];
+      const float *xr = xbuf + r * G::XSTR;
+#pragma unroll
+      for (int c0 = 0; c0 < D; c0 += 32) {
+        uint32_t z[32];
+        tmem_ld32(tl + G::Z_COL0 + 128 * hr + c0, z);
+        tmem_wait_ld();
+#pragma unroll
+        for (int i = 0; i < 32; ++i) o[c0 + i] = w_own * (__uint_as_float(z[i]) * inv_l) + w_peer * xr[c0 + i];
+      }
+    } else {
+#pragma unroll
+      for (int c0 = 0; c0 < D; c0 += 32) {
+        uint32_t z[32];
+        tmem_ld32(tl + G::Z_COL0 + c0, z);
+        tmem_wait_ld();
+#pragma unroll
+        for (int i = 0; i < 32; ++i) o[c0 + i] = __uint_as_float(z[i]) * inv_l;
+      }
+    }
+    if (p.gn) {  // group norm over the D channels of (token, head), then depth scale
+      float s = 0.f;
+#pragma unroll
+      for (int i = 0; i < D; ++i) s += o[i];
+      const float mu = s * (1.f / D);
+      float s2 = 0.f;
+#pragma unroll
+      for (int i = 0; i < D; ++i) { const float x = o[i] - mu; s2 += x * x; }
+      const float rstd = rsqrtf(s2 * (1.f / D) + p.eps);
+      const float *gm = p.gamma + static_cast<long long>(h) * D;
+      const float *bt = p.beta + static_cast<long long>(h) * D;
+#pragma unroll
+      for (int i = 0; i < D; ++i) o[i] = ((o[i] - mu) * rstd * gm[i] + bt[i]) * p.lam;
+    }
+    if (out_row) {
+      __nv_bfloat16 *dst = p.out + ((static_cast<long long>(b) * L + qi) * p.H + h) * D;
+#pragma unroll
+      for (int i = 0; i < D; i += 8) {
+        uint4 v;
+        v.x = pack_bf16x2(o[i], o[i + 1]);
+        v.y = pack_bf16x2(o[i + 2], o[i + 3]);
+        v.z = pack_bf16x2(o[i + 4], o[i + 5]);
+        v.w = pack_bf16x2(o[i + 6], o[i + 7]);
+        *reinterpret_cast<uint4 *>(dst + i) = v;
+      }
+    }
+  }
+  if (MIX == 2 && warp < kSmWarp0) {  // the other warps take part in the cluster barriers
+    __syncwarp();  // lanes 0 and 1 of warp 0 and lane 0 of warp 1 return from their roles
+    cluster_sync_all();
+    cluster_sync_all();
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, G::TMEM_COLS);
+  }
+}
+
+template <int D, int CQ, int CK, int MIX>
+cudaError_t launch_kq_one(const AttnArgs &a, const GnArgs *gn, const KqPrepArgs &pa) {
+  using G = KGeo<D, CQ, CK, MIX>;
+  alignas(64) CUtensorMap tq, tk, tv;
+  const unsigned long long dims[4] = {static_cast<unsigned long long>(D), static_cast<unsigned long long>(a.H),
+                                      static_cast<unsigned long long>(a.L), static_cast<unsigned long long>(a.B)};
+  const unsigned long long str[3] = {static_cast<unsigned long long>(D) * 2,
+                                     static_cast<unsigned long long>(a.rs) * 2,
+                                     static_cast<unsigned long long>(a.rs) * 2 * a.L};
+  const unsigned boxq[4] = {8, 1, G::QROWS, 1}, boxv[4] = {64, 1, G::BN, 1};
+  if (!encode_tmap_bf16(&tq, a.q, 4, dims, str, boxq, false)) return cudaErrorInvalidValue;
+  if (!encode_tmap_bf16(&tv, a.v, 4, dims, str, boxv, true)) return cudaErrorInvalidValue;
+  // Kt: [B*H*CQ][L][D] 16-bit elements (the copy moves bytes; fp16 as 16-bit)
+  const unsigned long long kdims[3] = {static_cast<unsigned long long>(D), static_cast<unsigned long long>(a.L),
+                                       static_cast<unsigned long long>(a.B) * a.H * CQ};
+  const unsigned long long kstr[2] = {static_cast<unsigned long long>(D) * 2,
+                                      static_cast<unsigned long long>(a.L) * D * 2};
+  const unsigned boxk[3] = {64, G::BN, 1};
+  if (!encode_tmap_bf16(&tk, pa.kt, 3, kdims, kstr, boxk, true)) return cudaErrorInvalidValue;
+  KqParams p;
+  p.theta = a.theta;
+  p.w = a.w;
+  p.out = static_cast<__nv_bfloat16 *>(a.out);
+  p.gn = gn != nullptr;
+  p.gamma = gn ? gn->gamma : nullptr;
+  p.beta = gn ? gn->beta : nullptr;
+  p.eps = gn ? gn->eps : 0.f;
+  p.lam = gn ? gn->lam : 1.f;
+  p.L = a.L;
+  p.H = a.H;
+  p.n_qtiles = (a.L + G::BM - 1) / G::BM;
+  p.qk_scale = a.scale;
+  p.fac = pa.fac;
+  p.vp = pa.vp;
+  p.err = a.err;
+  auto kern = attn_kq_kernel<D, CQ, CK, MIX>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, G::SMEM);
+  if (e != cudaSuccess) return e;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(a.H, a.B, p.n_qtiles);
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = G::SMEM;
+  cfg.stream = a.stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = G::CLUSTER;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, tq, tk, tv, p);
+}
+
+size_t align256(size_t x) { return (x + 255) / 256 * 256; }
+
+}  // namespace
+
+bool attn_kq_supported(const AttnArgs &a) {
+  if (a.dtype != 1 || (a.d != 64 && a.d != 128)) return false;
+  if (a.kq != 1 || a.cq != 6 || a.ck != 11) return false;
+  if (!(a.hp == 0 || (a.hp == 2 && a.ch == 2))) return false;
+  if (a.B > 65535 || a.H > 65535 || (a.L + 127) / 128 > 65535) return false;
+  const uintptr_t al = reinterpret_cast<uintptr_t>(a.q) | reinterpret_cast<uintptr_t>(a.k) |
+                       reinterpret_cast<uintptr_t>(a.v) | reinterpret_cast<uintptr_t>(a.out);
+  return al % 16 == 0 && a.rs % 8 == 0;
+}
+
+// Workspace of the contraction path: Kt [B][H][c_q][L][d] fp16 | fac [B][H][L] fp32 |
+// Vp [B][H][L][M] fp32, M = (c_q-1) + 2*(c_k/2); each part 256-byte aligned.
+size_t attn_kq_workspace_bytes(int B, int H, int L, int d, int cq, int ck) {
+  const size_t BHL = static_cast<size_t>(B) * H * L;
+  const size_t M = static_cast<size_t>(cq - 1 + 2 * (ck / 2));
+  return align256(BHL * cq * d * 2) + align256(BHL * 4) + align256(BHL * M * 4);
+}
+
+cudaError_t launch_attn_kq(const AttnArgs &a, const GnArgs *gn, void *ws) {
+  KqPrepArgs pa;
+  pa.q = a.q;
+  pa.k = a.k;
+  pa.rs = a.rs;
+  pa.theta = a.theta;
+  pa.B = a.B; pa.H = a.H; pa.L = a.L; pa.d = a.d; pa.cq = a.cq; pa.ck = a.ck;
+  pa.M = a.cq - 1 + 2 * (a.ck / 2);
+  pa.n_tiles = (a.L + 127) / 128;
+  const size_t BHL = static_cast<size_t>(a.B) * a.H * a.L;
+  char *base = static_cast<char *>(ws);
+  pa.kt = base;
+  pa.fac = reinterpret_cast<float *>(base + align256(BHL * a.cq * a.d * 2));
+  pa.vp = reinterpret_cast<float *>(reinterpret_cast<char *>(pa.fac) + align256(BHL * 4));
+  cudaError_t e = launch_kq_prep(pa, a.stream);
+  if (e != cudaSuccess) return e;
+  const bool post = a.hp == 2;
+  if (a.d == 128) return post ? launch_kq_one<128, 6, 11, 2>(a, gn, pa) : launch_kq_one<128, 6, 11, 0>(a, gn, pa);
+  return post ? launch_kq_one<64, 6, 11, 2>(a, gn, pa) : launch_kq_one<64, 6, 11, 0>(a, gn, pa);
+}
+
+}  // namespace mta

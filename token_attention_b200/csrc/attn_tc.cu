@@ -56,47 +56,6 @@ constexpr int kBarMax = 2;      // row maxima exchanged between warpgroups
 constexpr int kBarSum = 3;      // row sums exchanged (end of the key loop)
 
 // ---------------------------------------------------------------------------
-// cluster helpers (distributed shared memory)
-// ---------------------------------------------------------------------------
-__device__ __forceinline__ void cluster_sync_all() {
-  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::
-                   : "memory");
-}
-__device__ __forceinline__ uint32_t map_peer(uint32_t local_saddr, uint32_t rank) {
-  uint32_t r;
-  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(local_saddr), "r"(rank));
-  return r;
-}
-__device__ __forceinline__ void st_cluster_v4(uint32_t addr, float a, float b, float c, float d) {
-  asm volatile("st.shared::cluster.v4.f32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "f"(a), "f"(b),
-               "f"(c), "f"(d)
-               : "memory");
-}
-
-__device__ __forceinline__ void drain_wait(uint64_t *bar, uint32_t parity) {
-  const unsigned long long t0 = globaltimer_ns();
-  while (!mbar_try_wait(bar, parity))
-    if (globaltimer_ns() - t0 > kWaitLimitNs) return;
-}
-
-// D[tmem] (+)= A[tmem] * B[smem], kind::f16 (bf16 A packed two per 32-bit column).
-__device__ __forceinline__ void mma_bf16_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc,
-                                            uint32_t idesc, uint32_t accumulate) {
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "setp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
-      "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
-      : "memory");
-}
-
-__device__ __forceinline__ float ex2(float x) {
-  float y;
-  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
-  return y;
-}
-
-// ---------------------------------------------------------------------------
 // compile-time geometry
 // ---------------------------------------------------------------------------
 // MIX: 0 = no head mixing, 1 = pre-softmax (group of 2), 2 = post-softmax (group of 2)
@@ -333,7 +292,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int hd = 0; hd < G::NV; ++hd)
 #pragma unroll
           for (int kk = 0; kk < G::BN / 16; ++kk)
-            mma_bf16_ts(tmem + G::Z_COL0 + 128 * hd, tmem + G::P_COL + 8 * kk,
+            mma_f16_ts(tmem + G::Z_COL0 + 128 * hd, tmem + G::P_COL + 8 * kk,
                         sdesc_sw128(v_base + hd * G::V_HEAD + kk * 16 * 128, G::V_CHUNK, 1024),
                         idesc_pv, (t > 0 || kk > 0));
         mma_commit(v_empty);
@@ -399,7 +358,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (out_row && live) {
           const float *th = th_s + hh * CQ * CK;
           conv_row<CK, G::WIN>(acc, X, th);
-#pragma unroll 1
+#pragma unroll
           for (int a = 1; a < CQ; ++a) {
             const float *src = Scr + (r - a) * G::SSTR + cb;
             float Y[G::WIN];

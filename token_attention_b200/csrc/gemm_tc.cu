@@ -25,13 +25,6 @@ constexpr int STAGE_BYTES = A_BYTES + B_BYTES;  // 48 KB
 constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 1024 /*align*/ + 256 /*barriers*/;
 constexpr uint32_t TMEM_COLS = 256;
 
-// bounded wait that ignores the abort flag (used to drain TMA copies in flight)
-__device__ __forceinline__ void drain_wait(uint64_t *bar, uint32_t parity) {
-  const unsigned long long t0 = globaltimer_ns();
-  while (!mbar_try_wait(bar, parity))
-    if (globaltimer_ns() - t0 > kWaitLimitNs) return;
-}
-
 __global__ void __launch_bounds__(192, 1)
     gemm_bf16_nt_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                         __nv_bfloat16 *__restrict__ C, int M, int N, int K, unsigned *err) {

@@ -37,6 +37,25 @@ cudaError_t launch_attn_simt(const AttnArgs &a);
 bool attn_tc_supported(const AttnArgs &a);
 cudaError_t launch_attn_tc(const AttnArgs &a, const GnArgs *gn);
 
+// Contraction form of the key-query convolution (tensor cores): a prepass
+// builds the per-row-convolved keys Kt and the near-diagonal dot products U,
+// then the attention kernel contracts shifted queries against Kt.
+struct KqPrepArgs {
+  const void *q, *k;      // [B][L][H][d] bf16, token stride rs
+  long long rs;
+  const float *theta;     // [H][c_q][c_k]
+  void *kt;               // [B][H][c_q][L][d] fp16, key row j scaled by 2^e_j
+  float *fac;             // [B][H][L] 2^-e_j
+  float *vp;              // [B][H][L][M] past dot products q[i] . k[i-m], m < M
+  int B, H, L, d, cq, ck, M, n_tiles;
+};
+cudaError_t launch_kq_prep(const KqPrepArgs &a, cudaStream_t stream);
+// Workspace bytes of the contraction path (beyond the error word) and whether it applies.
+bool attn_kq_supported(const AttnArgs &a);
+size_t attn_kq_workspace_bytes(int B, int H, int L, int d, int cq, int ck);
+// ws: workspace area for Kt / fac / Vp (attn_kq_workspace_bytes bytes, 256-byte aligned).
+cudaError_t launch_attn_kq(const AttnArgs &a, const GnArgs *gn, void *ws);
+
 // tcgen05 GEMM: C[M][N] = A[M][K] * B[N][K]^T (bf16 -> fp32 -> bf16).
 cudaError_t launch_gemm_bf16_nt(const void *A, const void *B, void *C, int M, int N, int K,
                                 unsigned *err, cudaStream_t stream);

@@ -23,6 +23,10 @@
 
 #include "mta.h"
 
+namespace mta {
+size_t layer_base_workspace_bytes(const mta_cfg *cfg);  // mta_api.cu
+}  // namespace mta
+
 namespace {
 
 __device__ __align__(256) unsigned char g_layer_scratch[MTA_STATIC_SCRATCH_BYTES];
@@ -52,7 +56,9 @@ extern "C" mta_status mta_layer_fwd_static(const void *x, const void *Wqkv, cons
                                            const float *w_head, const mta_gn *gn, const void *Wo,
                                            const mta_cfg *cfg, void *out) {
   if (!cfg) return MTA_ERR_INVALID;
-  const size_t need = mta_layer_workspace_bytes(cfg);
+  // the fixed scratch must fit; the contraction kernel's operands are used
+  // where the rest of the buffer holds them, else the layer takes another kernel
+  const size_t need = mta::layer_base_workspace_bytes(cfg);
   mta_cfg c = *cfg;
   if (need == 0) {
     // invalid configuration: let the layer's own checks report the precise status

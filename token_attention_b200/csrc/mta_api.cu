@@ -33,7 +33,7 @@ mta_status check_cfg(const mta_cfg *c) {
   if (c->head_place != MTA_OFF && c->head_place != MTA_PRE && c->head_place != MTA_POST)
     return MTA_ERR_INVALID;
   if (c->dtype != MTA_F32 && c->dtype != MTA_BF16) return MTA_ERR_INVALID;
-  if (c->path < 0 || c->path > 2) return MTA_ERR_INVALID;
+  if (c->path < 0 || c->path > 3) return MTA_ERR_INVALID;
   if (!isfinite(c->scale) || c->scale < 0.f) return MTA_ERR_INVALID;
   const long long hd = static_cast<long long>(c->H) * c->d;
   if (c->qkv_row_stride != 0 && c->qkv_row_stride < hd) return MTA_ERR_INVALID;
@@ -54,14 +54,50 @@ AttnArgs make_args(const void *q, const void *k, const void *v, const float *the
   return a;
 }
 
-// Which attention kernel serves `a` under cfg->path (0: the tensor-core kernel
-// where it applies, else the CUDA-core kernel; 1: CUDA-core; 2: tensor-core).
-mta_status select_kernel(const AttnArgs &a, int path, bool *use_tc) {
+enum Kernel { K_SIMT = 1, K_TC = 2, K_KQ = 3 };
+
+// Shape-level test for the contraction kernel (pointer alignment aside): used
+// to size the workspace.
+bool kq_shape_ok(const mta_cfg *c) {
+  return c->dtype == MTA_BF16 && (c->d == 64 || c->d == 128) && c->kq_place == MTA_PRE &&
+         c->c_q == 6 && c->c_k == 11 &&
+         (c->head_place == MTA_OFF || (c->head_place == MTA_POST && c->c_h == 2));
+}
+
+size_t kq_bytes(const mta_cfg *c) {
+  return kq_shape_ok(c) ? attn_kq_workspace_bytes(c->B, c->H, c->L, c->d, c->c_q, c->c_k) : 0;
+}
+
+// Which attention kernel serves `a` under cfg->path: 0 chooses the contraction
+// kernel where it applies and `kq_room` bytes of workspace hold its operands,
+// else the direct tensor-core kernel where it applies, else the CUDA-core
+// kernel; 1, 2, 3 force the CUDA-core, direct tensor-core, contraction kernel.
+mta_status select_kernel(const AttnArgs &a, int path, size_t kq_room, Kernel *k) {
+  const bool kq_ok = attn_kq_supported(a) &&
+                     kq_room >= attn_kq_workspace_bytes(a.B, a.H, a.L, a.d, a.cq, a.ck);
   const bool tc_ok = attn_tc_supported(a);
-  if (path == 2 && !tc_ok) return MTA_ERR_UNSUPPORTED;
-  *use_tc = tc_ok && path != 1;
-  if (!*use_tc && attn_simt_pick_rows(a, 32) == 0) return MTA_ERR_UNSUPPORTED;
+  const bool simt_ok = attn_simt_pick_rows(a, 32) != 0;
+  if (path == 3) {
+    if (!attn_kq_supported(a)) return MTA_ERR_UNSUPPORTED;
+    if (!kq_ok) return MTA_ERR_WORKSPACE;
+    *k = K_KQ;
+  } else if (path == 2) {
+    if (!tc_ok) return MTA_ERR_UNSUPPORTED;
+    *k = K_TC;
+  } else if (path == 1) {
+    if (!simt_ok) return MTA_ERR_UNSUPPORTED;
+    *k = K_SIMT;
+  } else {
+    *k = kq_ok ? K_KQ : tc_ok ? K_TC : K_SIMT;
+    if (*k == K_SIMT && !simt_ok) return MTA_ERR_UNSUPPORTED;
+  }
   return MTA_OK;
+}
+
+cudaError_t launch_kernel(Kernel k, const AttnArgs &a, const GnArgs *gn, void *kq_ws) {
+  if (k == K_KQ) return launch_attn_kq(a, gn, kq_ws);
+  if (k == K_TC) return launch_attn_tc(a, gn);
+  return launch_attn_simt(a);
 }
 
 mta_status check_attn_pointers(const void *q, const void *k, const void *v, const float *theta,
@@ -130,6 +166,14 @@ bool encode_tmap_bf16(void *map_out, const void *base, int rank, const unsigned 
   return r == CUDA_SUCCESS;
 }
 
+// The layer's fixed scratch: error word, QKV, attention output O, normalised Y
+// (the contraction kernel's operands come on top where they fit).
+size_t layer_base_workspace_bytes(const mta_cfg *cfg) {
+  if (check_cfg(cfg) != MTA_OK) return 0;
+  const size_t T = layer_tokens(cfg), D = static_cast<size_t>(cfg->H) * cfg->d;
+  return kStatusBytes + align_up(T * 3 * D * 2) + 2 * align_up(T * D * 2);
+}
+
 }  // namespace mta
 
 using namespace mta;
@@ -152,7 +196,7 @@ const char *mta_status_string(mta_status s) {
 
 size_t mta_attn_workspace_bytes(const mta_cfg *cfg) {
   if (check_cfg(cfg) != MTA_OK) return 0;
-  return kStatusBytes;
+  return kStatusBytes + kq_bytes(cfg);
 }
 
 mta_status mta_attn_fwd(const void *q, const void *k, const void *v, const float *theta_kq,
@@ -162,17 +206,16 @@ mta_status mta_attn_fwd(const void *q, const void *k, const void *v, const float
   if ((s = check_attn_pointers(q, k, v, theta_kq, w_head, cfg, out)) != MTA_OK) return s;
   if ((s = check_workspace(cfg, kStatusBytes)) != MTA_OK) return s;
   AttnArgs a = make_args(q, k, v, theta_kq, w_head, cfg, out);
-  bool use_tc = false;
-  if ((s = select_kernel(a, cfg->path, &use_tc)) != MTA_OK) return s;
+  Kernel kern = K_SIMT;
+  if ((s = select_kernel(a, cfg->path, cfg->workspace_bytes - kStatusBytes, &kern)) != MTA_OK) return s;
   if ((s = clear_status(cfg)) != MTA_OK) return s;
-  const cudaError_t e = use_tc ? launch_attn_tc(a, nullptr) : launch_attn_simt(a);
+  const cudaError_t e = launch_kernel(kern, a, nullptr, static_cast<char *>(cfg->workspace) + kStatusBytes);
   return e == cudaSuccess ? MTA_OK : MTA_ERR_CUDA;
 }
 
 size_t mta_layer_workspace_bytes(const mta_cfg *cfg) {
-  if (check_cfg(cfg) != MTA_OK) return 0;
-  const size_t T = layer_tokens(cfg), D = static_cast<size_t>(cfg->H) * cfg->d;
-  return kStatusBytes + align_up(T * 3 * D * 2) + 2 * align_up(T * D * 2);
+  const size_t base = layer_base_workspace_bytes(cfg);
+  return base ? base + kq_bytes(cfg) : 0;
 }
 
 mta_status mta_layer_fwd(const void *x, const void *Wqkv, const float *theta, const float *w_head,
@@ -189,7 +232,7 @@ mta_status mta_layer_fwd(const void *x, const void *Wqkv, const float *theta, co
   const size_t T = layer_tokens(cfg), D = static_cast<size_t>(cfg->H) * cfg->d;
   if (T > static_cast<size_t>(65535) * 128 || 3 * D > static_cast<size_t>(1) << 30)
     return MTA_ERR_UNSUPPORTED;
-  if ((s = check_workspace(cfg, mta_layer_workspace_bytes(cfg))) != MTA_OK) return s;
+  if ((s = check_workspace(cfg, layer_base_workspace_bytes(cfg))) != MTA_OK) return s;
 
   char *ws = static_cast<char *>(cfg->workspace);
   void *qkv = ws + kStatusBytes;
@@ -200,8 +243,10 @@ mta_status mta_layer_fwd(const void *x, const void *Wqkv, const float *theta, co
   mta_cfg acfg = *cfg;
   acfg.qkv_row_stride = static_cast<long long>(3 * D);
   AttnArgs a = make_args(qkvb, qkvb + D, qkvb + 2 * D, theta, w_head, &acfg, obuf);
-  bool use_tc = false;
-  if ((s = select_kernel(a, cfg->path, &use_tc)) != MTA_OK) return s;
+  void *kq_ws = static_cast<char *>(ybuf) + align_up(T * D * 2);
+  const size_t kq_room = cfg->workspace_bytes - (static_cast<char *>(kq_ws) - ws);
+  Kernel kern = K_SIMT;
+  if ((s = select_kernel(a, cfg->path, kq_room, &kern)) != MTA_OK) return s;
 
   const GnArgs g = make_gn(gn);
   cudaStream_t st = static_cast<cudaStream_t>(cfg->stream);
@@ -211,10 +256,10 @@ mta_status mta_layer_fwd(const void *x, const void *Wqkv, const float *theta, co
   if (launch_gemm_bf16_nt(x, Wqkv, qkv, static_cast<int>(T), static_cast<int>(3 * D),
                           static_cast<int>(D), err, st) != cudaSuccess)
     return MTA_ERR_CUDA;
-  if (use_tc) {
+  if (kern != K_SIMT) {
     // attention with the group norm and depth scale fused into its epilogue: Y
     a.out = ybuf;
-    if (launch_attn_tc(a, &g) != cudaSuccess) return MTA_ERR_CUDA;
+    if (launch_kernel(kern, a, &g, kq_ws) != cudaSuccess) return MTA_ERR_CUDA;
   } else {
     // attention output O, then the stand-alone group norm O -> Y
     a.out = obuf;

@@ -18,7 +18,7 @@ LIB_PATH = os.environ.get("MTA_LIB") or os.path.join(HERE, "libmta.so")
 
 OFF, PRE, POST = 0, 1, 2
 F32, BF16 = 0, 1
-PATH_AUTO, PATH_SIMT, PATH_TC = 0, 1, 2
+PATH_AUTO, PATH_SIMT, PATH_TC, PATH_KQ = 0, 1, 2, 3
 
 STATUS = {0: "MTA_OK", 1: "MTA_ERR_INVALID", 2: "MTA_ERR_UNSUPPORTED", 3: "MTA_ERR_WORKSPACE",
           4: "MTA_ERR_CUDA", 5: "MTA_ERR_TIMEOUT"}
