@@ -52,16 +52,17 @@ namespace {
 
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kRescaleLog2 = 8.0f;
-constexpr int kThreads = 256;   // warp 0 TMA, warp 1 MMA, warps 2-3 idle, warps 4-7 softmax
-constexpr int kSmWarp0 = 4;
-constexpr int kSmThreads = 128;
-constexpr int kNStage = 4;      // Kt ring stages
-constexpr int kBarSm = 1;       // named barrier of the softmax warpgroup
+// warps 0-7: two softmax warpgroups (warpgroup w takes key columns 64w .. 64w+63 of
+// every tile and half of the output channels); warp 8: TMA; warp 9: MMA
+constexpr int kThreads = 320;
+constexpr int kSmThreads = 256;
+constexpr int kTmaWarp = 8, kMmaWarp = 9;
+constexpr int kBarAll = 1;      // named barrier over both softmax warpgroups
 
 template <int D, int CQ, int CK, int MIX>
 struct KGeo {
   static constexpr int C = CK / 2, HALO = CQ - 1, W = HALO + C, M = HALO + 2 * C;
-  static constexpr int BM = 128, BN = 128;
+  static constexpr int BM = 128, BN = 128, HALF = BN / 2, DH = D / 2;
   static constexpr int QROWS = (BM + HALO + 7) / 8 * 8;  // query rows staged (with halo)
   static constexpr int NSTRIP = D / 8;
   static constexpr int STRIP = QROWS * 16;               // bytes of one 8-element strip
@@ -75,14 +76,23 @@ struct KGeo {
   static constexpr int V_HEAD = BN * D * 2;
   static constexpr int V_BYTES = NV * V_HEAD;
   static constexpr int UROWS = BM + HALO;
+  static constexpr int U_BYTES = (UROWS * M * 4 + 15) / 16 * 16;
+  static constexpr int CS_BYTES = 2 * BM * W * 4;        // band values, one block per warpgroup
+  static constexpr int RED_BYTES = 10 * BM * 4;          // row maxima (2 tiles x 2 groups), l, norm sums
+  static constexpr int FAC_BYTES = 2 * BN * 4;           // column factors of two key tiles
+  static constexpr int SMALL_BYTES = 2048;
+  // Kt ring: as many 16 KB stages as the shared memory left over holds (at most 8)
+  static constexpr int REST = (Q_BYTES + 1023) / 1024 * 1024 + V_BYTES + U_BYTES + CS_BYTES + RED_BYTES +
+                              FAC_BYTES + SMALL_BYTES + 1024;
+  static constexpr int NS = (232448 - REST) / KCHUNK < 8 ? (232448 - REST) / KCHUNK : 8;
   static constexpr int OFF_Q = 0;
   static constexpr int OFF_K = (Q_BYTES + 1023) / 1024 * 1024;
-  static constexpr int OFF_V = OFF_K + kNStage * KCHUNK;
+  static constexpr int OFF_V = OFF_K + NS * KCHUNK;
   static constexpr int OFF_U = OFF_V + V_BYTES;
-  static constexpr int OFF_CORR = (OFF_U + UROWS * M * 4 + 15) / 16 * 16;
-  static constexpr int OFF_FAC = (OFF_CORR + BM * W * 4 + 15) / 16 * 16;   // [2][BN] column scales
-  static constexpr int OFF_SMALL = (OFF_FAC + 2 * BN * 4 + 15) / 16 * 16;
-  static constexpr int SMALL_BYTES = 2048;
+  static constexpr int OFF_CS = OFF_U + U_BYTES;
+  static constexpr int OFF_RED = OFF_CS + CS_BYTES;
+  static constexpr int OFF_FAC = OFF_RED + RED_BYTES;
+  static constexpr int OFF_SMALL = OFF_FAC + FAC_BYTES;
   static constexpr int SMEM_USED = OFF_SMALL + SMALL_BYTES + 1024;
   // at least half the SM's shared memory: one CTA per SM, so the 512-column TMEM
   // allocation never waits for another CTA
@@ -91,22 +101,23 @@ struct KGeo {
   static constexpr uint32_t TMEM_COLS = 512, C_COL = 0, P_COL = 128, Z_COL0 = 256;
   static_assert(Z_COL0 + 128 * (NV - 1) + D <= TMEM_COLS, "tensor memory");
   static_assert(OFF_K % 1024 == 0 && OFF_V % 1024 == 0, "swizzle alignment");
-  static_assert(OFF_FAC % 16 == 0, "vector loads of the column scales");
-  static_assert(MIX != 2 || BM * XSTR * 4 <= kNStage * KCHUNK + V_BYTES, "exchange buffer");
+  static_assert(OFF_SMALL % 16 == 0, "alignment");
+  static_assert(NS >= 3, "Kt ring");
+  static_assert(MIX != 2 || BM * XSTR * 4 <= NS * KCHUNK + V_BYTES, "exchange buffer");
   static_assert(SMEM <= 232448, "shared memory");
   static_assert(CQ * CK <= 120, "kernel taps");
 };
 
 struct KqParams {
-  const float *theta;   // [H][CQ][CK] (raw; the Mask_0 correction uses it)
+  const float *theta;   // [H][CQ][CK]
   const float *w;       // [H/2][2][2]
   __nv_bfloat16 *out;   // [B][L][H][D]
   const float *gamma, *beta;
   float eps, lam;
   int gn;
-  int L, H, n_qtiles;
+  int L, H, n_qtiles, lpad;
   float qk_scale;
-  const float *fac;     // [B][H][L] 2^-e_j of the convolved key rows
+  const float *fac;     // [B][H][lpad] s*log2(e)*2^-e_j per convolved key row (0 past L)
   const float *vp;      // [B][H][L][M] past dot products
   unsigned *err;
 };
@@ -134,22 +145,25 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint8_t *Ks = smem + G::OFF_K;
   uint8_t *Vs = smem + G::OFF_V;
   float *Us = reinterpret_cast<float *>(smem + G::OFF_U);
-  float *Cs = reinterpret_cast<float *>(smem + G::OFF_CORR);
-  float *facs = reinterpret_cast<float *>(smem + G::OFF_FAC);
+  float *Cs = reinterpret_cast<float *>(smem + G::OFF_CS);
+  float *red = reinterpret_cast<float *>(smem + G::OFF_RED);
+  float *facs = reinterpret_cast<float *>(smem + G::OFF_FAC);  // [2][BN]
   uint8_t *small = smem + G::OFF_SMALL;
   float *th_s = reinterpret_cast<float *>(small);          // [CQ*CK]
   float *w_s = reinterpret_cast<float *>(small + 512);     // [4]
-  float *red = reinterpret_cast<float *>(small + 528);     // [4]
+  float *qred = reinterpret_cast<float *>(small + 528);    // [8] per-warp max |q|
   uint64_t *bars = reinterpret_cast<uint64_t *>(small + 640);
-  uint64_t *q_full = bars + 0, *q_ready = bars + 1, *k_full = bars + 2, *k_empty = bars + 2 + kNStage;
-  uint64_t *v_full = bars + 2 + 2 * kNStage, *v_empty = v_full + 1, *c_full = v_full + 2;
+  uint64_t *q_full = bars + 0, *q_ready = bars + 1, *k_full = bars + 2, *k_empty = bars + 2 + G::NS;
+  uint64_t *v_full = bars + 2 + 2 * G::NS, *v_empty = v_full + 1, *c_full = v_full + 2;
   uint64_t *c_free = v_full + 3, *p_full = v_full + 4, *mma_done = v_full + 5;
   uint32_t *tslot = reinterpret_cast<uint32_t *>(small + 640 + 8 * 24);
   volatile int *abort_flag = reinterpret_cast<volatile int *>(small + 640 + 8 * 24 + 8);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int h = blockIdx.x, b = blockIdx.y;
-  const int qt = p.n_qtiles - 1 - static_cast<int>(blockIdx.z);  // longest tiles first
+  // the query tiles of one (batch, head) are adjacent in the grid (they share the
+  // head's Kt stream in L2), longest first
+  const int qt = p.n_qtiles - 1 - static_cast<int>(blockIdx.x);
+  const int h = blockIdx.y, b = blockIdx.z;
   const int hr = h & 1, g = h >> 1;
   const int L = p.L;
   const int i0 = qt * G::BM;
@@ -158,10 +172,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int n_kv = last_q / G::BN + 1;
 
   if (threadIdx.x == 0) {
-    mbar_init(q_full, 1); mbar_init(q_ready, 4);
-    for (int s = 0; s < kNStage; ++s) { mbar_init(k_full + s, 1); mbar_init(k_empty + s, 1); }
-    mbar_init(v_full, 1); mbar_init(v_empty, 1); mbar_init(c_full, 1); mbar_init(c_free, 4);
-    mbar_init(p_full, 4); mbar_init(mma_done, 1);
+    mbar_init(q_full, 1); mbar_init(q_ready, 8);
+    for (int s = 0; s < G::NS; ++s) { mbar_init(k_full + s, 1); mbar_init(k_empty + s, 1); }
+    mbar_init(v_full, 1); mbar_init(v_empty, 1); mbar_init(c_full, 1); mbar_init(c_free, 8);
+    mbar_init(p_full, 8); mbar_init(mma_done, 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -169,13 +183,13 @@ __global__ void __launch_bounds__(kThreads, 1)
     th_s[threadIdx.x - 32] = p.theta[static_cast<long long>(h) * CQ * CK + (threadIdx.x - 32)];
   if (MIX == 2 && threadIdx.x >= 192 && threadIdx.x < 196)
     w_s[threadIdx.x - 192] = p.w[static_cast<long long>(g) * 4 + (threadIdx.x - 192)];
-  if (warp == 1) { tmem_alloc(tslot, G::TMEM_COLS); tmem_relinquish(); }
+  if (warp == kMmaWarp) { tmem_alloc(tslot, G::TMEM_COLS); tmem_relinquish(); }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tslot;
 
-  if (warp == 0) {
+  if (warp == kTmaWarp) {
     // -------------------------------------------------------------- TMA
     if (lane == 0) {
       prefetch_tmap(&tmQ); prefetch_tmap(&tmK);
@@ -186,15 +200,15 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int zbase = (b * p.H + h) * CQ;
       for (int t = 0; t < n_kv && !*abort_flag; ++t)
         for (int ch = 0; ch < G::NCH; ++ch, ++cnt) {
-          const int st = cnt % kNStage;
-          if (!mbar_wait(k_empty + st, ((cnt / kNStage) & 1) ^ 1, abort_flag, p.err)) break;
+          const int st = cnt % G::NS;
+          if (!mbar_wait(k_empty + st, ((cnt / G::NS) & 1) ^ 1, abort_flag, p.err)) break;
           mbar_arrive_expect_tx(k_full + st, G::KCHUNK);
           tma_load_3d(Ks + st * G::KCHUNK, &tmK, k_full + st, (ch % G::NDC) * 64, t * G::BN, zbase + ch / G::NDC);
         }
       drain_wait(q_full, 0);
       if (*abort_flag)
-        for (int c2 = (cnt > kNStage ? cnt - kNStage : 0); c2 < cnt; ++c2)
-          drain_wait(k_full + c2 % kNStage, (c2 / kNStage) & 1);
+        for (int c2 = (cnt > G::NS ? cnt - G::NS : 0); c2 < cnt; ++c2)
+          drain_wait(k_full + c2 % G::NS, (c2 / G::NS) & 1);
     } else if (lane == 1) {
       prefetch_tmap(&tmV);
       int nv = 0;
@@ -211,29 +225,32 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       if (*abort_flag && nv) drain_wait(v_full, (nv - 1) & 1);
     }
-  } else if (warp == 1) {
+  } else if (warp == kMmaWarp) {
     // -------------------------------------------------------------- MMA
     if (lane == 0) {
       const uint32_t idesc_c = idesc_f16_f32(128, G::BN);
       const uint32_t idesc_pv = idesc_bf16_f32(128, D, 0, 1);
-      const uint32_t q_base = smem_u32(Qs), k_base = smem_u32(Ks), v_base = smem_u32(Vs);
+      // descriptors of the first operand tiles; every other tile differs only in its
+      // start address (field bits 0-13, address / 16), added below
+      const uint64_t qdesc0 = sdesc_noswz(smem_u32(Qs), G::STRIP, 128);
+      const uint64_t kdesc0 = sdesc_sw128(smem_u32(Ks), 16, 1024);
+      const uint64_t vdesc0 = sdesc_sw128(smem_u32(Vs), G::V_CHUNK, 1024);
       int cnt = 0;
       bool ok = mbar_wait(q_ready, 0, abort_flag, p.err);
       // C(t) = sum over the NCH chunks (a, 64-wide d block) of Q shifted by a rows x Kt_a
       auto issue_c = [&](int t) -> bool {
         if (t > 0 && !mbar_wait(c_free, (t - 1) & 1, abort_flag, p.err)) return false;
         for (int ch = 0; ch < G::NCH; ++ch, ++cnt) {
-          const int st = cnt % kNStage;
-          if (!mbar_wait(k_full + st, (cnt / kNStage) & 1, abort_flag, p.err)) return false;
+          const int st = cnt % G::NS;
+          if (!mbar_wait(k_full + st, (cnt / G::NS) & 1, abort_flag, p.err)) return false;
           tc_fence_after();
           const int a = ch / G::NDC, dc = ch % G::NDC;
+          // Q rows shifted up by a (16 bytes per row), 64-channel block dc
+          const uint64_t qd = qdesc0 + static_cast<uint32_t>((8 * dc * G::STRIP + 16 * (G::HALO - a)) >> 4);
+          const uint64_t kd = kdesc0 + static_cast<uint32_t>((st * G::KCHUNK) >> 4);
 #pragma unroll
-          for (int kk = 0; kk < 4; ++kk) {
-            const uint32_t qa = q_base + (8 * dc + 2 * kk) * G::STRIP + 16 * (G::HALO - a);
-            mma_bf16_ss(tmem + G::C_COL, sdesc_noswz(qa, G::STRIP, 128),
-                        sdesc_sw128(k_base + st * G::KCHUNK + kk * 32, 16, 1024), idesc_c,
-                        (ch > 0 || kk > 0));
-          }
+          for (int kk = 0; kk < 4; ++kk)
+            mma_bf16_ss(tmem + G::C_COL, qd + (2 * kk * G::STRIP >> 4), kd + 2 * kk, idesc_c, (ch > 0 || kk > 0));
           mma_commit(k_empty + st);
         }
         mma_commit(c_full);
@@ -250,23 +267,25 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
           for (int kk = 0; kk < G::BN / 16; ++kk)
             mma_f16_ts(tmem + G::Z_COL0 + 128 * hd, tmem + G::P_COL + 8 * kk,
-                       sdesc_sw128(v_base + hd * G::V_HEAD + kk * 16 * 128, G::V_CHUNK, 1024),
-                       idesc_pv, (t > 0 || kk > 0));
+                       vdesc0 + ((hd * G::V_HEAD + kk * 16 * 128) >> 4), idesc_pv, (t > 0 || kk > 0));
         mma_commit(v_empty);
       }
       mma_commit(mma_done);
       drain_wait(mma_done, 0);
     }
-  } else if (warp >= kSmWarp0) {
-    // ------------------------------------------------------ softmax group
-    const int q4 = warp & 3;
+  } else {
+    // ---------------------------------------------- softmax warpgroups
+    const int wg = warp >> 2, q4 = warp & 3;
     const int r = 32 * q4 + lane;            // query row of this thread = TMEM lane
     const int qi = i0 + r;
     const bool out_row = qi < L;
-    const int st_id = threadIdx.x - 32 * kSmWarp0;  // 0..127
+    const int st_id = threadIdx.x;           // 0..255
+    const int cb = G::HALF * wg;             // key columns of this warpgroup
+    const int zc = G::DH * wg;               // output channels of this warpgroup
     const uint32_t tl = tmem + (static_cast<uint32_t>(32 * q4) << 16);
 
-    // stage: queries in fp16 with a power-of-2 scale (no overflow), and U rows
+    // stage: queries in fp16 (scaled down by a power of 2 only if |q| > 2^14), and
+    // the past dot products of the staged rows
     mbar_wait(q_full, 0, abort_flag, p.err);
     float qmax = 0.f;
     for (int c16 = st_id; c16 < G::Q_BYTES / 16; c16 += kSmThreads) {
@@ -278,10 +297,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) qmax = fmaxf(qmax, __shfl_xor_sync(0xffffffffu, qmax, o));
-    if (lane == 0) red[q4] = qmax;
-    named_bar_sync(kBarSm, kSmThreads);
-    qmax = fmaxf(fmaxf(red[0], red[1]), fmaxf(red[2], red[3]));
-    // scale down only (|q| > 2^14): otherwise the fp16 queries are the bf16 ones
+    if (lane == 0) qred[warp] = qmax;
+    named_bar_sync(kBarAll, kSmThreads);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) qmax = fmaxf(qmax, qred[i]);
     int eq = 0;
     if (qmax > 16384.f) eq = max(-60, static_cast<int>(floorf(log2f(16384.f / qmax))));
     const float qsc = exp2f(static_cast<float>(eq));
@@ -305,71 +324,91 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int rr = e / G::M, k = e % G::M, iq = row0 + rr;
       Us[e] = (iq >= 0 && iq < L) ? p.vp[(bh * L + iq) * G::M + k] : 0.f;
     }
+    // column factors of key tile t are staged in facs[t & 1] one tile ahead; the
+    // barrier of tile t-1 (here: the one below) publishes them
+    const float *fac = p.fac + bh * p.lpad;
+    if (st_id < G::BN) facs[st_id] = fac[st_id];
+    named_bar_sync(kBarAll, kSmThreads);
 
     const float sc0 = p.qk_scale * kLog2e;
-    const float sc = sc0 * exp2f(static_cast<float>(-eq));
-    const float *fac = p.fac + bh * L;
+    const float qinv = exp2f(static_cast<float>(-eq));
+    float *crow = Cs + (wg * G::BM + r) * G::W;
     float m_run = -INFINITY, l_run = 0.f;
     for (int t = 0; t < n_kv; ++t) {
       const int j0 = t * G::BN;
-      // column scales of this key tile (double-buffered: the barrier below also
-      // tells every thread that the others are done with tile t-2's buffer)
-      float *fs = facs + (t & 1) * G::BN;
-      fs[st_id] = fac[min(j0 + st_id, L - 1)] * sc;
-      named_bar_sync(kBarSm, kSmThreads);
+      // next tile's column factors (stored before this tile's barrier, read after it)
+      const float fnext = (st_id < G::BN && t + 1 < n_kv) ? fac[j0 + G::BN + st_id] : 0.f;
+      const float4 *f4 = reinterpret_cast<const float4 *>(facs + (t & 1) * G::BN + cb);
       mbar_wait(c_full, t & 1, abort_flag, p.err);
       tc_fence_after();
-      float cv[G::BN];
+      float cv[G::HALF];
 #pragma unroll
-      for (int c0 = 0; c0 < G::BN; c0 += 32) {
+      for (int c0 = 0; c0 < G::HALF; c0 += 32) {
         uint32_t u32[32];
-        tmem_ld32(tl + G::C_COL + c0, u32);
+        tmem_ld32(tl + G::C_COL + cb + c0, u32);
+        float4 f[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) f[i] = f4[c0 / 4 + i];
         tmem_wait_ld();
 #pragma unroll
-        for (int i = 0; i < 32; i += 4) {
-          const float4 f4 = *reinterpret_cast<const float4 *>(fs + c0 + i);
-          cv[c0 + i] = __uint_as_float(u32[i]) * f4.x;
-          cv[c0 + i + 1] = __uint_as_float(u32[i + 1]) * f4.y;
-          cv[c0 + i + 2] = __uint_as_float(u32[i + 2]) * f4.z;
-          cv[c0 + i + 3] = __uint_as_float(u32[i + 3]) * f4.w;
+        for (int i = 0; i < 8; ++i) {
+          cv[c0 + 4 * i] = __uint_as_float(u32[4 * i]) * f[i].x;
+          cv[c0 + 4 * i + 1] = __uint_as_float(u32[4 * i + 1]) * f[i].y;
+          cv[c0 + 4 * i + 2] = __uint_as_float(u32[4 * i + 2]) * f[i].z;
+          cv[c0 + 4 * i + 3] = __uint_as_float(u32[4 * i + 3]) * f[i].w;
         }
       }
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(c_free);
+      if (eq != 0) {  // queries were scaled down (|q| > 2^14)
+#pragma unroll
+        for (int jj = 0; jj < G::HALF; ++jj) cv[jj] *= qinv;
+      }
       // the band 0 <= i-j < W, where Mask_0 removes taps: the convolution tap by
-      // tap over the unmasked taps, from the past dot products
-      const int dmax = qi - j0;  // i - j for jj = 0
-      if (out_row && dmax >= 0 && dmax - (G::BN - 1) < G::W) {
-        float *crow = Cs + r * G::W;
-#pragma unroll 1
-        for (int dd = 0; dd < G::W; ++dd) {
-          float val = 0.f;
-          const int j = qi - dd;
-          if (j >= j0 && j < j0 + G::BN) {
-#pragma unroll 1
-            for (int a = 0; a < CQ; ++a) {
-              if (qi - a < 0) break;
-              const float *vrow = Us + (r + G::HALO - a) * G::M;
-              // tap t reads key j-(t-c) = (i-a) - m with m = dd - a + (t - c) >= 0
-              for (int t = max(0, a + G::C - dd); t < CK; ++t)
-                val = fmaf(th_s[a * CK + t], vrow[dd - a + t - G::C], val);
+      // tap over the unmasked taps, from the past dot products:
+      //   C[i][i-dd] = s * sum_{a,t: m = dd - a + (t - c) >= 0} theta[a][t] Vp[i-a][m]
+      const int dmax = qi - j0 - cb;  // i - j for this warpgroup's first column
+      if (out_row && dmax >= 0 && dmax - (G::W - 1) < G::HALF) {
+        float acc[G::W];
+#pragma unroll
+        for (int dd = 0; dd < G::W; ++dd) acc[dd] = 0.f;
+#pragma unroll
+        for (int a = 0; a < CQ; ++a) {
+          const float *vrow = Us + (r + G::HALO - a) * G::M;  // rows before query 0 are zero
+          float vr[G::M];
+#pragma unroll
+          for (int m = 0; m < G::M; ++m) vr[m] = vrow[m];
+#pragma unroll
+          for (int t = 0; t < CK; ++t) {
+            const float th = th_s[a * CK + t];
+#pragma unroll
+            for (int dd = 0; dd < G::W; ++dd) {
+              const int m = dd - a + t - G::C;
+              if (m >= 0 && m < G::M) acc[dd] = fmaf(th, vr[m], acc[dd]);
             }
           }
-          crow[dd] = val * sc0;
         }
 #pragma unroll
-        for (int jj = 0; jj < G::BN; ++jj) {
+        for (int dd = 0; dd < G::W; ++dd) crow[dd] = acc[dd] * sc0;
+#pragma unroll
+        for (int jj = 0; jj < G::HALF; ++jj) {
           const int dd = dmax - jj;
           if (static_cast<unsigned>(dd) < static_cast<unsigned>(G::W)) cv[jj] = crow[dd];
         }
       }
-      __syncwarp();  // the warp-collective tensor-memory accesses below need the whole warp
-      // Mask_-inf and the tile's row max (log2 units)
+      // Mask_-inf (only the diagonal tile holds keys after a query) and the row max
+      // over both warpgroups' columns (log2 units)
+      if (t == n_kv - 1) {
 #pragma unroll
-      for (int jj = 0; jj < G::BN; ++jj)
-        if (j0 + jj > qi) cv[jj] = -INFINITY;
-      const float mt = out_row ? tree_max<G::BN>(cv) : -INFINITY;
+        for (int jj = 0; jj < G::HALF; ++jj)
+          if (j0 + cb + jj > qi) cv[jj] = -INFINITY;
+      }
+      float *rmx = red + (t & 1) * 2 * G::BM;
+      rmx[wg * G::BM + r] = out_row ? tree_max<G::HALF>(cv) : -INFINITY;
+      if (st_id < G::BN) facs[((t + 1) & 1) * G::BN + st_id] = fnext;
+      named_bar_sync(kBarAll, kSmThreads);
+      const float mt = fmaxf(rmx[r], rmx[G::BM + r]);
       const float m_new = fmaxf(m_run, mt);
       bool resc = false;
       float alpha = 1.f;
@@ -387,30 +426,28 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (__any_sync(0xffffffffu, resc)) {  // warp-collective tensor-memory access
         l_run *= alpha;
 #pragma unroll 1
-        for (int c0 = 0; c0 < 128 * (G::NV - 1) + D; c0 += 32) {
-          if (G::NV == 2 && c0 >= D && c0 < 128) continue;
-          uint32_t z[32];
-          tmem_ld32(tl + G::Z_COL0 + c0, z);
-          tmem_wait_ld();
+        for (int hd = 0; hd < G::NV; ++hd)
+#pragma unroll 1
+          for (int c0 = 0; c0 < G::DH; c0 += 32) {
+            uint32_t z[32];
+            const uint32_t za = tl + G::Z_COL0 + 128 * hd + zc + c0;
+            tmem_ld32(za, z);
+            tmem_wait_ld();
 #pragma unroll
-          for (int i = 0; i < 32; ++i) z[i] = __float_as_uint(__uint_as_float(z[i]) * alpha);
-          tmem_st32(tl + G::Z_COL0 + c0, z);
-        }
+            for (int i = 0; i < 32; ++i) z[i] = __float_as_uint(__uint_as_float(z[i]) * alpha);
+            tmem_st32(za, z);
+          }
       }
       float ls = 0.f;
+      uint32_t pk[32];
 #pragma unroll
-      for (int half = 0; half < 2; ++half) {
-        uint32_t pk[32];
-#pragma unroll
-        for (int q2 = 0; q2 < 32; ++q2) {
-          const int jj = 64 * half + 2 * q2;
-          const float p0 = out_row ? ex2(cv[jj] - m_run) : 0.f;
-          const float p1 = out_row ? ex2(cv[jj + 1] - m_run) : 0.f;
-          ls += p0 + p1;
-          pk[q2] = pack_bf16x2(p0, p1);
-        }
-        tmem_st32(tl + G::P_COL + 32 * half, pk);
+      for (int q2 = 0; q2 < 32; ++q2) {
+        const float p0 = out_row ? ex2(cv[2 * q2] - m_run) : 0.f;
+        const float p1 = out_row ? ex2(cv[2 * q2 + 1] - m_run) : 0.f;
+        ls += p0 + p1;
+        pk[q2] = pack_bf16x2(p0, p1);
       }
+      tmem_st32(tl + G::P_COL + 32 * wg, pk);
       l_run += ls;
       tmem_wait_st();
       tc_fence_before();
@@ -419,19 +456,22 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     mbar_wait(v_empty, (n_kv - 1) & 1, abort_flag, p.err);
     tc_fence_after();
-    const float inv_l = (out_row && l_run > 0.f) ? 1.f / l_run : 0.f;
+    red[(4 + wg) * G::BM + r] = l_run;
+    named_bar_sync(kBarAll, kSmThreads);
+    const float l_tot = l_run + red[(4 + (wg ^ 1)) * G::BM + r];
+    const float inv_l = (out_row && l_tot > 0.f) ? 1.f / l_tot : 0.f;
 
     // ---------------------------------------------------------- epilogue
-    float o[D];
+    float o[G::DH];
     if constexpr (MIX == 2) {
       float *xbuf = reinterpret_cast<float *>(Ks);  // [BM][XSTR] fp32, reuses the ring and V
       __syncwarp();
       cluster_sync_all();                           // both CTAs are done with their ring and V
-      const uint32_t dst = map_peer(smem_u32(xbuf + r * G::XSTR), static_cast<uint32_t>(hr ^ 1));
+      const uint32_t dst = map_peer(smem_u32(xbuf + r * G::XSTR + zc), static_cast<uint32_t>(hr ^ 1));
 #pragma unroll
-      for (int c0 = 0; c0 < D; c0 += 32) {
+      for (int c0 = 0; c0 < G::DH; c0 += 32) {
         uint32_t z[32];
-        tmem_ld32(tl + G::Z_COL0 + 128 * (hr ^ 1) + c0, z);
+        tmem_ld32(tl + G::Z_COL0 + 128 * (hr ^ 1) + zc + c0, z);
         tmem_wait_ld();
 #pragma unroll
         for (int i = 0; i < 32; i += 4)
@@ -440,20 +480,20 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       cluster_sync_all();  // the peer's Z_{peer->h} / l_peer is in xbuf
       const float w_own = w_s[hr * 2 + hr], w_peer = w_s[hr * 2 + (hr ^ 1)];
-      const float *xr = xbuf + r * G::XSTR;
+      const float *xr = xbuf + r * G::XSTR + zc;
 #pragma unroll
-      for (int c0 = 0; c0 < D; c0 += 32) {
+      for (int c0 = 0; c0 < G::DH; c0 += 32) {
         uint32_t z[32];
-        tmem_ld32(tl + G::Z_COL0 + 128 * hr + c0, z);
+        tmem_ld32(tl + G::Z_COL0 + 128 * hr + zc + c0, z);
         tmem_wait_ld();
 #pragma unroll
         for (int i = 0; i < 32; ++i) o[c0 + i] = w_own * (__uint_as_float(z[i]) * inv_l) + w_peer * xr[c0 + i];
       }
     } else {
 #pragma unroll
-      for (int c0 = 0; c0 < D; c0 += 32) {
+      for (int c0 = 0; c0 < G::DH; c0 += 32) {
         uint32_t z[32];
-        tmem_ld32(tl + G::Z_COL0 + c0, z);
+        tmem_ld32(tl + G::Z_COL0 + zc + c0, z);
         tmem_wait_ld();
 #pragma unroll
         for (int i = 0; i < 32; ++i) o[c0 + i] = __uint_as_float(z[i]) * inv_l;
@@ -462,21 +502,25 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (p.gn) {  // group norm over the D channels of (token, head), then depth scale
       float s = 0.f;
 #pragma unroll
-      for (int i = 0; i < D; ++i) s += o[i];
-      const float mu = s * (1.f / D);
+      for (int i = 0; i < G::DH; ++i) s += o[i];
+      red[(6 + wg) * G::BM + r] = s;
+      named_bar_sync(kBarAll, kSmThreads);
+      const float mu = (s + red[(6 + (wg ^ 1)) * G::BM + r]) * (1.f / D);
       float s2 = 0.f;
 #pragma unroll
-      for (int i = 0; i < D; ++i) { const float x = o[i] - mu; s2 += x * x; }
-      const float rstd = rsqrtf(s2 * (1.f / D) + p.eps);
-      const float *gm = p.gamma + static_cast<long long>(h) * D;
-      const float *bt = p.beta + static_cast<long long>(h) * D;
+      for (int i = 0; i < G::DH; ++i) { const float x = o[i] - mu; s2 += x * x; }
+      red[(8 + wg) * G::BM + r] = s2;
+      named_bar_sync(kBarAll, kSmThreads);
+      const float rstd = rsqrtf((s2 + red[(8 + (wg ^ 1)) * G::BM + r]) * (1.f / D) + p.eps);
+      const float *gm = p.gamma + static_cast<long long>(h) * D + zc;
+      const float *bt = p.beta + static_cast<long long>(h) * D + zc;
 #pragma unroll
-      for (int i = 0; i < D; ++i) o[i] = ((o[i] - mu) * rstd * gm[i] + bt[i]) * p.lam;
+      for (int i = 0; i < G::DH; ++i) o[i] = ((o[i] - mu) * rstd * gm[i] + bt[i]) * p.lam;
     }
     if (out_row) {
-      __nv_bfloat16 *dst = p.out + ((static_cast<long long>(b) * L + qi) * p.H + h) * D;
+      __nv_bfloat16 *dst = p.out + ((static_cast<long long>(b) * L + qi) * p.H + h) * D + zc;
 #pragma unroll
-      for (int i = 0; i < D; i += 8) {
+      for (int i = 0; i < G::DH; i += 8) {
         uint4 v;
         v.x = pack_bf16x2(o[i], o[i + 1]);
         v.y = pack_bf16x2(o[i + 2], o[i + 3]);
@@ -486,14 +530,14 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
     }
   }
-  if (MIX == 2 && warp < kSmWarp0) {  // the other warps take part in the cluster barriers
-    __syncwarp();  // lanes 0 and 1 of warp 0 and lane 0 of warp 1 return from their roles
+  if (MIX == 2 && warp >= kTmaWarp) {  // the producer warps take part in the cluster barriers
+    __syncwarp();  // their lanes return from their roles separately
     cluster_sync_all();
     cluster_sync_all();
   }
   tc_fence_before();
   __syncthreads();
-  if (warp == 1) {
+  if (warp == kMmaWarp) {
     tc_fence_after();
     tmem_dealloc(tmem, G::TMEM_COLS);
   }
@@ -531,6 +575,7 @@ cudaError_t launch_kq_one(const AttnArgs &a, const GnArgs *gn, const KqPrepArgs 
   p.H = a.H;
   p.n_qtiles = (a.L + G::BM - 1) / G::BM;
   p.qk_scale = a.scale;
+  p.lpad = pa.lpad;
   p.fac = pa.fac;
   p.vp = pa.vp;
   p.err = a.err;
@@ -538,14 +583,14 @@ cudaError_t launch_kq_one(const AttnArgs &a, const GnArgs *gn, const KqPrepArgs 
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, G::SMEM);
   if (e != cudaSuccess) return e;
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(a.H, a.B, p.n_qtiles);
+  cfg.gridDim = dim3(p.n_qtiles, a.H, a.B);
   cfg.blockDim = dim3(kThreads);
   cfg.dynamicSmemBytes = G::SMEM;
   cfg.stream = a.stream;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = G::CLUSTER;
-  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.x = 1;
+  attr[0].val.clusterDim.y = G::CLUSTER;  // the two heads of a group
   attr[0].val.clusterDim.z = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
@@ -566,12 +611,14 @@ bool attn_kq_supported(const AttnArgs &a) {
   return al % 16 == 0 && a.rs % 8 == 0;
 }
 
-// Workspace of the contraction path: Kt [B][H][c_q][L][d] fp16 | fac [B][H][L] fp32 |
-// Vp [B][H][L][M] fp32, M = (c_q-1) + 2*(c_k/2); each part 256-byte aligned.
+// Workspace of the contraction path: Kt [B][H][c_q][L][d] fp16 | fac [B][H][Lpad] fp32 |
+// Vp [B][H][L][M] fp32, Lpad = L rounded up to 128, M = (c_q-1) + 2*(c_k/2); each part
+// 256-byte aligned.
 size_t attn_kq_workspace_bytes(int B, int H, int L, int d, int cq, int ck) {
-  const size_t BHL = static_cast<size_t>(B) * H * L;
+  const size_t BH = static_cast<size_t>(B) * H, BHL = BH * L;
+  const size_t lpad = (static_cast<size_t>(L) + 127) / 128 * 128;
   const size_t M = static_cast<size_t>(cq - 1 + 2 * (ck / 2));
-  return align256(BHL * cq * d * 2) + align256(BHL * 4) + align256(BHL * M * 4);
+  return align256(BHL * cq * d * 2) + align256(BH * lpad * 4) + align256(BHL * M * 4);
 }
 
 cudaError_t launch_attn_kq(const AttnArgs &a, const GnArgs *gn, void *ws) {
@@ -583,11 +630,13 @@ cudaError_t launch_attn_kq(const AttnArgs &a, const GnArgs *gn, void *ws) {
   pa.B = a.B; pa.H = a.H; pa.L = a.L; pa.d = a.d; pa.cq = a.cq; pa.ck = a.ck;
   pa.M = a.cq - 1 + 2 * (a.ck / 2);
   pa.n_tiles = (a.L + 127) / 128;
-  const size_t BHL = static_cast<size_t>(a.B) * a.H * a.L;
+  pa.lpad = pa.n_tiles * 128;
+  pa.scale_log2 = a.scale * 1.4426950408889634f;
+  const size_t BH = static_cast<size_t>(a.B) * a.H, BHL = BH * a.L;
   char *base = static_cast<char *>(ws);
   pa.kt = base;
   pa.fac = reinterpret_cast<float *>(base + align256(BHL * a.cq * a.d * 2));
-  pa.vp = reinterpret_cast<float *>(reinterpret_cast<char *>(pa.fac) + align256(BHL * 4));
+  pa.vp = reinterpret_cast<float *>(reinterpret_cast<char *>(pa.fac) + align256(BH * pa.lpad * 4));
   cudaError_t e = launch_kq_prep(pa, a.stream);
   if (e != cudaSuccess) return e;
   const bool post = a.hp == 2;

@@ -45,9 +45,10 @@ struct KqPrepArgs {
   long long rs;
   const float *theta;     // [H][c_q][c_k]
   void *kt;               // [B][H][c_q][L][d] fp16, key row j scaled by 2^e_j
-  float *fac;             // [B][H][L] 2^-e_j
+  float *fac;             // [B][H][lpad] scale_log2 * 2^-e_j (0 for j >= L)
   float *vp;              // [B][H][L][M] past dot products q[i] . k[i-m], m < M
-  int B, H, L, d, cq, ck, M, n_tiles;
+  float scale_log2;       // logit scale times log2(e)
+  int B, H, L, d, cq, ck, M, n_tiles, lpad;
 };
 cudaError_t launch_kq_prep(const KqPrepArgs &a, cudaStream_t stream);
 // Workspace bytes of the contraction path (beyond the error word) and whether it applies.

@@ -15,7 +15,8 @@
 //   Kt  [B][H][c_q][L][d] fp16: Kt_a[j] * 2^e_j, e_j a power-of-2 exponent per key
 //       row chosen from max|k| over the rows j-c .. j+c that Kt_a[j] reads (so no
 //       value exceeds 2^14 and small keys keep fp16's relative precision);
-//   fac [B][H][L] fp32: 2^-e_j;
+//   fac [B][H][Lpad] fp32: s * log2(e) * 2^-e_j (the attention kernel's column
+//       factor; 0 for the padding keys L <= j < Lpad, Lpad = L rounded up to 128);
 //   Vp  [B][H][L][M] fp32: raw past dot products (no scale).
 // Every value written for key or query j depends on inputs at positions <= j + c
 // only, and Kt_a[j] is used only for queries i >= j + W > j + c: the path stays
@@ -41,15 +42,33 @@ struct PrepGeo {
   static constexpr int M = (CQ - 1) + 2 * C;          // past dot products per query
   static constexpr int LO = M - 1;                    // staged rows before the tile
   static constexpr int ROWS = kTile + LO + C;         // keys j0-LO .. j0+kTile-1+C
-  static constexpr int SMEM = ROWS * D * 4;
+  static constexpr int KSTR = D + 8;                  // staged row stride (floats): fewer bank conflicts
+  static constexpr int SMEM = ROWS * KSTR * 4;
+  static_assert(M - 1 + 16 <= 32, "past dot products of a 16-row block span 32 keys");
 };
+
+// D[16x8] += A[16x16] * B[16x8], bf16 inputs, fp32 accumulate (warp-wide).
+__device__ __forceinline__ void mma_m16n8k16_bf16(float (&c)[4], const uint32_t (&a)[4], uint32_t b0,
+                                                  uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+      "{%0,%1,%2,%3};"
+      : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
+// two floats that are bf16 values, packed exactly (low half = first)
+__device__ __forceinline__ uint32_t pack2_bf16(float lo, float hi) {
+  const __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
+  return *reinterpret_cast<const uint32_t *>(&v);
+}
 
 __device__ __forceinline__ float pow2i(int e) { return __int_as_float((127 + e) << 23); }  // |e| <= 126
 
 template <int D, int CQ, int CK>
 __global__ void __launch_bounds__(kPrepThreads) kq_prep_kernel(KqPrepArgs p) {
   using G = PrepGeo<D, CQ, CK>;
-  extern __shared__ float ks[];  // [ROWS][D] fp32, row r = key j0 - LO + r
+  extern __shared__ float ks[];  // [ROWS][KSTR] fp32, row r = key j0 - LO + r
   __shared__ float rmax[G::ROWS];
   __shared__ int es[kTile];
   __shared__ float th[CQ * CK];
@@ -79,7 +98,7 @@ __global__ void __launch_bounds__(kPrepThreads) kq_prep_kernel(KqPrepArgs p) {
     float m = 0.f;
 #pragma unroll
     for (int u = 0; u < 8; ++u) {
-      ks[r * D + e8 + u] = v[u];
+      ks[r * G::KSTR + e8 + u] = v[u];
       m = fmaxf(m, fabsf(v[u]));
     }
     atomicMax(reinterpret_cast<int *>(rmax + r), __float_as_int(m));  // non-negative floats order as ints
@@ -102,66 +121,92 @@ __global__ void __launch_bounds__(kPrepThreads) kq_prep_kernel(KqPrepArgs p) {
     int e = 0;
     if (bound > 0.f) e = max(-60, min(60, static_cast<int>(floorf(log2f(16384.f / bound)))));
     es[tid] = e;
-    if (j0 + tid < L) p.fac[bh * L + j0 + tid] = pow2i(-e);
+    p.fac[bh * p.lpad + j0 + tid] = j0 + tid < L ? pow2i(-e) * p.scale_log2 : 0.f;
   }
   __syncthreads();
 
   // Kt_a[j] = sum_t theta[a][t] k[j - (t - c)]: each work item is one pair of
   // channels x kRun consecutive keys, convolved from a register window of rows.
   __half *kt = static_cast<__half *>(p.kt);
+  const long long LD = static_cast<long long>(L) * D;  // elements between the Kt_a of one head
   constexpr int NPAIR = D / 2, NRUN = kTile / kRun;
   for (int item = tid; item < NPAIR * NRUN; item += kPrepThreads) {
     const int e2 = (item % NPAIR) * 2, jr = (item / NPAIR) * kRun;
+    if (j0 + jr >= L) continue;
+    const int nkeys = min(kRun, L - (j0 + jr));
     float2 win[kRun + 2 * G::C];  // keys j0+jr-c .. j0+jr+kRun-1+c
 #pragma unroll
     for (int w = 0; w < kRun + 2 * G::C; ++w)
-      win[w] = *reinterpret_cast<const float2 *>(ks + (jr + w + G::LO - G::C) * D + e2);
+      win[w] = *reinterpret_cast<const float2 *>(ks + (jr + w + G::LO - G::C) * G::KSTR + e2);
+    float scu[kRun];
+#pragma unroll
+    for (int u = 0; u < kRun; ++u) scu[u] = pow2i(es[jr + u]);
+    __half *o0 = kt + (bh * CQ * L + j0 + jr) * D + e2;
 #pragma unroll
     for (int a = 0; a < CQ; ++a) {
       float ta[CK];
 #pragma unroll
       for (int t = 0; t < CK; ++t) ta[t] = th[a * CK + t];
+      __half *oa = o0 + a * LD;
 #pragma unroll
       for (int u = 0; u < kRun; ++u) {
-        const int key = j0 + jr + u;
         float s0 = 0.f, s1 = 0.f;
 #pragma unroll
         for (int t = 0; t < CK; ++t) {  // key j - (t - c) is window entry u + 2c - t
           s0 = fmaf(ta[t], win[u + 2 * G::C - t].x, s0);
           s1 = fmaf(ta[t], win[u + 2 * G::C - t].y, s1);
         }
-        if (key < L) {
-          const float sc = pow2i(es[jr + u]);
-          const long long o = ((bh * CQ + a) * L + key) * D + e2;
-          *reinterpret_cast<__half2 *>(kt + o) = __floats2half2_rn(s0 * sc, s1 * sc);
-        }
+        if (nkeys == kRun || u < nkeys)
+          *reinterpret_cast<__half2 *>(oa + u * D) = __floats2half2_rn(s0 * scu[u], s1 * scu[u]);
       }
     }
   }
 
-  // Vp[i][m] = q[i] . k[i-m]: one warp per query row, channels spread over lanes
-  constexpr int PER_LANE = D / 32;
-  const int warp = tid >> 5, lane = tid & 31;
-  for (int r = warp; r < kTile; r += kPrepThreads / 32) {
-    const int qi = j0 + r;
-    if (qi >= L) break;
-    const __nv_bfloat16 *qr = qb + (static_cast<long long>(b) * L + qi) * p.rs + static_cast<long long>(h) * D;
-    float qv[PER_LANE];
+  // Vp[i][m] = q[i] . k[i-m]: per warp a block of 16 query rows i0 .. i0+15 against
+  // the 32 keys i0-(M-1) .. i0+32-M (a 16x32 tile of Q K^T on the tensor cores,
+  // exact products of bf16 values, fp32 sums), of which the band m < M is kept.
+  const int warp = tid >> 5, lane = tid & 31, g = lane >> 2, tq = lane & 3;
+  const int i0 = 16 * warp;                 // local query row of the block
+  const int krow0 = i0;                     // staged row of key j0+i0-(M-1) (= LO - (M-1) + i0)
+  float acc[4][4];
 #pragma unroll
-    for (int u = 0; u < PER_LANE; ++u) qv[u] = __bfloat162float(qr[lane * PER_LANE + u]);
-    float mine = 0.f;
+  for (int nt = 0; nt < 4; ++nt)
 #pragma unroll
-    for (int m = 0; m < G::M; ++m) {
-      const float *kr = ks + (r + G::LO - m) * D + lane * PER_LANE;
-      float s = 0.f;
+    for (int u = 0; u < 4; ++u) acc[nt][u] = 0.f;
+  const uint32_t *q32[2];
+  bool qok[2];
 #pragma unroll
-      for (int u = 0; u < PER_LANE; ++u) s = fmaf(qv[u], kr[u], s);
-#pragma unroll
-      for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
-      if (lane == m) mine = s;
-    }
-    if (lane < G::M) p.vp[(bh * L + qi) * G::M + lane] = mine;
+  for (int hh = 0; hh < 2; ++hh) {
+    const int qi = j0 + i0 + g + 8 * hh;
+    qok[hh] = qi < L;
+    q32[hh] = reinterpret_cast<const uint32_t *>(qb + (static_cast<long long>(b) * L + (qok[hh] ? qi : 0)) * p.rs +
+                                                 static_cast<long long>(h) * D);
   }
+#pragma unroll
+  for (int kc = 0; kc < D / 16; ++kc) {
+    const int c0 = kc * 16 + 2 * tq;
+    uint32_t a[4];
+    a[0] = qok[0] ? q32[0][c0 / 2] : 0u;
+    a[1] = qok[1] ? q32[1][c0 / 2] : 0u;
+    a[2] = qok[0] ? q32[0][c0 / 2 + 4] : 0u;
+    a[3] = qok[1] ? q32[1][c0 / 2 + 4] : 0u;
+#pragma unroll
+    for (int nt = 0; nt < 4; ++nt) {
+      const float *kr = ks + (krow0 + 8 * nt + g) * G::KSTR + c0;
+      const float2 lo = *reinterpret_cast<const float2 *>(kr);
+      const float2 hi = *reinterpret_cast<const float2 *>(kr + 8);
+      mma_m16n8k16_bf16(acc[nt], a, pack2_bf16(lo.x, lo.y), pack2_bf16(hi.x, hi.y));
+    }
+  }
+  // acc[nt][u]: row i0 + g + 8*(u/2), key column kk = 8*nt + 2*tq + (u&1); m = row - key
+#pragma unroll
+  for (int nt = 0; nt < 4; ++nt)
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int il = g + 8 * (u >> 1), kk = 8 * nt + 2 * tq + (u & 1);
+      const int m = il + (G::M - 1) - kk, qi = j0 + i0 + il;
+      if (m >= 0 && m < G::M && qi < L) p.vp[(bh * L + qi) * G::M + m] = acc[nt][u];
+    }
 }
 
 template <int D, int CQ, int CK>
