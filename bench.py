@@ -133,6 +133,12 @@ def read_traffic(kernel_key: str, workload: str):
     return None if e is None else e.get("bytes_per_launch")
 
 
+def call_traffic(kernel_keys, workload: str):
+    """dram bytes of one call made of several launches (null unless every one is known)."""
+    parts = [read_traffic(k, workload) for k in kernel_keys]
+    return None if any(x is None for x in parts) else sum(parts)
+
+
 # ---------------------------------------------------------------------------
 # clocks during the timed region
 # ---------------------------------------------------------------------------
@@ -525,7 +531,7 @@ def main():
         executed = contraction_tensor_flops(wl) / s / 1e12
         roof = {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
                 "frac": achieved / peak,
-                "traffic": read_traffic("attn_kq_kernel", wl.name),
+                "traffic": call_traffic(("kq_prep_kernel", "attn_kq_kernel"), wl.name),
                 "kernel": "mta_attn_fwd call = kq_prep_kernel + attn_kq_kernel",
                 "per_unit": f"F_mta = 4d + 2 c_q c_k + 2 c_h = {fl['attn_mta'] // wl.causal_pairs} flop "
                             f"per causal pair-head, x {wl.causal_pairs} pair-heads per launch",

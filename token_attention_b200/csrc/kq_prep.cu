@@ -144,21 +144,24 @@ __global__ void __launch_bounds__(kPrepThreads) kq_prep_kernel(KqPrepArgs p) {
     __half *o0 = kt + (bh * CQ * L + j0 + jr) * D + e2;
 #pragma unroll
     for (int a = 0; a < CQ; ++a) {
-      float ta[CK];
+      // kRun x 2 independent accumulators; taps in the outer loop (no dependent chains)
+      float2 acc[kRun];
 #pragma unroll
-      for (int t = 0; t < CK; ++t) ta[t] = th[a * CK + t];
+      for (int u = 0; u < kRun; ++u) acc[u] = make_float2(0.f, 0.f);
+#pragma unroll
+      for (int t = 0; t < CK; ++t) {
+        const float ta = th[a * CK + t];
+#pragma unroll
+        for (int u = 0; u < kRun; ++u) {  // key j - (t - c) is window entry u + 2c - t
+          acc[u].x = fmaf(ta, win[u + 2 * G::C - t].x, acc[u].x);
+          acc[u].y = fmaf(ta, win[u + 2 * G::C - t].y, acc[u].y);
+        }
+      }
       __half *oa = o0 + a * LD;
 #pragma unroll
-      for (int u = 0; u < kRun; ++u) {
-        float s0 = 0.f, s1 = 0.f;
-#pragma unroll
-        for (int t = 0; t < CK; ++t) {  // key j - (t - c) is window entry u + 2c - t
-          s0 = fmaf(ta[t], win[u + 2 * G::C - t].x, s0);
-          s1 = fmaf(ta[t], win[u + 2 * G::C - t].y, s1);
-        }
+      for (int u = 0; u < kRun; ++u)
         if (nkeys == kRun || u < nkeys)
-          *reinterpret_cast<__half2 *>(oa + u * D) = __floats2half2_rn(s0 * scu[u], s1 * scu[u]);
-      }
+          *reinterpret_cast<__half2 *>(oa + u * D) = __floats2half2_rn(acc[u].x * scu[u], acc[u].y * scu[u]);
     }
   }
 
