@@ -106,9 +106,10 @@ typedef struct mta_gn {
 
 /* Bytes of workspace mta_attn_fwd needs for cfg (0 if cfg is invalid): 256
  * bytes, plus, where the contraction kernel applies, its per-call operands
- * (the convolved keys, c_q*B*H*L*d fp16, their B*H*L fp32 scales, and
- * B*H*L*(c_q-1+2*(c_k/2)) fp32 dot products).  With a smaller workspace path 0
- * uses another kernel. */
+ * (the convolved keys, c_q*B*H*L*d fp16, their B*H*L fp32 scales,
+ * B*H*L*(c_q-1+2*(c_k/2)) fp32 dot products and, with post-softmax mixing, an
+ * exchange buffer of at most 160*2*d*128 fp32 for the kernel's persistent CTAs).
+ * With a smaller workspace path 0 uses another kernel. */
 size_t mta_attn_workspace_bytes(const mta_cfg *cfg);
 
 /* MTA attention core, sections 2, 3.1, 3.2 (steps: logits, Mask_0, key-query

@@ -39,6 +39,8 @@
 //     Z_{s->peer}/l_s through distributed shared memory in the epilogue.
 //   * Every mbarrier wait is bounded (error word + early exit).
 #include <cuda.h>
+
+#include <algorithm>
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 #include <math.h>
@@ -58,6 +60,7 @@ constexpr int kThreads = 320;
 constexpr int kSmThreads = 256;
 constexpr int kTmaWarp = 8, kMmaWarp = 9;
 constexpr int kBarAll = 1;      // named barrier over both softmax warpgroups
+constexpr int kKqMaxClusters = 160;  // persistent grid: at most this many CTAs (>= SM count)
 
 template <int D, int CQ, int CK, int MIX>
 struct KGeo {
@@ -71,7 +74,7 @@ struct KGeo {
   static constexpr int NCH = CQ * NDC;                   // Kt chunks per key tile
   static constexpr int KCHUNK = BN * 128;                // 128 keys x 64 elements, fp16
   static constexpr int NV = MIX == 2 ? 2 : 1;
-  static constexpr int CLUSTER = MIX == 2 ? 2 : 1;
+  static constexpr int CLUSTER = MIX == 2 ? 2 : 1;       // CTAs of a cluster: the heads of a group
   static constexpr int V_CHUNK = BN * 128;
   static constexpr int V_HEAD = BN * D * 2;
   static constexpr int V_BYTES = NV * V_HEAD;
@@ -97,13 +100,12 @@ struct KGeo {
   // at least half the SM's shared memory: one CTA per SM, so the 512-column TMEM
   // allocation never waits for another CTA
   static constexpr int SMEM = SMEM_USED > 232448 / 2 + 1024 ? SMEM_USED : 232448 / 2 + 1024;
-  static constexpr int XSTR = D + 4;  // exchange buffer row (post-softmax mix), reuses ring + V
   static constexpr uint32_t TMEM_COLS = 512, C_COL = 0, P_COL = 128, Z_COL0 = 256;
   static_assert(Z_COL0 + 128 * (NV - 1) + D <= TMEM_COLS, "tensor memory");
   static_assert(OFF_K % 1024 == 0 && OFF_V % 1024 == 0, "swizzle alignment");
   static_assert(OFF_SMALL % 16 == 0, "alignment");
   static_assert(NS >= 3, "Kt ring");
-  static_assert(MIX != 2 || BM * XSTR * 4 <= NS * KCHUNK + V_BYTES, "exchange buffer");
+  static_assert(11 + 2 * NS <= 32, "barrier slots");
   static_assert(SMEM <= 232448, "shared memory");
   static_assert(CQ * CK <= 120, "kernel taps");
 };
@@ -115,10 +117,11 @@ struct KqParams {
   const float *gamma, *beta;
   float eps, lam;
   int gn;
-  int L, H, n_qtiles, lpad;
+  int B, L, H, n_qtiles, lpad;
   float qk_scale;
   const float *fac;     // [B][H][lpad] s*log2(e)*2^-e_j per convolved key row (0 past L)
   const float *vp;      // [B][H][L][M] past dot products
+  float *xg;            // post-softmax mixing exchange: [CTA][2][D/4][BM] float4
   unsigned *err;
 };
 
@@ -132,6 +135,24 @@ __device__ __forceinline__ float tree_max(const float (&x)[N]) {
 #pragma unroll
     for (int i = 0; i < s; ++i) m[i] = fmaxf(m[i], m[i + s]);
   return m[0];
+}
+
+// Work item k of a cluster (longest first: query tile qt descending, then batch and
+// head group); clusters take items in a snake order over rounds of n_clusters.
+struct Item {
+  int qt, b, g;
+};
+__device__ __forceinline__ Item item_of(int k, int B, int G, int n_qtiles) {
+  const int per_qt = B * G;
+  Item it;
+  it.qt = n_qtiles - 1 - k / per_qt;
+  const int rem = k % per_qt;
+  it.b = rem / G;
+  it.g = rem % G;
+  return it;
+}
+__device__ __forceinline__ int item_index(int c, int r, int n_clusters) {
+  return r * n_clusters + ((r & 1) ? n_clusters - 1 - c : c);
 }
 
 template <int D, int CQ, int CK, int MIX>
@@ -149,81 +170,99 @@ __global__ void __launch_bounds__(kThreads, 1)
   float *red = reinterpret_cast<float *>(smem + G::OFF_RED);
   float *facs = reinterpret_cast<float *>(smem + G::OFF_FAC);  // [2][BN]
   uint8_t *small = smem + G::OFF_SMALL;
-  float *th_s = reinterpret_cast<float *>(small);          // [CQ*CK]
-  float *w_s = reinterpret_cast<float *>(small + 512);     // [4]
-  float *qred = reinterpret_cast<float *>(small + 528);    // [8] per-warp max |q|
-  uint64_t *bars = reinterpret_cast<uint64_t *>(small + 640);
-  uint64_t *q_full = bars + 0, *q_ready = bars + 1, *k_full = bars + 2, *k_empty = bars + 2 + G::NS;
-  uint64_t *v_full = bars + 2 + 2 * G::NS, *v_empty = v_full + 1, *c_full = v_full + 2;
+  float *th_s = reinterpret_cast<float *>(small);          // [2][CQ*CK] by item parity
+  float *qred = reinterpret_cast<float *>(small + 1024);   // [8] per-warp max |q|
+  uint64_t *bars = reinterpret_cast<uint64_t *>(small + 1088);
+  uint64_t *q_full = bars + 0, *q_ready = bars + 1, *q_free = bars + 2, *z_free = bars + 3;
+  uint64_t *x_ready = bars + 4, *k_full = bars + 5, *k_empty = bars + 5 + G::NS;
+  uint64_t *v_full = bars + 5 + 2 * G::NS, *v_empty = v_full + 1, *c_full = v_full + 2;
   uint64_t *c_free = v_full + 3, *p_full = v_full + 4, *mma_done = v_full + 5;
-  uint32_t *tslot = reinterpret_cast<uint32_t *>(small + 640 + 8 * 24);
-  volatile int *abort_flag = reinterpret_cast<volatile int *>(small + 640 + 8 * 24 + 8);
+  uint32_t *tslot = reinterpret_cast<uint32_t *>(small + 1088 + 8 * 32);
+  volatile int *abort_flag = reinterpret_cast<volatile int *>(small + 1088 + 8 * 32 + 8);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  // the query tiles of one (batch, head) are adjacent in the grid (they share the
-  // head's Kt stream in L2), longest first
-  const int qt = p.n_qtiles - 1 - static_cast<int>(blockIdx.x);
-  const int h = blockIdx.y, b = blockIdx.z;
-  const int hr = h & 1, g = h >> 1;
+  // cluster c (the two heads of a group with post-softmax mixing, else one CTA)
+  const int hr = MIX == 2 ? static_cast<int>(blockIdx.x) : 0;
+  const int c = static_cast<int>(blockIdx.y), n_clusters = static_cast<int>(gridDim.y);
+  constexpr int CL = MIX == 2 ? 2 : 1;
+  const int n_groups = p.H / CL;
+  const int n_items = p.B * n_groups * p.n_qtiles;
   const int L = p.L;
-  const int i0 = qt * G::BM;
-  const int row0 = i0 - G::HALO;  // query index of staged row 0
-  const int last_q = min(L - 1, i0 + G::BM - 1);
-  const int n_kv = last_q / G::BN + 1;
+  // this cluster's items: item_index(c, r) for r = 0, 1, ... while below n_items
+  auto item_at = [&](int r, Item &it) -> bool {
+    const int k = item_index(c, r, n_clusters);
+    if (k >= n_items) return false;
+    it = item_of(k, p.B, n_groups, p.n_qtiles);
+    return true;
+  };
+  auto kv_tiles = [&](const Item &it) { return min(L - 1, it.qt * G::BM + G::BM - 1) / G::BN + 1; };
 
   if (threadIdx.x == 0) {
-    mbar_init(q_full, 1); mbar_init(q_ready, 8);
+    mbar_init(q_full, 1); mbar_init(q_ready, 8); mbar_init(q_free, 1); mbar_init(z_free, 8);
+    mbar_init(x_ready, kSmThreads);
     for (int s = 0; s < G::NS; ++s) { mbar_init(k_full + s, 1); mbar_init(k_empty + s, 1); }
     mbar_init(v_full, 1); mbar_init(v_empty, 1); mbar_init(c_full, 1); mbar_init(c_free, 8);
     mbar_init(p_full, 8); mbar_init(mma_done, 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
-  if (threadIdx.x >= 32 && threadIdx.x < 32 + CQ * CK)
-    th_s[threadIdx.x - 32] = p.theta[static_cast<long long>(h) * CQ * CK + (threadIdx.x - 32)];
-  if (MIX == 2 && threadIdx.x >= 192 && threadIdx.x < 196)
-    w_s[threadIdx.x - 192] = p.w[static_cast<long long>(g) * 4 + (threadIdx.x - 192)];
   if (warp == kMmaWarp) { tmem_alloc(tslot, G::TMEM_COLS); tmem_relinquish(); }
   tc_fence_before();
   __syncthreads();
+  if (MIX == 2) cluster_sync_all();  // the peer's barriers are initialised before remote arrivals
   tc_fence_after();
   const uint32_t tmem = *tslot;
 
   if (warp == kTmaWarp) {
     // -------------------------------------------------------------- TMA
-    if (lane == 0) {
-      prefetch_tmap(&tmQ); prefetch_tmap(&tmK);
-      mbar_arrive_expect_tx(q_full, G::Q_BYTES);
-#pragma unroll 1
-      for (int s = 0; s < G::NSTRIP; ++s) tma_load_4d(Qs + s * G::STRIP, &tmQ, q_full, 8 * s, h, row0, b);
+    if (lane == 0) {  // Kt chunks of every key tile of every item, through the ring
+      prefetch_tmap(&tmK);
       int cnt = 0;
-      const int zbase = (b * p.H + h) * CQ;
-      for (int t = 0; t < n_kv && !*abort_flag; ++t)
-        for (int ch = 0; ch < G::NCH; ++ch, ++cnt) {
-          const int st = cnt % G::NS;
-          if (!mbar_wait(k_empty + st, ((cnt / G::NS) & 1) ^ 1, abort_flag, p.err)) break;
-          mbar_arrive_expect_tx(k_full + st, G::KCHUNK);
-          tma_load_3d(Ks + st * G::KCHUNK, &tmK, k_full + st, (ch % G::NDC) * 64, t * G::BN, zbase + ch / G::NDC);
-        }
-      drain_wait(q_full, 0);
-      if (*abort_flag)
+      Item it;
+      for (int r = 0; item_at(r, it) && !*abort_flag; ++r) {
+        const int h = it.g * CL + hr, n_kv = kv_tiles(it);
+        const int zbase = (it.b * p.H + h) * CQ;
+        for (int t = 0; t < n_kv && !*abort_flag; ++t)
+          for (int ch = 0; ch < G::NCH; ++ch, ++cnt) {
+            const int st = cnt % G::NS;
+            if (!mbar_wait(k_empty + st, ((cnt / G::NS) & 1) ^ 1, abort_flag, p.err)) break;
+            mbar_arrive_expect_tx(k_full + st, G::KCHUNK);
+            tma_load_3d(Ks + st * G::KCHUNK, &tmK, k_full + st, (ch % G::NDC) * 64, t * G::BN, zbase + ch / G::NDC);
+          }
+      }
+      if (*abort_flag)  // copies still in flight land before the CTA exits
         for (int c2 = (cnt > G::NS ? cnt - G::NS : 0); c2 < cnt; ++c2)
           drain_wait(k_full + c2 % G::NS, (c2 / G::NS) & 1);
-    } else if (lane == 1) {
+    } else if (lane == 1) {  // V of both heads of the group, per key tile
       prefetch_tmap(&tmV);
       int nv = 0;
-      for (int t = 0; t < n_kv; ++t) {
-        if (!mbar_wait(v_empty, (t & 1) ^ 1, abort_flag, p.err)) break;
-        mbar_arrive_expect_tx(v_full, G::V_BYTES);
+      Item it;
+      for (int r = 0; item_at(r, it) && !*abort_flag; ++r) {
+        const int h = it.g * CL + hr, n_kv = kv_tiles(it);
+        for (int t = 0; t < n_kv; ++t, ++nv) {
+          if (!mbar_wait(v_empty, (nv & 1) ^ 1, abort_flag, p.err)) break;
+          mbar_arrive_expect_tx(v_full, G::V_BYTES);
 #pragma unroll
-        for (int hd = 0; hd < G::NV; ++hd)
+          for (int hd = 0; hd < G::NV; ++hd)
 #pragma unroll
-          for (int dc = 0; dc < G::NDC; ++dc)
-            tma_load_4d(Vs + hd * G::V_HEAD + dc * G::V_CHUNK, &tmV, v_full, dc * 64,
-                        G::NV == 2 ? 2 * g + hd : h, t * G::BN, b);
-        ++nv;
+            for (int dc = 0; dc < G::NDC; ++dc)
+              tma_load_4d(Vs + hd * G::V_HEAD + dc * G::V_CHUNK, &tmV, v_full, dc * 64,
+                          G::NV == 2 ? 2 * it.g + hd : h, t * G::BN, it.b);
+        }
       }
       if (*abort_flag && nv) drain_wait(v_full, (nv - 1) & 1);
+    } else if (lane == 2) {  // the query rows of each item, once the previous item's C is done
+      prefetch_tmap(&tmQ);
+      int nq = 0;
+      Item it;
+      for (int r = 0; item_at(r, it) && !*abort_flag; ++r, ++nq) {
+        if (r > 0 && !mbar_wait(q_free, (r - 1) & 1, abort_flag, p.err)) break;
+        const int h = it.g * CL + hr, row0 = it.qt * G::BM - G::HALO;
+        mbar_arrive_expect_tx(q_full, G::Q_BYTES);
+#pragma unroll 1
+        for (int s2 = 0; s2 < G::NSTRIP; ++s2) tma_load_4d(Qs + s2 * G::STRIP, &tmQ, q_full, 8 * s2, h, row0, it.b);
+      }
+      if (nq) drain_wait(q_full, (nq - 1) & 1);
     }
   } else if (warp == kMmaWarp) {
     // -------------------------------------------------------------- MMA
@@ -235,11 +274,12 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint64_t qdesc0 = sdesc_noswz(smem_u32(Qs), G::STRIP, 128);
       const uint64_t kdesc0 = sdesc_sw128(smem_u32(Ks), 16, 1024);
       const uint64_t vdesc0 = sdesc_sw128(smem_u32(Vs), G::V_CHUNK, 1024);
-      int cnt = 0;
-      bool ok = mbar_wait(q_ready, 0, abort_flag, p.err);
-      // C(t) = sum over the NCH chunks (a, 64-wide d block) of Q shifted by a rows x Kt_a
-      auto issue_c = [&](int t) -> bool {
-        if (t > 0 && !mbar_wait(c_free, (t - 1) & 1, abort_flag, p.err)) return false;
+      int cnt = 0, T = 0;  // Kt chunks and key tiles issued so far (all items)
+      bool ok = true;
+      // C of global key tile T = sum over the NCH chunks (a, 64-wide d block) of Q
+      // shifted by a rows x Kt_a
+      auto issue_c = [&](bool last_of_item) -> bool {
+        if (T > 0 && !mbar_wait(c_free, (T - 1) & 1, abort_flag, p.err)) return false;
         for (int ch = 0; ch < G::NCH; ++ch, ++cnt) {
           const int st = cnt % G::NS;
           if (!mbar_wait(k_full + st, (cnt / G::NS) & 1, abort_flag, p.err)) return false;
@@ -254,21 +294,36 @@ __global__ void __launch_bounds__(kThreads, 1)
           mma_commit(k_empty + st);
         }
         mma_commit(c_full);
+        if (last_of_item) mma_commit(q_free);  // the query buffer may take the next item
         return true;
       };
-      if (ok) ok = issue_c(0);
-      for (int t = 0; ok && t < n_kv; ++t) {
-        if (t + 1 < n_kv && !issue_c(t + 1)) break;
-        if (!mbar_wait(p_full, t & 1, abort_flag, p.err)) break;
-        if (!mbar_wait(v_full, t & 1, abort_flag, p.err)) break;
-        tc_fence_after();
+      Item it;
+      for (int r = 0; ok && item_at(r, it); ++r) {
+        const int n_kv = kv_tiles(it);
+        if (!mbar_wait(q_ready, r & 1, abort_flag, p.err)) break;
+        const int T0 = T;
+        ok = issue_c(n_kv == 1);
+        for (int t = 0; ok && t < n_kv; ++t) {
+          const int Tt = T0 + t;
+          if (t + 1 < n_kv) {
+            T = Tt + 1;
+            if (!issue_c(t + 2 == n_kv)) { ok = false; break; }
+          }
+          if (!mbar_wait(p_full, Tt & 1, abort_flag, p.err)) { ok = false; break; }
+          if (!mbar_wait(v_full, Tt & 1, abort_flag, p.err)) { ok = false; break; }
+          // Z is overwritten (accumulate off) by the first P V of an item: the previous
+          // item's epilogue must have read it
+          if (t == 0 && r > 0 && !mbar_wait(z_free, (r - 1) & 1, abort_flag, p.err)) { ok = false; break; }
+          tc_fence_after();
 #pragma unroll
-        for (int hd = 0; hd < G::NV; ++hd)
+          for (int hd = 0; hd < G::NV; ++hd)
 #pragma unroll
-          for (int kk = 0; kk < G::BN / 16; ++kk)
-            mma_f16_ts(tmem + G::Z_COL0 + 128 * hd, tmem + G::P_COL + 8 * kk,
-                       vdesc0 + ((hd * G::V_HEAD + kk * 16 * 128) >> 4), idesc_pv, (t > 0 || kk > 0));
-        mma_commit(v_empty);
+            for (int kk = 0; kk < G::BN / 16; ++kk)
+              mma_f16_ts(tmem + G::Z_COL0 + 128 * hd, tmem + G::P_COL + 8 * kk,
+                         vdesc0 + ((hd * G::V_HEAD + kk * 16 * 128) >> 4), idesc_pv, (t > 0 || kk > 0));
+          mma_commit(v_empty);
+        }
+        T = T0 + n_kv;
       }
       mma_commit(mma_done);
       drain_wait(mma_done, 0);
@@ -276,267 +331,305 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else {
     // ---------------------------------------------- softmax warpgroups
     const int wg = warp >> 2, q4 = warp & 3;
-    const int r = 32 * q4 + lane;            // query row of this thread = TMEM lane
-    const int qi = i0 + r;
-    const bool out_row = qi < L;
+    const int r_ = 32 * q4 + lane;           // query row of this thread = TMEM lane
     const int st_id = threadIdx.x;           // 0..255
     const int cb = G::HALF * wg;             // key columns of this warpgroup
     const int zc = G::DH * wg;               // output channels of this warpgroup
     const uint32_t tl = tmem + (static_cast<uint32_t>(32 * q4) << 16);
-
-    // stage: queries in fp16 (scaled down by a power of 2 only if |q| > 2^14), and
-    // the past dot products of the staged rows
-    mbar_wait(q_full, 0, abort_flag, p.err);
-    float qmax = 0.f;
-    for (int c16 = st_id; c16 < G::Q_BYTES / 16; c16 += kSmThreads) {
-      const uint4 raw = *reinterpret_cast<const uint4 *>(Qs + 16 * c16);
-      const __nv_bfloat162 *p2 = reinterpret_cast<const __nv_bfloat162 *>(&raw);
-#pragma unroll
-      for (int u = 0; u < 4; ++u)
-        qmax = fmaxf(qmax, fmaxf(fabsf(__low2float(p2[u])), fabsf(__high2float(p2[u]))));
-    }
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) qmax = fmaxf(qmax, __shfl_xor_sync(0xffffffffu, qmax, o));
-    if (lane == 0) qred[warp] = qmax;
-    named_bar_sync(kBarAll, kSmThreads);
-#pragma unroll
-    for (int i = 0; i < 8; ++i) qmax = fmaxf(qmax, qred[i]);
-    int eq = 0;
-    if (qmax > 16384.f) eq = max(-60, static_cast<int>(floorf(log2f(16384.f / qmax))));
-    const float qsc = exp2f(static_cast<float>(eq));
-    for (int c16 = st_id; c16 < G::Q_BYTES / 16; c16 += kSmThreads) {
-      uint4 raw = *reinterpret_cast<const uint4 *>(Qs + 16 * c16);
-      __nv_bfloat162 *p2 = reinterpret_cast<__nv_bfloat162 *>(&raw);
-      uint4 o;
-      uint32_t *ow = reinterpret_cast<uint32_t *>(&o);
-#pragma unroll
-      for (int u = 0; u < 4; ++u) {
-        __half2 hv = __floats2half2_rn(__low2float(p2[u]) * qsc, __high2float(p2[u]) * qsc);
-        ow[u] = *reinterpret_cast<uint32_t *>(&hv);
-      }
-      *reinterpret_cast<uint4 *>(Qs + 16 * c16) = o;
-    }
-    fence_proxy_async_smem();
-    __syncwarp();
-    if (lane == 0) mbar_arrive(q_ready);
-    const long long bh = static_cast<long long>(b) * p.H + h;
-    for (int e = st_id; e < G::UROWS * G::M; e += kSmThreads) {
-      const int rr = e / G::M, k = e % G::M, iq = row0 + rr;
-      Us[e] = (iq >= 0 && iq < L) ? p.vp[(bh * L + iq) * G::M + k] : 0.f;
-    }
-    // column factors of key tile t are staged in facs[t & 1] one tile ahead; the
-    // barrier of tile t-1 (here: the one below) publishes them
-    const float *fac = p.fac + bh * p.lpad;
-    if (st_id < G::BN) facs[st_id] = fac[st_id];
-    named_bar_sync(kBarAll, kSmThreads);
-
     const float sc0 = p.qk_scale * kLog2e;
-    const float qinv = exp2f(static_cast<float>(-eq));
-    float *crow = Cs + (wg * G::BM + r) * G::W;
-    float m_run = -INFINITY, l_run = 0.f;
-    for (int t = 0; t < n_kv; ++t) {
-      const int j0 = t * G::BN;
-      // next tile's column factors (stored before this tile's barrier, read after it)
-      const float fnext = (st_id < G::BN && t + 1 < n_kv) ? fac[j0 + G::BN + st_id] : 0.f;
-      const float4 *f4 = reinterpret_cast<const float4 *>(facs + (t & 1) * G::BN + cb);
-      mbar_wait(c_full, t & 1, abort_flag, p.err);
-      tc_fence_after();
-      float cv[G::HALF];
+    float *crow = Cs + (wg * G::BM + r_) * G::W;
+
+    // Stage item r: its query rows in fp16 (scaled down by a power of 2 only if
+    // |q| > 2^14), the past dot products of its staged rows and its kernel taps.
+    // Returns the query exponent.
+    auto prepare = [&](int r, const Item &it) -> int {
+      const int h = it.g * CL + hr, row0 = it.qt * G::BM - G::HALO;
+      mbar_wait(q_full, r & 1, abort_flag, p.err);
+      float qmax = 0.f;
+      for (int c16 = st_id; c16 < G::Q_BYTES / 16; c16 += kSmThreads) {
+        const uint4 raw = *reinterpret_cast<const uint4 *>(Qs + 16 * c16);
+        const __nv_bfloat162 *p2 = reinterpret_cast<const __nv_bfloat162 *>(&raw);
 #pragma unroll
-      for (int c0 = 0; c0 < G::HALF; c0 += 32) {
-        uint32_t u32[32];
-        tmem_ld32(tl + G::C_COL + cb + c0, u32);
-        float4 f[8];
+        for (int u = 0; u < 4; ++u)
+          qmax = fmaxf(qmax, fmaxf(fabsf(__low2float(p2[u])), fabsf(__high2float(p2[u]))));
+      }
 #pragma unroll
-        for (int i = 0; i < 8; ++i) f[i] = f4[c0 / 4 + i];
-        tmem_wait_ld();
+      for (int o = 16; o > 0; o >>= 1) qmax = fmaxf(qmax, __shfl_xor_sync(0xffffffffu, qmax, o));
+      if (lane == 0) qred[warp] = qmax;
+      named_bar_sync(kBarAll, kSmThreads);
 #pragma unroll
-        for (int i = 0; i < 8; ++i) {
-          cv[c0 + 4 * i] = __uint_as_float(u32[4 * i]) * f[i].x;
-          cv[c0 + 4 * i + 1] = __uint_as_float(u32[4 * i + 1]) * f[i].y;
-          cv[c0 + 4 * i + 2] = __uint_as_float(u32[4 * i + 2]) * f[i].z;
-          cv[c0 + 4 * i + 3] = __uint_as_float(u32[4 * i + 3]) * f[i].w;
+      for (int i = 0; i < 8; ++i) qmax = fmaxf(qmax, qred[i]);
+      int eq = 0;
+      if (qmax > 16384.f) eq = max(-60, static_cast<int>(floorf(log2f(16384.f / qmax))));
+      const float qsc = exp2f(static_cast<float>(eq));
+      for (int c16 = st_id; c16 < G::Q_BYTES / 16; c16 += kSmThreads) {
+        uint4 raw = *reinterpret_cast<const uint4 *>(Qs + 16 * c16);
+        __nv_bfloat162 *p2 = reinterpret_cast<__nv_bfloat162 *>(&raw);
+        uint4 o;
+        uint32_t *ow = reinterpret_cast<uint32_t *>(&o);
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          __half2 hv = __floats2half2_rn(__low2float(p2[u]) * qsc, __high2float(p2[u]) * qsc);
+          ow[u] = *reinterpret_cast<uint32_t *>(&hv);
         }
+        *reinterpret_cast<uint4 *>(Qs + 16 * c16) = o;
       }
-      tc_fence_before();
+      fence_proxy_async_smem();
       __syncwarp();
-      if (lane == 0) mbar_arrive(c_free);
-      if (eq != 0) {  // queries were scaled down (|q| > 2^14)
-#pragma unroll
-        for (int jj = 0; jj < G::HALF; ++jj) cv[jj] *= qinv;
+      if (lane == 0) mbar_arrive(q_ready);
+      const long long bh = static_cast<long long>(it.b) * p.H + h;
+      for (int e = st_id; e < G::UROWS * G::M; e += kSmThreads) {
+        const int rr = e / G::M, k = e % G::M, iq = row0 + rr;
+        Us[e] = (iq >= 0 && iq < L) ? p.vp[(bh * L + iq) * G::M + k] : 0.f;
       }
-      // the band 0 <= i-j < W, where Mask_0 removes taps: the convolution tap by
-      // tap over the unmasked taps, from the past dot products:
-      //   C[i][i-dd] = s * sum_{a,t: m = dd - a + (t - c) >= 0} theta[a][t] Vp[i-a][m]
-      const int dmax = qi - j0 - cb;  // i - j for this warpgroup's first column
-      if (out_row && dmax >= 0 && dmax - (G::W - 1) < G::HALF) {
-        float acc[G::W];
+      if (st_id < CQ * CK) th_s[(r & 1) * 128 + st_id] = p.theta[static_cast<long long>(h) * CQ * CK + st_id];
+      return eq;
+    };
+
+    int T = 0;  // key tiles processed so far (all items)
+    Item it, nx;
+    bool have = item_at(0, it);
+    int eq = 0;
+    if (have) {
+      eq = prepare(0, it);
+      const float *fac0 = p.fac + (static_cast<long long>(it.b) * p.H + it.g * CL + hr) * p.lpad;
+      if (st_id < G::BN) facs[(T & 1) * G::BN + st_id] = fac0[st_id];
+      named_bar_sync(kBarAll, kSmThreads);
+    }
+    for (int r = 0; have; ++r) {
+      const int h = it.g * CL + hr, g = it.g;
+      const int i0 = it.qt * G::BM, qi = i0 + r_;
+      const bool out_row = qi < L;
+      const int n_kv = kv_tiles(it);
+      const long long bh = static_cast<long long>(it.b) * p.H + h;
+      const float *fac = p.fac + bh * p.lpad;
+      const bool more = item_at(r + 1, nx);
+      const float *fac_nx = more ? p.fac + (static_cast<long long>(nx.b) * p.H + nx.g * CL + hr) * p.lpad : fac;
+      const float *th = th_s + (r & 1) * 128;
+      const float qinv = exp2f(static_cast<float>(-eq));
+      float m_run = -INFINITY, l_run = 0.f;
+      for (int t = 0; t < n_kv; ++t, ++T) {
+        const int j0 = t * G::BN;
+        // next key tile's column factors (stored before this tile's barrier, read after it)
+        float fnext = 0.f;
+        if (st_id < G::BN) fnext = t + 1 < n_kv ? fac[j0 + G::BN + st_id] : (more ? fac_nx[st_id] : 0.f);
+        const float4 *f4 = reinterpret_cast<const float4 *>(facs + (T & 1) * G::BN + cb);
+        mbar_wait(c_full, T & 1, abort_flag, p.err);
+        tc_fence_after();
+        float cv[G::HALF];
 #pragma unroll
-        for (int dd = 0; dd < G::W; ++dd) acc[dd] = 0.f;
+        for (int c0 = 0; c0 < G::HALF; c0 += 32) {
+          uint32_t u32[32];
+          tmem_ld32(tl + G::C_COL + cb + c0, u32);
+          float4 f[8];
 #pragma unroll
-        for (int a = 0; a < CQ; ++a) {
-          const float *vrow = Us + (r + G::HALO - a) * G::M;  // rows before query 0 are zero
-          float vr[G::M];
+          for (int i = 0; i < 8; ++i) f[i] = f4[c0 / 4 + i];
+          tmem_wait_ld();
 #pragma unroll
-          for (int m = 0; m < G::M; ++m) vr[m] = vrow[m];
+          for (int i = 0; i < 8; ++i) {
+            cv[c0 + 4 * i] = __uint_as_float(u32[4 * i]) * f[i].x;
+            cv[c0 + 4 * i + 1] = __uint_as_float(u32[4 * i + 1]) * f[i].y;
+            cv[c0 + 4 * i + 2] = __uint_as_float(u32[4 * i + 2]) * f[i].z;
+            cv[c0 + 4 * i + 3] = __uint_as_float(u32[4 * i + 3]) * f[i].w;
+          }
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(c_free);
+        if (eq != 0) {  // queries were scaled down (|q| > 2^14)
 #pragma unroll
-          for (int t = 0; t < CK; ++t) {
-            const float th = th_s[a * CK + t];
+          for (int jj = 0; jj < G::HALF; ++jj) cv[jj] *= qinv;
+        }
+        // the band 0 <= i-j < W, where Mask_0 removes taps: the convolution tap by
+        // tap over the unmasked taps, from the past dot products:
+        //   C[i][i-dd] = s * sum_{a,t: m = dd - a + (t - c) >= 0} theta[a][t] Vp[i-a][m]
+        const int dmax = qi - j0 - cb;  // i - j for this warpgroup's first column
+        if (out_row && dmax >= 0 && dmax - (G::W - 1) < G::HALF) {
+          float acc[G::W];
 #pragma unroll
-            for (int dd = 0; dd < G::W; ++dd) {
-              const int m = dd - a + t - G::C;
-              if (m >= 0 && m < G::M) acc[dd] = fmaf(th, vr[m], acc[dd]);
+          for (int dd = 0; dd < G::W; ++dd) acc[dd] = 0.f;
+#pragma unroll
+          for (int a = 0; a < CQ; ++a) {
+            const float *vrow = Us + (r_ + G::HALO - a) * G::M;  // rows before query 0 are zero
+            float vr[G::M];
+#pragma unroll
+            for (int m = 0; m < G::M; ++m) vr[m] = vrow[m];
+#pragma unroll
+            for (int tp = 0; tp < CK; ++tp) {
+              const float thv = th[a * CK + tp];
+#pragma unroll
+              for (int dd = 0; dd < G::W; ++dd) {
+                const int m = dd - a + tp - G::C;
+                if (m >= 0 && m < G::M) acc[dd] = fmaf(thv, vr[m], acc[dd]);
+              }
             }
           }
-        }
 #pragma unroll
-        for (int dd = 0; dd < G::W; ++dd) crow[dd] = acc[dd] * sc0;
+          for (int dd = 0; dd < G::W; ++dd) crow[dd] = acc[dd] * sc0;
 #pragma unroll
-        for (int jj = 0; jj < G::HALF; ++jj) {
-          const int dd = dmax - jj;
-          if (static_cast<unsigned>(dd) < static_cast<unsigned>(G::W)) cv[jj] = crow[dd];
-        }
-      }
-      // Mask_-inf (only the diagonal tile holds keys after a query) and the row max
-      // over both warpgroups' columns (log2 units)
-      if (t == n_kv - 1) {
-#pragma unroll
-        for (int jj = 0; jj < G::HALF; ++jj)
-          if (j0 + cb + jj > qi) cv[jj] = -INFINITY;
-      }
-      float *rmx = red + (t & 1) * 2 * G::BM;
-      rmx[wg * G::BM + r] = out_row ? tree_max<G::HALF>(cv) : -INFINITY;
-      if (st_id < G::BN) facs[((t + 1) & 1) * G::BN + st_id] = fnext;
-      named_bar_sync(kBarAll, kSmThreads);
-      const float mt = fmaxf(rmx[r], rmx[G::BM + r]);
-      const float m_new = fmaxf(m_run, mt);
-      bool resc = false;
-      float alpha = 1.f;
-      if (t == 0) {
-        m_run = m_new;
-      } else if (m_new > m_run + kRescaleLog2) {
-        resc = true;
-        alpha = ex2(m_run - m_new);
-        m_run = m_new;
-      }
-      if (t > 0) {  // P(t-1) consumed and Z(t-1) complete
-        mbar_wait(v_empty, (t - 1) & 1, abort_flag, p.err);
-        tc_fence_after();
-      }
-      if (__any_sync(0xffffffffu, resc)) {  // warp-collective tensor-memory access
-        l_run *= alpha;
-#pragma unroll 1
-        for (int hd = 0; hd < G::NV; ++hd)
-#pragma unroll 1
-          for (int c0 = 0; c0 < G::DH; c0 += 32) {
-            uint32_t z[32];
-            const uint32_t za = tl + G::Z_COL0 + 128 * hd + zc + c0;
-            tmem_ld32(za, z);
-            tmem_wait_ld();
-#pragma unroll
-            for (int i = 0; i < 32; ++i) z[i] = __float_as_uint(__uint_as_float(z[i]) * alpha);
-            tmem_st32(za, z);
+          for (int jj = 0; jj < G::HALF; ++jj) {
+            const int dd = dmax - jj;
+            if (static_cast<unsigned>(dd) < static_cast<unsigned>(G::W)) cv[jj] = crow[dd];
           }
-      }
-      float ls = 0.f;
-      uint32_t pk[32];
+        }
+        // Mask_-inf (only the diagonal tile holds keys after a query) and the row max
+        // over both warpgroups' columns (log2 units)
+        if (t == n_kv - 1) {
 #pragma unroll
-      for (int q2 = 0; q2 < 32; ++q2) {
-        const float p0 = out_row ? ex2(cv[2 * q2] - m_run) : 0.f;
-        const float p1 = out_row ? ex2(cv[2 * q2 + 1] - m_run) : 0.f;
-        ls += p0 + p1;
-        pk[q2] = pack_bf16x2(p0, p1);
+          for (int jj = 0; jj < G::HALF; ++jj)
+            if (j0 + cb + jj > qi) cv[jj] = -INFINITY;
+        }
+        float *rmx = red + (T & 1) * 2 * G::BM;
+        rmx[wg * G::BM + r_] = out_row ? tree_max<G::HALF>(cv) : -INFINITY;
+        if (st_id < G::BN) facs[((T + 1) & 1) * G::BN + st_id] = fnext;
+        named_bar_sync(kBarAll, kSmThreads);
+        const float mt = fmaxf(rmx[r_], rmx[G::BM + r_]);
+        const float m_new = fmaxf(m_run, mt);
+        bool resc = false;
+        float alpha = 1.f;
+        if (t == 0) {
+          m_run = m_new;
+        } else if (m_new > m_run + kRescaleLog2) {
+          resc = true;
+          alpha = ex2(m_run - m_new);
+          m_run = m_new;
+        }
+        if (T > 0) {  // P and Z of the previous key tile are consumed / complete
+          mbar_wait(v_empty, (T - 1) & 1, abort_flag, p.err);
+          tc_fence_after();
+        }
+        if (__any_sync(0xffffffffu, resc)) {  // warp-collective tensor-memory access
+          l_run *= alpha;
+#pragma unroll 1
+          for (int hd = 0; hd < G::NV; ++hd)
+#pragma unroll 1
+            for (int c0 = 0; c0 < G::DH; c0 += 32) {
+              uint32_t z[32];
+              const uint32_t za = tl + G::Z_COL0 + 128 * hd + zc + c0;
+              tmem_ld32(za, z);
+              tmem_wait_ld();
+#pragma unroll
+              for (int i = 0; i < 32; ++i) z[i] = __float_as_uint(__uint_as_float(z[i]) * alpha);
+              tmem_st32(za, z);
+            }
+        }
+        float ls = 0.f;
+        uint32_t pk[32];
+#pragma unroll
+        for (int q2 = 0; q2 < 32; ++q2) {
+          const float p0 = out_row ? ex2(cv[2 * q2] - m_run) : 0.f;
+          const float p1 = out_row ? ex2(cv[2 * q2 + 1] - m_run) : 0.f;
+          ls += p0 + p1;
+          pk[q2] = pack_bf16x2(p0, p1);
+        }
+        tmem_st32(tl + G::P_COL + 32 * wg, pk);
+        l_run += ls;
+        tmem_wait_st();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(p_full);
       }
-      tmem_st32(tl + G::P_COL + 32 * wg, pk);
-      l_run += ls;
-      tmem_wait_st();
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(p_full);
-    }
-    mbar_wait(v_empty, (n_kv - 1) & 1, abort_flag, p.err);
-    tc_fence_after();
-    red[(4 + wg) * G::BM + r] = l_run;
-    named_bar_sync(kBarAll, kSmThreads);
-    const float l_tot = l_run + red[(4 + (wg ^ 1)) * G::BM + r];
-    const float inv_l = (out_row && l_tot > 0.f) ? 1.f / l_tot : 0.f;
+      // the next item's queries, dot products and taps, while this item's last P V runs
+      const int eq_next = more ? prepare(r + 1, nx) : 0;
 
-    // ---------------------------------------------------------- epilogue
-    float o[G::DH];
-    if constexpr (MIX == 2) {
-      float *xbuf = reinterpret_cast<float *>(Ks);  // [BM][XSTR] fp32, reuses the ring and V
-      __syncwarp();
-      cluster_sync_all();                           // both CTAs are done with their ring and V
-      const uint32_t dst = map_peer(smem_u32(xbuf + r * G::XSTR + zc), static_cast<uint32_t>(hr ^ 1));
-#pragma unroll
-      for (int c0 = 0; c0 < G::DH; c0 += 32) {
-        uint32_t z[32];
-        tmem_ld32(tl + G::Z_COL0 + 128 * (hr ^ 1) + zc + c0, z);
-        tmem_wait_ld();
-#pragma unroll
-        for (int i = 0; i < 32; i += 4)
-          st_cluster_v4(dst + 4 * (c0 + i), __uint_as_float(z[i]) * inv_l, __uint_as_float(z[i + 1]) * inv_l,
-                        __uint_as_float(z[i + 2]) * inv_l, __uint_as_float(z[i + 3]) * inv_l);
-      }
-      cluster_sync_all();  // the peer's Z_{peer->h} / l_peer is in xbuf
-      const float w_own = w_s[hr * 2 + hr], w_peer = w_s[hr * 2 + (hr ^ 1)];
-      const float *xr = xbuf + r * G::XSTR + zc;
-#pragma unroll
-      for (int c0 = 0; c0 < G::DH; c0 += 32) {
-        uint32_t z[32];
-        tmem_ld32(tl + G::Z_COL0 + 128 * hr + zc + c0, z);
-        tmem_wait_ld();
-#pragma unroll
-        for (int i = 0; i < 32; ++i) o[c0 + i] = w_own * (__uint_as_float(z[i]) * inv_l) + w_peer * xr[c0 + i];
-      }
-    } else {
-#pragma unroll
-      for (int c0 = 0; c0 < G::DH; c0 += 32) {
-        uint32_t z[32];
-        tmem_ld32(tl + G::Z_COL0 + zc + c0, z);
-        tmem_wait_ld();
-#pragma unroll
-        for (int i = 0; i < 32; ++i) o[c0 + i] = __uint_as_float(z[i]) * inv_l;
-      }
-    }
-    if (p.gn) {  // group norm over the D channels of (token, head), then depth scale
-      float s = 0.f;
-#pragma unroll
-      for (int i = 0; i < G::DH; ++i) s += o[i];
-      red[(6 + wg) * G::BM + r] = s;
+      // ---------------------------------------------------------- epilogue
+      mbar_wait(v_empty, (T - 1) & 1, abort_flag, p.err);
+      tc_fence_after();
+      red[(4 + wg) * G::BM + r_] = l_run;
       named_bar_sync(kBarAll, kSmThreads);
-      const float mu = (s + red[(6 + (wg ^ 1)) * G::BM + r]) * (1.f / D);
-      float s2 = 0.f;
+      const float l_tot = l_run + red[(4 + (wg ^ 1)) * G::BM + r_];
+      const float inv_l = (out_row && l_tot > 0.f) ? 1.f / l_tot : 0.f;
+      float o[G::DH];
+      if constexpr (MIX == 2) {
+        // Z_{h->peer} / l_h goes to the peer through L2: [parity][column/4][row] float4
+        float4 *mine = reinterpret_cast<float4 *>(p.xg) + (static_cast<long long>(2 * c + hr) * 2 + (r & 1)) * (G::BM * D / 4);
+        const float4 *theirs = reinterpret_cast<const float4 *>(p.xg) +
+                               (static_cast<long long>(2 * c + (hr ^ 1)) * 2 + (r & 1)) * (G::BM * D / 4);
 #pragma unroll
-      for (int i = 0; i < G::DH; ++i) { const float x = o[i] - mu; s2 += x * x; }
-      red[(8 + wg) * G::BM + r] = s2;
-      named_bar_sync(kBarAll, kSmThreads);
-      const float rstd = rsqrtf((s2 + red[(8 + (wg ^ 1)) * G::BM + r]) * (1.f / D) + p.eps);
-      const float *gm = p.gamma + static_cast<long long>(h) * D + zc;
-      const float *bt = p.beta + static_cast<long long>(h) * D + zc;
+        for (int c0 = 0; c0 < G::DH; c0 += 32) {
+          uint32_t z[32];
+          tmem_ld32(tl + G::Z_COL0 + 128 * (hr ^ 1) + zc + c0, z);
+          tmem_wait_ld();
 #pragma unroll
-      for (int i = 0; i < G::DH; ++i) o[i] = ((o[i] - mu) * rstd * gm[i] + bt[i]) * p.lam;
-    }
-    if (out_row) {
-      __nv_bfloat16 *dst = p.out + ((static_cast<long long>(b) * L + qi) * p.H + h) * D + zc;
+          for (int i = 0; i < 32; i += 4)
+            mine[((zc + c0 + i) / 4) * G::BM + r_] =
+                make_float4(__uint_as_float(z[i]) * inv_l, __uint_as_float(z[i + 1]) * inv_l,
+                            __uint_as_float(z[i + 2]) * inv_l, __uint_as_float(z[i + 3]) * inv_l);
+        }
+        const float w_own = p.w[g * 4 + hr * 2 + hr], w_peer = p.w[g * 4 + hr * 2 + (hr ^ 1)];
 #pragma unroll
-      for (int i = 0; i < G::DH; i += 8) {
-        uint4 v;
-        v.x = pack_bf16x2(o[i], o[i + 1]);
-        v.y = pack_bf16x2(o[i + 2], o[i + 3]);
-        v.z = pack_bf16x2(o[i + 4], o[i + 5]);
-        v.w = pack_bf16x2(o[i + 6], o[i + 7]);
-        *reinterpret_cast<uint4 *>(dst + i) = v;
+        for (int c0 = 0; c0 < G::DH; c0 += 32) {
+          uint32_t z[32];
+          tmem_ld32(tl + G::Z_COL0 + 128 * hr + zc + c0, z);
+          tmem_wait_ld();
+#pragma unroll
+          for (int i = 0; i < 32; ++i) o[c0 + i] = w_own * (__uint_as_float(z[i]) * inv_l);
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(z_free);  // the next item's first P V may overwrite Z
+        // every thread's stores are released to the peer by its own arrival
+        mbar_arrive_cluster(map_peer(smem_u32(x_ready), static_cast<uint32_t>(hr ^ 1)));
+        mbar_wait_cluster(x_ready, r & 1, abort_flag, p.err);
+#pragma unroll
+        for (int c4 = 0; c4 < G::DH / 4; ++c4) {
+          const float4 x = theirs[(zc / 4 + c4) * G::BM + r_];
+          o[4 * c4] += w_peer * x.x;
+          o[4 * c4 + 1] += w_peer * x.y;
+          o[4 * c4 + 2] += w_peer * x.z;
+          o[4 * c4 + 3] += w_peer * x.w;
+        }
+      } else {
+#pragma unroll
+        for (int c0 = 0; c0 < G::DH; c0 += 32) {
+          uint32_t z[32];
+          tmem_ld32(tl + G::Z_COL0 + zc + c0, z);
+          tmem_wait_ld();
+#pragma unroll
+          for (int i = 0; i < 32; ++i) o[c0 + i] = __uint_as_float(z[i]) * inv_l;
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(z_free);
       }
+      if (p.gn) {  // group norm over the D channels of (token, head), then depth scale
+        float s = 0.f;
+#pragma unroll
+        for (int i = 0; i < G::DH; ++i) s += o[i];
+        red[(6 + wg) * G::BM + r_] = s;
+        named_bar_sync(kBarAll, kSmThreads);
+        const float mu = (s + red[(6 + (wg ^ 1)) * G::BM + r_]) * (1.f / D);
+        float s2 = 0.f;
+#pragma unroll
+        for (int i = 0; i < G::DH; ++i) { const float x = o[i] - mu; s2 += x * x; }
+        red[(8 + wg) * G::BM + r_] = s2;
+        named_bar_sync(kBarAll, kSmThreads);
+        const float rstd = rsqrtf((s2 + red[(8 + (wg ^ 1)) * G::BM + r_]) * (1.f / D) + p.eps);
+        const float *gm = p.gamma + static_cast<long long>(h) * D + zc;
+        const float *bt = p.beta + static_cast<long long>(h) * D + zc;
+#pragma unroll
+        for (int i = 0; i < G::DH; ++i) o[i] = ((o[i] - mu) * rstd * gm[i] + bt[i]) * p.lam;
+      }
+      if (out_row) {
+        __nv_bfloat16 *dst = p.out + ((static_cast<long long>(it.b) * L + qi) * p.H + h) * D + zc;
+#pragma unroll
+        for (int i = 0; i < G::DH; i += 8) {
+          uint4 v;
+          v.x = pack_bf16x2(o[i], o[i + 1]);
+          v.y = pack_bf16x2(o[i + 2], o[i + 3]);
+          v.z = pack_bf16x2(o[i + 4], o[i + 5]);
+          v.w = pack_bf16x2(o[i + 6], o[i + 7]);
+          *reinterpret_cast<uint4 *>(dst + i) = v;
+        }
+      }
+      have = more;
+      it = nx;
+      eq = eq_next;
     }
-  }
-  if (MIX == 2 && warp >= kTmaWarp) {  // the producer warps take part in the cluster barriers
-    __syncwarp();  // their lanes return from their roles separately
-    cluster_sync_all();
-    cluster_sync_all();
   }
   tc_fence_before();
   __syncthreads();
+  if (MIX == 2) cluster_sync_all();  // no remote arrival reaches a CTA that has exited
   if (warp == kMmaWarp) {
     tc_fence_after();
     tmem_dealloc(tmem, G::TMEM_COLS);
@@ -544,7 +637,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 }
 
 template <int D, int CQ, int CK, int MIX>
-cudaError_t launch_kq_one(const AttnArgs &a, const GnArgs *gn, const KqPrepArgs &pa) {
+cudaError_t launch_kq_one(const AttnArgs &a, const GnArgs *gn, const KqPrepArgs &pa, float *xg) {
   using G = KGeo<D, CQ, CK, MIX>;
   alignas(64) CUtensorMap tq, tk, tv;
   const unsigned long long dims[4] = {static_cast<unsigned long long>(D), static_cast<unsigned long long>(a.H),
@@ -571,6 +664,7 @@ cudaError_t launch_kq_one(const AttnArgs &a, const GnArgs *gn, const KqPrepArgs 
   p.beta = gn ? gn->beta : nullptr;
   p.eps = gn ? gn->eps : 0.f;
   p.lam = gn ? gn->lam : 1.f;
+  p.B = a.B;
   p.L = a.L;
   p.H = a.H;
   p.n_qtiles = (a.L + G::BM - 1) / G::BM;
@@ -578,22 +672,32 @@ cudaError_t launch_kq_one(const AttnArgs &a, const GnArgs *gn, const KqPrepArgs 
   p.lpad = pa.lpad;
   p.fac = pa.fac;
   p.vp = pa.vp;
+  p.xg = xg;
   p.err = a.err;
   auto kern = attn_kq_kernel<D, CQ, CK, MIX>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, G::SMEM);
   if (e != cudaSuccess) return e;
+  // persistent: as many clusters as can be resident at once (at most one per work
+  // item and kKqMaxClusters), each walking its share of the work items
+  const long long n_items = static_cast<long long>(a.B) * (a.H / G::CLUSTER) * p.n_qtiles;
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(p.n_qtiles, a.H, a.B);
   cfg.blockDim = dim3(kThreads);
   cfg.dynamicSmemBytes = G::SMEM;
   cfg.stream = a.stream;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = 1;
-  attr[0].val.clusterDim.y = G::CLUSTER;  // the two heads of a group
+  attr[0].val.clusterDim.x = G::CLUSTER;  // the two heads of a group
+  attr[0].val.clusterDim.y = 1;
   attr[0].val.clusterDim.z = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
+  cfg.gridDim = dim3(G::CLUSTER, kKqMaxClusters / G::CLUSTER);
+  int resident = 0;
+  e = cudaOccupancyMaxActiveClusters(&resident, kern, &cfg);
+  if (e != cudaSuccess) return e;
+  if (resident < 1) return cudaErrorInvalidConfiguration;
+  const long long nc = std::min<long long>(std::min<long long>(resident, n_items), kKqMaxClusters / G::CLUSTER);
+  cfg.gridDim = dim3(G::CLUSTER, static_cast<unsigned>(nc));
   return cudaLaunchKernelEx(&cfg, kern, tq, tk, tv, p);
 }
 
@@ -612,13 +716,19 @@ bool attn_kq_supported(const AttnArgs &a) {
 }
 
 // Workspace of the contraction path: Kt [B][H][c_q][L][d] fp16 | fac [B][H][Lpad] fp32 |
-// Vp [B][H][L][M] fp32, Lpad = L rounded up to 128, M = (c_q-1) + 2*(c_k/2); each part
-// 256-byte aligned.
-size_t attn_kq_workspace_bytes(int B, int H, int L, int d, int cq, int ck) {
+// Vp [B][H][L][M] fp32 | (post-softmax mixing) the exchange buffer of the persistent
+// CTAs, [CTAs][2][d][128] fp32; Lpad = L rounded up to 128,
+// M = (c_q-1) + 2*(c_k/2); each part 256-byte aligned.
+size_t attn_kq_workspace_bytes(int B, int H, int L, int d, int cq, int ck, int hp) {
   const size_t BH = static_cast<size_t>(B) * H, BHL = BH * L;
   const size_t lpad = (static_cast<size_t>(L) + 127) / 128 * 128;
   const size_t M = static_cast<size_t>(cq - 1 + 2 * (ck / 2));
-  return align256(BHL * cq * d * 2) + align256(BH * lpad * 4) + align256(BHL * M * 4);
+  // one slot pair per persistent CTA: at most kKqMaxClusters CTAs, and at most two per
+  // work item (batch, head group, query tile)
+  const size_t items = static_cast<size_t>(B) * (H / 2) * ((static_cast<size_t>(L) + 127) / 128);
+  const size_t ctas = std::min<size_t>(kKqMaxClusters, 2 * items);
+  const size_t xg = hp == 2 ? ctas * 2 * d * 128 * 4 : 0;
+  return align256(BHL * cq * d * 2) + align256(BH * lpad * 4) + align256(BHL * M * 4) + xg;
 }
 
 cudaError_t launch_attn_kq(const AttnArgs &a, const GnArgs *gn, void *ws) {
@@ -637,11 +747,13 @@ cudaError_t launch_attn_kq(const AttnArgs &a, const GnArgs *gn, void *ws) {
   pa.kt = base;
   pa.fac = reinterpret_cast<float *>(base + align256(BHL * a.cq * a.d * 2));
   pa.vp = reinterpret_cast<float *>(reinterpret_cast<char *>(pa.fac) + align256(BH * pa.lpad * 4));
+  float *xg = reinterpret_cast<float *>(reinterpret_cast<char *>(pa.vp) + align256(BHL * pa.M * 4));
   cudaError_t e = launch_kq_prep(pa, a.stream);
   if (e != cudaSuccess) return e;
   const bool post = a.hp == 2;
-  if (a.d == 128) return post ? launch_kq_one<128, 6, 11, 2>(a, gn, pa) : launch_kq_one<128, 6, 11, 0>(a, gn, pa);
-  return post ? launch_kq_one<64, 6, 11, 2>(a, gn, pa) : launch_kq_one<64, 6, 11, 0>(a, gn, pa);
+  if (a.d == 128)
+    return post ? launch_kq_one<128, 6, 11, 2>(a, gn, pa, xg) : launch_kq_one<128, 6, 11, 0>(a, gn, pa, xg);
+  return post ? launch_kq_one<64, 6, 11, 2>(a, gn, pa, xg) : launch_kq_one<64, 6, 11, 0>(a, gn, pa, xg);
 }
 
 }  // namespace mta

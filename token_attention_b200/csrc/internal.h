@@ -53,7 +53,7 @@ struct KqPrepArgs {
 cudaError_t launch_kq_prep(const KqPrepArgs &a, cudaStream_t stream);
 // Workspace bytes of the contraction path (beyond the error word) and whether it applies.
 bool attn_kq_supported(const AttnArgs &a);
-size_t attn_kq_workspace_bytes(int B, int H, int L, int d, int cq, int ck);
+size_t attn_kq_workspace_bytes(int B, int H, int L, int d, int cq, int ck, int hp);
 // ws: workspace area for Kt / fac / Vp (attn_kq_workspace_bytes bytes, 256-byte aligned).
 cudaError_t launch_attn_kq(const AttnArgs &a, const GnArgs *gn, void *ws);
 

@@ -65,7 +65,7 @@ bool kq_shape_ok(const mta_cfg *c) {
 }
 
 size_t kq_bytes(const mta_cfg *c) {
-  return kq_shape_ok(c) ? attn_kq_workspace_bytes(c->B, c->H, c->L, c->d, c->c_q, c->c_k) : 0;
+  return kq_shape_ok(c) ? attn_kq_workspace_bytes(c->B, c->H, c->L, c->d, c->c_q, c->c_k, c->head_place) : 0;
 }
 
 // Which attention kernel serves `a` under cfg->path: 0 chooses the contraction
@@ -74,7 +74,7 @@ size_t kq_bytes(const mta_cfg *c) {
 // kernel; 1, 2, 3 force the CUDA-core, direct tensor-core, contraction kernel.
 mta_status select_kernel(const AttnArgs &a, int path, size_t kq_room, Kernel *k) {
   const bool kq_ok = attn_kq_supported(a) &&
-                     kq_room >= attn_kq_workspace_bytes(a.B, a.H, a.L, a.d, a.cq, a.ck);
+                     kq_room >= attn_kq_workspace_bytes(a.B, a.H, a.L, a.d, a.cq, a.ck, a.hp);
   const bool tc_ok = attn_tc_supported(a);
   const bool simt_ok = attn_simt_pick_rows(a, 32) != 0;
   if (path == 3) {
