@@ -39,14 +39,23 @@ Readings where the pages leave a step open (all listed in the design doc):
     the mixed map of head r multiplies head r's own values.
   * Group norm: per (token, head) over the d channels, biased variance,
     eps, affine gamma/beta of length D; then times lambda.
+  * Exact causal indicator (the variant section 3.1 contrasts with Mask_0: the
+    simpler mask "removes slightly more information than necessary"): a tap of
+    the convolution at output (i, j) reads A_hat[i - a][j - b] whenever its key
+    j - b is not after the output query i, even if it is after the shifted
+    query i - a.  Outputs stay causal (nothing after i is read).
+  * Sigmoid scalar gate (section 3.3: "a learned sigmoid scalar gate, a bounded
+    multiplier"): one learned logit g_h per head; the normalised output of head h
+    is multiplied by sigmoid(g_h) in place of the depth scale.
 """
 from __future__ import annotations
 
 import numpy as np
 
-OFF, PRE, POST = 0, 1, 2
+OFF, PRE, POST, PRE_EXACT = 0, 1, 2, 3
 
-__all__ = ["OFF", "PRE", "POST", "attention_logits", "mask_zero", "key_query_conv",
+__all__ = ["OFF", "PRE", "POST", "PRE_EXACT", "attention_logits", "mask_zero", "key_query_conv",
+           "key_query_conv_exact", "sigmoid_gate",
            "head_mix", "mask_neg_inf", "softmax_rows", "mta_attention_group",
            "mta_attention", "mta_attention_rows", "group_norm_scale", "mta_layer",
            "mta_layer_rows"]
@@ -98,6 +107,38 @@ def key_query_conv(m: np.ndarray, theta: np.ndarray) -> np.ndarray:
     return out
 
 
+def key_query_conv_exact(a_hat: np.ndarray, theta: np.ndarray, qpos: np.ndarray) -> np.ndarray:
+    """Conv2d_theta over (query, key) with the exact causal indicator  [MTA-3.1].
+
+    a_hat [c_h, R, L] (unmasked logits; rows are consecutive queries qpos).
+    out[h, r, j] = sum_a sum_t theta[h, a, t] * a_hat[h, r - a, j - b] * [j - b <= qpos[r]],
+    b = t - c_k//2; rows before the first and keys outside [0, L) count as 0."""
+    ch, R, L = a_hat.shape
+    cq, ck = theta.shape[1], theta.shape[2]
+    c = ck // 2
+    out = np.zeros_like(a_hat, dtype=np.float64)
+    keys = np.arange(L)
+    for a in range(cq):
+        if a >= R:
+            break
+        for t in range(ck):
+            b = t - c
+            j_lo, j_hi = max(0, b), min(L, L + b)
+            if j_lo >= j_hi:
+                continue
+            shifted = np.zeros((ch, R, L), np.float64)
+            shifted[:, a:, j_lo:j_hi] = a_hat[:, :R - a, j_lo - b:j_hi - b]
+            allowed = (keys[None, :] - b) <= np.asarray(qpos)[:, None]       # [R, L]
+            coef = theta[:, a, t].astype(np.float64)[:, None, None]
+            out += coef * np.where(allowed[None], shifted, 0.0)
+    return out
+
+
+def sigmoid_gate(gate: np.ndarray) -> np.ndarray:
+    """The bounded per-head multiplier sigmoid(g) of the scalar gate  [MTA-3.3]."""
+    return 1.0 / (1.0 + np.exp(-np.asarray(gate, np.float64)))
+
+
 def head_mix(a: np.ndarray, w: np.ndarray) -> np.ndarray:
     """Within-group linear combination: out[r] = sum_s w[r, s] * a[s]  [MTA-3.2]."""
     return np.einsum("rs,s...->r...", w.astype(np.float64), a)
@@ -125,6 +166,8 @@ def mta_attention_group(q_rows, k, v, theta, w, qpos, scale, kq_place, head_plac
     a_hat = attention_logits(q_rows, k, scale)
     if kq_place == PRE:
         c = key_query_conv(mask_zero(a_hat, qpos), theta)
+    elif kq_place == PRE_EXACT:
+        c = key_query_conv_exact(a_hat, theta, qpos)
     else:
         c = a_hat
     if head_place == PRE:
@@ -190,14 +233,16 @@ def mta_attention_rows(q, k, v, theta, w, c_h, rows, kq_place=PRE, head_place=PO
 
 def group_norm_scale(o, gamma, beta, eps, lam):
     """Per-(token, head) normalisation over d, affine, then depth scale
-    [MTA-3.3, bycloud].  o [..., H, d]; gamma, beta [H*d].  Returns float64."""
+    [MTA-3.3, bycloud].  o [..., H, d]; gamma, beta [H*d]; lam a scalar (depth
+    scale) or a per-head [H] multiplier (the sigmoid gate).  Returns float64."""
     o = o.astype(np.float64)
     H, d = o.shape[-2], o.shape[-1]
     mu = np.mean(o, axis=-1, keepdims=True)
     var = np.mean((o - mu) ** 2, axis=-1, keepdims=True)
     y = (o - mu) / np.sqrt(var + eps)
     y = y * gamma.astype(np.float64).reshape(H, d) + beta.astype(np.float64).reshape(H, d)
-    return lam * y
+    lam = np.asarray(lam, np.float64)
+    return (lam.reshape(H, 1) if lam.ndim else lam) * y
 
 
 def _split_qkv(qkv, H, d):

@@ -331,3 +331,116 @@ def test_layer_matches_library_pipeline():
                             O.PRE, O.POST)
     for n, (b, i) in enumerate(rows):
         np.testing.assert_allclose(part[n], out[b, i], rtol=0, atol=1e-11)
+
+
+# ---------------------------------------------------------------------------
+# exact causal indicator (the variant section 3.1 contrasts with Mask_0)
+# ---------------------------------------------------------------------------
+
+@pytest.mark.parametrize("a", [1, 2])
+def test_exact_indicator_query_shift_closed_form(qkv, a):
+    """theta = delta at (a, 0) with the exact indicator: C[i,j] = s q[i-a].k[j] for
+    every causal j <= i (keys after the shifted query i-a are kept, unlike Mask_0),
+    and 0 when i-a < 0."""
+    q, k, v = qkv
+    B, L, H, d = q.shape
+    cq, ck = 3, 5
+    s = 1 / np.sqrt(d)
+    th = delta_theta(H, cq, ck, a, ck // 2)
+    out = O.mta_attention(q, k, v, th, np.tile(np.eye(1), (H, 1, 1)), 1, O.PRE_EXACT, O.OFF)
+    for b, h in [(0, 2), (1, 0)]:
+        qq, kk, vv = q[b, :, h], k[b, :, h], v[b, :, h]
+        fn = lambda i, j: s * qq[i - a] @ kk[j] if i - a >= 0 else 0.0
+        np.testing.assert_allclose(out[b, :, h], _closed_form_attention(qq, kk, vv, fn, s),
+                                   rtol=0, atol=1e-12)
+
+
+@pytest.mark.parametrize("boff", [-2, 1])
+def test_exact_indicator_key_shift_closed_form(qkv, boff):
+    """theta = delta at (1, b) with the exact indicator: C[i,j] = s q[i-1].k[j-b]
+    when 0 <= j-b <= i (the key may lie after the shifted query i-1)."""
+    q, k, v = qkv
+    B, L, H, d = q.shape
+    cq, ck = 2, 5
+    s = 1 / np.sqrt(d)
+    th = delta_theta(H, cq, ck, 1, ck // 2 + boff)
+    out = O.mta_attention(q, k, v, th, np.tile(np.eye(1), (H, 1, 1)), 1, O.PRE_EXACT, O.OFF)
+    for b, h in [(0, 3), (1, 1)]:
+        qq, kk, vv = q[b, :, h], k[b, :, h], v[b, :, h]
+        fn = lambda i, j: s * qq[i - 1] @ kk[j - boff] if (i >= 1 and 0 <= j - boff <= i) else 0.0
+        np.testing.assert_allclose(out[b, :, h], _closed_form_attention(qq, kk, vv, fn, s),
+                                   rtol=0, atol=1e-12)
+
+
+def test_exact_indicator_equals_mask0_for_one_query_row(qkv):
+    """With c_q = 1 the shifted query is the output query, so the two masks agree."""
+    q, k, v = qkv
+    H = q.shape[2]
+    th = rand((H, 1, 5), 31, 0.4)
+    w = rand((H // 2, 2, 2), 32, 0.5)
+    a = O.mta_attention(q, k, v, th, w, 2, O.PRE, O.POST)
+    b = O.mta_attention(q, k, v, th, w, 2, O.PRE_EXACT, O.POST)
+    np.testing.assert_allclose(a, b, rtol=0, atol=1e-13)
+
+
+def test_exact_indicator_differs_from_mask0_only_near_the_diagonal():
+    """The two convolutions differ only where a tap reads a key after the shifted
+    query but not after the output query: 0 <= i-j < (c_q-1) + c."""
+    cq, ck, L = 4, 5, 20
+    c = ck // 2
+    a_hat = rand((1, L, L), 33)
+    th = rand((1, cq, ck), 34)
+    qpos = np.arange(L)
+    m0 = O.key_query_conv(O.mask_zero(a_hat, qpos), th)[0]
+    ex = O.key_query_conv_exact(a_hat, th, qpos)[0]
+    i, j = np.indices((L, L))
+    band = (i - j >= 0) & (i - j < cq - 1 + c)
+    causal = j <= i
+    np.testing.assert_array_equal(ex[causal & ~band], m0[causal & ~band])
+    assert np.abs(ex[band] - m0[band]).max() > 1e-3
+
+
+@pytest.mark.parametrize("head_place", [O.PRE, O.POST])
+def test_exact_indicator_causality_bit_exact(qkv, head_place):
+    """The exact indicator still reads nothing after the output query."""
+    q, k, v = qkv
+    H = q.shape[2]
+    th = rand((H, 3, 5), 35, 0.3)
+    w = rand((H // 2, 2, 2), 36, 0.5)
+    base = O.mta_attention(q, k, v, th, w, 2, O.PRE_EXACT, head_place)
+    t = 11
+    q2, k2, v2 = q.copy(), k.copy(), v.copy()
+    q2[:, t:] += rand(q2[:, t:].shape, 37)
+    k2[:, t:] += rand(k2[:, t:].shape, 38)
+    v2[:, t:] += rand(v2[:, t:].shape, 39)
+    pert = O.mta_attention(q2, k2, v2, th, w, 2, O.PRE_EXACT, head_place)
+    assert np.array_equal(base[:, :t], pert[:, :t])
+    assert not np.allclose(base[:, t:], pert[:, t:])
+
+
+# ---------------------------------------------------------------------------
+# sigmoid scalar gate (section 3.3)
+# ---------------------------------------------------------------------------
+
+def test_sigmoid_gate_values():
+    """sigmoid(0) = 1/2, sigmoid(-g) = 1 - sigmoid(g), bounded in (0, 1)."""
+    g = np.array([-30.0, -2.0, 0.0, 0.5, 3.0, 30.0])
+    m = O.sigmoid_gate(g)
+    assert m[2] == 0.5
+    np.testing.assert_allclose(O.sigmoid_gate(-g), 1.0 - m, rtol=0, atol=1e-15)
+    assert np.all(m > 0) and np.all(m < 1)
+    np.testing.assert_allclose(m, scipy.special.expit(g), rtol=1e-15)
+
+
+def test_gated_group_norm_invariants():
+    """With gamma = 1, beta = 0 each (token, head) output has mean 0 and standard
+    deviation sigmoid(g_h) * sqrt(var / (var + eps)): the gate scales head h alone."""
+    T, H, d = 6, 4, 16
+    o = rand((T, H, d), 45, 1.5)
+    g = np.array([-1.0, 0.0, 0.7, 2.5])
+    eps = 1e-5
+    y = O.group_norm_scale(o, np.ones(H * d), np.zeros(H * d), eps, O.sigmoid_gate(g))
+    np.testing.assert_allclose(y.mean(-1), 0.0, atol=1e-12)
+    var = o.var(-1)
+    np.testing.assert_allclose(y.std(-1), scipy.special.expit(g)[None, :] * np.sqrt(var / (var + eps)),
+                               rtol=1e-12)
