@@ -60,10 +60,13 @@ typedef enum {
 
 typedef enum { MTA_F32 = 0, MTA_BF16 = 1 } mta_dtype;
 
-/* Where a mixing step sits relative to the softmax.  kq_place: OFF or PRE
- * (pre-softmax key-query convolution, section 3.1).  head_place: OFF, PRE or
- * POST (section 3.2). */
-typedef enum { MTA_OFF = 0, MTA_PRE = 1, MTA_POST = 2 } mta_place;
+/* Where a mixing step sits relative to the softmax.  kq_place: OFF, PRE
+ * (pre-softmax key-query convolution of Mask_0(A_hat), section 3.1) or
+ * PRE_EXACT (the same convolution with the exact causal indicator: a tap at
+ * output (i, j) reads A_hat[i-a][j-b] whenever its key j-b is not after the
+ * output query i; section 3.1 contrasts it with the Mask_0 form).  head_place:
+ * OFF, PRE or POST (section 3.2). */
+typedef enum { MTA_OFF = 0, MTA_PRE = 1, MTA_POST = 2, MTA_PRE_EXACT = 3 } mta_place;
 
 typedef struct mta_cfg {
   int B;                 /* batch size, >= 1                                     */
@@ -73,7 +76,7 @@ typedef struct mta_cfg {
   int c_q;               /* query taps of the key-query kernel, 1..8             */
   int c_k;               /* key taps, odd, 1..15                                 */
   int c_h;               /* heads per mixing group, 1..16 (1 = no mixing)        */
-  int kq_place;          /* MTA_OFF or MTA_PRE                                   */
+  int kq_place;          /* MTA_OFF, MTA_PRE or MTA_PRE_EXACT                    */
   int head_place;        /* MTA_OFF, MTA_PRE or MTA_POST (OFF when c_h == 1)     */
   int dtype;             /* mta_dtype of q, k, v and out (x, W and out in a layer) */
   int path;              /* attention kernel: 0 = choose (the contraction kernel
@@ -93,15 +96,18 @@ typedef struct mta_cfg {
   size_t workspace_bytes;
 } mta_cfg;
 
-/* Depth-scaled group normalisation of head outputs (section 3.3; bycloud item 3):
- * y = lambda * ((o - mean_d) / sqrt(var_d + eps) * gamma + beta) per (token, head),
- * biased variance over the d channels of one head. */
+/* Scaled group normalisation of head outputs (section 3.3; bycloud item 3):
+ * y = m_h * ((o - mean_d) / sqrt(var_d + eps) * gamma + beta) per (token, head h),
+ * biased variance over the d channels of one head.  The multiplier m_h is the
+ * depth scale lambda, or, with a gate, the sigmoid scalar gate of section 3.3:
+ * m_h = 1 / (1 + exp(-gate[h])). */
 typedef struct mta_gn {
   const float *gamma;    /* [H*d] device, fp32                                   */
   const float *beta;     /* [H*d] device, fp32                                   */
   float eps;             /* <= 0 selects 1e-5                                    */
   int layer;             /* layer index for the default depth scale             */
   float depth_scale;     /* lambda; < 0 selects 1 - 0.8*exp(-0.3*layer)         */
+  const float *gate;     /* [H] device, fp32 gate logits; NULL = depth scale     */
 } mta_gn;
 
 /* Bytes of workspace mta_attn_fwd needs for cfg (0 if cfg is invalid): 256

@@ -86,7 +86,7 @@ def test_workspace_query(L):
 @pytest.mark.parametrize("kw,code", [
     (dict(c_k=4), 1), (dict(c_k=17), 1), (dict(c_q=0), 1), (dict(c_q=9), 1),
     (dict(H=5), 1), (dict(c_h=0), 1), (dict(B=0), 1), (dict(L=0), 1),
-    (dict(kq_place=2), 1), (dict(head_place=3), 1), (dict(dtype=7), 1), (dict(path=4), 1), (dict(path=-1), 1),
+    (dict(kq_place=2), 1), (dict(kq_place=4), 1), (dict(head_place=3), 1), (dict(dtype=7), 1), (dict(path=4), 1), (dict(path=-1), 1),
     (dict(scale=-1.0), 1), (dict(qkv_row_stride=10), 1),
     (dict(d=200), 2), (dict(d=20), 2), (dict(B=70000), 2),
 ])

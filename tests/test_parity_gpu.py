@@ -294,3 +294,92 @@ def test_layer_full_size_sampled(name):
                            wl.kq_place, wl.head_place)
     got = torch.stack([out[b, i] for b, i in rows])
     assert_close(got, ref, "bf16")
+
+
+# ---------------------------------------------------------------------------
+# exact causal indicator (kq_place = PRE_EXACT) and the sigmoid scalar gate
+# ---------------------------------------------------------------------------
+
+def oracle_exact(wl, inp):
+    return O.mta_attention(inp["q"], inp["k"], inp["v"], inp["theta"], inp["w"], wl.c_h,
+                           O.PRE_EXACT, wl.head_place)
+
+
+@pytest.mark.parametrize("d,hp,L", [(64, synth.OFF, 9), (128, synth.POST, 300), (64, synth.POST, 300),
+                                    (128, synth.OFF, 1)])
+@pytest.mark.parametrize("path", [mta.PATH_AUTO, mta.PATH_SIMT, mta.PATH_KQ])
+def test_exact_indicator_small(d, hp, L, path):
+    base = synth.WORKLOADS["pretrain_d128_L2048"]
+    wl = synth.shrink(base, B=2, H=4, L=L, d=d, head_place=hp, kq_place=mta.PRE_EXACT,
+                      seed=301 + L + d + hp)
+    inp = synth.make_attn_inputs(wl)
+    assert_close(run_attn(wl, inp, path), oracle_exact(wl, inp), "bf16")
+
+
+def test_exact_indicator_differs_from_mask0_on_gpu():
+    """The two kernels of section 3.1 give different outputs near the diagonal."""
+    base = synth.WORKLOADS["pretrain_d128_L2048"]
+    wl = synth.shrink(base, B=1, H=4, L=260, d=128, kq_place=mta.PRE_EXACT, seed=33)
+    inp = synth.make_attn_inputs(wl)
+    a = run_attn(wl, inp, mta.PATH_KQ)
+    wl0 = synth.shrink(wl, kq_place=mta.PRE)
+    b = run_attn(wl0, inp, mta.PATH_KQ)
+    rel, _ = errs(a, b.double().cpu().numpy())
+    assert rel > 1e-3
+
+
+def test_exact_indicator_causality_on_gpu():
+    base = synth.WORKLOADS["pretrain_d128_L2048"]
+    wl = synth.shrink(base, B=1, H=4, L=400, d=128, kq_place=mta.PRE_EXACT, seed=34)
+    inp = synth.make_attn_inputs(wl)
+    a = run_attn(wl, inp, mta.PATH_KQ)
+    t = 201
+    for n, s in (("q", 1), ("k", 2), ("v", 3)):
+        x = inp[n].copy()
+        x[:, t:] = synth.round_bf16(synth.normal(98, s, x[:, t:].shape))
+        inp[n] = x
+    b = run_attn(wl, inp, mta.PATH_KQ)
+    assert torch.equal(a[:, :t], b[:, :t])
+    assert not torch.equal(a[:, t:], b[:, t:])
+
+
+def test_exact_indicator_full_size_sampled():
+    wl = synth.shrink(synth.WORKLOADS["pretrain_d128_L2048"], kq_place=mta.PRE_EXACT)
+    inp = synth.make_attn_inputs(wl)
+    out = run_attn(wl, inp)
+    rows = sample_rows(wl, seed=5)
+    ref = O.mta_attention_rows(inp["q"], inp["k"], inp["v"], inp["theta"], inp["w"], wl.c_h, rows,
+                               O.PRE_EXACT, wl.head_place)
+    got = torch.stack([out[b, i] for b, i in rows])
+    assert_close(got, ref, "bf16")
+
+
+@pytest.mark.parametrize("name,path", [("layer_post_D2048_L4096", mta.PATH_AUTO),
+                                       ("layer_pre_D2048_L4096", mta.PATH_AUTO),
+                                       ("layer_post_D2048_L4096", mta.PATH_SIMT)])
+def test_layer_sigmoid_gate(name, path):
+    """The sigmoid scalar gate replaces the depth scale in every epilogue."""
+    wl = synth.shrink(synth.WORKLOADS[name], B=2, L=300, D=256, H=2, d=128, seed=124)
+    inp = synth.make_layer_inputs(wl)
+    gate = np.array([-0.8, 1.3], np.float32)
+    x, wqkv, wo = dev(inp["x"]), dev(inp["wqkv"]), dev(inp["wo"])
+    out = mta.layer_fwd(x, wqkv, dev(inp["theta"], "f32"), dev(inp["w"], "f32"),
+                        dev(inp["gamma"], "f32"), dev(inp["beta"], "f32"), wo, wl.H, wl.c_q,
+                        wl.c_k, wl.c_h, wl.kq_place, wl.head_place, eps=inp["eps"],
+                        layer=wl.depth, gate=dev(gate, "f32"), path=path, check=True)
+    torch.cuda.synchronize()
+    ref = O.mta_layer(inp["x"], inp["wqkv"], inp["theta"], inp["w"], inp["gamma"], inp["beta"],
+                      inp["eps"], O.sigmoid_gate(gate), inp["wo"], wl.H, wl.c_h, wl.kq_place,
+                      wl.head_place)
+    assert_close(out, ref, "bf16")
+
+
+def test_group_norm_sigmoid_gate():
+    o = synth.round_bf16(synth.normal(5, 1, (300, 4, 128), mean=0.1, std=1.5))
+    gamma = synth.normal(5, 2, (4 * 128,), mean=1.0, std=0.1)
+    beta = synth.normal(5, 3, (4 * 128,), std=0.1)
+    gate = np.array([-2.0, 0.0, 0.4, 3.0], np.float32)
+    y = mta.group_norm_scale(dev(o), dev(gamma, "f32"), dev(beta, "f32"), 1e-5, 1.0,
+                             gate=dev(gate, "f32"))
+    torch.cuda.synchronize()
+    assert_close(y, O.group_norm_scale(o, gamma, beta, 1e-5, O.sigmoid_gate(gate)), "bf16")

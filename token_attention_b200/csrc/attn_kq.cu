@@ -62,9 +62,12 @@ constexpr int kTmaWarp = 8, kMmaWarp = 9;
 constexpr int kBarAll = 1;      // named barrier over both softmax warpgroups
 constexpr int kKqMaxClusters = 160;  // persistent grid: at most this many CTAs (>= SM count)
 
-template <int D, int CQ, int CK, int MIX>
+template <int D, int CQ, int CK, int MIX, bool EXACT>
 struct KGeo {
-  static constexpr int C = CK / 2, HALO = CQ - 1, W = HALO + C, M = HALO + 2 * C;
+  // band 0 <= i-j < W where taps are masked: keys after the shifted query (Mask_0)
+  // or after the output query (exact indicator); Vp[i][m] = q[i] . k[i-m+OFF]
+  static constexpr int C = CK / 2, HALO = CQ - 1, W = EXACT ? C : HALO + C, M = HALO + 2 * C;
+  static constexpr int OFF = EXACT ? HALO : 0;
   static constexpr int BM = 128, BN = 128, HALF = BN / 2, DH = D / 2;
   static constexpr int QROWS = (BM + HALO + 7) / 8 * 8;  // query rows staged (with halo)
   static constexpr int NSTRIP = D / 8;
@@ -116,6 +119,7 @@ struct KqParams {
   __nv_bfloat16 *out;   // [B][L][H][D]
   const float *gamma, *beta;
   float eps, lam;
+  const float *gate;    // [H] sigmoid gate logits (replace lam) or null
   int gn;
   int B, L, H, n_qtiles, lpad;
   float qk_scale;
@@ -155,11 +159,11 @@ __device__ __forceinline__ int item_index(int c, int r, int n_clusters) {
   return r * n_clusters + ((r & 1) ? n_clusters - 1 - c : c);
 }
 
-template <int D, int CQ, int CK, int MIX>
+template <int D, int CQ, int CK, int MIX, bool EXACT>
 __global__ void __launch_bounds__(kThreads, 1)
     attn_kq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                    const __grid_constant__ CUtensorMap tmV, const KqParams p) {
-  using G = KGeo<D, CQ, CK, MIX>;
+  using G = KGeo<D, CQ, CK, MIX, EXACT>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t *Qs = smem + G::OFF_Q;
@@ -440,9 +444,10 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
           for (int jj = 0; jj < G::HALF; ++jj) cv[jj] *= qinv;
         }
-        // the band 0 <= i-j < W, where Mask_0 removes taps: the convolution tap by
-        // tap over the unmasked taps, from the past dot products:
-        //   C[i][i-dd] = s * sum_{a,t: m = dd - a + (t - c) >= 0} theta[a][t] Vp[i-a][m]
+        // the band 0 <= i-j < W, where the mask removes taps: the convolution tap by
+        // tap over the kept taps, from the dot products (key (i-a) - m, m = dd - a + t - c):
+        //   Mask_0: taps with m >= 0; exact indicator: taps with key <= i, i.e. t >= c - dd
+        //   C[i][i-dd] = s * sum_{kept a,t} theta[a][t] q[i-a] . k[i-a-m]
         const int dmax = qi - j0 - cb;  // i - j for this warpgroup's first column
         if (out_row && dmax >= 0 && dmax - (G::W - 1) < G::HALF) {
           float acc[G::W];
@@ -460,7 +465,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
               for (int dd = 0; dd < G::W; ++dd) {
                 const int m = dd - a + tp - G::C;
-                if (m >= 0 && m < G::M) acc[dd] = fmaf(thv, vr[m], acc[dd]);
+                const bool kept = EXACT ? tp >= G::C - dd : m >= 0;
+                if (kept && m + G::OFF >= 0 && m + G::OFF < G::M) acc[dd] = fmaf(thv, vr[m + G::OFF], acc[dd]);
               }
             }
           }
@@ -608,7 +614,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         const float *gm = p.gamma + static_cast<long long>(h) * D + zc;
         const float *bt = p.beta + static_cast<long long>(h) * D + zc;
 #pragma unroll
-        for (int i = 0; i < G::DH; ++i) o[i] = ((o[i] - mu) * rstd * gm[i] + bt[i]) * p.lam;
+        const float mh = head_multiplier(p.gate, p.lam, h);
+#pragma unroll
+        for (int i = 0; i < G::DH; ++i) o[i] = ((o[i] - mu) * rstd * gm[i] + bt[i]) * mh;
       }
       if (out_row) {
         __nv_bfloat16 *dst = p.out + ((static_cast<long long>(it.b) * L + qi) * p.H + h) * D + zc;
@@ -636,9 +644,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 }
 
-template <int D, int CQ, int CK, int MIX>
+template <int D, int CQ, int CK, int MIX, bool EXACT>
 cudaError_t launch_kq_one(const AttnArgs &a, const GnArgs *gn, const KqPrepArgs &pa, float *xg) {
-  using G = KGeo<D, CQ, CK, MIX>;
+  using G = KGeo<D, CQ, CK, MIX, EXACT>;
   alignas(64) CUtensorMap tq, tk, tv;
   const unsigned long long dims[4] = {static_cast<unsigned long long>(D), static_cast<unsigned long long>(a.H),
                                       static_cast<unsigned long long>(a.L), static_cast<unsigned long long>(a.B)};
@@ -664,6 +672,7 @@ cudaError_t launch_kq_one(const AttnArgs &a, const GnArgs *gn, const KqPrepArgs 
   p.beta = gn ? gn->beta : nullptr;
   p.eps = gn ? gn->eps : 0.f;
   p.lam = gn ? gn->lam : 1.f;
+  p.gate = gn ? gn->gate : nullptr;
   p.B = a.B;
   p.L = a.L;
   p.H = a.H;
@@ -674,7 +683,7 @@ cudaError_t launch_kq_one(const AttnArgs &a, const GnArgs *gn, const KqPrepArgs 
   p.vp = pa.vp;
   p.xg = xg;
   p.err = a.err;
-  auto kern = attn_kq_kernel<D, CQ, CK, MIX>;
+  auto kern = attn_kq_kernel<D, CQ, CK, MIX, EXACT>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, G::SMEM);
   if (e != cudaSuccess) return e;
   // persistent: as many clusters as can be resident at once (at most one per work
@@ -707,7 +716,7 @@ size_t align256(size_t x) { return (x + 255) / 256 * 256; }
 
 bool attn_kq_supported(const AttnArgs &a) {
   if (a.dtype != 1 || (a.d != 64 && a.d != 128)) return false;
-  if (a.kq != 1 || a.cq != 6 || a.ck != 11) return false;
+  if ((a.kq != 1 && a.kq != 3) || a.cq != 6 || a.ck != 11) return false;
   if (!(a.hp == 0 || (a.hp == 2 && a.ch == 2))) return false;
   if (a.B > 65535 || a.H > 65535 || (a.L + 127) / 128 > 65535) return false;
   const uintptr_t al = reinterpret_cast<uintptr_t>(a.q) | reinterpret_cast<uintptr_t>(a.k) |
@@ -742,6 +751,7 @@ cudaError_t launch_attn_kq(const AttnArgs &a, const GnArgs *gn, void *ws) {
   pa.n_tiles = (a.L + 127) / 128;
   pa.lpad = pa.n_tiles * 128;
   pa.scale_log2 = a.scale * 1.4426950408889634f;
+  pa.exact = a.kq == 3;
   const size_t BH = static_cast<size_t>(a.B) * a.H, BHL = BH * a.L;
   char *base = static_cast<char *>(ws);
   pa.kt = base;
@@ -752,8 +762,10 @@ cudaError_t launch_attn_kq(const AttnArgs &a, const GnArgs *gn, void *ws) {
   if (e != cudaSuccess) return e;
   const bool post = a.hp == 2;
   if (a.d == 128)
-    return post ? launch_kq_one<128, 6, 11, 2>(a, gn, pa, xg) : launch_kq_one<128, 6, 11, 0>(a, gn, pa, xg);
-  return post ? launch_kq_one<64, 6, 11, 2>(a, gn, pa, xg) : launch_kq_one<64, 6, 11, 0>(a, gn, pa, xg);
+    return post ? (pa.exact ? launch_kq_one<128, 6, 11, 2, true>(a, gn, pa, xg) : launch_kq_one<128, 6, 11, 2, false>(a, gn, pa, xg))
+                : (pa.exact ? launch_kq_one<128, 6, 11, 0, true>(a, gn, pa, xg) : launch_kq_one<128, 6, 11, 0, false>(a, gn, pa, xg));
+  return post ? (pa.exact ? launch_kq_one<64, 6, 11, 2, true>(a, gn, pa, xg) : launch_kq_one<64, 6, 11, 2, false>(a, gn, pa, xg))
+              : (pa.exact ? launch_kq_one<64, 6, 11, 0, true>(a, gn, pa, xg) : launch_kq_one<64, 6, 11, 0, false>(a, gn, pa, xg));
 }
 
 }  // namespace mta

@@ -75,7 +75,8 @@ __global__ void __launch_bounds__(kThreads) attn_simt_kernel(AttnArgs a, int BR)
   const T *v = static_cast<const T *>(a.v);
   T *out = static_cast<T *>(a.out);
   const float NEG_INF = -INFINITY;
-  const bool kq = (a.kq == 1);
+  const bool kq = (a.kq != 0);
+  const bool exact = (a.kq == 3);  // exact causal indicator instead of Mask_0
 
   for (int i = tid; i < ch * cq * ck; i += kThreads) th[i] = kq ? a.theta[g * ch * cq * ck + i] : 0.f;
   for (int i = tid; i < ch * ch; i += kThreads)
@@ -100,10 +101,11 @@ __global__ void __launch_bounds__(kThreads) attn_simt_kernel(AttnArgs a, int BR)
         }
         __syncthreads();
         // Mask_0(A_hat) on the halo tile: future keys of each (shifted) query are 0
+        // (with the exact indicator the logits stay unmasked here; see below)
         for (int i = tid; i < HR * HC; i += kThreads) {
           const int r = i / HC, s = i % HC, iq = i0 - (cq - 1) + r, jk = j0 - c + s;
           float val = 0.f;
-          if (iq >= 0 && iq < L && jk >= 0 && jk < L && (!kq || jk <= iq)) {
+          if (iq >= 0 && iq < L && jk >= 0 && jk < L && (!kq || exact || jk <= iq)) {
             const float *qr = Qs + r * dp, *kr = Ks + s * dp;
             for (int e = 0; e < d; ++e) val = fmaf(qr[e], kr[e], val);
             val *= a.scale;
@@ -111,16 +113,18 @@ __global__ void __launch_bounds__(kThreads) attn_simt_kernel(AttnArgs a, int BR)
           Sh[i] = val;
         }
         __syncthreads();
-        // key-query convolution: C[i][j] = sum_a sum_t theta[a][t] M0[i-a][j-(t-c)]
+        // key-query convolution: C[i][j] = sum_a sum_t theta[a][t] M0[i-a][j-(t-c)];
+        // with the exact indicator a tap counts when its key j-(t-c) <= i
         for (int i = tid; i < tile; i += kThreads) {
           const int r = i / BC, j = i % BC;
           float val;
           if (kq) {
             val = 0.f;
             const float *tk = th + hl * cq * ck;
+            const int t0 = exact ? max(0, (j0 + j) + c - (i0 + r)) : 0;
             for (int aa = 0; aa < cq; ++aa) {
               const float *srow = Sh + (r + cq - 1 - aa) * HC + j + 2 * c;
-              for (int t = 0; t < ck; ++t) val = fmaf(tk[aa * ck + t], srow[-t], val);
+              for (int t = t0; t < ck; ++t) val = fmaf(tk[aa * ck + t], srow[-t], val);
             }
           } else {
             val = Sh[(r + cq - 1) * HC + j + c];

@@ -120,6 +120,7 @@ struct TcParams {
   __nv_bfloat16 *out;   // [B][L][H][D]
   const float *gamma, *beta;
   float eps, lam;
+  const float *gate;    // [H] sigmoid gate logits (replace lam) or null
   int gn;               // fuse group norm + depth scale
   int L, H, n_qtiles;
   float qk_scale;       // logit scale (1/sqrt(d) unless the caller chose another)
@@ -523,7 +524,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       const float *gm = p.gamma + static_cast<long long>(h) * D + cbase;
       const float *bt = p.beta + static_cast<long long>(h) * D + cbase;
 #pragma unroll
-      for (int i = 0; i < G::DQ; ++i) o[i] = ((o[i] - mu) * rstd * gm[i] + bt[i]) * p.lam;
+      const float mh = head_multiplier(p.gate, p.lam, h);
+#pragma unroll
+      for (int i = 0; i < G::DQ; ++i) o[i] = ((o[i] - mu) * rstd * gm[i] + bt[i]) * mh;
     }
   }
   if (conv_thread && r >= G::HALO && qrow < L) {
@@ -568,6 +571,7 @@ cudaError_t launch_one(const AttnArgs &a, const GnArgs *gn) {
   p.beta = gn ? gn->beta : nullptr;
   p.eps = gn ? gn->eps : 0.f;
   p.lam = gn ? gn->lam : 1.f;
+  p.gate = gn ? gn->gate : nullptr;
   p.L = a.L;
   p.H = a.H;
   p.n_qtiles = (a.L + G::BR - 1) / G::BR;

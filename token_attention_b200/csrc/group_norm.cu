@@ -12,6 +12,7 @@
 #include <stdint.h>
 
 #include "internal.h"
+#include "ptx.cuh"
 
 namespace mta {
 namespace {
@@ -41,8 +42,9 @@ __global__ void __launch_bounds__(256) group_norm_d128_kernel(const __nv_bfloat1
     const float rstd = rsqrtf(warp_sum(s2) * (1.f / 128.f) + gn.eps);
     const float4 g4 = reinterpret_cast<const float4 *>(gn.gamma + h * 128)[lane];
     const float4 b4 = reinterpret_cast<const float4 *>(gn.beta + h * 128)[lane];
-    const float y0 = (x[0] * rstd * g4.x + b4.x) * gn.lam, y1 = (x[1] * rstd * g4.y + b4.y) * gn.lam;
-    const float y2 = (x[2] * rstd * g4.z + b4.z) * gn.lam, y3 = (x[3] * rstd * g4.w + b4.w) * gn.lam;
+    const float m = head_multiplier(gn.gate, gn.lam, h);
+    const float y0 = (x[0] * rstd * g4.x + b4.x) * m, y1 = (x[1] * rstd * g4.y + b4.y) * m;
+    const float y2 = (x[2] * rstd * g4.z + b4.z) * m, y3 = (x[3] * rstd * g4.w + b4.w) * m;
     __nv_bfloat162 q0 = __floats2bfloat162_rn(y0, y1), q1 = __floats2bfloat162_rn(y2, y3);
     uint2 outw;
     outw.x = *reinterpret_cast<uint32_t *>(&q0);
@@ -82,7 +84,7 @@ __global__ void __launch_bounds__(256) group_norm_any_kernel(const __nv_bfloat16
       const int e = lane + 32 * i;
       if (e < d)
         y[r * d + e] = __float2bfloat16_rn((x[i] * rstd * gn.gamma[h * d + e] + gn.beta[h * d + e]) *
-                                           gn.lam);
+                                           head_multiplier(gn.gate, gn.lam, h));
     }
   }
 }

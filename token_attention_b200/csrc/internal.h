@@ -26,6 +26,7 @@ struct AttnArgs {
 struct GnArgs {
   const float *gamma, *beta;  // [H*d]
   float eps, lam;
+  const float *gate;          // [H] sigmoid gate logits, replacing lam; may be null
 };
 
 // Generic CUDA-core kernel: every supported configuration, fp32 arithmetic.
@@ -49,6 +50,7 @@ struct KqPrepArgs {
   float *vp;              // [B][H][L][M] past dot products q[i] . k[i-m], m < M
   float scale_log2;       // logit scale times log2(e)
   int B, H, L, d, cq, ck, M, n_tiles, lpad;
+  int exact;              // exact causal indicator: Vp[i][m] = q[i] . k[i-m+(cq-1)]
 };
 cudaError_t launch_kq_prep(const KqPrepArgs &a, cudaStream_t stream);
 // Workspace bytes of the contraction path (beyond the error word) and whether it applies.

@@ -17,7 +17,9 @@
 //       value exceeds 2^14 and small keys keep fp16's relative precision);
 //   fac [B][H][Lpad] fp32: s * log2(e) * 2^-e_j (the attention kernel's column
 //       factor; 0 for the padding keys L <= j < Lpad, Lpad = L rounded up to 128);
-//   Vp  [B][H][L][M] fp32: raw past dot products (no scale).
+//   Vp  [B][H][L][M] fp32: raw past dot products (no scale); with the exact causal
+//       indicator shifted by c_q-1: Vp[i][m] = q[i] . k[i-m+(c_q-1)], so that the
+//       band can also read keys up to c_q-1 after a shifted query.
 // Every value written for key or query j depends on inputs at positions <= j + c
 // only, and Kt_a[j] is used only for queries i >= j + W > j + c: the path stays
 // exactly causal.  One CTA per (key tile, head, batch); the key rows with their
@@ -36,12 +38,15 @@ constexpr int kPrepThreads = 256;
 constexpr int kTile = 128;
 constexpr int kRun = 16;  // consecutive keys one thread convolves from a register window
 
-template <int D, int CQ, int CK>
+template <int D, int CQ, int CK, bool EXACT>
 struct PrepGeo {
   static constexpr int C = CK / 2;
-  static constexpr int M = (CQ - 1) + 2 * C;          // past dot products per query
+  static constexpr int M = (CQ - 1) + 2 * C;          // dot products per query
+  static constexpr int OFF = EXACT ? CQ - 1 : 0;      // Vp[i][m] = q[i] . k[i-m+OFF]
   static constexpr int LO = M - 1;                    // staged rows before the tile
-  static constexpr int ROWS = kTile + LO + C;         // keys j0-LO .. j0+kTile-1+C
+  // keys j0-LO .. : the Kt window reaches kTile-1+C past j0, a warp's 32-key tile of
+  // dot products 16*7+31+OFF-LO
+  static constexpr int ROWS = (kTile + LO + C) > (16 * 7 + 32 + OFF) ? (kTile + LO + C) : (16 * 7 + 32 + OFF);
   static constexpr int KSTR = D + 8;                  // staged row stride (floats): fewer bank conflicts
   static constexpr int SMEM = ROWS * KSTR * 4;
   static_assert(M - 1 + 16 <= 32, "past dot products of a 16-row block span 32 keys");
@@ -65,9 +70,9 @@ __device__ __forceinline__ uint32_t pack2_bf16(float lo, float hi) {
 
 __device__ __forceinline__ float pow2i(int e) { return __int_as_float((127 + e) << 23); }  // |e| <= 126
 
-template <int D, int CQ, int CK>
+template <int D, int CQ, int CK, bool EXACT>
 __global__ void __launch_bounds__(kPrepThreads) kq_prep_kernel(KqPrepArgs p) {
-  using G = PrepGeo<D, CQ, CK>;
+  using G = PrepGeo<D, CQ, CK, EXACT>;
   extern __shared__ float ks[];  // [ROWS][KSTR] fp32, row r = key j0 - LO + r
   __shared__ float rmax[G::ROWS];
   __shared__ int es[kTile];
@@ -165,12 +170,12 @@ __global__ void __launch_bounds__(kPrepThreads) kq_prep_kernel(KqPrepArgs p) {
     }
   }
 
-  // Vp[i][m] = q[i] . k[i-m]: per warp a block of 16 query rows i0 .. i0+15 against
-  // the 32 keys i0-(M-1) .. i0+32-M (a 16x32 tile of Q K^T on the tensor cores,
-  // exact products of bf16 values, fp32 sums), of which the band m < M is kept.
+  // Vp[i][m] = q[i] . k[i-m+OFF]: per warp a block of 16 query rows i0 .. i0+15
+  // against the 32 keys i0-(M-1)+OFF .. i0+32-M+OFF (a 16x32 tile of Q K^T on the
+  // tensor cores, exact products of bf16 values, fp32 sums), of which m < M is kept.
   const int warp = tid >> 5, lane = tid & 31, g = lane >> 2, tq = lane & 3;
   const int i0 = 16 * warp;                 // local query row of the block
-  const int krow0 = i0;                     // staged row of key j0+i0-(M-1) (= LO - (M-1) + i0)
+  const int krow0 = i0 + G::OFF;            // staged row of key j0+i0-(M-1)+OFF (LO = M-1)
   float acc[4][4];
 #pragma unroll
   for (int nt = 0; nt < 4; ++nt)
@@ -212,10 +217,10 @@ __global__ void __launch_bounds__(kPrepThreads) kq_prep_kernel(KqPrepArgs p) {
     }
 }
 
-template <int D, int CQ, int CK>
+template <int D, int CQ, int CK, bool EXACT>
 cudaError_t launch_prep_one(const KqPrepArgs &p, cudaStream_t stream) {
-  using G = PrepGeo<D, CQ, CK>;
-  auto kern = kq_prep_kernel<D, CQ, CK>;
+  using G = PrepGeo<D, CQ, CK, EXACT>;
+  auto kern = kq_prep_kernel<D, CQ, CK, EXACT>;
   const cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, G::SMEM);
   if (e != cudaSuccess) return e;
   kern<<<dim3(p.n_tiles, p.H, p.B), kPrepThreads, G::SMEM, stream>>>(p);
@@ -225,8 +230,10 @@ cudaError_t launch_prep_one(const KqPrepArgs &p, cudaStream_t stream) {
 }  // namespace
 
 cudaError_t launch_kq_prep(const KqPrepArgs &p, cudaStream_t stream) {
-  if (p.cq != 6 || p.ck != 11 || p.M != PrepGeo<128, 6, 11>::M) return cudaErrorInvalidValue;
-  return p.d == 128 ? launch_prep_one<128, 6, 11>(p, stream) : launch_prep_one<64, 6, 11>(p, stream);
+  if (p.cq != 6 || p.ck != 11 || p.M != PrepGeo<128, 6, 11, false>::M) return cudaErrorInvalidValue;
+  if (p.exact)
+    return p.d == 128 ? launch_prep_one<128, 6, 11, true>(p, stream) : launch_prep_one<64, 6, 11, true>(p, stream);
+  return p.d == 128 ? launch_prep_one<128, 6, 11, false>(p, stream) : launch_prep_one<64, 6, 11, false>(p, stream);
 }
 
 }  // namespace mta

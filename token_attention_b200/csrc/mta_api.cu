@@ -29,7 +29,8 @@ mta_status check_cfg(const mta_cfg *c) {
   if (c->c_q < 1 || c->c_q > 8) return MTA_ERR_INVALID;
   if (c->c_k < 1 || c->c_k > 15 || c->c_k % 2 == 0) return MTA_ERR_INVALID;
   if (c->c_h < 1 || c->c_h > 16 || c->H % c->c_h != 0) return MTA_ERR_INVALID;
-  if (c->kq_place != MTA_OFF && c->kq_place != MTA_PRE) return MTA_ERR_INVALID;
+  if (c->kq_place != MTA_OFF && c->kq_place != MTA_PRE && c->kq_place != MTA_PRE_EXACT)
+    return MTA_ERR_INVALID;
   if (c->head_place != MTA_OFF && c->head_place != MTA_PRE && c->head_place != MTA_POST)
     return MTA_ERR_INVALID;
   if (c->dtype != MTA_F32 && c->dtype != MTA_BF16) return MTA_ERR_INVALID;
@@ -59,7 +60,8 @@ enum Kernel { K_SIMT = 1, K_TC = 2, K_KQ = 3 };
 // Shape-level test for the contraction kernel (pointer alignment aside): used
 // to size the workspace.
 bool kq_shape_ok(const mta_cfg *c) {
-  return c->dtype == MTA_BF16 && (c->d == 64 || c->d == 128) && c->kq_place == MTA_PRE &&
+  return c->dtype == MTA_BF16 && (c->d == 64 || c->d == 128) &&
+         (c->kq_place == MTA_PRE || c->kq_place == MTA_PRE_EXACT) &&
          c->c_q == 6 && c->c_k == 11 &&
          (c->head_place == MTA_OFF || (c->head_place == MTA_POST && c->c_h == 2));
 }
@@ -103,7 +105,7 @@ cudaError_t launch_kernel(Kernel k, const AttnArgs &a, const GnArgs *gn, void *k
 mta_status check_attn_pointers(const void *q, const void *k, const void *v, const float *theta,
                                const float *w, const mta_cfg *c, const void *out) {
   if (!q || !k || !v || !out) return MTA_ERR_INVALID;
-  if (c->kq_place == MTA_PRE && !theta) return MTA_ERR_INVALID;
+  if (c->kq_place != MTA_OFF && !theta) return MTA_ERR_INVALID;
   if (c->head_place != MTA_OFF && !w) return MTA_ERR_INVALID;
   const size_t es = c->dtype == MTA_F32 ? 4 : 2;
   if (!aligned(q, es) || !aligned(k, es) || !aligned(v, es) || !aligned(out, es))
@@ -134,6 +136,7 @@ GnArgs make_gn(const mta_gn *gn) {
   g.eps = gn->eps > 0.f ? gn->eps : 1e-5f;
   g.lam = gn->depth_scale >= 0.f ? gn->depth_scale
                                  : static_cast<float>(1.0 - 0.8 * exp(-0.3 * gn->layer));
+  g.gate = gn->gate;
   return g;
 }
 
@@ -224,7 +227,7 @@ mta_status mta_layer_fwd(const void *x, const void *Wqkv, const float *theta, co
   if (s != MTA_OK) return s;
   if (cfg->dtype != MTA_BF16) return MTA_ERR_UNSUPPORTED;
   if (!x || !Wqkv || !Wo || !out || !gn || !gn->gamma || !gn->beta) return MTA_ERR_INVALID;
-  if (cfg->kq_place == MTA_PRE && !theta) return MTA_ERR_INVALID;
+  if (cfg->kq_place != MTA_OFF && !theta) return MTA_ERR_INVALID;
   if (cfg->head_place != MTA_OFF && !w_head) return MTA_ERR_INVALID;
   if (!aligned(x, 16) || !aligned(Wqkv, 16) || !aligned(Wo, 16) || !aligned(out, 16) ||
       !aligned(gn->gamma, 4) || !aligned(gn->beta, 4))

@@ -80,6 +80,12 @@ __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, volati
   }
 }
 
+// Multiplier of head h's normalised output: the sigmoid scalar gate when gate
+// logits are given, else the depth scale (section 3.3).
+__device__ __forceinline__ float head_multiplier(const float *gate, float lam, int h) {
+  return gate ? 1.f / (1.f + expf(-gate[h])) : lam;
+}
+
 // ----------------------------------------------------------------------------
 // proxies and fences
 // ----------------------------------------------------------------------------

@@ -16,7 +16,7 @@ HERE = os.path.dirname(os.path.abspath(__file__))
 # the in-tree libmta.so next to this file.
 LIB_PATH = os.environ.get("MTA_LIB") or os.path.join(HERE, "libmta.so")
 
-OFF, PRE, POST = 0, 1, 2
+OFF, PRE, POST, PRE_EXACT = 0, 1, 2, 3   # PRE_EXACT: key-query convolution with the exact causal indicator
 F32, BF16 = 0, 1
 PATH_AUTO, PATH_SIMT, PATH_TC, PATH_KQ = 0, 1, 2, 3
 
@@ -40,7 +40,7 @@ class MtaCfg(ctypes.Structure):
 
 class MtaGn(ctypes.Structure):
     _fields_ = [("gamma", ctypes.c_void_p), ("beta", ctypes.c_void_p), ("eps", ctypes.c_float),
-                ("layer", ctypes.c_int), ("depth_scale", ctypes.c_float)]
+                ("layer", ctypes.c_int), ("depth_scale", ctypes.c_float), ("gate", ctypes.c_void_p)]
 
 
 class MtaError(RuntimeError):
@@ -160,10 +160,11 @@ def depth_scale(layer: int) -> float:
 
 
 def layer_fwd(x, wqkv, theta, w, gamma, beta, wo, H, c_q, c_k, c_h, kq_place=PRE,
-              head_place=POST, *, eps=1e-5, layer=12, lam=-1.0, out=None, ws=None,
+              head_place=POST, *, eps=1e-5, layer=12, lam=-1.0, gate=None, out=None, ws=None,
               path=PATH_AUTO, stream=None, check=False):
     """Full MTA layer, bf16.  x [B, L, D]; wqkv [3D, D]; wo [D, D]; gamma, beta [D]
-    fp32.  Returns out [B, L, D] bf16."""
+    fp32; gate: optional [H] fp32 sigmoid-gate logits replacing the depth scale.
+    Returns out [B, L, D] bf16."""
     import torch
     B, L, D = x.shape
     d = D // H
@@ -174,7 +175,8 @@ def layer_fwd(x, wqkv, theta, w, gamma, beta, wo, H, c_q, c_k, c_h, kq_place=PRE
     if ws is None:
         ws = workspace(lib().mta_layer_workspace_bytes(ctypes.byref(cfg)), x.device)
     cfg.workspace, cfg.workspace_bytes = ws.data_ptr(), ws.numel()
-    gn = MtaGn(gamma.data_ptr(), beta.data_ptr(), eps, layer, lam)
+    gn = MtaGn(gamma.data_ptr(), beta.data_ptr(), eps, layer, lam,
+               gate.data_ptr() if gate is not None else None)
     _check("mta_layer_fwd", lib().mta_layer_fwd(_ptr(x), _ptr(wqkv), _ptr(theta), _ptr(w),
                                                ctypes.byref(gn), _ptr(wo), ctypes.byref(cfg),
                                                _ptr(out)))
@@ -200,14 +202,15 @@ def gemm_bf16_nt(a, b, out=None, stream=None):
     return out
 
 
-def group_norm_scale(o, gamma, beta, eps=1e-5, lam=1.0, out=None, stream=None):
+def group_norm_scale(o, gamma, beta, eps=1e-5, lam=1.0, out=None, stream=None, gate=None):
     """Depth-scaled group norm of o [..., H, d] bf16 (dense)."""
     import torch
     H, d = o.shape[-2], o.shape[-1]
     tokens = o.numel() // (H * d)
     if out is None:
         out = torch.empty_like(o)
-    gn = MtaGn(gamma.data_ptr(), beta.data_ptr(), eps, 0, lam)
+    gn = MtaGn(gamma.data_ptr(), beta.data_ptr(), eps, 0, lam,
+               gate.data_ptr() if gate is not None else None)
     _check("mta_group_norm_scale", lib().mta_group_norm_scale(_ptr(o), ctypes.byref(gn), tokens, H,
                                                              d, _ptr(out), _stream_handle(stream)))
     return out
