@@ -68,18 +68,20 @@ def uses_contraction(wl: synth.Workload) -> bool:
     prepass) for this workload."""
     return (wl.dtype == "bf16" and wl.d in (64, 128) and wl.kq_place == synth.PRE
             and (wl.c_q, wl.c_k) == (6, 11)
-            and (wl.head_place == synth.OFF or (wl.head_place == synth.POST and wl.c_h == 2)))
+            and (wl.head_place == synth.OFF or wl.c_h == 2))
 
 
 def contraction_tensor_flops(wl: synth.Workload) -> float:
     """Tensor flops the contraction kernel executes per launch: per (batch, head,
     query tile, key tile at or below the diagonal) a 128x128 tile of the
-    c_q*d-long contraction and, per destination head of the group, a 128x128xd
-    P V product."""
+    c_q*d-long contraction (for each source head of the group with pre-softmax
+    mixing) and, per V head held (both heads of the group with post-softmax
+    mixing), a 128x128xd P V product."""
     nt = -(-wl.L // 128)
     tiles = wl.B * wl.H * nt * (nt + 1) // 2
     nv = 2 if wl.head_place == synth.POST else 1
-    return tiles * 2.0 * 128 * 128 * (wl.c_q * wl.d + nv * wl.d)
+    nsrc = 2 if wl.head_place == synth.PRE else 1
+    return tiles * 2.0 * 128 * 128 * (nsrc * wl.c_q * wl.d + nv * wl.d)
 
 
 def launches_per_step(wl: synth.Workload) -> int:

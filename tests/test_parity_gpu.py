@@ -90,9 +90,9 @@ def tc_applies(wl):
 
 def kq_applies(wl):
     """Whether the contraction kernel serves this configuration."""
-    return (wl.dtype == "bf16" and wl.d in (64, 128) and wl.kq_place == synth.PRE
+    return (wl.dtype == "bf16" and wl.d in (64, 128) and wl.kq_place in (synth.PRE, 3)
             and (wl.c_q, wl.c_k) == (6, 11)
-            and (wl.head_place == synth.OFF or (wl.head_place == synth.POST and wl.c_h == 2)))
+            and (wl.head_place == synth.OFF or wl.c_h == 2))
 
 
 @pytest.mark.parametrize("d,hp,L", SMALL)
@@ -306,7 +306,7 @@ def oracle_exact(wl, inp):
 
 
 @pytest.mark.parametrize("d,hp,L", [(64, synth.OFF, 9), (128, synth.POST, 300), (64, synth.POST, 300),
-                                    (128, synth.OFF, 1)])
+                                    (128, synth.OFF, 1), (128, synth.PRE, 300), (64, synth.PRE, 130)])
 @pytest.mark.parametrize("path", [mta.PATH_AUTO, mta.PATH_SIMT, mta.PATH_KQ])
 def test_exact_indicator_small(d, hp, L, path):
     base = synth.WORKLOADS["pretrain_d128_L2048"]

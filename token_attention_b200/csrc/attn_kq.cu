@@ -41,6 +41,7 @@
 #include <cuda.h>
 
 #include <algorithm>
+#include <type_traits>
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 #include <math.h>
@@ -76,7 +77,8 @@ struct KGeo {
   static constexpr int NDC = D / 64;
   static constexpr int NCH = CQ * NDC;                   // Kt chunks per key tile
   static constexpr int KCHUNK = BN * 128;                // 128 keys x 64 elements, fp16
-  static constexpr int NV = MIX == 2 ? 2 : 1;
+  static constexpr int NV = MIX == 2 ? 2 : 1;            // V heads per CTA (post-softmax mixing: both)
+  static constexpr int NSRC = MIX == 1 ? 2 : 1;          // heads whose C a CTA computes (pre-softmax mixing: both)
   static constexpr int CLUSTER = MIX == 2 ? 2 : 1;       // CTAs of a cluster: the heads of a group
   static constexpr int V_CHUNK = BN * 128;
   static constexpr int V_HEAD = BN * D * 2;
@@ -85,17 +87,21 @@ struct KGeo {
   static constexpr int U_BYTES = (UROWS * M * 4 + 15) / 16 * 16;
   static constexpr int CS_BYTES = 2 * BM * W * 4;        // band values, one block per warpgroup
   static constexpr int RED_BYTES = 10 * BM * 4;          // row maxima (2 tiles x 2 groups), l, norm sums
-  static constexpr int FAC_BYTES = 2 * BN * 4;           // column factors of two key tiles
-  static constexpr int SMALL_BYTES = 2048;
+  static constexpr int FAC_BYTES = NSRC * 2 * BN * 4;    // column factors of two key tiles, per source head
+  static constexpr int Q_ALLOC = (Q_BYTES + 1023) / 1024 * 1024;
+  // small area: taps [2 items][NSRC][128], per-warp |q| maxima, barriers, TMEM slot, abort flag
+  static constexpr int TH_OFF = 0, QRED_OFF = 2 * NSRC * 128 * 4, BAR_OFF = QRED_OFF + 64;
+  static constexpr int TSLOT_OFF = BAR_OFF + 8 * 32, ABORT_OFF = TSLOT_OFF + 8;
+  static constexpr int SMALL_BYTES = (ABORT_OFF + 8 + 255) / 256 * 256;
   // Kt ring: as many 16 KB stages as the shared memory left over holds (at most 8)
-  static constexpr int REST = (Q_BYTES + 1023) / 1024 * 1024 + V_BYTES + U_BYTES + CS_BYTES + RED_BYTES +
+  static constexpr int REST = NSRC * Q_ALLOC + V_BYTES + NSRC * U_BYTES + CS_BYTES + RED_BYTES +
                               FAC_BYTES + SMALL_BYTES + 1024;
   static constexpr int NS = (232448 - REST) / KCHUNK < 8 ? (232448 - REST) / KCHUNK : 8;
   static constexpr int OFF_Q = 0;
-  static constexpr int OFF_K = (Q_BYTES + 1023) / 1024 * 1024;
+  static constexpr int OFF_K = NSRC * Q_ALLOC;
   static constexpr int OFF_V = OFF_K + NS * KCHUNK;
   static constexpr int OFF_U = OFF_V + V_BYTES;
-  static constexpr int OFF_CS = OFF_U + U_BYTES;
+  static constexpr int OFF_CS = OFF_U + NSRC * U_BYTES;
   static constexpr int OFF_RED = OFF_CS + CS_BYTES;
   static constexpr int OFF_FAC = OFF_RED + RED_BYTES;
   static constexpr int OFF_SMALL = OFF_FAC + FAC_BYTES;
@@ -103,8 +109,10 @@ struct KGeo {
   // at least half the SM's shared memory: one CTA per SM, so the 512-column TMEM
   // allocation never waits for another CTA
   static constexpr int SMEM = SMEM_USED > 232448 / 2 + 1024 ? SMEM_USED : 232448 / 2 + 1024;
-  static constexpr uint32_t TMEM_COLS = 512, C_COL = 0, P_COL = 128, Z_COL0 = 256;
+  // tensor memory: C of each source head (128 columns each), P (64), Z
+  static constexpr uint32_t TMEM_COLS = 512, C_COL = 0, P_COL = 128 * NSRC, Z_COL0 = P_COL + 128;
   static_assert(Z_COL0 + 128 * (NV - 1) + D <= TMEM_COLS, "tensor memory");
+  static_assert(MIX != 1 || NV == 1, "pre-softmax mixing uses the destination head's V only");
   static_assert(OFF_K % 1024 == 0 && OFF_V % 1024 == 0, "swizzle alignment");
   static_assert(OFF_SMALL % 16 == 0, "alignment");
   static_assert(NS >= 3, "Kt ring");
@@ -172,17 +180,17 @@ __global__ void __launch_bounds__(kThreads, 1)
   float *Us = reinterpret_cast<float *>(smem + G::OFF_U);
   float *Cs = reinterpret_cast<float *>(smem + G::OFF_CS);
   float *red = reinterpret_cast<float *>(smem + G::OFF_RED);
-  float *facs = reinterpret_cast<float *>(smem + G::OFF_FAC);  // [2][BN]
+  float *facs = reinterpret_cast<float *>(smem + G::OFF_FAC);  // [NSRC][2][BN]
   uint8_t *small = smem + G::OFF_SMALL;
-  float *th_s = reinterpret_cast<float *>(small);          // [2][CQ*CK] by item parity
-  float *qred = reinterpret_cast<float *>(small + 1024);   // [8] per-warp max |q|
-  uint64_t *bars = reinterpret_cast<uint64_t *>(small + 1088);
+  float *th_s = reinterpret_cast<float *>(small + G::TH_OFF);   // [2 items][NSRC][128]
+  float *qred = reinterpret_cast<float *>(small + G::QRED_OFF); // [8] per-warp max |q|
+  uint64_t *bars = reinterpret_cast<uint64_t *>(small + G::BAR_OFF);
   uint64_t *q_full = bars + 0, *q_ready = bars + 1, *q_free = bars + 2, *z_free = bars + 3;
   uint64_t *x_ready = bars + 4, *k_full = bars + 5, *k_empty = bars + 5 + G::NS;
   uint64_t *v_full = bars + 5 + 2 * G::NS, *v_empty = v_full + 1, *c_full = v_full + 2;
   uint64_t *c_free = v_full + 3, *p_full = v_full + 4, *mma_done = v_full + 5;
-  uint32_t *tslot = reinterpret_cast<uint32_t *>(small + 1088 + 8 * 32);
-  volatile int *abort_flag = reinterpret_cast<volatile int *>(small + 1088 + 8 * 32 + 8);
+  uint32_t *tslot = reinterpret_cast<uint32_t *>(small + G::TSLOT_OFF);
+  volatile int *abort_flag = reinterpret_cast<volatile int *>(small + G::ABORT_OFF);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   // cluster c (the two heads of a group with post-softmax mixing, else one CTA)
@@ -200,6 +208,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     return true;
   };
   auto kv_tiles = [&](const Item &it) { return min(L - 1, it.qt * G::BM + G::BM - 1) / G::BN + 1; };
+  // the head whose C is accumulated as source s of destination head h
+  auto src_head = [&](int h, int s) { return G::NSRC == 2 ? (h & ~1) + s : h; };
 
   if (threadIdx.x == 0) {
     mbar_init(q_full, 1); mbar_init(q_ready, 8); mbar_init(q_free, 1); mbar_init(z_free, 8);
@@ -225,13 +235,13 @@ __global__ void __launch_bounds__(kThreads, 1)
       Item it;
       for (int r = 0; item_at(r, it) && !*abort_flag; ++r) {
         const int h = it.g * CL + hr, n_kv = kv_tiles(it);
-        const int zbase = (it.b * p.H + h) * CQ;
         for (int t = 0; t < n_kv && !*abort_flag; ++t)
-          for (int ch = 0; ch < G::NCH; ++ch, ++cnt) {
-            const int st = cnt % G::NS;
+          for (int ch = 0; ch < G::NSRC * G::NCH; ++ch, ++cnt) {
+            const int st = cnt % G::NS, sc = ch / G::NCH, cs = ch % G::NCH;
+            const int zbase = (it.b * p.H + src_head(h, sc)) * CQ;
             if (!mbar_wait(k_empty + st, ((cnt / G::NS) & 1) ^ 1, abort_flag, p.err)) break;
             mbar_arrive_expect_tx(k_full + st, G::KCHUNK);
-            tma_load_3d(Ks + st * G::KCHUNK, &tmK, k_full + st, (ch % G::NDC) * 64, t * G::BN, zbase + ch / G::NDC);
+            tma_load_3d(Ks + st * G::KCHUNK, &tmK, k_full + st, (cs % G::NDC) * 64, t * G::BN, zbase + cs / G::NDC);
           }
       }
       if (*abort_flag)  // copies still in flight land before the CTA exits
@@ -262,9 +272,12 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int r = 0; item_at(r, it) && !*abort_flag; ++r, ++nq) {
         if (r > 0 && !mbar_wait(q_free, (r - 1) & 1, abort_flag, p.err)) break;
         const int h = it.g * CL + hr, row0 = it.qt * G::BM - G::HALO;
-        mbar_arrive_expect_tx(q_full, G::Q_BYTES);
+        mbar_arrive_expect_tx(q_full, G::NSRC * G::Q_BYTES);
 #pragma unroll 1
-        for (int s2 = 0; s2 < G::NSTRIP; ++s2) tma_load_4d(Qs + s2 * G::STRIP, &tmQ, q_full, 8 * s2, h, row0, it.b);
+        for (int sc = 0; sc < G::NSRC; ++sc)
+#pragma unroll 1
+          for (int s2 = 0; s2 < G::NSTRIP; ++s2)
+            tma_load_4d(Qs + sc * G::Q_ALLOC + s2 * G::STRIP, &tmQ, q_full, 8 * s2, src_head(h, sc), row0, it.b);
       }
       if (nq) drain_wait(q_full, (nq - 1) & 1);
     }
@@ -284,17 +297,19 @@ __global__ void __launch_bounds__(kThreads, 1)
       // shifted by a rows x Kt_a
       auto issue_c = [&](bool last_of_item) -> bool {
         if (T > 0 && !mbar_wait(c_free, (T - 1) & 1, abort_flag, p.err)) return false;
-        for (int ch = 0; ch < G::NCH; ++ch, ++cnt) {
+        for (int ch = 0; ch < G::NSRC * G::NCH; ++ch, ++cnt) {
           const int st = cnt % G::NS;
           if (!mbar_wait(k_full + st, (cnt / G::NS) & 1, abort_flag, p.err)) return false;
           tc_fence_after();
-          const int a = ch / G::NDC, dc = ch % G::NDC;
+          // source head sc (its own accumulator and query rows), tap row a, 64-channel block dc
+          const int sc = ch / G::NCH, cs = ch % G::NCH, a = cs / G::NDC, dc = cs % G::NDC;
           // Q rows shifted up by a (16 bytes per row), 64-channel block dc
-          const uint64_t qd = qdesc0 + static_cast<uint32_t>((8 * dc * G::STRIP + 16 * (G::HALO - a)) >> 4);
+          const uint64_t qd = qdesc0 + static_cast<uint32_t>((sc * G::Q_ALLOC + 8 * dc * G::STRIP + 16 * (G::HALO - a)) >> 4);
           const uint64_t kd = kdesc0 + static_cast<uint32_t>((st * G::KCHUNK) >> 4);
 #pragma unroll
           for (int kk = 0; kk < 4; ++kk)
-            mma_bf16_ss(tmem + G::C_COL, qd + (2 * kk * G::STRIP >> 4), kd + 2 * kk, idesc_c, (ch > 0 || kk > 0));
+            mma_bf16_ss(tmem + G::C_COL + 128 * sc, qd + (2 * kk * G::STRIP >> 4), kd + 2 * kk, idesc_c,
+                        (cs > 0 || kk > 0));
           mma_commit(k_empty + st);
         }
         mma_commit(c_full);
@@ -350,7 +365,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int h = it.g * CL + hr, row0 = it.qt * G::BM - G::HALO;
       mbar_wait(q_full, r & 1, abort_flag, p.err);
       float qmax = 0.f;
-      for (int c16 = st_id; c16 < G::Q_BYTES / 16; c16 += kSmThreads) {
+      // (the query tiles of the source heads lie Q_ALLOC = Q_BYTES apart)
+      static_assert(G::Q_ALLOC == G::Q_BYTES, "contiguous query tiles");
+      for (int c16 = st_id; c16 < G::NSRC * G::Q_BYTES / 16; c16 += kSmThreads) {
         const uint4 raw = *reinterpret_cast<const uint4 *>(Qs + 16 * c16);
         const __nv_bfloat162 *p2 = reinterpret_cast<const __nv_bfloat162 *>(&raw);
 #pragma unroll
@@ -366,7 +383,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       int eq = 0;
       if (qmax > 16384.f) eq = max(-60, static_cast<int>(floorf(log2f(16384.f / qmax))));
       const float qsc = exp2f(static_cast<float>(eq));
-      for (int c16 = st_id; c16 < G::Q_BYTES / 16; c16 += kSmThreads) {
+      for (int c16 = st_id; c16 < G::NSRC * G::Q_BYTES / 16; c16 += kSmThreads) {
         uint4 raw = *reinterpret_cast<const uint4 *>(Qs + 16 * c16);
         __nv_bfloat162 *p2 = reinterpret_cast<__nv_bfloat162 *>(&raw);
         uint4 o;
@@ -381,12 +398,18 @@ __global__ void __launch_bounds__(kThreads, 1)
       fence_proxy_async_smem();
       __syncwarp();
       if (lane == 0) mbar_arrive(q_ready);
-      const long long bh = static_cast<long long>(it.b) * p.H + h;
-      for (int e = st_id; e < G::UROWS * G::M; e += kSmThreads) {
-        const int rr = e / G::M, k = e % G::M, iq = row0 + rr;
-        Us[e] = (iq >= 0 && iq < L) ? p.vp[(bh * L + iq) * G::M + k] : 0.f;
+#pragma unroll 1
+      for (int sc = 0; sc < G::NSRC; ++sc) {
+        const int hs = src_head(h, sc);
+        const long long bh = static_cast<long long>(it.b) * p.H + hs;
+        float *us = Us + sc * (G::U_BYTES / 4);
+        for (int e = st_id; e < G::UROWS * G::M; e += kSmThreads) {
+          const int rr = e / G::M, k = e % G::M, iq = row0 + rr;
+          us[e] = (iq >= 0 && iq < L) ? p.vp[(bh * L + iq) * G::M + k] : 0.f;
+        }
+        if (st_id < CQ * CK)
+          th_s[((r & 1) * G::NSRC + sc) * 128 + st_id] = p.theta[static_cast<long long>(hs) * CQ * CK + st_id];
       }
-      if (st_id < CQ * CK) th_s[(r & 1) * 128 + st_id] = p.theta[static_cast<long long>(h) * CQ * CK + st_id];
       return eq;
     };
 
@@ -396,8 +419,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     int eq = 0;
     if (have) {
       eq = prepare(0, it);
-      const float *fac0 = p.fac + (static_cast<long long>(it.b) * p.H + it.g * CL + hr) * p.lpad;
-      if (st_id < G::BN) facs[(T & 1) * G::BN + st_id] = fac0[st_id];
+      const int h0 = it.g * CL + hr;
+      if (st_id < G::BN)
+#pragma unroll
+        for (int sc = 0; sc < G::NSRC; ++sc)
+          facs[sc * 2 * G::BN + st_id] = p.fac[(static_cast<long long>(it.b) * p.H + src_head(h0, sc)) * p.lpad + st_id];
       named_bar_sync(kBarAll, kSmThreads);
     }
     for (int r = 0; have; ++r) {
@@ -405,36 +431,53 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int i0 = it.qt * G::BM, qi = i0 + r_;
       const bool out_row = qi < L;
       const int n_kv = kv_tiles(it);
-      const long long bh = static_cast<long long>(it.b) * p.H + h;
-      const float *fac = p.fac + bh * p.lpad;
       const bool more = item_at(r + 1, nx);
-      const float *fac_nx = more ? p.fac + (static_cast<long long>(nx.b) * p.H + nx.g * CL + hr) * p.lpad : fac;
-      const float *th = th_s + (r & 1) * 128;
+      const int h_nx = nx.g * CL + hr;
+      // column factors of source s for the key tile after t (this item's or the next item's first)
+      auto fac_next = [&](int sc, int t) -> float {
+        if (t + 1 < n_kv) return p.fac[(static_cast<long long>(it.b) * p.H + src_head(h, sc)) * p.lpad + (t + 1) * G::BN + st_id];
+        if (more) return p.fac[(static_cast<long long>(nx.b) * p.H + src_head(h_nx, sc)) * p.lpad + st_id];
+        return 0.f;
+      };
       const float qinv = exp2f(static_cast<float>(-eq));
+      // pre-softmax mixing weights of the sources: w[g][destination][source]
+      float wmix[G::NSRC];
+#pragma unroll
+      for (int sc = 0; sc < G::NSRC; ++sc) wmix[sc] = G::NSRC == 2 ? p.w[(h >> 1) * 4 + (h & 1) * 2 + sc] : 1.f;
       float m_run = -INFINITY, l_run = 0.f;
       for (int t = 0; t < n_kv; ++t, ++T) {
         const int j0 = t * G::BN;
         // next key tile's column factors (stored before this tile's barrier, read after it)
-        float fnext = 0.f;
-        if (st_id < G::BN) fnext = t + 1 < n_kv ? fac[j0 + G::BN + st_id] : (more ? fac_nx[st_id] : 0.f);
-        const float4 *f4 = reinterpret_cast<const float4 *>(facs + (T & 1) * G::BN + cb);
+        float fnext[G::NSRC];
+#pragma unroll
+        for (int sc = 0; sc < G::NSRC; ++sc) fnext[sc] = st_id < G::BN ? fac_next(sc, t) : 0.f;
         mbar_wait(c_full, T & 1, abort_flag, p.err);
         tc_fence_after();
+        // C' = sum over source heads of w * (C_s x its column factors); one source without mixing
         float cv[G::HALF];
 #pragma unroll
-        for (int c0 = 0; c0 < G::HALF; c0 += 32) {
-          uint32_t u32[32];
-          tmem_ld32(tl + G::C_COL + cb + c0, u32);
-          float4 f[8];
+        for (int sc = 0; sc < G::NSRC; ++sc) {
+          const float4 *f4 = reinterpret_cast<const float4 *>(facs + (sc * 2 + (T & 1)) * G::BN + cb);
 #pragma unroll
-          for (int i = 0; i < 8; ++i) f[i] = f4[c0 / 4 + i];
-          tmem_wait_ld();
+          for (int c0 = 0; c0 < G::HALF; c0 += 32) {
+            uint32_t u32[32];
+            tmem_ld32(tl + G::C_COL + 128 * sc + cb + c0, u32);
+            float4 f[8];
 #pragma unroll
-          for (int i = 0; i < 8; ++i) {
-            cv[c0 + 4 * i] = __uint_as_float(u32[4 * i]) * f[i].x;
-            cv[c0 + 4 * i + 1] = __uint_as_float(u32[4 * i + 1]) * f[i].y;
-            cv[c0 + 4 * i + 2] = __uint_as_float(u32[4 * i + 2]) * f[i].z;
-            cv[c0 + 4 * i + 3] = __uint_as_float(u32[4 * i + 3]) * f[i].w;
+            for (int i = 0; i < 8; ++i) {
+              f[i] = f4[c0 / 4 + i];
+              if (G::NSRC == 2) { f[i].x *= wmix[sc]; f[i].y *= wmix[sc]; f[i].z *= wmix[sc]; f[i].w *= wmix[sc]; }
+            }
+            tmem_wait_ld();
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+#pragma unroll
+              for (int e = 0; e < 4; ++e) {
+                const float fe = e == 0 ? f[i].x : e == 1 ? f[i].y : e == 2 ? f[i].z : f[i].w;
+                const float x = __uint_as_float(u32[4 * i + e]) * fe;
+                cv[c0 + 4 * i + e] = sc == 0 ? x : cv[c0 + 4 * i + e] + x;
+              }
+            }
           }
         }
         tc_fence_before();
@@ -454,14 +497,18 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
           for (int dd = 0; dd < G::W; ++dd) acc[dd] = 0.f;
 #pragma unroll
+          for (int sc = 0; sc < G::NSRC; ++sc)
+#pragma unroll
           for (int a = 0; a < CQ; ++a) {
-            const float *vrow = Us + (r_ + G::HALO - a) * G::M;  // rows before query 0 are zero
+            // rows before query 0 are zero; the source's taps carry its mixing weight
+            const float *vrow = Us + sc * (G::U_BYTES / 4) + (r_ + G::HALO - a) * G::M;
+            const float *th = th_s + ((r & 1) * G::NSRC + sc) * 128;
             float vr[G::M];
 #pragma unroll
             for (int m = 0; m < G::M; ++m) vr[m] = vrow[m];
 #pragma unroll
             for (int tp = 0; tp < CK; ++tp) {
-              const float thv = th[a * CK + tp];
+              const float thv = th[a * CK + tp] * wmix[sc];
 #pragma unroll
               for (int dd = 0; dd < G::W; ++dd) {
                 const int m = dd - a + tp - G::C;
@@ -487,7 +534,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         float *rmx = red + (T & 1) * 2 * G::BM;
         rmx[wg * G::BM + r_] = out_row ? tree_max<G::HALF>(cv) : -INFINITY;
-        if (st_id < G::BN) facs[((T + 1) & 1) * G::BN + st_id] = fnext;
+        if (st_id < G::BN)
+#pragma unroll
+          for (int sc = 0; sc < G::NSRC; ++sc) facs[(sc * 2 + ((T + 1) & 1)) * G::BN + st_id] = fnext[sc];
         named_bar_sync(kBarAll, kSmThreads);
         const float mt = fmaxf(rmx[r_], rmx[G::BM + r_]);
         const float m_new = fmaxf(m_run, mt);
@@ -717,7 +766,7 @@ size_t align256(size_t x) { return (x + 255) / 256 * 256; }
 bool attn_kq_supported(const AttnArgs &a) {
   if (a.dtype != 1 || (a.d != 64 && a.d != 128)) return false;
   if ((a.kq != 1 && a.kq != 3) || a.cq != 6 || a.ck != 11) return false;
-  if (!(a.hp == 0 || (a.hp == 2 && a.ch == 2))) return false;
+  if (!(a.hp == 0 || ((a.hp == 1 || a.hp == 2) && a.ch == 2))) return false;
   if (a.B > 65535 || a.H > 65535 || (a.L + 127) / 128 > 65535) return false;
   const uintptr_t al = reinterpret_cast<uintptr_t>(a.q) | reinterpret_cast<uintptr_t>(a.k) |
                        reinterpret_cast<uintptr_t>(a.v) | reinterpret_cast<uintptr_t>(a.out);
@@ -760,12 +809,19 @@ cudaError_t launch_attn_kq(const AttnArgs &a, const GnArgs *gn, void *ws) {
   float *xg = reinterpret_cast<float *>(reinterpret_cast<char *>(pa.vp) + align256(BHL * pa.M * 4));
   cudaError_t e = launch_kq_prep(pa, a.stream);
   if (e != cudaSuccess) return e;
-  const bool post = a.hp == 2;
-  if (a.d == 128)
-    return post ? (pa.exact ? launch_kq_one<128, 6, 11, 2, true>(a, gn, pa, xg) : launch_kq_one<128, 6, 11, 2, false>(a, gn, pa, xg))
-                : (pa.exact ? launch_kq_one<128, 6, 11, 0, true>(a, gn, pa, xg) : launch_kq_one<128, 6, 11, 0, false>(a, gn, pa, xg));
-  return post ? (pa.exact ? launch_kq_one<64, 6, 11, 2, true>(a, gn, pa, xg) : launch_kq_one<64, 6, 11, 2, false>(a, gn, pa, xg))
-              : (pa.exact ? launch_kq_one<64, 6, 11, 0, true>(a, gn, pa, xg) : launch_kq_one<64, 6, 11, 0, false>(a, gn, pa, xg));
+  // MIX: 0 no head mixing, 1 pre-softmax mixing (both C of a group per CTA), 2 post-softmax
+  auto go = [&](auto d_tag, auto mix_tag) -> cudaError_t {
+    constexpr int DD = decltype(d_tag)::value, MX = decltype(mix_tag)::value;
+    return pa.exact ? launch_kq_one<DD, 6, 11, MX, true>(a, gn, pa, xg)
+                    : launch_kq_one<DD, 6, 11, MX, false>(a, gn, pa, xg);
+  };
+  using D64 = std::integral_constant<int, 64>;
+  using D128 = std::integral_constant<int, 128>;
+  using M0 = std::integral_constant<int, 0>;
+  using M1 = std::integral_constant<int, 1>;
+  using M2 = std::integral_constant<int, 2>;
+  if (a.d == 128) return a.hp == 2 ? go(D128{}, M2{}) : a.hp == 1 ? go(D128{}, M1{}) : go(D128{}, M0{});
+  return a.hp == 2 ? go(D64{}, M2{}) : a.hp == 1 ? go(D64{}, M1{}) : go(D64{}, M0{});
 }
 
 }  // namespace mta

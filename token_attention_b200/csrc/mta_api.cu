@@ -63,7 +63,7 @@ bool kq_shape_ok(const mta_cfg *c) {
   return c->dtype == MTA_BF16 && (c->d == 64 || c->d == 128) &&
          (c->kq_place == MTA_PRE || c->kq_place == MTA_PRE_EXACT) &&
          c->c_q == 6 && c->c_k == 11 &&
-         (c->head_place == MTA_OFF || (c->head_place == MTA_POST && c->c_h == 2));
+         (c->head_place == MTA_OFF || ((c->head_place == MTA_PRE || c->head_place == MTA_POST) && c->c_h == 2));
 }
 
 size_t kq_bytes(const mta_cfg *c) {
