@@ -47,6 +47,13 @@ Readings where the pages leave a step open (all listed in the design doc):
   * Sigmoid scalar gate (section 3.3: "a learned sigmoid scalar gate, a bounded
     multiplier"): one learned logit g_h per head; the normalised output of head h
     is multiplied by sigmoid(g_h) in place of the depth scale.
+  * Post-softmax key-query convolution (section 3.1 applies the kernel "before
+    or after" the softmax; section 4 uses both by default, and only the
+    pre-softmax formula is printed): its own per-head kernel theta_post of the
+    same c_q x c_k shape convolves the attention weights A (already 0 at future
+    keys), then Mask_0 zeroes the future keys again, so
+    A' = Mask_0(Conv2d_theta_post(A)); no renormalisation.  With head mixing
+    after the softmax, the convolution comes first, as before the softmax.
 """
 from __future__ import annotations
 
@@ -55,7 +62,7 @@ import numpy as np
 OFF, PRE, POST, PRE_EXACT = 0, 1, 2, 3
 
 __all__ = ["OFF", "PRE", "POST", "PRE_EXACT", "attention_logits", "mask_zero", "key_query_conv",
-           "key_query_conv_exact", "sigmoid_gate",
+           "key_query_conv_exact", "sigmoid_gate", "post_softmax_conv",
            "head_mix", "mask_neg_inf", "softmax_rows", "mta_attention_group",
            "mta_attention", "mta_attention_rows", "group_norm_scale", "mta_layer",
            "mta_layer_rows"]
@@ -156,11 +163,20 @@ def softmax_rows(c: np.ndarray) -> np.ndarray:
     return e / np.sum(e, axis=-1, keepdims=True)
 
 
-def mta_attention_group(q_rows, k, v, theta, w, qpos, scale, kq_place, head_place):
+def post_softmax_conv(attn: np.ndarray, theta_post: np.ndarray, qpos: np.ndarray) -> np.ndarray:
+    """Key-query convolution of the attention weights after the softmax, then
+    Mask_0 again  [MTA-3.1]: A' = Mask_0(Conv2d_theta_post(A)).  attn [c_h, R, L]
+    (rows are the consecutive queries qpos), theta_post [c_h, c_q, c_k]."""
+    return mask_zero(key_query_conv(attn, theta_post), qpos)
+
+
+def mta_attention_group(q_rows, k, v, theta, w, qpos, scale, kq_place, head_place,
+                        theta_post=None):
     """MTA attention of one head group for the query rows `qpos` (consecutive).
 
     q_rows [c_h, R, d] (queries at positions qpos), k, v [c_h, L, d],
-    theta [c_h, c_q, c_k], w [c_h, c_h].  Returns [c_h, R, d] float64.
+    theta [c_h, c_q, c_k], w [c_h, c_h], theta_post [c_h, c_q, c_k] or None (no
+    post-softmax convolution).  Returns [c_h, R, d] float64.
     Steps in the pages' order [MTA-2, MTA-3.1, MTA-3.2, MTA-3.3]."""
     qpos = np.asarray(qpos)
     a_hat = attention_logits(q_rows, k, scale)
@@ -173,6 +189,8 @@ def mta_attention_group(q_rows, k, v, theta, w, qpos, scale, kq_place, head_plac
     if head_place == PRE:
         c = head_mix(c, w)
     attn = softmax_rows(mask_neg_inf(c, qpos))
+    if theta_post is not None:
+        attn = post_softmax_conv(attn, theta_post, qpos)
     if head_place == POST:
         attn = head_mix(attn, w)
     return np.matmul(attn, v.astype(np.float64))        # head r: A_r V_r
@@ -187,13 +205,20 @@ def _group(x: np.ndarray, b: int, g: int, ch: int) -> np.ndarray:
     return np.ascontiguousarray(x[b, :, g * ch:(g + 1) * ch, :].transpose(1, 0, 2))
 
 
+def _sel(x, idx):
+    """x[idx], or None for a parameter that is absent (its step is off)."""
+    return None if x is None else x[idx]
+
+
 def _default_scale(d: int, scale) -> float:
     return 1.0 / np.sqrt(d) if not scale else float(scale)
 
 
-def mta_attention(q, k, v, theta, w, c_h, kq_place=PRE, head_place=POST, scale=None):
+def mta_attention(q, k, v, theta, w, c_h, kq_place=PRE, head_place=POST, scale=None,
+                  theta_post=None):
     """Full MTA attention.  q, k, v [B][L][H][d]; theta [H][c_q][c_k];
-    w [H/c_h][c_h][c_h].  Returns out [B][L][H][d] float64."""
+    w [H/c_h][c_h][c_h]; theta_post [H][c_q][c_k] or None.
+    Returns out [B][L][H][d] float64."""
     B, L, H, d = q.shape
     s = _default_scale(d, scale)
     out = np.zeros((B, L, H, d), np.float64)
@@ -202,31 +227,36 @@ def mta_attention(q, k, v, theta, w, c_h, kq_place=PRE, head_place=POST, scale=N
         for g in range(H // c_h):
             hs = slice(g * c_h, (g + 1) * c_h)
             og = mta_attention_group(_group(q, b, g, c_h), _group(k, b, g, c_h),
-                                     _group(v, b, g, c_h), theta[hs], w[g], qpos, s,
-                                     kq_place, head_place)
+                                     _group(v, b, g, c_h), _sel(theta, hs), _sel(w, g),
+                                     qpos, s, kq_place, head_place,
+                                     None if theta_post is None else theta_post[hs])
             out[b, :, hs, :] = og.transpose(1, 0, 2)
     return out
 
 
 def mta_attention_rows(q, k, v, theta, w, c_h, rows, kq_place=PRE, head_place=POST,
-                       scale=None):
+                       scale=None, theta_post=None):
     """MTA attention output at selected tokens only.
 
     rows: sequence of (b, i).  Returns [n, H, d] float64.  Each row is computed
-    from the window of the c_q queries ending at i (the only rows the
-    convolution reads), with exactly the same steps as mta_attention."""
+    from the window of queries ending at i that the convolutions read (c_q rows,
+    2 c_q - 1 with the post-softmax convolution), with exactly the same steps as
+    mta_attention."""
     B, L, H, d = q.shape
-    cq = theta.shape[1]
+    cq = 1 if theta is None else theta.shape[1]
+    back = cq - 1 + (0 if theta_post is None else theta_post.shape[1] - 1)
     s = _default_scale(d, scale)
     out = np.zeros((len(rows), H, d), np.float64)
     for n, (b, i) in enumerate(rows):
-        lo = max(0, i - cq + 1)
+        lo = max(0, i - back)
         qpos = np.arange(lo, i + 1)
         for g in range(H // c_h):
             hs = slice(g * c_h, (g + 1) * c_h)
             qg = np.ascontiguousarray(q[b, lo:i + 1, hs, :].transpose(1, 0, 2))
             og = mta_attention_group(qg, _group(k, b, g, c_h), _group(v, b, g, c_h),
-                                     theta[hs], w[g], qpos, s, kq_place, head_place)
+                                     _sel(theta, hs), _sel(w, g), qpos, s, kq_place,
+                                     head_place,
+                                     None if theta_post is None else theta_post[hs])
             out[n, hs, :] = og[:, -1, :]
     return out
 
@@ -253,20 +283,20 @@ def _split_qkv(qkv, H, d):
 
 
 def mta_layer(x, wqkv, theta, w, gamma, beta, eps, lam, wo, H, c_h,
-              kq_place=PRE, head_place=POST):
+              kq_place=PRE, head_place=POST, theta_post=None):
     """Full MTA attention layer  [MTA-2, MTA-3.x, bycloud].
     x [B][L][D]; wqkv [3D][D]; wo [D][D].  Returns out [B][L][D] float64."""
     B, L, D = x.shape
     d = D // H
     qkv = np.matmul(x.astype(np.float64), wqkv.astype(np.float64).T)      # x W^T
     q, k, v = _split_qkv(qkv, H, d)
-    o = mta_attention(q, k, v, theta, w, c_h, kq_place, head_place)
+    o = mta_attention(q, k, v, theta, w, c_h, kq_place, head_place, theta_post=theta_post)
     y = group_norm_scale(o, gamma, beta, eps, lam).reshape(B, L, D)
     return np.matmul(y, wo.astype(np.float64).T)
 
 
 def mta_layer_rows(x, wqkv, theta, w, gamma, beta, eps, lam, wo, H, c_h, rows,
-                   kq_place=PRE, head_place=POST):
+                   kq_place=PRE, head_place=POST, theta_post=None):
     """mta_layer at selected tokens (b, i) only: K, V of the token's batch in
     full, queries of the convolution window.  Returns [n, D] float64."""
     B, L, D = x.shape
@@ -280,7 +310,7 @@ def mta_layer_rows(x, wqkv, theta, w, gamma, beta, eps, lam, wo, H, c_h, rows,
             cache = {b: _split_qkv(qkv_b, H, d)}
         q, k, v = cache[b]
         o = mta_attention_rows(q[None], k[None], v[None], theta, w, c_h, [(0, i)],
-                               kq_place, head_place)[0]                     # [H, d]
+                               kq_place, head_place, theta_post=theta_post)[0]  # [H, d]
         y = group_norm_scale(o, gamma, beta, eps, lam).reshape(D)
         out[n] = y @ wo.astype(np.float64).T
     return out

@@ -444,3 +444,165 @@ def test_gated_group_norm_invariants():
     var = o.var(-1)
     np.testing.assert_allclose(y.std(-1), scipy.special.expit(g)[None, :] * np.sqrt(var / (var + eps)),
                                rtol=1e-12)
+
+
+# ----------------------------------------------------------------------------
+# post-softmax key-query convolution (section 3.1: the kernel acts before or
+# after the softmax; after it, it combines attention weights additively)
+# ----------------------------------------------------------------------------
+
+def _softmax_weights(q, k, scale):
+    """Causal softmax weights of one head by torch's library routine.  q,k [L,d]."""
+    L = q.shape[0]
+    lg = torch.from_numpy(scale * (q @ k.T))
+    lg = lg.masked_fill(torch.triu(torch.ones(L, L, dtype=torch.bool), 1), float("-inf"))
+    return torch.softmax(lg, dim=1).numpy()
+
+
+def test_post_conv_identity_is_no_op(qkv):
+    """theta_post = delta at (0,0) leaves the attention unchanged."""
+    q, k, v = qkv
+    H = q.shape[2]
+    th = rand((H, 3, 5), 61, 0.3)
+    w = rand((H // 2, 2, 2), 62)
+    for hp in (O.OFF, O.PRE, O.POST):
+        base = O.mta_attention(q, k, v, th, w, 2, O.PRE, hp)
+        ident = O.mta_attention(q, k, v, th, w, 2, O.PRE, hp,
+                                theta_post=delta_theta(H, 3, 5, 0, 2))
+        np.testing.assert_allclose(ident, base, rtol=0, atol=1e-13)
+
+
+@pytest.mark.parametrize("a", [1, 3])
+def test_post_conv_query_shift_moves_output_rows(qkv, a):
+    """theta_post = delta at (a, 0): A'[i] = A[i-a] (row i-a never reaches a key
+    after i, so the final Mask_0 removes nothing), hence the output at i is the
+    output the plain map gives at i-a, and 0 for i < a; with post-softmax mixing
+    the mixed rows move the same way."""
+    q, k, v = qkv
+    H = q.shape[2]
+    th = rand((H, 3, 5), 63, 0.3)
+    w = rand((H // 2, 2, 2), 64)
+    for hp in (O.OFF, O.POST):
+        base = O.mta_attention(q, k, v, th, w, 2, O.PRE, hp)
+        out = O.mta_attention(q, k, v, th, w, 2, O.PRE, hp, theta_post=delta_theta(H, 4, 5, a, 2))
+        np.testing.assert_allclose(out[:, a:], base[:, :-a], rtol=0, atol=1e-13)
+        assert np.all(out[:, :a] == 0.0)
+
+
+@pytest.mark.parametrize("boff", [-2, 1, 2])
+def test_post_conv_key_shift_closed_form(qkv, boff):
+    """theta_post = delta at (0, b): A'[i][j] = A[i][j-b] for keys j <= i, so
+    out[i] = sum over keys j' with 0 <= j'+b <= i of A[i][j'] v[j'+b]: the weights
+    move b keys later (b > 0: the last b weights of the row fall past the query
+    and are dropped) or |b| keys earlier (b < 0: the first |b| fall off the
+    sequence).  A from torch's softmax, the sum by loops."""
+    q, k, v = qkv
+    B, L, H, d = q.shape
+    ck = 5
+    th_post = delta_theta(H, 2, ck, 0, ck // 2 + boff)
+    out = O.mta_attention(q, k, v, None, None, 1, O.OFF, O.OFF, theta_post=th_post)
+    for b in range(B):
+        for h in range(H):
+            A = _softmax_weights(q[b, :, h], k[b, :, h], 1 / np.sqrt(d))
+            ref = np.zeros((L, d))
+            for i in range(L):
+                for jp in range(L):
+                    if 0 <= jp + boff <= i:
+                        ref[i] += A[i, jp] * v[b, jp + boff, h]
+            np.testing.assert_allclose(out[b, :, h], ref, rtol=0, atol=1e-12)
+
+
+def test_post_conv_is_linear_in_theta_post(qkv):
+    """After the softmax the convolution combines weights additively (section 3.1):
+    the output is linear in theta_post."""
+    q, k, v = qkv
+    H = q.shape[2]
+    th = rand((H, 3, 5), 65, 0.3)
+    w = rand((H // 2, 2, 2), 66)
+    t1, t2 = rand((H, 3, 5), 67), rand((H, 3, 5), 68)
+    f = lambda tp: O.mta_attention(q, k, v, th, w, 2, O.PRE, O.POST, theta_post=tp)
+    np.testing.assert_allclose(f(t1 + t2), f(t1) + f(t2), rtol=0, atol=1e-11)
+    np.testing.assert_allclose(f(-2.5 * t1), -2.5 * f(t1), rtol=0, atol=1e-11)
+
+
+@pytest.mark.parametrize("head_place", [O.OFF, O.PRE, O.POST])
+def test_post_conv_causality_bit_exact(qkv, head_place):
+    """With the convolution on both sides of the softmax, perturbing position t
+    still leaves outputs at i < t bit-identical."""
+    q, k, v = qkv
+    H = q.shape[2]
+    th = rand((H, 3, 5), 69, 0.3)
+    tp = rand((H, 3, 5), 70, 0.3)
+    w = rand((H // 2, 2, 2), 71, 0.5)
+    base = O.mta_attention(q, k, v, th, w, 2, O.PRE, head_place, theta_post=tp)
+    t = 11
+    q2, k2, v2 = q.copy(), k.copy(), v.copy()
+    q2[:, t:] += rand(q2[:, t:].shape, 72)
+    k2[:, t:] += rand(k2[:, t:].shape, 73)
+    v2[:, t:] += rand(v2[:, t:].shape, 74)
+    pert = O.mta_attention(q2, k2, v2, th, w, 2, O.PRE, head_place, theta_post=tp)
+    assert np.array_equal(base[:, :t], pert[:, :t])
+    assert not np.allclose(base[:, t:], pert[:, t:])
+
+
+def test_both_sides_bruteforce_tiny():
+    """Pure-Python restatement on a tiny case: pre-softmax convolution of the
+    Mask_0 logits, softmax over past keys, post-softmax convolution of the weights
+    with the future keys zeroed again, post-softmax head mixing, times the
+    destination head's V; every sum an explicit loop."""
+    L, H, d, cq, ck, ch = 7, 2, 3, 3, 3, 2
+    c = ck // 2
+    q, k, v = rand((1, L, H, d), 75), rand((1, L, H, d), 76), rand((1, L, H, d), 77)
+    th, tp = rand((H, cq, ck), 78, 0.5), rand((H, cq, ck), 79, 0.5)
+    w = rand((1, ch, ch), 80)
+    s = 1 / np.sqrt(d)
+
+    def m0(h, i, j):
+        if i < 0 or j < 0 or j >= L or j > i:
+            return 0.0
+        return s * sum(q[0, i, h, e] * k[0, j, h, e] for e in range(d))
+
+    A = np.zeros((H, L, L))
+    for h in range(H):
+        for i in range(L):
+            C = [sum(th[h, a, t] * m0(h, i - a, j - (t - c)) for a in range(cq) for t in range(ck))
+                 for j in range(i + 1)]
+            mx = max(C)
+            e = [np.exp(x - mx) for x in C]
+            for j in range(i + 1):
+                A[h, i, j] = e[j] / sum(e)
+
+    def a_at(h, i, j):
+        return A[h, i, j] if 0 <= i < L and 0 <= j < L else 0.0
+
+    Ap = np.zeros((H, L, L))
+    for h in range(H):
+        for i in range(L):
+            for j in range(i + 1):
+                Ap[h, i, j] = sum(tp[h, a, t] * a_at(h, i - a, j - (t - c))
+                                  for a in range(cq) for t in range(ck))
+    ref = np.zeros((1, L, H, d))
+    for r in range(H):
+        for i in range(L):
+            for j in range(L):
+                wt = sum(w[0, r, s_] * Ap[s_, i, j] for s_ in range(H))
+                ref[0, i, r] += wt * v[0, j, r]
+    out = O.mta_attention(q, k, v, th, w, ch, O.PRE, O.POST, theta_post=tp)
+    np.testing.assert_allclose(out, ref, rtol=0, atol=1e-12)
+
+
+def test_post_conv_rows_match_full(qkv):
+    """The row-wise oracle widens its query window to 2 c_q - 1 rows when the
+    convolution also acts after the softmax."""
+    q, k, v = qkv
+    H = q.shape[2]
+    th = rand((H, 3, 5), 81, 0.3)
+    tp = rand((H, 3, 5), 82, 0.3)
+    w = rand((H // 2, 2, 2), 83)
+    rows = [(0, 0), (0, 3), (1, 4), (1, 9), (0, 22)]
+    for kq in (O.PRE, O.OFF):
+        for hp in (O.PRE, O.POST, O.OFF):
+            full = O.mta_attention(q, k, v, th, w, 2, kq, hp, theta_post=tp)
+            part = O.mta_attention_rows(q, k, v, th, w, 2, rows, kq, hp, theta_post=tp)
+            for n, (b, i) in enumerate(rows):
+                np.testing.assert_allclose(part[n], full[b, i], rtol=0, atol=1e-12)
