@@ -23,7 +23,7 @@
 // Every value written for key or query j depends on inputs at positions <= j + c
 // only, and Kt_a[j] is used only for queries i >= j + W > j + c: the path stays
 // exactly causal.  One CTA per (key tile, head, batch); the key rows with their
-// halo are staged in shared memory as fp32.
+// halo are staged in shared memory as bf16.
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 #include <math.h>
@@ -36,7 +36,7 @@ namespace {
 
 constexpr int kPrepThreads = 256;
 constexpr int kTile = 128;
-constexpr int kRun = 16;  // consecutive keys one thread convolves from a register window
+constexpr int kRun = 8;   // consecutive keys one thread convolves from a register window
 
 template <int D, int CQ, int CK, bool EXACT>
 struct PrepGeo {
@@ -47,8 +47,8 @@ struct PrepGeo {
   // keys j0-LO .. : the Kt window reaches kTile-1+C past j0, a warp's 32-key tile of
   // dot products 16*7+31+OFF-LO
   static constexpr int ROWS = (kTile + LO + C) > (16 * 7 + 32 + OFF) ? (kTile + LO + C) : (16 * 7 + 32 + OFF);
-  static constexpr int KSTR = D + 8;                  // staged row stride (floats): fewer bank conflicts
-  static constexpr int SMEM = ROWS * KSTR * 4;
+  static constexpr int KSTR = D + 8;                  // staged row stride (bf16): conflict-free fragments
+  static constexpr int SMEM = ROWS * KSTR * 2;
   static_assert(M - 1 + 16 <= 32, "past dot products of a 16-row block span 32 keys");
 };
 
@@ -62,18 +62,17 @@ __device__ __forceinline__ void mma_m16n8k16_bf16(float (&c)[4], const uint32_t 
       : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
 }
 
-// two floats that are bf16 values, packed exactly (low half = first)
-__device__ __forceinline__ uint32_t pack2_bf16(float lo, float hi) {
-  const __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
-  return *reinterpret_cast<const uint32_t *>(&v);
+// two bf16 values (low half = first) as floats
+__device__ __forceinline__ float2 bf16x2_to_float2(uint32_t v) {
+  return make_float2(__uint_as_float(v << 16), __uint_as_float(v & 0xffff0000u));
 }
 
 __device__ __forceinline__ float pow2i(int e) { return __int_as_float((127 + e) << 23); }  // |e| <= 126
 
 template <int D, int CQ, int CK, bool EXACT>
-__global__ void __launch_bounds__(kPrepThreads) kq_prep_kernel(KqPrepArgs p) {
+__global__ void __launch_bounds__(kPrepThreads, 3) kq_prep_kernel(KqPrepArgs p) {
   using G = PrepGeo<D, CQ, CK, EXACT>;
-  extern __shared__ float ks[];  // [ROWS][KSTR] fp32, row r = key j0 - LO + r
+  extern __shared__ uint32_t ks[];  // [ROWS][KSTR/2] bf16 pairs, row r = key j0 - LO + r
   __shared__ float rmax[G::ROWS];
   __shared__ int es[kTile];
   __shared__ float th[CQ * CK];
@@ -86,25 +85,20 @@ __global__ void __launch_bounds__(kPrepThreads) kq_prep_kernel(KqPrepArgs p) {
   for (int i = tid; i < CQ * CK; i += kPrepThreads) th[i] = p.theta[static_cast<long long>(h) * CQ * CK + i];
   for (int i = tid; i < G::ROWS; i += kPrepThreads) rmax[i] = 0.f;
   __syncthreads();
-  // stage key rows (zero outside [0, L)) and their max |k|
+  // stage key rows as bf16 (zero outside [0, L)) and their max |k|
   for (int i = tid; i < G::ROWS * (D / 8); i += kPrepThreads) {
     const int r = i / (D / 8), e8 = (i % (D / 8)) * 8, key = j0 - G::LO + r;
-    float v[8];
-    if (key >= 0 && key < L) {
-      const uint4 raw = *reinterpret_cast<const uint4 *>(kb + (static_cast<long long>(b) * L + key) * p.rs +
-                                                         static_cast<long long>(h) * D + e8);
-      const __nv_bfloat162 *p2 = reinterpret_cast<const __nv_bfloat162 *>(&raw);
-#pragma unroll
-      for (int u = 0; u < 4; ++u) { v[2 * u] = __low2float(p2[u]); v[2 * u + 1] = __high2float(p2[u]); }
-    } else {
-#pragma unroll
-      for (int u = 0; u < 8; ++u) v[u] = 0.f;
-    }
+    uint4 raw = make_uint4(0u, 0u, 0u, 0u);
+    if (key >= 0 && key < L)
+      raw = *reinterpret_cast<const uint4 *>(kb + (static_cast<long long>(b) * L + key) * p.rs +
+                                             static_cast<long long>(h) * D + e8);
+    *reinterpret_cast<uint4 *>(ks + (r * G::KSTR + e8) / 2) = raw;
+    const uint32_t wds[4] = {raw.x, raw.y, raw.z, raw.w};
     float m = 0.f;
 #pragma unroll
-    for (int u = 0; u < 8; ++u) {
-      ks[r * G::KSTR + e8 + u] = v[u];
-      m = fmaxf(m, fabsf(v[u]));
+    for (int u = 0; u < 4; ++u) {
+      const float2 f = bf16x2_to_float2(wds[u]);
+      m = fmaxf(m, fmaxf(fabsf(f.x), fabsf(f.y)));
     }
     atomicMax(reinterpret_cast<int *>(rmax + r), __float_as_int(m));  // non-negative floats order as ints
   }
@@ -142,7 +136,7 @@ __global__ void __launch_bounds__(kPrepThreads) kq_prep_kernel(KqPrepArgs p) {
     float2 win[kRun + 2 * G::C];  // keys j0+jr-c .. j0+jr+kRun-1+c
 #pragma unroll
     for (int w = 0; w < kRun + 2 * G::C; ++w)
-      win[w] = *reinterpret_cast<const float2 *>(ks + (jr + w + G::LO - G::C) * G::KSTR + e2);
+      win[w] = bf16x2_to_float2(ks[((jr + w + G::LO - G::C) * G::KSTR + e2) / 2]);
     float scu[kRun];
 #pragma unroll
     for (int u = 0; u < kRun; ++u) scu[u] = pow2i(es[jr + u]);
@@ -200,10 +194,8 @@ __global__ void __launch_bounds__(kPrepThreads) kq_prep_kernel(KqPrepArgs p) {
     a[3] = qok[1] ? q32[1][c0 / 2 + 4] : 0u;
 #pragma unroll
     for (int nt = 0; nt < 4; ++nt) {
-      const float *kr = ks + (krow0 + 8 * nt + g) * G::KSTR + c0;
-      const float2 lo = *reinterpret_cast<const float2 *>(kr);
-      const float2 hi = *reinterpret_cast<const float2 *>(kr + 8);
-      mma_m16n8k16_bf16(acc[nt], a, pack2_bf16(lo.x, lo.y), pack2_bf16(hi.x, hi.y));
+      const uint32_t *kr = ks + ((krow0 + 8 * nt + g) * G::KSTR + c0) / 2;
+      mma_m16n8k16_bf16(acc[nt], a, kr[0], kr[4]);
     }
   }
   // acc[nt][u]: row i0 + g + 8*(u/2), key column kk = 8*nt + 2*tq + (u&1); m = row - key
