@@ -52,11 +52,12 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 def flops(wl: synth.Workload) -> dict:
     """Algorithmic flops of one step.  Per causal (query, key) pair and head:
     F_std = 4d (Q K^T and A V), F_mta = F_std + 2 c_q c_k + 2 c_h
-    (the key-query convolution and the head mix).  Layer adds 2 B L D 4D
+    (the key-query convolution and the head mix), plus 2 c_q c_k more when the
+    convolution also acts after the softmax.  Layer adds 2 B L D 4D
     (QKV and output projections)."""
     P = wl.causal_pairs
     f_std = 4 * wl.d * P
-    conv = (2 * wl.c_q * wl.c_k if wl.kq_place else 0) * P
+    conv = 2 * wl.c_q * wl.c_k * ((1 if wl.kq_place else 0) + (1 if wl.kq_post else 0)) * P
     mix = (2 * wl.c_h if wl.head_place else 0) * P
     gemm = 2 * wl.B * wl.L * wl.D * 4 * wl.D if wl.layer else 0
     return {"std": f_std + gemm, "mta": f_std + conv + mix + gemm, "conv": conv, "gemm": gemm,
@@ -67,7 +68,7 @@ def uses_contraction(wl: synth.Workload) -> bool:
     """Whether the library's default path runs the contraction kernel (with its
     prepass) for this workload."""
     return (wl.dtype == "bf16" and wl.d in (64, 128) and wl.kq_place == synth.PRE
-            and (wl.c_q, wl.c_k) == (6, 11)
+            and not wl.kq_post and (wl.c_q, wl.c_k) == (6, 11)
             and (wl.head_place == synth.OFF or wl.c_h == 2))
 
 
@@ -84,14 +85,20 @@ def contraction_tensor_flops(wl: synth.Workload) -> float:
     return tiles * 2.0 * 128 * 128 * (nsrc * wl.c_q * wl.d + nv * wl.d)
 
 
+def uses_direct_tc(wl: synth.Workload) -> bool:
+    """Whether the default path runs the direct tensor-core kernel."""
+    return (not uses_contraction(wl) and wl.dtype == "bf16" and wl.d in (64, 128)
+            and not wl.kq_post and (wl.c_h == 2 or wl.head_place == synth.OFF)
+            and (wl.kq_place == synth.OFF or (wl.c_q, wl.c_k) == (6, 11)))
+
+
 def launches_per_step(wl: synth.Workload) -> int:
     """Kernels of this library one step launches: the attention kernel (and the
     prepass of the contraction kernel); a layer adds the two projection GEMMs,
     and the stand-alone group norm when the attention runs on the CUDA-core
     kernel."""
     kq = uses_contraction(wl)
-    tc = (wl.dtype == "bf16" and wl.d in (64, 128) and (wl.c_h == 2 or wl.head_place == synth.OFF)
-          and (wl.kq_place == synth.OFF or (wl.c_q, wl.c_k) == (6, 11)))
+    tc = uses_direct_tc(wl)
     attn = 2 if kq else 1  # the contraction kernel runs after its prepass
     if not wl.layer:
         return attn
@@ -217,12 +224,13 @@ def make_sets(wl, dev, n_sets):
         w = synth.shrink(wl, seed=wl.seed + 100 * s)
         if wl.layer:
             inp = synth.make_layer_inputs(w)
-            sets.append({k: to(inp[k], "bf16" if k in ("x", "wqkv", "wo") else "f32")
-                         for k in ("x", "wqkv", "wo", "theta", "w", "gamma", "beta")})
+            keys = ("x", "wqkv", "wo", "theta", "w", "gamma", "beta")
+            sets.append({k: to(inp[k], "bf16" if k in ("x", "wqkv", "wo") else "f32") for k in keys})
         else:
             inp = synth.make_attn_inputs(w)
             sets.append({k: to(inp[k], wl.dtype if k in "qkv" else "f32")
                          for k in ("q", "k", "v", "theta", "w")})
+        sets[-1]["theta_post"] = None if inp["theta_post"] is None else to(inp["theta_post"], "f32")
     return sets
 
 
@@ -233,12 +241,14 @@ def step_fn(wl, mta, sets, ws, outs, stream):
             s = sets[i % len(sets)]
             mta.layer_fwd(s["x"], s["wqkv"], s["theta"], s["w"], s["gamma"], s["beta"], s["wo"],
                           wl.H, wl.c_q, wl.c_k, wl.c_h, wl.kq_place, wl.head_place, eps=1e-5,
-                          layer=wl.depth, out=outs[i % len(outs)], ws=ws, stream=stream)
+                          layer=wl.depth, out=outs[i % len(outs)], ws=ws, stream=stream,
+                          theta_post=s["theta_post"])
     else:
         def f(i):
             s = sets[i % len(sets)]
             mta.attn_fwd(s["q"], s["k"], s["v"], s["theta"], s["w"], wl.c_q, wl.c_k, wl.c_h,
-                         wl.kq_place, wl.head_place, out=outs[i % len(outs)], ws=ws, stream=stream)
+                         wl.kq_place, wl.head_place, out=outs[i % len(outs)], ws=ws, stream=stream,
+                         theta_post=s["theta_post"])
     return f
 
 
@@ -256,7 +266,7 @@ def run_mine(args, wl, rank, world, local_rank):
     odt = torch.float32 if wl.dtype == "f32" else torch.bfloat16
     outs = [torch.empty(out_shape, dtype=odt, device=dev) for _ in range(N_SETS)]
     cfg = mta.make_cfg(wl.B, wl.H, wl.L, wl.d, wl.c_q, wl.c_k, wl.c_h, wl.kq_place, wl.head_place,
-                       mta.F32 if wl.dtype == "f32" else mta.BF16)
+                       mta.F32 if wl.dtype == "f32" else mta.BF16, kq_post=int(wl.kq_post))
     nbytes = (mta.lib().mta_layer_workspace_bytes if wl.layer else mta.lib().mta_attn_workspace_bytes)(
         ctypes.byref(cfg))
     ws = mta.workspace(nbytes, dev)
@@ -341,11 +351,11 @@ def run_e2e(args, wl, mta, sets, ws, stream, dev, barrier, world):
         if wl.layer:
             mta.layer_fwd(dev_in[0]["x"], s["wqkv"], s["theta"], s["w"], s["gamma"], s["beta"],
                           s["wo"], wl.H, wl.c_q, wl.c_k, wl.c_h, wl.kq_place, wl.head_place,
-                          layer=wl.depth, out=dout, ws=ws, stream=stream)
+                          layer=wl.depth, out=dout, ws=ws, stream=stream, theta_post=s["theta_post"])
         else:
             mta.attn_fwd(dev_in[0]["q"], dev_in[0]["k"], dev_in[0]["v"], s["theta"], s["w"],
                          wl.c_q, wl.c_k, wl.c_h, wl.kq_place, wl.head_place, out=dout, ws=ws,
-                         stream=stream)
+                         stream=stream, theta_post=s["theta_post"])
         hout.copy_(dout, non_blocking=True)
 
     with torch.cuda.stream(stream):
@@ -392,11 +402,12 @@ def oracle_sample(wl, budget_s: float, mode: str):
         t = time.perf_counter()
         O.mta_layer_rows(inp["x"][:1], inp["wqkv"], inp["theta"], inp["w"], inp["gamma"],
                          inp["beta"], inp["eps"], inp["lam"], inp["wo"], wl.H, wl.c_h, rows,
-                         wl.kq_place, wl.head_place)
+                         wl.kq_place, wl.head_place, theta_post=inp["theta_post"])
         dt = time.perf_counter() - t
         return 1 / dt, dt, "1 token of the layer (QKV of its batch, attention window, norm, projection)"
     inp = synth.make_attn_inputs(wl)
     q, k, v, th, w = inp["q"], inp["k"], inp["v"], inp["theta"], inp["w"]
+    tp = inp["theta_post"]
     ch = wl.c_h
     if mode == "groups":
         n_units = wl.B * (wl.H // ch)
@@ -408,7 +419,8 @@ def oracle_sample(wl, budget_s: float, mode: str):
                                   np.ascontiguousarray(k[b, :, hs].transpose(1, 0, 2)),
                                   np.ascontiguousarray(v[b, :, hs].transpose(1, 0, 2)),
                                   th[hs], w[g], np.arange(wl.L), 1 / math.sqrt(wl.d),
-                                  wl.kq_place, wl.head_place)
+                                  wl.kq_place, wl.head_place,
+                                  None if tp is None else tp[hs])
             done += 1
             if time.perf_counter() - t0 > budget_s:
                 break
@@ -424,7 +436,8 @@ def oracle_sample(wl, budget_s: float, mode: str):
     while True:
         i = int(rng.integers(wl.L))
         O.mta_attention_rows(q[:1, :, hs], k[:1, :, hs], v[:1, :, hs], th[hs], w[g:g + 1], ch,
-                             [(0, i)], wl.kq_place, wl.head_place)
+                             [(0, i)], wl.kq_place, wl.head_place,
+                             theta_post=None if tp is None else tp[hs])
         done += 1
         if time.perf_counter() - t0 > budget_s:
             break
@@ -475,7 +488,8 @@ def main():
     wl = synth.WORKLOADS[args.workload]
     fl = flops(wl)
     config = {"workload": wl.name, "B": wl.B, "H": wl.H, "L": wl.L, "d": wl.d, "c_q": wl.c_q,
-              "c_k": wl.c_k, "c_h": wl.c_h, "kq_place": ["off", "pre", "post"][wl.kq_place],
+              "c_k": wl.c_k, "c_h": wl.c_h, "kq_place": ["off", "pre", "post", "pre_exact"][wl.kq_place],
+              "kq_post": bool(wl.kq_post),
               "head_place": ["off", "pre", "post"][wl.head_place],
               "parallelism": f"replicas x{max(world, args.gpus)}" if max(world, args.gpus) > 1 else "single",
               "l2": f"{N_SETS} rotating input sets, each step reads a set not touched by the previous step"}
@@ -539,6 +553,17 @@ def main():
                             f"per causal pair-head, x {wl.causal_pairs} pair-heads per launch",
                 "executed_tensor_tflops": executed, "executed_frac": executed / peak,
                 "peak_source": f"{peak_src} bf16 sustained"}
+    elif not uses_direct_tc(wl):
+        # the CUDA-core kernel: every step in fp32 FMA on the CUDA cores
+        kernel = "attn_simt_kernel"
+        achieved = fl["attn_mta"] / s / 1e12
+        roof = {"bound": "alu", "achieved": achieved, "peak": FP32_PEAK_TFLOPS, "unit": "TFLOP/s",
+                "frac": achieved / FP32_PEAK_TFLOPS,
+                "traffic": read_traffic("attn_simt_kernel", wl.name),
+                "kernel": kernel,
+                "per_unit": f"F_mta = {fl['attn_mta'] // wl.causal_pairs} fp32 flop per causal "
+                            f"pair-head (both convolutions), x {wl.causal_pairs} pair-heads per launch",
+                "peak_source": "148 SMs x 128 FP32 lanes x 2 x 1965 MHz"}
     else:
         kernel = "attn_tc_kernel"
         achieved = fl["conv"] / s / 1e12

@@ -23,7 +23,9 @@
  *   w_head[g][r][s] weighs source head g*c_h+s in destination head g*c_h+r.
  *   Post-softmax mixing is not renormalised; the mixed map of head r
  *   multiplies head r's own values.  Pre-softmax mixing follows the
- *   key-query convolution.
+ *   key-query convolution.  The post-softmax kernel theta_post[h][a][t]
+ *   multiplies A[i-a][j-(t-c_k/2)] of the softmax weights in the same way;
+ *   post-softmax mixing follows it.
  *
  * Ownership and threading: every pointer is a DEVICE pointer owned by the
  * caller (theta, w_head, gamma and beta included).  The library allocates no
@@ -47,7 +49,7 @@
 extern "C" {
 #endif
 
-#define MTA_ABI_VERSION 1
+#define MTA_ABI_VERSION 2
 
 typedef enum {
   MTA_OK = 0,
@@ -78,6 +80,12 @@ typedef struct mta_cfg {
   int c_h;               /* heads per mixing group, 1..16 (1 = no mixing)        */
   int kq_place;          /* MTA_OFF, MTA_PRE or MTA_PRE_EXACT                    */
   int head_place;        /* MTA_OFF, MTA_PRE or MTA_POST (OFF when c_h == 1)     */
+  int kq_post;           /* 1: a second key-query convolution acts on the softmax
+                            weights (section 3.1: the kernel may act before or
+                            after the softmax; section 4 uses both), then Mask_0
+                            zeroes the future keys again: A' = Mask_0(Conv2d(A)),
+                            not renormalised, before any post-softmax head mix;
+                            0: none                                              */
   int dtype;             /* mta_dtype of q, k, v and out (x, W and out in a layer) */
   int path;              /* attention kernel: 0 = choose (the contraction kernel
                             where it applies and the workspace holds its operands,
@@ -122,7 +130,9 @@ size_t mta_attn_workspace_bytes(const mta_cfg *cfg);
  * convolution, pre-softmax head mix, Mask_-inf, softmax, post-softmax head mix,
  * A V).  Never materialises an L x L map.
  *   q, k, v  : [B][L][H][d] with token stride cfg->qkv_row_stride, cfg->dtype
- *   theta_kq : [H][c_q][c_k] fp32 (ignored when kq_place == MTA_OFF)
+ *   theta_kq : [n][H][c_q][c_k] fp32, n = (kq_place != MTA_OFF) + kq_post: the
+ *              pre-softmax kernels first, then the post-softmax kernels (NULL
+ *              allowed when n == 0)
  *   w_head   : [H/c_h][c_h][c_h] fp32 (ignored when head_place == MTA_OFF)
  *   out      : [B][L][H][d] dense, cfg->dtype
  * Pointers to bf16 data must be 16-byte aligned and the row stride a multiple

@@ -40,7 +40,7 @@ def test_every_declared_symbol_is_exported(L):
 
 
 def test_version_and_strings(L):
-    assert L.mta_abi_version() == 1
+    assert L.mta_abi_version() == 2
     for code in range(6):
         assert L.mta_status_string(code)
     assert L.mta_status_string(0) == b"ok"
@@ -79,6 +79,9 @@ def test_workspace_query(L):
     other = good_cfg(c_q=3)   # not a contraction shape: fixed scratch only
     assert L.mta_attn_workspace_bytes(ctypes.byref(other)) == 256
     assert L.mta_layer_workspace_bytes(ctypes.byref(other)) == base
+    post = good_cfg(kq_post=1)   # the post-softmax convolution runs on the CUDA-core kernel
+    assert L.mta_attn_workspace_bytes(ctypes.byref(post)) == 256
+    assert L.mta_layer_workspace_bytes(ctypes.byref(post)) == base
     assert L.mta_attn_workspace_bytes(ctypes.byref(good_cfg(c_k=4))) == 0
     assert L.mta_attn_workspace_bytes(None) == 0
 
@@ -87,7 +90,8 @@ def test_workspace_query(L):
     (dict(c_k=4), 1), (dict(c_k=17), 1), (dict(c_q=0), 1), (dict(c_q=9), 1),
     (dict(H=5), 1), (dict(c_h=0), 1), (dict(B=0), 1), (dict(L=0), 1),
     (dict(kq_place=2), 1), (dict(kq_place=4), 1), (dict(head_place=3), 1), (dict(dtype=7), 1), (dict(path=4), 1), (dict(path=-1), 1),
-    (dict(scale=-1.0), 1), (dict(qkv_row_stride=10), 1),
+    (dict(scale=-1.0), 1), (dict(qkv_row_stride=10), 1), (dict(kq_post=2), 1), (dict(kq_post=-1), 1),
+    (dict(kq_post=1, path=mta.PATH_KQ), 2), (dict(kq_post=1, path=mta.PATH_TC), 2),
     (dict(d=200), 2), (dict(d=20), 2), (dict(B=70000), 2),
 ])
 def test_bad_config_rejected(L, kw, code):
@@ -104,6 +108,9 @@ def test_null_and_workspace_errors(L):
     assert call_attn(L, cfg, out=None) == 1
     assert call_attn(L, cfg, theta=None) == 1           # kq_place PRE needs theta
     assert call_attn(L, cfg, w=None) == 1               # head mixing needs w
+    post_only = good_cfg(kq_place=mta.OFF, kq_post=1)
+    post_only.workspace, post_only.workspace_bytes = 0x100000, 1 << 20
+    assert call_attn(L, post_only, theta=None) == 1     # the post-softmax kernels are theta
     nomix = good_cfg(kq_place=mta.OFF, head_place=mta.OFF)
     nomix.workspace, nomix.workspace_bytes = 0x100000, 1 << 20
     assert call_attn(L, nomix, q=ctypes.c_void_p(0x10001)) == 1   # misaligned bf16

@@ -52,15 +52,16 @@ def assert_close(gpu, ref, dtype):
 def run_attn(wl, inp, path=mta.PATH_AUTO, **kw):
     q, k, v = (dev(inp[n], wl.dtype) for n in ("q", "k", "v"))
     th, w = dev(inp["theta"], "f32"), dev(inp["w"], "f32")
+    tp = None if inp.get("theta_post") is None else dev(inp["theta_post"], "f32")
     out = mta.attn_fwd(q, k, v, th, w, wl.c_q, wl.c_k, wl.c_h, wl.kq_place, wl.head_place,
-                       path=path, check=True, **kw)
+                       path=path, check=True, theta_post=tp, **kw)
     torch.cuda.synchronize()
     return out
 
 
 def oracle_full(wl, inp):
     return O.mta_attention(inp["q"], inp["k"], inp["v"], inp["theta"], inp["w"], wl.c_h,
-                           wl.kq_place, wl.head_place)
+                           wl.kq_place, wl.head_place, theta_post=inp.get("theta_post"))
 
 
 # ---------------------------------------------------------------------------
@@ -264,10 +265,11 @@ def test_group_norm_scale():
 
 def run_layer(wl, inp, path=mta.PATH_AUTO):
     x, wqkv, wo = dev(inp["x"]), dev(inp["wqkv"]), dev(inp["wo"])
+    tp = None if inp.get("theta_post") is None else dev(inp["theta_post"], "f32")
     out = mta.layer_fwd(x, wqkv, dev(inp["theta"], "f32"), dev(inp["w"], "f32"),
                         dev(inp["gamma"], "f32"), dev(inp["beta"], "f32"), wo, wl.H, wl.c_q,
                         wl.c_k, wl.c_h, wl.kq_place, wl.head_place, eps=inp["eps"],
-                        layer=wl.depth, path=path, check=True)
+                        layer=wl.depth, path=path, check=True, theta_post=tp)
     torch.cuda.synchronize()
     return out
 
@@ -383,3 +385,70 @@ def test_group_norm_sigmoid_gate():
                              gate=dev(gate, "f32"))
     torch.cuda.synchronize()
     assert_close(y, O.group_norm_scale(o, gamma, beta, 1e-5, O.sigmoid_gate(gate)), "bf16")
+
+
+# ---------------------------------------------------------------------------
+# key-query convolution after the softmax as well (kq_post)
+# ---------------------------------------------------------------------------
+
+POST_SMALL = [("f32", synth.PRE, synth.POST, 9), ("f32", synth.OFF, synth.OFF, 70),
+              ("bf16", synth.PRE, synth.POST, 150), ("bf16", synth.PRE, synth.PRE, 150),
+              ("bf16", synth.PRE, synth.OFF, 33), ("bf16", synth.OFF, synth.POST, 150),
+              ("bf16", mta.PRE_EXACT, synth.POST, 150), ("bf16", synth.PRE, synth.POST, 1)]
+
+
+@pytest.mark.parametrize("dtype,kq,hp,L", POST_SMALL)
+def test_post_conv_small(dtype, kq, hp, L):
+    base = synth.WORKLOADS["both_d128_L2048"]
+    wl = synth.shrink(base, B=2, H=4, L=L, d=64, kq_place=kq, head_place=hp, dtype=dtype,
+                      seed=401 + L + kq + 3 * hp)
+    inp = synth.make_attn_inputs(wl)
+    assert inp["theta_post"] is not None
+    assert_close(run_attn(wl, inp), oracle_full(wl, inp), dtype)
+
+
+def test_post_conv_other_kernel_sizes():
+    base = synth.WORKLOADS["both_d128_L2048"]
+    wl = synth.shrink(base, B=1, H=8, L=100, d=32, c_q=3, c_k=5, c_h=4, seed=455)
+    inp = synth.make_attn_inputs(wl)
+    assert_close(run_attn(wl, inp), oracle_full(wl, inp), "bf16")
+
+
+def test_post_conv_causality_on_gpu():
+    base = synth.WORKLOADS["both_d128_L2048"]
+    wl = synth.shrink(base, B=1, H=4, L=200, d=64, seed=456)
+    inp = synth.make_attn_inputs(wl)
+    a = run_attn(wl, inp)
+    t = 77
+    for n, s in (("q", 1), ("k", 2), ("v", 3)):
+        x = inp[n].copy()
+        x[:, t:] = synth.round_bf16(synth.normal(99, s, x[:, t:].shape))
+        inp[n] = x
+    b = run_attn(wl, inp)
+    assert torch.equal(a[:, :t], b[:, :t])
+    assert not torch.equal(a[:, t:], b[:, t:])
+
+
+def test_post_conv_full_size_sampled():
+    """The pretraining-shaped workload with the convolution on both sides of the
+    softmax, in the launch configuration the bench times."""
+    wl = synth.WORKLOADS["both_d128_L2048"]
+    inp = synth.make_attn_inputs(wl)
+    out = run_attn(wl, inp)
+    rows = sample_rows(wl, seed=6)
+    ref = O.mta_attention_rows(inp["q"], inp["k"], inp["v"], inp["theta"], inp["w"], wl.c_h, rows,
+                               wl.kq_place, wl.head_place, theta_post=inp["theta_post"])
+    got = torch.stack([out[b, i] for b, i in rows])
+    assert_close(got, ref, "bf16")
+
+
+@pytest.mark.parametrize("hp", [synth.PRE, synth.POST])
+def test_post_conv_layer_small(hp):
+    wl = synth.shrink(synth.WORKLOADS["layer_post_D2048_L4096"], B=2, L=200, D=256, H=2, d=128,
+                      head_place=hp, kq_post=True, seed=125)
+    inp = synth.make_layer_inputs(wl)
+    out = run_layer(wl, inp)
+    ref = O.mta_layer(inp["x"], inp["wqkv"], inp["theta"], inp["w"], inp["gamma"], inp["beta"],
+                      inp["eps"], inp["lam"], inp["wo"], wl.H, wl.c_h, wl.kq_place, wl.head_place,
+                      theta_post=inp["theta_post"])
+    assert_close(out, ref, "bf16")

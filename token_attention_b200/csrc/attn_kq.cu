@@ -764,7 +764,7 @@ size_t align256(size_t x) { return (x + 255) / 256 * 256; }
 }  // namespace
 
 bool attn_kq_supported(const AttnArgs &a) {
-  if (a.dtype != 1 || (a.d != 64 && a.d != 128)) return false;
+  if (a.dtype != 1 || a.kqp != 0 || (a.d != 64 && a.d != 128)) return false;
   if ((a.kq != 1 && a.kq != 3) || a.cq != 6 || a.ck != 11) return false;
   if (!(a.hp == 0 || ((a.hp == 1 || a.hp == 2) && a.ch == 2))) return false;
   if (a.B > 65535 || a.H > 65535 || (a.L + 127) / 128 > 65535) return false;

@@ -5,7 +5,9 @@
 // Steps per "Multi-Token Attention | Summary" (greeksharifa): logits Q K^T/sqrt(d)
 // (section 2), Mask_0, key-query convolution over (previous queries, neighbouring
 // keys) (section 3.1), pre-softmax head mix (section 3.2), Mask_-inf and softmax
-// (section 2), post-softmax head mix (section 3.2), A V (section 2).
+// (section 2), the key-query convolution of the softmax weights followed by
+// Mask_0 (section 3.1, after the softmax), post-softmax head mix (section 3.2),
+// A V (section 2).
 //
 // One CTA owns one (batch, head group, tile of BR queries).  Two sweeps over the
 // key tiles: the first gathers the exact row maxima and sums of the softmax, the
@@ -39,22 +41,28 @@ __device__ __forceinline__ __nv_bfloat16 from_f<__nv_bfloat16>(float x) { return
 
 // Offsets (in floats) of the shared-memory arrays.
 struct SimtLayout {
-  int Qs, Ks, Sh, Ct, Pm, m, l, acc, th, wg, total;
+  int Qs, Ks, Sh, Ct, Pm, m, l, acc, th, thp, wg, total;
 };
 
-__host__ __device__ inline SimtLayout simt_layout(int BR, int BC, int d, int cq, int ck, int ch) {
-  const int c = ck / 2, HR = BR + cq - 1, HC = BC + 2 * c, dp = d + 1;
+// With the post-softmax convolution the tile's weights are needed on a wider
+// region: pr = c_q-1 more query rows above and pc = c_k/2 more keys on each side.
+__host__ __device__ inline SimtLayout simt_layout(int BR, int BC, int d, int cq, int ck, int ch,
+                                                  int kqp) {
+  const int c = ck / 2, pr = kqp ? cq - 1 : 0, pc = kqp ? c : 0;
+  const int CR = BR + pr, CC = BC + 2 * pc;           // region of C and A
+  const int HR = CR + cq - 1, HC = CC + 2 * c, dp = d + 1;
   SimtLayout s;
   int o = 0;
-  s.Qs = o;  o += HR * dp;        // query rows i0-(cq-1) .. i0+BR-1 of one head
-  s.Ks = o;  o += HC * dp;        // key rows j0-c .. j0+BC+c-1 of one head
+  s.Qs = o;  o += HR * dp;        // query rows i0-pr-(cq-1) .. i0+BR-1 of one head
+  s.Ks = o;  o += HC * dp;        // key rows j0-pc-c .. j0+BC+pc+c-1 of one head
   s.Sh = o;  o += HR * HC;        // Mask_0(A_hat) on the halo tile
-  s.Ct = o;  o += ch * BR * BC;   // convolved (then mixed) logits / probabilities
-  s.Pm = o;  o += ch * BR * BC;   // mixing scratch
-  s.m = o;   o += ch * BR;        // row max
-  s.l = o;   o += ch * BR;        // row sum
+  s.Ct = o;  o += ch * CR * CC;   // convolved (then mixed) logits / probabilities
+  s.Pm = o;  o += ch * CR * CC;   // softmax weights / mixing scratch
+  s.m = o;   o += ch * CR;        // row max
+  s.l = o;   o += ch * CR;        // row sum
   s.acc = o; o += ch * BR * d;    // output accumulators
-  s.th = o;  o += ch * cq * ck;   // key-query kernels of the group
+  s.th = o;  o += ch * cq * ck;   // pre-softmax key-query kernels of the group
+  s.thp = o; o += ch * cq * ck;   // post-softmax key-query kernels of the group
   s.wg = o;  o += ch * ch;        // head-mixing weights of the group
   s.total = o;
   return s;
@@ -65,10 +73,13 @@ __global__ void __launch_bounds__(kThreads) attn_simt_kernel(AttnArgs a, int BR)
   extern __shared__ float sm[];
   const int BC = kBC;
   const int d = a.d, cq = a.cq, ck = a.ck, ch = a.ch, c = ck / 2, L = a.L, H = a.H;
-  const int HR = BR + cq - 1, HC = BC + 2 * c, dp = d + 1;
-  const SimtLayout S = simt_layout(BR, BC, d, cq, ck, ch);
+  const int kqp = a.kqp, pr = kqp ? cq - 1 : 0, pc = kqp ? c : 0;
+  const int CR = BR + pr, CC = BC + 2 * pc;
+  const int HR = CR + cq - 1, HC = CC + 2 * c, dp = d + 1;
+  const SimtLayout S = simt_layout(BR, BC, d, cq, ck, ch, kqp);
   float *Qs = sm + S.Qs, *Ks = sm + S.Ks, *Sh = sm + S.Sh, *Ct = sm + S.Ct, *Pm = sm + S.Pm;
-  float *rm = sm + S.m, *rl = sm + S.l, *acc = sm + S.acc, *th = sm + S.th, *wg = sm + S.wg;
+  float *rm = sm + S.m, *rl = sm + S.l, *acc = sm + S.acc, *th = sm + S.th, *thp = sm + S.thp;
+  float *wg = sm + S.wg;
   const int i0 = blockIdx.x * BR, g = blockIdx.y, b = blockIdx.z, tid = threadIdx.x;
   const T *q = static_cast<const T *>(a.q);
   const T *k = static_cast<const T *>(a.k);
@@ -78,32 +89,37 @@ __global__ void __launch_bounds__(kThreads) attn_simt_kernel(AttnArgs a, int BR)
   const bool kq = (a.kq != 0);
   const bool exact = (a.kq == 3);  // exact causal indicator instead of Mask_0
 
-  for (int i = tid; i < ch * cq * ck; i += kThreads) th[i] = kq ? a.theta[g * ch * cq * ck + i] : 0.f;
+  for (int i = tid; i < ch * cq * ck; i += kThreads) {
+    th[i] = kq ? a.theta[g * ch * cq * ck + i] : 0.f;
+    thp[i] = kqp ? a.theta_post[g * ch * cq * ck + i] : 0.f;
+  }
   for (int i = tid; i < ch * ch; i += kThreads)
     wg[i] = (a.hp != 0) ? a.w[g * ch * ch + i] : (i / ch == i % ch ? 1.f : 0.f);
-  for (int i = tid; i < ch * BR; i += kThreads) { rm[i] = NEG_INF; rl[i] = 0.f; }
+  for (int i = tid; i < ch * CR; i += kThreads) { rm[i] = NEG_INF; rl[i] = 0.f; }
   for (int i = tid; i < ch * BR * d; i += kThreads) acc[i] = 0.f;
   __syncthreads();
 
   const int q_end = min(L, i0 + BR);  // queries of this tile are i0 .. q_end-1
-  const int tile = BR * BC;
+  const int region = CR * CC, tile = BR * BC;
+  const int rq0 = i0 - pr, rk0_ofs = -pc;  // region row r is query rq0 + r, column s key j0 - pc + s
   for (int pass = 0; pass < 2; ++pass) {
     for (int j0 = 0; j0 < q_end; j0 += BC) {
+      const int rk0 = j0 + rk0_ofs;
       for (int hl = 0; hl < ch; ++hl) {
         const int h = g * ch + hl;
         for (int i = tid; i < HR * d; i += kThreads) {
-          const int r = i / d, e = i % d, iq = i0 - (cq - 1) + r;
+          const int r = i / d, e = i % d, iq = rq0 - (cq - 1) + r;
           Qs[r * dp + e] = (iq >= 0 && iq < L) ? to_f(q[((long long)b * L + iq) * a.rs + h * d + e]) : 0.f;
         }
         for (int i = tid; i < HC * d; i += kThreads) {
-          const int s = i / d, e = i % d, jk = j0 - c + s;
+          const int s = i / d, e = i % d, jk = rk0 - c + s;
           Ks[s * dp + e] = (jk >= 0 && jk < L) ? to_f(k[((long long)b * L + jk) * a.rs + h * d + e]) : 0.f;
         }
         __syncthreads();
         // Mask_0(A_hat) on the halo tile: future keys of each (shifted) query are 0
         // (with the exact indicator the logits stay unmasked here; see below)
         for (int i = tid; i < HR * HC; i += kThreads) {
-          const int r = i / HC, s = i % HC, iq = i0 - (cq - 1) + r, jk = j0 - c + s;
+          const int r = i / HC, s = i % HC, iq = rq0 - (cq - 1) + r, jk = rk0 - c + s;
           float val = 0.f;
           if (iq >= 0 && iq < L && jk >= 0 && jk < L && (!kq || exact || jk <= iq)) {
             const float *qr = Qs + r * dp, *kr = Ks + s * dp;
@@ -115,44 +131,44 @@ __global__ void __launch_bounds__(kThreads) attn_simt_kernel(AttnArgs a, int BR)
         __syncthreads();
         // key-query convolution: C[i][j] = sum_a sum_t theta[a][t] M0[i-a][j-(t-c)];
         // with the exact indicator a tap counts when its key j-(t-c) <= i
-        for (int i = tid; i < tile; i += kThreads) {
-          const int r = i / BC, j = i % BC;
+        for (int i = tid; i < region; i += kThreads) {
+          const int r = i / CC, s = i % CC;
           float val;
           if (kq) {
             val = 0.f;
             const float *tk = th + hl * cq * ck;
-            const int t0 = exact ? max(0, (j0 + j) + c - (i0 + r)) : 0;
+            const int t0 = exact ? max(0, (rk0 + s) + c - (rq0 + r)) : 0;
             for (int aa = 0; aa < cq; ++aa) {
-              const float *srow = Sh + (r + cq - 1 - aa) * HC + j + 2 * c;
+              const float *srow = Sh + (r + cq - 1 - aa) * HC + s + 2 * c;
               for (int t = t0; t < ck; ++t) val = fmaf(tk[aa * ck + t], srow[-t], val);
             }
           } else {
-            val = Sh[(r + cq - 1) * HC + j + c];
+            val = Sh[(r + cq - 1) * HC + s + c];
           }
-          Ct[hl * tile + i] = val;
+          Ct[hl * region + i] = val;
         }
         __syncthreads();
       }
       if (a.hp == 1) {  // pre-softmax head mix
-        for (int i = tid; i < ch * tile; i += kThreads) {
-          const int hl = i / tile, rem = i % tile;
+        for (int i = tid; i < ch * region; i += kThreads) {
+          const int hl = i / region, rem = i % region;
           float val = 0.f;
-          for (int s = 0; s < ch; ++s) val = fmaf(wg[hl * ch + s], Ct[s * tile + rem], val);
+          for (int s = 0; s < ch; ++s) val = fmaf(wg[hl * ch + s], Ct[s * region + rem], val);
           Pm[i] = val;
         }
         __syncthreads();
-        for (int i = tid; i < ch * tile; i += kThreads) Ct[i] = Pm[i];
+        for (int i = tid; i < ch * region; i += kThreads) Ct[i] = Pm[i];
         __syncthreads();
       }
-      // Mask_-inf: keys after the query (and past the sequence) get -inf
-      for (int i = tid; i < ch * tile; i += kThreads) {
-        const int rem = i % tile, r = rem / BC, j = rem % BC;
-        if (j0 + j > i0 + r || j0 + j >= L) Ct[i] = NEG_INF;
+      // Mask_-inf: keys after the query, outside the sequence, and rows before it get -inf
+      for (int i = tid; i < ch * region; i += kThreads) {
+        const int rem = i % region, iq = rq0 + rem / CC, jk = rk0 + rem % CC;
+        if (jk > iq || jk >= L || jk < 0 || iq < 0) Ct[i] = NEG_INF;
       }
       __syncthreads();
-      if (pass == 0) {
-        for (int i = tid; i < ch * BR; i += kThreads) {
-          const float *row = Ct + i * BC;
+      if (pass == 0) {  // statistics over this tile's own keys (columns pc .. pc+BC-1)
+        for (int i = tid; i < ch * CR; i += kThreads) {
+          const float *row = Ct + i * CC + pc;
           float mx = NEG_INF;
           for (int j = 0; j < BC; ++j) mx = fmaxf(mx, row[j]);
           const float mn = fmaxf(rm[i], mx);
@@ -164,9 +180,29 @@ __global__ void __launch_bounds__(kThreads) attn_simt_kernel(AttnArgs a, int BR)
         }
         __syncthreads();
       } else {
+        // softmax weights A on the region (0 at masked entries and empty rows)
+        for (int i = tid; i < ch * region; i += kThreads) {
+          const int hr = i / CC;
+          Pm[i] = (Ct[i] == NEG_INF || rm[hr] == NEG_INF) ? 0.f : expf(Ct[i] - rm[hr]) / rl[hr];
+        }
+        __syncthreads();
+        // post-softmax convolution, then Mask_0: A'[i][j] = [j <= i] sum theta_post[a][t] A[i-a][j-(t-c)]
         for (int i = tid; i < ch * tile; i += kThreads) {
-          const int hr = i / BC;
-          Pm[i] = expf(Ct[i] - rm[hr]) / rl[hr];
+          const int hl = i / tile, rem = i % tile, r = rem / BC, j = rem % BC;
+          float val;
+          if (kqp) {
+            val = 0.f;
+            if (j0 + j <= i0 + r) {
+              const float *tk = thp + hl * cq * ck;
+              for (int aa = 0; aa < cq; ++aa) {
+                const float *prow = Pm + hl * region + (r + pr - aa) * CC + j + pc + c;
+                for (int t = 0; t < ck; ++t) val = fmaf(tk[aa * ck + t], prow[-t], val);
+              }
+            }
+          } else {
+            val = Pm[hl * region + r * CC + j];
+          }
+          Ct[i] = val;
         }
         __syncthreads();
         for (int i = tid; i < ch * tile; i += kThreads) {  // post-softmax head mix
@@ -174,17 +210,17 @@ __global__ void __launch_bounds__(kThreads) attn_simt_kernel(AttnArgs a, int BR)
           float val;
           if (a.hp == 2) {
             val = 0.f;
-            for (int s = 0; s < ch; ++s) val = fmaf(wg[hl * ch + s], Pm[s * tile + rem], val);
+            for (int s = 0; s < ch; ++s) val = fmaf(wg[hl * ch + s], Ct[s * tile + rem], val);
           } else {
-            val = Pm[i];
+            val = Ct[i];
           }
-          Ct[i] = val;
+          Pm[i] = val;
         }
         __syncthreads();
         for (int i = tid; i < ch * BR * d; i += kThreads) {  // acc += A V (head's own V)
           const int hl = i / (BR * d), rem = i % (BR * d), r = rem / d, e = rem % d;
           const int h = g * ch + hl;
-          const float *prow = Ct + (hl * BR + r) * BC;
+          const float *prow = Pm + (hl * BR + r) * BC;
           float s = acc[i];
           const int jn = min(BC, L - j0);
           for (int j = 0; j < jn; ++j)
@@ -205,7 +241,7 @@ __global__ void __launch_bounds__(kThreads) attn_simt_kernel(AttnArgs a, int BR)
 }  // namespace
 
 size_t attn_simt_smem_bytes(const AttnArgs &a, int BR, int BC) {
-  return static_cast<size_t>(simt_layout(BR, BC, a.d, a.cq, a.ck, a.ch).total) * sizeof(float);
+  return static_cast<size_t>(simt_layout(BR, BC, a.d, a.cq, a.ck, a.ch, a.kqp).total) * sizeof(float);
 }
 
 int attn_simt_pick_rows(const AttnArgs &a, int BC) {

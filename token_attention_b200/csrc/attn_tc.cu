@@ -598,7 +598,7 @@ cudaError_t launch_one(const AttnArgs &a, const GnArgs *gn) {
 }  // namespace
 
 bool attn_tc_supported(const AttnArgs &a) {
-  if (a.dtype != 1) return false;
+  if (a.dtype != 1 || a.kqp != 0) return false;
   if (a.d != 64 && a.d != 128) return false;
   const bool kq_std = a.kq == 1 && a.cq == 6 && a.ck == 11;
   const bool kq_off = a.kq == 0;

@@ -13,10 +13,12 @@ enum : unsigned { ERRBIT_TIMEOUT = 1u };
 struct AttnArgs {
   const void *q, *k, *v;  // [B][L][H][d], token stride rs elements
   long long rs;
-  const float *theta;     // [H][c_q][c_k]
+  const float *theta;     // [H][c_q][c_k] pre-softmax kernels
+  const float *theta_post;  // [H][c_q][c_k] post-softmax kernels (kqp == 1)
   const float *w;         // [H/c_h][c_h][c_h]
   void *out;              // [B][L][H][d] dense
   int B, H, L, d, cq, ck, ch, kq, hp, dtype;
+  int kqp;                // 1: key-query convolution after the softmax as well
   float scale;
   unsigned *err;          // error word in the workspace
   cudaStream_t stream;

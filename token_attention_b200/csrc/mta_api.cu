@@ -33,6 +33,7 @@ mta_status check_cfg(const mta_cfg *c) {
     return MTA_ERR_INVALID;
   if (c->head_place != MTA_OFF && c->head_place != MTA_PRE && c->head_place != MTA_POST)
     return MTA_ERR_INVALID;
+  if (c->kq_post != 0 && c->kq_post != 1) return MTA_ERR_INVALID;
   if (c->dtype != MTA_F32 && c->dtype != MTA_BF16) return MTA_ERR_INVALID;
   if (c->path < 0 || c->path > 3) return MTA_ERR_INVALID;
   if (!isfinite(c->scale) || c->scale < 0.f) return MTA_ERR_INVALID;
@@ -45,6 +46,11 @@ AttnArgs make_args(const void *q, const void *k, const void *v, const float *the
                    const float *w, const mta_cfg *c, void *out) {
   AttnArgs a;
   a.q = q; a.k = k; a.v = v; a.theta = theta; a.w = w; a.out = out;
+  // theta holds the pre-softmax kernels (when kq_place is on), then the post-softmax ones
+  a.kqp = c->kq_post;
+  a.theta_post = (c->kq_post && theta)
+                     ? theta + (c->kq_place != MTA_OFF ? static_cast<size_t>(c->H) * c->c_q * c->c_k : 0)
+                     : nullptr;
   a.rs = c->qkv_row_stride ? c->qkv_row_stride : static_cast<long long>(c->H) * c->d;
   a.B = c->B; a.H = c->H; a.L = c->L; a.d = c->d;
   a.cq = c->c_q; a.ck = c->c_k; a.ch = c->c_h;
@@ -60,7 +66,7 @@ enum Kernel { K_SIMT = 1, K_TC = 2, K_KQ = 3 };
 // Shape-level test for the contraction kernel (pointer alignment aside): used
 // to size the workspace.
 bool kq_shape_ok(const mta_cfg *c) {
-  return c->dtype == MTA_BF16 && (c->d == 64 || c->d == 128) &&
+  return c->dtype == MTA_BF16 && c->kq_post == 0 && (c->d == 64 || c->d == 128) &&
          (c->kq_place == MTA_PRE || c->kq_place == MTA_PRE_EXACT) &&
          c->c_q == 6 && c->c_k == 11 &&
          (c->head_place == MTA_OFF || ((c->head_place == MTA_PRE || c->head_place == MTA_POST) && c->c_h == 2));
@@ -105,7 +111,7 @@ cudaError_t launch_kernel(Kernel k, const AttnArgs &a, const GnArgs *gn, void *k
 mta_status check_attn_pointers(const void *q, const void *k, const void *v, const float *theta,
                                const float *w, const mta_cfg *c, const void *out) {
   if (!q || !k || !v || !out) return MTA_ERR_INVALID;
-  if (c->kq_place != MTA_OFF && !theta) return MTA_ERR_INVALID;
+  if ((c->kq_place != MTA_OFF || c->kq_post) && !theta) return MTA_ERR_INVALID;
   if (c->head_place != MTA_OFF && !w) return MTA_ERR_INVALID;
   const size_t es = c->dtype == MTA_F32 ? 4 : 2;
   if (!aligned(q, es) || !aligned(k, es) || !aligned(v, es) || !aligned(out, es))
@@ -227,8 +233,9 @@ mta_status mta_layer_fwd(const void *x, const void *Wqkv, const float *theta, co
   if (s != MTA_OK) return s;
   if (cfg->dtype != MTA_BF16) return MTA_ERR_UNSUPPORTED;
   if (!x || !Wqkv || !Wo || !out || !gn || !gn->gamma || !gn->beta) return MTA_ERR_INVALID;
-  if (cfg->kq_place != MTA_OFF && !theta) return MTA_ERR_INVALID;
+  if ((cfg->kq_place != MTA_OFF || cfg->kq_post) && !theta) return MTA_ERR_INVALID;
   if (cfg->head_place != MTA_OFF && !w_head) return MTA_ERR_INVALID;
+  if (theta && !aligned(theta, 4)) return MTA_ERR_INVALID;
   if (!aligned(x, 16) || !aligned(Wqkv, 16) || !aligned(Wo, 16) || !aligned(out, 16) ||
       !aligned(gn->gamma, 4) || !aligned(gn->beta, 4))
     return MTA_ERR_INVALID;

@@ -33,7 +33,7 @@ class MtaCfg(ctypes.Structure):
     _fields_ = [("B", ctypes.c_int), ("H", ctypes.c_int), ("L", ctypes.c_int), ("d", ctypes.c_int),
                 ("c_q", ctypes.c_int), ("c_k", ctypes.c_int), ("c_h", ctypes.c_int),
                 ("kq_place", ctypes.c_int), ("head_place", ctypes.c_int),
-                ("dtype", ctypes.c_int), ("path", ctypes.c_int), ("scale", ctypes.c_float),
+                ("kq_post", ctypes.c_int), ("dtype", ctypes.c_int), ("path", ctypes.c_int), ("scale", ctypes.c_float),
                 ("qkv_row_stride", ctypes.c_longlong), ("stream", ctypes.c_void_p),
                 ("workspace", ctypes.c_void_p), ("workspace_bytes", ctypes.c_size_t)]
 
@@ -100,11 +100,12 @@ def _stream_handle(stream):
 
 
 def make_cfg(B, H, L, d, c_q, c_k, c_h, kq_place, head_place, dtype, path=PATH_AUTO, scale=0.0,
-             qkv_row_stride=0, stream=None, workspace=None) -> MtaCfg:
+             qkv_row_stride=0, stream=None, workspace=None, kq_post=0) -> MtaCfg:
     cfg = MtaCfg()
     cfg.B, cfg.H, cfg.L, cfg.d = B, H, L, d
     cfg.c_q, cfg.c_k, cfg.c_h = c_q, c_k, c_h
     cfg.kq_place, cfg.head_place, cfg.dtype, cfg.path = kq_place, head_place, dtype, path
+    cfg.kq_post = kq_post
     cfg.scale = scale
     cfg.qkv_row_stride = qkv_row_stride
     cfg.stream = stream
@@ -129,11 +130,23 @@ def workspace(nbytes: int, device="cuda"):
     return torch.empty(max(int(nbytes), 256), dtype=torch.uint8, device=device)
 
 
+def _kernels(theta, theta_post, kq_place):
+    """The library's key-query kernel array: the pre-softmax kernels (when the
+    convolution before the softmax is on), then the post-softmax kernels."""
+    import torch
+    if theta_post is None:
+        return theta, 0
+    if kq_place == OFF:
+        return theta_post.contiguous(), 1
+    return torch.cat([theta.reshape(-1), theta_post.reshape(-1)]), 1
+
+
 def attn_fwd(q, k, v, theta, w, c_q, c_k, c_h, kq_place=PRE, head_place=POST, *, out=None,
-             ws=None, path=PATH_AUTO, scale=0.0, stream=None, check=False):
+             ws=None, path=PATH_AUTO, scale=0.0, stream=None, check=False, theta_post=None):
     """MTA attention.  q, k, v: [B, L, H, d] CUDA tensors (fp32 or bf16), dense in
     (H, d) with a common token stride; theta [H, c_q, c_k] fp32; w [H/c_h, c_h, c_h]
-    fp32.  Returns out [B, L, H, d] (dtype of q)."""
+    fp32; theta_post: optional [H, c_q, c_k] fp32 kernels of the key-query
+    convolution after the softmax.  Returns out [B, L, H, d] (dtype of q)."""
     import torch
     B, L, H, d = q.shape
     for t in (k, v):
@@ -143,8 +156,9 @@ def attn_fwd(q, k, v, theta, w, c_q, c_k, c_h, kq_place=PRE, head_place=POST, *,
         raise ValueError("q, k, v must be [B, L, H, d] with dense heads and a token stride")
     if out is None:
         out = torch.empty((B, L, H, d), dtype=q.dtype, device=q.device)
+    theta, kq_post = _kernels(theta, theta_post, kq_place)
     cfg = make_cfg(B, H, L, d, c_q, c_k, c_h, kq_place, head_place, _dtype_code(q), path, scale,
-                   q.stride(1), _stream_handle(stream))
+                   q.stride(1), _stream_handle(stream), kq_post=kq_post)
     if ws is None:
         ws = workspace(lib().mta_attn_workspace_bytes(ctypes.byref(cfg)), q.device)
     cfg.workspace, cfg.workspace_bytes = ws.data_ptr(), ws.numel()
@@ -161,17 +175,19 @@ def depth_scale(layer: int) -> float:
 
 def layer_fwd(x, wqkv, theta, w, gamma, beta, wo, H, c_q, c_k, c_h, kq_place=PRE,
               head_place=POST, *, eps=1e-5, layer=12, lam=-1.0, gate=None, out=None, ws=None,
-              path=PATH_AUTO, stream=None, check=False):
+              path=PATH_AUTO, stream=None, check=False, theta_post=None):
     """Full MTA layer, bf16.  x [B, L, D]; wqkv [3D, D]; wo [D, D]; gamma, beta [D]
-    fp32; gate: optional [H] fp32 sigmoid-gate logits replacing the depth scale.
+    fp32; gate: optional [H] fp32 sigmoid-gate logits replacing the depth scale;
+    theta_post: optional [H, c_q, c_k] post-softmax key-query kernels.
     Returns out [B, L, D] bf16."""
     import torch
     B, L, D = x.shape
     d = D // H
     if out is None:
         out = torch.empty((B, L, D), dtype=x.dtype, device=x.device)
+    theta, kq_post = _kernels(theta, theta_post, kq_place)
     cfg = make_cfg(B, H, L, d, c_q, c_k, c_h, kq_place, head_place, _dtype_code(x), path, 0.0, 0,
-                   _stream_handle(stream))
+                   _stream_handle(stream), kq_post=kq_post)
     if ws is None:
         ws = workspace(lib().mta_layer_workspace_bytes(ctypes.byref(cfg)), x.device)
     cfg.workspace, cfg.workspace_bytes = ws.data_ptr(), ws.numel()
@@ -185,8 +201,9 @@ def layer_fwd(x, wqkv, theta, w, gamma, beta, wo, H, c_q, c_k, c_h, kq_place=PRE
     return out
 
 
-def layer_workspace_bytes(B, L, H, d, c_q, c_k, c_h, kq_place=PRE, head_place=POST) -> int:
-    cfg = make_cfg(B, H, L, d, c_q, c_k, c_h, kq_place, head_place, BF16)
+def layer_workspace_bytes(B, L, H, d, c_q, c_k, c_h, kq_place=PRE, head_place=POST,
+                          kq_post=0) -> int:
+    cfg = make_cfg(B, H, L, d, c_q, c_k, c_h, kq_place, head_place, BF16, kq_post=kq_post)
     return lib().mta_layer_workspace_bytes(ctypes.byref(cfg))
 
 

@@ -83,6 +83,7 @@ class Workload:
     D: int = 0
     depth: int = 12       # layer index for the depth scale
     planted_pairs: int = 0
+    kq_post: bool = False # key-query convolution after the softmax as well (own kernels)
 
     @property
     def tokens(self) -> int:
@@ -126,6 +127,12 @@ WORKLOADS = {
                                        dtype="bf16", seed=1005, theta_kind="delta_noise",
                                        theta_std=0.05, w_kind="eye_noise", w_std=0.1,
                                        layer=True, D=2048),
+    # the convolution on both sides of the softmax (the pages' default setting),
+    # pretraining-shaped: post kernels drawn like the pre kernels
+    "both_d128_L2048": Workload("both_d128_L2048", B=4, H=16, L=2048, d=128, c_q=6, c_k=11,
+                                c_h=2, kq_place=PRE, head_place=POST, dtype="bf16", seed=1006,
+                                theta_kind="delta_noise", theta_std=0.05, w_kind="eye_noise",
+                                w_std=0.1, kq_post=True),
 }
 
 
@@ -136,18 +143,25 @@ def shrink(wl: Workload, **changes) -> Workload:
 
 # stream ids (fixed so that a tensor does not change when another one is added)
 _S_Q, _S_K, _S_V, _S_THETA, _S_W, _S_X, _S_WQKV, _S_WO, _S_GAMMA, _S_BETA, _S_PLANT = range(11)
+_S_THETA_POST = 11
 
 
-def make_theta(wl: Workload) -> np.ndarray:
+def make_theta(wl: Workload, stream: int = _S_THETA) -> np.ndarray:
     """Key-query kernels [H][c_q][c_k], float32.  "(0,0)" is the current query
     and the centre key: theta[h][0][c_k//2]."""
     th = np.zeros((wl.H, wl.c_q, wl.c_k), np.float32)
     if wl.theta_kind == "delta_noise":
-        th += normal(wl.seed, _S_THETA, th.shape, std=wl.theta_std)
+        th += normal(wl.seed, stream, th.shape, std=wl.theta_std)
     elif wl.theta_kind != "identity":
         raise ValueError(wl.theta_kind)
     th[:, 0, wl.c_k // 2] += 1.0
     return th
+
+
+def make_theta_post(wl: Workload):
+    """Post-softmax key-query kernels [H][c_q][c_k] (same recipe as the pre-softmax
+    ones, their own stream), or None when the workload has none."""
+    return make_theta(wl, _S_THETA_POST) if wl.kq_post else None
 
 
 def make_w(wl: Workload) -> np.ndarray:
@@ -188,7 +202,7 @@ def make_attn_inputs(wl: Workload) -> dict:
         _plant_pairs(wl, q, k)
     if wl.dtype == "bf16":
         q, k, v = round_bf16(q), round_bf16(k), round_bf16(v)
-    return dict(q=q, k=k, v=v, theta=make_theta(wl), w=make_w(wl))
+    return dict(q=q, k=k, v=v, theta=make_theta(wl), w=make_w(wl), theta_post=make_theta_post(wl))
 
 
 def make_layer_inputs(wl: Workload) -> dict:
@@ -201,4 +215,4 @@ def make_layer_inputs(wl: Workload) -> dict:
     gamma = normal(wl.seed, _S_GAMMA, (D,), mean=1.0, std=0.1)
     beta = normal(wl.seed, _S_BETA, (D,), std=0.1)
     return dict(x=x, wqkv=wqkv, wo=wo, theta=make_theta(wl), w=make_w(wl),
-                gamma=gamma, beta=beta, eps=1e-5, lam=depth_scale(wl.depth))
+                theta_post=make_theta_post(wl), gamma=gamma, beta=beta, eps=1e-5, lam=depth_scale(wl.depth))
