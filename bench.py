@@ -68,7 +68,7 @@ def uses_contraction(wl: synth.Workload) -> bool:
     """Whether the library's default path runs the contraction kernel (with its
     prepass) for this workload."""
     return (wl.dtype == "bf16" and wl.d in (64, 128) and wl.kq_place == synth.PRE
-            and not wl.kq_post and (wl.c_q, wl.c_k) == (6, 11)
+            and (wl.c_q, wl.c_k) == (6, 11)
             and (wl.head_place == synth.OFF or wl.c_h == 2))
 
 
@@ -77,11 +77,17 @@ def contraction_tensor_flops(wl: synth.Workload) -> float:
     query tile, key tile at or below the diagonal) a 128x128 tile of the
     c_q*d-long contraction (for each source head of the group with pre-softmax
     mixing) and, per V head held (both heads of the group with post-softmax
-    mixing), a 128x128xd P V product."""
-    nt = -(-wl.L // 128)
-    tiles = wl.B * wl.H * nt * (nt + 1) // 2
+    mixing), a 128x128xd P V product.  With the post-softmax convolution the
+    query tiles hold 123 output rows, the contraction runs in both passes and
+    P V becomes c_q row-shifted products with the convolved values."""
     nv = 2 if wl.head_place == synth.POST else 1
     nsrc = 2 if wl.head_place == synth.PRE else 1
+    if wl.kq_post:
+        nq = -(-wl.L // 123)
+        tiles = wl.B * wl.H * sum(min(wl.L - 1, qt * 123 - 5 + 127) // 128 + 1 for qt in range(nq))
+        return tiles * 2.0 * 128 * 128 * (2 * nsrc * wl.c_q * wl.d + nv * wl.c_q * wl.d)
+    nt = -(-wl.L // 128)
+    tiles = wl.B * wl.H * nt * (nt + 1) // 2
     return tiles * 2.0 * 128 * 128 * (nsrc * wl.c_q * wl.d + nv * wl.d)
 
 
@@ -99,7 +105,9 @@ def launches_per_step(wl: synth.Workload) -> int:
     kernel."""
     kq = uses_contraction(wl)
     tc = uses_direct_tc(wl)
-    attn = 2 if kq else 1  # the contraction kernel runs after its prepass
+    # the contraction kernel runs after its prepass (and the value prepass with the
+    # post-softmax convolution)
+    attn = (3 if wl.kq_post else 2) if kq else 1
     if not wl.layer:
         return attn
     return 2 + (attn if (kq or tc) else 2)
@@ -547,9 +555,12 @@ def main():
         executed = contraction_tensor_flops(wl) / s / 1e12
         roof = {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
                 "frac": achieved / peak,
-                "traffic": call_traffic(("kq_prep_kernel", "attn_kq_kernel"), wl.name),
-                "kernel": "mta_attn_fwd call = kq_prep_kernel + attn_kq_kernel",
-                "per_unit": f"F_mta = 4d + 2 c_q c_k + 2 c_h = {fl['attn_mta'] // wl.causal_pairs} flop "
+                "traffic": call_traffic(("kq_prep_kernel",) + (("vt_prep_kernel",) if wl.kq_post else ())
+                                        + ("attn_kq_kernel",), wl.name),
+                "kernel": "mta_attn_fwd call = kq_prep_kernel + " + ("vt_prep_kernel + " if wl.kq_post else "")
+                          + "attn_kq_kernel",
+                "per_unit": f"F_mta = 4d + 2 c_q c_k{' x 2' if wl.kq_post else ''} + 2 c_h = "
+                            f"{fl['attn_mta'] // wl.causal_pairs} flop "
                             f"per causal pair-head, x {wl.causal_pairs} pair-heads per launch",
                 "executed_tensor_tflops": executed, "executed_frac": executed / peak,
                 "peak_source": f"{peak_src} bf16 sustained"}

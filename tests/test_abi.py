@@ -79,9 +79,15 @@ def test_workspace_query(L):
     other = good_cfg(c_q=3)   # not a contraction shape: fixed scratch only
     assert L.mta_attn_workspace_bytes(ctypes.byref(other)) == 256
     assert L.mta_layer_workspace_bytes(ctypes.byref(other)) == base
-    post = good_cfg(kq_post=1)   # the post-softmax convolution runs on the CUDA-core kernel
-    assert L.mta_attn_workspace_bytes(ctypes.byref(post)) == 256
-    assert L.mta_layer_workspace_bytes(ctypes.byref(post)) == base
+    post = good_cfg(kq_post=1)   # adds the values convolved by the post-softmax kernels
+    vt = up(B * H * Ls * 2 * cq * d * 2)   # both heads of the group (post-softmax mixing)
+    assert L.mta_attn_workspace_bytes(ctypes.byref(post)) == 256 + kq + vt
+    assert L.mta_layer_workspace_bytes(ctypes.byref(post)) == base + kq + vt
+    post_nomix = good_cfg(kq_post=1, head_place=mta.OFF)
+    kq0 = kq - xg
+    assert L.mta_attn_workspace_bytes(ctypes.byref(post_nomix)) == 256 + kq0 + up(B * H * Ls * cq * d * 2)
+    post_off = good_cfg(kq_post=1, kq_place=mta.OFF)   # CUDA-core kernel only
+    assert L.mta_attn_workspace_bytes(ctypes.byref(post_off)) == 256
     assert L.mta_attn_workspace_bytes(ctypes.byref(good_cfg(c_k=4))) == 0
     assert L.mta_attn_workspace_bytes(None) == 0
 
@@ -91,7 +97,7 @@ def test_workspace_query(L):
     (dict(H=5), 1), (dict(c_h=0), 1), (dict(B=0), 1), (dict(L=0), 1),
     (dict(kq_place=2), 1), (dict(kq_place=4), 1), (dict(head_place=3), 1), (dict(dtype=7), 1), (dict(path=4), 1), (dict(path=-1), 1),
     (dict(scale=-1.0), 1), (dict(qkv_row_stride=10), 1), (dict(kq_post=2), 1), (dict(kq_post=-1), 1),
-    (dict(kq_post=1, path=mta.PATH_KQ), 2), (dict(kq_post=1, path=mta.PATH_TC), 2),
+    (dict(kq_post=1, kq_place=mta.OFF, path=mta.PATH_KQ), 2), (dict(kq_post=1, path=mta.PATH_TC), 2),
     (dict(d=200), 2), (dict(d=20), 2), (dict(B=70000), 2),
 ])
 def test_bad_config_rejected(L, kw, code):

@@ -407,6 +407,44 @@ def test_post_conv_small(dtype, kq, hp, L):
     assert_close(run_attn(wl, inp), oracle_full(wl, inp), dtype)
 
 
+POST_PATHS = [(d, hp, L) for d in (64, 128) for hp in (synth.OFF, synth.PRE, synth.POST)
+              for L in (9, 300)]
+
+
+@pytest.mark.parametrize("d,hp,L", POST_PATHS)
+@pytest.mark.parametrize("path", [mta.PATH_SIMT, mta.PATH_KQ])
+def test_post_conv_kernels(d, hp, L, path):
+    """Both kernels that take the post-softmax convolution, with tiles of 123
+    output rows on the contraction kernel (L = 300: three tiles, ragged tail)."""
+    base = synth.WORKLOADS["both_d128_L2048"]
+    wl = synth.shrink(base, B=2, H=4, L=L, d=d, head_place=hp, seed=501 + L + d + hp)
+    inp = synth.make_attn_inputs(wl)
+    assert_close(run_attn(wl, inp, path), oracle_full(wl, inp), "bf16")
+
+
+@pytest.mark.parametrize("hp,L", [(synth.POST, 300), (synth.OFF, 130)])
+def test_post_conv_exact_indicator_kq(hp, L):
+    base = synth.WORKLOADS["both_d128_L2048"]
+    wl = synth.shrink(base, B=1, H=4, L=L, d=128, head_place=hp, kq_place=mta.PRE_EXACT, seed=601 + L)
+    inp = synth.make_attn_inputs(wl)
+    assert_close(run_attn(wl, inp, mta.PATH_KQ), oracle_full(wl, inp), "bf16")
+
+
+def test_post_conv_causality_kq():
+    base = synth.WORKLOADS["both_d128_L2048"]
+    wl = synth.shrink(base, B=1, H=4, L=400, d=128, seed=457)
+    inp = synth.make_attn_inputs(wl)
+    a = run_attn(wl, inp, mta.PATH_KQ)
+    t = 250
+    for n, s in (("q", 1), ("k", 2), ("v", 3)):
+        x = inp[n].copy()
+        x[:, t:] = synth.round_bf16(synth.normal(97, s, x[:, t:].shape))
+        inp[n] = x
+    b = run_attn(wl, inp, mta.PATH_KQ)
+    assert torch.equal(a[:, :t], b[:, :t])
+    assert not torch.equal(a[:, t:], b[:, t:])
+
+
 def test_post_conv_other_kernel_sizes():
     base = synth.WORKLOADS["both_d128_L2048"]
     wl = synth.shrink(base, B=1, H=8, L=100, d=32, c_q=3, c_k=5, c_h=4, seed=455)

@@ -63,7 +63,7 @@ constexpr int kTmaWarp = 8, kMmaWarp = 9;
 constexpr int kBarAll = 1;      // named barrier over both softmax warpgroups
 constexpr int kKqMaxClusters = 160;  // persistent grid: at most this many CTAs (>= SM count)
 
-template <int D, int CQ, int CK, int MIX, bool EXACT>
+template <int D, int CQ, int CK, int MIX, bool EXACT, bool POST>
 struct KGeo {
   // band 0 <= i-j < W where taps are masked: keys after the shifted query (Mask_0)
   // or after the output query (exact indicator); Vp[i][m] = q[i] . k[i-m+OFF]
@@ -82,7 +82,18 @@ struct KGeo {
   static constexpr int CLUSTER = MIX == 2 ? 2 : 1;       // CTAs of a cluster: the heads of a group
   static constexpr int V_CHUNK = BN * 128;
   static constexpr int V_HEAD = BN * D * 2;
-  static constexpr int V_BYTES = NV * V_HEAD;
+  // with the post-softmax convolution the convolved values stream through the Kt
+  // ring, and the normalised weights go to shared memory (8-key strips, 16-byte
+  // rows, PS_PAD rows of padding above row 0 for the row shifts)
+  static constexpr int V_BYTES = POST ? 0 : NV * V_HEAD;
+  static constexpr int RSH = POST ? HALO : 0;            // rows of a tile above its output rows
+  static constexpr int BMO = BM - RSH;                   // output rows per query tile
+  static constexpr int PS_PAD = 8;
+  static constexpr int PS_STRIP = (BM + PS_PAD) * 16;
+  static constexpr int PS_BYTES = POST ? (BN / 8) * PS_STRIP : 0;
+  static constexpr int DG_BYTES = POST ? BM * C * 4 : 0;   // weights of the c keys ending at the diagonal
+  static constexpr int NVCH = NV * CQ * NDC;              // convolved-value chunks per key tile
+  static constexpr int UB = HALO + 2 * C;                 // diagonals of the near-diagonal value band
   static constexpr int UROWS = BM + HALO;
   static constexpr int U_BYTES = (UROWS * M * 4 + 15) / 16 * 16;
   static constexpr int CS_BYTES = 2 * BM * W * 4;        // band values, one block per warpgroup
@@ -90,17 +101,20 @@ struct KGeo {
   static constexpr int FAC_BYTES = NSRC * 2 * BN * 4;    // column factors of two key tiles, per source head
   static constexpr int Q_ALLOC = (Q_BYTES + 1023) / 1024 * 1024;
   // small area: taps [2 items][NSRC][128], per-warp |q| maxima, barriers, TMEM slot, abort flag
-  static constexpr int TH_OFF = 0, QRED_OFF = 2 * NSRC * 128 * 4, BAR_OFF = QRED_OFF + 64;
+  static constexpr int TH_OFF = 0, THP_OFF = 2 * NSRC * 128 * 4;
+  static constexpr int QRED_OFF = THP_OFF + (POST ? 2 * 128 * 4 : 0), BAR_OFF = QRED_OFF + 64;
   static constexpr int TSLOT_OFF = BAR_OFF + 8 * 32, ABORT_OFF = TSLOT_OFF + 8;
   static constexpr int SMALL_BYTES = (ABORT_OFF + 8 + 255) / 256 * 256;
   // Kt ring: as many 16 KB stages as the shared memory left over holds (at most 8)
-  static constexpr int REST = NSRC * Q_ALLOC + V_BYTES + NSRC * U_BYTES + CS_BYTES + RED_BYTES +
-                              FAC_BYTES + SMALL_BYTES + 1024;
+  static constexpr int REST = NSRC * Q_ALLOC + V_BYTES + PS_BYTES + DG_BYTES + NSRC * U_BYTES + CS_BYTES +
+                              RED_BYTES + FAC_BYTES + SMALL_BYTES + 1024;
   static constexpr int NS = (232448 - REST) / KCHUNK < 8 ? (232448 - REST) / KCHUNK : 8;
   static constexpr int OFF_Q = 0;
   static constexpr int OFF_K = NSRC * Q_ALLOC;
   static constexpr int OFF_V = OFF_K + NS * KCHUNK;
-  static constexpr int OFF_U = OFF_V + V_BYTES;
+  static constexpr int OFF_PS = OFF_V + V_BYTES;
+  static constexpr int OFF_DG = OFF_PS + PS_BYTES;
+  static constexpr int OFF_U = OFF_DG + DG_BYTES;
   static constexpr int OFF_CS = OFF_U + NSRC * U_BYTES;
   static constexpr int OFF_RED = OFF_CS + CS_BYTES;
   static constexpr int OFF_FAC = OFF_RED + RED_BYTES;
@@ -110,10 +124,12 @@ struct KGeo {
   // allocation never waits for another CTA
   static constexpr int SMEM = SMEM_USED > 232448 / 2 + 1024 ? SMEM_USED : 232448 / 2 + 1024;
   // tensor memory: C of each source head (128 columns each), P (64), Z
-  static constexpr uint32_t TMEM_COLS = 512, C_COL = 0, P_COL = 128 * NSRC, Z_COL0 = P_COL + 128;
+  static constexpr uint32_t TMEM_COLS = 512, C_COL = 0, P_COL = 128 * NSRC;
+  static constexpr uint32_t Z_COL0 = POST ? P_COL : P_COL + 128;  // P lives in shared memory with POST
   static_assert(Z_COL0 + 128 * (NV - 1) + D <= TMEM_COLS, "tensor memory");
   static_assert(MIX != 1 || NV == 1, "pre-softmax mixing uses the destination head's V only");
   static_assert(OFF_K % 1024 == 0 && OFF_V % 1024 == 0, "swizzle alignment");
+  static_assert(OFF_PS % 16 == 0 && OFF_DG % 16 == 0 && OFF_U % 16 == 0, "alignment");
   static_assert(OFF_SMALL % 16 == 0, "alignment");
   static_assert(NS >= 3, "Kt ring");
   static_assert(11 + 2 * NS <= 32, "barrier slots");
@@ -135,6 +151,10 @@ struct KqParams {
   const float *vp;      // [B][H][L][M] past dot products
   float *xg;            // post-softmax mixing exchange: [CTA][2][D/4][BM] float4
   unsigned *err;
+  // post-softmax convolution: its kernels and the values (for the band near the diagonal)
+  const float *theta_post;    // [H][CQ][CK]
+  const __nv_bfloat16 *v;     // [B][L][H][D], token stride rs
+  long long rs;
 };
 
 template <int N>
@@ -167,22 +187,26 @@ __device__ __forceinline__ int item_index(int c, int r, int n_clusters) {
   return r * n_clusters + ((r & 1) ? n_clusters - 1 - c : c);
 }
 
-template <int D, int CQ, int CK, int MIX, bool EXACT>
+template <int D, int CQ, int CK, int MIX, bool EXACT, bool POST>
 __global__ void __launch_bounds__(kThreads, 1)
     attn_kq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
-                   const __grid_constant__ CUtensorMap tmV, const KqParams p) {
-  using G = KGeo<D, CQ, CK, MIX, EXACT>;
+                   const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmVt,
+                   const KqParams p) {
+  using G = KGeo<D, CQ, CK, MIX, EXACT, POST>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t *Qs = smem + G::OFF_Q;
   uint8_t *Ks = smem + G::OFF_K;
   uint8_t *Vs = smem + G::OFF_V;
+  uint8_t *Ps = smem + G::OFF_PS;                                // normalised weights (POST)
+  float *Dg = reinterpret_cast<float *>(smem + G::OFF_DG);       // [BM][C] near-diagonal weights (POST)
   float *Us = reinterpret_cast<float *>(smem + G::OFF_U);
   float *Cs = reinterpret_cast<float *>(smem + G::OFF_CS);
   float *red = reinterpret_cast<float *>(smem + G::OFF_RED);
   float *facs = reinterpret_cast<float *>(smem + G::OFF_FAC);  // [NSRC][2][BN]
   uint8_t *small = smem + G::OFF_SMALL;
   float *th_s = reinterpret_cast<float *>(small + G::TH_OFF);   // [2 items][NSRC][128]
+  float *thp_s = reinterpret_cast<float *>(small + G::THP_OFF); // [2 items][128] post-softmax taps
   float *qred = reinterpret_cast<float *>(small + G::QRED_OFF); // [8] per-warp max |q|
   uint64_t *bars = reinterpret_cast<uint64_t *>(small + G::BAR_OFF);
   uint64_t *q_full = bars + 0, *q_ready = bars + 1, *q_free = bars + 2, *z_free = bars + 3;
@@ -207,7 +231,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     it = item_of(k, p.B, n_groups, p.n_qtiles);
     return true;
   };
-  auto kv_tiles = [&](const Item &it) { return min(L - 1, it.qt * G::BM + G::BM - 1) / G::BN + 1; };
+  // first query row of an item's tile (with POST, its c_q-1 rows above the output rows)
+  auto row_start = [&](const Item &it) { return it.qt * G::BMO - G::RSH; };
+  auto kv_tiles = [&](const Item &it) { return min(L - 1, row_start(it) + G::BM - 1) / G::BN + 1; };
+  // key-tile passes of an item: one, or two with POST (exact row statistics first)
+  auto n_slots = [&](const Item &it) { return POST ? 2 * kv_tiles(it) : kv_tiles(it); };
   // the head whose C is accumulated as source s of destination head h
   auto src_head = [&](int h, int s) { return G::NSRC == 2 ? (h & ~1) + s : h; };
 
@@ -220,6 +248,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     *abort_flag = 0;
     fence_mbar_init();
   }
+  if constexpr (POST) {  // padding rows above the weights (read only for rows that are not output)
+    for (int i = threadIdx.x; i < (G::BN / 8) * G::PS_PAD * 4; i += kThreads)
+      reinterpret_cast<uint32_t *>(Ps + (i / (G::PS_PAD * 4)) * G::PS_STRIP)[i % (G::PS_PAD * 4)] = 0u;
+  }
   if (warp == kMmaWarp) { tmem_alloc(tslot, G::TMEM_COLS); tmem_relinquish(); }
   tc_fence_before();
   __syncthreads();
@@ -229,25 +261,49 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (warp == kTmaWarp) {
     // -------------------------------------------------------------- TMA
-    if (lane == 0) {  // Kt chunks of every key tile of every item, through the ring
+    if (lane == 0) {  // Kt chunks (and with POST the convolved values), through the ring
       prefetch_tmap(&tmK);
+      if (POST) prefetch_tmap(&tmVt);
       int cnt = 0;
+      auto push = [&](const CUtensorMap *map, int x, int y, int z) -> bool {
+        const int st = cnt % G::NS;
+        if (!mbar_wait(k_empty + st, ((cnt / G::NS) & 1) ^ 1, abort_flag, p.err)) return false;
+        mbar_arrive_expect_tx(k_full + st, G::KCHUNK);
+        tma_load_3d(Ks + st * G::KCHUNK, map, k_full + st, x, y, z);
+        ++cnt;
+        return true;
+      };
       Item it;
-      for (int r = 0; item_at(r, it) && !*abort_flag; ++r) {
-        const int h = it.g * CL + hr, n_kv = kv_tiles(it);
-        for (int t = 0; t < n_kv && !*abort_flag; ++t)
-          for (int ch = 0; ch < G::NSRC * G::NCH; ++ch, ++cnt) {
-            const int st = cnt % G::NS, sc = ch / G::NCH, cs = ch % G::NCH;
+      bool ok = true;
+      for (int r = 0; ok && item_at(r, it) && !*abort_flag; ++r) {
+        const int h = it.g * CL + hr, n_kv = kv_tiles(it), nsl = n_slots(it);
+        auto load_c = [&](int t) -> bool {
+          for (int ch = 0; ch < G::NSRC * G::NCH; ++ch) {
+            const int sc = ch / G::NCH, cs = ch % G::NCH;
             const int zbase = (it.b * p.H + src_head(h, sc)) * CQ;
-            if (!mbar_wait(k_empty + st, ((cnt / G::NS) & 1) ^ 1, abort_flag, p.err)) break;
-            mbar_arrive_expect_tx(k_full + st, G::KCHUNK);
-            tma_load_3d(Ks + st * G::KCHUNK, &tmK, k_full + st, (cs % G::NDC) * 64, t * G::BN, zbase + cs / G::NDC);
+            if (!push(&tmK, (cs % G::NDC) * 64, t * G::BN, zbase + cs / G::NDC)) return false;
           }
+          return true;
+        };
+        auto load_pv = [&](int t) -> bool {  // chunk (value head hd, tap row a, 64-channel block dc)
+          for (int ch = 0; ch < G::NVCH; ++ch) {
+            const int hd = ch / (CQ * G::NDC), a = (ch / G::NDC) % CQ, dc = ch % G::NDC;
+            const int z = ((it.b * p.H + h) * G::NV + hd) * CQ + a;
+            if (!push(&tmVt, dc * 64, t * G::BN, z)) return false;
+          }
+          return true;
+        };
+        // the order the MMA issuer consumes: C of slot s+1 before P V of slot s
+        for (int sl = 0; ok && sl < nsl && !*abort_flag; ++sl) {
+          ok = load_c(sl % n_kv);
+          if (POST && ok && sl >= n_kv + 1) ok = load_pv(sl - 1 - n_kv);
+        }
+        if (POST && ok && !*abort_flag) ok = load_pv(n_kv - 1);
       }
       if (*abort_flag)  // copies still in flight land before the CTA exits
         for (int c2 = (cnt > G::NS ? cnt - G::NS : 0); c2 < cnt; ++c2)
           drain_wait(k_full + c2 % G::NS, (c2 / G::NS) & 1);
-    } else if (lane == 1) {  // V of both heads of the group, per key tile
+    } else if (lane == 1 && !POST) {  // V of both heads of the group, per key tile
       prefetch_tmap(&tmV);
       int nv = 0;
       Item it;
@@ -271,7 +327,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       Item it;
       for (int r = 0; item_at(r, it) && !*abort_flag; ++r, ++nq) {
         if (r > 0 && !mbar_wait(q_free, (r - 1) & 1, abort_flag, p.err)) break;
-        const int h = it.g * CL + hr, row0 = it.qt * G::BM - G::HALO;
+        const int h = it.g * CL + hr, row0 = row_start(it) - G::HALO;
         mbar_arrive_expect_tx(q_full, G::NSRC * G::Q_BYTES);
 #pragma unroll 1
         for (int sc = 0; sc < G::NSRC; ++sc)
@@ -291,7 +347,13 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint64_t qdesc0 = sdesc_noswz(smem_u32(Qs), G::STRIP, 128);
       const uint64_t kdesc0 = sdesc_sw128(smem_u32(Ks), 16, 1024);
       const uint64_t vdesc0 = sdesc_sw128(smem_u32(Vs), G::V_CHUNK, 1024);
-      int cnt = 0, T = 0;  // Kt chunks and key tiles issued so far (all items)
+      // POST: weights in shared memory (row shift a = 16a bytes earlier) times the
+      // convolved values in the ring (N = 64 channels per chunk)
+      const uint32_t idesc_pv64 = idesc_bf16_f32(128, 64, 0, 1);
+      const uint64_t psdesc0 = sdesc_noswz(smem_u32(Ps), G::PS_STRIP, 128);
+      const uint64_t vtdesc0 = sdesc_sw128(smem_u32(Ks), G::KCHUNK, 1024);  // a ring stage as MN-major B
+      int cnt = 0, T = 0;  // ring chunks and C tiles issued so far (all items)
+      int npv = 0;         // P V tiles issued (POST)
       bool ok = true;
       // C of global key tile T = sum over the NCH chunks (a, 64-wide d block) of Q
       // shifted by a rows x Kt_a
@@ -316,33 +378,62 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (last_of_item) mma_commit(q_free);  // the query buffer may take the next item
         return true;
       };
+      // Z_hd += sum_a (weights shifted down by a rows) x Vt_{hd,a}, from the ring
+      auto issue_pv = [&](bool first_of_item) -> bool {
+        for (int ch = 0; ch < G::NVCH; ++ch, ++cnt) {
+          const int st = cnt % G::NS;
+          if (!mbar_wait(k_full + st, (cnt / G::NS) & 1, abort_flag, p.err)) return false;
+          tc_fence_after();
+          const int hd = ch / (CQ * G::NDC), a = (ch / G::NDC) % CQ, dc = ch % G::NDC;
+          const uint64_t pd = psdesc0 + static_cast<uint32_t>(G::PS_PAD - a);
+          const uint64_t vd = vtdesc0 + static_cast<uint32_t>((st * G::KCHUNK) >> 4);
+#pragma unroll
+          for (int kk = 0; kk < G::BN / 16; ++kk)
+            mma_bf16_ss(tmem + G::Z_COL0 + 128 * hd + 64 * dc, pd + static_cast<uint32_t>((2 * kk * G::PS_STRIP) >> 4),
+                        vd + static_cast<uint32_t>((kk * 16 * 128) >> 4), idesc_pv64,
+                        !(first_of_item && a == 0 && kk == 0));
+          mma_commit(k_empty + st);
+        }
+        mma_commit(v_empty);
+        return true;
+      };
       Item it;
       for (int r = 0; ok && item_at(r, it); ++r) {
-        const int n_kv = kv_tiles(it);
+        const int n_kv = kv_tiles(it), nsl = n_slots(it);
         if (!mbar_wait(q_ready, r & 1, abort_flag, p.err)) break;
         const int T0 = T;
-        ok = issue_c(n_kv == 1);
-        for (int t = 0; ok && t < n_kv; ++t) {
-          const int Tt = T0 + t;
-          if (t + 1 < n_kv) {
+        ok = issue_c(nsl == 1);
+        for (int sl = 0; ok && sl < nsl; ++sl) {
+          const int Tt = T0 + sl;
+          if (sl + 1 < nsl) {
             T = Tt + 1;
-            if (!issue_c(t + 2 == n_kv)) { ok = false; break; }
+            if (!issue_c(sl + 2 == nsl)) { ok = false; break; }
           }
-          if (!mbar_wait(p_full, Tt & 1, abort_flag, p.err)) { ok = false; break; }
-          if (!mbar_wait(v_full, Tt & 1, abort_flag, p.err)) { ok = false; break; }
-          // Z is overwritten (accumulate off) by the first P V of an item: the previous
-          // item's epilogue must have read it
-          if (t == 0 && r > 0 && !mbar_wait(z_free, (r - 1) & 1, abort_flag, p.err)) { ok = false; break; }
-          tc_fence_after();
+          if constexpr (POST) {
+            if (sl < n_kv) continue;  // first pass: statistics only
+            if (!mbar_wait(p_full, npv & 1, abort_flag, p.err)) { ok = false; break; }
+            if (sl == n_kv && r > 0 && !mbar_wait(z_free, (r - 1) & 1, abort_flag, p.err)) { ok = false; break; }
+            tc_fence_after();
+            if (!issue_pv(sl == n_kv)) { ok = false; break; }
+            ++npv;
+          } else {
+            const int t = sl;
+            if (!mbar_wait(p_full, Tt & 1, abort_flag, p.err)) { ok = false; break; }
+            if (!mbar_wait(v_full, Tt & 1, abort_flag, p.err)) { ok = false; break; }
+            // Z is overwritten (accumulate off) by the first P V of an item: the previous
+            // item's epilogue must have read it
+            if (t == 0 && r > 0 && !mbar_wait(z_free, (r - 1) & 1, abort_flag, p.err)) { ok = false; break; }
+            tc_fence_after();
 #pragma unroll
-          for (int hd = 0; hd < G::NV; ++hd)
+            for (int hd = 0; hd < G::NV; ++hd)
 #pragma unroll
-            for (int kk = 0; kk < G::BN / 16; ++kk)
-              mma_f16_ts(tmem + G::Z_COL0 + 128 * hd, tmem + G::P_COL + 8 * kk,
-                         vdesc0 + ((hd * G::V_HEAD + kk * 16 * 128) >> 4), idesc_pv, (t > 0 || kk > 0));
-          mma_commit(v_empty);
+              for (int kk = 0; kk < G::BN / 16; ++kk)
+                mma_f16_ts(tmem + G::Z_COL0 + 128 * hd, tmem + G::P_COL + 8 * kk,
+                           vdesc0 + ((hd * G::V_HEAD + kk * 16 * 128) >> 4), idesc_pv, (t > 0 || kk > 0));
+            mma_commit(v_empty);
+          }
         }
-        T = T0 + n_kv;
+        T = T0 + nsl;
       }
       mma_commit(mma_done);
       drain_wait(mma_done, 0);
@@ -362,7 +453,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     // |q| > 2^14), the past dot products of its staged rows and its kernel taps.
     // Returns the query exponent.
     auto prepare = [&](int r, const Item &it) -> int {
-      const int h = it.g * CL + hr, row0 = it.qt * G::BM - G::HALO;
+      const int h = it.g * CL + hr, row0 = row_start(it) - G::HALO;
       mbar_wait(q_full, r & 1, abort_flag, p.err);
       float qmax = 0.f;
       // (the query tiles of the source heads lie Q_ALLOC = Q_BYTES apart)
@@ -410,10 +501,13 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (st_id < CQ * CK)
           th_s[((r & 1) * G::NSRC + sc) * 128 + st_id] = p.theta[static_cast<long long>(hs) * CQ * CK + st_id];
       }
+      if (POST && st_id < CQ * CK)  // the post-softmax kernel of this CTA's head
+        thp_s[(r & 1) * 128 + st_id] = p.theta_post[static_cast<long long>(h) * CQ * CK + st_id];
       return eq;
     };
 
-    int T = 0;  // key tiles processed so far (all items)
+    int T = 0;   // C tiles processed so far (all items, both passes with POST)
+    int NP = 0;  // weight tiles handed to the P V issuer so far (POST)
     Item it, nx;
     bool have = item_at(0, it);
     int eq = 0;
@@ -428,14 +522,17 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     for (int r = 0; have; ++r) {
       const int h = it.g * CL + hr, g = it.g;
-      const int i0 = it.qt * G::BM, qi = i0 + r_;
-      const bool out_row = qi < L;
-      const int n_kv = kv_tiles(it);
+      const int R0 = row_start(it), qi = R0 + r_;
+      const bool row_ok = qi >= 0 && qi < L;          // a query of the sequence
+      const bool out_row = row_ok && r_ >= G::RSH;     // an output row of this tile
+      const int n_kv = kv_tiles(it), nsl = n_slots(it);
       const bool more = item_at(r + 1, nx);
       const int h_nx = nx.g * CL + hr;
-      // column factors of source s for the key tile after t (this item's or the next item's first)
-      auto fac_next = [&](int sc, int t) -> float {
-        if (t + 1 < n_kv) return p.fac[(static_cast<long long>(it.b) * p.H + src_head(h, sc)) * p.lpad + (t + 1) * G::BN + st_id];
+      // column factors of source s for the key tile of the slot after sl (this
+      // item's or the next item's first)
+      auto fac_next = [&](int sc, int sl) -> float {
+        if (sl + 1 < nsl)
+          return p.fac[(static_cast<long long>(it.b) * p.H + src_head(h, sc)) * p.lpad + ((sl + 1) % n_kv) * G::BN + st_id];
         if (more) return p.fac[(static_cast<long long>(nx.b) * p.H + src_head(h_nx, sc)) * p.lpad + st_id];
         return 0.f;
       };
@@ -444,13 +541,51 @@ __global__ void __launch_bounds__(kThreads, 1)
       float wmix[G::NSRC];
 #pragma unroll
       for (int sc = 0; sc < G::NSRC; ++sc) wmix[sc] = G::NSRC == 2 ? p.w[(h >> 1) * 4 + (h & 1) * 2 + sc] : 1.f;
+      // the band 0 <= i-j < W, where the mask removes taps: the convolution tap by
+      // tap over the kept taps, from the dot products (key (i-a) - m, m = dd - a + t - c):
+      //   Mask_0: taps with m >= 0; exact indicator: taps with key <= i, i.e. t >= c - dd
+      //   C[i][i-dd] = s * sum_{kept a,t} theta[a][t] q[i-a] . k[i-a-m]   (acc[dd] / s)
+      auto band_acc = [&](float (&acc)[G::W]) {
+#pragma unroll
+        for (int dd = 0; dd < G::W; ++dd) acc[dd] = 0.f;
+#pragma unroll
+        for (int sc = 0; sc < G::NSRC; ++sc)
+#pragma unroll
+        for (int a = 0; a < CQ; ++a) {
+          // rows before query 0 are zero; the source's taps carry its mixing weight
+          const float *vrow = Us + sc * (G::U_BYTES / 4) + (r_ + G::HALO - a) * G::M;
+          const float *th = th_s + ((r & 1) * G::NSRC + sc) * 128;
+          float vr[G::M];
+#pragma unroll
+          for (int m = 0; m < G::M; ++m) vr[m] = vrow[m];
+#pragma unroll
+          for (int tp = 0; tp < CK; ++tp) {
+            const float thv = th[a * CK + tp] * wmix[sc];
+#pragma unroll
+            for (int dd = 0; dd < G::W; ++dd) {
+              const int m = dd - a + tp - G::C;
+              const bool kept = EXACT ? tp >= G::C - dd : m >= 0;
+              if (kept && m + G::OFF >= 0 && m + G::OFF < G::M) acc[dd] = fmaf(thv, vr[m + G::OFF], acc[dd]);
+            }
+          }
+        }
+      };
       float m_run = -INFINITY, l_run = 0.f;
-      for (int t = 0; t < n_kv; ++t, ++T) {
+      float mm = INFINITY;  // POST: log2 of (row max x row sum), final after the first pass
+      for (int sl = 0; sl < nsl; ++sl, ++T) {
+        const int t = POST ? sl % n_kv : sl;
+        const bool pass2 = POST && sl >= n_kv;
         const int j0 = t * G::BN;
+        if (POST && sl == n_kv) {  // exact statistics of the row: one normaliser for the second pass
+          red[(4 + wg) * G::BM + r_] = l_run;
+          named_bar_sync(kBarAll, kSmThreads);
+          const float l_tot = l_run + red[(4 + (wg ^ 1)) * G::BM + r_];
+          mm = (row_ok && l_tot > 0.f) ? m_run + log2f(l_tot) : INFINITY;
+        }
         // next key tile's column factors (stored before this tile's barrier, read after it)
         float fnext[G::NSRC];
 #pragma unroll
-        for (int sc = 0; sc < G::NSRC; ++sc) fnext[sc] = st_id < G::BN ? fac_next(sc, t) : 0.f;
+        for (int sc = 0; sc < G::NSRC; ++sc) fnext[sc] = st_id < G::BN ? fac_next(sc, sl) : 0.f;
         mbar_wait(c_full, T & 1, abort_flag, p.err);
         tc_fence_after();
         // C' = sum over source heads of w * (C_s x its column factors); one source without mixing
@@ -487,36 +622,10 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
           for (int jj = 0; jj < G::HALF; ++jj) cv[jj] *= qinv;
         }
-        // the band 0 <= i-j < W, where the mask removes taps: the convolution tap by
-        // tap over the kept taps, from the dot products (key (i-a) - m, m = dd - a + t - c):
-        //   Mask_0: taps with m >= 0; exact indicator: taps with key <= i, i.e. t >= c - dd
-        //   C[i][i-dd] = s * sum_{kept a,t} theta[a][t] q[i-a] . k[i-a-m]
         const int dmax = qi - j0 - cb;  // i - j for this warpgroup's first column
-        if (out_row && dmax >= 0 && dmax - (G::W - 1) < G::HALF) {
+        if (row_ok && dmax >= 0 && dmax - (G::W - 1) < G::HALF) {
           float acc[G::W];
-#pragma unroll
-          for (int dd = 0; dd < G::W; ++dd) acc[dd] = 0.f;
-#pragma unroll
-          for (int sc = 0; sc < G::NSRC; ++sc)
-#pragma unroll
-          for (int a = 0; a < CQ; ++a) {
-            // rows before query 0 are zero; the source's taps carry its mixing weight
-            const float *vrow = Us + sc * (G::U_BYTES / 4) + (r_ + G::HALO - a) * G::M;
-            const float *th = th_s + ((r & 1) * G::NSRC + sc) * 128;
-            float vr[G::M];
-#pragma unroll
-            for (int m = 0; m < G::M; ++m) vr[m] = vrow[m];
-#pragma unroll
-            for (int tp = 0; tp < CK; ++tp) {
-              const float thv = th[a * CK + tp] * wmix[sc];
-#pragma unroll
-              for (int dd = 0; dd < G::W; ++dd) {
-                const int m = dd - a + tp - G::C;
-                const bool kept = EXACT ? tp >= G::C - dd : m >= 0;
-                if (kept && m + G::OFF >= 0 && m + G::OFF < G::M) acc[dd] = fmaf(thv, vr[m + G::OFF], acc[dd]);
-              }
-            }
-          }
+          band_acc(acc);
 #pragma unroll
           for (int dd = 0; dd < G::W; ++dd) crow[dd] = acc[dd] * sc0;
 #pragma unroll
@@ -525,75 +634,179 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (static_cast<unsigned>(dd) < static_cast<unsigned>(G::W)) cv[jj] = crow[dd];
           }
         }
-        // Mask_-inf (only the diagonal tile holds keys after a query) and the row max
-        // over both warpgroups' columns (log2 units)
-        if (t == n_kv - 1) {
+        // Mask_-inf: keys after the query (only tiles reaching past the tile's first row)
+        if (j0 + G::BN - 1 > R0) {
 #pragma unroll
           for (int jj = 0; jj < G::HALF; ++jj)
             if (j0 + cb + jj > qi) cv[jj] = -INFINITY;
         }
-        float *rmx = red + (T & 1) * 2 * G::BM;
-        rmx[wg * G::BM + r_] = out_row ? tree_max<G::HALF>(cv) : -INFINITY;
-        if (st_id < G::BN)
+        if (!pass2) {
+          // the row max over both warpgroups' columns (log2 units)
+          float *rmx = red + (T & 1) * 2 * G::BM;
+          rmx[wg * G::BM + r_] = row_ok ? tree_max<G::HALF>(cv) : -INFINITY;
+          if (st_id < G::BN)
 #pragma unroll
-          for (int sc = 0; sc < G::NSRC; ++sc) facs[(sc * 2 + ((T + 1) & 1)) * G::BN + st_id] = fnext[sc];
-        named_bar_sync(kBarAll, kSmThreads);
-        const float mt = fmaxf(rmx[r_], rmx[G::BM + r_]);
-        const float m_new = fmaxf(m_run, mt);
-        bool resc = false;
-        float alpha = 1.f;
-        if (t == 0) {
-          m_run = m_new;
-        } else if (m_new > m_run + kRescaleLog2) {
-          resc = true;
-          alpha = ex2(m_run - m_new);
-          m_run = m_new;
-        }
-        if (T > 0) {  // P and Z of the previous key tile are consumed / complete
-          mbar_wait(v_empty, (T - 1) & 1, abort_flag, p.err);
-          tc_fence_after();
-        }
-        if (__any_sync(0xffffffffu, resc)) {  // warp-collective tensor-memory access
-          l_run *= alpha;
-#pragma unroll 1
-          for (int hd = 0; hd < G::NV; ++hd)
-#pragma unroll 1
-            for (int c0 = 0; c0 < G::DH; c0 += 32) {
-              uint32_t z[32];
-              const uint32_t za = tl + G::Z_COL0 + 128 * hd + zc + c0;
-              tmem_ld32(za, z);
-              tmem_wait_ld();
+            for (int sc = 0; sc < G::NSRC; ++sc) facs[(sc * 2 + ((T + 1) & 1)) * G::BN + st_id] = fnext[sc];
+          named_bar_sync(kBarAll, kSmThreads);
+          const float mt = fmaxf(rmx[r_], rmx[G::BM + r_]);
+          const float m_new = fmaxf(m_run, mt);
+          if constexpr (POST) {  // first pass: row sums only
+            if (m_new != -INFINITY) {
+              float ls = 0.f;
 #pragma unroll
-              for (int i = 0; i < 32; ++i) z[i] = __float_as_uint(__uint_as_float(z[i]) * alpha);
-              tmem_st32(za, z);
+              for (int jj = 0; jj < G::HALF; ++jj) ls += ex2(cv[jj] - m_new);
+              l_run = l_run * ex2(m_run - m_new) + ls;
+              m_run = m_new;
             }
-        }
-        float ls = 0.f;
-        uint32_t pk[32];
+          } else {
+            bool resc = false;
+            float alpha = 1.f;
+            if (t == 0) {
+              m_run = m_new;
+            } else if (m_new > m_run + kRescaleLog2) {
+              resc = true;
+              alpha = ex2(m_run - m_new);
+              m_run = m_new;
+            }
+            if (T > 0) {  // P and Z of the previous key tile are consumed / complete
+              mbar_wait(v_empty, (T - 1) & 1, abort_flag, p.err);
+              tc_fence_after();
+            }
+            if (__any_sync(0xffffffffu, resc)) {  // warp-collective tensor-memory access
+              l_run *= alpha;
+#pragma unroll 1
+              for (int hd = 0; hd < G::NV; ++hd)
+#pragma unroll 1
+                for (int c0 = 0; c0 < G::DH; c0 += 32) {
+                  uint32_t z[32];
+                  const uint32_t za = tl + G::Z_COL0 + 128 * hd + zc + c0;
+                  tmem_ld32(za, z);
+                  tmem_wait_ld();
 #pragma unroll
-        for (int q2 = 0; q2 < 32; ++q2) {
-          const float p0 = out_row ? ex2(cv[2 * q2] - m_run) : 0.f;
-          const float p1 = out_row ? ex2(cv[2 * q2 + 1] - m_run) : 0.f;
-          ls += p0 + p1;
-          pk[q2] = pack_bf16x2(p0, p1);
+                  for (int i = 0; i < 32; ++i) z[i] = __float_as_uint(__uint_as_float(z[i]) * alpha);
+                  tmem_st32(za, z);
+                }
+            }
+            float ls = 0.f;
+            uint32_t pk[32];
+#pragma unroll
+            for (int q2 = 0; q2 < 32; ++q2) {
+              const float p0 = row_ok ? ex2(cv[2 * q2] - m_run) : 0.f;
+              const float p1 = row_ok ? ex2(cv[2 * q2 + 1] - m_run) : 0.f;
+              ls += p0 + p1;
+              pk[q2] = pack_bf16x2(p0, p1);
+            }
+            tmem_st32(tl + G::P_COL + 32 * wg, pk);
+            l_run += ls;
+            tmem_wait_st();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(p_full);
+          }
+        } else {
+          // second pass: normalised weights A = 2^(C - mm); the c keys ending at the
+          // diagonal go through the band below (their convolved values would reach
+          // past the query), so they are 0 here
+          if (st_id < G::BN)
+#pragma unroll
+            for (int sc = 0; sc < G::NSRC; ++sc) facs[(sc * 2 + ((T + 1) & 1)) * G::BN + st_id] = fnext[sc];
+          named_bar_sync(kBarAll, kSmThreads);
+          const bool cut = j0 + G::BN - 1 > R0 - G::C;
+          uint32_t pk[32];
+#pragma unroll
+          for (int q2 = 0; q2 < 32; ++q2) {
+            float p0 = ex2(cv[2 * q2] - mm), p1 = ex2(cv[2 * q2 + 1] - mm);
+            if (cut) {
+              if (j0 + cb + 2 * q2 > qi - G::C) p0 = 0.f;
+              if (j0 + cb + 2 * q2 + 1 > qi - G::C) p1 = 0.f;
+            }
+            pk[q2] = pack_bf16x2(p0, p1);
+          }
+          if (NP > 0) mbar_wait(v_empty, (NP - 1) & 1, abort_flag, p.err);  // the previous P V read the buffer
+          uint8_t *prow = Ps + (cb / 8) * G::PS_STRIP + 16 * (r_ + G::PS_PAD);
+#pragma unroll
+          for (int k8 = 0; k8 < G::HALF / 8; ++k8)
+            *reinterpret_cast<uint4 *>(prow + k8 * G::PS_STRIP) =
+                make_uint4(pk[4 * k8], pk[4 * k8 + 1], pk[4 * k8 + 2], pk[4 * k8 + 3]);
+          fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(p_full);
+          ++NP;
         }
-        tmem_st32(tl + G::P_COL + 32 * wg, pk);
-        l_run += ls;
-        tmem_wait_st();
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(p_full);
+      }
+      if constexpr (POST) {
+        // normalised weights of the c keys ending at each row's diagonal, for the band
+        if (wg == 0) {
+          float acc[G::W];
+          band_acc(acc);
+#pragma unroll
+          for (int dl = 0; dl < G::C; ++dl)
+            Dg[r_ * G::C + dl] = (row_ok && qi - dl >= 0) ? ex2(acc[dl] * sc0 - mm) : 0.f;
+        }
       }
       // the next item's queries, dot products and taps, while this item's last P V runs
       const int eq_next = more ? prepare(r + 1, nx) : 0;
 
       // ---------------------------------------------------------- epilogue
-      mbar_wait(v_empty, (T - 1) & 1, abort_flag, p.err);
+      mbar_wait(v_empty, ((POST ? NP : T) - 1) & 1, abort_flag, p.err);
       tc_fence_after();
-      red[(4 + wg) * G::BM + r_] = l_run;
-      named_bar_sync(kBarAll, kSmThreads);
-      const float l_tot = l_run + red[(4 + (wg ^ 1)) * G::BM + r_];
-      const float inv_l = (out_row && l_tot > 0.f) ? 1.f / l_tot : 0.f;
+      float inv_l = 1.f;
+      // POST: the band near the diagonal, sum_u Gb[u] v[i-u] (u < UB), with
+      //   Gb[u] = sum over tap rows a, diagonal offsets dl < c and taps t with
+      //           a + dl + c - t = u of theta_post[a][t] A[i-a][i-a-dl]
+      float Gb[G::UB];
+#pragma unroll
+      for (int u = 0; u < G::UB; ++u) Gb[u] = 0.f;
+      if constexpr (POST) {
+        named_bar_sync(kBarAll, kSmThreads);  // every row's Dg is written
+        if (out_row) {
+          const float *tp = thp_s + (r & 1) * 128;
+#pragma unroll
+          for (int a = 0; a < CQ; ++a)
+#pragma unroll
+            for (int dl = 0; dl < G::C; ++dl) {
+              const float pv = Dg[(r_ - a) * G::C + dl];
+#pragma unroll
+              for (int tq = 0; tq < CK; ++tq) {
+                const int u = a + dl + G::C - tq;
+                if (u >= 0 && u < G::UB) Gb[u] = fmaf(tp[a * CK + tq], pv, Gb[u]);
+              }
+            }
+        }
+      } else {
+        red[(4 + wg) * G::BM + r_] = l_run;
+        named_bar_sync(kBarAll, kSmThreads);
+        const float l_tot = l_run + red[(4 + (wg ^ 1)) * G::BM + r_];
+        inv_l = (out_row && l_tot > 0.f) ? 1.f / l_tot : 0.f;
+      }
+      // 32 output channels zc+c0 .. of head vh: Z (times 1/l) plus, with POST, the band
+      auto z_chunk = [&](int hd, int vh, int c0, float (&zo)[32]) {
+        uint32_t z[32];
+        tmem_ld32(tl + G::Z_COL0 + 128 * hd + zc + c0, z);
+        tmem_wait_ld();
+#pragma unroll
+        for (int i = 0; i < 32; ++i) zo[i] = __uint_as_float(z[i]) * inv_l;
+        if constexpr (POST) {
+          if (out_row) {
+#pragma unroll
+            for (int u = 0; u < G::UB; ++u) {
+              if (qi - u < 0) break;
+              const uint4 *vr = reinterpret_cast<const uint4 *>(
+                  p.v + (static_cast<long long>(it.b) * L + (qi - u)) * p.rs + static_cast<long long>(vh) * D + zc + c0);
+#pragma unroll
+              for (int q8 = 0; q8 < 4; ++q8) {
+                const uint4 w4 = vr[q8];
+                const uint32_t wv[4] = {w4.x, w4.y, w4.z, w4.w};
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                  zo[8 * q8 + 2 * e] = fmaf(Gb[u], __uint_as_float(wv[e] << 16), zo[8 * q8 + 2 * e]);
+                  zo[8 * q8 + 2 * e + 1] = fmaf(Gb[u], __uint_as_float(wv[e] & 0xffff0000u), zo[8 * q8 + 2 * e + 1]);
+                }
+              }
+            }
+          }
+        }
+      };
       float o[G::DH];
       if constexpr (MIX == 2) {
         // Z_{h->peer} / l_h goes to the peer through L2: [parity][column/4][row] float4
@@ -602,23 +815,19 @@ __global__ void __launch_bounds__(kThreads, 1)
                                (static_cast<long long>(2 * c + (hr ^ 1)) * 2 + (r & 1)) * (G::BM * D / 4);
 #pragma unroll
         for (int c0 = 0; c0 < G::DH; c0 += 32) {
-          uint32_t z[32];
-          tmem_ld32(tl + G::Z_COL0 + 128 * (hr ^ 1) + zc + c0, z);
-          tmem_wait_ld();
+          float zo[32];
+          z_chunk(hr ^ 1, 2 * g + (hr ^ 1), c0, zo);
 #pragma unroll
           for (int i = 0; i < 32; i += 4)
-            mine[((zc + c0 + i) / 4) * G::BM + r_] =
-                make_float4(__uint_as_float(z[i]) * inv_l, __uint_as_float(z[i + 1]) * inv_l,
-                            __uint_as_float(z[i + 2]) * inv_l, __uint_as_float(z[i + 3]) * inv_l);
+            mine[((zc + c0 + i) / 4) * G::BM + r_] = make_float4(zo[i], zo[i + 1], zo[i + 2], zo[i + 3]);
         }
         const float w_own = p.w[g * 4 + hr * 2 + hr], w_peer = p.w[g * 4 + hr * 2 + (hr ^ 1)];
 #pragma unroll
         for (int c0 = 0; c0 < G::DH; c0 += 32) {
-          uint32_t z[32];
-          tmem_ld32(tl + G::Z_COL0 + 128 * hr + zc + c0, z);
-          tmem_wait_ld();
+          float zo[32];
+          z_chunk(hr, 2 * g + hr, c0, zo);
 #pragma unroll
-          for (int i = 0; i < 32; ++i) o[c0 + i] = w_own * (__uint_as_float(z[i]) * inv_l);
+          for (int i = 0; i < 32; ++i) o[c0 + i] = w_own * zo[i];
         }
         tc_fence_before();
         __syncwarp();
@@ -637,11 +846,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       } else {
 #pragma unroll
         for (int c0 = 0; c0 < G::DH; c0 += 32) {
-          uint32_t z[32];
-          tmem_ld32(tl + G::Z_COL0 + zc + c0, z);
-          tmem_wait_ld();
+          float zo[32];
+          z_chunk(0, h, c0, zo);
 #pragma unroll
-          for (int i = 0; i < 32; ++i) o[c0 + i] = __uint_as_float(z[i]) * inv_l;
+          for (int i = 0; i < 32; ++i) o[c0 + i] = zo[i];
         }
         tc_fence_before();
         __syncwarp();
@@ -662,7 +870,6 @@ __global__ void __launch_bounds__(kThreads, 1)
         const float rstd = rsqrtf((s2 + red[(8 + (wg ^ 1)) * G::BM + r_]) * (1.f / D) + p.eps);
         const float *gm = p.gamma + static_cast<long long>(h) * D + zc;
         const float *bt = p.beta + static_cast<long long>(h) * D + zc;
-#pragma unroll
         const float mh = head_multiplier(p.gate, p.lam, h);
 #pragma unroll
         for (int i = 0; i < G::DH; ++i) o[i] = ((o[i] - mu) * rstd * gm[i] + bt[i]) * mh;
@@ -693,10 +900,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 }
 
-template <int D, int CQ, int CK, int MIX, bool EXACT>
-cudaError_t launch_kq_one(const AttnArgs &a, const GnArgs *gn, const KqPrepArgs &pa, float *xg) {
-  using G = KGeo<D, CQ, CK, MIX, EXACT>;
-  alignas(64) CUtensorMap tq, tk, tv;
+template <int D, int CQ, int CK, int MIX, bool EXACT, bool POST>
+cudaError_t launch_kq_one(const AttnArgs &a, const GnArgs *gn, const KqPrepArgs &pa, float *xg, void *vt) {
+  using G = KGeo<D, CQ, CK, MIX, EXACT, POST>;
+  alignas(64) CUtensorMap tq, tk, tv, tvt;
   const unsigned long long dims[4] = {static_cast<unsigned long long>(D), static_cast<unsigned long long>(a.H),
                                       static_cast<unsigned long long>(a.L), static_cast<unsigned long long>(a.B)};
   const unsigned long long str[3] = {static_cast<unsigned long long>(D) * 2,
@@ -712,6 +919,12 @@ cudaError_t launch_kq_one(const AttnArgs &a, const GnArgs *gn, const KqPrepArgs 
                                       static_cast<unsigned long long>(a.L) * D * 2};
   const unsigned boxk[3] = {64, G::BN, 1};
   if (!encode_tmap_bf16(&tk, pa.kt, 3, kdims, kstr, boxk, true)) return cudaErrorInvalidValue;
+  tvt = tk;
+  if (POST) {  // convolved values: [B*H*NV*CQ][L][D] bf16, 64-channel x 128-key boxes
+    const unsigned long long vdims[3] = {static_cast<unsigned long long>(D), static_cast<unsigned long long>(a.L),
+                                         static_cast<unsigned long long>(a.B) * a.H * G::NV * CQ};
+    if (!encode_tmap_bf16(&tvt, vt, 3, vdims, kstr, boxk, true)) return cudaErrorInvalidValue;
+  }
   KqParams p;
   p.theta = a.theta;
   p.w = a.w;
@@ -725,14 +938,17 @@ cudaError_t launch_kq_one(const AttnArgs &a, const GnArgs *gn, const KqPrepArgs 
   p.B = a.B;
   p.L = a.L;
   p.H = a.H;
-  p.n_qtiles = (a.L + G::BM - 1) / G::BM;
+  p.n_qtiles = (a.L + G::BMO - 1) / G::BMO;
   p.qk_scale = a.scale;
   p.lpad = pa.lpad;
   p.fac = pa.fac;
   p.vp = pa.vp;
   p.xg = xg;
   p.err = a.err;
-  auto kern = attn_kq_kernel<D, CQ, CK, MIX, EXACT>;
+  p.theta_post = a.theta_post;
+  p.v = static_cast<const __nv_bfloat16 *>(a.v);
+  p.rs = a.rs;
+  auto kern = attn_kq_kernel<D, CQ, CK, MIX, EXACT, POST>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, G::SMEM);
   if (e != cudaSuccess) return e;
   // persistent: as many clusters as can be resident at once (at most one per work
@@ -756,7 +972,7 @@ cudaError_t launch_kq_one(const AttnArgs &a, const GnArgs *gn, const KqPrepArgs 
   if (resident < 1) return cudaErrorInvalidConfiguration;
   const long long nc = std::min<long long>(std::min<long long>(resident, n_items), kKqMaxClusters / G::CLUSTER);
   cfg.gridDim = dim3(G::CLUSTER, static_cast<unsigned>(nc));
-  return cudaLaunchKernelEx(&cfg, kern, tq, tk, tv, p);
+  return cudaLaunchKernelEx(&cfg, kern, tq, tk, tv, tvt, p);
 }
 
 size_t align256(size_t x) { return (x + 255) / 256 * 256; }
@@ -764,7 +980,7 @@ size_t align256(size_t x) { return (x + 255) / 256 * 256; }
 }  // namespace
 
 bool attn_kq_supported(const AttnArgs &a) {
-  if (a.dtype != 1 || a.kqp != 0 || (a.d != 64 && a.d != 128)) return false;
+  if (a.dtype != 1 || (a.d != 64 && a.d != 128)) return false;
   if ((a.kq != 1 && a.kq != 3) || a.cq != 6 || a.ck != 11) return false;
   if (!(a.hp == 0 || ((a.hp == 1 || a.hp == 2) && a.ch == 2))) return false;
   if (a.B > 65535 || a.H > 65535 || (a.L + 127) / 128 > 65535) return false;
@@ -773,20 +989,30 @@ bool attn_kq_supported(const AttnArgs &a) {
   return al % 16 == 0 && a.rs % 8 == 0;
 }
 
+namespace {
+// rows of the query tiles: 128, or 123 output rows with the post-softmax convolution
+size_t kq_items(int B, int H, int L, int kqp) {
+  const size_t bmo = kqp ? 128 - 5 : 128;
+  return static_cast<size_t>(B) * (H / 2) * ((static_cast<size_t>(L) + bmo - 1) / bmo);
+}
+}  // namespace
+
 // Workspace of the contraction path: Kt [B][H][c_q][L][d] fp16 | fac [B][H][Lpad] fp32 |
 // Vp [B][H][L][M] fp32 | (post-softmax mixing) the exchange buffer of the persistent
-// CTAs, [CTAs][2][d][128] fp32; Lpad = L rounded up to 128,
-// M = (c_q-1) + 2*(c_k/2); each part 256-byte aligned.
-size_t attn_kq_workspace_bytes(int B, int H, int L, int d, int cq, int ck, int hp) {
+// CTAs, [CTAs][2][d][128] fp32 | (post-softmax convolution) the convolved values
+// Vt [B][H][nvh][c_q][L][d] bf16, nvh = 2 with post-softmax mixing, else 1;
+// Lpad = L rounded up to 128, M = (c_q-1) + 2*(c_k/2); each part 256-byte aligned.
+size_t attn_kq_workspace_bytes(int B, int H, int L, int d, int cq, int ck, int hp, int kqp) {
   const size_t BH = static_cast<size_t>(B) * H, BHL = BH * L;
   const size_t lpad = (static_cast<size_t>(L) + 127) / 128 * 128;
   const size_t M = static_cast<size_t>(cq - 1 + 2 * (ck / 2));
   // one slot pair per persistent CTA: at most kKqMaxClusters CTAs, and at most two per
   // work item (batch, head group, query tile)
-  const size_t items = static_cast<size_t>(B) * (H / 2) * ((static_cast<size_t>(L) + 127) / 128);
+  const size_t items = kq_items(B, H, L, kqp);
   const size_t ctas = std::min<size_t>(kKqMaxClusters, 2 * items);
   const size_t xg = hp == 2 ? ctas * 2 * d * 128 * 4 : 0;
-  return align256(BHL * cq * d * 2) + align256(BH * lpad * 4) + align256(BHL * M * 4) + xg;
+  const size_t vt = kqp ? align256(BHL * (hp == 2 ? 2 : 1) * cq * d * 2) : 0;
+  return align256(BHL * cq * d * 2) + align256(BH * lpad * 4) + align256(BHL * M * 4) + xg + vt;
 }
 
 cudaError_t launch_attn_kq(const AttnArgs &a, const GnArgs *gn, void *ws) {
@@ -807,13 +1033,30 @@ cudaError_t launch_attn_kq(const AttnArgs &a, const GnArgs *gn, void *ws) {
   pa.fac = reinterpret_cast<float *>(base + align256(BHL * a.cq * a.d * 2));
   pa.vp = reinterpret_cast<float *>(reinterpret_cast<char *>(pa.fac) + align256(BH * pa.lpad * 4));
   float *xg = reinterpret_cast<float *>(reinterpret_cast<char *>(pa.vp) + align256(BHL * pa.M * 4));
+  const size_t items = kq_items(a.B, a.H, a.L, a.kqp);
+  void *vt = reinterpret_cast<char *>(xg) +
+             (a.hp == 2 ? std::min<size_t>(kKqMaxClusters, 2 * items) * 2 * a.d * 128 * 4 : 0);
   cudaError_t e = launch_kq_prep(pa, a.stream);
   if (e != cudaSuccess) return e;
+  if (a.kqp) {
+    VtPrepArgs va;
+    va.v = a.v;
+    va.rs = a.rs;
+    va.theta_post = a.theta_post;
+    va.vt = vt;
+    va.B = a.B; va.H = a.H; va.L = a.L; va.d = a.d; va.cq = a.cq; va.ck = a.ck;
+    va.nvh = a.hp == 2 ? 2 : 1;
+    va.n_tiles = pa.n_tiles;
+    if ((e = launch_vt_prep(va, a.stream)) != cudaSuccess) return e;
+  }
   // MIX: 0 no head mixing, 1 pre-softmax mixing (both C of a group per CTA), 2 post-softmax
   auto go = [&](auto d_tag, auto mix_tag) -> cudaError_t {
     constexpr int DD = decltype(d_tag)::value, MX = decltype(mix_tag)::value;
-    return pa.exact ? launch_kq_one<DD, 6, 11, MX, true>(a, gn, pa, xg)
-                    : launch_kq_one<DD, 6, 11, MX, false>(a, gn, pa, xg);
+    if (a.kqp)
+      return pa.exact ? launch_kq_one<DD, 6, 11, MX, true, true>(a, gn, pa, xg, vt)
+                      : launch_kq_one<DD, 6, 11, MX, false, true>(a, gn, pa, xg, vt);
+    return pa.exact ? launch_kq_one<DD, 6, 11, MX, true, false>(a, gn, pa, xg, vt)
+                    : launch_kq_one<DD, 6, 11, MX, false, false>(a, gn, pa, xg, vt);
   };
   using D64 = std::integral_constant<int, 64>;
   using D128 = std::integral_constant<int, 128>;

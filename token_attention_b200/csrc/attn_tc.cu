@@ -523,7 +523,6 @@ __global__ void __launch_bounds__(kThreads, 1)
       rstd = rsqrtf((redgn[r] + redgn[128 + r] + redgn[256 + r] + redgn[384 + r]) * (1.f / D) + p.eps);
       const float *gm = p.gamma + static_cast<long long>(h) * D + cbase;
       const float *bt = p.beta + static_cast<long long>(h) * D + cbase;
-#pragma unroll
       const float mh = head_multiplier(p.gate, p.lam, h);
 #pragma unroll
       for (int i = 0; i < G::DQ; ++i) o[i] = ((o[i] - mu) * rstd * gm[i] + bt[i]) * mh;

@@ -55,9 +55,21 @@ struct KqPrepArgs {
   int exact;              // exact causal indicator: Vp[i][m] = q[i] . k[i-m+(cq-1)]
 };
 cudaError_t launch_kq_prep(const KqPrepArgs &a, cudaStream_t stream);
+// Values convolved by the post-softmax kernels along the keys (bf16):
+//   Vt[b][s][hd][a][j] = sum_t theta_post[s][a][t] v_{head(s,hd)}[j + t - c_k/2]
+// for the source head s and, with post-softmax mixing (nvh = 2), both heads hd of
+// its group, else (nvh = 1) head s itself; zero outside [0, L).
+struct VtPrepArgs {
+  const void *v;            // [B][L][H][d] bf16, token stride rs
+  long long rs;
+  const float *theta_post;  // [H][c_q][c_k]
+  void *vt;                 // [B][H][nvh][c_q][L][d] bf16
+  int B, H, L, d, cq, ck, nvh, n_tiles;
+};
+cudaError_t launch_vt_prep(const VtPrepArgs &a, cudaStream_t stream);
 // Workspace bytes of the contraction path (beyond the error word) and whether it applies.
 bool attn_kq_supported(const AttnArgs &a);
-size_t attn_kq_workspace_bytes(int B, int H, int L, int d, int cq, int ck, int hp);
+size_t attn_kq_workspace_bytes(int B, int H, int L, int d, int cq, int ck, int hp, int kqp);
 // ws: workspace area for Kt / fac / Vp (attn_kq_workspace_bytes bytes, 256-byte aligned).
 cudaError_t launch_attn_kq(const AttnArgs &a, const GnArgs *gn, void *ws);
 

@@ -219,7 +219,89 @@ cudaError_t launch_prep_one(const KqPrepArgs &p, cudaStream_t stream) {
   return cudaGetLastError();
 }
 
+// ---------------------------------------------------------------------------
+// Values convolved by the post-softmax kernels.  Section 3.1's convolution after
+// the softmax, A'[i][j] = sum_a sum_t theta_post[a][t] A[i-a][j-(t-c)], moves onto
+// the values away from the diagonal:
+//   sum_j A'[i][j] v[j] = sum_a sum_j' A[i-a][j'] Vt_a[j'],  Vt_a[j'] = sum_t theta_post[a][t] v[j'+t-c],
+// so the attention kernel multiplies row-shifted weights by Vt_a on the tensor
+// cores.  One CTA per (key tile, source head, batch); the value rows with their
+// +-c halo are staged as bf16, and each thread convolves a channel pair over
+// kRun consecutive keys from a register window.
+template <int D, int CQ, int CK, int NVH>
+__global__ void __launch_bounds__(kPrepThreads, 3) vt_prep_kernel(VtPrepArgs p) {
+  constexpr int C = CK / 2, ROWS = kTile + 2 * C, VSTR = D + 8;
+  extern __shared__ uint32_t vs[];  // [ROWS][VSTR/2] bf16 pairs, row r = key j0 - C + r
+  __shared__ float th[CQ * CK];
+  const int tile = blockIdx.x, s = blockIdx.y, b = blockIdx.z, tid = threadIdx.x;
+  const int L = p.L, j0 = tile * kTile;
+  const __nv_bfloat16 *vb = static_cast<const __nv_bfloat16 *>(p.v);
+  __nv_bfloat16 *vt = static_cast<__nv_bfloat16 *>(p.vt);
+  for (int i = tid; i < CQ * CK; i += kPrepThreads) th[i] = p.theta_post[static_cast<long long>(s) * CQ * CK + i];
+  constexpr int NPAIR = D / 2, NRUN = kTile / kRun;
+#pragma unroll 1
+  for (int hd = 0; hd < NVH; ++hd) {
+    const int hv = NVH == 2 ? (s & ~1) + hd : s;
+    __syncthreads();  // the previous head's window is consumed (and th is loaded)
+    for (int i = tid; i < ROWS * (D / 8); i += kPrepThreads) {
+      const int r = i / (D / 8), e8 = (i % (D / 8)) * 8, key = j0 - C + r;
+      uint4 raw = make_uint4(0u, 0u, 0u, 0u);
+      if (key >= 0 && key < L)
+        raw = *reinterpret_cast<const uint4 *>(vb + (static_cast<long long>(b) * L + key) * p.rs +
+                                               static_cast<long long>(hv) * D + e8);
+      *reinterpret_cast<uint4 *>(vs + (r * VSTR + e8) / 2) = raw;
+    }
+    __syncthreads();
+    const long long z0 = ((static_cast<long long>(b) * p.H + s) * NVH + hd) * CQ;
+    for (int item = tid; item < NPAIR * NRUN; item += kPrepThreads) {
+      const int e2 = (item % NPAIR) * 2, jr = (item / NPAIR) * kRun;
+      if (j0 + jr >= L) continue;
+      const int nkeys = min(kRun, L - (j0 + jr));
+      float2 win[kRun + 2 * C];  // keys j0+jr-c .. j0+jr+kRun-1+c
+#pragma unroll
+      for (int w = 0; w < kRun + 2 * C; ++w) win[w] = bf16x2_to_float2(vs[((jr + w) * VSTR + e2) / 2]);
+#pragma unroll
+      for (int a = 0; a < CQ; ++a) {
+        float2 acc[kRun];
+#pragma unroll
+        for (int u = 0; u < kRun; ++u) acc[u] = make_float2(0.f, 0.f);
+#pragma unroll
+        for (int t = 0; t < CK; ++t) {
+          const float ta = th[a * CK + t];
+#pragma unroll
+          for (int u = 0; u < kRun; ++u) {  // value j + (t - c) is window entry u + t
+            acc[u].x = fmaf(ta, win[u + t].x, acc[u].x);
+            acc[u].y = fmaf(ta, win[u + t].y, acc[u].y);
+          }
+        }
+        __nv_bfloat16 *oa = vt + ((z0 + a) * L + j0 + jr) * D + e2;
+#pragma unroll
+        for (int u = 0; u < kRun; ++u)
+          if (nkeys == kRun || u < nkeys)
+            *reinterpret_cast<__nv_bfloat162 *>(oa + u * D) = __floats2bfloat162_rn(acc[u].x, acc[u].y);
+      }
+    }
+  }
+}
+
+template <int D, int NVH>
+cudaError_t launch_vt_one(const VtPrepArgs &p, cudaStream_t stream) {
+  constexpr int SMEM = (kTile + 2 * (11 / 2)) * (D + 8) * 2;
+  auto kern = vt_prep_kernel<D, 6, 11, NVH>;
+  const cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM);
+  if (e != cudaSuccess) return e;
+  kern<<<dim3(p.n_tiles, p.H, p.B), kPrepThreads, SMEM, stream>>>(p);
+  return cudaGetLastError();
+}
+
 }  // namespace
+
+cudaError_t launch_vt_prep(const VtPrepArgs &p, cudaStream_t stream) {
+  if (p.cq != 6 || p.ck != 11 || (p.nvh != 1 && p.nvh != 2)) return cudaErrorInvalidValue;
+  if (p.d == 128) return p.nvh == 2 ? launch_vt_one<128, 2>(p, stream) : launch_vt_one<128, 1>(p, stream);
+  if (p.d == 64) return p.nvh == 2 ? launch_vt_one<64, 2>(p, stream) : launch_vt_one<64, 1>(p, stream);
+  return cudaErrorInvalidValue;
+}
 
 cudaError_t launch_kq_prep(const KqPrepArgs &p, cudaStream_t stream) {
   if (p.cq != 6 || p.ck != 11 || p.M != PrepGeo<128, 6, 11, false>::M) return cudaErrorInvalidValue;

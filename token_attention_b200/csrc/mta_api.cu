@@ -66,14 +66,16 @@ enum Kernel { K_SIMT = 1, K_TC = 2, K_KQ = 3 };
 // Shape-level test for the contraction kernel (pointer alignment aside): used
 // to size the workspace.
 bool kq_shape_ok(const mta_cfg *c) {
-  return c->dtype == MTA_BF16 && c->kq_post == 0 && (c->d == 64 || c->d == 128) &&
+  return c->dtype == MTA_BF16 && (c->d == 64 || c->d == 128) &&
          (c->kq_place == MTA_PRE || c->kq_place == MTA_PRE_EXACT) &&
          c->c_q == 6 && c->c_k == 11 &&
          (c->head_place == MTA_OFF || ((c->head_place == MTA_PRE || c->head_place == MTA_POST) && c->c_h == 2));
 }
 
 size_t kq_bytes(const mta_cfg *c) {
-  return kq_shape_ok(c) ? attn_kq_workspace_bytes(c->B, c->H, c->L, c->d, c->c_q, c->c_k, c->head_place) : 0;
+  return kq_shape_ok(c) ? attn_kq_workspace_bytes(c->B, c->H, c->L, c->d, c->c_q, c->c_k, c->head_place,
+                                                  c->kq_post)
+                        : 0;
 }
 
 // Which attention kernel serves `a` under cfg->path: 0 chooses the contraction
@@ -82,7 +84,7 @@ size_t kq_bytes(const mta_cfg *c) {
 // kernel; 1, 2, 3 force the CUDA-core, direct tensor-core, contraction kernel.
 mta_status select_kernel(const AttnArgs &a, int path, size_t kq_room, Kernel *k) {
   const bool kq_ok = attn_kq_supported(a) &&
-                     kq_room >= attn_kq_workspace_bytes(a.B, a.H, a.L, a.d, a.cq, a.ck, a.hp);
+                     kq_room >= attn_kq_workspace_bytes(a.B, a.H, a.L, a.d, a.cq, a.ck, a.hp, a.kqp);
   const bool tc_ok = attn_tc_supported(a);
   const bool simt_ok = attn_simt_pick_rows(a, 32) != 0;
   if (path == 3) {
