@@ -65,6 +65,8 @@ __all__ = ["OFF", "PRE", "POST", "PRE_EXACT", "attention_logits", "mask_zero", "
            "key_query_conv_exact", "sigmoid_gate", "post_softmax_conv",
            "head_mix", "mask_neg_inf", "softmax_rows", "mta_attention_group",
            "mta_attention", "mta_attention_rows", "group_norm_scale", "mta_layer",
+           "key_query_conv_adjoint", "key_query_conv_grad_theta", "mta_attention_group_bwd",
+           "mta_attention_bwd",
            "mta_layer_rows"]
 
 
@@ -197,6 +199,134 @@ def mta_attention_group(q_rows, k, v, theta, w, qpos, scale, kq_place, head_plac
 
 
 # ----------------------------------------------------------------------------
+# backward pass of one head group (gradients by the chain rule, each forward
+# step taken in reverse order; the pages train with this forward, section 4)
+# ----------------------------------------------------------------------------
+
+def key_query_conv_adjoint(g: np.ndarray, theta: np.ndarray) -> np.ndarray:
+    """Adjoint of key_query_conv in its input: for out = key_query_conv(m, theta),
+    d m[h, r', j'] = sum_a sum_t theta[h, a, t] * g[h, r' + a, j' + (t - c_k//2)]
+    (entries outside the array count as 0)."""
+    ch, R, L = g.shape
+    cq, ck = theta.shape[1], theta.shape[2]
+    c = ck // 2
+    out = np.zeros_like(g, dtype=np.float64)
+    for a in range(cq):
+        if a >= R:
+            break
+        for t in range(ck):
+            b = t - c
+            j_lo, j_hi = max(0, b), min(L, L + b)
+            if j_lo >= j_hi:
+                continue
+            coef = theta[:, a, t].astype(np.float64)[:, None, None]
+            out[:, :R - a, j_lo - b:j_hi - b] += coef * g[:, a:, j_lo:j_hi]
+    return out
+
+
+def key_query_conv_grad_theta(g: np.ndarray, m: np.ndarray, cq: int, ck: int) -> np.ndarray:
+    """Gradient of key_query_conv in its kernel: d theta[h, a, t] =
+    sum_{r, j} g[h, r, j] * m[h, r - a, j - (t - c_k//2)]."""
+    ch, R, L = g.shape
+    c = ck // 2
+    out = np.zeros((ch, cq, ck), np.float64)
+    for a in range(cq):
+        if a >= R:
+            break
+        for t in range(ck):
+            b = t - c
+            j_lo, j_hi = max(0, b), min(L, L + b)
+            if j_lo >= j_hi:
+                continue
+            out[:, a, t] = np.einsum("hrj,hrj->h", g[:, a:, j_lo:j_hi], m[:, :R - a, j_lo - b:j_hi - b])
+    return out
+
+
+def _exact_indicator_terms(a_hat, theta, qpos):
+    """The shifted, indicator-masked logits of key_query_conv_exact, one per tap:
+    yields (a, t, shifted * [key <= query])."""
+    ch, R, L = a_hat.shape
+    cq, ck = theta.shape[1], theta.shape[2]
+    c = ck // 2
+    keys = np.arange(L)
+    for a in range(min(cq, R)):
+        for t in range(ck):
+            b = t - c
+            j_lo, j_hi = max(0, b), min(L, L + b)
+            if j_lo >= j_hi:
+                continue
+            allowed = ((keys[None, :] - b) <= np.asarray(qpos)[:, None]).astype(np.float64)
+            yield a, t, b, j_lo, j_hi, allowed
+
+
+def mta_attention_group_bwd(q_rows, k, v, theta, w, qpos, scale, kq_place, head_place, dout,
+                            theta_post=None):
+    """Gradients of mta_attention_group for all its query rows (qpos = 0 .. L-1).
+
+    dout [c_h, R, d]: gradient of the output.  Returns dict with dq [c_h, R, d],
+    dk, dv [c_h, L, d], dtheta [c_h, c_q, c_k] (None if the convolution is off),
+    dw [c_h, c_h] (None without head mixing) and dtheta_post (None without the
+    post-softmax convolution), all float64."""
+    qpos = np.asarray(qpos)
+    q64, k64, v64 = (x.astype(np.float64) for x in (q_rows, k, v))
+    g_out = dout.astype(np.float64)
+    # forward, keeping every intermediate map
+    a_hat = attention_logits(q_rows, k, scale)
+    if kq_place == PRE:
+        m0 = mask_zero(a_hat, qpos)
+        c = key_query_conv(m0, theta)
+    elif kq_place == PRE_EXACT:
+        c = key_query_conv_exact(a_hat, theta, qpos)
+    else:
+        c = a_hat
+    c2 = head_mix(c, w) if head_place == PRE else c
+    attn = softmax_rows(mask_neg_inf(c2, qpos))
+    attn2 = post_softmax_conv(attn, theta_post, qpos) if theta_post is not None else attn
+    attn3 = head_mix(attn2, w) if head_place == POST else attn2
+    res = {"dtheta": None, "dw": None, "dtheta_post": None}
+    # out[r] = attn3[r] v[r]
+    res["dv"] = np.matmul(attn3.transpose(0, 2, 1), g_out)
+    d_attn3 = np.matmul(g_out, v64.transpose(0, 2, 1))
+    if head_place == POST:                      # attn3[r] = sum_s w[r, s] attn2[s]
+        res["dw"] = np.einsum("rij,sij->rs", d_attn3, attn2)
+        d_attn2 = np.einsum("rs,rij->sij", w.astype(np.float64), d_attn3)
+    else:
+        d_attn2 = d_attn3
+    if theta_post is not None:                  # attn2 = Mask_0(conv(attn, theta_post))
+        g_pre = mask_zero(d_attn2, qpos)
+        res["dtheta_post"] = key_query_conv_grad_theta(g_pre, attn, theta_post.shape[1], theta_post.shape[2])
+        d_attn = key_query_conv_adjoint(g_pre, theta_post)
+    else:
+        d_attn = d_attn2
+    # softmax over keys: d c2 = attn * (d attn - sum_j d attn * attn); masked keys have attn 0
+    dc2 = attn * (d_attn - np.sum(d_attn * attn, axis=-1, keepdims=True))
+    if head_place == PRE:                       # c2[r] = sum_s w[r, s] c[s]
+        res["dw"] = np.einsum("rij,sij->rs", dc2, c)
+        dc = np.einsum("rs,rij->sij", w.astype(np.float64), dc2)
+    else:
+        dc = dc2
+    if kq_place == PRE:                         # c = conv(Mask_0(a_hat), theta)
+        res["dtheta"] = key_query_conv_grad_theta(dc, m0, theta.shape[1], theta.shape[2])
+        d_a_hat = mask_zero(key_query_conv_adjoint(dc, theta), qpos)
+    elif kq_place == PRE_EXACT:                 # c = sum_taps theta * shifted(a_hat) * [key <= query]
+        ch, R, L = a_hat.shape
+        d_a_hat = np.zeros_like(a_hat)
+        dth = np.zeros(theta.shape, np.float64)
+        for a, t, b, j_lo, j_hi, allowed in _exact_indicator_terms(a_hat, theta, qpos):
+            g = dc * allowed[None]               # gradient reaching the shifted logits
+            dth[:, a, t] = np.einsum("hrj,hrj->h", g[:, a:, j_lo:j_hi], a_hat[:, :R - a, j_lo - b:j_hi - b])
+            coef = theta[:, a, t].astype(np.float64)[:, None, None]
+            d_a_hat[:, :R - a, j_lo - b:j_hi - b] += coef * g[:, a:, j_lo:j_hi]
+        res["dtheta"] = dth
+    else:
+        d_a_hat = dc
+    # a_hat = scale q k^T
+    res["dq"] = scale * np.matmul(d_a_hat, k64)
+    res["dk"] = scale * np.matmul(d_a_hat.transpose(0, 2, 1), q64)
+    return res
+
+
+# ----------------------------------------------------------------------------
 # whole tensors in the library's layout: q, k, v, out [B][L][H][d]
 # ----------------------------------------------------------------------------
 
@@ -231,6 +361,38 @@ def mta_attention(q, k, v, theta, w, c_h, kq_place=PRE, head_place=POST, scale=N
                                      qpos, s, kq_place, head_place,
                                      None if theta_post is None else theta_post[hs])
             out[b, :, hs, :] = og.transpose(1, 0, 2)
+    return out
+
+
+def mta_attention_bwd(q, k, v, theta, w, c_h, dout, kq_place=PRE, head_place=POST, scale=None,
+                      theta_post=None):
+    """Gradients of mta_attention.  q, k, v, dout [B][L][H][d].  Returns dict with
+    dq, dk, dv [B][L][H][d], dtheta [H][c_q][c_k] (summed over batches),
+    dw [H/c_h][c_h][c_h] and dtheta_post, float64 (None where the step is off)."""
+    B, L, H, d = q.shape
+    s = _default_scale(d, scale)
+    G = H // c_h
+    out = {n: np.zeros((B, L, H, d), np.float64) for n in ("dq", "dk", "dv")}
+    dth = np.zeros((H,) + theta.shape[1:], np.float64) if theta is not None and kq_place else None
+    dw = np.zeros((G, c_h, c_h), np.float64) if head_place else None
+    dtp = np.zeros(theta_post.shape, np.float64) if theta_post is not None else None
+    qpos = np.arange(L)
+    for b in range(B):
+        for g in range(G):
+            hs = slice(g * c_h, (g + 1) * c_h)
+            r = mta_attention_group_bwd(_group(q, b, g, c_h), _group(k, b, g, c_h), _group(v, b, g, c_h),
+                                        _sel(theta, hs), _sel(w, g), qpos, s, kq_place, head_place,
+                                        _group(dout, b, g, c_h),
+                                        None if theta_post is None else theta_post[hs])
+            for n in ("dq", "dk", "dv"):
+                out[n][b, :, hs, :] = r[n].transpose(1, 0, 2)
+            if dth is not None:
+                dth[hs] += r["dtheta"]
+            if dw is not None:
+                dw[g] += r["dw"]
+            if dtp is not None:
+                dtp[hs] += r["dtheta_post"]
+    out["dtheta"], out["dw"], out["dtheta_post"] = dth, dw, dtp
     return out
 
 

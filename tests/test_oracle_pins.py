@@ -606,3 +606,70 @@ def test_post_conv_rows_match_full(qkv):
             part = O.mta_attention_rows(q, k, v, th, w, 2, rows, kq, hp, theta_post=tp)
             for n, (b, i) in enumerate(rows):
                 np.testing.assert_allclose(part[n], full[b, i], rtol=0, atol=1e-12)
+
+
+# ----------------------------------------------------------------------------
+# backward pass: pinned to central finite differences of the forward, and to
+# torch's autograd of its causal attention for identity kernels
+# ----------------------------------------------------------------------------
+
+def _fd_check(kq, hp, post, seed):
+    B, L, H, d, cq, ck, ch = 1, 7, 2, 3, 3, 3, 2
+    rng = np.random.default_rng(seed)
+    q, k, v = (rng.standard_normal((B, L, H, d)) for _ in range(3))
+    th = rng.standard_normal((H, cq, ck)) * 0.5
+    tp = rng.standard_normal((H, cq, ck)) * 0.5 if post else None
+    w = rng.standard_normal((1, ch, ch))
+    dout = rng.standard_normal((B, L, H, d))
+    hpl = hp if hp != O.OFF else O.OFF
+
+    def f(q_, k_, v_, th_, w_, tp_):
+        o = O.mta_attention(q_, k_, v_, th_, w_, ch, kq, hpl, theta_post=tp_)
+        return float(np.sum(o * dout))
+
+    g = O.mta_attention_bwd(q, k, v, th, w, ch, dout, kq, hpl, theta_post=tp)
+    base = dict(q_=q, k_=k, v_=v, th_=th, w_=w, tp_=tp)
+    checks = [("q_", "dq"), ("k_", "dk"), ("v_", "dv")]
+    if kq != O.OFF:
+        checks.append(("th_", "dtheta"))
+    if hp != O.OFF:
+        checks.append(("w_", "dw"))
+    if post:
+        checks.append(("tp_", "dtheta_post"))
+    eps = 1e-6
+    for name, gname in checks:
+        for rep in range(2):
+            u = rng.standard_normal(base[name].shape)
+            plus = dict(base); plus[name] = base[name] + eps * u
+            minus = dict(base); minus[name] = base[name] - eps * u
+            fd = (f(**plus) - f(**minus)) / (2 * eps)
+            an = float(np.sum(g[gname] * u))
+            assert abs(fd - an) <= 1e-6 * max(1.0, abs(an)), (kq, hp, post, gname, fd, an)
+
+
+@pytest.mark.parametrize("kq", [O.OFF, O.PRE, O.PRE_EXACT])
+@pytest.mark.parametrize("hp", [O.OFF, O.PRE, O.POST])
+@pytest.mark.parametrize("post", [False, True])
+def test_backward_matches_finite_differences(kq, hp, post):
+    """Every gradient (q, k, v, the kernels, the mixing weights) against central
+    differences of the forward, along random directions."""
+    _fd_check(kq, hp, post, seed=900 + 7 * kq + 3 * hp + post)
+
+
+def test_backward_identity_kernels_equal_torch_autograd():
+    """theta = delta(0,0), w = I: the gradients are those of causal softmax
+    attention, taken here by torch's autograd through its SDPA routine."""
+    B, L, H, d, cq, ck, ch = 2, 11, 4, 5, 3, 5, 2
+    rng = np.random.default_rng(5)
+    q, k, v, dout = (rng.standard_normal((B, L, H, d)) for _ in range(4))
+    th = delta_theta(H, cq, ck, 0, ck // 2)
+    w = np.tile(np.eye(ch), (H // ch, 1, 1))
+    g = O.mta_attention_bwd(q, k, v, th, w, ch, dout, O.PRE, O.POST)
+    t = lambda x: torch.from_numpy(np.ascontiguousarray(x.transpose(0, 2, 1, 3))).requires_grad_(True)
+    tq, tk, tv = t(q), t(k), t(v)
+    o = torch.nn.functional.scaled_dot_product_attention(tq, tk, tv, is_causal=True, scale=1 / np.sqrt(d))
+    o.backward(torch.from_numpy(np.ascontiguousarray(dout.transpose(0, 2, 1, 3))))
+    for name, tt in (("dq", tq), ("dk", tk), ("dv", tv)):
+        np.testing.assert_allclose(g[name], tt.grad.numpy().transpose(0, 2, 1, 3), rtol=0, atol=1e-12)
+    # the kernel gradient of the identity kernel's centre tap is the logits' own gradient . logits
+    assert g["dtheta"].shape == (H, cq, ck)
