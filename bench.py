@@ -37,6 +37,7 @@ sys.path.insert(0, ROOT)
 from token_attention_b200 import synth  # noqa: E402
 
 METRIC = "MTA fwd tokens/s and TFLOP/s at L=2048 on 1 B200; % of BF16 tensor peak"
+METRIC_BWD = "MTA attention backward (mta_attn_bwd) tokens/s on 1 B200"
 UNIT = "tokens/s"
 DEFAULT_WORKLOAD = "pretrain_d128_L2048"
 N_SETS = 3
@@ -67,7 +68,7 @@ def flops(wl: synth.Workload) -> dict:
 def uses_contraction(wl: synth.Workload) -> bool:
     """Whether the library's default path runs the contraction kernel (with its
     prepass) for this workload."""
-    return (wl.dtype == "bf16" and wl.d in (64, 128) and wl.kq_place == synth.PRE
+    return (wl.dtype == "bf16" and wl.d in (64, 96, 128) and wl.kq_place == synth.PRE
             and (wl.c_q, wl.c_k) == (6, 11)
             and (wl.head_place == synth.OFF or wl.c_h == 2))
 
@@ -220,7 +221,7 @@ class ClockSampler:
 # the library arm
 # ---------------------------------------------------------------------------
 
-def make_sets(wl, dev, n_sets):
+def make_sets(wl, dev, n_sets, bwd=False):
     import torch
 
     def to(x, dt):
@@ -239,12 +240,20 @@ def make_sets(wl, dev, n_sets):
             sets.append({k: to(inp[k], wl.dtype if k in "qkv" else "f32")
                          for k in ("q", "k", "v", "theta", "w")})
         sets[-1]["theta_post"] = None if inp["theta_post"] is None else to(inp["theta_post"], "f32")
+        if bwd:  # gradient of the output, drawn like the values
+            dout = synth.normal(w.seed, 20, (wl.B, wl.L, wl.H, wl.d))
+            sets[-1]["dout"] = to(synth.round_bf16(dout) if wl.dtype == "bf16" else dout, wl.dtype)
     return sets
 
 
-def step_fn(wl, mta, sets, ws, outs, stream):
+def step_fn(wl, mta, sets, ws, outs, stream, bwd=False):
     """Returns f(i): enqueue step i (input set i % n) on `stream`."""
-    if wl.layer:
+    if bwd:
+        def f(i):
+            s = sets[i % len(sets)]
+            mta.attn_bwd(s["q"], s["k"], s["v"], s["theta"], s["w"], s["dout"], wl.c_q, wl.c_k, wl.c_h,
+                         wl.kq_place, wl.head_place, ws=ws, stream=stream, grads=outs[i % len(outs)])
+    elif wl.layer:
         def f(i):
             s = sets[i % len(sets)]
             mta.layer_fwd(s["x"], s["wqkv"], s["theta"], s["w"], s["gamma"], s["beta"], s["wo"],
@@ -269,16 +278,25 @@ def run_mine(args, wl, rank, world, local_rank):
     dev = torch.device("cuda", local_rank)
     mta.lib()
     stream = torch.cuda.Stream(device=dev)
-    sets = make_sets(wl, dev, N_SETS)
+    sets = make_sets(wl, dev, N_SETS, args.bwd)
     out_shape = (wl.B, wl.L, wl.D) if wl.layer else (wl.B, wl.L, wl.H, wl.d)
     odt = torch.float32 if wl.dtype == "f32" else torch.bfloat16
-    outs = [torch.empty(out_shape, dtype=odt, device=dev) for _ in range(N_SETS)]
+    if args.bwd:  # fp32 gradients of q, k, v, the kernels and the mixing weights
+        z = lambda *shape: torch.empty(shape, dtype=torch.float32, device=dev)
+        outs = [{"dq": z(*out_shape), "dk": z(*out_shape), "dv": z(*out_shape),
+                 "dtheta": z(wl.H, wl.c_q, wl.c_k) if wl.kq_place else None,
+                 "dw": z(wl.H // wl.c_h, wl.c_h, wl.c_h) if wl.head_place else None} for _ in range(N_SETS)]
+    else:
+        outs = [torch.empty(out_shape, dtype=odt, device=dev) for _ in range(N_SETS)]
     cfg = mta.make_cfg(wl.B, wl.H, wl.L, wl.d, wl.c_q, wl.c_k, wl.c_h, wl.kq_place, wl.head_place,
                        mta.F32 if wl.dtype == "f32" else mta.BF16, kq_post=int(wl.kq_post))
-    nbytes = (mta.lib().mta_layer_workspace_bytes if wl.layer else mta.lib().mta_attn_workspace_bytes)(
-        ctypes.byref(cfg))
+    if args.bwd:
+        nbytes = mta.lib().mta_attn_bwd_workspace_bytes(ctypes.byref(cfg))
+    else:
+        nbytes = (mta.lib().mta_layer_workspace_bytes if wl.layer else mta.lib().mta_attn_workspace_bytes)(
+            ctypes.byref(cfg))
     ws = mta.workspace(nbytes, dev)
-    f = step_fn(wl, mta, sets, ws, outs, stream)
+    f = step_fn(wl, mta, sets, ws, outs, stream, args.bwd)
 
     def barrier():
         if world > 1:
@@ -330,7 +348,7 @@ def run_mine(args, wl, rank, world, local_rank):
     t_max = max_over_ranks(total_ms, world, dev)
 
     e2e = None
-    if not args.no_e2e:
+    if not args.no_e2e and not args.bwd:
         e2e = run_e2e(args, wl, mta, sets, ws, stream, dev, barrier, world)
     return {"total_ms": t_max, "per_launch_ms": per_launch, "clocks": clocks, "e2e": e2e,
             "warmup": warm}
@@ -417,6 +435,23 @@ def oracle_sample(wl, budget_s: float, mode: str):
     q, k, v, th, w = inp["q"], inp["k"], inp["v"], inp["theta"], inp["w"]
     tp = inp["theta_post"]
     ch = wl.c_h
+    if mode == "bwd_groups":  # the backward oracle on whole head groups at full length
+        n_units = wl.B * (wl.H // ch)
+        dout = synth.normal(wl.seed, 20, (wl.B, wl.L, wl.H, wl.d))
+        done, t0 = 0, time.perf_counter()
+        for u in range(n_units):
+            b, g = divmod(u, wl.H // ch)
+            hs = slice(g * ch, (g + 1) * ch)
+            grp = lambda x: np.ascontiguousarray(x[b, :, hs].transpose(1, 0, 2))
+            O.mta_attention_group_bwd(grp(q), grp(k), grp(v), th[hs], w[g], np.arange(wl.L),
+                                      1 / math.sqrt(wl.d), wl.kq_place, wl.head_place, grp(dout))
+            done += 1
+            if time.perf_counter() - t0 > budget_s:
+                break
+        dt = time.perf_counter() - t0
+        tok = done * ch / wl.H * wl.L
+        return tok / dt, dt, (f"backward of {done} of {n_units} (batch, head-group) units at full length "
+                              f"L={wl.L} ({tok:.0f} token-equivalents)")
     if mode == "groups":
         n_units = wl.B * (wl.H // ch)
         done, t0 = 0, time.perf_counter()
@@ -488,6 +523,8 @@ def main():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu", action="store_true")
     ap.add_argument("--no-clocks", action="store_true")
+    ap.add_argument("--bwd", action="store_true",
+                    help="time the backward pass (mta_attn_bwd) of an attention workload instead")
     args = ap.parse_args()
 
     world = int(os.environ.get("WORLD_SIZE", "1"))
@@ -536,7 +573,21 @@ def main():
     launch_ms = statistics.mean(res["per_launch_ms"])
     peaks, peak_src = read_peaks()
     s = launch_ms / 1e3
-    if wl.layer:
+    if args.bwd:
+        # the backward on the CUDA cores: F_bwd = 8d + 4 c_q c_k + 4 c_h fp32 flop per causal
+        # pair-head (dS, dQ, dK, dV products; the convolution's adjoint and kernel gradient;
+        # the mixing adjoints)
+        kernel = "attn_bwd_simt_kernel"
+        f_bwd = (8 * wl.d + (4 * wl.c_q * wl.c_k if wl.kq_place else 0) + (4 * wl.c_h if wl.head_place else 0)) \
+            * wl.causal_pairs
+        achieved = f_bwd / s / 1e12
+        roof = {"bound": "alu", "achieved": achieved, "peak": FP32_PEAK_TFLOPS, "unit": "TFLOP/s",
+                "frac": achieved / FP32_PEAK_TFLOPS, "traffic": read_traffic(kernel, wl.name),
+                "kernel": kernel,
+                "per_unit": f"F_bwd = 8d + 4 c_q c_k + 4 c_h = {f_bwd // wl.causal_pairs} fp32 flop per "
+                            f"causal pair-head, x {wl.causal_pairs} pair-heads per launch",
+                "peak_source": "148 SMs x 128 FP32 lanes x 2 x 1965 MHz"}
+    elif wl.layer:
         kernel = "mta_layer_fwd"
         achieved = fl["mta"] / s / 1e12
         roof = {"bound": "tensor", "achieved": achieved, "peak": peaks["bf16_tflops"],
@@ -586,7 +637,8 @@ def main():
                             f"(key-query convolution), x {wl.causal_pairs} pair-heads per launch",
                 "peak_source": "148 SMs x 128 FP32 lanes x 2 x 1965 MHz"}
     line = {
-        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "metric": METRIC_BWD if args.bwd else METRIC, "value": value, "unit": UNIT, "n_gpus": world,
+        "steps": args.steps,
         "warmup": res["warmup"], "ms_per_step": ms / args.steps, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "bf16" if wl.dtype == "bf16" else "f32",
         "data": "synthetic", "config": config,
@@ -594,11 +646,12 @@ def main():
         "pct_bf16_peak": {"std": fl["std"] / s / 1e12 / peaks["bf16_tflops"],
                           "mta": fl["mta"] / s / 1e12 / peaks["bf16_tflops"],
                           "peak_tflops": peaks["bf16_tflops"], "peak_source": peak_src},
-        "roofline": roof, "gpu_launches": args.steps * launches_per_step(wl),
+        "roofline": roof, "gpu_launches": args.steps * (1 if args.bwd else launches_per_step(wl)),
         "clocks": res["clocks"], "e2e": res["e2e"],
     }
     if world == 1 and not args.no_cpu:
-        v, secs, desc = oracle_sample(wl, args.cpu_budget, "groups" if not wl.layer else "rows")
+        mode = "bwd_groups" if args.bwd else "groups" if not wl.layer else "rows"
+        v, secs, desc = oracle_sample(wl, args.cpu_budget, mode)
         line["cpu_baseline"] = {"value": v, "unit": UNIT, "cores": blas_threads(), "kind": "oracle",
                                 "sample": f"{desc}; {secs:.1f} s"}
     print(json.dumps(line), flush=True)

@@ -195,6 +195,29 @@ mta_status mta_gemm_bf16_nt(const void *A, const void *Bm, void *C, int M, int N
 mta_status mta_group_norm_scale(const void *o, const mta_gn *gn, int tokens, int H, int d,
                                 void *y, void *stream);
 
+/* Backward pass of mta_attn_fwd (the pages train with this forward; section 4).
+ * Given dout = dL/dout, writes the gradients of q, k, v, of the key-query kernels
+ * and of the head-mixing weights, each forward step taken in reverse order (see
+ * attn_bwd_simt.cu for the chain of adjoints):
+ *   q, k, v      : as for mta_attn_fwd (cfg->dtype, token stride cfg->qkv_row_stride)
+ *   theta_kq     : [H][c_q][c_k] fp32 (ignored when kq_place == MTA_OFF)
+ *   w_head       : [H/c_h][c_h][c_h] fp32 (ignored when head_place == MTA_OFF)
+ *   dout         : [B][L][H][d] dense, cfg->dtype
+ *   dq, dk, dv   : [B][L][H][d] dense fp32, overwritten
+ *   dtheta       : [H][c_q][c_k] fp32, overwritten (may be NULL; ignored when
+ *                  kq_place == MTA_OFF)
+ *   dw           : [H/c_h][c_h][c_h] fp32, overwritten (may be NULL; ignored when
+ *                  head_place == MTA_OFF)
+ * Runs on the CUDA cores in fp32 arithmetic for every forward configuration except
+ * the post-softmax convolution (cfg->kq_post = 1: MTA_ERR_UNSUPPORTED).  cfg->path
+ * must be 0 or 1.  dk, dv, dtheta and dw are summed with atomic additions, so their
+ * last bits may differ between runs.  The workspace holds the error word only
+ * (mta_attn_bwd_workspace_bytes).  No L x L map is stored. */
+size_t mta_attn_bwd_workspace_bytes(const mta_cfg *cfg);
+mta_status mta_attn_bwd(const void *q, const void *k, const void *v, const float *theta_kq,
+                        const float *w_head, const void *dout, const mta_cfg *cfg, float *dq,
+                        float *dk, float *dv, float *dtheta, float *dw);
+
 /* Waits for cfg->stream and reports whether a kernel of the last call that used
  * cfg->workspace gave up a bounded wait (MTA_ERR_TIMEOUT), else MTA_OK or
  * MTA_ERR_CUDA.  Blocking; for tests and diagnostics. */

@@ -76,7 +76,7 @@ def test_tiny_f32_L256(path):
 
 
 SMALL = []
-for d in (64, 128):
+for d in (64, 96, 128):
     for hp in (synth.OFF, synth.PRE, synth.POST):
         for L in (1, 9, 300):
             SMALL.append((d, hp, L))
@@ -91,7 +91,7 @@ def tc_applies(wl):
 
 def kq_applies(wl):
     """Whether the contraction kernel serves this configuration."""
-    return (wl.dtype == "bf16" and wl.d in (64, 128) and wl.kq_place in (synth.PRE, 3)
+    return (wl.dtype == "bf16" and wl.d in (64, 96, 128) and wl.kq_place in (synth.PRE, 3)
             and (wl.c_q, wl.c_k) == (6, 11)
             and (wl.head_place == synth.OFF or wl.c_h == 2))
 
@@ -103,6 +103,8 @@ def test_small_bf16(d, hp, L, path):
     wl = synth.shrink(base, B=2, H=4, L=L, d=d, head_place=hp, seed=77 + L + d + hp)
     if path == mta.PATH_KQ and not kq_applies(wl):
         pytest.skip("the contraction kernel does not take this configuration")
+    if path == mta.PATH_TC and not tc_applies(wl):
+        pytest.skip("the direct tensor-core kernel does not take this configuration")
     inp = synth.make_attn_inputs(wl)
     assert_close(run_attn(wl, inp, path), oracle_full(wl, inp), "bf16")
 
@@ -407,7 +409,7 @@ def test_post_conv_small(dtype, kq, hp, L):
     assert_close(run_attn(wl, inp), oracle_full(wl, inp), dtype)
 
 
-POST_PATHS = [(d, hp, L) for d in (64, 128) for hp in (synth.OFF, synth.PRE, synth.POST)
+POST_PATHS = [(d, hp, L) for d in (64, 96, 128) for hp in (synth.OFF, synth.PRE, synth.POST)
               for L in (9, 300)]
 
 
@@ -490,3 +492,115 @@ def test_post_conv_layer_small(hp):
                       inp["eps"], inp["lam"], inp["wo"], wl.H, wl.c_h, wl.kq_place, wl.head_place,
                       theta_post=inp["theta_post"])
     assert_close(out, ref, "bf16")
+
+
+# ---------------------------------------------------------------------------
+# head dimension 96 (the pages' 880M model: dimension 1536 over 16 heads)
+# ---------------------------------------------------------------------------
+
+def test_d96_full_size_sampled():
+    wl = synth.WORKLOADS["pretrain_d96_L2048"]
+    assert kq_applies(wl)
+    inp = synth.make_attn_inputs(wl)
+    out = run_attn(wl, inp)
+    rows = sample_rows(wl, seed=7)
+    ref = O.mta_attention_rows(inp["q"], inp["k"], inp["v"], inp["theta"], inp["w"], wl.c_h, rows,
+                               wl.kq_place, wl.head_place)
+    got = torch.stack([out[b, i] for b, i in rows])
+    assert_close(got, ref, "bf16")
+
+
+@pytest.mark.parametrize("kq,post", [(synth.PRE, False), (mta.PRE_EXACT, False), (synth.PRE, True)])
+def test_d96_kq_variants(kq, post):
+    base = synth.WORKLOADS["pretrain_d96_L2048"]
+    wl = synth.shrink(base, B=1, H=4, L=260, kq_place=kq, kq_post=post, seed=701 + kq + 2 * post)
+    inp = synth.make_attn_inputs(wl)
+    assert_close(run_attn(wl, inp, mta.PATH_KQ), oracle_full(wl, inp), "bf16")
+
+
+@pytest.mark.parametrize("hp", [synth.PRE, synth.POST])
+def test_d96_layer_small(hp):
+    wl = synth.shrink(synth.WORKLOADS["layer_post_D2048_L4096"], B=2, L=200, D=192, H=2, d=96,
+                      head_place=hp, seed=126)
+    inp = synth.make_layer_inputs(wl)
+    out = run_layer(wl, inp)
+    ref = O.mta_layer(inp["x"], inp["wqkv"], inp["theta"], inp["w"], inp["gamma"], inp["beta"],
+                      inp["eps"], inp["lam"], inp["wo"], wl.H, wl.c_h, wl.kq_place, wl.head_place)
+    assert_close(out, ref, "bf16")
+
+
+# ---------------------------------------------------------------------------
+# backward pass (mta_attn_bwd): every gradient against the fp64 oracle
+# ---------------------------------------------------------------------------
+
+GRAD_NAMES = ("dq", "dk", "dv", "dtheta", "dw")
+
+
+def run_bwd(wl, inp, dout):
+    q, k, v = (dev(inp[n], wl.dtype) for n in ("q", "k", "v"))
+    g = mta.attn_bwd(q, k, v, dev(inp["theta"], "f32"), dev(inp["w"], "f32"), dev(dout, wl.dtype),
+                     wl.c_q, wl.c_k, wl.c_h, wl.kq_place, wl.head_place, check=True)
+    torch.cuda.synchronize()
+    return g
+
+
+def check_grads(wl, inp, dout, tol=TOL_F32):
+    got = run_bwd(wl, inp, dout)
+    ref = O.mta_attention_bwd(inp["q"], inp["k"], inp["v"], inp["theta"], inp["w"], wl.c_h, dout,
+                              wl.kq_place, wl.head_place)
+    for n in GRAD_NAMES:
+        if ref[n] is None:
+            assert got[n] is None
+            continue
+        rel, mx = errs(got[n], ref[n])
+        assert rel <= tol, (n, rel, mx)
+
+
+BWD_SMALL = [("f32", synth.PRE, synth.POST, 9), ("f32", synth.PRE, synth.PRE, 70),
+             ("f32", synth.OFF, synth.OFF, 70), ("f32", mta.PRE_EXACT, synth.POST, 70),
+             ("bf16", synth.PRE, synth.POST, 70), ("bf16", synth.PRE, synth.OFF, 33),
+             ("bf16", synth.OFF, synth.POST, 40), ("bf16", mta.PRE_EXACT, synth.PRE, 50)]
+
+
+@pytest.mark.parametrize("dtype,kq,hp,L", BWD_SMALL)
+def test_bwd_small(dtype, kq, hp, L):
+    base = synth.WORKLOADS["pretrain_d128_L2048"]
+    wl = synth.shrink(base, B=2, H=4, L=L, d=32, kq_place=kq, head_place=hp, dtype=dtype,
+                      seed=801 + L + kq + 3 * hp)
+    inp = synth.make_attn_inputs(wl)
+    dout = synth.normal(wl.seed, 20, (wl.B, wl.L, wl.H, wl.d))
+    if dtype == "bf16":
+        dout = synth.round_bf16(dout)
+    check_grads(wl, inp, dout)
+
+
+def test_bwd_other_kernel_sizes():
+    base = synth.WORKLOADS["pretrain_d128_L2048"]
+    wl = synth.shrink(base, B=1, H=8, L=45, d=16, c_q=3, c_k=5, c_h=4, seed=850)
+    inp = synth.make_attn_inputs(wl)
+    dout = synth.round_bf16(synth.normal(wl.seed, 20, (wl.B, wl.L, wl.H, wl.d)))
+    check_grads(wl, inp, dout)
+
+
+def test_bwd_pretrain_recipe_L512():
+    """The pretraining recipe (d = 128, c_q = 6, c_k = 11, post-softmax mixing) at a
+    length the fp64 oracle finishes in seconds: four tiles of 128 keys."""
+    wl = synth.shrink(synth.WORKLOADS["pretrain_d128_L2048"], B=1, H=4, L=512, seed=851)
+    inp = synth.make_attn_inputs(wl)
+    dout = synth.round_bf16(synth.normal(wl.seed, 20, (wl.B, wl.L, wl.H, wl.d)))
+    check_grads(wl, inp, dout)
+
+
+def test_bwd_rejects_post_softmax_convolution():
+    wl = synth.shrink(synth.WORKLOADS["both_d128_L2048"], B=1, H=2, L=16, d=32)
+    inp = synth.make_attn_inputs(wl)
+    q, k, v = (dev(inp[n]) for n in "qkv")
+    cfg = mta.make_cfg(1, 2, 16, 32, 6, 11, 2, synth.PRE, synth.POST, mta.BF16, kq_post=1)
+    ws = mta.workspace(256)
+    cfg.workspace, cfg.workspace_bytes = ws.data_ptr(), ws.numel()
+    z = torch.zeros((1, 16, 2, 32), dtype=torch.float32, device="cuda")
+    th = dev(np.concatenate([inp["theta"], inp["theta_post"]]), "f32")
+    code = mta.lib().mta_attn_bwd(mta._ptr(q), mta._ptr(k), mta._ptr(v), mta._ptr(th),
+                                  mta._ptr(dev(inp["w"], "f32")), mta._ptr(q), ctypes.byref(cfg),
+                                  mta._ptr(z), mta._ptr(z), mta._ptr(z), None, None)
+    assert code == 2

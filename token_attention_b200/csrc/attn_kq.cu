@@ -69,19 +69,22 @@ struct KGeo {
   // or after the output query (exact indicator); Vp[i][m] = q[i] . k[i-m+OFF]
   static constexpr int C = CK / 2, HALO = CQ - 1, W = EXACT ? C : HALO + C, M = HALO + 2 * C;
   static constexpr int OFF = EXACT ? HALO : 0;
-  static constexpr int BM = 128, BN = 128, HALF = BN / 2, DH = D / 2;
+  static constexpr int BM = 128, BN = 128, HALF = BN / 2;
+  // output channels: warpgroup 0 takes DH (a multiple of 32), warpgroup 1 the other DH1
+  static constexpr int DH = (D / 2 + 31) / 32 * 32, DH1 = D - DH;
   static constexpr int QROWS = (BM + HALO + 7) / 8 * 8;  // query rows staged (with halo)
   static constexpr int NSTRIP = D / 8;
   static constexpr int STRIP = QROWS * 16;               // bytes of one 8-element strip
   static constexpr int Q_BYTES = NSTRIP * STRIP;
-  static constexpr int NDC = D / 64;
-  static constexpr int NCH = CQ * NDC;                   // Kt chunks per key tile
+  static constexpr int NDC = (D + 63) / 64;              // 64-channel blocks of a V row
+  // Kt row of a key = the c_q*D contraction operand, in 64-element chunks
+  static constexpr int NCH = CQ * D / 64;                // Kt chunks per key tile
   static constexpr int KCHUNK = BN * 128;                // 128 keys x 64 elements, fp16
   static constexpr int NV = MIX == 2 ? 2 : 1;            // V heads per CTA (post-softmax mixing: both)
   static constexpr int NSRC = MIX == 1 ? 2 : 1;          // heads whose C a CTA computes (pre-softmax mixing: both)
   static constexpr int CLUSTER = MIX == 2 ? 2 : 1;       // CTAs of a cluster: the heads of a group
   static constexpr int V_CHUNK = BN * 128;
-  static constexpr int V_HEAD = BN * D * 2;
+  static constexpr int V_HEAD = NDC * V_CHUNK;            // a V tile: 64-channel boxes (the last may pass D)
   // with the post-softmax convolution the convolved values stream through the Kt
   // ring, and the normalised weights go to shared memory (8-key strips, 16-byte
   // rows, PS_PAD rows of padding above row 0 for the row shifts)
@@ -99,18 +102,19 @@ struct KGeo {
   static constexpr int CS_BYTES = 2 * BM * W * 4;        // band values, one block per warpgroup
   static constexpr int RED_BYTES = 10 * BM * 4;          // row maxima (2 tiles x 2 groups), l, norm sums
   static constexpr int FAC_BYTES = NSRC * 2 * BN * 4;    // column factors of two key tiles, per source head
-  static constexpr int Q_ALLOC = (Q_BYTES + 1023) / 1024 * 1024;
+  static constexpr int Q_ALLOC = Q_BYTES;                              // query tiles of the sources, back to back
+  static constexpr int Q_AREA = (NSRC * Q_ALLOC + 1023) / 1024 * 1024;  // up to the 1024-aligned ring
   // small area: taps [2 items][NSRC][128], per-warp |q| maxima, barriers, TMEM slot, abort flag
   static constexpr int TH_OFF = 0, THP_OFF = 2 * NSRC * 128 * 4;
   static constexpr int QRED_OFF = THP_OFF + (POST ? 2 * 128 * 4 : 0), BAR_OFF = QRED_OFF + 64;
   static constexpr int TSLOT_OFF = BAR_OFF + 8 * 32, ABORT_OFF = TSLOT_OFF + 8;
   static constexpr int SMALL_BYTES = (ABORT_OFF + 8 + 255) / 256 * 256;
   // Kt ring: as many 16 KB stages as the shared memory left over holds (at most 8)
-  static constexpr int REST = NSRC * Q_ALLOC + V_BYTES + PS_BYTES + DG_BYTES + NSRC * U_BYTES + CS_BYTES +
+  static constexpr int REST = Q_AREA + V_BYTES + PS_BYTES + DG_BYTES + NSRC * U_BYTES + CS_BYTES +
                               RED_BYTES + FAC_BYTES + SMALL_BYTES + 1024;
   static constexpr int NS = (232448 - REST) / KCHUNK < 8 ? (232448 - REST) / KCHUNK : 8;
   static constexpr int OFF_Q = 0;
-  static constexpr int OFF_K = NSRC * Q_ALLOC;
+  static constexpr int OFF_K = Q_AREA;
   static constexpr int OFF_V = OFF_K + NS * KCHUNK;
   static constexpr int OFF_PS = OFF_V + V_BYTES;
   static constexpr int OFF_DG = OFF_PS + PS_BYTES;
@@ -135,6 +139,7 @@ struct KGeo {
   static_assert(11 + 2 * NS <= 32, "barrier slots");
   static_assert(SMEM <= 232448, "shared memory");
   static_assert(CQ * CK <= 120, "kernel taps");
+  static_assert(CQ * D % 64 == 0 && D % 16 == 0, "contraction chunks");
 };
 
 struct KqParams {
@@ -280,8 +285,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         auto load_c = [&](int t) -> bool {
           for (int ch = 0; ch < G::NSRC * G::NCH; ++ch) {
             const int sc = ch / G::NCH, cs = ch % G::NCH;
-            const int zbase = (it.b * p.H + src_head(h, sc)) * CQ;
-            if (!push(&tmK, (cs % G::NDC) * 64, t * G::BN, zbase + cs / G::NDC)) return false;
+            if (!push(&tmK, 0, t * G::BN, (it.b * p.H + src_head(h, sc)) * G::NCH + cs)) return false;
           }
           return true;
         };
@@ -355,23 +359,29 @@ __global__ void __launch_bounds__(kThreads, 1)
       int cnt = 0, T = 0;  // ring chunks and C tiles issued so far (all items)
       int npv = 0;         // P V tiles issued (POST)
       bool ok = true;
-      // C of global key tile T = sum over the NCH chunks (a, 64-wide d block) of Q
-      // shifted by a rows x Kt_a
+      // C of global key tile T = sum over the NCH 64-element chunks of the c_q*D
+      // contraction; element kappa = a*D + e pairs Q shifted by a rows with Kt_a
       auto issue_c = [&](bool last_of_item) -> bool {
         if (T > 0 && !mbar_wait(c_free, (T - 1) & 1, abort_flag, p.err)) return false;
         for (int ch = 0; ch < G::NSRC * G::NCH; ++ch, ++cnt) {
           const int st = cnt % G::NS;
+          // source head sc (its own accumulator and query rows); the 16 elements
+          // kappa = 64 cs + 16 kk of step kk: tap row a, channels e0 .. e0+15 (D is a
+          // multiple of 16, so a step never straddles two tap rows); Q rows shifted up
+          // by a (16 bytes per row), 8-channel strips e0/8 and e0/8 + 1
+          const int sc = ch / G::NCH, cs = ch % G::NCH;
+          uint64_t qd[4];
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk) {
+            const int kap = 64 * cs + 16 * kk, a = kap / D, e0 = kap % D;
+            qd[kk] = qdesc0 + static_cast<uint32_t>((sc * G::Q_ALLOC + (e0 / 8) * G::STRIP + 16 * (G::HALO - a)) >> 4);
+          }
+          const uint64_t kd = kdesc0 + static_cast<uint32_t>((st * G::KCHUNK) >> 4);
           if (!mbar_wait(k_full + st, (cnt / G::NS) & 1, abort_flag, p.err)) return false;
           tc_fence_after();
-          // source head sc (its own accumulator and query rows), tap row a, 64-channel block dc
-          const int sc = ch / G::NCH, cs = ch % G::NCH, a = cs / G::NDC, dc = cs % G::NDC;
-          // Q rows shifted up by a (16 bytes per row), 64-channel block dc
-          const uint64_t qd = qdesc0 + static_cast<uint32_t>((sc * G::Q_ALLOC + 8 * dc * G::STRIP + 16 * (G::HALO - a)) >> 4);
-          const uint64_t kd = kdesc0 + static_cast<uint32_t>((st * G::KCHUNK) >> 4);
 #pragma unroll
           for (int kk = 0; kk < 4; ++kk)
-            mma_bf16_ss(tmem + G::C_COL + 128 * sc, qd + (2 * kk * G::STRIP >> 4), kd + 2 * kk, idesc_c,
-                        (cs > 0 || kk > 0));
+            mma_bf16_ss(tmem + G::C_COL + 128 * sc, qd[kk], kd + 2 * kk, idesc_c, (cs > 0 || kk > 0));
           mma_commit(k_empty + st);
         }
         mma_commit(c_full);
@@ -444,7 +454,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int r_ = 32 * q4 + lane;           // query row of this thread = TMEM lane
     const int st_id = threadIdx.x;           // 0..255
     const int cb = G::HALF * wg;             // key columns of this warpgroup
-    const int zc = G::DH * wg;               // output channels of this warpgroup
+    const int zc = G::DH * wg;               // output channels of this warpgroup: zc .. zc+zn-1
+    const int zn = wg ? G::DH1 : G::DH;
     const uint32_t tl = tmem + (static_cast<uint32_t>(32 * q4) << 16);
     const float sc0 = p.qk_scale * kLog2e;
     float *crow = Cs + (wg * G::BM + r_) * G::W;
@@ -532,7 +543,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       // item's or the next item's first)
       auto fac_next = [&](int sc, int sl) -> float {
         if (sl + 1 < nsl)
-          return p.fac[(static_cast<long long>(it.b) * p.H + src_head(h, sc)) * p.lpad + ((sl + 1) % n_kv) * G::BN + st_id];
+          return p.fac[(static_cast<long long>(it.b) * p.H + src_head(h, sc)) * p.lpad +
+                       (POST ? (sl + 1) % n_kv : sl + 1) * G::BN + st_id];
         if (more) return p.fac[(static_cast<long long>(nx.b) * p.H + src_head(h_nx, sc)) * p.lpad + st_id];
         return 0.f;
       };
@@ -678,6 +690,7 @@ __global__ void __launch_bounds__(kThreads, 1)
               for (int hd = 0; hd < G::NV; ++hd)
 #pragma unroll 1
                 for (int c0 = 0; c0 < G::DH; c0 += 32) {
+                  if (c0 >= zn) break;
                   uint32_t z[32];
                   const uint32_t za = tl + G::Z_COL0 + 128 * hd + zc + c0;
                   tmem_ld32(za, z);
@@ -815,6 +828,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                                (static_cast<long long>(2 * c + (hr ^ 1)) * 2 + (r & 1)) * (G::BM * D / 4);
 #pragma unroll
         for (int c0 = 0; c0 < G::DH; c0 += 32) {
+          if (c0 >= zn) break;
           float zo[32];
           z_chunk(hr ^ 1, 2 * g + (hr ^ 1), c0, zo);
 #pragma unroll
@@ -825,9 +839,9 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
         for (int c0 = 0; c0 < G::DH; c0 += 32) {
           float zo[32];
-          z_chunk(hr, 2 * g + hr, c0, zo);
+          if (c0 < zn) z_chunk(hr, 2 * g + hr, c0, zo);
 #pragma unroll
-          for (int i = 0; i < 32; ++i) o[c0 + i] = w_own * zo[i];
+          for (int i = 0; i < 32; ++i) o[c0 + i] = c0 < zn ? w_own * zo[i] : 0.f;
         }
         tc_fence_before();
         __syncwarp();
@@ -837,6 +851,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         mbar_wait_cluster(x_ready, r & 1, abort_flag, p.err);
 #pragma unroll
         for (int c4 = 0; c4 < G::DH / 4; ++c4) {
+          if (4 * c4 >= zn) break;
           const float4 x = theirs[(zc / 4 + c4) * G::BM + r_];
           o[4 * c4] += w_peer * x.x;
           o[4 * c4 + 1] += w_peer * x.y;
@@ -847,9 +862,9 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
         for (int c0 = 0; c0 < G::DH; c0 += 32) {
           float zo[32];
-          z_chunk(0, h, c0, zo);
+          if (c0 < zn) z_chunk(0, h, c0, zo);
 #pragma unroll
-          for (int i = 0; i < 32; ++i) o[c0 + i] = zo[i];
+          for (int i = 0; i < 32; ++i) o[c0 + i] = c0 < zn ? zo[i] : 0.f;
         }
         tc_fence_before();
         __syncwarp();
@@ -858,13 +873,13 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (p.gn) {  // group norm over the D channels of (token, head), then depth scale
         float s = 0.f;
 #pragma unroll
-        for (int i = 0; i < G::DH; ++i) s += o[i];
+        for (int i = 0; i < G::DH; ++i) s += o[i];  // channels past zn are 0
         red[(6 + wg) * G::BM + r_] = s;
         named_bar_sync(kBarAll, kSmThreads);
         const float mu = (s + red[(6 + (wg ^ 1)) * G::BM + r_]) * (1.f / D);
         float s2 = 0.f;
 #pragma unroll
-        for (int i = 0; i < G::DH; ++i) { const float x = o[i] - mu; s2 += x * x; }
+        for (int i = 0; i < G::DH; ++i) { const float x = i < zn ? o[i] - mu : 0.f; s2 += x * x; }
         red[(8 + wg) * G::BM + r_] = s2;
         named_bar_sync(kBarAll, kSmThreads);
         const float rstd = rsqrtf((s2 + red[(8 + (wg ^ 1)) * G::BM + r_]) * (1.f / D) + p.eps);
@@ -872,12 +887,14 @@ __global__ void __launch_bounds__(kThreads, 1)
         const float *bt = p.beta + static_cast<long long>(h) * D + zc;
         const float mh = head_multiplier(p.gate, p.lam, h);
 #pragma unroll
-        for (int i = 0; i < G::DH; ++i) o[i] = ((o[i] - mu) * rstd * gm[i] + bt[i]) * mh;
+        for (int i = 0; i < G::DH; ++i)
+          if (i < zn) o[i] = ((o[i] - mu) * rstd * gm[i] + bt[i]) * mh;
       }
       if (out_row) {
         __nv_bfloat16 *dst = p.out + ((static_cast<long long>(it.b) * L + qi) * p.H + h) * D + zc;
 #pragma unroll
         for (int i = 0; i < G::DH; i += 8) {
+          if (i >= zn) break;
           uint4 v;
           v.x = pack_bf16x2(o[i], o[i + 1]);
           v.y = pack_bf16x2(o[i + 2], o[i + 3]);
@@ -912,18 +929,19 @@ cudaError_t launch_kq_one(const AttnArgs &a, const GnArgs *gn, const KqPrepArgs 
   const unsigned boxq[4] = {8, 1, G::QROWS, 1}, boxv[4] = {64, 1, G::BN, 1};
   if (!encode_tmap_bf16(&tq, a.q, 4, dims, str, boxq, false)) return cudaErrorInvalidValue;
   if (!encode_tmap_bf16(&tv, a.v, 4, dims, str, boxv, true)) return cudaErrorInvalidValue;
-  // Kt: [B*H*CQ][L][D] 16-bit elements (the copy moves bytes; fp16 as 16-bit)
-  const unsigned long long kdims[3] = {static_cast<unsigned long long>(D), static_cast<unsigned long long>(a.L),
-                                       static_cast<unsigned long long>(a.B) * a.H * CQ};
-  const unsigned long long kstr[2] = {static_cast<unsigned long long>(D) * 2,
-                                      static_cast<unsigned long long>(a.L) * D * 2};
+  // Kt: [B*H*NCH][L][64] 16-bit elements (the copy moves bytes; fp16 as 16-bit)
+  const unsigned long long kdims[3] = {64, static_cast<unsigned long long>(a.L),
+                                       static_cast<unsigned long long>(a.B) * a.H * G::NCH};
+  const unsigned long long kstr[2] = {128, static_cast<unsigned long long>(a.L) * 128};
   const unsigned boxk[3] = {64, G::BN, 1};
   if (!encode_tmap_bf16(&tk, pa.kt, 3, kdims, kstr, boxk, true)) return cudaErrorInvalidValue;
   tvt = tk;
   if (POST) {  // convolved values: [B*H*NV*CQ][L][D] bf16, 64-channel x 128-key boxes
     const unsigned long long vdims[3] = {static_cast<unsigned long long>(D), static_cast<unsigned long long>(a.L),
                                          static_cast<unsigned long long>(a.B) * a.H * G::NV * CQ};
-    if (!encode_tmap_bf16(&tvt, vt, 3, vdims, kstr, boxk, true)) return cudaErrorInvalidValue;
+    const unsigned long long vstr[2] = {static_cast<unsigned long long>(D) * 2,
+                                        static_cast<unsigned long long>(a.L) * D * 2};
+    if (!encode_tmap_bf16(&tvt, vt, 3, vdims, vstr, boxk, true)) return cudaErrorInvalidValue;
   }
   KqParams p;
   p.theta = a.theta;
@@ -980,7 +998,7 @@ size_t align256(size_t x) { return (x + 255) / 256 * 256; }
 }  // namespace
 
 bool attn_kq_supported(const AttnArgs &a) {
-  if (a.dtype != 1 || (a.d != 64 && a.d != 128)) return false;
+  if (a.dtype != 1 || (a.d != 64 && a.d != 96 && a.d != 128)) return false;
   if ((a.kq != 1 && a.kq != 3) || a.cq != 6 || a.ck != 11) return false;
   if (!(a.hp == 0 || ((a.hp == 1 || a.hp == 2) && a.ch == 2))) return false;
   if (a.B > 65535 || a.H > 65535 || (a.L + 127) / 128 > 65535) return false;
@@ -997,7 +1015,7 @@ size_t kq_items(int B, int H, int L, int kqp) {
 }
 }  // namespace
 
-// Workspace of the contraction path: Kt [B][H][c_q][L][d] fp16 | fac [B][H][Lpad] fp32 |
+// Workspace of the contraction path: Kt [B][H][c_q*d/64][L][64] fp16 | fac [B][H][Lpad] fp32 |
 // Vp [B][H][L][M] fp32 | (post-softmax mixing) the exchange buffer of the persistent
 // CTAs, [CTAs][2][d][128] fp32 | (post-softmax convolution) the convolved values
 // Vt [B][H][nvh][c_q][L][d] bf16, nvh = 2 with post-softmax mixing, else 1;
@@ -1059,11 +1077,13 @@ cudaError_t launch_attn_kq(const AttnArgs &a, const GnArgs *gn, void *ws) {
                     : launch_kq_one<DD, 6, 11, MX, false, false>(a, gn, pa, xg, vt);
   };
   using D64 = std::integral_constant<int, 64>;
+  using D96 = std::integral_constant<int, 96>;
   using D128 = std::integral_constant<int, 128>;
   using M0 = std::integral_constant<int, 0>;
   using M1 = std::integral_constant<int, 1>;
   using M2 = std::integral_constant<int, 2>;
   if (a.d == 128) return a.hp == 2 ? go(D128{}, M2{}) : a.hp == 1 ? go(D128{}, M1{}) : go(D128{}, M0{});
+  if (a.d == 96) return a.hp == 2 ? go(D96{}, M2{}) : a.hp == 1 ? go(D96{}, M1{}) : go(D96{}, M0{});
   return a.hp == 2 ? go(D64{}, M2{}) : a.hp == 1 ? go(D64{}, M1{}) : go(D64{}, M0{});
 }
 

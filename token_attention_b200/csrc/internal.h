@@ -36,6 +36,23 @@ size_t attn_simt_smem_bytes(const AttnArgs &a, int BR, int BC);
 int attn_simt_pick_rows(const AttnArgs &a, int BC);  // 0 if nothing fits
 cudaError_t launch_attn_simt(const AttnArgs &a);
 
+// Backward pass of the attention (CUDA cores, fp32 arithmetic).
+struct BwdArgs {
+  const void *q, *k, *v;  // [B][L][H][d], token stride rs
+  long long rs;
+  const void *dout;       // [B][L][H][d] dense, gradient of the output
+  const float *theta;     // [H][c_q][c_k]
+  const float *w;         // [H/c_h][c_h][c_h]
+  float *dq, *dk, *dv;    // [B][L][H][d] dense fp32
+  float *dtheta;          // [H][c_q][c_k] or null
+  float *dw;              // [H/c_h][c_h][c_h] or null
+  int B, H, L, d, cq, ck, ch, kq, hp, dtype;
+  float scale;
+  cudaStream_t stream;
+};
+int attn_bwd_simt_pick_rows(const BwdArgs &a);  // 0 if nothing fits
+cudaError_t launch_attn_bwd_simt(const BwdArgs &a);
+
 // tcgen05 kernel (bf16, fused); attn_tc_supported() says whether it applies.
 bool attn_tc_supported(const AttnArgs &a);
 cudaError_t launch_attn_tc(const AttnArgs &a, const GnArgs *gn);
@@ -47,7 +64,7 @@ struct KqPrepArgs {
   const void *q, *k;      // [B][L][H][d] bf16, token stride rs
   long long rs;
   const float *theta;     // [H][c_q][c_k]
-  void *kt;               // [B][H][c_q][L][d] fp16, key row j scaled by 2^e_j
+  void *kt;               // [B][H][c_q*d/64][L][64] fp16, key j's contraction operand by 64-element chunks, times 2^e_j
   float *fac;             // [B][H][lpad] scale_log2 * 2^-e_j (0 for j >= L)
   float *vp;              // [B][H][L][M] past dot products q[i] . k[i-m], m < M
   float scale_log2;       // logit scale times log2(e)

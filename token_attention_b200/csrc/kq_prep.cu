@@ -12,7 +12,10 @@
 // which covers every unmasked tap of the band (m = i-a - key >= 0).
 //
 // This kernel writes, per (batch, head, tile of 128 keys):
-//   Kt  [B][H][c_q][L][d] fp16: Kt_a[j] * 2^e_j, e_j a power-of-2 exponent per key
+//   Kt  [B][H][c_q*d/64][L][64] fp16: element kappa = a*d + e of key j's contraction
+//       operand (Kt_a[j][e]) sits in chunk kappa/64 at column kappa%64, so that the 128
+//       keys of a tile form one contiguous 16 KB block per chunk; every value is
+//       Kt_a[j] * 2^e_j, e_j a power-of-2 exponent per key
 //       row chosen from max|k| over the rows j-c .. j+c that Kt_a[j] reads (so no
 //       value exceeds 2^14 and small keys keep fp16's relative precision);
 //   fac [B][H][Lpad] fp32: s * log2(e) * 2^-e_j (the attention kernel's column
@@ -28,6 +31,8 @@
 #include <cuda_fp16.h>
 #include <math.h>
 #include <stdint.h>
+
+#include <type_traits>
 
 #include "internal.h"
 
@@ -127,7 +132,7 @@ __global__ void __launch_bounds__(kPrepThreads, 3) kq_prep_kernel(KqPrepArgs p) 
   // Kt_a[j] = sum_t theta[a][t] k[j - (t - c)]: each work item is one pair of
   // channels x kRun consecutive keys, convolved from a register window of rows.
   __half *kt = static_cast<__half *>(p.kt);
-  const long long LD = static_cast<long long>(L) * D;  // elements between the Kt_a of one head
+  constexpr int NCHK = CQ * D / 64;  // 64-element chunks of a key's contraction operand
   constexpr int NPAIR = D / 2, NRUN = kTile / kRun;
   for (int item = tid; item < NPAIR * NRUN; item += kPrepThreads) {
     const int e2 = (item % NPAIR) * 2, jr = (item / NPAIR) * kRun;
@@ -140,7 +145,7 @@ __global__ void __launch_bounds__(kPrepThreads, 3) kq_prep_kernel(KqPrepArgs p) 
     float scu[kRun];
 #pragma unroll
     for (int u = 0; u < kRun; ++u) scu[u] = pow2i(es[jr + u]);
-    __half *o0 = kt + (bh * CQ * L + j0 + jr) * D + e2;
+    __half *o0 = kt + (bh * NCHK * L + j0 + jr) * 64;  // chunk 0, key j0+jr
 #pragma unroll
     for (int a = 0; a < CQ; ++a) {
       // kRun x 2 independent accumulators; taps in the outer loop (no dependent chains)
@@ -156,11 +161,12 @@ __global__ void __launch_bounds__(kPrepThreads, 3) kq_prep_kernel(KqPrepArgs p) 
           acc[u].y = fmaf(ta, win[u + 2 * G::C - t].y, acc[u].y);
         }
       }
-      __half *oa = o0 + a * LD;
+      const int kap = a * D + e2;  // contraction element of channel pair e2 in tap row a
+      __half *oa = o0 + static_cast<long long>(kap / 64) * L * 64 + kap % 64;
 #pragma unroll
       for (int u = 0; u < kRun; ++u)
         if (nkeys == kRun || u < nkeys)
-          *reinterpret_cast<__half2 *>(oa + u * D) = __floats2half2_rn(acc[u].x * scu[u], acc[u].y * scu[u]);
+          *reinterpret_cast<__half2 *>(oa + u * 64) = __floats2half2_rn(acc[u].x * scu[u], acc[u].y * scu[u]);
     }
   }
 
@@ -299,15 +305,21 @@ cudaError_t launch_vt_one(const VtPrepArgs &p, cudaStream_t stream) {
 cudaError_t launch_vt_prep(const VtPrepArgs &p, cudaStream_t stream) {
   if (p.cq != 6 || p.ck != 11 || (p.nvh != 1 && p.nvh != 2)) return cudaErrorInvalidValue;
   if (p.d == 128) return p.nvh == 2 ? launch_vt_one<128, 2>(p, stream) : launch_vt_one<128, 1>(p, stream);
+  if (p.d == 96) return p.nvh == 2 ? launch_vt_one<96, 2>(p, stream) : launch_vt_one<96, 1>(p, stream);
   if (p.d == 64) return p.nvh == 2 ? launch_vt_one<64, 2>(p, stream) : launch_vt_one<64, 1>(p, stream);
   return cudaErrorInvalidValue;
 }
 
 cudaError_t launch_kq_prep(const KqPrepArgs &p, cudaStream_t stream) {
   if (p.cq != 6 || p.ck != 11 || p.M != PrepGeo<128, 6, 11, false>::M) return cudaErrorInvalidValue;
-  if (p.exact)
-    return p.d == 128 ? launch_prep_one<128, 6, 11, true>(p, stream) : launch_prep_one<64, 6, 11, true>(p, stream);
-  return p.d == 128 ? launch_prep_one<128, 6, 11, false>(p, stream) : launch_prep_one<64, 6, 11, false>(p, stream);
+  auto go = [&](auto d_tag) -> cudaError_t {
+    constexpr int DD = decltype(d_tag)::value;
+    return p.exact ? launch_prep_one<DD, 6, 11, true>(p, stream) : launch_prep_one<DD, 6, 11, false>(p, stream);
+  };
+  if (p.d == 128) return go(std::integral_constant<int, 128>{});
+  if (p.d == 96) return go(std::integral_constant<int, 96>{});
+  if (p.d == 64) return go(std::integral_constant<int, 64>{});
+  return cudaErrorInvalidValue;
 }
 
 }  // namespace mta

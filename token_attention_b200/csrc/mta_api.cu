@@ -66,7 +66,7 @@ enum Kernel { K_SIMT = 1, K_TC = 2, K_KQ = 3 };
 // Shape-level test for the contraction kernel (pointer alignment aside): used
 // to size the workspace.
 bool kq_shape_ok(const mta_cfg *c) {
-  return c->dtype == MTA_BF16 && (c->d == 64 || c->d == 128) &&
+  return c->dtype == MTA_BF16 && (c->d == 64 || c->d == 96 || c->d == 128) &&
          (c->kq_place == MTA_PRE || c->kq_place == MTA_PRE_EXACT) &&
          c->c_q == 6 && c->c_k == 11 &&
          (c->head_place == MTA_OFF || ((c->head_place == MTA_PRE || c->head_place == MTA_POST) && c->c_h == 2));
@@ -284,6 +284,37 @@ mta_status mta_layer_fwd(const void *x, const void *Wqkv, const float *theta, co
                           static_cast<int>(D), err, st) != cudaSuccess)
     return MTA_ERR_CUDA;
   return MTA_OK;
+}
+
+size_t mta_attn_bwd_workspace_bytes(const mta_cfg *cfg) {
+  return check_cfg(cfg) == MTA_OK ? kStatusBytes : 0;
+}
+
+mta_status mta_attn_bwd(const void *q, const void *k, const void *v, const float *theta_kq,
+                        const float *w_head, const void *dout, const mta_cfg *cfg, float *dq,
+                        float *dk, float *dv, float *dtheta, float *dw) {
+  mta_status s = check_cfg(cfg);
+  if (s != MTA_OK) return s;
+  if (cfg->kq_post || cfg->path > 1) return MTA_ERR_UNSUPPORTED;
+  if ((s = check_attn_pointers(q, k, v, theta_kq, w_head, cfg, dout)) != MTA_OK) return s;
+  if (!dq || !dk || !dv || !aligned(dq, 4) || !aligned(dk, 4) || !aligned(dv, 4)) return MTA_ERR_INVALID;
+  if ((dtheta && !aligned(dtheta, 4)) || (dw && !aligned(dw, 4))) return MTA_ERR_INVALID;
+  if ((s = check_workspace(cfg, kStatusBytes)) != MTA_OK) return s;
+  BwdArgs a;
+  a.q = q; a.k = k; a.v = v; a.dout = dout;
+  a.rs = cfg->qkv_row_stride ? cfg->qkv_row_stride : static_cast<long long>(cfg->H) * cfg->d;
+  a.theta = theta_kq; a.w = w_head;
+  a.dq = dq; a.dk = dk; a.dv = dv;
+  a.dtheta = cfg->kq_place != MTA_OFF ? dtheta : nullptr;
+  a.dw = cfg->head_place != MTA_OFF ? dw : nullptr;
+  a.B = cfg->B; a.H = cfg->H; a.L = cfg->L; a.d = cfg->d;
+  a.cq = cfg->c_q; a.ck = cfg->c_k; a.ch = cfg->c_h;
+  a.kq = cfg->kq_place; a.hp = cfg->head_place; a.dtype = cfg->dtype;
+  a.scale = cfg->scale > 0.f ? cfg->scale : 1.0f / sqrtf(static_cast<float>(cfg->d));
+  a.stream = static_cast<cudaStream_t>(cfg->stream);
+  if (attn_bwd_simt_pick_rows(a) == 0) return MTA_ERR_UNSUPPORTED;
+  if ((s = clear_status(cfg)) != MTA_OK) return s;
+  return launch_attn_bwd_simt(a) == cudaSuccess ? MTA_OK : MTA_ERR_CUDA;
 }
 
 mta_status mta_gemm_bf16_nt(const void *A, const void *Bm, void *C, int M, int N, int K, void *stream) {

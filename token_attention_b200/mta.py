@@ -26,7 +26,8 @@ STATUS = {0: "MTA_OK", 1: "MTA_ERR_INVALID", 2: "MTA_ERR_UNSUPPORTED", 3: "MTA_E
 # Every function include/mta.h declares.
 EXPORTS = ["mta_attn_workspace_bytes", "mta_attn_fwd", "mta_layer_workspace_bytes",
            "mta_layer_fwd", "mta_gemm_bf16_nt", "mta_group_norm_scale", "mta_sync_status",
-           "mta_status_string", "mta_abi_version", "mta_layer_fwd_static"]
+           "mta_status_string", "mta_abi_version", "mta_layer_fwd_static",
+           "mta_attn_bwd_workspace_bytes", "mta_attn_bwd"]
 
 
 class MtaCfg(ctypes.Structure):
@@ -74,6 +75,10 @@ def lib() -> ctypes.CDLL:
         L.mta_gemm_bf16_nt.restype = I
         L.mta_group_norm_scale.argtypes = [P, ctypes.POINTER(MtaGn), I, I, I, P, P]
         L.mta_group_norm_scale.restype = I
+        L.mta_attn_bwd_workspace_bytes.argtypes = [cfgp]
+        L.mta_attn_bwd_workspace_bytes.restype = S
+        L.mta_attn_bwd.argtypes = [P, P, P, P, P, P, cfgp, P, P, P, P, P]
+        L.mta_attn_bwd.restype = I
         L.mta_sync_status.argtypes = [cfgp]
         L.mta_sync_status.restype = I
         L.mta_status_string.argtypes = [I]
@@ -167,6 +172,34 @@ def attn_fwd(q, k, v, theta, w, c_q, c_k, c_h, kq_place=PRE, head_place=POST, *,
     if check:
         _check("mta_sync_status", lib().mta_sync_status(ctypes.byref(cfg)))
     return out
+
+
+def attn_bwd(q, k, v, theta, w, dout, c_q, c_k, c_h, kq_place=PRE, head_place=POST, *, ws=None,
+             path=PATH_AUTO, scale=0.0, stream=None, check=False, grads=None):
+    """Gradients of attn_fwd.  dout: [B, L, H, d] dense, dtype of q.  Returns a dict
+    of fp32 tensors: dq, dk, dv [B, L, H, d], dtheta [H, c_q, c_k] (kq_place on)
+    and dw [H/c_h, c_h, c_h] (head_place on).  `grads` may pass that dict to reuse."""
+    import torch
+    B, L, H, d = q.shape
+    if dout.shape != q.shape or dout.dtype != q.dtype or not dout.is_contiguous():
+        raise ValueError("dout must be a dense [B, L, H, d] tensor of q's dtype")
+    if grads is None:
+        z = lambda *shape: torch.empty(shape, dtype=torch.float32, device=q.device)
+        grads = {"dq": z(B, L, H, d), "dk": z(B, L, H, d), "dv": z(B, L, H, d),
+                 "dtheta": z(H, c_q, c_k) if kq_place != OFF else None,
+                 "dw": z(H // c_h, c_h, c_h) if head_place != OFF else None}
+    cfg = make_cfg(B, H, L, d, c_q, c_k, c_h, kq_place, head_place, _dtype_code(q), path, scale,
+                   q.stride(1), _stream_handle(stream))
+    if ws is None:
+        ws = workspace(lib().mta_attn_bwd_workspace_bytes(ctypes.byref(cfg)), q.device)
+    cfg.workspace, cfg.workspace_bytes = ws.data_ptr(), ws.numel()
+    _check("mta_attn_bwd", lib().mta_attn_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(theta), _ptr(w),
+                                             _ptr(dout), ctypes.byref(cfg), _ptr(grads["dq"]),
+                                             _ptr(grads["dk"]), _ptr(grads["dv"]),
+                                             _ptr(grads["dtheta"]), _ptr(grads["dw"])))
+    if check:
+        _check("mta_sync_status", lib().mta_sync_status(ctypes.byref(cfg)))
+    return grads
 
 
 def depth_scale(layer: int) -> float:

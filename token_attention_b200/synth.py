@@ -127,6 +127,11 @@ WORKLOADS = {
                                        dtype="bf16", seed=1005, theta_kind="delta_noise",
                                        theta_std=0.05, w_kind="eye_noise", w_std=0.1,
                                        layer=True, D=2048),
+    # the pages' 880M pretraining shape: dimension 1536 over 16 heads (d = 96), L = 2048
+    "pretrain_d96_L2048": Workload("pretrain_d96_L2048", B=4, H=16, L=2048, d=96, c_q=6, c_k=11,
+                                   c_h=2, kq_place=PRE, head_place=POST, dtype="bf16", seed=1007,
+                                   theta_kind="delta_noise", theta_std=0.05, w_kind="eye_noise",
+                                   w_std=0.1),
     # the convolution on both sides of the softmax (the pages' default setting),
     # pretraining-shaped: post kernels drawn like the pre kernels
     "both_d128_L2048": Workload("both_d128_L2048", B=4, H=16, L=2048, d=128, c_q=6, c_k=11,
