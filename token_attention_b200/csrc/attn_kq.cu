@@ -56,10 +56,12 @@ namespace {
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kRescaleLog2 = 8.0f;
 // warps 0-7: two softmax warpgroups (warpgroup w takes key columns 64w .. 64w+63 of
-// every tile and half of the output channels); warp 8: TMA; warp 9: MMA
-constexpr int kThreads = 320;
+// every tile and half of the output channels); warp 8: TMA of the convolved keys
+// (and values); warp 9: MMA; warp 10: TMA of V and of the query rows (a warp of its
+// own, so that these waits never hold up the busier key stream)
+constexpr int kThreads = 352;
 constexpr int kSmThreads = 256;
-constexpr int kTmaWarp = 8, kMmaWarp = 9;
+constexpr int kTmaWarp = 8, kMmaWarp = 9, kTma2Warp = 10;
 constexpr int kBarAll = 1;      // named barrier over both softmax warpgroups
 constexpr int kKqMaxClusters = 160;  // persistent grid: at most this many CTAs (>= SM count)
 
@@ -80,6 +82,7 @@ struct KGeo {
   // Kt row of a key = the c_q*D contraction operand, in 64-element chunks
   static constexpr int NCH = CQ * D / 64;                // Kt chunks per key tile
   static constexpr int KCHUNK = BN * 128;                // 128 keys x 64 elements, fp16
+
   static constexpr int NV = MIX == 2 ? 2 : 1;            // V heads per CTA (post-softmax mixing: both)
   static constexpr int NSRC = MIX == 1 ? 2 : 1;          // heads whose C a CTA computes (pre-softmax mixing: both)
   static constexpr int CLUSTER = MIX == 2 ? 2 : 1;       // CTAs of a cluster: the heads of a group
@@ -112,10 +115,14 @@ struct KGeo {
   // Kt ring: as many 16 KB stages as the shared memory left over holds (at most 8)
   static constexpr int REST = Q_AREA + V_BYTES + PS_BYTES + DG_BYTES + NSRC * U_BYTES + CS_BYTES +
                               RED_BYTES + FAC_BYTES + SMALL_BYTES + 1024;
-  static constexpr int NS = (232448 - REST) / KCHUNK < 8 ? (232448 - REST) / KCHUNK : 8;
+  // a ring stage holds SB boxes: a whole tap row when d is a multiple of 64 and at
+  // least three such stages fit, else one box
+  static constexpr int SB = (D % 64 == 0 && (232448 - REST) / (NDC * KCHUNK) >= 3) ? NDC : 1;
+  static constexpr int KSTAGE = SB * KCHUNK;
+  static constexpr int NS = (232448 - REST) / KSTAGE < 8 ? (232448 - REST) / KSTAGE : 8;
   static constexpr int OFF_Q = 0;
   static constexpr int OFF_K = Q_AREA;
-  static constexpr int OFF_V = OFF_K + NS * KCHUNK;
+  static constexpr int OFF_V = OFF_K + NS * KSTAGE;
   static constexpr int OFF_PS = OFF_V + V_BYTES;
   static constexpr int OFF_DG = OFF_PS + PS_BYTES;
   static constexpr int OFF_U = OFF_DG + DG_BYTES;
@@ -136,6 +143,7 @@ struct KGeo {
   static_assert(OFF_PS % 16 == 0 && OFF_DG % 16 == 0 && OFF_U % 16 == 0, "alignment");
   static_assert(OFF_SMALL % 16 == 0, "alignment");
   static_assert(NS >= 3, "Kt ring");
+  static_assert(NCH % SB == 0 && NDC % SB == 0, "whole stages");
   static_assert(11 + 2 * NS <= 32, "barrier slots");
   static_assert(SMEM <= 232448, "shared memory");
   static_assert(CQ * CK <= 120, "kernel taps");
@@ -264,17 +272,20 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_after();
   const uint32_t tmem = *tslot;
 
-  if (warp == kTmaWarp) {
+  if (warp == kTmaWarp || warp == kTma2Warp) {
     // -------------------------------------------------------------- TMA
-    if (lane == 0) {  // Kt chunks (and with POST the convolved values), through the ring
+    if (warp == kTmaWarp && lane == 0) {  // Kt chunks (and with POST the convolved values), through the ring
       prefetch_tmap(&tmK);
       if (POST) prefetch_tmap(&tmVt);
       int cnt = 0;
-      auto push = [&](const CUtensorMap *map, int x, int y, int z) -> bool {
+      // one ring stage: SB boxes, box bx at (x[bx], y, z[bx])
+      auto push = [&](const CUtensorMap *map, const int (&x)[G::SB], int y, const int (&z)[G::SB]) -> bool {
         const int st = cnt % G::NS;
         if (!mbar_wait(k_empty + st, ((cnt / G::NS) & 1) ^ 1, abort_flag, p.err)) return false;
-        mbar_arrive_expect_tx(k_full + st, G::KCHUNK);
-        tma_load_3d(Ks + st * G::KCHUNK, map, k_full + st, x, y, z);
+        mbar_arrive_expect_tx(k_full + st, G::KSTAGE);
+#pragma unroll
+        for (int bx = 0; bx < G::SB; ++bx)
+          tma_load_3d(Ks + st * G::KSTAGE + bx * G::KCHUNK, map, k_full + st, x[bx], y, z[bx]);
         ++cnt;
         return true;
       };
@@ -283,17 +294,29 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int r = 0; ok && item_at(r, it) && !*abort_flag; ++r) {
         const int h = it.g * CL + hr, n_kv = kv_tiles(it), nsl = n_slots(it);
         auto load_c = [&](int t) -> bool {
-          for (int ch = 0; ch < G::NSRC * G::NCH; ++ch) {
-            const int sc = ch / G::NCH, cs = ch % G::NCH;
-            if (!push(&tmK, 0, t * G::BN, (it.b * p.H + src_head(h, sc)) * G::NCH + cs)) return false;
+          for (int ch = 0; ch < G::NSRC * G::NCH; ch += G::SB) {
+            const int sc = ch / G::NCH, zh = it.b * p.H + src_head(h, sc);
+            int x[G::SB], z[G::SB];
+#pragma unroll
+            for (int bx = 0; bx < G::SB; ++bx) {
+              const int cs = ch % G::NCH + bx;
+              x[bx] = D % 64 == 0 ? (cs % G::NDC) * 64 : 0;
+              z[bx] = D % 64 == 0 ? zh * CQ + cs / G::NDC : zh * G::NCH + cs;
+            }
+            if (!push(&tmK, x, t * G::BN, z)) return false;
           }
           return true;
         };
         auto load_pv = [&](int t) -> bool {  // chunk (value head hd, tap row a, 64-channel block dc)
-          for (int ch = 0; ch < G::NVCH; ++ch) {
-            const int hd = ch / (CQ * G::NDC), a = (ch / G::NDC) % CQ, dc = ch % G::NDC;
-            const int z = ((it.b * p.H + h) * G::NV + hd) * CQ + a;
-            if (!push(&tmVt, dc * 64, t * G::BN, z)) return false;
+          for (int ch = 0; ch < G::NVCH; ch += G::SB) {
+            int x[G::SB], z[G::SB];
+#pragma unroll
+            for (int bx = 0; bx < G::SB; ++bx) {
+              const int c2 = ch + bx, hd = c2 / (CQ * G::NDC), a = (c2 / G::NDC) % CQ, dc = c2 % G::NDC;
+              x[bx] = dc * 64;
+              z[bx] = ((it.b * p.H + h) * G::NV + hd) * CQ + a;
+            }
+            if (!push(&tmVt, x, t * G::BN, z)) return false;
           }
           return true;
         };
@@ -307,7 +330,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (*abort_flag)  // copies still in flight land before the CTA exits
         for (int c2 = (cnt > G::NS ? cnt - G::NS : 0); c2 < cnt; ++c2)
           drain_wait(k_full + c2 % G::NS, (c2 / G::NS) & 1);
-    } else if (lane == 1 && !POST) {  // V of both heads of the group, per key tile
+    } else if (warp == kTma2Warp && lane == 0 && !POST) {  // V of both heads of the group, per key tile
       prefetch_tmap(&tmV);
       int nv = 0;
       Item it;
@@ -325,7 +348,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
       if (*abort_flag && nv) drain_wait(v_full, (nv - 1) & 1);
-    } else if (lane == 2) {  // the query rows of each item, once the previous item's C is done
+    } else if (warp == kTma2Warp && lane == 1) {  // the query rows of each item, once the previous item's C is done
       prefetch_tmap(&tmQ);
       int nq = 0;
       Item it;
@@ -363,25 +386,43 @@ __global__ void __launch_bounds__(kThreads, 1)
       // contraction; element kappa = a*D + e pairs Q shifted by a rows with Kt_a
       auto issue_c = [&](bool last_of_item) -> bool {
         if (T > 0 && !mbar_wait(c_free, (T - 1) & 1, abort_flag, p.err)) return false;
-        for (int ch = 0; ch < G::NSRC * G::NCH; ++ch, ++cnt) {
+        for (int ch = 0; ch < G::NSRC * G::NCH; ch += G::SB, ++cnt) {
           const int st = cnt % G::NS;
           // source head sc (its own accumulator and query rows); the 16 elements
           // kappa = 64 cs + 16 kk of step kk: tap row a, channels e0 .. e0+15 (D is a
           // multiple of 16, so a step never straddles two tap rows); Q rows shifted up
           // by a (16 bytes per row), 8-channel strips e0/8 and e0/8 + 1
-          const int sc = ch / G::NCH, cs = ch % G::NCH;
-          uint64_t qd[4];
+          if constexpr (D % 64 == 0) {
+            if (!mbar_wait(k_full + st, (cnt / G::NS) & 1, abort_flag, p.err)) return false;
+            tc_fence_after();
+            // box bx of the stage is chunk cs: tap row a = cs / NDC, channels 64 dc ..
+            // 64 dc + 63 (a stage is a whole tap row when SB = NDC)
+            const int sc = ch / G::NCH;
+            const uint64_t kd = kdesc0 + static_cast<uint32_t>((st * G::KSTAGE) >> 4);
 #pragma unroll
-          for (int kk = 0; kk < 4; ++kk) {
-            const int kap = 64 * cs + 16 * kk, a = kap / D, e0 = kap % D;
-            qd[kk] = qdesc0 + static_cast<uint32_t>((sc * G::Q_ALLOC + (e0 / 8) * G::STRIP + 16 * (G::HALO - a)) >> 4);
+            for (int bx = 0; bx < G::SB; ++bx) {
+              const int cs = ch % G::NCH + bx, a = cs / G::NDC, dc = cs % G::NDC;
+              const uint64_t qd = qdesc0 + static_cast<uint32_t>((sc * G::Q_ALLOC + 8 * dc * G::STRIP + 16 * (G::HALO - a)) >> 4);
+#pragma unroll
+              for (int kk = 0; kk < 4; ++kk)
+                mma_bf16_ss(tmem + G::C_COL + 128 * sc, qd + (2 * kk * G::STRIP >> 4),
+                            kd + (bx * G::KCHUNK >> 4) + 2 * kk, idesc_c, (cs > 0 || kk > 0));
+            }
+          } else {
+            const int sc = ch / G::NCH, cs = ch % G::NCH;
+            const uint64_t kd = kdesc0 + static_cast<uint32_t>((st * G::KSTAGE) >> 4);
+            uint64_t qd[4];
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk) {
+              const int kap = 64 * cs + 16 * kk, a = kap / D, e0 = kap % D;
+              qd[kk] = qdesc0 + static_cast<uint32_t>((sc * G::Q_ALLOC + (e0 / 8) * G::STRIP + 16 * (G::HALO - a)) >> 4);
+            }
+            if (!mbar_wait(k_full + st, (cnt / G::NS) & 1, abort_flag, p.err)) return false;
+            tc_fence_after();
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk)
+              mma_bf16_ss(tmem + G::C_COL + 128 * sc, qd[kk], kd + 2 * kk, idesc_c, (cs > 0 || kk > 0));
           }
-          const uint64_t kd = kdesc0 + static_cast<uint32_t>((st * G::KCHUNK) >> 4);
-          if (!mbar_wait(k_full + st, (cnt / G::NS) & 1, abort_flag, p.err)) return false;
-          tc_fence_after();
-#pragma unroll
-          for (int kk = 0; kk < 4; ++kk)
-            mma_bf16_ss(tmem + G::C_COL + 128 * sc, qd[kk], kd + 2 * kk, idesc_c, (cs > 0 || kk > 0));
           mma_commit(k_empty + st);
         }
         mma_commit(c_full);
@@ -390,18 +431,33 @@ __global__ void __launch_bounds__(kThreads, 1)
       };
       // Z_hd += sum_a (weights shifted down by a rows) x Vt_{hd,a}, from the ring
       auto issue_pv = [&](bool first_of_item) -> bool {
-        for (int ch = 0; ch < G::NVCH; ++ch, ++cnt) {
+        for (int ch = 0; ch < G::NVCH; ch += G::SB, ++cnt) {
           const int st = cnt % G::NS;
           if (!mbar_wait(k_full + st, (cnt / G::NS) & 1, abort_flag, p.err)) return false;
           tc_fence_after();
-          const int hd = ch / (CQ * G::NDC), a = (ch / G::NDC) % CQ, dc = ch % G::NDC;
-          const uint64_t pd = psdesc0 + static_cast<uint32_t>(G::PS_PAD - a);
-          const uint64_t vd = vtdesc0 + static_cast<uint32_t>((st * G::KCHUNK) >> 4);
+          if constexpr (G::SB == 2) {
+            // the stage holds both 64-channel boxes of (hd, a): one N = 128 MMA per key step
+            const int hd = ch / (CQ * G::NDC), a = (ch / G::NDC) % CQ;
+            const uint64_t pd = psdesc0 + static_cast<uint32_t>(G::PS_PAD - a);
+            const uint64_t vd = vtdesc0 + static_cast<uint32_t>((st * G::KSTAGE) >> 4);
 #pragma unroll
-          for (int kk = 0; kk < G::BN / 16; ++kk)
-            mma_bf16_ss(tmem + G::Z_COL0 + 128 * hd + 64 * dc, pd + static_cast<uint32_t>((2 * kk * G::PS_STRIP) >> 4),
-                        vd + static_cast<uint32_t>((kk * 16 * 128) >> 4), idesc_pv64,
-                        !(first_of_item && a == 0 && kk == 0));
+            for (int kk = 0; kk < G::BN / 16; ++kk)
+              mma_bf16_ss(tmem + G::Z_COL0 + 128 * hd, pd + static_cast<uint32_t>((2 * kk * G::PS_STRIP) >> 4),
+                          vd + static_cast<uint32_t>((kk * 16 * 128) >> 4), idesc_bf16_f32(128, 128, 0, 1),
+                          !(first_of_item && a == 0 && kk == 0));
+          } else {
+#pragma unroll
+            for (int bx = 0; bx < G::SB; ++bx) {
+              const int c2 = ch + bx, hd = c2 / (CQ * G::NDC), a = (c2 / G::NDC) % CQ, dc = c2 % G::NDC;
+              const uint64_t pd = psdesc0 + static_cast<uint32_t>(G::PS_PAD - a);
+              const uint64_t vd = vtdesc0 + static_cast<uint32_t>((st * G::KSTAGE + bx * G::KCHUNK) >> 4);
+#pragma unroll
+              for (int kk = 0; kk < G::BN / 16; ++kk)
+                mma_bf16_ss(tmem + G::Z_COL0 + 128 * hd + 64 * dc, pd + static_cast<uint32_t>((2 * kk * G::PS_STRIP) >> 4),
+                            vd + static_cast<uint32_t>((kk * 16 * 128) >> 4), idesc_pv64,
+                            !(first_of_item && a == 0 && kk == 0));
+            }
+          }
           mma_commit(k_empty + st);
         }
         mma_commit(v_empty);
@@ -434,12 +490,21 @@ __global__ void __launch_bounds__(kThreads, 1)
             // item's epilogue must have read it
             if (t == 0 && r > 0 && !mbar_wait(z_free, (r - 1) & 1, abort_flag, p.err)) { ok = false; break; }
             tc_fence_after();
-#pragma unroll
-            for (int hd = 0; hd < G::NV; ++hd)
+            if constexpr (G::NV * G::NDC * 64 == 256) {
+              // both heads' V tiles are four consecutive 64-channel boxes and both Z
+              // accumulators 256 consecutive columns: one N = 256 MMA per key step
 #pragma unroll
               for (int kk = 0; kk < G::BN / 16; ++kk)
-                mma_f16_ts(tmem + G::Z_COL0 + 128 * hd, tmem + G::P_COL + 8 * kk,
-                           vdesc0 + ((hd * G::V_HEAD + kk * 16 * 128) >> 4), idesc_pv, (t > 0 || kk > 0));
+                mma_f16_ts(tmem + G::Z_COL0, tmem + G::P_COL + 8 * kk, vdesc0 + ((kk * 16 * 128) >> 4),
+                           idesc_bf16_f32(128, 256, 0, 1), (t > 0 || kk > 0));
+            } else {
+#pragma unroll
+              for (int hd = 0; hd < G::NV; ++hd)
+#pragma unroll
+                for (int kk = 0; kk < G::BN / 16; ++kk)
+                  mma_f16_ts(tmem + G::Z_COL0 + 128 * hd, tmem + G::P_COL + 8 * kk,
+                             vdesc0 + ((hd * G::V_HEAD + kk * 16 * 128) >> 4), idesc_pv, (t > 0 || kk > 0));
+            }
             mma_commit(v_empty);
           }
         }
@@ -455,7 +520,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int st_id = threadIdx.x;           // 0..255
     const int cb = G::HALF * wg;             // key columns of this warpgroup
     const int zc = G::DH * wg;               // output channels of this warpgroup: zc .. zc+zn-1
-    const int zn = wg ? G::DH1 : G::DH;
+    const int zn = G::DH1 == G::DH ? G::DH : (wg ? G::DH1 : G::DH);  // a constant unless d = 96
     const uint32_t tl = tmem + (static_cast<uint32_t>(32 * q4) << 16);
     const float sc0 = p.qk_scale * kLog2e;
     float *crow = Cs + (wg * G::BM + r_) * G::W;
@@ -929,10 +994,14 @@ cudaError_t launch_kq_one(const AttnArgs &a, const GnArgs *gn, const KqPrepArgs 
   const unsigned boxq[4] = {8, 1, G::QROWS, 1}, boxv[4] = {64, 1, G::BN, 1};
   if (!encode_tmap_bf16(&tq, a.q, 4, dims, str, boxq, false)) return cudaErrorInvalidValue;
   if (!encode_tmap_bf16(&tv, a.v, 4, dims, str, boxv, true)) return cudaErrorInvalidValue;
-  // Kt: [B*H*NCH][L][64] 16-bit elements (the copy moves bytes; fp16 as 16-bit)
-  const unsigned long long kdims[3] = {64, static_cast<unsigned long long>(a.L),
-                                       static_cast<unsigned long long>(a.B) * a.H * G::NCH};
-  const unsigned long long kstr[2] = {128, static_cast<unsigned long long>(a.L) * 128};
+  // Kt (16-bit elements; the copy moves bytes, fp16 as 16-bit): [B*H*CQ][L][D] when D is
+  // a multiple of 64, else [B*H*NCH][L][64]
+  const bool krows = D % 64 == 0;
+  const unsigned long long kdims[3] = {krows ? static_cast<unsigned long long>(D) : 64ull,
+                                       static_cast<unsigned long long>(a.L),
+                                       static_cast<unsigned long long>(a.B) * a.H * (krows ? CQ : G::NCH)};
+  const unsigned long long kstr[2] = {krows ? static_cast<unsigned long long>(D) * 2 : 128ull,
+                                      static_cast<unsigned long long>(a.L) * (krows ? D * 2 : 128)};
   const unsigned boxk[3] = {64, G::BN, 1};
   if (!encode_tmap_bf16(&tk, pa.kt, 3, kdims, kstr, boxk, true)) return cudaErrorInvalidValue;
   tvt = tk;

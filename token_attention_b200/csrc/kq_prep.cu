@@ -134,6 +134,11 @@ __global__ void __launch_bounds__(kPrepThreads, 3) kq_prep_kernel(KqPrepArgs p) 
   __half *kt = static_cast<__half *>(p.kt);
   constexpr int NCHK = CQ * D / 64;  // 64-element chunks of a key's contraction operand
   constexpr int NPAIR = D / 2, NRUN = kTile / kRun;
+  // d a multiple of 64: rows [c_q][L][d] (a 64-element chunk = 64 channels of one tap
+  // row); else chunk-major [c_q*d/64][L][64]
+  constexpr bool ROWS = D % 64 == 0;
+  constexpr int KSTEP = ROWS ? D : 64;  // elements between consecutive keys
+  const long long LD = static_cast<long long>(L) * D;  // elements between the Kt_a of one head (rows)
   for (int item = tid; item < NPAIR * NRUN; item += kPrepThreads) {
     const int e2 = (item % NPAIR) * 2, jr = (item / NPAIR) * kRun;
     if (j0 + jr >= L) continue;
@@ -145,7 +150,7 @@ __global__ void __launch_bounds__(kPrepThreads, 3) kq_prep_kernel(KqPrepArgs p) 
     float scu[kRun];
 #pragma unroll
     for (int u = 0; u < kRun; ++u) scu[u] = pow2i(es[jr + u]);
-    __half *o0 = kt + (bh * NCHK * L + j0 + jr) * 64;  // chunk 0, key j0+jr
+    __half *o0 = ROWS ? kt + (bh * CQ * L + j0 + jr) * D + e2 : kt + (bh * NCHK * L + j0 + jr) * 64;
 #pragma unroll
     for (int a = 0; a < CQ; ++a) {
       // kRun x 2 independent accumulators; taps in the outer loop (no dependent chains)
@@ -161,12 +166,17 @@ __global__ void __launch_bounds__(kPrepThreads, 3) kq_prep_kernel(KqPrepArgs p) 
           acc[u].y = fmaf(ta, win[u + 2 * G::C - t].y, acc[u].y);
         }
       }
-      const int kap = a * D + e2;  // contraction element of channel pair e2 in tap row a
-      __half *oa = o0 + static_cast<long long>(kap / 64) * L * 64 + kap % 64;
+      __half *oa;
+      if constexpr (ROWS) {
+        oa = o0 + a * LD;
+      } else {
+        const int kap = a * D + e2;  // contraction element of channel pair e2 in tap row a
+        oa = o0 + static_cast<long long>(kap / 64) * L * 64 + kap % 64;
+      }
 #pragma unroll
       for (int u = 0; u < kRun; ++u)
         if (nkeys == kRun || u < nkeys)
-          *reinterpret_cast<__half2 *>(oa + u * 64) = __floats2half2_rn(acc[u].x * scu[u], acc[u].y * scu[u]);
+          *reinterpret_cast<__half2 *>(oa + u * KSTEP) = __floats2half2_rn(acc[u].x * scu[u], acc[u].y * scu[u]);
     }
   }
 
