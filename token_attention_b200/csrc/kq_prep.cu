@@ -74,6 +74,17 @@ __device__ __forceinline__ float2 bf16x2_to_float2(uint32_t v) {
 
 __device__ __forceinline__ float pow2i(int e) { return __int_as_float((127 + e) << 23); }  // |e| <= 126
 
+// c + a * b on a pair of floats with one packed instruction (each lane rounds as fmaf)
+__device__ __forceinline__ float2 fma2(float2 a, float2 b, float2 c) {
+  float2 r;
+  asm("{\n\t.reg .b64 pa, pb, pc, pd;\n\t"
+      "mov.b64 pa, {%2, %3};\n\tmov.b64 pb, {%4, %5};\n\tmov.b64 pc, {%6, %7};\n\t"
+      "fma.rn.f32x2 pd, pa, pb, pc;\n\tmov.b64 {%0, %1}, pd;\n\t}"
+      : "=f"(r.x), "=f"(r.y)
+      : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y), "f"(c.x), "f"(c.y));
+  return r;
+}
+
 template <int D, int CQ, int CK, bool EXACT>
 __global__ void __launch_bounds__(kPrepThreads, 3) kq_prep_kernel(KqPrepArgs p) {
   using G = PrepGeo<D, CQ, CK, EXACT>;
@@ -159,12 +170,10 @@ __global__ void __launch_bounds__(kPrepThreads, 3) kq_prep_kernel(KqPrepArgs p) 
       for (int u = 0; u < kRun; ++u) acc[u] = make_float2(0.f, 0.f);
 #pragma unroll
       for (int t = 0; t < CK; ++t) {
-        const float ta = th[a * CK + t];
+        const float2 ta = make_float2(th[a * CK + t], th[a * CK + t]);
 #pragma unroll
-        for (int u = 0; u < kRun; ++u) {  // key j - (t - c) is window entry u + 2c - t
-          acc[u].x = fmaf(ta, win[u + 2 * G::C - t].x, acc[u].x);
-          acc[u].y = fmaf(ta, win[u + 2 * G::C - t].y, acc[u].y);
-        }
+        for (int u = 0; u < kRun; ++u)  // key j - (t - c) is window entry u + 2c - t
+          acc[u] = fma2(ta, win[u + 2 * G::C - t], acc[u]);
       }
       __half *oa;
       if constexpr (ROWS) {
@@ -283,12 +292,10 @@ __global__ void __launch_bounds__(kPrepThreads, 3) vt_prep_kernel(VtPrepArgs p) 
         for (int u = 0; u < kRun; ++u) acc[u] = make_float2(0.f, 0.f);
 #pragma unroll
         for (int t = 0; t < CK; ++t) {
-          const float ta = th[a * CK + t];
+          const float2 ta = make_float2(th[a * CK + t], th[a * CK + t]);
 #pragma unroll
-          for (int u = 0; u < kRun; ++u) {  // value j + (t - c) is window entry u + t
-            acc[u].x = fmaf(ta, win[u + t].x, acc[u].x);
-            acc[u].y = fmaf(ta, win[u + t].y, acc[u].y);
-          }
+          for (int u = 0; u < kRun; ++u)  // value j + (t - c) is window entry u + t
+            acc[u] = fma2(ta, win[u + t], acc[u]);
         }
         __nv_bfloat16 *oa = vt + ((z0 + a) * L + j0 + jr) * D + e2;
 #pragma unroll
