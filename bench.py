@@ -285,9 +285,13 @@ def run_mine(args, wl, rank, world, local_rank):
     odt = torch.float32 if wl.dtype == "f32" else torch.bfloat16
     if args.bwd:  # fp32 gradients of q, k, v, the kernels and the mixing weights
         z = lambda *shape: torch.empty(shape, dtype=torch.float32, device=dev)
-        outs = [{"dq": z(*out_shape), "dk": z(*out_shape), "dv": z(*out_shape),
-                 "dtheta": z(wl.H, wl.c_q, wl.c_k) if wl.kq_place else None,
-                 "dw": z(wl.H // wl.c_h, wl.c_h, wl.c_h) if wl.head_place else None} for _ in range(N_SETS)]
+        n_th = (1 if wl.kq_place else 0) + (1 if wl.kq_post else 0)
+        outs = []
+        for _ in range(N_SETS):
+            dth = z(n_th, wl.H, wl.c_q, wl.c_k) if n_th else None
+            outs.append({"dq": z(*out_shape), "dk": z(*out_shape), "dv": z(*out_shape), "dtheta_all": dth,
+                         "dtheta": None, "dtheta_post": None,
+                         "dw": z(wl.H // wl.c_h, wl.c_h, wl.c_h) if wl.head_place else None})
     else:
         outs = [torch.empty(out_shape, dtype=odt, device=dev) for _ in range(N_SETS)]
     cfg = mta.make_cfg(wl.B, wl.H, wl.L, wl.d, wl.c_q, wl.c_k, wl.c_h, wl.kq_place, wl.head_place,
@@ -446,7 +450,8 @@ def oracle_sample(wl, budget_s: float, mode: str):
             hs = slice(g * ch, (g + 1) * ch)
             grp = lambda x: np.ascontiguousarray(x[b, :, hs].transpose(1, 0, 2))
             O.mta_attention_group_bwd(grp(q), grp(k), grp(v), th[hs], w[g], np.arange(wl.L),
-                                      1 / math.sqrt(wl.d), wl.kq_place, wl.head_place, grp(dout))
+                                      1 / math.sqrt(wl.d), wl.kq_place, wl.head_place, grp(dout),
+                                      None if tp is None else tp[hs])
             done += 1
             if time.perf_counter() - t0 > budget_s:
                 break
@@ -579,14 +584,15 @@ def main():
         # the backward on the CUDA cores: F_bwd = 8d + 4 c_q c_k + 4 c_h fp32 flop per causal
         # pair-head (dS, dQ, dK, dV products; the convolution's adjoint and kernel gradient;
         # the mixing adjoints)
-        kernel = "attn_bwd_simt_kernel"
-        f_bwd = (8 * wl.d + (4 * wl.c_q * wl.c_k if wl.kq_place else 0) + (4 * wl.c_h if wl.head_place else 0)) \
+        kernel = "attn_bwd_post_kernel" if wl.kq_post else "attn_bwd_simt_kernel"
+        n_conv = (1 if wl.kq_place else 0) + (1 if wl.kq_post else 0)
+        f_bwd = (8 * wl.d + 4 * wl.c_q * wl.c_k * n_conv + (4 * wl.c_h if wl.head_place else 0)) \
             * wl.causal_pairs
         achieved = f_bwd / s / 1e12
         roof = {"bound": "alu", "achieved": achieved, "peak": FP32_PEAK_TFLOPS, "unit": "TFLOP/s",
                 "frac": achieved / FP32_PEAK_TFLOPS, "traffic": read_traffic(kernel, wl.name),
                 "kernel": kernel,
-                "per_unit": f"F_bwd = 8d + 4 c_q c_k + 4 c_h = {f_bwd // wl.causal_pairs} fp32 flop per "
+                "per_unit": f"F_bwd = 8d + 4 c_q c_k (per convolution) + 4 c_h = {f_bwd // wl.causal_pairs} fp32 flop per "
                             f"causal pair-head, x {wl.causal_pairs} pair-heads per launch",
                 "peak_source": "148 SMs x 128 FP32 lanes x 2 x 1965 MHz"}
     elif wl.layer:

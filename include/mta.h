@@ -85,7 +85,10 @@ typedef struct mta_cfg {
                             after the softmax; section 4 uses both), then Mask_0
                             zeroes the future keys again: A' = Mask_0(Conv2d(A)),
                             not renormalised, before any post-softmax head mix;
-                            0: none                                              */
+                            its kernels follow the pre-softmax ones in theta_kq.
+                            Served by the contraction kernel (bf16, c_q x c_k =
+                            6 x 11, a pre-softmax convolution on) and by the
+                            CUDA-core kernel; 0: none                            */
   int dtype;             /* mta_dtype of q, k, v and out (x, W and out in a layer) */
   int path;              /* attention kernel: 0 = choose (the contraction kernel
                             where it applies and the workspace holds its operands,
@@ -121,8 +124,10 @@ typedef struct mta_gn {
 /* Bytes of workspace mta_attn_fwd needs for cfg (0 if cfg is invalid): 256
  * bytes, plus, where the contraction kernel applies, its per-call operands
  * (the convolved keys, c_q*B*H*L*d fp16, their B*H*L fp32 scales,
- * B*H*L*(c_q-1+2*(c_k/2)) fp32 dot products and, with post-softmax mixing, an
- * exchange buffer of at most 160*2*d*128 fp32 for the kernel's persistent CTAs).
+ * B*H*L*(c_q-1+2*(c_k/2)) fp32 dot products, with post-softmax mixing an
+ * exchange buffer of at most 160*2*d*128 fp32 for the kernel's persistent CTAs,
+ * and with kq_post the values convolved by the post-softmax kernels,
+ * n_v*c_q*B*H*L*d bf16, n_v = 2 with post-softmax mixing, else 1).
  * With a smaller workspace path 0 uses another kernel. */
 size_t mta_attn_workspace_bytes(const mta_cfg *cfg);
 
@@ -200,17 +205,19 @@ mta_status mta_group_norm_scale(const void *o, const mta_gn *gn, int tokens, int
  * and of the head-mixing weights, each forward step taken in reverse order (see
  * attn_bwd_simt.cu for the chain of adjoints):
  *   q, k, v      : as for mta_attn_fwd (cfg->dtype, token stride cfg->qkv_row_stride)
- *   theta_kq     : [H][c_q][c_k] fp32 (ignored when kq_place == MTA_OFF)
+ *   theta_kq     : [n][H][c_q][c_k] fp32 as for mta_attn_fwd (the pre-softmax
+ *                  kernels when kq_place is on, then the post-softmax ones when
+ *                  kq_post = 1)
  *   w_head       : [H/c_h][c_h][c_h] fp32 (ignored when head_place == MTA_OFF)
  *   dout         : [B][L][H][d] dense, cfg->dtype
  *   dq, dk, dv   : [B][L][H][d] dense fp32, overwritten
- *   dtheta       : [H][c_q][c_k] fp32, overwritten (may be NULL; ignored when
- *                  kq_place == MTA_OFF)
+ *   dtheta       : [n][H][c_q][c_k] fp32, laid out as theta_kq, overwritten (may be
+ *                  NULL; n = 0 leaves it unused)
  *   dw           : [H/c_h][c_h][c_h] fp32, overwritten (may be NULL; ignored when
  *                  head_place == MTA_OFF)
- * Runs on the CUDA cores in fp32 arithmetic for every forward configuration except
- * the post-softmax convolution (cfg->kq_post = 1: MTA_ERR_UNSUPPORTED).  cfg->path
- * must be 0 or 1.  dk, dv, dtheta and dw are summed with atomic additions, so their
+ * Runs on the CUDA cores in fp32 arithmetic for every forward configuration
+ * (attn_bwd_simt.cu; attn_bwd_post_simt.cu with the post-softmax convolution).
+ * cfg->path must be 0 or 1.  dk, dv, dtheta and dw are summed with atomic additions, so their
  * last bits may differ between runs.  The workspace holds the error word only
  * (mta_attn_bwd_workspace_bytes).  No L x L map is stored. */
 size_t mta_attn_bwd_workspace_bytes(const mta_cfg *cfg);

@@ -533,13 +533,14 @@ def test_d96_layer_small(hp):
 # backward pass (mta_attn_bwd): every gradient against the fp64 oracle
 # ---------------------------------------------------------------------------
 
-GRAD_NAMES = ("dq", "dk", "dv", "dtheta", "dw")
+GRAD_NAMES = ("dq", "dk", "dv", "dtheta", "dw", "dtheta_post")
 
 
 def run_bwd(wl, inp, dout):
     q, k, v = (dev(inp[n], wl.dtype) for n in ("q", "k", "v"))
+    tp = None if inp.get("theta_post") is None else dev(inp["theta_post"], "f32")
     g = mta.attn_bwd(q, k, v, dev(inp["theta"], "f32"), dev(inp["w"], "f32"), dev(dout, wl.dtype),
-                     wl.c_q, wl.c_k, wl.c_h, wl.kq_place, wl.head_place, check=True)
+                     wl.c_q, wl.c_k, wl.c_h, wl.kq_place, wl.head_place, check=True, theta_post=tp)
     torch.cuda.synchronize()
     return g
 
@@ -547,7 +548,7 @@ def run_bwd(wl, inp, dout):
 def check_grads(wl, inp, dout, tol=TOL_F32):
     got = run_bwd(wl, inp, dout)
     ref = O.mta_attention_bwd(inp["q"], inp["k"], inp["v"], inp["theta"], inp["w"], wl.c_h, dout,
-                              wl.kq_place, wl.head_place)
+                              wl.kq_place, wl.head_place, theta_post=inp.get("theta_post"))
     for n in GRAD_NAMES:
         if ref[n] is None:
             assert got[n] is None
@@ -591,31 +592,37 @@ def test_bwd_pretrain_recipe_L512():
     check_grads(wl, inp, dout)
 
 
-def test_bwd_rejects_post_softmax_convolution():
-    wl = synth.shrink(synth.WORKLOADS["both_d128_L2048"], B=1, H=2, L=16, d=32)
-    inp = synth.make_attn_inputs(wl)
-    q, k, v = (dev(inp[n]) for n in "qkv")
-    cfg = mta.make_cfg(1, 2, 16, 32, 6, 11, 2, synth.PRE, synth.POST, mta.BF16, kq_post=1)
-    ws = mta.workspace(256)
-    cfg.workspace, cfg.workspace_bytes = ws.data_ptr(), ws.numel()
-    z = torch.zeros((1, 16, 2, 32), dtype=torch.float32, device="cuda")
-    th = dev(np.concatenate([inp["theta"], inp["theta_post"]]), "f32")
-    code = mta.lib().mta_attn_bwd(mta._ptr(q), mta._ptr(k), mta._ptr(v), mta._ptr(th),
-                                  mta._ptr(dev(inp["w"], "f32")), mta._ptr(q), ctypes.byref(cfg),
-                                  mta._ptr(z), mta._ptr(z), mta._ptr(z), None, None)
-    assert code == 2
+BWD_POST = [("f32", synth.PRE, synth.POST, 9), ("f32", synth.PRE, synth.PRE, 40),
+            ("bf16", synth.PRE, synth.POST, 70), ("bf16", synth.OFF, synth.POST, 50),
+            ("bf16", mta.PRE_EXACT, synth.OFF, 45), ("bf16", synth.PRE, synth.OFF, 33)]
 
 
-def test_post_conv_stacked_kernel_array():
-    """Passing the pre- and post-softmax kernels as one stacked array (what the
-    library reads) gives the same bits as passing them separately."""
+@pytest.mark.parametrize("dtype,kq,hp,L", BWD_POST)
+def test_bwd_post_conv_small(dtype, kq, hp, L):
+    """The backward with the key-query convolution also after the softmax: every
+    gradient, the post-softmax kernels' included."""
     base = synth.WORKLOADS["both_d128_L2048"]
-    wl = synth.shrink(base, B=1, H=4, L=140, seed=461)
+    wl = synth.shrink(base, B=2, H=4, L=L, d=32, kq_place=kq, head_place=hp, dtype=dtype,
+                      seed=861 + L + kq + 3 * hp)
     inp = synth.make_attn_inputs(wl)
-    a = run_attn(wl, inp)
-    q, k, v = (dev(inp[n]) for n in "qkv")
-    stacked = mta.kq_kernels(dev(inp["theta"], "f32"), dev(inp["theta_post"], "f32"))
-    b = mta.attn_fwd(q, k, v, stacked, dev(inp["w"], "f32"), wl.c_q, wl.c_k, wl.c_h, wl.kq_place,
-                     wl.head_place, check=True)
-    torch.cuda.synchronize()
-    assert torch.equal(a, b)
+    dout = synth.normal(wl.seed, 20, (wl.B, wl.L, wl.H, wl.d))
+    if dtype == "bf16":
+        dout = synth.round_bf16(dout)
+    check_grads(wl, inp, dout)
+
+
+def test_bwd_post_conv_recipe_L300():
+    wl = synth.shrink(synth.WORKLOADS["both_d128_L2048"], B=1, H=2, L=300, seed=862)
+    inp = synth.make_attn_inputs(wl)
+    dout = synth.round_bf16(synth.normal(wl.seed, 20, (wl.B, wl.L, wl.H, wl.d)))
+    check_grads(wl, inp, dout)
+
+
+def test_bwd_full_length_one_group():
+    """The pretraining recipe at its full length L = 2048 (the length the bench's
+    backward line runs) for one batch and one head group, against the fp64
+    oracle's full L x L backward of that group."""
+    wl = synth.shrink(synth.WORKLOADS["pretrain_d128_L2048"], B=1, H=2, seed=852)
+    inp = synth.make_attn_inputs(wl)
+    dout = synth.round_bf16(synth.normal(wl.seed, 20, (wl.B, wl.L, wl.H, wl.d)))
+    check_grads(wl, inp, dout)

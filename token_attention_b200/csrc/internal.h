@@ -46,12 +46,18 @@ struct BwdArgs {
   float *dq, *dk, *dv;    // [B][L][H][d] dense fp32
   float *dtheta;          // [H][c_q][c_k] or null
   float *dw;              // [H/c_h][c_h][c_h] or null
+  const float *theta_post;  // [H][c_q][c_k] post-softmax kernels (kq_post)
+  float *dtheta_post;       // their gradient (kq_post) or null
   int B, H, L, d, cq, ck, ch, kq, hp, dtype;
+  int kqp;                // 1: the convolution also acts after the softmax
   float scale;
   cudaStream_t stream;
 };
 int attn_bwd_simt_pick_rows(const BwdArgs &a);  // 0 if nothing fits
 cudaError_t launch_attn_bwd_simt(const BwdArgs &a);
+// With the post-softmax convolution (kqp == 1).
+int attn_bwd_post_pick_rows(const BwdArgs &a);
+cudaError_t launch_attn_bwd_post(const BwdArgs &a);
 
 // tcgen05 kernel (bf16, fused); attn_tc_supported() says whether it applies.
 bool attn_tc_supported(const AttnArgs &a);

@@ -295,7 +295,7 @@ mta_status mta_attn_bwd(const void *q, const void *k, const void *v, const float
                         float *dk, float *dv, float *dtheta, float *dw) {
   mta_status s = check_cfg(cfg);
   if (s != MTA_OK) return s;
-  if (cfg->kq_post || cfg->path > 1) return MTA_ERR_UNSUPPORTED;
+  if (cfg->path > 1) return MTA_ERR_UNSUPPORTED;
   if ((s = check_attn_pointers(q, k, v, theta_kq, w_head, cfg, dout)) != MTA_OK) return s;
   if (!dq || !dk || !dv || !aligned(dq, 4) || !aligned(dk, 4) || !aligned(dv, 4)) return MTA_ERR_INVALID;
   if ((dtheta && !aligned(dtheta, 4)) || (dw && !aligned(dw, 4))) return MTA_ERR_INVALID;
@@ -305,16 +305,21 @@ mta_status mta_attn_bwd(const void *q, const void *k, const void *v, const float
   a.rs = cfg->qkv_row_stride ? cfg->qkv_row_stride : static_cast<long long>(cfg->H) * cfg->d;
   a.theta = theta_kq; a.w = w_head;
   a.dq = dq; a.dk = dk; a.dv = dv;
+  // theta_kq (and dtheta) hold the pre-softmax kernels when on, then the post-softmax ones
+  const size_t nth = static_cast<size_t>(cfg->H) * cfg->c_q * cfg->c_k;
   a.dtheta = cfg->kq_place != MTA_OFF ? dtheta : nullptr;
+  a.kqp = cfg->kq_post;
+  a.theta_post = cfg->kq_post ? theta_kq + (cfg->kq_place != MTA_OFF ? nth : 0) : nullptr;
+  a.dtheta_post = (cfg->kq_post && dtheta) ? dtheta + (cfg->kq_place != MTA_OFF ? nth : 0) : nullptr;
   a.dw = cfg->head_place != MTA_OFF ? dw : nullptr;
   a.B = cfg->B; a.H = cfg->H; a.L = cfg->L; a.d = cfg->d;
   a.cq = cfg->c_q; a.ck = cfg->c_k; a.ch = cfg->c_h;
   a.kq = cfg->kq_place; a.hp = cfg->head_place; a.dtype = cfg->dtype;
   a.scale = cfg->scale > 0.f ? cfg->scale : 1.0f / sqrtf(static_cast<float>(cfg->d));
   a.stream = static_cast<cudaStream_t>(cfg->stream);
-  if (attn_bwd_simt_pick_rows(a) == 0) return MTA_ERR_UNSUPPORTED;
+  if ((a.kqp ? attn_bwd_post_pick_rows(a) : attn_bwd_simt_pick_rows(a)) == 0) return MTA_ERR_UNSUPPORTED;
   if ((s = clear_status(cfg)) != MTA_OK) return s;
-  return launch_attn_bwd_simt(a) == cudaSuccess ? MTA_OK : MTA_ERR_CUDA;
+  return (a.kqp ? launch_attn_bwd_post(a) : launch_attn_bwd_simt(a)) == cudaSuccess ? MTA_OK : MTA_ERR_CUDA;
 }
 
 mta_status mta_gemm_bf16_nt(const void *A, const void *Bm, void *C, int M, int N, int K, void *stream) {

@@ -187,28 +187,35 @@ def attn_fwd(q, k, v, theta, w, c_q, c_k, c_h, kq_place=PRE, head_place=POST, *,
 
 
 def attn_bwd(q, k, v, theta, w, dout, c_q, c_k, c_h, kq_place=PRE, head_place=POST, *, ws=None,
-             path=PATH_AUTO, scale=0.0, stream=None, check=False, grads=None):
-    """Gradients of attn_fwd.  dout: [B, L, H, d] dense, dtype of q.  Returns a dict
-    of fp32 tensors: dq, dk, dv [B, L, H, d], dtheta [H, c_q, c_k] (kq_place on)
-    and dw [H/c_h, c_h, c_h] (head_place on).  `grads` may pass that dict to reuse."""
+             path=PATH_AUTO, scale=0.0, stream=None, check=False, grads=None, theta_post=None):
+    """Gradients of attn_fwd.  dout: [B, L, H, d] dense, dtype of q.  theta,
+    theta_post: as for attn_fwd (a stacked [n, H, c_q, c_k] theta included).
+    Returns a dict of fp32 tensors: dq, dk, dv [B, L, H, d]; dtheta [H, c_q, c_k]
+    (kq_place on) and dtheta_post [H, c_q, c_k] (post-softmax convolution), views of
+    one dtheta_all [n, H, c_q, c_k] laid out as the kernel array; dw
+    [H/c_h, c_h, c_h] (head_place on).  `grads` may pass that dict to reuse."""
     import torch
     B, L, H, d = q.shape
     if dout.shape != q.shape or dout.dtype != q.dtype or not dout.is_contiguous():
         raise ValueError("dout must be a dense [B, L, H, d] tensor of q's dtype")
+    theta, kq_post = _kernels(theta, theta_post, kq_place)
+    n_th = (1 if kq_place != OFF else 0) + kq_post
     if grads is None:
         z = lambda *shape: torch.empty(shape, dtype=torch.float32, device=q.device)
-        grads = {"dq": z(B, L, H, d), "dk": z(B, L, H, d), "dv": z(B, L, H, d),
-                 "dtheta": z(H, c_q, c_k) if kq_place != OFF else None,
+        dth = z(n_th, H, c_q, c_k) if n_th else None
+        grads = {"dq": z(B, L, H, d), "dk": z(B, L, H, d), "dv": z(B, L, H, d), "dtheta_all": dth,
+                 "dtheta": dth[0] if kq_place != OFF else None,
+                 "dtheta_post": dth[n_th - 1] if kq_post else None,
                  "dw": z(H // c_h, c_h, c_h) if head_place != OFF else None}
     cfg = make_cfg(B, H, L, d, c_q, c_k, c_h, kq_place, head_place, _dtype_code(q), path, scale,
-                   q.stride(1), _stream_handle(stream))
+                   q.stride(1), _stream_handle(stream), kq_post=kq_post)
     if ws is None:
         ws = workspace(lib().mta_attn_bwd_workspace_bytes(ctypes.byref(cfg)), q.device)
     cfg.workspace, cfg.workspace_bytes = ws.data_ptr(), ws.numel()
     _check("mta_attn_bwd", lib().mta_attn_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(theta), _ptr(w),
                                              _ptr(dout), ctypes.byref(cfg), _ptr(grads["dq"]),
                                              _ptr(grads["dk"]), _ptr(grads["dv"]),
-                                             _ptr(grads["dtheta"]), _ptr(grads["dw"])))
+                                             _ptr(grads["dtheta_all"]), _ptr(grads["dw"])))
     if check:
         _check("mta_sync_status", lib().mta_sync_status(ctypes.byref(cfg)))
     return grads
