@@ -154,3 +154,25 @@ def test_building_block_argument_errors(L):
     gn = mta.MtaGn(0x20000, 0x20000, 1e-5, 12, -1.0)
     assert L.mta_group_norm_scale(FAKE, ctypes.byref(gn), 4, 2, 0, FAKE, None) == 1
     assert L.mta_group_norm_scale(FAKE, None, 4, 2, 64, FAKE, None) == 1
+
+
+def test_backward_argument_errors(L):
+    """mta_attn_bwd checks its arguments on the host and enqueues nothing on error."""
+    cfg = good_cfg()
+    cfg.workspace, cfg.workspace_bytes = 0x100000, 1 << 20
+    f = lambda c, dq=FAKE, theta=FAKE, dout=FAKE: L.mta_attn_bwd(FAKE, FAKE, FAKE, theta, FAKE, dout,
+                                                                  ctypes.byref(c) if c else None,
+                                                                  dq, FAKE, FAKE, FAKE, FAKE)
+    assert f(None) == 1
+    assert f(cfg, dq=None) == 1
+    assert f(cfg, dout=None) == 1
+    assert f(cfg, theta=None) == 1                      # kq_place PRE needs the kernels
+    assert f(cfg, dq=ctypes.c_void_p(0x10002)) == 1     # fp32 gradients, 4-byte aligned
+    forced = good_cfg(path=mta.PATH_TC)                 # only the CUDA-core backward exists
+    forced.workspace, forced.workspace_bytes = 0x100000, 1 << 20
+    assert f(forced) == 2
+    small = good_cfg()
+    small.workspace, small.workspace_bytes = 0x100000, 16
+    assert f(small) == 3
+    assert L.mta_attn_bwd_workspace_bytes(ctypes.byref(good_cfg())) == 256
+    assert L.mta_attn_bwd_workspace_bytes(ctypes.byref(good_cfg(c_k=4))) == 0
