@@ -32,6 +32,7 @@ namespace {
 constexpr int kThreads = 256;
 constexpr int kBC = 32;
 constexpr int kSmemCap = 200 * 1024;
+constexpr int kTwoPerSm = 112 * 1024;  // two CTAs per SM (228 KB of shared memory)
 
 template <typename T>
 __device__ __forceinline__ float ld(const T *p);
@@ -353,11 +354,16 @@ __global__ void __launch_bounds__(kThreads) attn_bwd_simt_kernel(BwdArgs a, int 
 
 }  // namespace
 
+// Rows per CTA: the largest BR whose tile lets two CTAs share an SM (the kernel is
+// latency-bound at one), else the largest that fits at all.
 int attn_bwd_simt_pick_rows(const BwdArgs &a) {
+  auto bytes = [&](int BR) {
+    return static_cast<size_t>(bwd_layout(BR, kBC, a.d, a.cq, a.ck, a.ch, a.kq != 0).total) * sizeof(float);
+  };
+  for (int BR = 16; BR >= 4; BR /= 2)
+    if (bytes(BR) <= static_cast<size_t>(kTwoPerSm)) return BR;
   for (int BR = 16; BR >= 1; BR /= 2)
-    if (static_cast<size_t>(bwd_layout(BR, kBC, a.d, a.cq, a.ck, a.ch, a.kq != 0).total) * sizeof(float) <=
-        static_cast<size_t>(kSmemCap))
-      return BR;
+    if (bytes(BR) <= static_cast<size_t>(kSmemCap)) return BR;
   return 0;
 }
 
