@@ -94,11 +94,14 @@ __host__ __device__ inline PostLayout post_layout(int BR, int BC, int d, int cq,
   return s;
 }
 
-template <typename T>
-__global__ void __launch_bounds__(kThreads) attn_bwd_post_kernel(BwdArgs a, int BR) {
+// The shape parameters DT, CQT, CKT, CHT, BRT are compile-time constants when
+// nonzero (the index arithmetic of every loop then folds), else read at run time.
+template <typename T, int DT, int CQT, int CKT, int CHT, int BRT>
+__global__ void __launch_bounds__(kThreads) attn_bwd_post_kernel(BwdArgs a, int BR_) {
+  const int BR = BRT ? BRT : BR_;
   extern __shared__ float sm[];
   const int BC = kBC;
-  const int d = a.d, cq = a.cq, ck = a.ck, ch = a.ch, L = a.L, H = a.H;
+  const int d = DT ? DT : a.d, cq = CQT ? CQT : a.cq, ck = CKT ? CKT : a.ck, ch = CHT ? CHT : a.ch, L = a.L, H = a.H;
   const bool kq = a.kq != 0, exact = a.kq == 3;
   const PostGeo q = post_geo(BR, BC, d, cq, ck);
   const int P1 = q.P1, c = q.c, NRA = q.NRA, NKA = q.NKA, NRM = q.NRM, NKM = q.NKM;
@@ -452,18 +455,20 @@ cudaError_t launch_attn_bwd_post(const BwdArgs &a) {
       (e = cudaMemsetAsync(a.dw, 0, static_cast<size_t>(a.H) * a.ch * sizeof(float), a.stream)) != cudaSuccess)
     return e;
   dim3 grid((a.L + BR - 1) / BR, a.H / a.ch, a.B);
-  if (a.dtype == 0) {
-    e = cudaFuncSetAttribute(attn_bwd_post_kernel<float>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             static_cast<int>(smem));
-    if (e != cudaSuccess) return e;
-    attn_bwd_post_kernel<float><<<grid, kThreads, smem, a.stream>>>(a, BR);
-  } else {
-    e = cudaFuncSetAttribute(attn_bwd_post_kernel<__nv_bfloat16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             static_cast<int>(smem));
-    if (e != cudaSuccess) return e;
-    attn_bwd_post_kernel<__nv_bfloat16><<<grid, kThreads, smem, a.stream>>>(a, BR);
+  auto run = [&](auto kern) -> cudaError_t {
+    cudaError_t e2 = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+    if (e2 != cudaSuccess) return e2;
+    kern<<<grid, kThreads, smem, a.stream>>>(a, BR);
+    return cudaGetLastError();
+  };
+  // specialisations of the pretraining recipe (bf16, c_q = 6, c_k = 11, groups of 2)
+  if (a.dtype == 1 && a.cq == 6 && a.ck == 11 && a.ch == 2) {
+    if (a.d == 128 && BR == 8) return run(attn_bwd_post_kernel<__nv_bfloat16, 128, 6, 11, 2, 8>);
+    if (a.d == 64 && BR == 8) return run(attn_bwd_post_kernel<__nv_bfloat16, 64, 6, 11, 2, 8>);
+    if (a.d == 64 && BR == 16) return run(attn_bwd_post_kernel<__nv_bfloat16, 64, 6, 11, 2, 16>);
   }
-  return cudaGetLastError();
+  if (a.dtype == 0) return run(attn_bwd_post_kernel<float, 0, 0, 0, 0, 0>);
+  return run(attn_bwd_post_kernel<__nv_bfloat16, 0, 0, 0, 0, 0>);
 }
 
 }  // namespace mta
