@@ -27,6 +27,7 @@
 #include <cuda_bf16.h>
 #include <math.h>
 
+#include "bwd_common.cuh"
 #include "internal.h"
 
 namespace mta {
@@ -156,16 +157,11 @@ __global__ void __launch_bounds__(kThreads) attn_bwd_post_kernel(BwdArgs a, int 
         }
         __syncthreads();
         float *sh = Sh + hl * NRM * NKM;
-        for (int i = tid; i < NRM * NKM; i += kThreads) {
-          const int r = i / NKM, s = i % NKM, iq = i0 - 2 * P1 + r, jk = j0 - 2 * c + s;
-          float val = 0.f;
-          if (iq >= 0 && iq < L && jk >= 0 && jk < L && (!kq || exact || jk <= iq)) {
-            const float *qr = Qs + r * dp, *kr = Ks + s * dp;
-            for (int e = 0; e < d; ++e) val = fmaf(qr[e], kr[e], val);
-            val *= a.scale;
-          }
-          sh[i] = val;
-        }
+        dot_rows4<kThreads>(Qs, Ks, NRM, NKM, d, dp, [&](int r, int s, float v) {
+          const int iq = i0 - 2 * P1 + r, jk = j0 - 2 * c + s;
+          const bool ok = iq >= 0 && iq < L && jk >= 0 && jk < L && (!kq || exact || jk <= iq);
+          sh[r * NKM + s] = ok ? v * a.scale : 0.f;
+        });
         __syncthreads();
         for (int i = tid; i < RA; i += kThreads) {  // C on the A region
           const int ra = i / NKA, ka = i % NKA;
@@ -190,13 +186,8 @@ __global__ void __launch_bounds__(kThreads) attn_bwd_post_kernel(BwdArgs a, int 
           Ks[s * dp + e] = (jk >= 0 && jk < L) ? ldv(vp + gidx(jk, h) + e) : 0.f;
         }
         __syncthreads();
-        for (int i = tid; i < RG; i += kThreads) {
-          const int rg = i / NKG, kg = i % NKG;
-          const float *dr = DO + (hl * NRG + rg) * dp, *vr = Ks + kg * dp;
-          float val = 0.f;
-          for (int e = 0; e < d; ++e) val = fmaf(dr[e], vr[e], val);
-          Gd[hl * RG + i] = val;
-        }
+        dot_rows4<kThreads>(DO + hl * NRG * dp, Ks, NRG, NKG, d, dp,
+                            [&](int r, int s, float v) { Gd[hl * RG + r * NKG + s] = v; });
         __syncthreads();
       }
       // ---- mixed logits with Mask_-inf (A region); g = Mask_0(post-mix adjoint of G)

@@ -24,6 +24,7 @@
 #include <cuda_bf16.h>
 #include <math.h>
 
+#include "bwd_common.cuh"
 #include "internal.h"
 
 namespace mta {
@@ -130,16 +131,11 @@ __global__ void __launch_bounds__(kThreads) attn_bwd_simt_kernel(BwdArgs a, int 
         }
         __syncthreads();
         float *sh = Sh + hl * HR * HC;
-        for (int i = tid; i < HR * HC; i += kThreads) {
-          const int r = i / HC, s = i % HC, iq = i0 - (cq - 1) + r, jk = j0 - PC - c + s;
-          float val = 0.f;
-          if (iq >= 0 && iq < L && jk >= 0 && jk < L && (!kq || exact || jk <= iq)) {
-            const float *qr = Qs + r * dp, *kr = Ks + s * dp;
-            for (int e = 0; e < d; ++e) val = fmaf(qr[e], kr[e], val);
-            val *= a.scale;
-          }
-          sh[i] = val;
-        }
+        dot_rows4<kThreads>(Qs, Ks, HR, HC, d, dp, [&](int r, int s, float v) {
+          const int iq = i0 - (cq - 1) + r, jk = j0 - PC - c + s;
+          const bool ok = iq >= 0 && iq < L && jk >= 0 && jk < L && (!kq || exact || jk <= iq);
+          sh[r * HC + s] = ok ? v * a.scale : 0.f;
+        });
         __syncthreads();
         for (int i = tid; i < region; i += kThreads) {
           const int r = i / CC, s = i % CC;
@@ -164,13 +160,8 @@ __global__ void __launch_bounds__(kThreads) attn_bwd_simt_kernel(BwdArgs a, int 
           Ks[s * dp + e] = (jk >= 0 && jk < L) ? ld(v + gidx(jk, h) + e) : 0.f;
         }
         __syncthreads();
-        for (int i = tid; i < region; i += kThreads) {
-          const int r = i / CC, s = i % CC;
-          const float *dr = DO + (hl * CR + r) * dp, *vr = Ks + s * dp;
-          float val = 0.f;
-          for (int e = 0; e < d; ++e) val = fmaf(dr[e], vr[e], val);
-          Gd[hl * region + i] = val;
-        }
+        dot_rows4<kThreads>(DO + hl * CR * dp, Ks, CR, CC, d, dp,
+                            [&](int r, int s, float v) { Gd[hl * region + r * CC + s] = v; });
         __syncthreads();
       }
       // ---- mixed logits (pre-softmax mix), Mask_-inf; dA (post-softmax mix adjoint)
