@@ -304,26 +304,29 @@ __global__ void __launch_bounds__(kThreads) attn_bwd_post_kernel(BwdArgs a, int 
         atomicAdd(dthp + at, acc);
       }
       __syncthreads();
-      // dV_h[j] += sum over the tile's rows of A3_h[i][j] dO_h[i], A3 = post mix of A2
+      // A3 = post mix of A2, in place (the parameter gradients above are done with A2),
+      // then dV_h[j] += sum over the tile's rows of A3_h[i][j] dO_h[i]
+      if (a.hp == 2) {
+        for (int i = tid; i < TILE; i += kThreads) {
+          float x[16];
+          for (int s2 = 0; s2 < ch; ++s2) x[s2] = A2[s2 * TILE + i];
+          for (int hl = 0; hl < ch; ++hl) {
+            float pa = 0.f;
+            for (int s2 = 0; s2 < ch; ++s2) pa = fmaf(wg[hl * ch + s2], x[s2], pa);
+            A2[hl * TILE + i] = pa;
+          }
+        }
+        __syncthreads();
+      }
       for (int i = tid; i < ch * BC * d; i += kThreads) {
         const int hl = i / (BC * d), rem = i % (BC * d), s = rem / d, e = rem % d, jk = j0 + s;
         if (jk >= L) continue;
         float acc = 0.f;
-        for (int r = 0; r < BR; ++r) {
-          if (i0 + r >= L) break;
-          float pa;
-          if (a.hp == 2) {
-            pa = 0.f;
-            for (int s2 = 0; s2 < ch; ++s2) pa = fmaf(wg[hl * ch + s2], A2[s2 * TILE + r * BC + s], pa);
-          } else {
-            pa = A2[hl * TILE + r * BC + s];
-          }
-          acc = fmaf(pa, DO[(hl * NRG + r) * dp + e], acc);
-        }
+        for (int r = 0; r < BR; ++r) acc = fmaf(A2[hl * TILE + r * BC + s], DO[(hl * NRG + r) * dp + e], acc);
         atomicAdd(a.dv + oidx(jk, g * ch + hl) + e, acc);
       }
-      // dC_s = sum_h w[h][s] dC'_h (pre-softmax mixing), into gg's space is not free: reuse A2? no --
-      // write it over Cp (C_s is no longer needed once dw is taken)
+      // dC_s = sum_h w[h][s] dC'_h (pre-softmax mixing), written over C_s (no longer needed
+      // once dw is taken)
       __syncthreads();
       const float *dcs = dA;
       if (a.hp == 1) {
@@ -382,18 +385,33 @@ __global__ void __launch_bounds__(kThreads) attn_bwd_post_kernel(BwdArgs a, int 
           Ks[s * dp + e] = jk < L ? ldv(kp + gidx(jk, h) + e) : 0.f;
         }
         __syncthreads();
-        for (int i = tid; i < BR * d; i += kThreads) {  // dQ += dA_hat K
-          const int r = i / d, e = i % d;
-          float acc = dqa[(sl * BR + r) * d + e];
-          for (int s = 0; s < BC; ++s) acc = fmaf(Tmp[r * BC + s], Ks[s * dp + e], acc);
-          dqa[(sl * BR + r) * d + e] = acc;
+        // dQ += dA_hat K and dK += dA_hat^T Q, four rows (columns) per thread sharing
+        // each K (Q) load
+        for (int i = tid; i < (BR + 3) / 4 * d; i += kThreads) {
+          const int r0 = 4 * (i / d), e = i % d;
+          float acc[4];
+#pragma unroll
+          for (int k2 = 0; k2 < 4; ++k2) acc[k2] = r0 + k2 < BR ? dqa[(sl * BR + r0 + k2) * d + e] : 0.f;
+          for (int s = 0; s < BC; ++s) {
+            const float x = Ks[s * dp + e];
+#pragma unroll
+            for (int k2 = 0; k2 < 4; ++k2) acc[k2] = fmaf(Tmp[min(r0 + k2, BR - 1) * BC + s], x, acc[k2]);
+          }
+#pragma unroll
+          for (int k2 = 0; k2 < 4; ++k2)
+            if (r0 + k2 < BR) dqa[(sl * BR + r0 + k2) * d + e] = acc[k2];
         }
-        for (int i = tid; i < BC * d; i += kThreads) {  // dK += dA_hat^T Q
-          const int s = i / d, e = i % d, jk = j0 + s;
-          if (jk >= L) continue;
-          float acc = 0.f;
-          for (int r = 0; r < BR; ++r) acc = fmaf(Tmp[r * BC + s], Qs[r * dp + e], acc);
-          atomicAdd(a.dk + oidx(jk, h) + e, acc);
+        for (int i = tid; i < BC / 4 * d; i += kThreads) {
+          const int s0 = 4 * (i / d), e = i % d;
+          float acc[4] = {0.f, 0.f, 0.f, 0.f};
+          for (int r = 0; r < BR; ++r) {
+            const float x = Qs[r * dp + e];
+#pragma unroll
+            for (int k2 = 0; k2 < 4; ++k2) acc[k2] = fmaf(Tmp[r * BC + s0 + k2], x, acc[k2]);
+          }
+#pragma unroll
+          for (int k2 = 0; k2 < 4; ++k2)
+            if (j0 + s0 + k2 < L) atomicAdd(a.dk + oidx(j0 + s0 + k2, h) + e, acc[k2]);
         }
         __syncthreads();
       }

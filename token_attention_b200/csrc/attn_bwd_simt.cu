@@ -43,7 +43,7 @@ template <>
 __device__ __forceinline__ float ld<__nv_bfloat16>(const __nv_bfloat16 *p) { return __bfloat162float(*p); }
 
 struct BwdLayout {
-  int Qs, Ks, DO, Sh, Cp, P, Gd, Dc, Tmp, m, l, Ds, dqa, th, wg, dth, dwa, total;
+  int Qs, Ks, DO, Sh, Cp, P, Gd, Dc, Tmp, A3, m, l, Ds, dqa, th, wg, dth, dwa, total;
 };
 
 __host__ __device__ inline BwdLayout bwd_layout(int BR, int BC, int d, int cq, int ck, int ch, bool kq) {
@@ -60,6 +60,7 @@ __host__ __device__ inline BwdLayout bwd_layout(int BR, int BC, int d, int cq, i
   s.Gd = o;  o += ch * CR * CC;       // dO_h . v_h
   s.Dc = o;  o += ch * CR * CC;       // dA, then dC' and dC
   s.Tmp = o; o += BR * BC;            // dA_hat of the tile, one head
+  s.A3 = o;  o += ch * BR * BC;       // post-softmax-mixed weights A'' of the tile
   s.m = o;   o += ch * CR;
   s.l = o;   o += ch * CR;
   s.Ds = o;  o += ch * CR;            // D (row sums), accumulated then normalised
@@ -86,7 +87,7 @@ __global__ void __launch_bounds__(kThreads) attn_bwd_simt_kernel(BwdArgs a, int 
   const int region = CR * CC;
   const BwdLayout S = bwd_layout(BR, BC, d, cq, ck, ch, kq);
   float *Qs = sm + S.Qs, *Ks = sm + S.Ks, *DO = sm + S.DO, *Sh = sm + S.Sh, *Cp = sm + S.Cp;
-  float *P = sm + S.P, *Gd = sm + S.Gd, *Dc = sm + S.Dc, *Tmp = sm + S.Tmp;
+  float *P = sm + S.P, *Gd = sm + S.Gd, *Dc = sm + S.Dc, *Tmp = sm + S.Tmp, *A3 = sm + S.A3;
   float *rm = sm + S.m, *rl = sm + S.l, *Ds = sm + S.Ds, *dqa = sm + S.dqa;
   float *th = sm + S.th, *wg = sm + S.wg, *dth = sm + S.dth, *dwa = sm + S.dwa;
   const int i0 = blockIdx.x * BR, g = blockIdx.y, b = blockIdx.z, tid = threadIdx.x;
@@ -246,22 +247,26 @@ __global__ void __launch_bounds__(kThreads) attn_bwd_simt_kernel(BwdArgs a, int 
         __syncthreads();
         dcs = Gd;
       }
-      // dV_h[j] += sum over the tile's rows of A''_h[i][j] dO_h[i], A'' = post-softmax mix of A
-      for (int i = tid; i < ch * BC * d; i += kThreads) {
-        const int hl = i / (BC * d), rem = i % (BC * d), s = rem / d, e = rem % d, jk = j0 + s;
-        if (jk >= L) continue;
-        float acc = 0.f;
-        for (int r = 0; r < BR; ++r) {
-          if (i0 + r >= L) break;
-          float pa;
+      // A'' = post-softmax mix of A on the tile (rows past L are 0), then
+      // dV_h[j] += sum over the tile's rows of A''_h[i][j] dO_h[i]
+      for (int i = tid; i < ch * BR * BC; i += kThreads) {
+        const int hl = i / (BR * BC), rem = i % (BR * BC), r = rem / BC, s = rem % BC;
+        float pa = 0.f;
+        if (i0 + r < L) {
           if (a.hp == 2) {
-            pa = 0.f;
             for (int s2 = 0; s2 < ch; ++s2) pa = fmaf(wg[hl * ch + s2], P[(s2 * CR + r) * CC + s + PC], pa);
           } else {
             pa = P[(hl * CR + r) * CC + s + PC];
           }
-          acc = fmaf(pa, DO[(hl * CR + r) * dp + e], acc);
         }
+        A3[i] = pa;
+      }
+      __syncthreads();
+      for (int i = tid; i < ch * BC * d; i += kThreads) {
+        const int hl = i / (BC * d), rem = i % (BC * d), s = rem / d, e = rem % d, jk = j0 + s;
+        if (jk >= L) continue;
+        float acc = 0.f;
+        for (int r = 0; r < BR; ++r) acc = fmaf(A3[(hl * BR + r) * BC + s], DO[(hl * CR + r) * dp + e], acc);
         atomicAdd(a.dv + oidx(jk, g * ch + hl) + e, acc);
       }
       // per source head: dtheta, dA_hat of the tile, dQ, dK
@@ -314,18 +319,33 @@ __global__ void __launch_bounds__(kThreads) attn_bwd_simt_kernel(BwdArgs a, int 
           Ks[s * dp + e] = jk < L ? ld(k + gidx(jk, h) + e) : 0.f;
         }
         __syncthreads();
-        for (int i = tid; i < BR * d; i += kThreads) {  // dQ += dA_hat K
-          const int r = i / d, e = i % d;
-          float acc = dqa[(sl * BR + r) * d + e];
-          for (int s = 0; s < BC; ++s) acc = fmaf(Tmp[r * BC + s], Ks[s * dp + e], acc);
-          dqa[(sl * BR + r) * d + e] = acc;
+        // dQ += dA_hat K and dK += dA_hat^T Q, four rows (columns) per thread sharing
+        // each K (Q) load
+        for (int i = tid; i < (BR + 3) / 4 * d; i += kThreads) {
+          const int r0 = 4 * (i / d), e = i % d;
+          float acc[4];
+#pragma unroll
+          for (int k2 = 0; k2 < 4; ++k2) acc[k2] = r0 + k2 < BR ? dqa[(sl * BR + r0 + k2) * d + e] : 0.f;
+          for (int s = 0; s < BC; ++s) {
+            const float x = Ks[s * dp + e];
+#pragma unroll
+            for (int k2 = 0; k2 < 4; ++k2) acc[k2] = fmaf(Tmp[min(r0 + k2, BR - 1) * BC + s], x, acc[k2]);
+          }
+#pragma unroll
+          for (int k2 = 0; k2 < 4; ++k2)
+            if (r0 + k2 < BR) dqa[(sl * BR + r0 + k2) * d + e] = acc[k2];
         }
-        for (int i = tid; i < BC * d; i += kThreads) {  // dK += dA_hat^T Q
-          const int s = i / d, e = i % d, jk = j0 + s;
-          if (jk >= L) continue;
-          float acc = 0.f;
-          for (int r = 0; r < BR; ++r) acc = fmaf(Tmp[r * BC + s], Qs[r * dp + e], acc);
-          atomicAdd(a.dk + oidx(jk, h) + e, acc);
+        for (int i = tid; i < BC / 4 * d; i += kThreads) {
+          const int s0 = 4 * (i / d), e = i % d;
+          float acc[4] = {0.f, 0.f, 0.f, 0.f};
+          for (int r = 0; r < BR; ++r) {
+            const float x = Qs[r * dp + e];
+#pragma unroll
+            for (int k2 = 0; k2 < 4; ++k2) acc[k2] = fmaf(Tmp[r * BC + s0 + k2], x, acc[k2]);
+          }
+#pragma unroll
+          for (int k2 = 0; k2 < 4; ++k2)
+            if (j0 + s0 + k2 < L) atomicAdd(a.dk + oidx(j0 + s0 + k2, h) + e, acc[k2]);
         }
         __syncthreads();
       }
