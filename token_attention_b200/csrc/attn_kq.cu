@@ -3,10 +3,13 @@
 //
 // What it computes ("Multi-Token Attention | Summary" (greeksharifa)):
 //   section 2  : logits A_hat = Q K^T / sqrt(d), causal softmax, A V;
-//   section 3.1: A = Softmax(Mask_-inf(Conv2d_theta(Mask_0(A_hat))));
-//   section 3.2: post-softmax head mixing inside groups of 2 heads (appendix B:
-//                through the values, O^h = sum_s w[h][s] A^s V^h);
-//   section 3.3: optional group norm + depth scale (fused epilogue).
+//   section 3.1: A = Softmax(Mask_-inf(Conv2d_theta(Mask_0(A_hat)))) (or the exact
+//                causal indicator), and optionally the convolution after the
+//                softmax, A' = Mask_0(Conv2d_theta_post(A));
+//   section 3.2: head mixing inside groups of 2 heads, before the softmax or after
+//                it (appendix B: through the values, O^h = sum_s w[h][s] A^s V^h);
+//   section 3.3: optional group norm with a depth scale or sigmoid gate (fused
+//                epilogue).
 //
 // The convolution is linear in the logits, and the logits are bilinear in q and
 // k, so without the mask
@@ -21,22 +24,28 @@
 // kernel reads for query i depends on an input after position i, so outputs are
 // exactly causal (the query tile's fp16 scale only scales down, when |q| > 2^14).
 //
-// Design (one CTA = one (batch, head, tile of 128 queries)):
-//   * TMA loads the query rows i0-(c_q-1) .. i0+127 once, as 8-element strips in
-//     which consecutive rows are 16 bytes apart; the softmax warpgroup converts
-//     them in place to fp16 with a power-of-2 scale.  A row shift by a is then a
-//     16*a-byte offset of the MMA descriptor (SWIZZLE_NONE layout).
-//   * Per key tile of 128: TMA streams the c_q*d/64 chunks of Kt (fp16, 128-byte
-//     swizzle) through a 4-stage ring; one thread issues the 4*c_q*d/64 MMAs
-//     (M=128, N=128, K=16) of C into tensor memory, then P V (P read from tensor
-//     memory) into Z for every destination head of the group.
-//   * One softmax warpgroup (a whole query row per thread, so the row max needs
-//     no exchange) reads C, rescales it, applies the Mask_0 correction near the
-//     diagonal and Mask_-inf, keeps an exact online softmax (the running max
-//     moves only when it grows by more than 2^8, then Z is rescaled) and writes
+// Design (persistent: one CTA, or a 2-CTA cluster with post-softmax mixing, per SM,
+// walking (query tile of 128, batch, head group) work items longest first):
+//   * Warp 10's TMA loads the query rows i0-(c_q-1) .. i0+127 of each item as
+//     8-element strips in which consecutive rows are 16 bytes apart; the softmax
+//     warps convert them in place to fp16 with a power-of-2 scale.  A row shift
+//     by a is then a 16*a-byte offset of the MMA descriptor (SWIZZLE_NONE layout).
+//   * Per key tile of 128: warp 8's TMA streams Kt (fp16, 128-byte swizzle)
+//     through a ring whose stage is a whole tap row when d is a multiple of 64;
+//     warp 9's single thread issues the contraction MMAs (M=128, N=128, K=16) of C
+//     into tensor memory, then P V (P read from tensor memory; one N=256 MMA for
+//     both heads' V with post-softmax mixing).
+//   * Two softmax warpgroups (64 key columns and half of the output channels each,
+//     a whole query row per thread) read C, scale it, apply the Mask_0 correction
+//     near the diagonal and Mask_-inf, keep an exact online softmax (the running
+//     max moves only when it grows by more than 2^8, then Z is rescaled) and write
 //     P (bf16) to tensor memory.
-//   * Post-softmax mixing runs as a 2-CTA cluster with one exchange of
-//     Z_{s->peer}/l_s through distributed shared memory in the epilogue.
+//   * Post-softmax mixing runs as a 2-CTA cluster exchanging Z_{s->peer}/l_s through
+//     an L2 buffer in the workspace once per item, handshaked by cluster mbarriers.
+//   * With the post-softmax convolution (POST) each item makes two passes (exact
+//     row statistics, then normalised weights in shared memory times the values
+//     convolved by the post-softmax kernels, c_q row-shifted products), with the c
+//     keys ending at each diagonal added on the CUDA cores (see POST below).
 //   * Every mbarrier wait is bounded (error word + early exit).
 #include <cuda.h>
 
