@@ -12,12 +12,12 @@
 // which covers every unmasked tap of the band (m = i-a - key >= 0).
 //
 // This kernel writes, per (batch, head, tile of 128 keys):
-//   Kt  [B][H][c_q*d/64][L][64] fp16: element kappa = a*d + e of key j's contraction
-//       operand (Kt_a[j][e]) sits in chunk kappa/64 at column kappa%64, so that the 128
-//       keys of a tile form one contiguous 16 KB block per chunk; every value is
-//       Kt_a[j] * 2^e_j, e_j a power-of-2 exponent per key
-//       row chosen from max|k| over the rows j-c .. j+c that Kt_a[j] reads (so no
-//       value exceeds 2^14 and small keys keep fp16's relative precision);
+//   Kt  fp16, every value Kt_a[j] * 2^e_j, e_j a power-of-2 exponent per key row
+//       chosen from max|k| over the rows j-c .. j+c that Kt_a[j] reads (so no value
+//       exceeds 2^14 and small keys keep fp16's relative precision); laid out as
+//       [B][H][c_q][L][d] when d is a multiple of 64, else as [B][H][c_q*d/64][L][64]:
+//       element kappa = a*d + e of key j's contraction operand in chunk kappa/64 at
+//       column kappa%64, so that a 64-element box of 128 keys is contiguous;
 //   fac [B][H][Lpad] fp32: s * log2(e) * 2^-e_j (the attention kernel's column
 //       factor; 0 for the padding keys L <= j < Lpad, Lpad = L rounded up to 128);
 //   Vp  [B][H][L][M] fp32: raw past dot products (no scale); with the exact causal
@@ -26,7 +26,8 @@
 // Every value written for key or query j depends on inputs at positions <= j + c
 // only, and Kt_a[j] is used only for queries i >= j + W > j + c: the path stays
 // exactly causal.  One CTA per (key tile, head, batch); the key rows with their
-// halo are staged in shared memory as bf16.
+// halo are staged in shared memory as bf16, and the convolution runs in packed
+// fp32 FMAs on channel pairs.
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 #include <math.h>
