@@ -47,7 +47,7 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 
 
 # ---------------------------------------------------------------------------
-# workload arithmetic (algorithmic counts, measurement)
+# workload arithmetic (algorithmic counts per step)
 # ---------------------------------------------------------------------------
 
 def flops(wl: synth.Workload) -> dict:

@@ -29,7 +29,7 @@ section):
             Attention (MTA) Mechanism", item 3: group normalisation with depth
             scaling.
 
-Readings where the pages leave a step open (all listed in the design doc):
+Readings where the pages leave a step open:
   * Mask_0 zeroes logits of future keys (key j > query i) before the
     convolution; indices outside [0, L) contribute 0 (zero padding).
   * theta[h][a][t] multiplies Mask_0(A_hat)[i - a][j - (t - c_k//2)]:
