@@ -54,7 +54,7 @@ extern "C" {
 typedef enum {
   MTA_OK = 0,
   MTA_ERR_INVALID = 1,      /* null pointer, bad shape or inconsistent configuration */
-  MTA_ERR_UNSUPPORTED = 2,  /* a valid configuration this build has no kernel for */
+  MTA_ERR_UNSUPPORTED = 2,  /* a valid configuration the library has no kernel for */
   MTA_ERR_WORKSPACE = 3,    /* workspace missing, misaligned or smaller than required */
   MTA_ERR_CUDA = 4,         /* a CUDA runtime call or a kernel launch failed */
   MTA_ERR_TIMEOUT = 5       /* a kernel's bounded wait ran out (see mta_sync_status) */
