@@ -626,3 +626,27 @@ def test_bwd_full_length_one_group():
     inp = synth.make_attn_inputs(wl)
     dout = synth.round_bf16(synth.normal(wl.seed, 20, (wl.B, wl.L, wl.H, wl.d)))
     check_grads(wl, inp, dout)
+
+
+@pytest.mark.parametrize("post", [False, True])
+def test_autograd_function_matches_oracle(post):
+    """mta.mta_attention as a torch op: torch.autograd.grad through it returns the
+    oracle's gradients (the op calls mta_attn_fwd and mta_attn_bwd)."""
+    base = synth.WORKLOADS["both_d128_L2048" if post else "pretrain_d128_L2048"]
+    wl = synth.shrink(base, B=1, H=4, L=90, d=64, dtype="f32", seed=871 + post)
+    inp = synth.make_attn_inputs(wl)
+    dout = synth.normal(wl.seed, 20, (wl.B, wl.L, wl.H, wl.d))
+    t = lambda x: torch.from_numpy(np.ascontiguousarray(x)).cuda().requires_grad_(True)
+    q, k, v, th, w = (t(inp[n]) for n in ("q", "k", "v", "theta", "w"))
+    tp = t(inp["theta_post"]) if post else None
+    out = mta.mta_attention(q, k, v, th, w, wl.c_q, wl.c_k, wl.c_h, wl.kq_place, wl.head_place,
+                            theta_post=tp)
+    leaves = [q, k, v, th, w] + ([tp] if post else [])
+    grads = torch.autograd.grad(out, leaves, torch.from_numpy(dout).cuda())
+    ref = O.mta_attention_bwd(inp["q"], inp["k"], inp["v"], inp["theta"], inp["w"], wl.c_h, dout,
+                              wl.kq_place, wl.head_place, theta_post=inp["theta_post"])
+    names = ["dq", "dk", "dv", "dtheta", "dw"] + (["dtheta_post"] if post else [])
+    for n, g in zip(names, grads):
+        rel, _ = errs(g, ref[n])
+        assert rel <= TOL_F32, (n, rel)
+    assert_close(out, oracle_full(wl, inp), "f32")

@@ -221,6 +221,46 @@ def attn_bwd(q, k, v, theta, w, dout, c_q, c_k, c_h, kq_place=PRE, head_place=PO
     return grads
 
 
+def _attention_function():
+    """torch.autograd.Function over mta_attn_fwd / mta_attn_bwd (built on first use,
+    so that importing this module needs no torch)."""
+    import torch
+
+    class _MtaAttention(torch.autograd.Function):
+        @staticmethod
+        def forward(ctx, q, k, v, theta, w, c_q, c_k, c_h, kq_place, head_place, theta_post):
+            out = attn_fwd(q, k, v, theta, w, c_q, c_k, c_h, kq_place, head_place, theta_post=theta_post)
+            ctx.save_for_backward(q, k, v, theta, w, theta_post)
+            ctx.shape = (c_q, c_k, c_h, kq_place, head_place)
+            return out
+
+        @staticmethod
+        def backward(ctx, dout):
+            q, k, v, theta, w, theta_post = ctx.saved_tensors
+            c_q, c_k, c_h, kq_place, head_place = ctx.shape
+            g = attn_bwd(q, k, v, theta, w, dout.contiguous().to(q.dtype), c_q, c_k, c_h, kq_place,
+                         head_place, theta_post=theta_post)
+            cast = lambda x, like: None if x is None or like is None else x.to(like.dtype)
+            return (cast(g["dq"], q), cast(g["dk"], k), cast(g["dv"], v), cast(g["dtheta"], theta),
+                    cast(g["dw"], w), None, None, None, None, None, cast(g["dtheta_post"], theta_post))
+
+    return _MtaAttention
+
+
+_MTA_FN = None
+
+
+def mta_attention(q, k, v, theta, w, c_q, c_k, c_h, kq_place=PRE, head_place=POST, theta_post=None):
+    """MTA attention as a differentiable torch op: the forward runs mta_attn_fwd, the
+    backward mta_attn_bwd (gradients of q, k, v, theta, w and theta_post, cast to
+    their dtypes).  Arguments as for attn_fwd; theta and theta_post are separate
+    [H, c_q, c_k] tensors here."""
+    global _MTA_FN
+    if _MTA_FN is None:
+        _MTA_FN = _attention_function()
+    return _MTA_FN.apply(q, k, v, theta, w, c_q, c_k, c_h, kq_place, head_place, theta_post)
+
+
 def depth_scale(layer: int) -> float:
     return 1.0 - 0.8 * math.exp(-0.3 * layer)
 
