@@ -176,3 +176,63 @@ def test_backward_argument_errors(L):
     assert f(small) == 3
     assert L.mta_attn_bwd_workspace_bytes(ctypes.byref(good_cfg())) == 256
     assert L.mta_attn_bwd_workspace_bytes(ctypes.byref(good_cfg(c_k=4))) == 0
+
+
+# ---------------------------------------------------------------------------
+# the Python binding rejects tensors the C ABI cannot take, before any call
+# ---------------------------------------------------------------------------
+
+class FakeCuda:
+    """Stands in for a CUDA tensor on a machine without a GPU: only the
+    attributes the binding's checks read."""
+
+    def __init__(self, shape, dtype, contiguous=True, index=0):
+        import torch
+        self.shape, self.dtype, self._c = tuple(shape), dtype, contiguous
+        self.is_cuda, self.device = True, torch.device("cuda", index)
+
+    def is_contiguous(self):
+        return self._c
+
+
+def test_binding_checks_device_dtype_shape_layout():
+    import torch
+    dv = torch.device("cuda", 0)
+    f32 = torch.float32
+    mta._need("t", None, dv, f32, (2, 3))                     # optional argument left out
+    mta._need("t", FakeCuda((2, 3), f32), dv, f32, (2, 3))
+    with pytest.raises(ValueError, match="CUDA tensor"):
+        mta._need("t", torch.zeros(2, 3), dv, f32, (2, 3))   # host memory
+    with pytest.raises(ValueError, match="CUDA tensor"):
+        mta._need("t", FakeCuda((2, 3), f32, index=1), dv)    # another GPU
+    with pytest.raises(TypeError, match="bfloat16"):
+        mta._need("t", FakeCuda((2, 3), f32), dv, torch.bfloat16)
+    with pytest.raises(ValueError, match="shape"):
+        mta._need("t", FakeCuda((3, 2), f32), dv, f32, (2, 3))
+    with pytest.raises(ValueError, match="contiguous"):
+        mta._need("t", FakeCuda((2, 3), f32, contiguous=False), dv, f32)
+    mta._need("t", FakeCuda((2, 3), f32, contiguous=False), dv, f32, contiguous=False)
+
+
+def test_binding_rejects_host_tensors():
+    """Host tensors would hand host pointers to the kernels: every entry point
+    refuses them with a ValueError before calling the library."""
+    import torch
+    B, L, H, d = 1, 8, 2, 32
+    bf = lambda *s: torch.zeros(s, dtype=torch.bfloat16)
+    f32 = lambda *s: torch.zeros(s, dtype=torch.float32)
+    q = bf(B, L, H, d)
+    th, w = f32(H, 3, 5), f32(1, 2, 2)
+    with pytest.raises(ValueError, match="CUDA tensor"):
+        mta.attn_fwd(q, q, q, th, w, 3, 5, 2)
+    with pytest.raises(ValueError, match="CUDA tensor"):
+        mta.attn_bwd(q, q, q, th, w, q, 3, 5, 2)
+    D = H * d
+    with pytest.raises(ValueError, match="CUDA tensor"):
+        mta.layer_fwd(bf(B, L, D), bf(3 * D, D), th, w, f32(D), f32(D), bf(D, D), H, 3, 5, 2)
+    with pytest.raises(ValueError, match="multiple of H"):
+        mta.layer_fwd(bf(B, L, 65), bf(195, 65), th, w, f32(65), f32(65), bf(65, 65), H, 3, 5, 2)
+    with pytest.raises(ValueError, match="CUDA tensor"):
+        mta.gemm_bf16_nt(bf(16, 8), bf(4, 8))
+    with pytest.raises(ValueError, match="CUDA tensor"):
+        mta.group_norm_scale(q, f32(H * d), f32(H * d))

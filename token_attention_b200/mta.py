@@ -98,6 +98,27 @@ def _ptr(t):
     return None if t is None else ctypes.c_void_p(t.data_ptr())
 
 
+def _need(name, t, device, dtype=None, shape=None, contiguous=True):
+    """Rejects, before the library sees it, a tensor the C ABI cannot take.  The
+    library reads raw device pointers, so a host tensor, a tensor on another GPU,
+    another dtype or a strided view would be read as something else.  None passes
+    (an optional argument)."""
+    if t is None:
+        return
+    if not t.is_cuda or t.device != device:
+        raise ValueError(f"{name} must be a CUDA tensor on {device}, not on {t.device}")
+    if dtype is not None and t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, not {t.dtype}")
+    if shape is not None and tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} must have shape {tuple(shape)}, not {tuple(t.shape)}")
+    if contiguous and not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+
+
+def _nbytes(t) -> int:
+    return t.numel() * t.element_size()
+
+
 def _stream_handle(stream):
     import torch
     s = stream if stream is not None else torch.cuda.current_stream()
@@ -171,6 +192,13 @@ def attn_fwd(q, k, v, theta, w, c_q, c_k, c_h, kq_place=PRE, head_place=POST, *,
             raise ValueError("q, k, v must share shape, strides and dtype")
     if q.stride(3) != 1 or q.stride(2) != d or q.stride(0) != L * q.stride(1):
         raise ValueError("q, k, v must be [B, L, H, d] with dense heads and a token stride")
+    dv = q.device
+    for name, t in (("q", q), ("k", k), ("v", v)):
+        _need(name, t, dv, contiguous=False)
+    for name, t in (("theta", theta), ("w", w), ("theta_post", theta_post)):
+        _need(name, t, dv, torch.float32)
+    _need("out", out, dv, q.dtype, (B, L, H, d))
+    _need("ws", ws, dv)
     if out is None:
         out = torch.empty((B, L, H, d), dtype=q.dtype, device=q.device)
     theta, kq_post = _kernels(theta, theta_post, kq_place)
@@ -178,7 +206,7 @@ def attn_fwd(q, k, v, theta, w, c_q, c_k, c_h, kq_place=PRE, head_place=POST, *,
                    q.stride(1), _stream_handle(stream), kq_post=kq_post)
     if ws is None:
         ws = workspace(lib().mta_attn_workspace_bytes(ctypes.byref(cfg)), q.device)
-    cfg.workspace, cfg.workspace_bytes = ws.data_ptr(), ws.numel()
+    cfg.workspace, cfg.workspace_bytes = ws.data_ptr(), _nbytes(ws)
     _check("mta_attn_fwd", lib().mta_attn_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(theta), _ptr(w),
                                              ctypes.byref(cfg), _ptr(out)))
     if check:
@@ -198,6 +226,17 @@ def attn_bwd(q, k, v, theta, w, dout, c_q, c_k, c_h, kq_place=PRE, head_place=PO
     B, L, H, d = q.shape
     if dout.shape != q.shape or dout.dtype != q.dtype or not dout.is_contiguous():
         raise ValueError("dout must be a dense [B, L, H, d] tensor of q's dtype")
+    if q.stride(3) != 1 or q.stride(2) != d or q.stride(0) != L * q.stride(1):
+        raise ValueError("q, k, v must be [B, L, H, d] with dense heads and a token stride")
+    dv = q.device
+    for name, t in (("q", q), ("k", k), ("v", v)):
+        _need(name, t, dv, q.dtype, q.shape, contiguous=False)
+        if t.stride() != q.stride():
+            raise ValueError("q, k, v must share strides")
+    _need("dout", dout, dv)
+    for name, t in (("theta", theta), ("w", w), ("theta_post", theta_post)):
+        _need(name, t, dv, torch.float32)
+    _need("ws", ws, dv)
     theta, kq_post = _kernels(theta, theta_post, kq_place)
     n_th = (1 if kq_place != OFF else 0) + kq_post
     if grads is None:
@@ -207,11 +246,21 @@ def attn_bwd(q, k, v, theta, w, dout, c_q, c_k, c_h, kq_place=PRE, head_place=PO
                  "dtheta": dth[0] if kq_place != OFF else None,
                  "dtheta_post": dth[n_th - 1] if kq_post else None,
                  "dw": z(H // c_h, c_h, c_h) if head_place != OFF else None}
+    else:
+        want = {"dq": (B, L, H, d), "dk": (B, L, H, d), "dv": (B, L, H, d),
+                "dtheta_all": (n_th, H, c_q, c_k) if n_th else None,
+                "dw": (H // c_h, c_h, c_h) if head_place != OFF else None}
+        for name, shape in want.items():
+            if shape is None:
+                continue
+            if grads.get(name) is None:
+                raise ValueError(f"grads[{name!r}] is missing")
+            _need(f"grads[{name!r}]", grads[name], dv, torch.float32, shape)
     cfg = make_cfg(B, H, L, d, c_q, c_k, c_h, kq_place, head_place, _dtype_code(q), path, scale,
                    q.stride(1), _stream_handle(stream), kq_post=kq_post)
     if ws is None:
         ws = workspace(lib().mta_attn_bwd_workspace_bytes(ctypes.byref(cfg)), q.device)
-    cfg.workspace, cfg.workspace_bytes = ws.data_ptr(), ws.numel()
+    cfg.workspace, cfg.workspace_bytes = ws.data_ptr(), _nbytes(ws)
     _check("mta_attn_bwd", lib().mta_attn_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(theta), _ptr(w),
                                              _ptr(dout), ctypes.byref(cfg), _ptr(grads["dq"]),
                                              _ptr(grads["dk"]), _ptr(grads["dv"]),
@@ -274,7 +323,20 @@ def layer_fwd(x, wqkv, theta, w, gamma, beta, wo, H, c_q, c_k, c_h, kq_place=PRE
     Returns out [B, L, D] bf16."""
     import torch
     B, L, D = x.shape
+    if D % H:
+        raise ValueError(f"D = {D} is not a multiple of H = {H}")
     d = D // H
+    dv = x.device
+    _need("x", x, dv)
+    _need("wqkv", wqkv, dv, x.dtype, (3 * D, D))
+    _need("wo", wo, dv, x.dtype, (D, D))
+    for name, t in (("theta", theta), ("w", w), ("theta_post", theta_post)):
+        _need(name, t, dv, torch.float32)
+    _need("gamma", gamma, dv, torch.float32, (D,))
+    _need("beta", beta, dv, torch.float32, (D,))
+    _need("gate", gate, dv, torch.float32, (H,))
+    _need("out", out, dv, x.dtype, (B, L, D))
+    _need("ws", ws, dv)
     if out is None:
         out = torch.empty((B, L, D), dtype=x.dtype, device=x.device)
     theta, kq_post = _kernels(theta, theta_post, kq_place)
@@ -282,7 +344,7 @@ def layer_fwd(x, wqkv, theta, w, gamma, beta, wo, H, c_q, c_k, c_h, kq_place=PRE
                    _stream_handle(stream), kq_post=kq_post)
     if ws is None:
         ws = workspace(lib().mta_layer_workspace_bytes(ctypes.byref(cfg)), x.device)
-    cfg.workspace, cfg.workspace_bytes = ws.data_ptr(), ws.numel()
+    cfg.workspace, cfg.workspace_bytes = ws.data_ptr(), _nbytes(ws)
     gn = MtaGn(gamma.data_ptr(), beta.data_ptr(), eps, layer, lam,
                gate.data_ptr() if gate is not None else None)
     _check("mta_layer_fwd", lib().mta_layer_fwd(_ptr(x), _ptr(wqkv), _ptr(theta), _ptr(w),
@@ -304,6 +366,9 @@ def gemm_bf16_nt(a, b, out=None, stream=None):
     import torch
     M, K = a.shape
     N = b.shape[0]
+    _need("a", a, a.device, torch.bfloat16)
+    _need("b", b, a.device, torch.bfloat16, (N, K))
+    _need("out", out, a.device, torch.bfloat16, (M, N))
     if out is None:
         out = torch.empty((M, N), dtype=torch.bfloat16, device=a.device)
     _check("mta_gemm_bf16_nt", lib().mta_gemm_bf16_nt(_ptr(a), _ptr(b), _ptr(out), M, N, K,
@@ -316,6 +381,13 @@ def group_norm_scale(o, gamma, beta, eps=1e-5, lam=1.0, out=None, stream=None, g
     import torch
     H, d = o.shape[-2], o.shape[-1]
     tokens = o.numel() // (H * d)
+    _need("o", o, o.device, torch.bfloat16)
+    for name, t in (("gamma", gamma), ("beta", beta)):
+        _need(name, t, o.device, torch.float32)
+        if t.numel() != H * d:
+            raise ValueError(f"{name} must hold H*d = {H * d} values, not {t.numel()}")
+    _need("gate", gate, o.device, torch.float32, (H,))
+    _need("out", out, o.device, torch.bfloat16, tuple(o.shape))
     if out is None:
         out = torch.empty_like(o)
     gn = MtaGn(gamma.data_ptr(), beta.data_ptr(), eps, 0, lam,
