@@ -236,3 +236,18 @@ def test_binding_rejects_host_tensors():
         mta.gemm_bf16_nt(bf(16, 8), bf(4, 8))
     with pytest.raises(ValueError, match="CUDA tensor"):
         mta.group_norm_scale(q, f32(H * d), f32(H * d))
+
+
+def test_plain_c_caller(L, tmp_path):
+    """include/mta.h is plain C99: a C program that includes only the header
+    compiles warning-free against it, links libmta.so and gets the documented
+    status codes from the host-side checks (tests/abi_host.c)."""
+    exe = tmp_path / "abi_host"
+    lib_dir = os.path.dirname(mta.LIB_PATH)
+    cc = subprocess.run(["gcc", "-std=c99", "-pedantic", "-Wall", "-Wextra", "-Werror",
+                         "-I", os.path.join(ROOT, "include"), os.path.join(ROOT, "tests", "abi_host.c"),
+                         "-o", str(exe), mta.LIB_PATH, f"-Wl,-rpath,{lib_dir}"],
+                        capture_output=True, text=True, timeout=120)
+    assert cc.returncode == 0, cc.stderr
+    run = subprocess.run([str(exe)], capture_output=True, text=True, timeout=60)
+    assert run.returncode == 0 and run.stdout.strip() == "ok", run.stdout + run.stderr
