@@ -146,6 +146,16 @@ mta_status mta_attn_fwd(const void *q, const void *k, const void *v,
                         const float *theta_kq, const float *w_head,
                         const mta_cfg *cfg, void *out);
 
+/* The attention kernel mta_attn_fwd would run for cfg, decided on the host
+ * without enqueuing anything or calling CUDA: 1 = the CUDA-core kernel, 2 = the
+ * direct tensor-core kernel, 3 = the contraction kernel (after its prepasses).
+ * cfg->workspace_bytes counts as for mta_attn_fwd (the contraction kernel needs
+ * its operands there); cfg->workspace is not read, and the tensors are taken to
+ * be 16-byte aligned.  Returns -s for the status s the call would return
+ * instead of launching (-MTA_ERR_INVALID, -MTA_ERR_UNSUPPORTED or
+ * -MTA_ERR_WORKSPACE). */
+int mta_attn_kernel(const mta_cfg *cfg);
+
 /* Bytes of workspace mta_layer_fwd uses for cfg (0 if cfg is invalid): the
  * error word, QKV, the attention output and the normalised output (all bf16),
  * plus the contraction kernel's operands where it applies (as for

@@ -251,3 +251,79 @@ def test_plain_c_caller(L, tmp_path):
     assert cc.returncode == 0, cc.stderr
     run = subprocess.run([str(exe)], capture_output=True, text=True, timeout=60)
     assert run.returncode == 0 and run.stdout.strip() == "ok", run.stdout + run.stderr
+
+
+# ---------------------------------------------------------------------------
+# kernel selection, asked of the library on the host (mta_attn_kernel)
+# ---------------------------------------------------------------------------
+
+def _cfg_for(wl, ws_bytes=None, path=mta.PATH_AUTO):
+    d = wl.D // wl.H if wl.layer else wl.d
+    cfg = mta.make_cfg(wl.B, wl.H, wl.L, d, wl.c_q, wl.c_k, wl.c_h, wl.kq_place, wl.head_place,
+                       mta.F32 if wl.dtype == "f32" else mta.BF16, path=path, kq_post=int(wl.kq_post))
+    cfg.workspace_bytes = mta.lib().mta_attn_workspace_bytes(ctypes.byref(cfg)) if ws_bytes is None else ws_bytes
+    return cfg
+
+
+def test_kernel_choice_matches_the_bench_launch_count(L):
+    """bench.py counts the kernels a step launches from its own reading of the
+    selection rules; the library's own choice (with the workspace the bench
+    gives it) must agree for every workload."""
+    import bench
+    from token_attention_b200 import synth
+    for name, wl in synth.WORKLOADS.items():
+        want = mta.PATH_KQ if bench.uses_contraction(wl) else mta.PATH_TC if bench.uses_direct_tc(wl) \
+            else mta.PATH_SIMT
+        assert mta.attn_kernel(_cfg_for(wl)) == want, name
+
+
+def test_kernel_choice_rules(L):
+    from token_attention_b200 import synth
+    wl = synth.WORKLOADS["pretrain_d128_L2048"]
+    assert mta.attn_kernel(_cfg_for(wl)) == mta.PATH_KQ
+    # without room for the convolved keys, path 0 takes the direct tensor-core kernel,
+    # and a forced contraction kernel reports the workspace
+    assert mta.attn_kernel(_cfg_for(wl, ws_bytes=256)) == mta.PATH_TC
+    with pytest.raises(mta.MtaError) as e:
+        mta.attn_kernel(_cfg_for(wl, ws_bytes=256, path=mta.PATH_KQ))
+    assert e.value.code == 3
+    assert mta.attn_kernel(_cfg_for(wl, path=mta.PATH_SIMT)) == mta.PATH_SIMT
+    assert mta.attn_kernel(_cfg_for(wl, path=mta.PATH_TC)) == mta.PATH_TC
+    # fp32 has only the CUDA-core kernel
+    tiny = synth.WORKLOADS["tiny_f32_L256"]
+    for path, code in ((mta.PATH_TC, 2), (mta.PATH_KQ, 2)):
+        with pytest.raises(mta.MtaError) as e:
+            mta.attn_kernel(_cfg_for(tiny, path=path))
+        assert e.value.code == code
+    # the post-softmax convolution: contraction kernel or CUDA-core kernel, never the direct form
+    both = synth.WORKLOADS["both_d128_L2048"]
+    assert mta.attn_kernel(_cfg_for(both, ws_bytes=256)) == mta.PATH_SIMT
+    with pytest.raises(mta.MtaError) as e:
+        mta.attn_kernel(_cfg_for(both, path=mta.PATH_TC))
+    assert e.value.code == 2
+    # an invalid configuration, and a workspace too small for the error word
+    bad = _cfg_for(wl)
+    bad.c_k = 4
+    with pytest.raises(mta.MtaError) as e:
+        mta.attn_kernel(bad)
+    assert e.value.code == 1
+    with pytest.raises(mta.MtaError) as e:
+        mta.attn_kernel(_cfg_for(wl, ws_bytes=64))
+    assert e.value.code == 3
+
+
+@pytest.mark.parametrize("B,H,L_,d,cq,ck,ch,kq,hp,dt,post", [
+    (1, 16, 300, 128, 8, 15, 16, mta.PRE, mta.POST, mta.F32, 1),
+    (1, 16, 300, 128, 8, 15, 16, mta.PRE_EXACT, mta.PRE, mta.BF16, 1),
+    (1, 16, 300, 16, 1, 1, 1, mta.OFF, mta.OFF, mta.F32, 0),
+    (65535, 1, 1, 16, 1, 1, 1, mta.OFF, mta.OFF, mta.BF16, 0),
+])
+def test_extreme_documented_shapes_have_a_kernel(L, B, H, L_, d, cq, ck, ch, kq, hp, dt, post):
+    """The ends of the ranges the header documents (c_q = 8, c_k = 15, c_h = 16,
+    d = 16 and 128, B = 65535, both convolutions) are not refused: the library
+    selects a kernel for them (the CUDA-core kernel with fewer rows per CTA).
+    This checks the host's choice only; these shapes are not among the GPU
+    parity cases."""
+    cfg = mta.make_cfg(B, H, L_, d, cq, ck, ch, kq, hp, dt, kq_post=post)
+    cfg.workspace_bytes = L.mta_attn_workspace_bytes(ctypes.byref(cfg))
+    assert mta.attn_kernel(cfg) == mta.PATH_SIMT

@@ -224,6 +224,18 @@ mta_status mta_attn_fwd(const void *q, const void *k, const void *v, const float
   return e == cudaSuccess ? MTA_OK : MTA_ERR_CUDA;
 }
 
+int mta_attn_kernel(const mta_cfg *cfg) {
+  mta_status s = check_cfg(cfg);
+  if (s != MTA_OK) return -static_cast<int>(s);
+  if (cfg->workspace_bytes < kStatusBytes) return -static_cast<int>(MTA_ERR_WORKSPACE);
+  // no tensor is read: null pointers stand for 16-byte aligned ones
+  const AttnArgs a = make_args(nullptr, nullptr, nullptr, nullptr, nullptr, cfg, nullptr);
+  Kernel kern = K_SIMT;
+  if ((s = select_kernel(a, cfg->path, cfg->workspace_bytes - kStatusBytes, &kern)) != MTA_OK)
+    return -static_cast<int>(s);
+  return static_cast<int>(kern);
+}
+
 size_t mta_layer_workspace_bytes(const mta_cfg *cfg) {
   const size_t base = layer_base_workspace_bytes(cfg);
   return base ? base + kq_bytes(cfg) : 0;

@@ -27,7 +27,7 @@ STATUS = {0: "MTA_OK", 1: "MTA_ERR_INVALID", 2: "MTA_ERR_UNSUPPORTED", 3: "MTA_E
 EXPORTS = ["mta_attn_workspace_bytes", "mta_attn_fwd", "mta_layer_workspace_bytes",
            "mta_layer_fwd", "mta_gemm_bf16_nt", "mta_group_norm_scale", "mta_sync_status",
            "mta_status_string", "mta_abi_version", "mta_layer_fwd_static",
-           "mta_attn_bwd_workspace_bytes", "mta_attn_bwd"]
+           "mta_attn_bwd_workspace_bytes", "mta_attn_bwd", "mta_attn_kernel"]
 
 
 class MtaCfg(ctypes.Structure):
@@ -79,6 +79,8 @@ def lib() -> ctypes.CDLL:
         L.mta_attn_bwd_workspace_bytes.restype = S
         L.mta_attn_bwd.argtypes = [P, P, P, P, P, P, cfgp, P, P, P, P, P]
         L.mta_attn_bwd.restype = I
+        L.mta_attn_kernel.argtypes = [cfgp]
+        L.mta_attn_kernel.restype = I
         L.mta_sync_status.argtypes = [cfgp]
         L.mta_sync_status.restype = I
         L.mta_status_string.argtypes = [I]
@@ -177,6 +179,19 @@ def _kernels(theta, theta_post, kq_place):
             raise ValueError("a stacked theta holds the pre-softmax kernels (if on), then the post-softmax ones")
         return theta, 1
     return theta, 0
+
+
+KERNEL_NAMES = {PATH_SIMT: "attn_simt_kernel", PATH_TC: "attn_tc_kernel", PATH_KQ: "attn_kq_kernel"}
+
+
+def attn_kernel(cfg: MtaCfg) -> int:
+    """The kernel mta_attn_fwd picks for cfg (PATH_SIMT, PATH_TC or PATH_KQ), asked
+    of the library on the host; raises MtaError with the status the call would
+    return instead of launching."""
+    r = lib().mta_attn_kernel(ctypes.byref(cfg))
+    if r < 0:
+        raise MtaError("mta_attn_kernel", -r)
+    return r
 
 
 def attn_fwd(q, k, v, theta, w, c_q, c_k, c_h, kq_place=PRE, head_place=POST, *, out=None,
