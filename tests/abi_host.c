@@ -50,6 +50,14 @@ int main(void) {
   EXPECT(mta_layer_workspace_bytes(&c) > ws);
   EXPECT(mta_attn_bwd_workspace_bytes(&c) == 256);
 
+  /* kernel choice on the host: the contraction kernel once its operands fit */
+  EXPECT(mta_attn_kernel(&c) == -MTA_ERR_WORKSPACE);
+  c.workspace_bytes = ws;
+  EXPECT(mta_attn_kernel(&c) == 3);
+  c.workspace_bytes = 256;
+  EXPECT(mta_attn_kernel(&c) == 2);
+  c = recipe();
+
   /* invalid configurations: no workspace size, MTA_ERR_INVALID from the call */
   bad = c; bad.c_k = 4;
   EXPECT(mta_attn_workspace_bytes(&bad) == 0);
