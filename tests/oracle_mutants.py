@@ -7,8 +7,9 @@ of tests/test_oracle_pins.py run.  Every variant is a plausible slip in
 writing the method down: a dropped tap, a flipped key or query offset, a
 transposed mixing matrix, a mask off by one, a wrong scale, a missing re-mask,
 mixing with the source heads' values instead of the destination head's, the
-unbiased variance in the norm, and wrong adjoints in the backward pass.  The
-mistakes live in the CPU oracle only; nothing here touches the CUDA library.
+unbiased variance in the norm, a strict exact indicator, the gate's sign, and
+wrong adjoints in the backward pass.  The mistakes live in the CPU oracle only;
+nothing here touches the CUDA library.
 """
 import os
 
@@ -20,7 +21,8 @@ import oracle.mta_oracle as M
 _ORIG = {n: getattr(M, n) for n in (
     "attention_logits", "mask_zero", "mask_neg_inf", "key_query_conv", "head_mix",
     "post_softmax_conv", "mta_attention_group", "group_norm_scale",
-    "key_query_conv_adjoint", "key_query_conv_grad_theta")}
+    "key_query_conv_adjoint", "key_query_conv_grad_theta", "key_query_conv_exact",
+    "sigmoid_gate")}
 
 
 def _drop_tap(m, theta):
@@ -99,6 +101,17 @@ def _grad_theta_flipped(g, m, cq, ck):
     return _ORIG["key_query_conv_grad_theta"](g, m, cq, ck)[:, :, ::-1]
 
 
+def _exact_strict(a_hat, theta, qpos):
+    """The exact indicator with a strict inequality: a tap may not read the
+    output query's own key."""
+    return _ORIG["key_query_conv_exact"](a_hat, theta, np.asarray(qpos) - 1)
+
+
+def _gate_sign(gate):
+    """The scalar gate with the wrong sign inside the sigmoid."""
+    return _ORIG["sigmoid_gate"](-np.asarray(gate, np.float64))
+
+
 MUTANTS = {
     "drop_tap": ("key_query_conv", _drop_tap),
     "flip_key_offset": ("key_query_conv", _flip_key),
@@ -113,6 +126,8 @@ MUTANTS = {
     "unbiased_variance": ("group_norm_scale", _unbiased_variance),
     "adjoint_flipped": ("key_query_conv_adjoint", _adjoint_flipped),
     "grad_theta_flipped": ("key_query_conv_grad_theta", _grad_theta_flipped),
+    "exact_indicator_strict": ("key_query_conv_exact", _exact_strict),
+    "gate_sign": ("sigmoid_gate", _gate_sign),
 }
 
 
