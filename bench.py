@@ -221,7 +221,10 @@ class ClockSampler:
 # the library arm
 # ---------------------------------------------------------------------------
 
-def make_sets(wl, dev, n_sets, bwd=False):
+def make_sets(wl, dev, n_sets, bwd=False, rank=0):
+    """n_sets input sets of the workload.  Under N ranks each rank draws its own
+    batches (a seed offset per rank): the ranks process different units of the
+    same shape, with no exchange between them."""
     import torch
 
     def to(x, dt):
@@ -230,7 +233,7 @@ def make_sets(wl, dev, n_sets, bwd=False):
 
     sets = []
     for s in range(n_sets):
-        w = synth.shrink(wl, seed=wl.seed + 100 * s)
+        w = synth.shrink(wl, seed=wl.seed + 100 * s + 100_000 * rank)
         if wl.layer:
             inp = synth.make_layer_inputs(w)
             keys = ("x", "wqkv", "wo", "theta", "w", "gamma", "beta")
@@ -280,7 +283,7 @@ def run_mine(args, wl, rank, world, local_rank):
     dev = torch.device("cuda", local_rank)
     mta.lib()
     stream = torch.cuda.Stream(device=dev)
-    sets = make_sets(wl, dev, N_SETS, args.bwd)
+    sets = make_sets(wl, dev, N_SETS, args.bwd, rank)
     out_shape = (wl.B, wl.L, wl.D) if wl.layer else (wl.B, wl.L, wl.H, wl.d)
     odt = torch.float32 if wl.dtype == "f32" else torch.bfloat16
     if args.bwd:  # fp32 gradients of q, k, v, the kernels and the mixing weights

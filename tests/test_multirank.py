@@ -84,3 +84,17 @@ def test_reference_arm_line_on_rank0():
     assert cb["kind"] == "oracle" and cb["cores"] >= 1 and cb["value"] == line["value"] and cb["sample"]
     assert line["e2e"] == {"value": line["value"], "unit": "tokens/s",
                            "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}
+
+
+def test_ranks_draw_their_own_batches():
+    """Weak scaling over replicas: every rank times the same shape on its own
+    inputs; rank 0 keeps the single-GPU inputs."""
+    import torch
+    from token_attention_b200 import synth
+    wl = synth.WORKLOADS["tiny_f32_L256"]
+    r0 = bench.make_sets(wl, "cpu", 2, rank=0)
+    r1 = bench.make_sets(wl, "cpu", 2, rank=1)
+    single = synth.make_attn_inputs(synth.shrink(wl, seed=wl.seed))
+    assert torch.equal(r0[0]["q"], torch.from_numpy(single["q"]))
+    assert not torch.equal(r0[0]["q"], r0[1]["q"])
+    assert not torch.equal(r0[0]["q"], r1[0]["q"]) and r0[0]["q"].shape == r1[0]["q"].shape
