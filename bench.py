@@ -140,15 +140,46 @@ def read_peaks() -> tuple[dict, str]:
     return dict(FALLBACK_PEAKS), "fallback"
 
 
+# source files each kernel's code comes from (a committed traffic figure counts only
+# while these files are unchanged since its capture)
+KERNEL_SOURCES = {
+    "attn_kq_kernel": ("attn_kq.cu", "ptx.cuh"),
+    "kq_prep_kernel": ("kq_prep.cu",),
+    "vt_prep_kernel": ("kq_prep.cu",),
+    "attn_tc_kernel": ("attn_tc.cu", "ptx.cuh"),
+    "attn_simt_kernel": ("attn_simt.cu",),
+    "attn_bwd_simt_kernel": ("attn_bwd_simt.cu", "bwd_common.cuh"),
+    "attn_bwd_post_kernel": ("attn_bwd_post_simt.cu", "bwd_common.cuh"),
+    "group_norm_d128_kernel": ("group_norm.cu",),
+    "gemm_bf16_nt_kernel": ("gemm_tc.cu", "ptx.cuh"),
+}
+
+
+def source_sha(kernel_key: str) -> str | None:
+    """sha1 (16 hex digits) over the source files of a kernel, as committed."""
+    import hashlib
+    files = KERNEL_SOURCES.get(kernel_key)
+    if not files:
+        return None
+    h = hashlib.sha1()
+    for f in files:
+        with open(os.path.join(ROOT, "token_attention_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
 def read_traffic(kernel_key: str, workload: str):
-    """dram bytes per launch from a committed ncu summary, if one matches."""
+    """dram bytes per launch from a committed ncu summary, if one matches this
+    workload and was taken from the kernel's current source (else None)."""
     p = os.path.join(ROOT, "profiles", "traffic.json")
     if not os.path.exists(p):
         return None
     with open(p) as f:
         t = json.load(f)
     e = t.get(kernel_key, {}).get(workload)
-    return None if e is None else e.get("bytes_per_launch")
+    if e is None or e.get("source_sha") != source_sha(kernel_key):
+        return None
+    return e.get("bytes_per_launch")
 
 
 def call_traffic(kernel_keys, workload: str):
@@ -252,26 +283,82 @@ def make_sets(wl, dev, n_sets, bwd=False, rank=0):
 
 
 def step_fn(wl, mta, sets, ws, outs, stream, bwd=False):
-    """Returns f(i): enqueue step i (input set i % n) on `stream`."""
+    """Returns f(i, events=None): enqueue step i (input set i % n) on `stream`;
+    the library records `events` around the step's kernels (mta_cfg.events)."""
     if bwd:
-        def f(i):
+        def f(i, events=None):
             s = sets[i % len(sets)]
             mta.attn_bwd(s["q"], s["k"], s["v"], s["theta"], s["w"], s["dout"], wl.c_q, wl.c_k, wl.c_h,
-                         wl.kq_place, wl.head_place, ws=ws, stream=stream, grads=outs[i % len(outs)])
+                         wl.kq_place, wl.head_place, ws=ws, stream=stream, grads=outs[i % len(outs)],
+                         events=events)
     elif wl.layer:
-        def f(i):
+        def f(i, events=None):
             s = sets[i % len(sets)]
             mta.layer_fwd(s["x"], s["wqkv"], s["theta"], s["w"], s["gamma"], s["beta"], s["wo"],
                           wl.H, wl.c_q, wl.c_k, wl.c_h, wl.kq_place, wl.head_place, eps=1e-5,
                           layer=wl.depth, out=outs[i % len(outs)], ws=ws, stream=stream,
-                          theta_post=s["theta_post"])
+                          theta_post=s["theta_post"], events=events)
     else:
-        def f(i):
+        def f(i, events=None):
             s = sets[i % len(sets)]
             mta.attn_fwd(s["q"], s["k"], s["v"], s["theta"], s["w"], wl.c_q, wl.c_k, wl.c_h,
                          wl.kq_place, wl.head_place, out=outs[i % len(outs)], ws=ws, stream=stream,
-                         theta_post=s["theta_post"])
+                         theta_post=s["theta_post"], events=events)
     return f
+
+
+def dominant_kernel(wl: synth.Workload, bwd: bool) -> tuple[int, int, str]:
+    """(a, b, name): the step's dominant kernel runs between the library's timing
+    events a and b of a step (event 0 before the first kernel, event k after the
+    k-th; see mta_cfg.events), and its name."""
+    if bwd:
+        return 0, 1, "attn_bwd_post_kernel" if wl.kq_post else "attn_bwd_simt_kernel"
+    n = launches_per_step(wl) + 1
+    if uses_contraction(wl):
+        # ... key prepass, (value prepass), attention kernel, (output GEMM)
+        return (n - 3, n - 2, "attn_kq_kernel") if wl.layer else (n - 2, n - 1, "attn_kq_kernel")
+    name = "attn_tc_kernel" if uses_direct_tc(wl) else "attn_simt_kernel"
+    return (1, 2, name) if wl.layer else (0, 1, name)
+
+
+def choose_peak(peaks: dict, region_ms: float, clocks) -> tuple[float, str]:
+    """The bf16 denominator for the timed region: the sustained figure only for a
+    region of a second or more that ran under the power cap, else the burst one."""
+    capped = bool(clocks) and "sw_power_cap" in clocks.get("reasons", [])
+    if region_ms >= 1000.0 and capped:
+        return peaks["bf16_tflops_sustained"], f"sustained (timed region {region_ms:.0f} ms under sw_power_cap)"
+    why = "no power cap" if not capped else "region shorter than 1 s"
+    return peaks["bf16_tflops"], f"burst (timed region {region_ms:.1f} ms, {why})"
+
+
+def run_epilogue(mta, dev, stream, launches=20):
+    """The group norm with depth scale as its own kernel (mta_group_norm_scale) on the
+    full layer's Y: 8192 tokens x 16 heads x 128 channels bf16 (B*L = 2*4096,
+    D = 2048).  Four input/output pairs rotate (4 x 67 MB, above the 126 MB L2), so
+    that no launch reads data the previous one left in L2.  Returns achieved
+    HBM GB/s on the algorithmic bytes (2 B read + 2 B written per element)."""
+    import torch
+    T, H, d = 8192, 16, 128
+    g = torch.Generator(device="cpu").manual_seed(5)
+    xs = [torch.randn((T, H, d), generator=g).to(torch.bfloat16).to(dev) for _ in range(4)]
+    ys = [torch.empty_like(xs[0]) for _ in range(4)]
+    gamma = (1 + 0.1 * torch.randn(H * d, generator=g)).to(dev)
+    beta = (0.1 * torch.randn(H * d, generator=g)).to(dev)
+    for i in range(3):
+        mta.group_norm_scale(xs[i % 4], gamma, beta, 1e-5, 0.978141, out=ys[i % 4], stream=stream)
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(launches)]
+    torch.cuda.synchronize()
+    with torch.cuda.stream(stream):
+        for i in range(launches):
+            ev[i][0].record(stream)
+            mta.group_norm_scale(xs[i % 4], gamma, beta, 1e-5, 0.978141, out=ys[i % 4], stream=stream)
+            ev[i][1].record(stream)
+    stream.synchronize()
+    ms = statistics.mean(a.elapsed_time(b) for a, b in ev)
+    nbytes = 2 * T * H * d * 2
+    return {"kernel": "group_norm_d128_kernel", "workload": "Y of layer_*_D2048_L4096: 8192 x 16 x 128 bf16",
+            "bytes_per_launch": nbytes, "ms_per_launch": ms, "achieved_gbs": nbytes / (ms / 1e3) / 1e9,
+            "launches": launches, "l2": "4 rotating input/output pairs (268 MB)"}
 
 
 def run_mine(args, wl, rank, world, local_rank):
@@ -327,8 +414,15 @@ def run_mine(args, wl, rank, world, local_rank):
     if st != 0:
         raise RuntimeError(f"warm-up status {mta.STATUS.get(st, st)}")
 
-    starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
-    ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    # the library records n_ev events per step around its kernels (mta_cfg.events);
+    # each is recorded once here first, so that torch has created it
+    n_ev = (1 if args.bwd else launches_per_step(wl)) + 1
+    step_ev = [[torch.cuda.Event(enable_timing=True) for _ in range(n_ev)] for _ in range(args.steps)]
+    with torch.cuda.stream(stream):
+        for evs in step_ev:
+            for e in evs:
+                e.record(stream)
+    stream.synchronize()
     barrier()
     torch.cuda.synchronize()
     if sampler:
@@ -338,9 +432,7 @@ def run_mine(args, wl, rank, world, local_rank):
     with torch.cuda.stream(stream):
         t_begin.record(stream)
         for i in range(args.steps):
-            starts[i].record(stream)
-            f(warm + i)
-            ends[i].record(stream)
+            f(warm + i, step_ev[i])
         t_end.record(stream)
     stream.synchronize()
     barrier()
@@ -348,7 +440,9 @@ def run_mine(args, wl, rank, world, local_rank):
     if sampler:
         sampler.mark_end()
     total_ms = t_begin.elapsed_time(t_end)
-    per_launch = [s.elapsed_time(e) for s, e in zip(starts, ends)]
+    ka, kb, kname = dominant_kernel(wl, args.bwd)
+    kernel_ms = [evs[ka].elapsed_time(evs[kb]) for evs in step_ev]
+    step_ms = [evs[0].elapsed_time(evs[-1]) for evs in step_ev]
     st = mta.lib().mta_sync_status(ctypes.byref(cfg))
     if st != 0:
         raise RuntimeError(f"timed-region status {mta.STATUS.get(st, st)}")
@@ -359,8 +453,12 @@ def run_mine(args, wl, rank, world, local_rank):
     e2e = None
     if not args.no_e2e and not args.bwd:
         e2e = run_e2e(args, wl, mta, sets, ws, stream, dev, barrier, world)
-    return {"total_ms": t_max, "per_launch_ms": per_launch, "clocks": clocks, "e2e": e2e,
-            "warmup": warm}
+    epi = None
+    if not args.no_epilogue and not args.bwd and rank == 0:
+        epi = run_epilogue(mta, dev, stream)
+    return {"total_ms": t_max, "region_ms": total_ms, "kernel_ms": statistics.mean(kernel_ms),
+            "kernel": kname, "kernel_calls_ms": statistics.mean(step_ms), "clocks": clocks, "e2e": e2e,
+            "warmup": warm, "epilogue": epi}
 
 
 def run_e2e(args, wl, mta, sets, ws, stream, dev, barrier, world):
@@ -461,7 +559,7 @@ def oracle_sample(wl, budget_s: float, mode: str):
         rows = [(0, 0)]
         t = time.perf_counter()
         O.mta_layer_rows(inp["x"][:1], inp["wqkv"], inp["theta"], inp["w"], inp["gamma"],
-                         inp["beta"], inp["eps"], inp["lam"], inp["wo"], wl.H, wl.c_h, rows,
+                         inp["beta"], inp["eps"], O.depth_scale(wl.depth), inp["wo"], wl.H, wl.c_h, rows,
                          wl.kq_place, wl.head_place, theta_post=inp["theta_post"])
         dt = time.perf_counter() - t
         return 1 / dt, dt, "1 token of the layer (QKV of its batch, attention window, norm, projection)"
@@ -558,6 +656,8 @@ def main():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu", action="store_true")
     ap.add_argument("--no-clocks", action="store_true")
+    ap.add_argument("--no-epilogue", action="store_true",
+                    help="skip the stand-alone group-norm bandwidth measurement")
     ap.add_argument("--bwd", action="store_true",
                     help="time the backward pass (mta_attn_bwd) of an attention workload instead")
     args = ap.parse_args()
@@ -605,73 +705,73 @@ def main():
 
     ms = res["total_ms"]
     value = job_tokens_per_s(world, wl.tokens, args.steps, ms)
-    launch_ms = statistics.mean(res["per_launch_ms"])
     peaks, peak_src = read_peaks()
-    s = launch_ms / 1e3
+    # one time everywhere: the step time is the timed region / steps; the dominant
+    # kernel's time is the mean, over the timed steps, of the library's events around it
+    s = ms / args.steps / 1e3
+    ks = res["kernel_ms"] / 1e3
+    kernel = res["kernel"]
+    bf16_peak, peak_kind = choose_peak(peaks, res["region_ms"], res["clocks"])
+    fp32_src = "148 SMs x 128 FP32 lanes x 2 x 1965 MHz"
+    timing = (f"achieved = per_unit x units / {kernel}'s mean duration over the {args.steps} timed "
+              f"steps (CUDA events the library records around it on the launch stream)")
     if args.bwd:
         # the backward on the CUDA cores: F_bwd = 8d + 4 c_q c_k + 4 c_h fp32 flop per causal
         # pair-head (dS, dQ, dK, dV products; the convolution's adjoint and kernel gradient;
         # the mixing adjoints)
-        kernel = "attn_bwd_post_kernel" if wl.kq_post else "attn_bwd_simt_kernel"
         n_conv = (1 if wl.kq_place else 0) + (1 if wl.kq_post else 0)
         f_bwd = (8 * wl.d + 4 * wl.c_q * wl.c_k * n_conv + (4 * wl.c_h if wl.head_place else 0)) \
             * wl.causal_pairs
-        achieved = f_bwd / s / 1e12
+        achieved = f_bwd / ks / 1e12
         roof = {"bound": "alu", "achieved": achieved, "peak": FP32_PEAK_TFLOPS, "unit": "TFLOP/s",
                 "frac": achieved / FP32_PEAK_TFLOPS, "traffic": read_traffic(kernel, wl.name),
-                "kernel": kernel,
+                "kernel": kernel, "kernel_ms": ks * 1e3,
                 "per_unit": f"F_bwd = 8d + 4 c_q c_k (per convolution) + 4 c_h = {f_bwd // wl.causal_pairs} fp32 flop per "
                             f"causal pair-head, x {wl.causal_pairs} pair-heads per launch",
-                "peak_source": "148 SMs x 128 FP32 lanes x 2 x 1965 MHz"}
-    elif wl.layer:
-        kernel = "mta_layer_fwd"
-        achieved = fl["mta"] / s / 1e12
-        roof = {"bound": "tensor", "achieved": achieved, "peak": peaks["bf16_tflops"],
-                "unit": "TFLOP/s", "frac": achieved / peaks["bf16_tflops"],
-                "traffic": read_traffic("layer", wl.name),
-                "kernel": "layer step (QKV GEMM + fused attention + output GEMM)",
-                "per_unit": "F_mta per causal pair-head + 8 B L D^2 GEMM flops",
-                "peak_source": f"{peak_src} bf16 burst"}
+                "peak_source": fp32_src, "timing": timing}
     elif uses_contraction(wl):
-        # the attention call: kq_prep_kernel + attn_kq_kernel (the dominant one);
-        # algorithmic flops F_mta per causal pair-head against the bf16 tensor peak
-        # sustained under the power cap (the timed loop runs for about a second)
-        kernel = "attn_kq_kernel"
-        peak = peaks["bf16_tflops_sustained"]
-        achieved = fl["attn_mta"] / s / 1e12
-        executed = contraction_tensor_flops(wl) / s / 1e12
-        roof = {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
-                "frac": achieved / peak,
-                "traffic": call_traffic(("kq_prep_kernel",) + (("vt_prep_kernel",) if wl.kq_post else ())
-                                        + ("attn_kq_kernel",), wl.name),
-                "kernel": "mta_attn_fwd call = kq_prep_kernel + " + ("vt_prep_kernel + " if wl.kq_post else "")
-                          + "attn_kq_kernel",
+        # the dominant kernel is attn_kq_kernel (after its prepass, inside the layer between
+        # the two projection GEMMs): algorithmic flops F_mta per causal pair-head
+        achieved = fl["attn_mta"] / ks / 1e12
+        executed = contraction_tensor_flops(wl) / ks / 1e12
+        roof = {"bound": "tensor", "achieved": achieved, "peak": bf16_peak, "unit": "TFLOP/s",
+                "frac": achieved / bf16_peak, "traffic": read_traffic(kernel, wl.name),
+                "kernel": kernel, "kernel_ms": ks * 1e3,
                 "per_unit": f"F_mta = 4d + 2 c_q c_k{' x 2' if wl.kq_post else ''} + 2 c_h = "
                             f"{fl['attn_mta'] // wl.causal_pairs} flop "
                             f"per causal pair-head, x {wl.causal_pairs} pair-heads per launch",
-                "executed_tensor_tflops": executed, "executed_frac": executed / peak,
-                "peak_source": f"{peak_src} bf16 sustained"}
+                "executed_tensor_tflops": executed, "executed_frac": executed / bf16_peak,
+                "executed_note": "MMA work the kernel issues (the contraction of length c_q*d, P V for "
+                                 "the heads held): a design figure, not the roofline",
+                "peak_source": f"{peak_src} bf16 {peak_kind}", "timing": timing}
     elif not uses_direct_tc(wl):
         # the CUDA-core kernel: every step in fp32 FMA on the CUDA cores
-        kernel = "attn_simt_kernel"
-        achieved = fl["attn_mta"] / s / 1e12
+        achieved = fl["attn_mta"] / ks / 1e12
         roof = {"bound": "alu", "achieved": achieved, "peak": FP32_PEAK_TFLOPS, "unit": "TFLOP/s",
-                "frac": achieved / FP32_PEAK_TFLOPS,
-                "traffic": read_traffic("attn_simt_kernel", wl.name),
-                "kernel": kernel,
+                "frac": achieved / FP32_PEAK_TFLOPS, "traffic": read_traffic(kernel, wl.name),
+                "kernel": kernel, "kernel_ms": ks * 1e3,
                 "per_unit": f"F_mta = {fl['attn_mta'] // wl.causal_pairs} fp32 flop per causal "
                             f"pair-head (both convolutions), x {wl.causal_pairs} pair-heads per launch",
-                "peak_source": "148 SMs x 128 FP32 lanes x 2 x 1965 MHz"}
+                "peak_source": fp32_src, "timing": timing}
     else:
-        kernel = "attn_tc_kernel"
-        achieved = fl["conv"] / s / 1e12
+        achieved = fl["conv"] / ks / 1e12
         roof = {"bound": "alu", "achieved": achieved, "peak": FP32_PEAK_TFLOPS, "unit": "TFLOP/s",
-                "frac": achieved / FP32_PEAK_TFLOPS,
-                "traffic": read_traffic("attn_tc_kernel", wl.name),
-                "kernel": kernel,
+                "frac": achieved / FP32_PEAK_TFLOPS, "traffic": read_traffic(kernel, wl.name),
+                "kernel": kernel, "kernel_ms": ks * 1e3,
                 "per_unit": f"2*c_q*c_k = {2 * wl.c_q * wl.c_k} fp32 flop per causal pair-head "
                             f"(key-query convolution), x {wl.causal_pairs} pair-heads per launch",
-                "peak_source": "148 SMs x 128 FP32 lanes x 2 x 1965 MHz"}
+                "peak_source": fp32_src, "timing": timing}
+    # the whole call (every kernel of the step) against the bf16 peak
+    call_f = fl["mta"] if not args.bwd else None
+    roof["call"] = None if args.bwd else {
+        "achieved": call_f / s / 1e12, "frac": call_f / s / 1e12 / bf16_peak, "unit": "TFLOP/s",
+        "ms": s * 1e3, "flops": "F_mta per causal pair-head" + (" + 8 B L D^2 projection GEMM flops" if wl.layer else ""),
+        "peak": bf16_peak, "peak_source": f"{peak_src} bf16 {peak_kind}"}
+    epi = res.get("epilogue")
+    if epi is not None:
+        epi = dict(epi, peak_gbs=peaks["hbm_gbs"], frac=epi["achieved_gbs"] / peaks["hbm_gbs"],
+                   peak_source=f"{peak_src} HBM copy bandwidth",
+                   traffic=read_traffic("group_norm_d128_kernel", "layer_Y_T8192_H16_d128"))
     line = {
         "metric": METRIC_BWD if args.bwd else METRIC, "value": value, "unit": UNIT, "n_gpus": world,
         "steps": args.steps,
@@ -679,17 +779,22 @@ def main():
         "scaling": "weak", "vs_baseline": None, "dtype": "bf16" if wl.dtype == "bf16" else "f32",
         "data": "synthetic", "config": config,
         "tflops": {"std": fl["std"] / s / 1e12, "mta": fl["mta"] / s / 1e12},
-        "pct_bf16_peak": {"std": fl["std"] / s / 1e12 / peaks["bf16_tflops"],
-                          "mta": fl["mta"] / s / 1e12 / peaks["bf16_tflops"],
-                          "peak_tflops": peaks["bf16_tflops"], "peak_source": peak_src},
+        "pct_bf16_peak": {"std": fl["std"] / s / 1e12 / bf16_peak,
+                          "mta": fl["mta"] / s / 1e12 / bf16_peak,
+                          "peak_tflops": bf16_peak, "peak_source": f"{peak_src} bf16 {peak_kind}"},
         "roofline": roof, "gpu_launches": args.steps * (1 if args.bwd else launches_per_step(wl)),
-        "clocks": res["clocks"], "e2e": res["e2e"],
+        "timed_region_ms": res["region_ms"],
+        "clocks": res["clocks"], "e2e": res["e2e"], "epilogue_group_norm": epi,
     }
     if world == 1 and not args.no_cpu:
         mode = "bwd_groups" if args.bwd else "groups" if not wl.layer else "rows"
         v, secs, desc = oracle_sample(wl, args.cpu_budget, mode)
         line["cpu_baseline"] = {"value": v, "unit": UNIT, "cores": blas_threads(), "kind": "oracle",
-                                "sample": f"{desc}; {secs:.1f} s"}
+                                "sample": f"{desc}; {secs:.1f} s",
+                                "note": "the stated CPU baseline: the oracle on whole head groups at full "
+                                        "length, its natural unit (the --impl reference arm samples single "
+                                        "query rows instead, which recomputes every key's logits per row and "
+                                        "so runs several times slower per token)"}
     print(json.dumps(line), flush=True)
     return 0
 

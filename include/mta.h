@@ -38,7 +38,9 @@
  * and enqueues nothing.  A failed launch returns MTA_ERR_CUDA.  Kernels never
  * wait without a bound: a wait that runs out sets a flag in the workspace and
  * the kernel returns; mta_sync_status() reports it as MTA_ERR_TIMEOUT.
- * Outputs must not alias inputs.
+ * Outputs must not alias inputs: an output whose bytes overlap an input's
+ * (q, k, v or dout of the attention; x, Wqkv or Wo of the layer), or another
+ * output's, is refused with MTA_ERR_INVALID.
  */
 #ifndef MTA_H
 #define MTA_H
@@ -49,7 +51,7 @@
 extern "C" {
 #endif
 
-#define MTA_ABI_VERSION 2
+#define MTA_ABI_VERSION 3
 
 typedef enum {
   MTA_OK = 0,
@@ -105,6 +107,22 @@ typedef struct mta_cfg {
   void *stream;          /* cudaStream_t to enqueue on; NULL = legacy default    */
   void *workspace;       /* device scratch, 256-byte aligned                      */
   size_t workspace_bytes;
+  void *const *events;   /* optional timing events (cudaEvent_t handles created by
+                            the caller, 0 .. 64 of them; NULL when n_events = 0):
+                            a call records events[0] on cfg->stream just before
+                            its first kernel and events[k] just after its k-th
+                            kernel, while k < n_events, so that the time of each
+                            kernel of the call can be read with
+                            cudaEventElapsedTime.  The kernels of a call, in
+                            order: mta_attn_fwd, the contraction path: the key
+                            prepass, (with kq_post) the value prepass, the
+                            attention kernel; other paths: the attention kernel.
+                            mta_layer_fwd: the QKV GEMM, the attention kernels
+                            as above (with the norm fused), or, on the CUDA-core
+                            path, the attention kernel and then the stand-alone
+                            group norm; the output GEMM.  mta_attn_bwd: its one
+                            kernel.                                              */
+  int n_events;          /* number of handles in events, 0 .. 64                 */
 } mta_cfg;
 
 /* Scaled group normalisation of head outputs (section 3.3; bycloud item 3):
@@ -188,7 +206,9 @@ mta_status mta_layer_fwd(const void *x, const void *Wqkv, const float *theta,
  * (mta_layer_workspace_bytes(cfg) less the contraction kernel's operands)
  * exceeds MTA_STATIC_SCRATCH_BYTES; the contraction kernel runs where the
  * whole of mta_layer_workspace_bytes(cfg) fits.  The first call on a device looks up the
- * buffer's address on that device (make it before any stream capture).  All
+ * buffer's address on that device (make it before any stream capture) and keeps
+ * it for the life of the process; after cudaDeviceReset on a device that address
+ * is stale, so do not call this entry point on a device after resetting it.  All
  * calls on a device share the buffer: calls that overlap on the GPU race, so
  * order them on one stream.  A bounded wait that runs out is recorded in the
  * static buffer and is not reported; use mta_layer_fwd with a workspace and
@@ -239,6 +259,22 @@ mta_status mta_attn_bwd(const void *q, const void *k, const void *v, const float
  * cfg->workspace gave up a bounded wait (MTA_ERR_TIMEOUT), else MTA_OK or
  * MTA_ERR_CUDA.  Blocking; for tests and diagnostics. */
 mta_status mta_sync_status(const mta_cfg *cfg);
+
+/* Diagnostic of the library's failure reporting (the pages have no counterpart
+ * to it): enqueues on cfg->stream one small kernel whose
+ * mbarrier waits can never complete, with every wait bounded by limit_us
+ * microseconds (1 .. 2,000,000) instead of the library's 2 s.  The kernel gives
+ * up through the same path as the attention kernels: the first wait to run out
+ * sets the error word at the start of cfg->workspace (which the call clears
+ * first) and an abort flag, the other threads' waits then return at once, and
+ * the kernel ends.  mta_sync_status(cfg) then returns MTA_ERR_TIMEOUT, and the
+ * next call on the same workspace starts from a clear error word.  The two
+ * unsigned words after the error word count the threads (128) whose first and
+ * second wait gave up.  Nothing faults and no wait is unbounded.  Returns
+ * MTA_ERR_INVALID for a null cfg or a limit out of range, MTA_ERR_WORKSPACE
+ * without a 256-byte aligned workspace of at least 256 bytes (only
+ * cfg->workspace, cfg->workspace_bytes and cfg->stream are read). */
+mta_status mta_selftest_wait_timeout(const mta_cfg *cfg, unsigned limit_us);
 
 /* Static description of a status code. */
 const char *mta_status_string(mta_status s);

@@ -64,7 +64,7 @@ OFF, PRE, POST, PRE_EXACT = 0, 1, 2, 3
 __all__ = ["OFF", "PRE", "POST", "PRE_EXACT", "attention_logits", "mask_zero", "key_query_conv",
            "key_query_conv_exact", "sigmoid_gate", "post_softmax_conv",
            "head_mix", "mask_neg_inf", "softmax_rows", "mta_attention_group",
-           "mta_attention", "mta_attention_rows", "group_norm_scale", "mta_layer",
+           "mta_attention", "mta_attention_rows", "depth_scale", "group_norm_scale", "mta_layer",
            "key_query_conv_adjoint", "key_query_conv_grad_theta", "mta_attention_group_bwd",
            "mta_attention_bwd",
            "mta_layer_rows"]
@@ -421,6 +421,13 @@ def mta_attention_rows(q, k, v, theta, w, c_h, rows, kq_place=PRE, head_place=PO
                                      None if theta_post is None else theta_post[hs])
             out[n, hs, :] = og[:, -1, :]
     return out
+
+
+def depth_scale(layer: int) -> float:
+    """Depth-dependent multiplier of the normalised head outputs [bycloud, MTA-3.3]:
+    lambda = 1 - 0.8 * exp(-0.3 * layer).  The pages name the scaling without a
+    formula; this form (the Differential-Transformer one) is the workload's reading."""
+    return 1.0 - 0.8 * np.exp(-0.3 * float(layer))
 
 
 def group_norm_scale(o, gamma, beta, eps, lam):

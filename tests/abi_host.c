@@ -19,9 +19,10 @@ static int fails = 0;
     }                                                         \
   } while (0)
 
-/* Distinct, 256-byte aligned addresses that the library never dereferences on
- * the host: every call below returns before any CUDA call. */
-static void *fake(uintptr_t i) { return (void *)(uintptr_t)(0x100000u + 0x1000u * i); }
+/* Distinct, 256-byte aligned addresses 1 GiB apart (so that no two tensors of
+ * these shapes overlap) that the library never dereferences on the host: every
+ * call below returns before any CUDA call. */
+static void *fake(uintptr_t i) { return (void *)(((uintptr_t)1 << 36) + (i << 30)); }
 
 static mta_cfg recipe(void) {
   mta_cfg c;
@@ -93,6 +94,13 @@ int main(void) {
   EXPECT(mta_attn_bwd(fake(1), fake(2), fake(3), th, w, fake(10), &bad, (float *)fake(11),
                       (float *)fake(12), (float *)fake(13), NULL, NULL) == MTA_ERR_UNSUPPORTED);
   EXPECT(mta_gemm_bf16_nt(fake(1), fake(2), fake(3), 128, 256, 60, NULL) == MTA_ERR_INVALID);
+
+  /* an output that overlaps an input is refused before anything is enqueued */
+  c.workspace = fake(7);
+  c.workspace_bytes = ws;
+  EXPECT(mta_attn_fwd(fake(1), fake(2), fake(3), th, w, &c, fake(3)) == MTA_ERR_INVALID);
+  EXPECT(mta_attn_fwd(fake(1), fake(2), fake(3), th, w, &c, (char *)fake(1) + 4096) == MTA_ERR_INVALID);
+  c = recipe();
   EXPECT(mta_sync_status(NULL) == MTA_ERR_INVALID);
 
   if (fails) return 1;

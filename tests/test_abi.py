@@ -40,7 +40,7 @@ def test_every_declared_symbol_is_exported(L):
 
 
 def test_version_and_strings(L):
-    assert L.mta_abi_version() == 2
+    assert L.mta_abi_version() == 3
     for code in range(6):
         assert L.mta_status_string(code)
     assert L.mta_status_string(0) == b"ok"
@@ -56,8 +56,17 @@ def good_cfg(**kw):
 FAKE = ctypes.c_void_p(0x10000)  # never dereferenced: every case below fails a host check
 
 
-def call_attn(L, cfg, q=FAKE, theta=FAKE, w=FAKE, out=FAKE):
-    return L.mta_attn_fwd(q, FAKE, FAKE, theta, w, ctypes.byref(cfg) if cfg else None, out)
+def fake(i):
+    """Distinct addresses 1 GiB apart (no two tensors of these shapes overlap),
+    never dereferenced."""
+    return ctypes.c_void_p((1 << 36) + (i << 30))
+
+
+def call_attn(L, cfg, q=None, theta=FAKE, w=FAKE, out=None, k=None, v=None, default_q=True):
+    q = fake(1) if q is None and default_q else q
+    out = fake(6) if out is None else out
+    return L.mta_attn_fwd(q, fake(2) if k is None else k, fake(3) if v is None else v, theta, w,
+                          ctypes.byref(cfg) if cfg else None, out)
 
 
 def up(x):
@@ -99,6 +108,7 @@ def test_workspace_query(L):
     (dict(scale=-1.0), 1), (dict(qkv_row_stride=10), 1), (dict(kq_post=2), 1), (dict(kq_post=-1), 1),
     (dict(kq_post=1, kq_place=mta.OFF, path=mta.PATH_KQ), 2), (dict(kq_post=1, path=mta.PATH_TC), 2),
     (dict(d=200), 2), (dict(d=20), 2), (dict(B=70000), 2),
+    (dict(n_events=-1), 1), (dict(n_events=65), 1), (dict(n_events=2), 1),
 ])
 def test_bad_config_rejected(L, kw, code):
     cfg = good_cfg(**kw)
@@ -110,8 +120,8 @@ def test_null_and_workspace_errors(L):
     assert call_attn(L, None) == 1
     cfg = good_cfg()
     cfg.workspace, cfg.workspace_bytes = 0x100000, 1 << 20
-    assert call_attn(L, cfg, q=None) == 1
-    assert call_attn(L, cfg, out=None) == 1
+    assert call_attn(L, cfg, default_q=False) == 1
+    assert L.mta_attn_fwd(fake(1), fake(2), fake(3), FAKE, FAKE, ctypes.byref(cfg), None) == 1
     assert call_attn(L, cfg, theta=None) == 1           # kq_place PRE needs theta
     assert call_attn(L, cfg, w=None) == 1               # head mixing needs w
     post_only = good_cfg(kq_place=mta.OFF, kq_post=1)
@@ -119,7 +129,7 @@ def test_null_and_workspace_errors(L):
     assert call_attn(L, post_only, theta=None) == 1     # the post-softmax kernels are theta
     nomix = good_cfg(kq_place=mta.OFF, head_place=mta.OFF)
     nomix.workspace, nomix.workspace_bytes = 0x100000, 1 << 20
-    assert call_attn(L, nomix, q=ctypes.c_void_p(0x10001)) == 1   # misaligned bf16
+    assert call_attn(L, nomix, q=ctypes.c_void_p(fake(1).value + 1)) == 1   # misaligned bf16
     cfg.workspace_bytes = 16
     assert call_attn(L, cfg) == 3
     cfg.workspace, cfg.workspace_bytes = 0x100010, 1 << 20   # not 256-byte aligned
@@ -132,8 +142,8 @@ def test_layer_argument_errors(L):
     cfg = good_cfg()
     cfg.workspace, cfg.workspace_bytes = 0x100000, 1 << 30
     gn = mta.MtaGn(0x20000, 0x20000, 1e-5, 12, -1.0)
-    f = lambda c, g=ctypes.byref(gn), x=FAKE: L.mta_layer_fwd(x, FAKE, FAKE, FAKE, g, FAKE,
-                                                              ctypes.byref(c), FAKE)
+    f = lambda c, g=ctypes.byref(gn), x=fake(1), out=fake(6): L.mta_layer_fwd(
+        x, fake(2), FAKE, FAKE, g, fake(3), ctypes.byref(c), out)
     assert f(cfg, g=None) == 1
     assert f(cfg, x=None) == 1
     f32 = good_cfg(dtype=mta.F32)
@@ -146,6 +156,39 @@ def test_layer_argument_errors(L):
     base = L.mta_layer_workspace_bytes(ctypes.byref(good_cfg(c_q=3)))
     forced.workspace, forced.workspace_bytes = 0x100000, base
     assert f(forced) == 3
+    # the output must not overlap x, Wqkv or Wo
+    assert f(cfg, out=fake(1)) == 1
+    assert f(cfg, out=ctypes.c_void_p(fake(2).value + 256)) == 1
+    assert f(cfg, out=fake(3)) == 1
+
+
+def test_output_aliasing_rejected(L):
+    """An output that shares bytes with an input is refused (MTA_ERR_INVALID)
+    before anything is enqueued; distinct buffers pass on to the workspace check."""
+    cfg = good_cfg()
+    cfg.workspace, cfg.workspace_bytes = 0x100000, 16   # too small: a call that passes the
+    assert call_attn(L, cfg) == 3                        # pointer checks stops at the workspace
+    for n in ("q", "k", "v"):
+        i = {"q": 1, "k": 2, "v": 3}[n]
+        assert call_attn(L, cfg, out=fake(i)) == 1
+        # a view starting inside the input (e.g. the second token)
+        assert call_attn(L, cfg, out=ctypes.c_void_p(fake(i).value + 4 * 64 * 2)) == 1
+    # an output ending just before q starts does not overlap
+    n_out = 2 * 64 * 4 * 64 * 2
+    assert call_attn(L, cfg, out=ctypes.c_void_p(fake(1).value - n_out)) == 3
+    # strided q/k/v (a [B][L][3][H][d] buffer): out inside the span of the last token
+    st = good_cfg(qkv_row_stride=3 * 4 * 64)
+    st.workspace, st.workspace_bytes = 0x100000, 16
+    span = ((2 * 64 - 1) * 3 * 4 * 64 + 4 * 64) * 2
+    assert call_attn(L, st, out=ctypes.c_void_p(fake(3).value + span - 2)) == 1
+    assert call_attn(L, st, out=ctypes.c_void_p(fake(3).value + span)) == 3
+    # the backward pass: gradients must not overlap the inputs or each other
+    g = lambda dq, dk, dv: L.mta_attn_bwd(fake(1), fake(2), fake(3), FAKE, FAKE, fake(4),
+                                         ctypes.byref(cfg), dq, dk, dv, None, None)
+    assert g(fake(11), fake(12), fake(13)) == 3
+    assert g(fake(4), fake(12), fake(13)) == 1
+    assert g(fake(11), fake(11), fake(13)) == 1
+    assert g(fake(11), fake(12), fake(2)) == 1
 
 
 def test_building_block_argument_errors(L):
@@ -160,14 +203,14 @@ def test_backward_argument_errors(L):
     """mta_attn_bwd checks its arguments on the host and enqueues nothing on error."""
     cfg = good_cfg()
     cfg.workspace, cfg.workspace_bytes = 0x100000, 1 << 20
-    f = lambda c, dq=FAKE, theta=FAKE, dout=FAKE: L.mta_attn_bwd(FAKE, FAKE, FAKE, theta, FAKE, dout,
-                                                                  ctypes.byref(c) if c else None,
-                                                                  dq, FAKE, FAKE, FAKE, FAKE)
+    f = lambda c, dq=fake(11), theta=FAKE, dout=fake(4): L.mta_attn_bwd(
+        fake(1), fake(2), fake(3), theta, FAKE, dout, ctypes.byref(c) if c else None,
+        dq, fake(12), fake(13), FAKE, FAKE)
     assert f(None) == 1
     assert f(cfg, dq=None) == 1
     assert f(cfg, dout=None) == 1
     assert f(cfg, theta=None) == 1                      # kq_place PRE needs the kernels
-    assert f(cfg, dq=ctypes.c_void_p(0x10002)) == 1     # fp32 gradients, 4-byte aligned
+    assert f(cfg, dq=ctypes.c_void_p(fake(11).value + 2)) == 1   # fp32 gradients, 4-byte aligned
     forced = good_cfg(path=mta.PATH_TC)                 # only the CUDA-core backward exists
     forced.workspace, forced.workspace_bytes = 0x100000, 1 << 20
     assert f(forced) == 2
@@ -327,3 +370,16 @@ def test_extreme_documented_shapes_have_a_kernel(L, B, H, L_, d, cq, ck, ch, kq,
     cfg = mta.make_cfg(B, H, L_, d, cq, ck, ch, kq, hp, dt, kq_post=post)
     cfg.workspace_bytes = L.mta_attn_workspace_bytes(ctypes.byref(cfg))
     assert mta.attn_kernel(cfg) == mta.PATH_SIMT
+
+
+def test_selftest_wait_timeout_argument_errors(L):
+    """The bounded-wait diagnostic checks its arguments on the host."""
+    cfg = good_cfg()
+    cfg.workspace, cfg.workspace_bytes = 0x100000, 1 << 20
+    assert L.mta_selftest_wait_timeout(None, 1000) == 1
+    assert L.mta_selftest_wait_timeout(ctypes.byref(cfg), 0) == 1
+    assert L.mta_selftest_wait_timeout(ctypes.byref(cfg), 2000001) == 1
+    cfg.workspace = None
+    assert L.mta_selftest_wait_timeout(ctypes.byref(cfg), 1000) == 3
+    cfg.workspace, cfg.workspace_bytes = 0x100010, 1 << 20
+    assert L.mta_selftest_wait_timeout(ctypes.byref(cfg), 1000) == 3

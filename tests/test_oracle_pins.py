@@ -285,6 +285,16 @@ def test_group_norm_matches_torch():
     np.testing.assert_allclose(y, ref, rtol=0, atol=1e-12)
 
 
+def test_depth_scale_values():
+    """The depth scale at the layer the workloads use (layer 12: 0.978141, the
+    value the workload description states to six digits), its value 0.2 at the
+    first layer, and its rise towards 1 with depth."""
+    assert abs(O.depth_scale(12) - 0.978141) < 5e-7
+    assert abs(O.depth_scale(0) - 0.2) < 1e-15
+    vals = [O.depth_scale(n) for n in range(40)]
+    assert all(b > a for a, b in zip(vals, vals[1:])) and 1 - vals[-1] < 1e-5
+
+
 def test_group_norm_invariants():
     T, H, d = 5, 3, 16
     o = rand((T, H, d), 44, 2.0)

@@ -185,10 +185,17 @@ def test_kq_operand_scales(eq, ek):
 # ---------------------------------------------------------------------------
 
 def sample_rows(wl, n_extra=6, seed=0):
+    """Tile-boundary rows, a few random ones and, for a workload with planted
+    pairs, every planted query row r with the c_q-1 rows after it (the
+    convolution carries q_r's spike into them) and every copied key p+1 as a
+    query, in every batch."""
     rng = np.random.default_rng(seed)
     fixed = [0, 1, 4, 5, 6, 122, 123, 127, 128, 129, 245, 246, wl.L // 2, wl.L - 2, wl.L - 1]
     rows = sorted({(int(rng.integers(wl.B)), i) for i in fixed if i < wl.L})
     rows += [(int(rng.integers(wl.B)), int(rng.integers(wl.L))) for _ in range(n_extra)]
+    for p, r in synth.planted_positions(wl):
+        for b in range(wl.B):
+            rows += [(b, i) for i in range(r, min(wl.L, r + wl.c_q))] + [(b, p + 1)]
     return sorted(set(rows))
 
 
@@ -206,6 +213,51 @@ def test_full_size_sampled(name, path):
                                rows, wl.kq_place, wl.head_place)
     got = torch.stack([out[b, i] for b, i in rows])
     assert_close(got, ref, "bf16")
+    if wl.planted_pairs:
+        # the planted rows are compared on their own too, so that a wrong spike row
+        # cannot hide in the norm of the other rows
+        planted = {(b, r + a) for p, r in synth.planted_positions(wl) for b in range(wl.B)
+                   for a in range(wl.c_q) if r + a < wl.L}
+        sel = [n for n, row in enumerate(rows) if row in planted]
+        assert len(sel) >= wl.planted_pairs
+        assert_close(got[sel], ref[sel], "bf16")
+
+
+def spike_logits(wl, inp, h, r):
+    """Row r of head h's convolved logits C (log2 units), composed from the
+    oracle's steps: Mask_0, the key-query convolution, nothing after it (no
+    pre-softmax mixing in these workloads)."""
+    qh, kh = inp["q"][0, :, h][None], inp["k"][0, :, h][None]
+    a_hat = O.attention_logits(qh, kh, 1 / np.sqrt(wl.d))
+    qpos = np.arange(wl.L)
+    c = O.key_query_conv(O.mask_zero(a_hat, qpos), inp["theta"][h:h + 1])
+    return c[0, r, :r + 1] * np.log2(np.e)
+
+
+SPIKES = [(140, 200), (150, 290), (20, 100)]  # spike in a diagonal key tile, an earlier one, the first
+
+
+@pytest.mark.parametrize("path", [mta.PATH_AUTO, mta.PATH_TC, mta.PATH_SIMT])
+def test_planted_spikes_small_full(path):
+    """Planted high-similarity pairs (the long-context workload's recipe) at a
+    size the oracle computes in full: the spike of row 200 sits in its own
+    (diagonal) key tile 128..255, the spike of row 290 in the earlier tile
+    128..255, and the spike of row 100 in the first tile.  For the first two the
+    convolved logit at the spike exceeds every logit of the earlier key tiles by
+    more than 8 (log2 units) in every head, so the kernels' online softmax takes
+    its lazy rescale branch there (it rescales Z only when the running max grows by more
+    than 2^8); every element is compared."""
+    wl = synth.shrink(synth.WORKLOADS["long_d128_L16384"], B=1, H=4, L=300, planted_pairs=0,
+                      seed=1104)
+    inp = synth.make_attn_inputs(wl)
+    synth.plant_pairs_at(inp["q"], inp["k"], SPIKES, wl.seed)
+    inp["q"], inp["k"] = synth.round_bf16(inp["q"]), synth.round_bf16(inp["k"])
+    for p, r in SPIKES[:2]:
+        for h in range(wl.H):
+            c = spike_logits(wl, inp, h, r)
+            t_p = p // 128
+            assert c[128 * t_p:].max() > c[:128 * t_p].max() + 8.0, (p, r, h)
+    assert_close(run_attn(wl, inp, path), oracle_full(wl, inp), "bf16")
 
 
 def test_identity_workload_equals_causal_attention():
@@ -283,7 +335,7 @@ def test_layer_small(name, path):
     inp = synth.make_layer_inputs(wl)
     out = run_layer(wl, inp, path)
     ref = O.mta_layer(inp["x"], inp["wqkv"], inp["theta"], inp["w"], inp["gamma"], inp["beta"],
-                      inp["eps"], inp["lam"], inp["wo"], wl.H, wl.c_h, wl.kq_place, wl.head_place)
+                      inp["eps"], O.depth_scale(wl.depth), inp["wo"], wl.H, wl.c_h, wl.kq_place, wl.head_place)
     assert_close(out, ref, "bf16")
 
 
@@ -294,7 +346,7 @@ def test_layer_full_size_sampled(name):
     out = run_layer(wl, inp)
     rows = [(0, 0), (0, 5), (0, 123), (0, 2048), (0, 4095), (1, 1), (1, 700), (1, 4094)]
     ref = O.mta_layer_rows(inp["x"], inp["wqkv"], inp["theta"], inp["w"], inp["gamma"],
-                           inp["beta"], inp["eps"], inp["lam"], inp["wo"], wl.H, wl.c_h, rows,
+                           inp["beta"], inp["eps"], O.depth_scale(wl.depth), inp["wo"], wl.H, wl.c_h, rows,
                            wl.kq_place, wl.head_place)
     got = torch.stack([out[b, i] for b, i in rows])
     assert_close(got, ref, "bf16")
@@ -489,7 +541,7 @@ def test_post_conv_layer_small(hp):
     inp = synth.make_layer_inputs(wl)
     out = run_layer(wl, inp)
     ref = O.mta_layer(inp["x"], inp["wqkv"], inp["theta"], inp["w"], inp["gamma"], inp["beta"],
-                      inp["eps"], inp["lam"], inp["wo"], wl.H, wl.c_h, wl.kq_place, wl.head_place,
+                      inp["eps"], O.depth_scale(wl.depth), inp["wo"], wl.H, wl.c_h, wl.kq_place, wl.head_place,
                       theta_post=inp["theta_post"])
     assert_close(out, ref, "bf16")
 
@@ -525,7 +577,7 @@ def test_d96_layer_small(hp):
     inp = synth.make_layer_inputs(wl)
     out = run_layer(wl, inp)
     ref = O.mta_layer(inp["x"], inp["wqkv"], inp["theta"], inp["w"], inp["gamma"], inp["beta"],
-                      inp["eps"], inp["lam"], inp["wo"], wl.H, wl.c_h, wl.kq_place, wl.head_place)
+                      inp["eps"], O.depth_scale(wl.depth), inp["wo"], wl.H, wl.c_h, wl.kq_place, wl.head_place)
     assert_close(out, ref, "bf16")
 
 

@@ -5,6 +5,10 @@ because allocation can synchronise the device).  Its scratch lives in a static
 buffer inside the library; these tests call it through the C ABI and compare
 it with mta_layer_fwd given an ordinary workspace.
 
+Each output is also compared with the fp64 oracle, so that a mistake shared by
+both entry points cannot pass unseen, and the device's free memory is read
+around calls to show that the entry point allocates nothing.
+
 Named so that pytest collects it last; it passes alone in a fresh process and
 after the other tests (the static buffer keeps whatever the last call left).
 """
@@ -14,6 +18,7 @@ import numpy as np
 import pytest
 import torch
 
+import oracle as O
 from token_attention_b200 import build, mta, synth
 
 pytestmark = pytest.mark.gpu
@@ -68,6 +73,30 @@ def test_static_scratch_layer_matches_workspace_layer(L, name):
         g, r = out.double().cpu().numpy(), ref.double().cpu().numpy()
         rel = np.linalg.norm(g - r) / np.linalg.norm(r)
         assert rel <= 1e-2 and np.abs(g - r).max() <= 3e-2, (call, rel)
+        o = O.mta_layer(inp["x"], inp["wqkv"], inp["theta"], inp["w"], inp["gamma"], inp["beta"],
+                        inp["eps"], O.depth_scale(wl.depth), inp["wo"], wl.H, wl.c_h, wl.kq_place,
+                        wl.head_place)
+        rel_o = np.linalg.norm(g - o) / np.linalg.norm(o)
+        assert rel_o <= 1e-2 and np.abs(g - o).max() <= 3e-2, (call, rel_o)
+
+
+def test_static_scratch_allocates_nothing(L):
+    """Once a first call has run (with lazy module loading, the library's static
+    buffer becomes resident on the device then), further calls leave the
+    device's free memory exactly as it was: nothing is allocated per call."""
+    wl = synth.shrink(synth.WORKLOADS["layer_post_D2048_L4096"], B=2, L=300, D=256, H=2, d=128, seed=503)
+    inp = synth.make_layer_inputs(wl)
+    t = {k: dev(inp[k], k in ("x", "wqkv", "wo")) for k in
+         ("x", "wqkv", "wo", "theta", "w", "gamma", "beta")}
+    out = torch.empty((wl.B, wl.L, wl.D), dtype=torch.bfloat16, device="cuda")
+    assert static_call(L, wl, t, out) == 0
+    torch.cuda.synchronize()
+    free0, _ = torch.cuda.mem_get_info()
+    for _ in range(3):
+        assert static_call(L, wl, t, out) == 0
+    torch.cuda.synchronize()
+    free1, _ = torch.cuda.mem_get_info()
+    assert free1 == free0
 
 
 def test_static_scratch_rejects_sizes_beyond_the_buffer(L):

@@ -1133,7 +1133,7 @@ cudaError_t launch_attn_kq(const AttnArgs &a, const GnArgs *gn, void *ws) {
   void *vt = reinterpret_cast<char *>(xg) +
              (a.hp == 2 ? std::min<size_t>(kKqMaxClusters, 2 * items) * 2 * a.d * 128 * 4 : 0);
   cudaError_t e = launch_kq_prep(pa, a.stream);
-  if (e != cudaSuccess) return e;
+  if (e != cudaSuccess || (e = mark(a)) != cudaSuccess) return e;
   if (a.kqp) {
     VtPrepArgs va;
     va.v = a.v;
@@ -1143,7 +1143,7 @@ cudaError_t launch_attn_kq(const AttnArgs &a, const GnArgs *gn, void *ws) {
     va.B = a.B; va.H = a.H; va.L = a.L; va.d = a.d; va.cq = a.cq; va.ck = a.ck;
     va.nvh = a.hp == 2 ? 2 : 1;
     va.n_tiles = pa.n_tiles;
-    if ((e = launch_vt_prep(va, a.stream)) != cudaSuccess) return e;
+    if ((e = launch_vt_prep(va, a.stream)) != cudaSuccess || (e = mark(a)) != cudaSuccess) return e;
   }
   // MIX: 0 no head mixing, 1 pre-softmax mixing (both C of a group per CTA), 2 post-softmax
   auto go = [&](auto d_tag, auto mix_tag) -> cudaError_t {
@@ -1160,9 +1160,10 @@ cudaError_t launch_attn_kq(const AttnArgs &a, const GnArgs *gn, void *ws) {
   using M0 = std::integral_constant<int, 0>;
   using M1 = std::integral_constant<int, 1>;
   using M2 = std::integral_constant<int, 2>;
-  if (a.d == 128) return a.hp == 2 ? go(D128{}, M2{}) : a.hp == 1 ? go(D128{}, M1{}) : go(D128{}, M0{});
-  if (a.d == 96) return a.hp == 2 ? go(D96{}, M2{}) : a.hp == 1 ? go(D96{}, M1{}) : go(D96{}, M0{});
-  return a.hp == 2 ? go(D64{}, M2{}) : a.hp == 1 ? go(D64{}, M1{}) : go(D64{}, M0{});
+  if (a.d == 128) e = a.hp == 2 ? go(D128{}, M2{}) : a.hp == 1 ? go(D128{}, M1{}) : go(D128{}, M0{});
+  else if (a.d == 96) e = a.hp == 2 ? go(D96{}, M2{}) : a.hp == 1 ? go(D96{}, M1{}) : go(D96{}, M0{});
+  else e = a.hp == 2 ? go(D64{}, M2{}) : a.hp == 1 ? go(D64{}, M1{}) : go(D64{}, M0{});
+  return e != cudaSuccess ? e : mark(a);
 }
 
 }  // namespace mta

@@ -6,8 +6,9 @@
 // y = lambda * ((o - mean) / sqrt(var + eps) * gamma + beta), statistics over the
 // d channels of one (token, head), biased variance.
 //
-// HBM-bound: one warp per (token, head) row, grid-stride over rows, vector loads
-// when d == 128.  Used by the layer when the attention epilogue does not fuse it.
+// HBM-bound (2 bytes read and 2 written per element): at d = 128 half a warp per
+// (token, head) row with 16-byte loads, several rows in flight per warp; other d
+// one warp per row.  Used by the layer when the attention epilogue does not fuse it.
 #include <cuda_bf16.h>
 #include <stdint.h>
 
@@ -23,33 +24,67 @@ __device__ __forceinline__ float warp_sum(float x) {
   return x;
 }
 
+// d = 128: 16 lanes per (token, head) row, 8 channels (16 bytes) per lane, so a
+// warp covers two rows; each warp loads kRowsAhead row pairs before it reduces
+// any of them, so that enough bytes are in flight to keep HBM busy.
+constexpr int kRowsAhead = 4;
+
+__device__ __forceinline__ float half_warp_sum(float x) {
+#pragma unroll
+  for (int o = 8; o > 0; o >>= 1) x += __shfl_xor_sync(0xffffffffu, x, o);
+  return x;
+}
+
 __global__ void __launch_bounds__(256) group_norm_d128_kernel(const __nv_bfloat16 *__restrict__ o,
                                                               GnArgs gn, long long rows, int H,
                                                               __nv_bfloat16 *__restrict__ y) {
-  const int lane = threadIdx.x & 31;
+  const int lane = threadIdx.x & 31, half = lane >> 4, hl = lane & 15;
   const long long warp = (static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
   const long long nwarps = (static_cast<long long>(gridDim.x) * blockDim.x) >> 5;
-  for (long long r = warp; r < rows; r += nwarps) {
-    const int h = static_cast<int>(r % H);
-    const uint2 raw = reinterpret_cast<const uint2 *>(o + r * 128)[lane];
-    const __nv_bfloat162 p0 = *reinterpret_cast<const __nv_bfloat162 *>(&raw.x);
-    const __nv_bfloat162 p1 = *reinterpret_cast<const __nv_bfloat162 *>(&raw.y);
-    float x[4] = {__low2float(p0), __high2float(p0), __low2float(p1), __high2float(p1)};
-    const float mu = warp_sum(x[0] + x[1] + x[2] + x[3]) * (1.f / 128.f);
-    float s2 = 0.f;
+  // the loop bound is the same for both halves of a warp (every lane reaches
+  // every shuffle); a half whose row is past the end works on zeros
+  for (long long pb = 2 * warp; pb < rows; pb += 2 * nwarps * kRowsAhead) {
+    uint4 raw[kRowsAhead];
+    long long rr[kRowsAhead];
 #pragma unroll
-    for (int i = 0; i < 4; ++i) { x[i] -= mu; s2 += x[i] * x[i]; }
-    const float rstd = rsqrtf(warp_sum(s2) * (1.f / 128.f) + gn.eps);
-    const float4 g4 = reinterpret_cast<const float4 *>(gn.gamma + h * 128)[lane];
-    const float4 b4 = reinterpret_cast<const float4 *>(gn.beta + h * 128)[lane];
-    const float m = head_multiplier(gn.gate, gn.lam, h);
-    const float y0 = (x[0] * rstd * g4.x + b4.x) * m, y1 = (x[1] * rstd * g4.y + b4.y) * m;
-    const float y2 = (x[2] * rstd * g4.z + b4.z) * m, y3 = (x[3] * rstd * g4.w + b4.w) * m;
-    __nv_bfloat162 q0 = __floats2bfloat162_rn(y0, y1), q1 = __floats2bfloat162_rn(y2, y3);
-    uint2 outw;
-    outw.x = *reinterpret_cast<uint32_t *>(&q0);
-    outw.y = *reinterpret_cast<uint32_t *>(&q1);
-    reinterpret_cast<uint2 *>(y + r * 128)[lane] = outw;
+    for (int u = 0; u < kRowsAhead; ++u) {
+      rr[u] = pb + 2 * nwarps * u + half;
+      raw[u] = rr[u] < rows ? reinterpret_cast<const uint4 *>(o + rr[u] * 128)[hl] : make_uint4(0u, 0u, 0u, 0u);
+    }
+#pragma unroll
+    for (int u = 0; u < kRowsAhead; ++u) {
+      const uint32_t wv[4] = {raw[u].x, raw[u].y, raw[u].z, raw[u].w};
+      float x[8];
+      float s = 0.f;
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        x[2 * i] = __uint_as_float(wv[i] << 16);
+        x[2 * i + 1] = __uint_as_float(wv[i] & 0xffff0000u);
+        s += x[2 * i] + x[2 * i + 1];
+      }
+      const float mu = half_warp_sum(s) * (1.f / 128.f);
+      float s2 = 0.f;
+#pragma unroll
+      for (int i = 0; i < 8; ++i) { x[i] -= mu; s2 += x[i] * x[i]; }
+      const float rstd = rsqrtf(half_warp_sum(s2) * (1.f / 128.f) + gn.eps);
+      if (rr[u] >= rows) continue;
+      const int h = static_cast<int>(rr[u] % H);
+      const float4 *g4 = reinterpret_cast<const float4 *>(gn.gamma + h * 128 + 8 * hl);
+      const float4 *b4 = reinterpret_cast<const float4 *>(gn.beta + h * 128 + 8 * hl);
+      const float4 ga = g4[0], gb = g4[1], ba = b4[0], bb = b4[1];
+      const float g[8] = {ga.x, ga.y, ga.z, ga.w, gb.x, gb.y, gb.z, gb.w};
+      const float b[8] = {ba.x, ba.y, ba.z, ba.w, bb.x, bb.y, bb.z, bb.w};
+      const float m = head_multiplier(gn.gate, gn.lam, h);
+      uint4 outw;
+      uint32_t *ow = reinterpret_cast<uint32_t *>(&outw);
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        __nv_bfloat162 q = __floats2bfloat162_rn((x[2 * i] * rstd * g[2 * i] + b[2 * i]) * m,
+                                                 (x[2 * i + 1] * rstd * g[2 * i + 1] + b[2 * i + 1]) * m);
+        ow[i] = *reinterpret_cast<uint32_t *>(&q);
+      }
+      reinterpret_cast<uint4 *>(y + rr[u] * 128)[hl] = outw;
+    }
   }
 }
 
@@ -99,13 +134,16 @@ cudaError_t launch_group_norm(const void *o, const GnArgs &gn, int tokens, int H
   int dev = 0;
   if (cudaGetDevice(&dev) == cudaSuccess)
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  const long long want = (rows + 7) / 8;  // 8 warps per block
-  const int blocks = static_cast<int>(want < 8LL * sms ? want : 8LL * sms);
   const __nv_bfloat16 *src = static_cast<const __nv_bfloat16 *>(o);
   __nv_bfloat16 *dst = static_cast<__nv_bfloat16 *>(y);
   const bool vec = d == 128 &&
                    ((reinterpret_cast<uintptr_t>(gn.gamma) | reinterpret_cast<uintptr_t>(gn.beta)) & 15) == 0 &&
-                   ((reinterpret_cast<uintptr_t>(o) | reinterpret_cast<uintptr_t>(y)) & 7) == 0;
+                   ((reinterpret_cast<uintptr_t>(o) | reinterpret_cast<uintptr_t>(y)) & 15) == 0;
+  // d = 128: a block of 8 warps covers 16 rows per step and kRowsAhead steps at once;
+  // otherwise a warp per row.  At most 8 blocks per SM (grid-stride beyond that).
+  const long long per_block = vec ? 16LL * kRowsAhead : 8LL;
+  const long long want = (rows + per_block - 1) / per_block;
+  const int blocks = static_cast<int>(want < 8LL * sms ? want : 8LL * sms);
   if (vec)
     group_norm_d128_kernel<<<blocks, 256, 0, stream>>>(src, gn, rows, H, dst);
   else

@@ -9,6 +9,19 @@ namespace mta {
 // Bits of the error word kept at the start of the caller's workspace.
 enum : unsigned { ERRBIT_TIMEOUT = 1u };
 
+// Optional timing events of one call (mta_cfg.events): next() records events[i]
+// on the call's stream, i = 0 just before the call's first kernel and i = k just
+// after its k-th kernel, while i < n.
+struct Marks {
+  void *const *ev = nullptr;
+  int n = 0, i = 0;
+  cudaStream_t st = nullptr;
+  cudaError_t next() {
+    if (!ev || i >= n) return cudaSuccess;
+    return cudaEventRecord(static_cast<cudaEvent_t>(ev[i++]), st);
+  }
+};
+
 // Arguments of one attention call, already validated by the C-ABI layer.
 struct AttnArgs {
   const void *q, *k, *v;  // [B][L][H][d], token stride rs elements
@@ -22,7 +35,9 @@ struct AttnArgs {
   float scale;
   unsigned *err;          // error word in the workspace
   cudaStream_t stream;
+  Marks *marks;           // timing events of the call, or null
 };
+inline cudaError_t mark(const AttnArgs &a) { return a.marks ? a.marks->next() : cudaSuccess; }
 
 // Depth-scaled group norm fused into an attention epilogue (optional).
 struct GnArgs {
@@ -103,6 +118,11 @@ cudaError_t launch_gemm_bf16_nt(const void *A, const void *B, void *C, int M, in
 // Depth-scaled group norm over [tokens][H][d] bf16.
 cudaError_t launch_group_norm(const void *o, const GnArgs &gn, int tokens, int H, int d, void *y,
                               cudaStream_t stream);
+
+// Diagnostic: one CTA whose bounded waits cannot complete (selftest.cu); err is the
+// workspace's error word, out[2] counters of the waits that gave up.
+cudaError_t launch_wait_timeout_selftest(unsigned long long limit_ns, unsigned *err, unsigned *out,
+                                         cudaStream_t stream);
 
 // cuTensorMapEncodeTiled through the runtime's driver entry point.
 // dims/strides innermost first; strides in bytes for dims 1..rank-1.

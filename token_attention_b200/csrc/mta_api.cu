@@ -37,6 +37,7 @@ mta_status check_cfg(const mta_cfg *c) {
   if (c->dtype != MTA_F32 && c->dtype != MTA_BF16) return MTA_ERR_INVALID;
   if (c->path < 0 || c->path > 3) return MTA_ERR_INVALID;
   if (!isfinite(c->scale) || c->scale < 0.f) return MTA_ERR_INVALID;
+  if (c->n_events < 0 || c->n_events > 64 || (c->n_events > 0 && !c->events)) return MTA_ERR_INVALID;
   const long long hd = static_cast<long long>(c->H) * c->d;
   if (c->qkv_row_stride != 0 && c->qkv_row_stride < hd) return MTA_ERR_INVALID;
   return MTA_OK;
@@ -58,7 +59,16 @@ AttnArgs make_args(const void *q, const void *k, const void *v, const float *the
   a.scale = c->scale > 0.f ? c->scale : 1.0f / sqrtf(static_cast<float>(c->d));
   a.err = static_cast<unsigned *>(c->workspace);
   a.stream = static_cast<cudaStream_t>(c->stream);
+  a.marks = nullptr;
   return a;
+}
+
+Marks make_marks(const mta_cfg *c) {
+  Marks m;
+  m.ev = c->events;
+  m.n = c->n_events;
+  m.st = static_cast<cudaStream_t>(c->stream);
+  return m;
 }
 
 enum Kernel { K_SIMT = 1, K_TC = 2, K_KQ = 3 };
@@ -104,10 +114,31 @@ mta_status select_kernel(const AttnArgs &a, int path, size_t kq_room, Kernel *k)
   return MTA_OK;
 }
 
+// Launches the attention kernel(s) of `k`, recording a timing mark after each.
 cudaError_t launch_kernel(Kernel k, const AttnArgs &a, const GnArgs *gn, void *kq_ws) {
   if (k == K_KQ) return launch_attn_kq(a, gn, kq_ws);
-  if (k == K_TC) return launch_attn_tc(a, gn);
-  return launch_attn_simt(a);
+  const cudaError_t e = k == K_TC ? launch_attn_tc(a, gn) : launch_attn_simt(a);
+  return e != cudaSuccess ? e : mark(a);
+}
+
+// Whether the byte ranges [a, a + na) and [b, b + nb) share a byte.
+bool overlaps(const void *a, size_t na, const void *b, size_t nb) {
+  const uintptr_t a0 = reinterpret_cast<uintptr_t>(a), b0 = reinterpret_cast<uintptr_t>(b);
+  return a0 < b0 + nb && b0 < a0 + na;
+}
+
+// Bytes spanned by q, k or v of cfg ([B][L][H][d] with token stride qkv_row_stride).
+size_t qkv_span(const mta_cfg *c, size_t es) {
+  const size_t rs = c->qkv_row_stride ? static_cast<size_t>(c->qkv_row_stride) : static_cast<size_t>(c->H) * c->d;
+  return ((static_cast<size_t>(c->B) * c->L - 1) * rs + static_cast<size_t>(c->H) * c->d) * es;
+}
+
+// A dense [B][L][H][d] output of element size oes must not share memory with q, k or v.
+bool output_aliases_qkv(const void *q, const void *k, const void *v, const mta_cfg *c, const void *out,
+                        size_t oes) {
+  const size_t es = c->dtype == MTA_F32 ? 4 : 2, n = qkv_span(c, es);
+  const size_t no = static_cast<size_t>(c->B) * c->L * c->H * c->d * oes;
+  return overlaps(out, no, q, n) || overlaps(out, no, k, n) || overlaps(out, no, v, n);
 }
 
 mta_status check_attn_pointers(const void *q, const void *k, const void *v, const float *theta,
@@ -215,11 +246,15 @@ mta_status mta_attn_fwd(const void *q, const void *k, const void *v, const float
   mta_status s = check_cfg(cfg);
   if (s != MTA_OK) return s;
   if ((s = check_attn_pointers(q, k, v, theta_kq, w_head, cfg, out)) != MTA_OK) return s;
+  if (output_aliases_qkv(q, k, v, cfg, out, cfg->dtype == MTA_F32 ? 4 : 2)) return MTA_ERR_INVALID;
   if ((s = check_workspace(cfg, kStatusBytes)) != MTA_OK) return s;
   AttnArgs a = make_args(q, k, v, theta_kq, w_head, cfg, out);
   Kernel kern = K_SIMT;
   if ((s = select_kernel(a, cfg->path, cfg->workspace_bytes - kStatusBytes, &kern)) != MTA_OK) return s;
   if ((s = clear_status(cfg)) != MTA_OK) return s;
+  Marks m = make_marks(cfg);
+  a.marks = &m;
+  if (m.next() != cudaSuccess) return MTA_ERR_CUDA;
   const cudaError_t e = launch_kernel(kern, a, nullptr, static_cast<char *>(cfg->workspace) + kStatusBytes);
   return e == cudaSuccess ? MTA_OK : MTA_ERR_CUDA;
 }
@@ -256,6 +291,9 @@ mta_status mta_layer_fwd(const void *x, const void *Wqkv, const float *theta, co
   const size_t T = layer_tokens(cfg), D = static_cast<size_t>(cfg->H) * cfg->d;
   if (T > static_cast<size_t>(65535) * 128 || 3 * D > static_cast<size_t>(1) << 30)
     return MTA_ERR_UNSUPPORTED;
+  if (overlaps(out, T * D * 2, x, T * D * 2) || overlaps(out, T * D * 2, Wqkv, 3 * D * D * 2) ||
+      overlaps(out, T * D * 2, Wo, D * D * 2))
+    return MTA_ERR_INVALID;
   if ((s = check_workspace(cfg, layer_base_workspace_bytes(cfg))) != MTA_OK) return s;
 
   char *ws = static_cast<char *>(cfg->workspace);
@@ -276,9 +314,12 @@ mta_status mta_layer_fwd(const void *x, const void *Wqkv, const float *theta, co
   cudaStream_t st = static_cast<cudaStream_t>(cfg->stream);
   unsigned *err = static_cast<unsigned *>(cfg->workspace);
   if ((s = clear_status(cfg)) != MTA_OK) return s;
+  Marks m = make_marks(cfg);
+  a.marks = &m;
+  if (m.next() != cudaSuccess) return MTA_ERR_CUDA;
   // QKV = x Wqkv^T
   if (launch_gemm_bf16_nt(x, Wqkv, qkv, static_cast<int>(T), static_cast<int>(3 * D),
-                          static_cast<int>(D), err, st) != cudaSuccess)
+                          static_cast<int>(D), err, st) != cudaSuccess || m.next() != cudaSuccess)
     return MTA_ERR_CUDA;
   if (kern != K_SIMT) {
     // attention with the group norm and depth scale fused into its epilogue: Y
@@ -287,13 +328,14 @@ mta_status mta_layer_fwd(const void *x, const void *Wqkv, const float *theta, co
   } else {
     // attention output O, then the stand-alone group norm O -> Y
     a.out = obuf;
-    if (launch_attn_simt(a) != cudaSuccess) return MTA_ERR_CUDA;
-    if (launch_group_norm(obuf, g, static_cast<int>(T), cfg->H, cfg->d, ybuf, st) != cudaSuccess)
+    if (launch_kernel(kern, a, nullptr, kq_ws) != cudaSuccess) return MTA_ERR_CUDA;
+    if (launch_group_norm(obuf, g, static_cast<int>(T), cfg->H, cfg->d, ybuf, st) != cudaSuccess ||
+        m.next() != cudaSuccess)
       return MTA_ERR_CUDA;
   }
   // out = Y Wo^T
   if (launch_gemm_bf16_nt(ybuf, Wo, out, static_cast<int>(T), static_cast<int>(D),
-                          static_cast<int>(D), err, st) != cudaSuccess)
+                          static_cast<int>(D), err, st) != cudaSuccess || m.next() != cudaSuccess)
     return MTA_ERR_CUDA;
   return MTA_OK;
 }
@@ -310,6 +352,13 @@ mta_status mta_attn_bwd(const void *q, const void *k, const void *v, const float
   if (cfg->path > 1) return MTA_ERR_UNSUPPORTED;
   if ((s = check_attn_pointers(q, k, v, theta_kq, w_head, cfg, dout)) != MTA_OK) return s;
   if (!dq || !dk || !dv || !aligned(dq, 4) || !aligned(dk, 4) || !aligned(dv, 4)) return MTA_ERR_INVALID;
+  {
+    const size_t es = cfg->dtype == MTA_F32 ? 4 : 2;
+    const size_t ng = static_cast<size_t>(cfg->B) * cfg->L * cfg->H * cfg->d * 4;
+    for (const float *g : {dq, dk, dv})
+      if (output_aliases_qkv(q, k, v, cfg, g, 4) || overlaps(g, ng, dout, ng / 4 * es)) return MTA_ERR_INVALID;
+    if (overlaps(dq, ng, dk, ng) || overlaps(dq, ng, dv, ng) || overlaps(dk, ng, dv, ng)) return MTA_ERR_INVALID;
+  }
   if ((dtheta && !aligned(dtheta, 4)) || (dw && !aligned(dw, 4))) return MTA_ERR_INVALID;
   if ((s = check_workspace(cfg, kStatusBytes)) != MTA_OK) return s;
   BwdArgs a;
@@ -331,7 +380,10 @@ mta_status mta_attn_bwd(const void *q, const void *k, const void *v, const float
   a.stream = static_cast<cudaStream_t>(cfg->stream);
   if ((a.kqp ? attn_bwd_post_pick_rows(a) : attn_bwd_simt_pick_rows(a)) == 0) return MTA_ERR_UNSUPPORTED;
   if ((s = clear_status(cfg)) != MTA_OK) return s;
-  return (a.kqp ? launch_attn_bwd_post(a) : launch_attn_bwd_simt(a)) == cudaSuccess ? MTA_OK : MTA_ERR_CUDA;
+  Marks m = make_marks(cfg);
+  if (m.next() != cudaSuccess) return MTA_ERR_CUDA;
+  if ((a.kqp ? launch_attn_bwd_post(a) : launch_attn_bwd_simt(a)) != cudaSuccess) return MTA_ERR_CUDA;
+  return m.next() == cudaSuccess ? MTA_OK : MTA_ERR_CUDA;
 }
 
 mta_status mta_gemm_bf16_nt(const void *A, const void *Bm, void *C, int M, int N, int K, void *stream) {
@@ -354,6 +406,20 @@ mta_status mta_group_norm_scale(const void *o, const mta_gn *gn, int tokens, int
                  cudaSuccess
              ? MTA_OK
              : MTA_ERR_CUDA;
+}
+
+mta_status mta_selftest_wait_timeout(const mta_cfg *cfg, unsigned limit_us) {
+  if (!cfg) return MTA_ERR_INVALID;
+  if (limit_us < 1 || limit_us > 2000000) return MTA_ERR_INVALID;
+  mta_status s = check_workspace(cfg, kStatusBytes);
+  if (s != MTA_OK) return s;
+  if ((s = clear_status(cfg)) != MTA_OK) return s;
+  // counters of the waits that gave up, after the error word
+  unsigned *word = static_cast<unsigned *>(cfg->workspace);
+  cudaStream_t st = static_cast<cudaStream_t>(cfg->stream);
+  if (cudaMemsetAsync(word + 1, 0, 2 * sizeof(unsigned), st) != cudaSuccess) return MTA_ERR_CUDA;
+  return launch_wait_timeout_selftest(1000ull * limit_us, word, word + 1, st) == cudaSuccess ? MTA_OK
+                                                                                              : MTA_ERR_CUDA;
 }
 
 mta_status mta_sync_status(const mta_cfg *cfg) {

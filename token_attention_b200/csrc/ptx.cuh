@@ -61,23 +61,29 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
 
 // Bounded wait for the phase of parity `parity` to complete.  Returns false
 // (after setting *abort and the workspace error bit) if it did not complete
-// within kWaitLimitNs; once *abort is set, later waits return at once so that
+// within limit_ns; once *abort is set, later waits return at once so that
 // every thread still reaches every CTA barrier and the kernel can end.
-__device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, volatile int *abort,
-                                          unsigned *err) {
+__device__ __forceinline__ bool mbar_wait_for(uint64_t *bar, uint32_t parity, volatile int *abort,
+                                              unsigned *err, unsigned long long limit_ns) {
   if (mbar_try_wait(bar, parity)) return true;
   unsigned long long t0 = globaltimer_ns();
   for (uint32_t it = 0;; ++it) {
     if (mbar_try_wait(bar, parity)) return true;
     if ((it & 63u) == 63u) {
       if (*abort) return false;
-      if (globaltimer_ns() - t0 > kWaitLimitNs) {
+      if (globaltimer_ns() - t0 > limit_ns) {
         *abort = 1;
         if (err) atomicOr(err, ERRBIT_TIMEOUT);
         return false;
       }
     }
   }
+}
+
+// The kernels' bounded wait: mbar_wait_for with the library's limit.
+__device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, volatile int *abort,
+                                          unsigned *err) {
+  return mbar_wait_for(bar, parity, abort, err, kWaitLimitNs);
 }
 
 // Multiplier of head h's normalised output: the sigmoid scalar gate when gate

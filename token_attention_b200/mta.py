@@ -8,7 +8,6 @@ module raises.
 from __future__ import annotations
 
 import ctypes
-import math
 import os
 
 HERE = os.path.dirname(os.path.abspath(__file__))
@@ -27,7 +26,8 @@ STATUS = {0: "MTA_OK", 1: "MTA_ERR_INVALID", 2: "MTA_ERR_UNSUPPORTED", 3: "MTA_E
 EXPORTS = ["mta_attn_workspace_bytes", "mta_attn_fwd", "mta_layer_workspace_bytes",
            "mta_layer_fwd", "mta_gemm_bf16_nt", "mta_group_norm_scale", "mta_sync_status",
            "mta_status_string", "mta_abi_version", "mta_layer_fwd_static",
-           "mta_attn_bwd_workspace_bytes", "mta_attn_bwd", "mta_attn_kernel"]
+           "mta_attn_bwd_workspace_bytes", "mta_attn_bwd", "mta_attn_kernel",
+           "mta_selftest_wait_timeout"]
 
 
 class MtaCfg(ctypes.Structure):
@@ -36,7 +36,8 @@ class MtaCfg(ctypes.Structure):
                 ("kq_place", ctypes.c_int), ("head_place", ctypes.c_int),
                 ("kq_post", ctypes.c_int), ("dtype", ctypes.c_int), ("path", ctypes.c_int), ("scale", ctypes.c_float),
                 ("qkv_row_stride", ctypes.c_longlong), ("stream", ctypes.c_void_p),
-                ("workspace", ctypes.c_void_p), ("workspace_bytes", ctypes.c_size_t)]
+                ("workspace", ctypes.c_void_p), ("workspace_bytes", ctypes.c_size_t),
+                ("events", ctypes.POINTER(ctypes.c_void_p)), ("n_events", ctypes.c_int)]
 
 
 class MtaGn(ctypes.Structure):
@@ -81,6 +82,8 @@ def lib() -> ctypes.CDLL:
         L.mta_attn_bwd.restype = I
         L.mta_attn_kernel.argtypes = [cfgp]
         L.mta_attn_kernel.restype = I
+        L.mta_selftest_wait_timeout.argtypes = [cfgp, ctypes.c_uint]
+        L.mta_selftest_wait_timeout.restype = I
         L.mta_sync_status.argtypes = [cfgp]
         L.mta_sync_status.restype = I
         L.mta_status_string.argtypes = [I]
@@ -127,8 +130,21 @@ def _stream_handle(stream):
     return ctypes.c_void_p(s.cuda_stream)
 
 
+def _set_events(cfg: MtaCfg, events, n_events=None) -> None:
+    """events: CUDA event handles (ints or objects with a cuda_event handle, such
+    as torch.cuda.Event after its first record) the call records; n_events
+    overrides the count (to test the library's checks)."""
+    if events:
+        hs = [e.cuda_event if hasattr(e, "cuda_event") else int(e) for e in events]
+        arr = (ctypes.c_void_p * len(hs))(*hs)
+        cfg._events_keep = arr          # keeps the array alive with the struct
+        cfg.events = ctypes.cast(arr, ctypes.POINTER(ctypes.c_void_p))
+    cfg.n_events = len(events or ()) if n_events is None else n_events
+
+
 def make_cfg(B, H, L, d, c_q, c_k, c_h, kq_place, head_place, dtype, path=PATH_AUTO, scale=0.0,
-             qkv_row_stride=0, stream=None, workspace=None, kq_post=0) -> MtaCfg:
+             qkv_row_stride=0, stream=None, workspace=None, kq_post=0, events=None,
+             n_events=None) -> MtaCfg:
     cfg = MtaCfg()
     cfg.B, cfg.H, cfg.L, cfg.d = B, H, L, d
     cfg.c_q, cfg.c_k, cfg.c_h = c_q, c_k, c_h
@@ -140,6 +156,7 @@ def make_cfg(B, H, L, d, c_q, c_k, c_h, kq_place, head_place, dtype, path=PATH_A
     if workspace is not None:
         cfg.workspace = workspace.data_ptr()
         cfg.workspace_bytes = workspace.numel() * workspace.element_size()
+    _set_events(cfg, events, n_events)
     return cfg
 
 
@@ -195,7 +212,8 @@ def attn_kernel(cfg: MtaCfg) -> int:
 
 
 def attn_fwd(q, k, v, theta, w, c_q, c_k, c_h, kq_place=PRE, head_place=POST, *, out=None,
-             ws=None, path=PATH_AUTO, scale=0.0, stream=None, check=False, theta_post=None):
+             ws=None, path=PATH_AUTO, scale=0.0, stream=None, check=False, theta_post=None,
+             events=None):
     """MTA attention.  q, k, v: [B, L, H, d] CUDA tensors (fp32 or bf16), dense in
     (H, d) with a common token stride; theta [H, c_q, c_k] fp32; w [H/c_h, c_h, c_h]
     fp32; theta_post: optional [H, c_q, c_k] fp32 kernels of the key-query
@@ -218,7 +236,7 @@ def attn_fwd(q, k, v, theta, w, c_q, c_k, c_h, kq_place=PRE, head_place=POST, *,
         out = torch.empty((B, L, H, d), dtype=q.dtype, device=q.device)
     theta, kq_post = _kernels(theta, theta_post, kq_place)
     cfg = make_cfg(B, H, L, d, c_q, c_k, c_h, kq_place, head_place, _dtype_code(q), path, scale,
-                   q.stride(1), _stream_handle(stream), kq_post=kq_post)
+                   q.stride(1), _stream_handle(stream), kq_post=kq_post, events=events)
     if ws is None:
         ws = workspace(lib().mta_attn_workspace_bytes(ctypes.byref(cfg)), q.device)
     cfg.workspace, cfg.workspace_bytes = ws.data_ptr(), _nbytes(ws)
@@ -230,7 +248,8 @@ def attn_fwd(q, k, v, theta, w, c_q, c_k, c_h, kq_place=PRE, head_place=POST, *,
 
 
 def attn_bwd(q, k, v, theta, w, dout, c_q, c_k, c_h, kq_place=PRE, head_place=POST, *, ws=None,
-             path=PATH_AUTO, scale=0.0, stream=None, check=False, grads=None, theta_post=None):
+             path=PATH_AUTO, scale=0.0, stream=None, check=False, grads=None, theta_post=None,
+             events=None):
     """Gradients of attn_fwd.  dout: [B, L, H, d] dense, dtype of q.  theta,
     theta_post: as for attn_fwd (a stacked [n, H, c_q, c_k] theta included).
     Returns a dict of fp32 tensors: dq, dk, dv [B, L, H, d]; dtheta [H, c_q, c_k]
@@ -272,7 +291,7 @@ def attn_bwd(q, k, v, theta, w, dout, c_q, c_k, c_h, kq_place=PRE, head_place=PO
                 raise ValueError(f"grads[{name!r}] is missing")
             _need(f"grads[{name!r}]", grads[name], dv, torch.float32, shape)
     cfg = make_cfg(B, H, L, d, c_q, c_k, c_h, kq_place, head_place, _dtype_code(q), path, scale,
-                   q.stride(1), _stream_handle(stream), kq_post=kq_post)
+                   q.stride(1), _stream_handle(stream), kq_post=kq_post, events=events)
     if ws is None:
         ws = workspace(lib().mta_attn_bwd_workspace_bytes(ctypes.byref(cfg)), q.device)
     cfg.workspace, cfg.workspace_bytes = ws.data_ptr(), _nbytes(ws)
@@ -325,13 +344,9 @@ def mta_attention(q, k, v, theta, w, c_q, c_k, c_h, kq_place=PRE, head_place=POS
     return _MTA_FN.apply(q, k, v, theta, w, c_q, c_k, c_h, kq_place, head_place, theta_post)
 
 
-def depth_scale(layer: int) -> float:
-    return 1.0 - 0.8 * math.exp(-0.3 * layer)
-
-
 def layer_fwd(x, wqkv, theta, w, gamma, beta, wo, H, c_q, c_k, c_h, kq_place=PRE,
               head_place=POST, *, eps=1e-5, layer=12, lam=-1.0, gate=None, out=None, ws=None,
-              path=PATH_AUTO, stream=None, check=False, theta_post=None):
+              path=PATH_AUTO, stream=None, check=False, theta_post=None, events=None):
     """Full MTA layer, bf16.  x [B, L, D]; wqkv [3D, D]; wo [D, D]; gamma, beta [D]
     fp32; gate: optional [H] fp32 sigmoid-gate logits replacing the depth scale;
     theta_post: optional [H, c_q, c_k] post-softmax key-query kernels.
@@ -356,7 +371,7 @@ def layer_fwd(x, wqkv, theta, w, gamma, beta, wo, H, c_q, c_k, c_h, kq_place=PRE
         out = torch.empty((B, L, D), dtype=x.dtype, device=x.device)
     theta, kq_post = _kernels(theta, theta_post, kq_place)
     cfg = make_cfg(B, H, L, d, c_q, c_k, c_h, kq_place, head_place, _dtype_code(x), path, 0.0, 0,
-                   _stream_handle(stream), kq_post=kq_post)
+                   _stream_handle(stream), kq_post=kq_post, events=events)
     if ws is None:
         ws = workspace(lib().mta_layer_workspace_bytes(ctypes.byref(cfg)), x.device)
     cfg.workspace, cfg.workspace_bytes = ws.data_ptr(), _nbytes(ws)

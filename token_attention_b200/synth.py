@@ -13,7 +13,6 @@ appendix D (880M model: D=1536, 16 heads, context 2048).
 from __future__ import annotations
 
 import dataclasses
-import math
 
 import numpy as np
 
@@ -55,12 +54,6 @@ def bf16_bits(x: np.ndarray) -> np.ndarray:
     return (u >> 16).astype(np.uint16)
 
 
-def depth_scale(layer: int) -> float:
-    """Depth-dependent output scale lambda = 1 - 0.8 exp(-0.3 layer) (the
-    Differential-Transformer form the pages name for MTA's group-norm scaling)."""
-    return 1.0 - 0.8 * math.exp(-0.3 * layer)
-
-
 @dataclasses.dataclass(frozen=True)
 class Workload:
     name: str
@@ -81,7 +74,7 @@ class Workload:
     w_std: float
     layer: bool = False   # full layer (QKV projection .. output projection)
     D: int = 0
-    depth: int = 12       # layer index for the depth scale
+    depth: int = 12       # layer index of the depth scale (the scale itself is the method's)
     planted_pairs: int = 0
     kq_post: bool = False # key-query convolution after the softmax as well (own kernels)
 
@@ -182,18 +175,46 @@ def make_w(wl: Workload) -> np.ndarray:
     return w
 
 
+def _plant_draws(wl: Workload) -> list:
+    """The seeded draws of the planted pairs, in stream order: (p, r, noise) with
+    noise [B][H][d] float32 for key p+1."""
+    rng = rng_for(wl.seed, _S_PLANT)
+    L = wl.L
+    draws = []
+    for _ in range(wl.planted_pairs):
+        p = int(rng.integers(wl.c_k, L - 2))
+        r = int(rng.integers(p + 2, L)) if p + 2 < L else L - 1
+        noise = rng.standard_normal(size=(wl.B, wl.H, wl.d), dtype=np.float32) * 0.05
+        draws.append((p, r, noise))
+    return draws
+
+
+def planted_positions(wl: Workload) -> list:
+    """(p, r) of every planted pair of the workload: key p+1 is a near copy of key
+    p and query r is 2*k_p (the same draws make_attn_inputs uses)."""
+    return [(p, r) for p, r, _ in _plant_draws(wl)]
+
+
+def plant_pairs_at(q: np.ndarray, k: np.ndarray, positions, seed: int) -> None:
+    """Plants pairs at the given (p, r) positions in q, k [B][L][H][d] (in place),
+    with the key noise drawn from the plant stream of `seed`."""
+    rng = rng_for(seed, _S_PLANT)
+    draws = [(p, r, rng.standard_normal(size=(k.shape[0], k.shape[2], k.shape[3]), dtype=np.float32) * 0.05)
+             for p, r in positions]
+    _apply_pairs(q, k, draws)
+
+
+def _apply_pairs(q: np.ndarray, k: np.ndarray, draws) -> None:
+    for p, r, noise in draws:
+        k[:, p + 1] = k[:, p] + noise
+        q[:, r] = 2.0 * k[:, p]
+
+
 def _plant_pairs(wl: Workload, q: np.ndarray, k: np.ndarray) -> None:
     """Planted high-similarity pairs (reading of "a few planted high-similarity
     key pairs at random positions"): for n seeded positions p, key p+1 becomes a
     near copy of key p and a later query r > p+1 becomes 2*k_p, in every head."""
-    rng = rng_for(wl.seed, _S_PLANT)
-    L = wl.L
-    for _ in range(wl.planted_pairs):
-        p = int(rng.integers(wl.c_k, L - 2))
-        r = int(rng.integers(p + 2, L)) if p + 2 < L else L - 1
-        noise = rng.standard_normal(size=k.shape[0:1] + k.shape[2:], dtype=np.float32) * 0.05
-        k[:, p + 1] = k[:, p] + noise
-        q[:, r] = 2.0 * k[:, p]
+    _apply_pairs(q, k, _plant_draws(wl))
 
 
 def make_attn_inputs(wl: Workload) -> dict:
@@ -220,4 +241,4 @@ def make_layer_inputs(wl: Workload) -> dict:
     gamma = normal(wl.seed, _S_GAMMA, (D,), mean=1.0, std=0.1)
     beta = normal(wl.seed, _S_BETA, (D,), std=0.1)
     return dict(x=x, wqkv=wqkv, wo=wo, theta=make_theta(wl), w=make_w(wl),
-                theta_post=make_theta_post(wl), gamma=gamma, beta=beta, eps=1e-5, lam=depth_scale(wl.depth))
+                theta_post=make_theta_post(wl), gamma=gamma, beta=beta, eps=1e-5)
