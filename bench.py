@@ -307,6 +307,20 @@ def step_fn(wl, mta, sets, ws, outs, stream, bwd=False):
     return f
 
 
+def step_kernels(wl: synth.Workload, bwd: bool) -> list[str]:
+    """Names of the library's kernels one step launches, in launch order (the
+    library records a timing event after each; see mta_cfg.events)."""
+    if bwd:
+        return ["attn_bwd_post_kernel" if wl.kq_post else "attn_bwd_simt_kernel"]
+    if uses_contraction(wl):
+        attn = ["kq_prep_kernel"] + (["vt_prep_kernel"] if wl.kq_post else []) + ["attn_kq_kernel"]
+    elif uses_direct_tc(wl):
+        attn = ["attn_tc_kernel"]
+    else:
+        attn = ["attn_simt_kernel"] + (["group_norm_kernel"] if wl.layer else [])
+    return ["gemm_qkv"] + attn + ["gemm_out"] if wl.layer else attn
+
+
 def dominant_kernel(wl: synth.Workload, bwd: bool) -> tuple[int, int, str]:
     """(a, b, name): the step's dominant kernel runs between the library's timing
     events a and b of a step (event 0 before the first kernel, event k after the
@@ -442,6 +456,9 @@ def run_mine(args, wl, rank, world, local_rank):
     total_ms = t_begin.elapsed_time(t_end)
     ka, kb, kname = dominant_kernel(wl, args.bwd)
     kernel_ms = [evs[ka].elapsed_time(evs[kb]) for evs in step_ev]
+    names = step_kernels(wl, args.bwd)
+    per_kernel = {f"{i}:{n}": statistics.mean(evs[i].elapsed_time(evs[i + 1]) for evs in step_ev)
+                  for i, n in enumerate(names) if i + 1 < n_ev}
     step_ms = [evs[0].elapsed_time(evs[-1]) for evs in step_ev]
     st = mta.lib().mta_sync_status(ctypes.byref(cfg))
     if st != 0:
@@ -457,6 +474,7 @@ def run_mine(args, wl, rank, world, local_rank):
     if not args.no_epilogue and not args.bwd and rank == 0:
         epi = run_epilogue(mta, dev, stream)
     return {"total_ms": t_max, "region_ms": total_ms, "kernel_ms": statistics.mean(kernel_ms),
+            "per_kernel_ms": per_kernel,
             "kernel": kname, "kernel_calls_ms": statistics.mean(step_ms), "clocks": clocks, "e2e": e2e,
             "warmup": warm, "epilogue": epi}
 
@@ -783,7 +801,7 @@ def main():
                           "mta": fl["mta"] / s / 1e12 / bf16_peak,
                           "peak_tflops": bf16_peak, "peak_source": f"{peak_src} bf16 {peak_kind}"},
         "roofline": roof, "gpu_launches": args.steps * (1 if args.bwd else launches_per_step(wl)),
-        "timed_region_ms": res["region_ms"],
+        "timed_region_ms": res["region_ms"], "per_kernel_ms": res["per_kernel_ms"],
         "clocks": res["clocks"], "e2e": res["e2e"], "epilogue_group_norm": epi,
     }
     if world == 1 and not args.no_cpu:

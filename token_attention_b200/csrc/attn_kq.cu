@@ -73,6 +73,7 @@ constexpr int kSmThreads = 256;
 constexpr int kTmaWarp = 8, kMmaWarp = 9, kTma2Warp = 10;
 constexpr int kBarAll = 1;      // named barrier over both softmax warpgroups
 constexpr int kKqMaxClusters = 160;  // persistent grid: at most this many CTAs (>= SM count)
+constexpr int kItemSlots = 4;        // item ring: indices taken from the queue ahead of their use
 
 template <int D, int CQ, int CK, int MIX, bool EXACT, bool POST>
 struct KGeo {
@@ -119,8 +120,9 @@ struct KGeo {
   // small area: taps [2 items][NSRC][128], per-warp |q| maxima, barriers, TMEM slot, abort flag
   static constexpr int TH_OFF = 0, THP_OFF = 2 * NSRC * 128 * 4;
   static constexpr int QRED_OFF = THP_OFF + (POST ? 2 * 128 * 4 : 0), BAR_OFF = QRED_OFF + 64;
-  static constexpr int TSLOT_OFF = BAR_OFF + 8 * 32, ABORT_OFF = TSLOT_OFF + 8;
-  static constexpr int SMALL_BYTES = (ABORT_OFF + 8 + 255) / 256 * 256;
+  static constexpr int TSLOT_OFF = BAR_OFF + 8 * 40, ABORT_OFF = TSLOT_OFF + 8;
+  static constexpr int ITEMS_OFF = ABORT_OFF + 8;         // the item ring: kItemSlots item indices
+  static constexpr int SMALL_BYTES = (ITEMS_OFF + 16 + 255) / 256 * 256;
   // Kt ring: as many 16 KB stages as the shared memory left over holds (at most 8)
   static constexpr int REST = Q_AREA + V_BYTES + PS_BYTES + DG_BYTES + NSRC * U_BYTES + CS_BYTES +
                               RED_BYTES + FAC_BYTES + SMALL_BYTES + 1024;
@@ -143,9 +145,13 @@ struct KGeo {
   // at least half the SM's shared memory: one CTA per SM, so the 512-column TMEM
   // allocation never waits for another CTA
   static constexpr int SMEM = SMEM_USED > 232448 / 2 + 1024 ? SMEM_USED : 232448 / 2 + 1024;
-  // tensor memory: C of each source head (128 columns each), P (64), Z
-  static constexpr uint32_t TMEM_COLS = 512, C_COL = 0, P_COL = 128 * NSRC;
-  static constexpr uint32_t Z_COL0 = POST ? P_COL : P_COL + 128;  // P lives in shared memory with POST
+  // tensor memory.  DB (one source head, no post-softmax convolution): C in two
+  // 128-column buffers used by alternate key tiles, each tile's P (bf16, 64
+  // columns) written over its own C, then Z.  Otherwise: C of each source head (128
+  // columns each), P (64), Z (P lives in shared memory with POST).
+  static constexpr bool DB = !POST && NSRC == 1;
+  static constexpr uint32_t TMEM_COLS = 512, C_COL = 0, P_COL = DB ? 0 : 128 * NSRC;
+  static constexpr uint32_t Z_COL0 = DB ? 256 : POST ? P_COL : P_COL + 128;
   static_assert(Z_COL0 + 128 * (NV - 1) + D <= TMEM_COLS, "tensor memory");
   static_assert(MIX != 1 || NV == 1, "pre-softmax mixing uses the destination head's V only");
   static_assert(OFF_K % 1024 == 0 && OFF_V % 1024 == 0, "swizzle alignment");
@@ -153,7 +159,7 @@ struct KGeo {
   static_assert(OFF_SMALL % 16 == 0, "alignment");
   static_assert(NS >= 3, "Kt ring");
   static_assert(NCH % SB == 0 && NDC % SB == 0, "whole stages");
-  static_assert(11 + 2 * NS <= 32, "barrier slots");
+  static_assert(13 + 2 * NS <= 32, "barrier slots (32 .. 39: the item ring)");
   static_assert(SMEM <= 232448, "shared memory");
   static_assert(CQ * CK <= 120, "kernel taps");
   static_assert(CQ * D % 64 == 0 && D % 16 == 0, "contraction chunks");
@@ -177,6 +183,8 @@ struct KqParams {
   const float *theta_post;    // [H][CQ][CK]
   const __nv_bfloat16 *v;     // [B][L][H][D], token stride rs
   long long rs;
+  unsigned *queue;            // work-queue counter (zero when the launch starts)
+  int wave;                   // units (batch, head group) per wave of the item order
 };
 
 template <int N>
@@ -191,22 +199,25 @@ __device__ __forceinline__ float tree_max(const float (&x)[N]) {
   return m[0];
 }
 
-// Work item k of a cluster (longest first: query tile qt descending, then batch and
-// head group); clusters take items in a snake order over rounds of n_clusters.
+// Work item k of the launch: (query tile qt, batch b, head group g).  The units
+// (b, g) are taken in waves of `wave` units (as many as keep their convolved keys
+// resident in L2 together); inside a wave, items go longest first (query tile
+// descending), then by unit.  The clusters take items from a queue in this order,
+// so the clusters running at any time read the keys of a few units, and the
+// shortest items come last.
 struct Item {
   int qt, b, g;
 };
-__device__ __forceinline__ Item item_of(int k, int B, int G, int n_qtiles) {
-  const int per_qt = B * G;
+__device__ __forceinline__ Item item_of(int k, int B, int G, int n_qtiles, int wave) {
+  const int per_wave = wave * n_qtiles;
+  const int w = k / per_wave, r = k - w * per_wave;
+  const int nu = min(wave, B * G - w * wave);  // units of this wave (the last may have fewer)
+  const int unit = w * wave + r % nu;
   Item it;
-  it.qt = n_qtiles - 1 - k / per_qt;
-  const int rem = k % per_qt;
-  it.b = rem / G;
-  it.g = rem % G;
+  it.qt = n_qtiles - 1 - r / nu;
+  it.b = unit / G;
+  it.g = unit % G;
   return it;
-}
-__device__ __forceinline__ int item_index(int c, int r, int n_clusters) {
-  return r * n_clusters + ((r & 1) ? n_clusters - 1 - c : c);
 }
 
 template <int D, int CQ, int CK, int MIX, bool EXACT, bool POST>
@@ -235,22 +246,57 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t *x_ready = bars + 4, *k_full = bars + 5, *k_empty = bars + 5 + G::NS;
   uint64_t *v_full = bars + 5 + 2 * G::NS, *v_empty = v_full + 1, *c_full = v_full + 2;
   uint64_t *c_free = v_full + 3, *p_full = v_full + 4, *mma_done = v_full + 5;
+  // DB: C complete and P written, per buffer (tile T uses buffer T & 1)
+  uint64_t *const c_fullb[2] = {c_full, v_full + 6};
+  uint64_t *const p_fullb[2] = {p_full, v_full + 7};
   uint32_t *tslot = reinterpret_cast<uint32_t *>(small + G::TSLOT_OFF);
   volatile int *abort_flag = reinterpret_cast<volatile int *>(small + G::ABORT_OFF);
+  // item ring: it_full[s] completes when slot s holds the next item index (or -1 at
+  // the end); it_empty[s] (in the cluster's first CTA) when every consumer of both
+  // CTAs has read it
+  uint64_t *it_full = bars + 32, *it_empty = bars + 36;
+  volatile int *item_slot = reinterpret_cast<volatile int *>(small + G::ITEMS_OFF);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   // cluster c (the two heads of a group with post-softmax mixing, else one CTA)
   const int hr = MIX == 2 ? static_cast<int>(blockIdx.x) : 0;
-  const int c = static_cast<int>(blockIdx.y), n_clusters = static_cast<int>(gridDim.y);
+  const int c = static_cast<int>(blockIdx.y);  // this cluster's slot of the exchange buffer
   constexpr int CL = MIX == 2 ? 2 : 1;
   const int n_groups = p.H / CL;
   const int n_items = p.B * n_groups * p.n_qtiles;
   const int L = p.L;
-  // this cluster's items: item_index(c, r) for r = 0, 1, ... while below n_items
-  auto item_at = [&](int r, Item &it) -> bool {
-    const int k = item_index(c, r, n_clusters);
-    if (k >= n_items) return false;
-    it = item_of(k, p.B, n_groups, p.n_qtiles);
+  // Consumers of the item ring: the r-th item of this cluster (r = 0, 1, ...), or
+  // false at the end of the queue (or after an abort).  Every consumer thread waits;
+  // one arrival per consumer (lane 0 of a warp, or a single thread) frees the slot.
+  auto take_item = [&](int r, Item &it, bool arrive) -> bool {
+    const int s = r % kItemSlots;
+    const bool ok = mbar_wait_cluster(it_full + s, (r / kItemSlots) & 1, abort_flag, p.err);
+    const int k = ok ? item_slot[s] : -1;
+    if (ok && arrive) {
+      if (CL == 2 && hr != 0)
+        mbar_arrive_cluster(map_peer(smem_u32(it_empty + s), 0u));
+      else
+        mbar_arrive(it_empty + s);
+    }
+    if (k < 0) return false;
+    it = item_of(k, p.B, n_groups, p.n_qtiles, p.wave);
+    return true;
+  };
+  // The producer (the cluster's first CTA, TMA warp lane 0): takes the next index
+  // from the queue and publishes it to both CTAs' rings; -1 once the queue is empty.
+  auto publish_item = [&](int r, Item &it) -> bool {
+    const int s = r % kItemSlots;
+    if (!mbar_wait_cluster(it_empty + s, ((r / kItemSlots) & 1) ^ 1, abort_flag, p.err)) return false;
+    int k = static_cast<int>(atomicAdd(p.queue, 1u));
+    if (k >= n_items) k = -1;
+    item_slot[s] = k;
+    if (CL == 2) {
+      st_cluster_s32(map_peer(smem_u32(const_cast<int *>(item_slot + s)), 1u), k);
+      mbar_arrive_cluster(map_peer(smem_u32(it_full + s), 1u));  // releases the store above
+    }
+    mbar_arrive(it_full + s);
+    if (k < 0) return false;
+    it = item_of(k, p.B, n_groups, p.n_qtiles, p.wave);
     return true;
   };
   // first query row of an item's tile (with POST, its c_q-1 rows above the output rows)
@@ -267,6 +313,14 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int s = 0; s < G::NS; ++s) { mbar_init(k_full + s, 1); mbar_init(k_empty + s, 1); }
     mbar_init(v_full, 1); mbar_init(v_empty, 1); mbar_init(c_full, 1); mbar_init(c_free, 8);
     mbar_init(p_full, 8); mbar_init(mma_done, 1);
+    mbar_init(c_fullb[1], 1); mbar_init(p_fullb[1], 8);
+    // consumers per item: the V and query loaders, the MMA thread and the 8 softmax
+    // warps of each CTA, and the second CTA's key loader (no V loader with POST)
+    constexpr int per_cta = (POST ? 1 : 2) + 1 + 8;
+    for (int s = 0; s < kItemSlots; ++s) {
+      mbar_init(it_full + s, 1);
+      mbar_init(it_empty + s, CL == 2 ? 2 * per_cta + 1 : per_cta);
+    }
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -280,6 +334,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (MIX == 2) cluster_sync_all();  // the peer's barriers are initialised before remote arrivals
   tc_fence_after();
   const uint32_t tmem = *tslot;
+  // launched as the prepasses' programmatic dependent: everything above overlapped
+  // their tail; from here on their outputs (convolved keys and values, column
+  // factors, dot products) are complete and visible
+  pdl_wait_primary();
 
   if (warp == kTmaWarp || warp == kTma2Warp) {
     // -------------------------------------------------------------- TMA
@@ -300,7 +358,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       };
       Item it;
       bool ok = true;
-      for (int r = 0; ok && item_at(r, it) && !*abort_flag; ++r) {
+      // the cluster's first CTA takes the items from the queue; the second reads them
+      for (int r = 0; ok && !*abort_flag && (hr == 0 ? publish_item(r, it) : take_item(r, it, true)); ++r) {
         const int h = it.g * CL + hr, n_kv = kv_tiles(it), nsl = n_slots(it);
         auto load_c = [&](int t) -> bool {
           for (int ch = 0; ch < G::NSRC * G::NCH; ch += G::SB) {
@@ -343,7 +402,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       prefetch_tmap(&tmV);
       int nv = 0;
       Item it;
-      for (int r = 0; item_at(r, it) && !*abort_flag; ++r) {
+      for (int r = 0; !*abort_flag && take_item(r, it, true); ++r) {
         const int h = it.g * CL + hr, n_kv = kv_tiles(it);
         for (int t = 0; t < n_kv; ++t, ++nv) {
           if (!mbar_wait(v_empty, (nv & 1) ^ 1, abort_flag, p.err)) break;
@@ -361,7 +420,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       prefetch_tmap(&tmQ);
       int nq = 0;
       Item it;
-      for (int r = 0; item_at(r, it) && !*abort_flag; ++r, ++nq) {
+      for (int r = 0; !*abort_flag && take_item(r, it, true); ++r, ++nq) {
         if (r > 0 && !mbar_wait(q_free, (r - 1) & 1, abort_flag, p.err)) break;
         const int h = it.g * CL + hr, row0 = row_start(it) - G::HALO;
         mbar_arrive_expect_tx(q_full, G::NSRC * G::Q_BYTES);
@@ -393,8 +452,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       bool ok = true;
       // C of global key tile T = sum over the NCH 64-element chunks of the c_q*D
       // contraction; element kappa = a*D + e pairs Q shifted by a rows with Kt_a
+      // DB: into buffer T & 1 without waiting for the softmax (the buffer's previous
+      // tile, T - 2, had its P V issued before, and MMAs run in issue order)
       auto issue_c = [&](bool last_of_item) -> bool {
-        if (T > 0 && !mbar_wait(c_free, (T - 1) & 1, abort_flag, p.err)) return false;
+        if (!G::DB && T > 0 && !mbar_wait(c_free, (T - 1) & 1, abort_flag, p.err)) return false;
+        const uint32_t c_dst = tmem + G::C_COL + (G::DB ? 128u * (T & 1) : 0u);
         for (int ch = 0; ch < G::NSRC * G::NCH; ch += G::SB, ++cnt) {
           const int st = cnt % G::NS;
           // source head sc (its own accumulator and query rows); the 16 elements
@@ -414,7 +476,7 @@ __global__ void __launch_bounds__(kThreads, 1)
               const uint64_t qd = qdesc0 + static_cast<uint32_t>((sc * G::Q_ALLOC + 8 * dc * G::STRIP + 16 * (G::HALO - a)) >> 4);
 #pragma unroll
               for (int kk = 0; kk < 4; ++kk)
-                mma_bf16_ss(tmem + G::C_COL + 128 * sc, qd + (2 * kk * G::STRIP >> 4),
+                mma_bf16_ss(c_dst + 128 * sc, qd + (2 * kk * G::STRIP >> 4),
                             kd + (bx * G::KCHUNK >> 4) + 2 * kk, idesc_c, (cs > 0 || kk > 0));
             }
           } else {
@@ -430,11 +492,11 @@ __global__ void __launch_bounds__(kThreads, 1)
             tc_fence_after();
 #pragma unroll
             for (int kk = 0; kk < 4; ++kk)
-              mma_bf16_ss(tmem + G::C_COL + 128 * sc, qd[kk], kd + 2 * kk, idesc_c, (cs > 0 || kk > 0));
+              mma_bf16_ss(c_dst + 128 * sc, qd[kk], kd + 2 * kk, idesc_c, (cs > 0 || kk > 0));
           }
           mma_commit(k_empty + st);
         }
-        mma_commit(c_full);
+        mma_commit(G::DB ? c_fullb[T & 1] : c_full);
         if (last_of_item) mma_commit(q_free);  // the query buffer may take the next item
         return true;
       };
@@ -473,9 +535,47 @@ __global__ void __launch_bounds__(kThreads, 1)
         return true;
       };
       Item it;
-      for (int r = 0; ok && item_at(r, it); ++r) {
+      for (int r = 0; ok && take_item(r, it, true); ++r) {
         const int n_kv = kv_tiles(it), nsl = n_slots(it);
         if (!mbar_wait(q_ready, r & 1, abort_flag, p.err)) break;
+        if constexpr (G::DB) {
+          // C of the first two tiles, then per tile: P V, and C two tiles ahead into
+          // the buffer that P V has just consumed
+          const int T0 = T;
+          ok = issue_c(nsl == 1);
+          if (ok && nsl > 1) {
+            T = T0 + 1;
+            ok = issue_c(nsl == 2);
+          }
+          for (int sl = 0; ok && sl < nsl; ++sl) {
+            const int Tt = T0 + sl;
+            if (!mbar_wait(p_fullb[Tt & 1], (Tt >> 1) & 1, abort_flag, p.err)) { ok = false; break; }
+            if (!mbar_wait(v_full, Tt & 1, abort_flag, p.err)) { ok = false; break; }
+            if (sl == 0 && r > 0 && !mbar_wait(z_free, (r - 1) & 1, abort_flag, p.err)) { ok = false; break; }
+            tc_fence_after();
+            const uint32_t pcol = tmem + 128u * (Tt & 1);
+            if constexpr (G::NV * G::NDC * 64 == 256) {
+#pragma unroll
+              for (int kk = 0; kk < G::BN / 16; ++kk)
+                mma_f16_ts(tmem + G::Z_COL0, pcol + 8 * kk, vdesc0 + ((kk * 16 * 128) >> 4),
+                           idesc_bf16_f32(128, 256, 0, 1), (sl > 0 || kk > 0));
+            } else {
+#pragma unroll
+              for (int hd = 0; hd < G::NV; ++hd)
+#pragma unroll
+                for (int kk = 0; kk < G::BN / 16; ++kk)
+                  mma_f16_ts(tmem + G::Z_COL0 + 128 * hd, pcol + 8 * kk,
+                             vdesc0 + ((hd * G::V_HEAD + kk * 16 * 128) >> 4), idesc_pv, (sl > 0 || kk > 0));
+            }
+            mma_commit(v_empty);
+            if (sl + 2 < nsl) {
+              T = Tt + 2;
+              ok = issue_c(sl + 3 == nsl);
+            }
+          }
+          T = T0 + nsl;
+          continue;
+        }
         const int T0 = T;
         ok = issue_c(nsl == 1);
         for (int sl = 0; ok && sl < nsl; ++sl) {
@@ -594,7 +694,20 @@ __global__ void __launch_bounds__(kThreads, 1)
     int T = 0;   // C tiles processed so far (all items, both passes with POST)
     int NP = 0;  // weight tiles handed to the P V issuer so far (POST)
     Item it, nx;
-    bool have = item_at(0, it);
+    // every softmax thread reads the ring; lane 0 of each warp frees the slot
+    auto take_sm = [&](int r, Item &x) -> bool {
+      const bool got = take_item(r, x, false);
+      __syncwarp();
+      if (lane == 0) {
+        const int s = r % kItemSlots;
+        if (CL == 2 && hr != 0)
+          mbar_arrive_cluster(map_peer(smem_u32(it_empty + s), 0u));
+        else
+          mbar_arrive(it_empty + s);
+      }
+      return got;
+    };
+    bool have = take_sm(0, it);
     int eq = 0;
     if (have) {
       eq = prepare(0, it);
@@ -611,15 +724,20 @@ __global__ void __launch_bounds__(kThreads, 1)
       const bool row_ok = qi >= 0 && qi < L;          // a query of the sequence
       const bool out_row = row_ok && r_ >= G::RSH;     // an output row of this tile
       const int n_kv = kv_tiles(it), nsl = n_slots(it);
-      const bool more = item_at(r + 1, nx);
-      const int h_nx = nx.g * CL + hr;
-      // column factors of source s for the key tile of the slot after sl (this
-      // item's or the next item's first)
+      // the next item, read from the ring at this item's last key tile
+      bool more = false, nx_known = false;
+      auto fetch_next = [&]() {
+        if (!nx_known) {
+          more = take_sm(r + 1, nx);
+          nx_known = true;
+        }
+      };
+      // column factors of source s for the key tile of the slot after sl (this item's;
+      // the next item's first tile's are loaded after the slot loop)
       auto fac_next = [&](int sc, int sl) -> float {
         if (sl + 1 < nsl)
           return p.fac[(static_cast<long long>(it.b) * p.H + src_head(h, sc)) * p.lpad +
                        (POST ? (sl + 1) % n_kv : sl + 1) * G::BN + st_id];
-        if (more) return p.fac[(static_cast<long long>(nx.b) * p.H + src_head(h_nx, sc)) * p.lpad + st_id];
         return 0.f;
       };
       const float qinv = exp2f(static_cast<float>(-eq));
@@ -672,8 +790,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         float fnext[G::NSRC];
 #pragma unroll
         for (int sc = 0; sc < G::NSRC; ++sc) fnext[sc] = st_id < G::BN ? fac_next(sc, sl) : 0.f;
-        mbar_wait(c_full, T & 1, abort_flag, p.err);
+        if constexpr (G::DB)
+          mbar_wait(c_fullb[T & 1], (T >> 1) & 1, abort_flag, p.err);
+        else
+          mbar_wait(c_full, T & 1, abort_flag, p.err);
         tc_fence_after();
+        const uint32_t cbuf = G::DB ? 128u * (T & 1) : 0u;  // this tile's C (and, with DB, P) buffer
         // C' = sum over source heads of w * (C_s x its column factors); one source without mixing
         float cv[G::HALF];
 #pragma unroll
@@ -682,7 +804,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
           for (int c0 = 0; c0 < G::HALF; c0 += 32) {
             uint32_t u32[32];
-            tmem_ld32(tl + G::C_COL + 128 * sc + cb + c0, u32);
+            tmem_ld32(tl + G::C_COL + cbuf + 128 * sc + cb + c0, u32);
             float4 f[8];
 #pragma unroll
             for (int i = 0; i < 8; ++i) {
@@ -701,9 +823,11 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
           }
         }
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(c_free);
+        tc_fence_before();  // (with DB: orders the C reads before the barrier that precedes the P writes)
+        if constexpr (!G::DB) {  // with DB the buffer is reused only after this tile's P V
+          __syncwarp();
+          if (lane == 0) mbar_arrive(c_free);
+        }
         if (eq != 0) {  // queries were scaled down (|q| > 2^14)
 #pragma unroll
           for (int jj = 0; jj < G::HALF; ++jj) cv[jj] *= qinv;
@@ -734,6 +858,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
             for (int sc = 0; sc < G::NSRC; ++sc) facs[(sc * 2 + ((T + 1) & 1)) * G::BN + st_id] = fnext[sc];
           named_bar_sync(kBarAll, kSmThreads);
+          tc_fence_after();  // both warpgroups have read this tile's C (P may overwrite it)
           const float mt = fmaxf(rmx[r_], rmx[G::BM + r_]);
           const float m_new = fmaxf(m_run, mt);
           if constexpr (POST) {  // first pass: row sums only
@@ -783,12 +908,13 @@ __global__ void __launch_bounds__(kThreads, 1)
               ls += p0 + p1;
               pk[q2] = pack_bf16x2(p0, p1);
             }
-            tmem_st32(tl + G::P_COL + 32 * wg, pk);
+            // (with DB, over this tile's C: both warpgroups have read it, see the barrier above)
+            tmem_st32(tl + G::P_COL + cbuf + 32 * wg, pk);
             l_run += ls;
             tmem_wait_st();
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive(p_full);
+            if (lane == 0) mbar_arrive(G::DB ? p_fullb[T & 1] : p_full);
           }
         } else {
           // second pass: normalised weights A = 2^(C - mm); the c keys ending at the
@@ -832,6 +958,17 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
       // the next item's queries, dot products and taps, while this item's last P V runs
+      // The next item, taken from the ring only now: its index may be published only
+      // after the key loader has issued this item's last loads, which (with POST) are
+      // the convolved values its last weights are multiplied by.  Its first key
+      // tile's column factors go to the factor buffer of tile T (the barriers of
+      // prepare() and of the epilogue order them before that tile reads them).
+      fetch_next();
+      if (more && st_id < G::BN)
+#pragma unroll
+        for (int sc = 0; sc < G::NSRC; ++sc)
+          facs[(sc * 2 + (T & 1)) * G::BN + st_id] =
+              p.fac[(static_cast<long long>(nx.b) * p.H + src_head(nx.g * CL + hr, sc)) * p.lpad + st_id];
       const int eq_next = more ? prepare(r + 1, nx) : 0;
 
       // ---------------------------------------------------------- epilogue
@@ -1044,6 +1181,15 @@ cudaError_t launch_kq_one(const AttnArgs &a, const GnArgs *gn, const KqPrepArgs 
   p.theta_post = a.theta_post;
   p.v = static_cast<const __nv_bfloat16 *>(a.v);
   p.rs = a.rs;
+  p.queue = a.err + 3;  // zeroed with the error word before every call
+  {
+    // units (batch, head group) per wave: as many as keep the convolved keys they read
+    // (c_q*L*d fp16 per source head, both heads of a group) within a quarter of L2
+    const long long unit_bytes = static_cast<long long>(CQ) * a.L * D * 2 * (G::CLUSTER == 2 || G::NSRC == 2 ? 2 : 1);
+    const long long units = static_cast<long long>(a.B) * (a.H / G::CLUSTER);
+    const long long w = (32ll << 20) / unit_bytes;
+    p.wave = static_cast<int>(std::max<long long>(1, std::min<long long>(w, units)));
+  }
   auto kern = attn_kq_kernel<D, CQ, CK, MIX, EXACT, POST>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, G::SMEM);
   if (e != cudaSuccess) return e;
@@ -1054,11 +1200,14 @@ cudaError_t launch_kq_one(const AttnArgs &a, const GnArgs *gn, const KqPrepArgs 
   cfg.blockDim = dim3(kThreads);
   cfg.dynamicSmemBytes = G::SMEM;
   cfg.stream = a.stream;
-  cudaLaunchAttribute attr[1];
+  cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeClusterDimension;
   attr[0].val.clusterDim.x = G::CLUSTER;  // the two heads of a group
   attr[0].val.clusterDim.y = 1;
   attr[0].val.clusterDim.z = 1;
+  // programmatic dependent of the prepass launched just before it on this stream
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   cfg.gridDim = dim3(G::CLUSTER, kKqMaxClusters / G::CLUSTER);
@@ -1068,6 +1217,7 @@ cudaError_t launch_kq_one(const AttnArgs &a, const GnArgs *gn, const KqPrepArgs 
   if (resident < 1) return cudaErrorInvalidConfiguration;
   const long long nc = std::min<long long>(std::min<long long>(resident, n_items), kKqMaxClusters / G::CLUSTER);
   cfg.gridDim = dim3(G::CLUSTER, static_cast<unsigned>(nc));
+  cfg.numAttrs = 2;
   return cudaLaunchKernelEx(&cfg, kern, tq, tk, tv, tvt, p);
 }
 

@@ -25,9 +25,11 @@ __device__ __forceinline__ float warp_sum(float x) {
 }
 
 // d = 128: 16 lanes per (token, head) row, 8 channels (16 bytes) per lane, so a
-// warp covers two rows; each warp loads kRowsAhead row pairs before it reduces
-// any of them, so that enough bytes are in flight to keep HBM busy.
-constexpr int kRowsAhead = 4;
+// warp covers two rows; a block of 8 warps covers 16 consecutive rows per step and
+// kRowsAhead steps.  Every load of a thread is issued before it reduces any row,
+// so that enough bytes are in flight to keep HBM busy; one block per 16*kRowsAhead
+// rows, no grid-stride loop, 32-bit row indices.
+constexpr int kRowsAhead = 8;
 
 __device__ __forceinline__ float half_warp_sum(float x) {
 #pragma unroll
@@ -35,56 +37,53 @@ __device__ __forceinline__ float half_warp_sum(float x) {
   return x;
 }
 
-__global__ void __launch_bounds__(256) group_norm_d128_kernel(const __nv_bfloat16 *__restrict__ o,
-                                                              GnArgs gn, long long rows, int H,
-                                                              __nv_bfloat16 *__restrict__ y) {
-  const int lane = threadIdx.x & 31, half = lane >> 4, hl = lane & 15;
-  const long long warp = (static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
-  const long long nwarps = (static_cast<long long>(gridDim.x) * blockDim.x) >> 5;
-  // the loop bound is the same for both halves of a warp (every lane reaches
-  // every shuffle); a half whose row is past the end works on zeros
-  for (long long pb = 2 * warp; pb < rows; pb += 2 * nwarps * kRowsAhead) {
-    uint4 raw[kRowsAhead];
-    long long rr[kRowsAhead];
+__global__ void __launch_bounds__(256, 4) group_norm_d128_kernel(const __nv_bfloat16 *__restrict__ o,
+                                                                 GnArgs gn, int rows, int H,
+                                                                 __nv_bfloat16 *__restrict__ y) {
+  const int lane = threadIdx.x & 31, hl = lane & 15;
+  const int row0 = blockIdx.x * 16 * kRowsAhead + 2 * (threadIdx.x >> 5) + (lane >> 4);
+  uint4 raw[kRowsAhead];
 #pragma unroll
-    for (int u = 0; u < kRowsAhead; ++u) {
-      rr[u] = pb + 2 * nwarps * u + half;
-      raw[u] = rr[u] < rows ? reinterpret_cast<const uint4 *>(o + rr[u] * 128)[hl] : make_uint4(0u, 0u, 0u, 0u);
+  for (int u = 0; u < kRowsAhead; ++u) {
+    const int r = row0 + 16 * u;
+    raw[u] = r < rows ? reinterpret_cast<const uint4 *>(o + static_cast<long long>(r) * 128)[hl]
+                      : make_uint4(0u, 0u, 0u, 0u);
+  }
+#pragma unroll
+  for (int u = 0; u < kRowsAhead; ++u) {
+    const int r = row0 + 16 * u;
+    const uint32_t wv[4] = {raw[u].x, raw[u].y, raw[u].z, raw[u].w};
+    float x[8];
+    float s = 0.f;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      x[2 * i] = __uint_as_float(wv[i] << 16);
+      x[2 * i + 1] = __uint_as_float(wv[i] & 0xffff0000u);
+      s += x[2 * i] + x[2 * i + 1];
     }
+    // both halves of the warp take every shuffle (a row past the end works on zeros)
+    const float mu = half_warp_sum(s) * (1.f / 128.f);
+    float s2 = 0.f;
 #pragma unroll
-    for (int u = 0; u < kRowsAhead; ++u) {
-      const uint32_t wv[4] = {raw[u].x, raw[u].y, raw[u].z, raw[u].w};
-      float x[8];
-      float s = 0.f;
+    for (int i = 0; i < 8; ++i) { x[i] -= mu; s2 += x[i] * x[i]; }
+    const float rstd = rsqrtf(half_warp_sum(s2) * (1.f / 128.f) + gn.eps);
+    if (r >= rows) continue;
+    const int h = r % H;
+    const float4 *g4 = reinterpret_cast<const float4 *>(gn.gamma + h * 128 + 8 * hl);
+    const float4 *b4 = reinterpret_cast<const float4 *>(gn.beta + h * 128 + 8 * hl);
+    const float4 ga = __ldg(g4), gb = __ldg(g4 + 1), ba = __ldg(b4), bb = __ldg(b4 + 1);
+    const float g[8] = {ga.x, ga.y, ga.z, ga.w, gb.x, gb.y, gb.z, gb.w};
+    const float b[8] = {ba.x, ba.y, ba.z, ba.w, bb.x, bb.y, bb.z, bb.w};
+    const float m = head_multiplier(gn.gate, gn.lam, h);
+    uint4 outw;
+    uint32_t *ow = reinterpret_cast<uint32_t *>(&outw);
 #pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        x[2 * i] = __uint_as_float(wv[i] << 16);
-        x[2 * i + 1] = __uint_as_float(wv[i] & 0xffff0000u);
-        s += x[2 * i] + x[2 * i + 1];
-      }
-      const float mu = half_warp_sum(s) * (1.f / 128.f);
-      float s2 = 0.f;
-#pragma unroll
-      for (int i = 0; i < 8; ++i) { x[i] -= mu; s2 += x[i] * x[i]; }
-      const float rstd = rsqrtf(half_warp_sum(s2) * (1.f / 128.f) + gn.eps);
-      if (rr[u] >= rows) continue;
-      const int h = static_cast<int>(rr[u] % H);
-      const float4 *g4 = reinterpret_cast<const float4 *>(gn.gamma + h * 128 + 8 * hl);
-      const float4 *b4 = reinterpret_cast<const float4 *>(gn.beta + h * 128 + 8 * hl);
-      const float4 ga = g4[0], gb = g4[1], ba = b4[0], bb = b4[1];
-      const float g[8] = {ga.x, ga.y, ga.z, ga.w, gb.x, gb.y, gb.z, gb.w};
-      const float b[8] = {ba.x, ba.y, ba.z, ba.w, bb.x, bb.y, bb.z, bb.w};
-      const float m = head_multiplier(gn.gate, gn.lam, h);
-      uint4 outw;
-      uint32_t *ow = reinterpret_cast<uint32_t *>(&outw);
-#pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        __nv_bfloat162 q = __floats2bfloat162_rn((x[2 * i] * rstd * g[2 * i] + b[2 * i]) * m,
-                                                 (x[2 * i + 1] * rstd * g[2 * i + 1] + b[2 * i + 1]) * m);
-        ow[i] = *reinterpret_cast<uint32_t *>(&q);
-      }
-      reinterpret_cast<uint4 *>(y + rr[u] * 128)[hl] = outw;
+    for (int i = 0; i < 4; ++i) {
+      __nv_bfloat162 q = __floats2bfloat162_rn((x[2 * i] * rstd * g[2 * i] + b[2 * i]) * m,
+                                               (x[2 * i + 1] * rstd * g[2 * i + 1] + b[2 * i + 1]) * m);
+      ow[i] = *reinterpret_cast<uint32_t *>(&q);
     }
+    reinterpret_cast<uint4 *>(y + static_cast<long long>(r) * 128)[hl] = outw;
   }
 }
 
@@ -130,24 +129,23 @@ cudaError_t launch_group_norm(const void *o, const GnArgs &gn, int tokens, int H
                               cudaStream_t stream) {
   const long long rows = static_cast<long long>(tokens) * H;
   if (rows == 0) return cudaSuccess;
-  int sms = 148;
-  int dev = 0;
-  if (cudaGetDevice(&dev) == cudaSuccess)
-    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   const __nv_bfloat16 *src = static_cast<const __nv_bfloat16 *>(o);
   __nv_bfloat16 *dst = static_cast<__nv_bfloat16 *>(y);
-  const bool vec = d == 128 &&
+  const bool vec = d == 128 && rows < (1ll << 31) - 16 * kRowsAhead &&
                    ((reinterpret_cast<uintptr_t>(gn.gamma) | reinterpret_cast<uintptr_t>(gn.beta)) & 15) == 0 &&
                    ((reinterpret_cast<uintptr_t>(o) | reinterpret_cast<uintptr_t>(y)) & 15) == 0;
-  // d = 128: a block of 8 warps covers 16 rows per step and kRowsAhead steps at once;
-  // otherwise a warp per row.  At most 8 blocks per SM (grid-stride beyond that).
-  const long long per_block = vec ? 16LL * kRowsAhead : 8LL;
-  const long long want = (rows + per_block - 1) / per_block;
-  const int blocks = static_cast<int>(want < 8LL * sms ? want : 8LL * sms);
-  if (vec)
-    group_norm_d128_kernel<<<blocks, 256, 0, stream>>>(src, gn, rows, H, dst);
-  else
+  if (vec) {
+    const long long blocks = (rows + 16 * kRowsAhead - 1) / (16 * kRowsAhead);
+    group_norm_d128_kernel<<<static_cast<unsigned>(blocks), 256, 0, stream>>>(src, gn, static_cast<int>(rows), H,
+                                                                             dst);
+  } else {
+    // a warp per row, grid-stride; at most 8 blocks of 8 warps per SM
+    int sms = 148, dev = 0;
+    if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    const long long want = (rows + 7) / 8;
+    const int blocks = static_cast<int>(want < 8LL * sms ? want : 8LL * sms);
     group_norm_any_kernel<<<blocks, 256, 0, stream>>>(src, gn, rows, H, d, dst);
+  }
   return cudaGetLastError();
 }
 

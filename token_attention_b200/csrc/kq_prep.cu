@@ -36,6 +36,7 @@
 #include <type_traits>
 
 #include "internal.h"
+#include "ptx.cuh"
 
 namespace mta {
 namespace {
@@ -97,6 +98,10 @@ __global__ void __launch_bounds__(kPrepThreads, 3) kq_prep_kernel(KqPrepArgs p) 
   const int L = p.L, j0 = tile * kTile;
   const long long bh = static_cast<long long>(b) * p.H + h;
   const __nv_bfloat16 *kb = static_cast<const __nv_bfloat16 *>(p.k);
+  // the attention kernel (launched as this grid's programmatic dependent) may start
+  // its prologue once every CTA of this grid is running; it waits for this grid's
+  // completion before it reads anything written here
+  pdl_launch_dependents();
   const __nv_bfloat16 *qb = static_cast<const __nv_bfloat16 *>(p.q);
 
   for (int i = tid; i < CQ * CK; i += kPrepThreads) th[i] = p.theta[static_cast<long long>(h) * CQ * CK + i];
@@ -261,6 +266,7 @@ __global__ void __launch_bounds__(kPrepThreads, 3) vt_prep_kernel(VtPrepArgs p) 
   __shared__ float th[CQ * CK];
   const int tile = blockIdx.x, s = blockIdx.y, b = blockIdx.z, tid = threadIdx.x;
   const int L = p.L, j0 = tile * kTile;
+  pdl_launch_dependents();  // as in kq_prep_kernel
   const __nv_bfloat16 *vb = static_cast<const __nv_bfloat16 *>(p.v);
   __nv_bfloat16 *vt = static_cast<__nv_bfloat16 *>(p.vt);
   for (int i = tid; i < CQ * CK; i += kPrepThreads) th[i] = p.theta_post[static_cast<long long>(s) * CQ * CK + i];

@@ -159,8 +159,10 @@ mta_status check_workspace(const mta_cfg *c, size_t need) {
   return MTA_OK;
 }
 
+// Clears the first 16 bytes of the status area: the error word (0), the
+// self-test's counters (1, 2) and the attention kernel's work-queue counter (3).
 mta_status clear_status(const mta_cfg *c) {
-  return cudaMemsetAsync(c->workspace, 0, sizeof(unsigned), static_cast<cudaStream_t>(c->stream)) ==
+  return cudaMemsetAsync(c->workspace, 0, 4 * sizeof(unsigned), static_cast<cudaStream_t>(c->stream)) ==
                  cudaSuccess
              ? MTA_OK
              : MTA_ERR_CUDA;
@@ -413,11 +415,10 @@ mta_status mta_selftest_wait_timeout(const mta_cfg *cfg, unsigned limit_us) {
   if (limit_us < 1 || limit_us > 2000000) return MTA_ERR_INVALID;
   mta_status s = check_workspace(cfg, kStatusBytes);
   if (s != MTA_OK) return s;
-  if ((s = clear_status(cfg)) != MTA_OK) return s;
+  if ((s = clear_status(cfg)) != MTA_OK) return s;  // also zeroes the counters
   // counters of the waits that gave up, after the error word
   unsigned *word = static_cast<unsigned *>(cfg->workspace);
   cudaStream_t st = static_cast<cudaStream_t>(cfg->stream);
-  if (cudaMemsetAsync(word + 1, 0, 2 * sizeof(unsigned), st) != cudaSuccess) return MTA_ERR_CUDA;
   return launch_wait_timeout_selftest(1000ull * limit_us, word, word + 1, st) == cudaSuccess ? MTA_OK
                                                                                               : MTA_ERR_CUDA;
 }
