@@ -159,7 +159,7 @@ __global__ void __launch_bounds__(192, 1)
 // (that memory's bandwidth, not the tensor pipe, bounds the one-CTA kernel).
 // The loads of both CTAs are counted on the first CTA's full barrier; the MMA
 // commits arrive on both CTAs' barriers; each CTA stores its own 128 rows.
-constexpr bool kPairs = false;  // launch the CTA-pair kernel for M >= 256
+constexpr bool kPairs = true;  // launch the CTA-pair kernel for M >= 256
 constexpr int P_STAGES = 6;
 constexpr int P_A_BYTES = 128 * BK * 2;                 // 16 KB
 constexpr int P_B_BYTES = 128 * BK * 2;                 // 16 KB (half of the 256 columns)
