@@ -143,7 +143,7 @@ typedef struct mta_gn {
  * bytes, plus, where the contraction kernel applies, its per-call operands
  * (the convolved keys, c_q*B*H*L*d fp16, their B*H*L fp32 scales,
  * B*H*L*(c_q-1+2*(c_k/2)) fp32 dot products, with post-softmax mixing an
- * exchange buffer of at most 160*2*d*128 fp32 for the kernel's persistent CTAs,
+ * exchange buffer of at most 160*4*d*128 fp32 for the kernel's persistent CTAs,
  * and with kq_post the values convolved by the post-softmax kernels,
  * n_v*c_q*B*H*L*d bf16, n_v = 2 with post-softmax mixing, else 1).
  * With a smaller workspace path 0 uses another kernel. */

@@ -78,7 +78,7 @@ def test_workspace_query(L):
     B, H, Ls, d, cq, M = 2, 4, 64, 64, 6, 6 - 1 + 2 * (11 // 2)
     lpad = -(-Ls // 128) * 128
     items = B * (H // 2) * 1     # (batch, head group, query tile) work items
-    xg = min(160, 2 * items) * 2 * d * 128 * 4   # exchange buffer of the persistent CTAs
+    xg = min(160, 2 * items) * 2 * 2 * d * 128 * 4   # exchange buffer of the persistent CTAs
     kq = up(B * H * cq * Ls * d * 2) + up(B * H * lpad * 4) + up(B * H * Ls * M * 4) + xg
     assert L.mta_attn_workspace_bytes(ctypes.byref(cfg)) == 256 + kq
     t = 2 * 64

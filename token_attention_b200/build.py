@@ -21,7 +21,7 @@ INCLUDE = os.path.join(ROOT, "include")
 BUILD_DIR = os.path.join(ROOT, "_build")
 LIB = os.path.join(HERE, "libmta.so")
 
-SOURCES = ["mta_api.cu", "attn_simt.cu", "attn_tc.cu", "attn_kq.cu", "kq_prep.cu", "gemm_tc.cu",
+SOURCES = ["mta_api.cu", "attn_simt.cu", "attn_tc.cu", "attn_kq.cu", "attn_kq_pair.cu", "kq_prep.cu", "gemm_tc.cu",
            "group_norm.cu", "layer_static.cu", "attn_bwd_simt.cu", "attn_bwd_post_simt.cu",
            "selftest.cu"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]

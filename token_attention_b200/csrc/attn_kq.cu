@@ -150,6 +150,10 @@ struct KGeo {
   // columns) written over its own C, then Z.  Otherwise: C of each source head (128
   // columns each), P (64), Z (P lives in shared memory with POST).
   static constexpr bool DB = !POST && NSRC == 1;
+  // DEFER (DB with post-softmax mixing): an item's epilogue releases Z, parks both
+  // halves (for the peer head and for its own) in the L2 exchange buffer, and
+  // finishes (mixing, group norm, store) only after the next item's first tile
+  static constexpr bool DEFER = DB && MIX == 2;
   static constexpr uint32_t TMEM_COLS = 512, C_COL = 0, P_COL = DB ? 0 : 128 * NSRC;
   static constexpr uint32_t Z_COL0 = DB ? 256 : POST ? P_COL : P_COL + 128;
   static_assert(Z_COL0 + 128 * (NV - 1) + D <= TMEM_COLS, "tensor memory");
@@ -177,7 +181,7 @@ struct KqParams {
   float qk_scale;
   const float *fac;     // [B][H][lpad] s*log2(e)*2^-e_j per convolved key row (0 past L)
   const float *vp;      // [B][H][L][M] past dot products
-  float *xg;            // post-softmax mixing exchange: [CTA][2][D/4][BM] float4
+  float *xg;            // post-softmax mixing exchange: [CTA][2 parities][2 parts][D/4][BM] float4
   unsigned *err;
   // post-softmax convolution: its kernels and the values (for the band near the diagonal)
   const float *theta_post;    // [H][CQ][CK]
@@ -679,9 +683,20 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int hs = src_head(h, sc);
         const long long bh = static_cast<long long>(it.b) * p.H + hs;
         float *us = Us + sc * (G::U_BYTES / 4);
-        for (int e = st_id; e < G::UROWS * G::M; e += kSmThreads) {
-          const int rr = e / G::M, k = e % G::M, iq = row0 + rr;
-          us[e] = (iq >= 0 && iq < L) ? p.vp[(bh * L + iq) * G::M + k] : 0.f;
+        // the staged rows are contiguous in Vp: every load of a thread is issued
+        // before any of them is stored, so their latencies overlap
+        constexpr int NU = (G::UROWS * G::M + kSmThreads - 1) / kSmThreads;
+        const float *vsrc = p.vp + (bh * L + row0) * G::M;
+        float vt[NU];
+#pragma unroll
+        for (int u = 0; u < NU; ++u) {
+          const int e = st_id + u * kSmThreads, iq = row0 + e / G::M;
+          vt[u] = (e < G::UROWS * G::M && iq >= 0 && iq < L) ? vsrc[e] : 0.f;
+        }
+#pragma unroll
+        for (int u = 0; u < NU; ++u) {
+          const int e = st_id + u * kSmThreads;
+          if (e < G::UROWS * G::M) us[e] = vt[u];
         }
         if (st_id < CQ * CK)
           th_s[((r & 1) * G::NSRC + sc) * 128 + st_id] = p.theta[static_cast<long long>(hs) * CQ * CK + st_id];
@@ -689,6 +704,74 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (POST && st_id < CQ * CK)  // the post-softmax kernel of this CTA's head
         thp_s[(r & 1) * 128 + st_id] = p.theta_post[static_cast<long long>(h) * CQ * CK + st_id];
       return eq;
+    };
+
+    // exchange buffer slot of CTA (cluster cc, head rank hh) for items of parity par:
+    // part 0 = for the peer head, part 1 (DEFER) = its own head's part
+    auto xslot = [&](int cc, int hh, int par, int part) -> float4 * {
+      return reinterpret_cast<float4 *>(p.xg) +
+             ((static_cast<long long>(2 * cc + hh) * 2 + par) * 2 + part) * (G::BM * D / 4);
+    };
+    // DEFER: the item whose epilogue is still to be finished
+    bool pend = false;
+    int pend_r = 0;
+    Item pend_it{0, 0, 0};
+    // the rest of item pr's epilogue: its own part plus the peer's, group norm and
+    // depth scale (or gate), bf16 store
+    auto finish = [&](int pr, const Item &pi) {
+      const int ph = pi.g * CL + hr, pg = pi.g;
+      const int pq = row_start(pi) + r_;
+      const bool pout = pq >= 0 && pq < L && r_ >= G::RSH;
+      mbar_wait_cluster(x_ready, pr & 1, abort_flag, p.err);
+      const float4 *own = xslot(c, hr, pr & 1, 1);
+      const float4 *theirs = xslot(c, hr ^ 1, pr & 1, 0);
+      const float w_peer = p.w[pg * 4 + hr * 2 + (hr ^ 1)];
+      float o[G::DH];
+#pragma unroll
+      for (int c4 = 0; c4 < G::DH / 4; ++c4) {
+        float4 x = make_float4(0.f, 0.f, 0.f, 0.f), y = x;
+        if (4 * c4 < zn) {
+          x = own[(zc / 4 + c4) * G::BM + r_];
+          y = theirs[(zc / 4 + c4) * G::BM + r_];
+        }
+        o[4 * c4] = x.x + w_peer * y.x;
+        o[4 * c4 + 1] = x.y + w_peer * y.y;
+        o[4 * c4 + 2] = x.z + w_peer * y.z;
+        o[4 * c4 + 3] = x.w + w_peer * y.w;
+      }
+      if (p.gn) {
+        float s1 = 0.f;
+#pragma unroll
+        for (int i = 0; i < G::DH; ++i) s1 += o[i];  // channels past zn are 0
+        red[(6 + wg) * G::BM + r_] = s1;
+        named_bar_sync(kBarAll, kSmThreads);
+        const float mu = (s1 + red[(6 + (wg ^ 1)) * G::BM + r_]) * (1.f / D);
+        float s2 = 0.f;
+#pragma unroll
+        for (int i = 0; i < G::DH; ++i) { const float x = i < zn ? o[i] - mu : 0.f; s2 += x * x; }
+        red[(8 + wg) * G::BM + r_] = s2;
+        named_bar_sync(kBarAll, kSmThreads);
+        const float rstd = rsqrtf((s2 + red[(8 + (wg ^ 1)) * G::BM + r_]) * (1.f / D) + p.eps);
+        const float *gm = p.gamma + static_cast<long long>(ph) * D + zc;
+        const float *bt = p.beta + static_cast<long long>(ph) * D + zc;
+        const float mh = head_multiplier(p.gate, p.lam, ph);
+#pragma unroll
+        for (int i = 0; i < G::DH; ++i)
+          if (i < zn) o[i] = ((o[i] - mu) * rstd * gm[i] + bt[i]) * mh;
+      }
+      if (pout) {
+        __nv_bfloat16 *dst = p.out + ((static_cast<long long>(pi.b) * L + pq) * p.H + ph) * D + zc;
+#pragma unroll
+        for (int i = 0; i < G::DH; i += 8) {
+          if (i >= zn) break;
+          uint4 v;
+          v.x = pack_bf16x2(o[i], o[i + 1]);
+          v.y = pack_bf16x2(o[i + 2], o[i + 3]);
+          v.z = pack_bf16x2(o[i + 4], o[i + 5]);
+          v.w = pack_bf16x2(o[i + 6], o[i + 7]);
+          *reinterpret_cast<uint4 *>(dst + i) = v;
+        }
+      }
     };
 
     int T = 0;   // C tiles processed so far (all items, both passes with POST)
@@ -915,6 +998,13 @@ __global__ void __launch_bounds__(kThreads, 1)
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(G::DB ? p_fullb[T & 1] : p_full);
+            if constexpr (G::DEFER) {
+              // the previous item's epilogue, while this tile's P V and the next C run
+              if (pend && sl == 0) {
+                finish(pend_r, pend_it);
+                pend = false;
+              }
+            }
           }
         } else {
           // second pass: normalised weights A = 2^(C - mm); the c keys ending at the
@@ -1032,11 +1122,41 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       };
       float o[G::DH];
-      if constexpr (MIX == 2) {
+      if constexpr (G::DEFER) {
+        // Z_{h->peer} / l_h and w_own * Z_{h->h} / l_h go to the L2 exchange buffer;
+        // Z is released at once, the rest of the epilogue waits for finish()
+        float4 *mine = xslot(c, hr, r & 1, 0), *own = xslot(c, hr, r & 1, 1);
+        const float w_own = p.w[g * 4 + hr * 2 + hr];
+#pragma unroll
+        for (int c0 = 0; c0 < G::DH; c0 += 32) {
+          if (c0 >= zn) break;
+          float zo[32];
+          z_chunk(hr ^ 1, 2 * g + (hr ^ 1), c0, zo);
+#pragma unroll
+          for (int i = 0; i < 32; i += 4)
+            mine[((zc + c0 + i) / 4) * G::BM + r_] = make_float4(zo[i], zo[i + 1], zo[i + 2], zo[i + 3]);
+          z_chunk(hr, 2 * g + hr, c0, zo);
+#pragma unroll
+          for (int i = 0; i < 32; i += 4)
+            own[((zc + c0 + i) / 4) * G::BM + r_] =
+                make_float4(w_own * zo[i], w_own * zo[i + 1], w_own * zo[i + 2], w_own * zo[i + 3]);
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(z_free);  // the next item's first P V may overwrite Z
+        // every thread's stores are released to the peer by its own arrival
+        mbar_arrive_cluster(map_peer(smem_u32(x_ready), static_cast<uint32_t>(hr ^ 1)));
+        pend = true;
+        pend_r = r;
+        pend_it = it;
+        have = more;
+        it = nx;
+        eq = eq_next;
+        continue;
+      } else if constexpr (MIX == 2) {
         // Z_{h->peer} / l_h goes to the peer through L2: [parity][column/4][row] float4
-        float4 *mine = reinterpret_cast<float4 *>(p.xg) + (static_cast<long long>(2 * c + hr) * 2 + (r & 1)) * (G::BM * D / 4);
-        const float4 *theirs = reinterpret_cast<const float4 *>(p.xg) +
-                               (static_cast<long long>(2 * c + (hr ^ 1)) * 2 + (r & 1)) * (G::BM * D / 4);
+        float4 *mine = xslot(c, hr, r & 1, 0);
+        const float4 *theirs = xslot(c, hr ^ 1, r & 1, 0);
 #pragma unroll
         for (int c0 = 0; c0 < G::DH; c0 += 32) {
           if (c0 >= zn) break;
@@ -1117,6 +1237,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       have = more;
       it = nx;
       eq = eq_next;
+    }
+    if constexpr (G::DEFER) {
+      if (pend) finish(pend_r, pend_it);  // the last item's epilogue
     }
   }
   tc_fence_before();
@@ -1245,18 +1368,20 @@ size_t kq_items(int B, int H, int L, int kqp) {
 
 // Workspace of the contraction path: Kt [B][H][c_q*d/64][L][64] fp16 | fac [B][H][Lpad] fp32 |
 // Vp [B][H][L][M] fp32 | (post-softmax mixing) the exchange buffer of the persistent
-// CTAs, [CTAs][2][d][128] fp32 | (post-softmax convolution) the convolved values
+// CTAs, [CTAs][2 parities][2 parts][d][128] fp32 | (post-softmax convolution) the convolved values
 // Vt [B][H][nvh][c_q][L][d] bf16, nvh = 2 with post-softmax mixing, else 1;
 // Lpad = L rounded up to 128, M = (c_q-1) + 2*(c_k/2); each part 256-byte aligned.
 size_t attn_kq_workspace_bytes(int B, int H, int L, int d, int cq, int ck, int hp, int kqp) {
   const size_t BH = static_cast<size_t>(B) * H, BHL = BH * L;
   const size_t lpad = (static_cast<size_t>(L) + 127) / 128 * 128;
   const size_t M = static_cast<size_t>(cq - 1 + 2 * (ck / 2));
-  // one slot pair per persistent CTA: at most kKqMaxClusters CTAs, and at most two per
-  // work item (batch, head group, query tile)
+  // the CTA-pair kernel's mixing scratch, or one exchange slot pair per persistent CTA
+  // of this kernel (at most kKqMaxClusters CTAs, and at most two per work item)
   const size_t items = kq_items(B, H, L, kqp);
   const size_t ctas = std::min<size_t>(kKqMaxClusters, 2 * items);
-  const size_t xg = hp == 2 ? ctas * 2 * d * 128 * 4 : 0;
+  const size_t xg = attn_kq_pair_applies(d, 1, hp, kqp) ? attn_kq_pair_scratch_bytes(B, H, L, d, hp)
+                    : hp == 2                           ? ctas * 2 * 2 * d * 128 * 4
+                                                        : 0;
   const size_t vt = kqp ? align256(BHL * (hp == 2 ? 2 : 1) * cq * d * 2) : 0;
   return align256(BHL * cq * d * 2) + align256(BH * lpad * 4) + align256(BHL * M * 4) + xg + vt;
 }
@@ -1280,8 +1405,18 @@ cudaError_t launch_attn_kq(const AttnArgs &a, const GnArgs *gn, void *ws) {
   pa.vp = reinterpret_cast<float *>(reinterpret_cast<char *>(pa.fac) + align256(BH * pa.lpad * 4));
   float *xg = reinterpret_cast<float *>(reinterpret_cast<char *>(pa.vp) + align256(BHL * pa.M * 4));
   const size_t items = kq_items(a.B, a.H, a.L, a.kqp);
-  void *vt = reinterpret_cast<char *>(xg) +
-             (a.hp == 2 ? std::min<size_t>(kKqMaxClusters, 2 * items) * 2 * a.d * 128 * 4 : 0);
+  const bool pair = attn_kq_pair_applies(a.d, a.kq, a.hp, a.kqp);
+  const size_t xg_bytes = pair ? attn_kq_pair_scratch_bytes(a.B, a.H, a.L, a.d, a.hp)
+                          : a.hp == 2 ? std::min<size_t>(kKqMaxClusters, 2 * items) * 2 * 2 * a.d * 128 * 4
+                                      : 0;
+  void *vt = reinterpret_cast<char *>(xg) + xg_bytes;
+  pa.zero = nullptr;
+  pa.n_zero = 0;
+  if (pair && a.hp == 2) {  // the pair kernel's mixing counters, after its scratch slots
+    const size_t slots = static_cast<size_t>(a.B) * (a.H / 2) * ((static_cast<size_t>(a.L) + 127) / 128);
+    pa.zero = reinterpret_cast<unsigned *>(reinterpret_cast<char *>(xg) + slots * 2 * 2 * a.d * 128 * 4);
+    pa.n_zero = static_cast<int>(slots);
+  }
   cudaError_t e = launch_kq_prep(pa, a.stream);
   if (e != cudaSuccess || (e = mark(a)) != cudaSuccess) return e;
   if (a.kqp) {
@@ -1294,6 +1429,10 @@ cudaError_t launch_attn_kq(const AttnArgs &a, const GnArgs *gn, void *ws) {
     va.nvh = a.hp == 2 ? 2 : 1;
     va.n_tiles = pa.n_tiles;
     if ((e = launch_vt_prep(va, a.stream)) != cudaSuccess || (e = mark(a)) != cudaSuccess) return e;
+  }
+  if (pair) {
+    e = launch_attn_kq_pair(a, gn, pa, xg);
+    return e != cudaSuccess ? e : mark(a);
   }
   // MIX: 0 no head mixing, 1 pre-softmax mixing (both C of a group per CTA), 2 post-softmax
   auto go = [&](auto d_tag, auto mix_tag) -> cudaError_t {

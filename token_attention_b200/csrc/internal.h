@@ -91,6 +91,8 @@ struct KqPrepArgs {
   float scale_log2;       // logit scale times log2(e)
   int B, H, L, d, cq, ck, M, n_tiles, lpad;
   int exact;              // exact causal indicator: Vp[i][m] = q[i] . k[i-m+(cq-1)]
+  unsigned *zero;         // n_zero words the prepass sets to 0 (counters of the attention kernel), or null
+  int n_zero;
 };
 cudaError_t launch_kq_prep(const KqPrepArgs &a, cudaStream_t stream);
 // Values convolved by the post-softmax kernels along the keys (bf16):
@@ -110,6 +112,11 @@ bool attn_kq_supported(const AttnArgs &a);
 size_t attn_kq_workspace_bytes(int B, int H, int L, int d, int cq, int ck, int hp, int kqp);
 // ws: workspace area for Kt / fac / Vp (attn_kq_workspace_bytes bytes, 256-byte aligned).
 cudaError_t launch_attn_kq(const AttnArgs &a, const GnArgs *gn, void *ws);
+// The contraction kernel on CTA pairs (attn_kq_pair.cu): the shapes it serves, the
+// scratch it needs after the prepass's operands, and its launch.
+bool attn_kq_pair_applies(int d, int kq, int hp, int kqp);
+size_t attn_kq_pair_scratch_bytes(int B, int H, int L, int d, int hp);
+cudaError_t launch_attn_kq_pair(const AttnArgs &a, const GnArgs *gn, const KqPrepArgs &pa, void *scratch);
 
 // tcgen05 GEMM: C[M][N] = A[M][K] * B[N][K]^T (bf16 -> fp32 -> bf16).
 cudaError_t launch_gemm_bf16_nt(const void *A, const void *B, void *C, int M, int N, int K,

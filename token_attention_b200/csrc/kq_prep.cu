@@ -104,6 +104,8 @@ __global__ void __launch_bounds__(kPrepThreads, 3) kq_prep_kernel(KqPrepArgs p) 
   pdl_launch_dependents();
   const __nv_bfloat16 *qb = static_cast<const __nv_bfloat16 *>(p.q);
 
+  if (p.zero && tile == 0 && h == 0 && b == 0)  // counters the attention kernel starts from 0
+    for (int i = tid; i < p.n_zero; i += kPrepThreads) p.zero[i] = 0u;
   for (int i = tid; i < CQ * CK; i += kPrepThreads) th[i] = p.theta[static_cast<long long>(h) * CQ * CK + i];
   for (int i = tid; i < G::ROWS; i += kPrepThreads) rmax[i] = 0.f;
   __syncthreads();
