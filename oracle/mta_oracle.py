@@ -67,7 +67,7 @@ __all__ = ["OFF", "PRE", "POST", "PRE_EXACT", "attention_logits", "mask_zero", "
            "mta_attention", "mta_attention_rows", "depth_scale", "group_norm_scale", "mta_layer",
            "key_query_conv_adjoint", "key_query_conv_grad_theta", "mta_attention_group_bwd",
            "mta_attention_bwd",
-           "mta_layer_rows"]
+           "mta_layer_rows", "group_norm_scale_bwd", "mta_layer_bwd"]
 
 
 # ----------------------------------------------------------------------------
@@ -462,6 +462,63 @@ def mta_layer(x, wqkv, theta, w, gamma, beta, eps, lam, wo, H, c_h,
     o = mta_attention(q, k, v, theta, w, c_h, kq_place, head_place, theta_post=theta_post)
     y = group_norm_scale(o, gamma, beta, eps, lam).reshape(B, L, D)
     return np.matmul(y, wo.astype(np.float64).T)
+
+
+def group_norm_scale_bwd(o, gamma, beta, eps, lam, dy, gate=None):
+    """Gradients of group_norm_scale  [MTA-3.3, bycloud]: given dy = dL/dy,
+    returns (do, dgamma [H*d], dbeta [H*d], dgate [H] or None).  lam is the depth
+    scale (a scalar, no gradient); with gate logits the multiplier of head h is
+    sigmoid(gate[h]) and dgate is its gradient.  Chain rule of
+    y = m_h * (xhat * gamma + beta), xhat = (o - mean) / sqrt(var + eps), biased var."""
+    o = o.astype(np.float64)
+    dy = dy.astype(np.float64)
+    H, d = o.shape[-2], o.shape[-1]
+    g = gamma.astype(np.float64).reshape(H, d)
+    b = beta.astype(np.float64).reshape(H, d)
+    mu = np.mean(o, axis=-1, keepdims=True)
+    var = np.mean((o - mu) ** 2, axis=-1, keepdims=True)
+    rstd = 1.0 / np.sqrt(var + eps)
+    xhat = (o - mu) * rstd
+    m = sigmoid_gate(gate).reshape(H, 1) if gate is not None else np.asarray(lam, np.float64)
+    lead = tuple(range(o.ndim - 2))
+    dgamma = np.sum(m * dy * xhat, axis=lead).reshape(H * d)
+    dbeta = np.sum(m * dy, axis=lead).reshape(H * d)
+    dgate = None
+    if gate is not None:
+        sg = sigmoid_gate(gate)
+        dgate = np.sum(dy * (xhat * g + b), axis=lead + (o.ndim - 1,)) * sg * (1.0 - sg)
+    dxhat = m * dy * g
+    do = rstd * (dxhat - np.mean(dxhat, axis=-1, keepdims=True)
+                 - xhat * np.mean(dxhat * xhat, axis=-1, keepdims=True))
+    return do, dgamma, dbeta, dgate
+
+
+def mta_layer_bwd(x, wqkv, theta, w, gamma, beta, eps, lam, wo, H, c_h, dout,
+                  kq_place=PRE, head_place=POST, theta_post=None, gate=None):
+    """Gradients of mta_layer  [MTA-2, MTA-3.x, bycloud], each step of the forward
+    taken in reverse: out = Y Wo^T, Y = group norm (depth scale or gate) of the
+    attention output, attention as mta_attention_bwd, QKV = x Wqkv^T.
+    dout [B][L][D].  Returns dict with dx [B][L][D], dwqkv [3D][D], dwo [D][D],
+    dtheta, dw, dtheta_post (as mta_attention_bwd), dgamma, dbeta [D] and dgate [H]
+    (None without a gate), float64.  With a gate, lam is ignored."""
+    B, L, D = x.shape
+    d = D // H
+    x64 = x.astype(np.float64)
+    qkv = np.matmul(x64, wqkv.astype(np.float64).T)
+    q, k, v = _split_qkv(qkv, H, d)
+    o = mta_attention(q, k, v, theta, w, c_h, kq_place, head_place, theta_post=theta_post)
+    mult = sigmoid_gate(gate) if gate is not None else lam
+    y = group_norm_scale(o, gamma, beta, eps, mult).reshape(B, L, D)
+    g_out = dout.astype(np.float64)
+    dy = np.matmul(g_out, wo.astype(np.float64)).reshape(B, L, H, d)         # out = y Wo^T
+    dwo = np.matmul(g_out.reshape(-1, D).T, y.reshape(-1, D))
+    do, dgamma, dbeta, dgate = group_norm_scale_bwd(o, gamma, beta, eps, lam, dy, gate)
+    ga = mta_attention_bwd(q, k, v, theta, w, c_h, do, kq_place, head_place, theta_post=theta_post)
+    dqkv = np.concatenate([ga[n].reshape(B, L, D) for n in ("dq", "dk", "dv")], axis=-1)
+    dx = np.matmul(dqkv, wqkv.astype(np.float64))                            # qkv = x Wqkv^T
+    dwqkv = np.matmul(dqkv.reshape(-1, 3 * D).T, x64.reshape(-1, D))
+    return {"dx": dx, "dwqkv": dwqkv, "dwo": dwo, "dtheta": ga["dtheta"], "dw": ga["dw"],
+            "dtheta_post": ga["dtheta_post"], "dgamma": dgamma, "dbeta": dbeta, "dgate": dgate}
 
 
 def mta_layer_rows(x, wqkv, theta, w, gamma, beta, eps, lam, wo, H, c_h, rows,

@@ -683,3 +683,73 @@ def test_backward_identity_kernels_equal_torch_autograd():
         np.testing.assert_allclose(g[name], tt.grad.numpy().transpose(0, 2, 1, 3), rtol=0, atol=1e-12)
     # the kernel gradient of the identity kernel's centre tap is the logits' own gradient . logits
     assert g["dtheta"].shape == (H, cq, ck)
+
+
+# ----------------------------------------------------------------------------
+# backward of the full layer: central finite differences of mta_layer, and the
+# group norm's backward against torch's autograd of its group_norm routine
+# ----------------------------------------------------------------------------
+
+@pytest.mark.parametrize("hp,post,gated", [(O.POST, False, False), (O.PRE, False, False),
+                                           (O.POST, True, False), (O.POST, False, True)])
+def test_layer_backward_matches_finite_differences(hp, post, gated):
+    """Every gradient of the layer (x, Wqkv, Wo, the kernels, the mixing weights,
+    gamma, beta and the gate logits) against central differences of the forward
+    along random directions."""
+    B, L, H, d, cq, ck, ch = 1, 6, 2, 3, 3, 3, 2
+    D = H * d
+    rng = np.random.default_rng(950 + hp + 2 * post + 4 * gated)
+    x = rng.standard_normal((B, L, D))
+    wqkv = rng.standard_normal((3 * D, D)) * 0.4
+    wo = rng.standard_normal((D, D)) * 0.4
+    th = rng.standard_normal((H, cq, ck)) * 0.5
+    tp = rng.standard_normal((H, cq, ck)) * 0.5 if post else None
+    w = rng.standard_normal((1, ch, ch))
+    gamma = 1 + 0.2 * rng.standard_normal(D)
+    beta = 0.2 * rng.standard_normal(D)
+    gate = rng.standard_normal(H) if gated else None
+    eps, lam = 1e-5, 0.8
+    dout = rng.standard_normal((B, L, D))
+
+    def f(x_, wqkv_, wo_, th_, w_, tp_, gamma_, beta_, gate_):
+        mult = O.sigmoid_gate(gate_) if gate_ is not None else lam
+        out = O.mta_layer(x_, wqkv_, th_, w_, gamma_, beta_, eps, mult, wo_, H, ch, O.PRE, hp,
+                          theta_post=tp_)
+        return float(np.sum(out * dout))
+
+    g = O.mta_layer_bwd(x, wqkv, th, w, gamma, beta, eps, lam, wo, H, ch, dout, O.PRE, hp,
+                        theta_post=tp, gate=gate)
+    base = dict(x_=x, wqkv_=wqkv, wo_=wo, th_=th, w_=w, tp_=tp, gamma_=gamma, beta_=beta, gate_=gate)
+    checks = [("x_", "dx"), ("wqkv_", "dwqkv"), ("wo_", "dwo"), ("th_", "dtheta"), ("w_", "dw"),
+              ("gamma_", "dgamma"), ("beta_", "dbeta")]
+    if post:
+        checks.append(("tp_", "dtheta_post"))
+    if gated:
+        checks.append(("gate_", "dgate"))
+    eps_fd = 1e-6
+    for name, gname in checks:
+        for _ in range(2):
+            u = rng.standard_normal(base[name].shape)
+            plus = dict(base); plus[name] = base[name] + eps_fd * u
+            minus = dict(base); minus[name] = base[name] - eps_fd * u
+            fd = (f(**plus) - f(**minus)) / (2 * eps_fd)
+            an = float(np.sum(g[gname] * u))
+            assert abs(fd - an) <= 1e-6 * max(1.0, abs(an)), (hp, post, gated, gname, fd, an)
+
+
+def test_group_norm_backward_matches_torch_autograd():
+    T, H, d = 7, 3, 8
+    rng = np.random.default_rng(61)
+    o = rng.standard_normal((T, H, d)) * 2 + 0.5
+    gamma, beta = 1 + 0.1 * rng.standard_normal(H * d), 0.1 * rng.standard_normal(H * d)
+    dy = rng.standard_normal((T, H, d))
+    lam, eps = 0.9, 1e-5
+    do, dgamma, dbeta, _ = O.group_norm_scale_bwd(o, gamma, beta, eps, lam, dy)
+    to = torch.from_numpy(o.reshape(T, H * d)).requires_grad_(True)
+    tg = torch.from_numpy(gamma).requires_grad_(True)
+    tb = torch.from_numpy(beta).requires_grad_(True)
+    y = torch.nn.functional.group_norm(to, H, tg, tb, eps) * lam
+    y.backward(torch.from_numpy(dy.reshape(T, H * d)))
+    np.testing.assert_allclose(do.reshape(T, H * d), to.grad.numpy(), rtol=0, atol=1e-10)
+    np.testing.assert_allclose(dgamma, tg.grad.numpy(), rtol=0, atol=1e-10)
+    np.testing.assert_allclose(dbeta, tb.grad.numpy(), rtol=0, atol=1e-10)
