@@ -438,7 +438,18 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else if (warp == kMmaWarp) {
     // -------------------------------------------------------------- MMA
-    if (lane == 0) {
+    // The whole warp runs the issuing loop; one elected lane issues the instructions.
+    {
+      const bool issuer = elect_one();
+      // waits of the issuing loop, made warp-uniform (all lanes poll the same barrier)
+      auto wwait = [&](uint64_t *bar, uint32_t ph) -> bool {
+        return __all_sync(0xffffffffu, mbar_wait(bar, ph, abort_flag, p.err));
+      };
+      auto take_mma = [&](int r, Item &x) -> bool {
+        const bool got = __all_sync(0xffffffffu, take_item(r, x, lane == 0));
+        __syncwarp();
+        return got;
+      };
       const uint32_t idesc_c = idesc_f16_f32(128, G::BN);
       const uint32_t idesc_pv = idesc_bf16_f32(128, D, 0, 1);
       // descriptors of the first operand tiles; every other tile differs only in its
@@ -459,7 +470,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       // DB: into buffer T & 1 without waiting for the softmax (the buffer's previous
       // tile, T - 2, had its P V issued before, and MMAs run in issue order)
       auto issue_c = [&](bool last_of_item) -> bool {
-        if (!G::DB && T > 0 && !mbar_wait(c_free, (T - 1) & 1, abort_flag, p.err)) return false;
+        if (!G::DB && T > 0 && !wwait(c_free, (T - 1) & 1)) return false;
         const uint32_t c_dst = tmem + G::C_COL + (G::DB ? 128u * (T & 1) : 0u);
         for (int ch = 0; ch < G::NSRC * G::NCH; ch += G::SB, ++cnt) {
           const int st = cnt % G::NS;
@@ -468,7 +479,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           // multiple of 16, so a step never straddles two tap rows); Q rows shifted up
           // by a (16 bytes per row), 8-channel strips e0/8 and e0/8 + 1
           if constexpr (D % 64 == 0) {
-            if (!mbar_wait(k_full + st, (cnt / G::NS) & 1, abort_flag, p.err)) return false;
+            if (!wwait(k_full + st, (cnt / G::NS) & 1)) return false;
             tc_fence_after();
             // box bx of the stage is chunk cs: tap row a = cs / NDC, channels 64 dc ..
             // 64 dc + 63 (a stage is a whole tap row when SB = NDC)
@@ -480,7 +491,7 @@ __global__ void __launch_bounds__(kThreads, 1)
               const uint64_t qd = qdesc0 + static_cast<uint32_t>((sc * G::Q_ALLOC + 8 * dc * G::STRIP + 16 * (G::HALO - a)) >> 4);
 #pragma unroll
               for (int kk = 0; kk < 4; ++kk)
-                mma_bf16_ss(c_dst + 128 * sc, qd + (2 * kk * G::STRIP >> 4),
+                mma_ss_if(issuer, c_dst + 128 * sc, qd + (2 * kk * G::STRIP >> 4),
                             kd + (bx * G::KCHUNK >> 4) + 2 * kk, idesc_c, (cs > 0 || kk > 0));
             }
           } else {
@@ -492,23 +503,23 @@ __global__ void __launch_bounds__(kThreads, 1)
               const int kap = 64 * cs + 16 * kk, a = kap / D, e0 = kap % D;
               qd[kk] = qdesc0 + static_cast<uint32_t>((sc * G::Q_ALLOC + (e0 / 8) * G::STRIP + 16 * (G::HALO - a)) >> 4);
             }
-            if (!mbar_wait(k_full + st, (cnt / G::NS) & 1, abort_flag, p.err)) return false;
+            if (!wwait(k_full + st, (cnt / G::NS) & 1)) return false;
             tc_fence_after();
 #pragma unroll
             for (int kk = 0; kk < 4; ++kk)
-              mma_bf16_ss(c_dst + 128 * sc, qd[kk], kd + 2 * kk, idesc_c, (cs > 0 || kk > 0));
+              mma_ss_if(issuer, c_dst + 128 * sc, qd[kk], kd + 2 * kk, idesc_c, (cs > 0 || kk > 0));
           }
-          mma_commit(k_empty + st);
+          mma_commit_if(issuer, k_empty + st);
         }
-        mma_commit(G::DB ? c_fullb[T & 1] : c_full);
-        if (last_of_item) mma_commit(q_free);  // the query buffer may take the next item
+        mma_commit_if(issuer, G::DB ? c_fullb[T & 1] : c_full);
+        if (last_of_item) mma_commit_if(issuer, q_free);  // the query buffer may take the next item
         return true;
       };
       // Z_hd += sum_a (weights shifted down by a rows) x Vt_{hd,a}, from the ring
       auto issue_pv = [&](bool first_of_item) -> bool {
         for (int ch = 0; ch < G::NVCH; ch += G::SB, ++cnt) {
           const int st = cnt % G::NS;
-          if (!mbar_wait(k_full + st, (cnt / G::NS) & 1, abort_flag, p.err)) return false;
+          if (!wwait(k_full + st, (cnt / G::NS) & 1)) return false;
           tc_fence_after();
           if constexpr (G::SB == 2) {
             // the stage holds both 64-channel boxes of (hd, a): one N = 128 MMA per key step
@@ -517,7 +528,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             const uint64_t vd = vtdesc0 + static_cast<uint32_t>((st * G::KSTAGE) >> 4);
 #pragma unroll
             for (int kk = 0; kk < G::BN / 16; ++kk)
-              mma_bf16_ss(tmem + G::Z_COL0 + 128 * hd, pd + static_cast<uint32_t>((2 * kk * G::PS_STRIP) >> 4),
+              mma_ss_if(issuer, tmem + G::Z_COL0 + 128 * hd, pd + static_cast<uint32_t>((2 * kk * G::PS_STRIP) >> 4),
                           vd + static_cast<uint32_t>((kk * 16 * 128) >> 4), idesc_bf16_f32(128, 128, 0, 1),
                           !(first_of_item && a == 0 && kk == 0));
           } else {
@@ -528,20 +539,20 @@ __global__ void __launch_bounds__(kThreads, 1)
               const uint64_t vd = vtdesc0 + static_cast<uint32_t>((st * G::KSTAGE + bx * G::KCHUNK) >> 4);
 #pragma unroll
               for (int kk = 0; kk < G::BN / 16; ++kk)
-                mma_bf16_ss(tmem + G::Z_COL0 + 128 * hd + 64 * dc, pd + static_cast<uint32_t>((2 * kk * G::PS_STRIP) >> 4),
+                mma_ss_if(issuer, tmem + G::Z_COL0 + 128 * hd + 64 * dc, pd + static_cast<uint32_t>((2 * kk * G::PS_STRIP) >> 4),
                             vd + static_cast<uint32_t>((kk * 16 * 128) >> 4), idesc_pv64,
                             !(first_of_item && a == 0 && kk == 0));
             }
           }
-          mma_commit(k_empty + st);
+          mma_commit_if(issuer, k_empty + st);
         }
-        mma_commit(v_empty);
+        mma_commit_if(issuer, v_empty);
         return true;
       };
       Item it;
-      for (int r = 0; ok && take_item(r, it, true); ++r) {
+      for (int r = 0; ok && take_mma(r, it); ++r) {
         const int n_kv = kv_tiles(it), nsl = n_slots(it);
-        if (!mbar_wait(q_ready, r & 1, abort_flag, p.err)) break;
+        if (!wwait(q_ready, r & 1)) break;
         if constexpr (G::DB) {
           // C of the first two tiles, then per tile: P V, and C two tiles ahead into
           // the buffer that P V has just consumed
@@ -553,25 +564,25 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           for (int sl = 0; ok && sl < nsl; ++sl) {
             const int Tt = T0 + sl;
-            if (!mbar_wait(p_fullb[Tt & 1], (Tt >> 1) & 1, abort_flag, p.err)) { ok = false; break; }
-            if (!mbar_wait(v_full, Tt & 1, abort_flag, p.err)) { ok = false; break; }
-            if (sl == 0 && r > 0 && !mbar_wait(z_free, (r - 1) & 1, abort_flag, p.err)) { ok = false; break; }
+            if (!wwait(p_fullb[Tt & 1], (Tt >> 1) & 1)) { ok = false; break; }
+            if (!wwait(v_full, Tt & 1)) { ok = false; break; }
+            if (sl == 0 && r > 0 && !wwait(z_free, (r - 1) & 1)) { ok = false; break; }
             tc_fence_after();
             const uint32_t pcol = tmem + 128u * (Tt & 1);
             if constexpr (G::NV * G::NDC * 64 == 256) {
 #pragma unroll
               for (int kk = 0; kk < G::BN / 16; ++kk)
-                mma_f16_ts(tmem + G::Z_COL0, pcol + 8 * kk, vdesc0 + ((kk * 16 * 128) >> 4),
+                mma_ts_if(issuer, tmem + G::Z_COL0, pcol + 8 * kk, vdesc0 + ((kk * 16 * 128) >> 4),
                            idesc_bf16_f32(128, 256, 0, 1), (sl > 0 || kk > 0));
             } else {
 #pragma unroll
               for (int hd = 0; hd < G::NV; ++hd)
 #pragma unroll
                 for (int kk = 0; kk < G::BN / 16; ++kk)
-                  mma_f16_ts(tmem + G::Z_COL0 + 128 * hd, pcol + 8 * kk,
+                  mma_ts_if(issuer, tmem + G::Z_COL0 + 128 * hd, pcol + 8 * kk,
                              vdesc0 + ((hd * G::V_HEAD + kk * 16 * 128) >> 4), idesc_pv, (sl > 0 || kk > 0));
             }
-            mma_commit(v_empty);
+            mma_commit_if(issuer, v_empty);
             if (sl + 2 < nsl) {
               T = Tt + 2;
               ok = issue_c(sl + 3 == nsl);
@@ -590,40 +601,40 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           if constexpr (POST) {
             if (sl < n_kv) continue;  // first pass: statistics only
-            if (!mbar_wait(p_full, npv & 1, abort_flag, p.err)) { ok = false; break; }
-            if (sl == n_kv && r > 0 && !mbar_wait(z_free, (r - 1) & 1, abort_flag, p.err)) { ok = false; break; }
+            if (!wwait(p_full, npv & 1)) { ok = false; break; }
+            if (sl == n_kv && r > 0 && !wwait(z_free, (r - 1) & 1)) { ok = false; break; }
             tc_fence_after();
             if (!issue_pv(sl == n_kv)) { ok = false; break; }
             ++npv;
           } else {
             const int t = sl;
-            if (!mbar_wait(p_full, Tt & 1, abort_flag, p.err)) { ok = false; break; }
-            if (!mbar_wait(v_full, Tt & 1, abort_flag, p.err)) { ok = false; break; }
+            if (!wwait(p_full, Tt & 1)) { ok = false; break; }
+            if (!wwait(v_full, Tt & 1)) { ok = false; break; }
             // Z is overwritten (accumulate off) by the first P V of an item: the previous
             // item's epilogue must have read it
-            if (t == 0 && r > 0 && !mbar_wait(z_free, (r - 1) & 1, abort_flag, p.err)) { ok = false; break; }
+            if (t == 0 && r > 0 && !wwait(z_free, (r - 1) & 1)) { ok = false; break; }
             tc_fence_after();
             if constexpr (G::NV * G::NDC * 64 == 256) {
               // both heads' V tiles are four consecutive 64-channel boxes and both Z
               // accumulators 256 consecutive columns: one N = 256 MMA per key step
 #pragma unroll
               for (int kk = 0; kk < G::BN / 16; ++kk)
-                mma_f16_ts(tmem + G::Z_COL0, tmem + G::P_COL + 8 * kk, vdesc0 + ((kk * 16 * 128) >> 4),
+                mma_ts_if(issuer, tmem + G::Z_COL0, tmem + G::P_COL + 8 * kk, vdesc0 + ((kk * 16 * 128) >> 4),
                            idesc_bf16_f32(128, 256, 0, 1), (t > 0 || kk > 0));
             } else {
 #pragma unroll
               for (int hd = 0; hd < G::NV; ++hd)
 #pragma unroll
                 for (int kk = 0; kk < G::BN / 16; ++kk)
-                  mma_f16_ts(tmem + G::Z_COL0 + 128 * hd, tmem + G::P_COL + 8 * kk,
+                  mma_ts_if(issuer, tmem + G::Z_COL0 + 128 * hd, tmem + G::P_COL + 8 * kk,
                              vdesc0 + ((hd * G::V_HEAD + kk * 16 * 128) >> 4), idesc_pv, (t > 0 || kk > 0));
             }
-            mma_commit(v_empty);
+            mma_commit_if(issuer, v_empty);
           }
         }
         T = T0 + nsl;
       }
-      mma_commit(mma_done);
+      mma_commit_if(issuer, mma_done);
       drain_wait(mma_done, 0);
     }
   } else {
@@ -1379,7 +1390,7 @@ size_t attn_kq_workspace_bytes(int B, int H, int L, int d, int cq, int ck, int h
   // of this kernel (at most kKqMaxClusters CTAs, and at most two per work item)
   const size_t items = kq_items(B, H, L, kqp);
   const size_t ctas = std::min<size_t>(kKqMaxClusters, 2 * items);
-  const size_t xg = attn_kq_pair_applies(d, 1, hp, kqp) ? attn_kq_pair_scratch_bytes(B, H, L, d, hp)
+  const size_t xg = attn_kq_pair_applies(d, 1, hp, kqp, L) ? attn_kq_pair_scratch_bytes(B, H, L, d, hp)
                     : hp == 2                           ? ctas * 2 * 2 * d * 128 * 4
                                                         : 0;
   const size_t vt = kqp ? align256(BHL * (hp == 2 ? 2 : 1) * cq * d * 2) : 0;
@@ -1405,7 +1416,7 @@ cudaError_t launch_attn_kq(const AttnArgs &a, const GnArgs *gn, void *ws) {
   pa.vp = reinterpret_cast<float *>(reinterpret_cast<char *>(pa.fac) + align256(BH * pa.lpad * 4));
   float *xg = reinterpret_cast<float *>(reinterpret_cast<char *>(pa.vp) + align256(BHL * pa.M * 4));
   const size_t items = kq_items(a.B, a.H, a.L, a.kqp);
-  const bool pair = attn_kq_pair_applies(a.d, a.kq, a.hp, a.kqp);
+  const bool pair = attn_kq_pair_applies(a.d, a.kq, a.hp, a.kqp, a.L);
   const size_t xg_bytes = pair ? attn_kq_pair_scratch_bytes(a.B, a.H, a.L, a.d, a.hp)
                           : a.hp == 2 ? std::min<size_t>(kKqMaxClusters, 2 * items) * 2 * 2 * a.d * 128 * 4
                                       : 0;

@@ -54,7 +54,11 @@ constexpr int kTmaWarp = 8, kMmaWarp = 9, kTma2Warp = 10;
 constexpr int kBarAll = 1;
 constexpr int kItemSlots = 4;
 constexpr int kMaxPairs = 80;  // persistent grid: at most this many CTA pairs (>= SM count / 2)
-constexpr bool kPairKernel = false;  // serve the shapes below with this kernel
+// Sequences at least this long use this kernel for the shapes below (measured on
+// B200, one call, d = 128, groups of 2: the one-CTA kernel is faster at L = 2048
+// (316 vs 336 us) and L = 4096 (491 vs 516 us), this one at L = 16384 (3.32 vs
+// 3.53 ms), where each item runs over many more key tiles)
+constexpr int kPairMinL = 8192;
 
 template <int D, int MIX, bool EXACT>
 struct PGeo {
@@ -310,7 +314,13 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else if (warp == kMmaWarp) {
     // -------------------------------------------------------------- MMA (first CTA)
-    if (lane == 0 && rank == 0) {
+    // The whole warp runs the issuing loop; one elected lane issues the instructions.
+    if (rank == 0) {
+      const bool issuer = elect_one();
+      // waits of the issuing loop, made warp-uniform (all lanes poll the same barrier)
+      auto wwait = [&](uint64_t *bar, uint32_t ph) -> bool {
+        return __all_sync(0xffffffffu, mbar_wait_cluster(bar, ph, abort_flag, p.err));
+      };
       const uint32_t idesc_c = idesc_f16_f32(256, G::BN);
       const uint32_t idesc_pv = idesc_bf16_f32(256, G::NPV, 0, 1);
       const uint64_t qdesc0 = sdesc_noswz(smem_u32(Qs), G::STRIP, 128);
@@ -324,7 +334,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint32_t c_dst = tmem + 128u * (T & 1);
         for (int a = 0; a < CQ; ++a, ++cnt) {
           const int st = cnt % G::NS;
-          if (!mbar_wait_cluster(k_full + st, (cnt / G::NS) & 1, abort_flag, p.err)) return false;
+          if (!wwait(k_full + st, (cnt / G::NS) & 1)) return false;
           tc_fence_after();
           const uint64_t kd = kdesc0 + static_cast<uint32_t>((st * G::KSTAGE) >> 4);
 #pragma unroll
@@ -332,19 +342,25 @@ __global__ void __launch_bounds__(kThreads, 1)
             const uint64_t qd = qdesc0 + static_cast<uint32_t>((8 * dc * G::STRIP + 16 * (G::HALO - a)) >> 4);
 #pragma unroll
             for (int kk = 0; kk < 4; ++kk)
-              mma_f16_ss_pair(c_dst, qd + (2 * kk * G::STRIP >> 4), kd + (dc * G::KBOX >> 4) + 2 * kk, idesc_c,
-                              (a > 0 || dc > 0 || kk > 0));
+              mma_ss_pair_if(issuer, c_dst, qd + (2 * kk * G::STRIP >> 4), kd + (dc * G::KBOX >> 4) + 2 * kk,
+                             idesc_c, (a > 0 || dc > 0 || kk > 0));
           }
-          mma_commit_pair(k_empty + st, 0x3);
+          mma_commit_pair_if(issuer, k_empty + st, 0x3);
         }
-        mma_commit_pair(c_full + (T & 1), 0x3);
-        if (last_of_item) mma_commit_pair(q_free, 0x3);  // both query buffers may take the next item
+        mma_commit_pair_if(issuer, c_full + (T & 1), 0x3);
+        if (last_of_item) mma_commit_pair_if(issuer, q_free, 0x3);  // both query buffers may take the next item
         return true;
       };
       PItem it;
-      for (int r = 0; ok && take_item(r, it, true); ++r) {
+      // (one arrival per item on the ring: this warp counts as one consumer)
+      auto take_mma = [&](int r, PItem &x) -> bool {
+        const bool got = __all_sync(0xffffffffu, take_item(r, x, false));
+        if (lane == 0) arrive_first(it_empty + r % kItemSlots);
+        return got;
+      };
+      for (int r = 0; ok && take_mma(r, it); ++r) {
         const int nsl = kv_tiles(it);
-        if (!mbar_wait_cluster(q_ready, r & 1, abort_flag, p.err)) break;
+        if (!wwait(q_ready, r & 1)) break;
         const int T0 = T;
         ok = issue_c(nsl == 1);
         if (ok && nsl > 1) {
@@ -353,16 +369,16 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         for (int sl = 0; ok && sl < nsl; ++sl) {
           const int Tt = T0 + sl;
-          if (!mbar_wait_cluster(p_full + (Tt & 1), (Tt >> 1) & 1, abort_flag, p.err)) { ok = false; break; }
-          if (!mbar_wait_cluster(v_full, Tt & 1, abort_flag, p.err)) { ok = false; break; }
-          if (sl == 0 && r > 0 && !mbar_wait_cluster(z_free, (r - 1) & 1, abort_flag, p.err)) { ok = false; break; }
+          if (!wwait(p_full + (Tt & 1), (Tt >> 1) & 1)) { ok = false; break; }
+          if (!wwait(v_full, Tt & 1)) { ok = false; break; }
+          if (sl == 0 && r > 0 && !wwait(z_free, (r - 1) & 1)) { ok = false; break; }
           tc_fence_after();
           const uint32_t pcol = tmem + 128u * (Tt & 1);
 #pragma unroll
           for (int kk = 0; kk < G::BN / 16; ++kk)
-            mma_f16_ts_pair(tmem + G::Z_COL0, pcol + 8 * kk, vdesc0 + ((kk * 16 * 128) >> 4), idesc_pv,
-                            (sl > 0 || kk > 0));
-          mma_commit_pair(v_empty, 0x3);
+            mma_ts_pair_if(issuer, tmem + G::Z_COL0, pcol + 8 * kk, vdesc0 + ((kk * 16 * 128) >> 4), idesc_pv,
+                           (sl > 0 || kk > 0));
+          mma_commit_pair_if(issuer, v_empty, 0x3);
           if (sl + 2 < nsl) {
             T = Tt + 2;
             ok = issue_c(sl + 3 == nsl);
@@ -370,7 +386,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         T = T0 + nsl;
       }
-      mma_commit_pair(mma_done, 0x1);
+      mma_commit_pair_if(issuer, mma_done, 0x1);
       drain_wait(mma_done, 0);
     }
   } else {
@@ -821,8 +837,8 @@ cudaError_t launch_pair_one(const AttnArgs &a, const GnArgs *gn, const KqPrepArg
 
 }  // namespace
 
-bool attn_kq_pair_applies(int d, int kq, int hp, int kqp) {
-  return kPairKernel && kqp == 0 && (kq == 1 || kq == 3) && ((d == 128 && (hp == 0 || hp == 2)) || (d == 64 && hp == 2));
+bool attn_kq_pair_applies(int d, int kq, int hp, int kqp, int L) {
+  return L >= kPairMinL && kqp == 0 && (kq == 1 || kq == 3) && ((d == 128 && (hp == 0 || hp == 2)) || (d == 64 && hp == 2));
 }
 
 size_t attn_kq_pair_scratch_bytes(int B, int H, int L, int d, int hp) {
