@@ -38,6 +38,7 @@ from token_attention_b200 import synth  # noqa: E402
 
 METRIC = "MTA fwd tokens/s and TFLOP/s at L=2048 on 1 B200; % of BF16 tensor peak"
 METRIC_BWD = "MTA attention backward (mta_attn_bwd) tokens/s on 1 B200"
+METRIC_LAYER_BWD = "MTA layer backward (mta_layer_bwd) tokens/s on 1 B200"
 UNIT = "tokens/s"
 DEFAULT_WORKLOAD = "pretrain_d128_L2048"
 N_SETS = 3
@@ -277,7 +278,7 @@ def make_sets(wl, dev, n_sets, bwd=False, rank=0):
         if inp["theta_post"] is not None:  # pre- and post-softmax kernels stacked once, outside the timed steps
             sets[-1]["theta"] = to(np.stack([inp["theta"], inp["theta_post"]]), "f32")
         if bwd:  # gradient of the output, drawn like the values
-            dout = synth.normal(w.seed, 20, (wl.B, wl.L, wl.H, wl.d))
+            dout = synth.normal(w.seed, 20, (wl.B, wl.L, wl.D) if wl.layer else (wl.B, wl.L, wl.H, wl.d))
             sets[-1]["dout"] = to(synth.round_bf16(dout) if wl.dtype == "bf16" else dout, wl.dtype)
     return sets
 
@@ -285,7 +286,13 @@ def make_sets(wl, dev, n_sets, bwd=False, rank=0):
 def step_fn(wl, mta, sets, ws, outs, stream, bwd=False):
     """Returns f(i, events=None): enqueue step i (input set i % n) on `stream`;
     the library records `events` around the step's kernels (mta_cfg.events)."""
-    if bwd:
+    if bwd and wl.layer:
+        def f(i, events=None):
+            s = sets[i % len(sets)]
+            mta.layer_bwd(s["x"], s["wqkv"], s["theta"], s["w"], s["gamma"], s["beta"], s["wo"], s["dout"],
+                          wl.H, wl.c_q, wl.c_k, wl.c_h, wl.kq_place, wl.head_place, eps=1e-5,
+                          layer=wl.depth, ws=ws, stream=stream, theta_post=s["theta_post"], events=events)
+    elif bwd:
         def f(i, events=None):
             s = sets[i % len(sets)]
             mta.attn_bwd(s["q"], s["k"], s["v"], s["theta"], s["w"], s["dout"], wl.c_q, wl.c_k, wl.c_h,
@@ -310,8 +317,13 @@ def step_fn(wl, mta, sets, ws, outs, stream, bwd=False):
 def step_kernels(wl: synth.Workload, bwd: bool) -> list[str]:
     """Names of the library's kernels one step launches, in launch order (the
     library records a timing event after each; see mta_cfg.events)."""
+    bwd_kernel = "attn_bwd_post_kernel" if wl.kq_post else "attn_bwd_simt_kernel"
+    if bwd and wl.layer:
+        return (["gemm_qkv"] + [k for k in step_kernels(wl, False)[1:-1] if k != "group_norm_kernel"] +
+                ["gemm_dy", "group_norm_bwd_kernel", "gemm_dwo", bwd_kernel, "pack_qkv_grad_kernel",
+                 "gemm_dx", "gemm_dwqkv"])
     if bwd:
-        return ["attn_bwd_post_kernel" if wl.kq_post else "attn_bwd_simt_kernel"]
+        return [bwd_kernel]
     if uses_contraction(wl):
         attn = ["kq_prep_kernel"] + (["vt_prep_kernel"] if wl.kq_post else []) + ["attn_kq_kernel"]
     elif uses_direct_tc(wl):
@@ -326,7 +338,9 @@ def dominant_kernel(wl: synth.Workload, bwd: bool) -> tuple[int, int, str]:
     events a and b of a step (event 0 before the first kernel, event k after the
     k-th; see mta_cfg.events), and its name."""
     if bwd:
-        return 0, 1, "attn_bwd_post_kernel" if wl.kq_post else "attn_bwd_simt_kernel"
+        names = step_kernels(wl, True)
+        i = names.index("attn_bwd_post_kernel" if wl.kq_post else "attn_bwd_simt_kernel")
+        return i, i + 1, names[i]
     n = launches_per_step(wl) + 1
     if uses_contraction(wl):
         # ... key prepass, (value prepass), attention kernel, (output GEMM)
@@ -387,7 +401,9 @@ def run_mine(args, wl, rank, world, local_rank):
     sets = make_sets(wl, dev, N_SETS, args.bwd, rank)
     out_shape = (wl.B, wl.L, wl.D) if wl.layer else (wl.B, wl.L, wl.H, wl.d)
     odt = torch.float32 if wl.dtype == "f32" else torch.bfloat16
-    if args.bwd:  # fp32 gradients of q, k, v, the kernels and the mixing weights
+    if args.bwd and wl.layer:  # mta.layer_bwd allocates its gradients
+        outs = [None]
+    elif args.bwd:  # fp32 gradients of q, k, v, the kernels and the mixing weights
         z = lambda *shape: torch.empty(shape, dtype=torch.float32, device=dev)
         n_th = (1 if wl.kq_place else 0) + (1 if wl.kq_post else 0)
         outs = []
@@ -401,7 +417,8 @@ def run_mine(args, wl, rank, world, local_rank):
     cfg = mta.make_cfg(wl.B, wl.H, wl.L, wl.d, wl.c_q, wl.c_k, wl.c_h, wl.kq_place, wl.head_place,
                        mta.F32 if wl.dtype == "f32" else mta.BF16, kq_post=int(wl.kq_post))
     if args.bwd:
-        nbytes = mta.lib().mta_attn_bwd_workspace_bytes(ctypes.byref(cfg))
+        nbytes = (mta.lib().mta_layer_bwd_workspace_bytes if wl.layer else mta.lib().mta_attn_bwd_workspace_bytes)(
+            ctypes.byref(cfg))
     else:
         nbytes = (mta.lib().mta_layer_workspace_bytes if wl.layer else mta.lib().mta_attn_workspace_bytes)(
             ctypes.byref(cfg))
@@ -430,7 +447,7 @@ def run_mine(args, wl, rank, world, local_rank):
 
     # the library records n_ev events per step around its kernels (mta_cfg.events);
     # each is recorded once here first, so that torch has created it
-    n_ev = (1 if args.bwd else launches_per_step(wl)) + 1
+    n_ev = len(step_kernels(wl, args.bwd)) + 1
     step_ev = [[torch.cuda.Event(enable_timing=True) for _ in range(n_ev)] for _ in range(args.steps)]
     with torch.cuda.stream(stream):
         for evs in step_ev:
@@ -572,6 +589,30 @@ def oracle_sample(wl, budget_s: float, mode: str):
     whole head groups at full length; mode "rows": single query rows of one
     head group.  Returns (tokens-equivalent/s, seconds, description)."""
     import oracle as O
+    if wl.layer and mode == "bwd_groups":
+        # the layer backward's dominant step: the attention backward of whole head
+        # groups of batch 0 at full length, on its QKV (computed outside the timing)
+        inp = synth.make_layer_inputs(wl)
+        D, ch, H = wl.D, wl.c_h, wl.H
+        qkv = inp["x"][0].astype(np.float64) @ inp["wqkv"].astype(np.float64).T
+        q, k, v = (qkv[:, i * D:(i + 1) * D].reshape(wl.L, H, wl.d) for i in range(3))
+        dout = synth.normal(wl.seed, 20, (wl.L, H, wl.d))
+        tp = inp["theta_post"]
+        done, t0 = 0, time.perf_counter()
+        for g in range(H // ch):
+            hs = slice(g * ch, (g + 1) * ch)
+            grp = lambda x: np.ascontiguousarray(x[:, hs].transpose(1, 0, 2))
+            O.mta_attention_group_bwd(grp(q), grp(k), grp(v), inp["theta"][hs], inp["w"][g], np.arange(wl.L),
+                                      1 / math.sqrt(wl.d), wl.kq_place, wl.head_place, grp(dout),
+                                      None if tp is None else tp[hs])
+            done += 1
+            if time.perf_counter() - t0 > budget_s:
+                break
+        dt = time.perf_counter() - t0
+        tok = done * ch / H * wl.L
+        return tok / dt, dt, (f"attention backward (the layer backward's dominant step) of {done} of {H // ch} "
+                              f"head groups of one batch at full length L={wl.L} ({tok:.0f} token-equivalents; "
+                              f"the projections' and the norm's gradients are not in the sample)")
     if wl.layer:
         inp = synth.make_layer_inputs(wl)
         rows = [(0, 0)]
@@ -791,7 +832,7 @@ def main():
                    peak_source=f"{peak_src} HBM copy bandwidth",
                    traffic=read_traffic("group_norm_d128_kernel", "layer_Y_T8192_H16_d128"))
     line = {
-        "metric": METRIC_BWD if args.bwd else METRIC, "value": value, "unit": UNIT, "n_gpus": world,
+        "metric": (METRIC_LAYER_BWD if wl.layer else METRIC_BWD) if args.bwd else METRIC, "value": value, "unit": UNIT, "n_gpus": world,
         "steps": args.steps,
         "warmup": res["warmup"], "ms_per_step": ms / args.steps, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "bf16" if wl.dtype == "bf16" else "f32",
@@ -800,7 +841,7 @@ def main():
         "pct_bf16_peak": {"std": fl["std"] / s / 1e12 / bf16_peak,
                           "mta": fl["mta"] / s / 1e12 / bf16_peak,
                           "peak_tflops": bf16_peak, "peak_source": f"{peak_src} bf16 {peak_kind}"},
-        "roofline": roof, "gpu_launches": args.steps * (1 if args.bwd else launches_per_step(wl)),
+        "roofline": roof, "gpu_launches": args.steps * len(step_kernels(wl, args.bwd)),
         "timed_region_ms": res["region_ms"], "per_kernel_ms": res["per_kernel_ms"],
         "clocks": res["clocks"], "e2e": res["e2e"], "epilogue_group_norm": epi,
     }

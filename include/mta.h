@@ -230,6 +230,23 @@ mta_status mta_gemm_bf16_nt(const void *A, const void *Bm, void *C, int M, int N
 mta_status mta_group_norm_scale(const void *o, const mta_gn *gn, int tokens, int H, int d,
                                 void *y, void *stream);
 
+/* C[M][N] = A B^T, bf16 in, fp32 accumulate, as the layer's GEMMs run it.
+ * A is [M][K] (a_mn = 0) or stored transposed as [K][M] (a_mn = 1); B is [N][K]
+ * (b_mn = 0) or [K][N] (b_mn = 1); C is bf16 (f32_out = 0) or fp32 (1), dense.
+ * All pointers 16-byte aligned; the contiguous extent of each operand (K for a
+ * [rows][K] operand, M or N for a transposed one) a multiple of 8.  Enqueued on
+ * `stream`. */
+mta_status mta_gemm_bf16(const void *A, const void *Bm, void *C, int M, int N, int K, int a_mn, int b_mn,
+                         int f32_out, void *stream);
+
+/* Backward of mta_group_norm_scale as mta_layer_bwd runs it: for o [tokens][H][d]
+ * bf16 and dy [tokens][H][d] fp32 writes y (the forward output, bf16) and
+ * dout = dL/do (bf16), and overwrites dgamma, dbeta [H*d] and, with gn->gate,
+ * dgate [H] (fp32, summed with atomic additions).  d in {32, 64, 96, 128}. */
+mta_status mta_group_norm_scale_bwd(const void *o, const float *dy, const mta_gn *gn, int tokens, int H, int d,
+                                    void *y, void *dout, float *dgamma, float *dbeta, float *dgate,
+                                    void *stream);
+
 /* Backward pass of mta_attn_fwd (the pages train with this forward; section 4).
  * Given dout = dL/dout, writes the gradients of q, k, v, of the key-query kernels
  * and of the head-mixing weights, each forward step taken in reverse order (see
@@ -254,6 +271,51 @@ size_t mta_attn_bwd_workspace_bytes(const mta_cfg *cfg);
 mta_status mta_attn_bwd(const void *q, const void *k, const void *v, const float *theta_kq,
                         const float *w_head, const void *dout, const mta_cfg *cfg, float *dq,
                         float *dk, float *dv, float *dtheta, float *dw);
+
+/* Backward pass of mta_layer_fwd: the gradients of the layer's every input and
+ * parameter for dout = dL/dout, so that a training step of the layer runs through
+ * the library (the pages train with this layer, section 4 and appendix F).  Each
+ * forward step is taken in reverse ("Multi-Token Attention | Summary"
+ * (greeksharifa), section 2 projections, sections 3.1-3.2 attention, section 3.3
+ * group norm):
+ *   1. QKV = x Wqkv^T and the attention output O are recomputed (as in
+ *      mta_layer_fwd, cfg->path choosing the attention kernel);
+ *   2. dY = dout Wo;
+ *   3. the group norm's backward: Y, dO, dgamma, dbeta (and dgate);
+ *   4. dWo = dout^T Y;
+ *   5. the attention core's backward (as mta_attn_bwd, on the CUDA cores):
+ *      dq, dk, dv, dtheta, dw;
+ *   6. dx = dQKV Wqkv and dWqkv = dQKV^T x, dQKV = (dq | dk | dv) in bf16.
+ * The GEMMs run on the tensor cores with bf16 operands and fp32 accumulation,
+ * reading transposed operands in place (no transpose pass).
+ *   x, Wqkv, theta, w_head, gn, Wo : as for mta_layer_fwd (bf16 only; gn->depth_scale
+ *              has no gradient)
+ *   dout     : [B][L][D] bf16
+ *   dx       : [B][L][D] fp32, overwritten
+ *   dWqkv    : [3D][D] fp32, dWo: [D][D] fp32, overwritten
+ *   dtheta   : as for mta_attn_bwd (may be NULL); dw: as for mta_attn_bwd (may be NULL)
+ *   dgamma, dbeta : [H*d] fp32, overwritten
+ *   dgate    : [H] fp32, overwritten; required when gn->gate is set, else unused
+ * d must be 32, 64, 96 or 128; x, Wqkv, Wo, dout, dx, dWqkv and dWo 16-byte aligned.
+ * Outputs must not share memory with the inputs or with one another
+ * (MTA_ERR_INVALID).  dk, dv, dtheta, dw, dgamma, dbeta and dgate are summed with
+ * atomic additions, so the last bits of every gradient may differ between runs.
+ * The workspace (mta_layer_bwd_workspace_bytes) holds, in this order, each at a
+ * 256-byte boundary: 256 bytes of status; QKV [T][3D] bf16 (T = B*L); O [T][D]
+ * bf16 (the attention output); Y [T][D] bf16; dY [T][D] fp32; dO [T][D] bf16; dq,
+ * dk, dv [T][D] fp32 each; dQKV [T][3D] bf16; then the contraction kernel's
+ * operands where they apply.  Each keeps its value after the call, for
+ * inspection.  The call runs with the fixed part alone, the forward recompute
+ * then taking another attention kernel under path 0.  Timing events
+ * (cfg->events), in order: the QKV GEMM, the attention kernels as for
+ * mta_attn_fwd, the dY GEMM, the group-norm backward, the dWo GEMM, the
+ * attention backward, the dQKV pack, the dx GEMM, the dWqkv GEMM.  No L x L map
+ * is stored. */
+size_t mta_layer_bwd_workspace_bytes(const mta_cfg *cfg);
+mta_status mta_layer_bwd(const void *x, const void *Wqkv, const float *theta, const float *w_head,
+                         const mta_gn *gn, const void *Wo, const void *dout, const mta_cfg *cfg, float *dx,
+                         float *dWqkv, float *dWo, float *dtheta, float *dw, float *dgamma, float *dbeta,
+                         float *dgate);
 
 /* Waits for cfg->stream and reports whether a kernel of the last call that used
  * cfg->workspace gave up a bounded wait (MTA_ERR_TIMEOUT), else MTA_OK or

@@ -1,7 +1,11 @@
 // gemm_tc.cu -- bf16 GEMM on the sm_100a tensor cores: C[M][N] = A[M][K] B[N][K]^T.
 //
 // Used for the two projections of the MTA layer ("Multi-Token Attention |
-// Summary" (greeksharifa), section 2): QKV = x Wqkv^T and out = Y Wo^T.
+// Summary" (greeksharifa), section 2): QKV = x Wqkv^T and out = Y Wo^T, and for
+// their gradients in the layer's backward pass (dY = dOut Wo, dWo = dOut^T Y,
+// dx = dQKV Wqkv, dWqkv = dQKV^T x).  Either operand may be stored K-major
+// ([rows][K], the forward's case) or MN-major ([K][rows], a transposed operand,
+// read as such by the MMA: no transpose pass); C is bf16 or fp32.
 //
 // Persistent: one CTA per SM walks the 128 x 256 tiles of C (t = blockIdx.x,
 // + gridDim.x, ...).  Warp 0 streams 64-wide K slices of A and B with TMA
@@ -28,10 +32,81 @@ constexpr int B_BYTES = BN * BK * 2;            // 32 KB
 constexpr int STAGE_BYTES = A_BYTES + B_BYTES;  // 48 KB
 constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 1024 /*align*/ + 256 /*barriers*/;
 constexpr uint32_t TMEM_COLS = 512;             // two 256-column accumulators
+constexpr int PANEL_BYTES = 64 * BK * 2;        // MN-major operand: 64 rows x 64 K, 8 KB
 
+// Operand staging.  K-major: one TMA box {64 K, R rows} per stage, 128-byte rows
+// (64 K elements), swizzled.  MN-major ([K][rows] in memory): R/64 boxes {64 rows,
+// 64 K}, each a panel of 64 K-rows of 128 bytes (64 operand rows).
+template <bool MN>
+__device__ __forceinline__ void load_operand(uint8_t *dst, const CUtensorMap *map, uint64_t *bar, int k0, int r0,
+                                             int R) {
+  if constexpr (!MN) {
+    tma_load_2d(dst, map, bar, k0, r0);
+  } else {
+    for (int p = 0; p < R / 64; ++p) tma_load_2d(dst + p * PANEL_BYTES, map, bar, r0 + 64 * p, k0);
+  }
+}
+template <bool MN>
+__device__ __forceinline__ void load_operand_pair(uint8_t *dst, const CUtensorMap *map, uint32_t bar_cluster, int k0,
+                                                  int r0, int R) {
+  if constexpr (!MN) {
+    tma_load_2d_pair(dst, map, bar_cluster, k0, r0);
+  } else {
+    for (int p = 0; p < R / 64; ++p) tma_load_2d_pair(dst + p * PANEL_BYTES, map, bar_cluster, r0 + 64 * p, k0);
+  }
+}
+// Shared-memory descriptor of K step k (16 elements) of a staged operand.
+// K-major: +32 bytes inside the swizzled 128-byte row.  MN-major: +16 K-rows
+// (2048 bytes); the 64-row panels lie PANEL_BYTES apart (leading offset), 8-row
+// groups of K 1024 bytes apart (stride offset).
+template <bool MN>
+__device__ __forceinline__ uint64_t operand_desc(uint32_t base, int k) {
+  if constexpr (!MN)
+    return sdesc_sw128(base + 32 * k, 16, 1024);
+  else
+    return sdesc_sw128(base + 2048 * k, PANEL_BYTES, 1024);
+}
+
+// Stores 32 consecutive fp32 accumulator columns of one row of C.
+template <bool F32>
+__device__ __forceinline__ void store_row32(void *C, int row, int col, int M, int N, const uint32_t *r) {
+  if (row >= M || col >= N) return;
+  if constexpr (F32) {
+    float *dst = static_cast<float *>(C) + static_cast<long long>(row) * N + col;
+    if ((N % 4) == 0 && col + 32 <= N) {
+#pragma unroll
+      for (int i = 0; i < 8; ++i)
+        reinterpret_cast<float4 *>(dst)[i] = make_float4(__uint_as_float(r[4 * i + 0]), __uint_as_float(r[4 * i + 1]),
+                                                         __uint_as_float(r[4 * i + 2]), __uint_as_float(r[4 * i + 3]));
+    } else {
+#pragma unroll
+      for (int i = 0; i < 32; ++i)
+        if (col + i < N) dst[i] = __uint_as_float(r[i]);
+    }
+  } else {
+    __nv_bfloat16 *dst = static_cast<__nv_bfloat16 *>(C) + static_cast<long long>(row) * N + col;
+    if ((N % 8) == 0 && col + 32 <= N) {
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        uint4 w;
+        w.x = pack_bf16x2(__uint_as_float(r[8 * i + 0]), __uint_as_float(r[8 * i + 1]));
+        w.y = pack_bf16x2(__uint_as_float(r[8 * i + 2]), __uint_as_float(r[8 * i + 3]));
+        w.z = pack_bf16x2(__uint_as_float(r[8 * i + 4]), __uint_as_float(r[8 * i + 5]));
+        w.w = pack_bf16x2(__uint_as_float(r[8 * i + 6]), __uint_as_float(r[8 * i + 7]));
+        reinterpret_cast<uint4 *>(dst)[i] = w;
+      }
+    } else {
+#pragma unroll
+      for (int i = 0; i < 32; ++i)
+        if (col + i < N) dst[i] = __float2bfloat16_rn(__uint_as_float(r[i]));
+    }
+  }
+}
+
+template <bool AT, bool BT, bool F32>
 __global__ void __launch_bounds__(192, 1)
     gemm_bf16_nt_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-                        __nv_bfloat16 *__restrict__ C, int M, int N, int K, unsigned *err) {
+                        void *__restrict__ C, int M, int N, int K, unsigned *err) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t *full = reinterpret_cast<uint64_t *>(smem + STAGES * STAGE_BYTES);
@@ -73,8 +148,8 @@ __global__ void __launch_bounds__(192, 1)
           if (!mbar_wait(&empty[s], ph ^ 1, abort_flag, err)) break;
           uint8_t *a_s = smem + s * STAGE_BYTES;
           mbar_arrive_expect_tx(&full[s], STAGE_BYTES);
-          tma_load_2d(a_s, &tmA, &full[s], kt * BK, m0);
-          tma_load_2d(a_s + A_BYTES, &tmB, &full[s], kt * BK, n0);
+          load_operand<AT>(a_s, &tmA, &full[s], kt * BK, m0, BM);
+          load_operand<BT>(a_s + A_BYTES, &tmB, &full[s], kt * BK, n0, BN);
         }
       }
       if (*abort_flag)  // let copies in flight land before the CTA exits
@@ -83,7 +158,7 @@ __global__ void __launch_bounds__(192, 1)
     }
   } else if (warp == 1) {
     if (lane == 0) {
-      const uint32_t idesc = idesc_bf16_f32(BM, BN, 0, 0);
+      const uint32_t idesc = idesc_bf16_f32(BM, BN, AT ? 1 : 0, BT ? 1 : 0);
       int used = 0;  // K slices consumed so far (all tiles)
       int local = 0;
       bool ok = true;
@@ -100,9 +175,9 @@ __global__ void __launch_bounds__(192, 1)
           const uint32_t a_base = smem_u32(smem + s * STAGE_BYTES);
           const uint32_t b_base = a_base + A_BYTES;
 #pragma unroll
-          for (int k = 0; k < BK / 16; ++k)  // K=16 per MMA: +32 bytes inside the 128-byte swizzle row
-            mma_bf16_ss(tmem + 256u * b, sdesc_sw128(a_base + 32 * k, 16, 1024),
-                        sdesc_sw128(b_base + 32 * k, 16, 1024), idesc, (kt | k) != 0);
+          for (int k = 0; k < BK / 16; ++k)  // K=16 per MMA
+            mma_bf16_ss(tmem + 256u * b, operand_desc<AT>(a_base, k), operand_desc<BT>(b_base, k), idesc,
+                        (kt | k) != 0);
           mma_commit(&empty[s]);
         }
         if (ok) mma_commit(&acc_full[b]);
@@ -110,7 +185,6 @@ __global__ void __launch_bounds__(192, 1)
     }
   } else {
     const int qd = warp & 3;  // TMEM lane quadrant this warp may access
-    const bool vec = (N % 8) == 0;
     int local = 0;
     for (int t = blockIdx.x; t < n_tiles; t += gridDim.x, ++local) {
       const int b = local & 1;
@@ -122,25 +196,7 @@ __global__ void __launch_bounds__(192, 1)
         uint32_t r[32];
         tmem_ld32(tmem + 256u * b + (static_cast<uint32_t>(32 * qd) << 16) + c0, r);
         tmem_wait_ld();
-        const int col = n0 + c0;
-        if (row < M && col < N) {
-          __nv_bfloat16 *dst = C + static_cast<long long>(row) * N + col;
-          if (vec && col + 32 <= N) {
-#pragma unroll
-            for (int i = 0; i < 4; ++i) {
-              uint4 w;
-              w.x = pack_bf16x2(__uint_as_float(r[8 * i + 0]), __uint_as_float(r[8 * i + 1]));
-              w.y = pack_bf16x2(__uint_as_float(r[8 * i + 2]), __uint_as_float(r[8 * i + 3]));
-              w.z = pack_bf16x2(__uint_as_float(r[8 * i + 4]), __uint_as_float(r[8 * i + 5]));
-              w.w = pack_bf16x2(__uint_as_float(r[8 * i + 6]), __uint_as_float(r[8 * i + 7]));
-              reinterpret_cast<uint4 *>(dst)[i] = w;
-            }
-          } else {
-#pragma unroll
-            for (int i = 0; i < 32; ++i)
-              if (col + i < N) dst[i] = __float2bfloat16_rn(__uint_as_float(r[i]));
-          }
-        }
+        store_row32<F32>(C, row, n0 + c0, M, N, r);
       }
       tc_fence_before();
       __syncwarp();
@@ -166,9 +222,10 @@ constexpr int P_B_BYTES = 128 * BK * 2;                 // 16 KB (half of the 25
 constexpr int P_STAGE_BYTES = P_A_BYTES + P_B_BYTES;    // 32 KB
 constexpr int P_SMEM_BYTES = P_STAGES * P_STAGE_BYTES + 1024 + 256;
 
+template <bool AT, bool BT, bool F32>
 __global__ void __launch_bounds__(192, 1)
     gemm_bf16_nt_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-                             __nv_bfloat16 *__restrict__ C, int M, int N, int K, unsigned *err) {
+                             void *__restrict__ C, int M, int N, int K, unsigned *err) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t *full = reinterpret_cast<uint64_t *>(smem + P_STAGES * P_STAGE_BYTES);  // used in the first CTA
@@ -214,8 +271,8 @@ __global__ void __launch_bounds__(192, 1)
           if (rank == 0) mbar_arrive_expect_tx(&full[s], 2 * P_STAGE_BYTES);
           const uint32_t fb = map_peer(smem_u32(&full[s]), 0u);
           uint8_t *a_s = smem + s * P_STAGE_BYTES;
-          tma_load_2d_pair(a_s, &tmA, fb, kt * BK, am);
-          tma_load_2d_pair(a_s + P_A_BYTES, &tmB, fb, kt * BK, bn);
+          load_operand_pair<AT>(a_s, &tmA, fb, kt * BK, am, 128);
+          load_operand_pair<BT>(a_s + P_A_BYTES, &tmB, fb, kt * BK, bn, 128);
         }
       }
       // copies still in flight land before the CTA exits: both CTAs' loads are counted
@@ -226,7 +283,7 @@ __global__ void __launch_bounds__(192, 1)
     }
   } else if (warp == 1) {
     if (lane == 0 && rank == 0) {
-      const uint32_t idesc = idesc_bf16_f32(256, 256, 0, 0);
+      const uint32_t idesc = idesc_bf16_f32(256, 256, AT ? 1 : 0, BT ? 1 : 0);
       int used = 0, local = 0;
       bool ok = true;
       for (int t = pair; ok && t < n_tiles; t += n_pairs, ++local) {
@@ -241,8 +298,8 @@ __global__ void __launch_bounds__(192, 1)
           const uint32_t b_base = a_base + P_A_BYTES;
 #pragma unroll
           for (int k = 0; k < BK / 16; ++k)
-            mma_bf16_ss_pair(tmem + 256u * b, sdesc_sw128(a_base + 32 * k, 16, 1024),
-                             sdesc_sw128(b_base + 32 * k, 16, 1024), idesc, (kt | k) != 0);
+            mma_bf16_ss_pair(tmem + 256u * b, operand_desc<AT>(a_base, k), operand_desc<BT>(b_base, k), idesc,
+                             (kt | k) != 0);
           mma_commit_pair(&empty[s], 0x3);  // both CTAs' loaders may refill stage s
         }
         if (ok) mma_commit_pair(&acc_full[b], 0x3);
@@ -250,7 +307,6 @@ __global__ void __launch_bounds__(192, 1)
     }
   } else {
     const int qd = warp & 3;
-    const bool vec = (N % 8) == 0;
     const uint32_t acc_empty_first = map_peer(smem_u32(&acc_empty[0]), 0u);
     int local = 0;
     for (int t = pair; t < n_tiles; t += n_pairs, ++local) {
@@ -263,25 +319,7 @@ __global__ void __launch_bounds__(192, 1)
         uint32_t r[32];
         tmem_ld32(tmem + 256u * b + (static_cast<uint32_t>(32 * qd) << 16) + c0, r);
         tmem_wait_ld();
-        const int col = n0 + c0;
-        if (row < M && col < N) {
-          __nv_bfloat16 *dst = C + static_cast<long long>(row) * N + col;
-          if (vec && col + 32 <= N) {
-#pragma unroll
-            for (int i = 0; i < 4; ++i) {
-              uint4 w;
-              w.x = pack_bf16x2(__uint_as_float(r[8 * i + 0]), __uint_as_float(r[8 * i + 1]));
-              w.y = pack_bf16x2(__uint_as_float(r[8 * i + 2]), __uint_as_float(r[8 * i + 3]));
-              w.z = pack_bf16x2(__uint_as_float(r[8 * i + 4]), __uint_as_float(r[8 * i + 5]));
-              w.w = pack_bf16x2(__uint_as_float(r[8 * i + 6]), __uint_as_float(r[8 * i + 7]));
-              reinterpret_cast<uint4 *>(dst)[i] = w;
-            }
-          } else {
-#pragma unroll
-            for (int i = 0; i < 32; ++i)
-              if (col + i < N) dst[i] = __float2bfloat16_rn(__uint_as_float(r[i]));
-          }
-        }
+        store_row32<F32>(C, row, n0 + c0, M, N, r);
       }
       tc_fence_before();
       __syncwarp();
@@ -295,27 +333,28 @@ __global__ void __launch_bounds__(192, 1)
   if (warp == 1) { tc_fence_after(); tmem_dealloc_pair(tmem, TMEM_COLS); }
 }
 
-}  // namespace
-
-cudaError_t launch_gemm_bf16_nt(const void *A, const void *B, void *C, int M, int N, int K, unsigned *err,
-                                cudaStream_t stream) {
+template <bool AT, bool BT, bool F32>
+cudaError_t launch_gemm_impl(const void *A, const void *B, void *C, int M, int N, int K, unsigned *err,
+                             cudaStream_t stream) {
   alignas(64) CUtensorMap ta, tb;
-  const unsigned long long dA[2] = {static_cast<unsigned long long>(K), static_cast<unsigned long long>(M)};
-  const unsigned long long dB[2] = {static_cast<unsigned long long>(K), static_cast<unsigned long long>(N)};
-  const unsigned long long st[1] = {static_cast<unsigned long long>(K) * 2};
-  const unsigned boxA[2] = {BK, BM}, boxB[2] = {BK, BN};
-  if (!encode_tmap_bf16(&ta, A, 2, dA, st, boxA, true)) return cudaErrorInvalidValue;
-  if (!encode_tmap_bf16(&tb, B, 2, dB, st, boxB, true)) return cudaErrorInvalidValue;
+  // K-major operand [rows][K]: dims {K, rows}, box {64, R}; MN-major [K][rows]:
+  // dims {rows, K}, box {64, 64}
+  auto encode = [&](CUtensorMap *map, const void *base, bool mn, int rows, int R) {
+    const unsigned long long dims[2] = {static_cast<unsigned long long>(mn ? rows : K),
+                                        static_cast<unsigned long long>(mn ? K : rows)};
+    const unsigned long long st[1] = {static_cast<unsigned long long>(mn ? rows : K) * 2};
+    const unsigned box[2] = {64u, mn ? 64u : static_cast<unsigned>(R)};
+    return encode_tmap_bf16(map, base, 2, dims, st, box, true);
+  };
   int dev = 0, sms = 148;
   cudaError_t e;
   if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
   if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return e;
   if (kPairs && M >= 256) {
     // CTA pairs, persistent: as many pairs as are resident (at most one per 256 x 256 tile)
-    const unsigned boxB2[2] = {BK, 128};
-    if (!encode_tmap_bf16(&tb, B, 2, dB, st, boxB2, true)) return cudaErrorInvalidValue;
-    if ((e = cudaFuncSetAttribute(gemm_bf16_nt_pair_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                  P_SMEM_BYTES)) != cudaSuccess)
+    if (!encode(&ta, A, AT, M, 128) || !encode(&tb, B, BT, N, 128)) return cudaErrorInvalidValue;
+    auto kern = gemm_bf16_nt_pair_kernel<AT, BT, F32>;
+    if ((e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, P_SMEM_BYTES)) != cudaSuccess)
       return e;
     const long long tiles2 = static_cast<long long>((N + 255) / 256) * ((M + 255) / 256);
     cudaLaunchConfig_t cfg = {};
@@ -331,19 +370,42 @@ cudaError_t launch_gemm_bf16_nt(const void *A, const void *B, void *C, int M, in
     cfg.numAttrs = 1;
     cfg.gridDim = dim3(2 * (sms / 2));
     int pairs = 0;
-    if ((e = cudaOccupancyMaxActiveClusters(&pairs, gemm_bf16_nt_pair_kernel, &cfg)) != cudaSuccess) return e;
+    if ((e = cudaOccupancyMaxActiveClusters(&pairs, kern, &cfg)) != cudaSuccess) return e;
     if (pairs < 1) return cudaErrorInvalidConfiguration;
     const long long np = std::min<long long>(pairs, tiles2);
     cfg.gridDim = dim3(static_cast<unsigned>(2 * np));
-    return cudaLaunchKernelEx(&cfg, gemm_bf16_nt_pair_kernel, ta, tb, static_cast<__nv_bfloat16 *>(C), M, N, K, err);
+    return cudaLaunchKernelEx(&cfg, kern, ta, tb, C, M, N, K, err);
   }
-  if ((e = cudaFuncSetAttribute(gemm_bf16_nt_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES)) !=
-      cudaSuccess)
+  if (!encode(&ta, A, AT, M, BM) || !encode(&tb, B, BT, N, BN)) return cudaErrorInvalidValue;
+  auto kern = gemm_bf16_nt_kernel<AT, BT, F32>;
+  if ((e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES)) != cudaSuccess)
     return e;
   const long long tiles = static_cast<long long>((N + BN - 1) / BN) * ((M + BM - 1) / BM);
   const int grid = static_cast<int>(tiles < sms ? tiles : sms);
-  gemm_bf16_nt_kernel<<<grid, 192, SMEM_BYTES, stream>>>(ta, tb, static_cast<__nv_bfloat16 *>(C), M, N, K, err);
+  kern<<<grid, 192, SMEM_BYTES, stream>>>(ta, tb, C, M, N, K, err);
   return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_gemm(const void *A, const void *B, void *C, int M, int N, int K, bool a_mn, bool b_mn,
+                        bool f32_out, unsigned *err, cudaStream_t stream) {
+  const int sel = (a_mn ? 4 : 0) | (b_mn ? 2 : 0) | (f32_out ? 1 : 0);
+  switch (sel) {
+    case 0: return launch_gemm_impl<false, false, false>(A, B, C, M, N, K, err, stream);
+    case 1: return launch_gemm_impl<false, false, true>(A, B, C, M, N, K, err, stream);
+    case 3: return launch_gemm_impl<false, true, true>(A, B, C, M, N, K, err, stream);
+    case 7: return launch_gemm_impl<true, true, true>(A, B, C, M, N, K, err, stream);
+    case 2: return launch_gemm_impl<false, true, false>(A, B, C, M, N, K, err, stream);
+    case 4: return launch_gemm_impl<true, false, false>(A, B, C, M, N, K, err, stream);
+    case 5: return launch_gemm_impl<true, false, true>(A, B, C, M, N, K, err, stream);
+    default: return launch_gemm_impl<true, true, false>(A, B, C, M, N, K, err, stream);
+  }
+}
+
+cudaError_t launch_gemm_bf16_nt(const void *A, const void *B, void *C, int M, int N, int K, unsigned *err,
+                                cudaStream_t stream) {
+  return launch_gemm(A, B, C, M, N, K, false, false, false, err, stream);
 }
 
 }  // namespace mta

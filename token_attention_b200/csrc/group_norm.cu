@@ -123,7 +123,115 @@ __global__ void __launch_bounds__(256) group_norm_any_kernel(const __nv_bfloat16
   }
 }
 
+// Backward of the scaled group norm, for (token, head) rows of head h = blockIdx.x:
+// given dy, recomputes xhat = (o - mean) * rstd and returns
+//   y  = m (xhat gamma + beta)                        (bf16, the output projection's operand)
+//   do = rstd (g - mean(g) - xhat mean(g xhat)),  g = m gamma dy   (bf16)
+// and adds the block's sums of dgamma = m dy xhat, dbeta = m dy and, with a gate,
+// dgate_h = m (1 - m) sum dy (xhat gamma + beta) to the fp32 outputs (zeroed by the
+// caller).  A warp per row, channel e = lane + 32 c in lane `lane`, CPL = d / 32
+// channels per lane; 8 warps take kGnBwdRows consecutive tokens of the head, so a
+// block adds 2 d (+1) values instead of 2 d per row.
+constexpr int kGnBwdRows = 64;
+
+template <int CPL>
+__global__ void __launch_bounds__(256) group_norm_bwd_kernel(const __nv_bfloat16 *__restrict__ o,
+                                                             const float *__restrict__ dy, GnArgs gn, int tokens,
+                                                             int H, __nv_bfloat16 *__restrict__ y,
+                                                             __nv_bfloat16 *__restrict__ dout, float *dgamma,
+                                                             float *dbeta, float *dgate) {
+  constexpr int d = 32 * CPL;
+  __shared__ float red[8][2 * d + 1];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int h = blockIdx.x;
+  const float m = head_multiplier(gn.gate, gn.lam, h);
+  float gam[CPL], bet[CPL], dga[CPL], dbe[CPL];
+#pragma unroll
+  for (int c = 0; c < CPL; ++c) {
+    gam[c] = gn.gamma[h * d + lane + 32 * c];
+    bet[c] = gn.beta[h * d + lane + 32 * c];
+    dga[c] = 0.f;
+    dbe[c] = 0.f;
+  }
+  float dgt = 0.f;
+  const int t_end = min(tokens, (blockIdx.y + 1) * kGnBwdRows);
+  for (int t = blockIdx.y * kGnBwdRows + warp; t < t_end; t += 8) {
+    const long long base = (static_cast<long long>(t) * H + h) * d;
+    float x[CPL], g[CPL];
+    float s = 0.f;
+#pragma unroll
+    for (int c = 0; c < CPL; ++c) {
+      x[c] = __bfloat162float(o[base + lane + 32 * c]);
+      g[c] = dy[base + lane + 32 * c];
+      s += x[c];
+    }
+    const float mu = warp_sum(s) * (1.f / d);
+    float s2 = 0.f;
+#pragma unroll
+    for (int c = 0; c < CPL; ++c) {
+      x[c] -= mu;
+      s2 += x[c] * x[c];
+    }
+    const float rstd = rsqrtf(warp_sum(s2) * (1.f / d) + gn.eps);
+    float sg = 0.f, sgx = 0.f, sdg = 0.f;
+#pragma unroll
+    for (int c = 0; c < CPL; ++c) {
+      const float xh = x[c] * rstd, aff = xh * gam[c] + bet[c];
+      y[base + lane + 32 * c] = __float2bfloat16_rn(m * aff);
+      dga[c] += m * g[c] * xh;
+      dbe[c] += m * g[c];
+      sdg += g[c] * aff;
+      const float gx = m * gam[c] * g[c];
+      g[c] = gx;
+      x[c] = xh;
+      sg += gx;
+      sgx += gx * xh;
+    }
+    const float mg = warp_sum(sg) * (1.f / d), mgx = warp_sum(sgx) * (1.f / d);
+#pragma unroll
+    for (int c = 0; c < CPL; ++c)
+      dout[base + lane + 32 * c] = __float2bfloat16_rn(rstd * (g[c] - mg - x[c] * mgx));
+    dgt += sdg;
+  }
+#pragma unroll
+  for (int c = 0; c < CPL; ++c) {
+    red[warp][lane + 32 * c] = dga[c];
+    red[warp][d + lane + 32 * c] = dbe[c];
+  }
+  dgt = warp_sum(dgt);
+  if (lane == 0) red[warp][2 * d] = dgt;
+  __syncthreads();
+  for (int i = threadIdx.x; i < 2 * d + 1; i += blockDim.x) {
+    float v = 0.f;
+#pragma unroll
+    for (int w = 0; w < 8; ++w) v += red[w][i];
+    if (i < d)
+      atomicAdd(dgamma + h * d + i, v);
+    else if (i < 2 * d)
+      atomicAdd(dbeta + h * d + (i - d), v);
+    else if (gn.gate && dgate)
+      atomicAdd(dgate + h, v * m * (1.f - m));
+  }
+}
+
 }  // namespace
+
+cudaError_t launch_group_norm_bwd(const void *o, const float *dy, const GnArgs &gn, int tokens, int H, int d,
+                                  void *y, void *dout, float *dgamma, float *dbeta, float *dgate,
+                                  cudaStream_t stream) {
+  if (tokens == 0) return cudaSuccess;
+  const dim3 grid(static_cast<unsigned>(H), static_cast<unsigned>((tokens + kGnBwdRows - 1) / kGnBwdRows));
+  const __nv_bfloat16 *src = static_cast<const __nv_bfloat16 *>(o);
+  __nv_bfloat16 *yb = static_cast<__nv_bfloat16 *>(y), *db = static_cast<__nv_bfloat16 *>(dout);
+  switch (d) {
+    case 32: group_norm_bwd_kernel<1><<<grid, 256, 0, stream>>>(src, dy, gn, tokens, H, yb, db, dgamma, dbeta, dgate); break;
+    case 64: group_norm_bwd_kernel<2><<<grid, 256, 0, stream>>>(src, dy, gn, tokens, H, yb, db, dgamma, dbeta, dgate); break;
+    case 96: group_norm_bwd_kernel<3><<<grid, 256, 0, stream>>>(src, dy, gn, tokens, H, yb, db, dgamma, dbeta, dgate); break;
+    case 128: group_norm_bwd_kernel<4><<<grid, 256, 0, stream>>>(src, dy, gn, tokens, H, yb, db, dgamma, dbeta, dgate); break;
+    default: return cudaErrorInvalidValue;
+  }
+  return cudaGetLastError();
+}
 
 cudaError_t launch_group_norm(const void *o, const GnArgs &gn, int tokens, int H, int d, void *y,
                               cudaStream_t stream) {

@@ -114,17 +114,29 @@ size_t attn_kq_workspace_bytes(int B, int H, int L, int d, int cq, int ck, int h
 cudaError_t launch_attn_kq(const AttnArgs &a, const GnArgs *gn, void *ws);
 // The contraction kernel on CTA pairs (attn_kq_pair.cu): the shapes it serves, the
 // scratch it needs after the prepass's operands, and its launch.
-bool attn_kq_pair_applies(int d, int kq, int hp, int kqp);
+bool attn_kq_pair_applies(int d, int kq, int hp, int kqp, int L);
 size_t attn_kq_pair_scratch_bytes(int B, int H, int L, int d, int hp);
 cudaError_t launch_attn_kq_pair(const AttnArgs &a, const GnArgs *gn, const KqPrepArgs &pa, void *scratch);
 
 // tcgen05 GEMM: C[M][N] = A[M][K] * B[N][K]^T (bf16 -> fp32 -> bf16).
+// C[M][N] = A B^T with A [M][K] (a_mn: stored [K][M]) and B [N][K] (b_mn: stored
+// [K][N]), bf16 in, fp32 accumulate, bf16 or (f32_out) fp32 out.
+cudaError_t launch_gemm(const void *A, const void *B, void *C, int M, int N, int K, bool a_mn, bool b_mn,
+                        bool f32_out, unsigned *err, cudaStream_t stream);
 cudaError_t launch_gemm_bf16_nt(const void *A, const void *B, void *C, int M, int N, int K,
                                 unsigned *err, cudaStream_t stream);
 
 // Depth-scaled group norm over [tokens][H][d] bf16.
 cudaError_t launch_group_norm(const void *o, const GnArgs &gn, int tokens, int H, int d, void *y,
                               cudaStream_t stream);
+// Backward of the group norm (d in {32, 64, 96, 128}): o, y, dout bf16 and dy fp32,
+// all [tokens][H][d]; adds into dgamma, dbeta [H*d] and (with a gate) dgate [H].
+cudaError_t launch_group_norm_bwd(const void *o, const float *dy, const GnArgs &gn, int tokens, int H, int d,
+                                  void *y, void *dout, float *dgamma, float *dbeta, float *dgate,
+                                  cudaStream_t stream);
+// [tokens][3 H d] bf16 = (dq | dk | dv), each fp32 [tokens][H d]
+cudaError_t launch_pack_qkv_grad(const float *dq, const float *dk, const float *dv, long long tokens, int hd,
+                                 void *dqkv, cudaStream_t stream);
 
 // Diagnostic: one CTA whose bounded waits cannot complete (selftest.cu); err is the
 // workspace's error word, out[2] counters of the waits that gave up.

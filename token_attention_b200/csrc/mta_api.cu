@@ -181,6 +181,43 @@ GnArgs make_gn(const mta_gn *gn) {
   return g;
 }
 
+// The attention backward's arguments (see mta_attn_bwd).
+BwdArgs make_bwd_args(const void *q, const void *k, const void *v, const float *theta_kq, const float *w_head,
+                      const void *dout, const mta_cfg *cfg, float *dq, float *dk, float *dv, float *dtheta,
+                      float *dw) {
+  BwdArgs a;
+  a.q = q; a.k = k; a.v = v; a.dout = dout;
+  a.rs = cfg->qkv_row_stride ? cfg->qkv_row_stride : static_cast<long long>(cfg->H) * cfg->d;
+  a.theta = theta_kq; a.w = w_head;
+  a.dq = dq; a.dk = dk; a.dv = dv;
+  // theta_kq (and dtheta) hold the pre-softmax kernels when on, then the post-softmax ones
+  const size_t nth = static_cast<size_t>(cfg->H) * cfg->c_q * cfg->c_k;
+  a.dtheta = cfg->kq_place != MTA_OFF ? dtheta : nullptr;
+  a.kqp = cfg->kq_post;
+  a.theta_post = cfg->kq_post ? theta_kq + (cfg->kq_place != MTA_OFF ? nth : 0) : nullptr;
+  a.dtheta_post = (cfg->kq_post && dtheta) ? dtheta + (cfg->kq_place != MTA_OFF ? nth : 0) : nullptr;
+  a.dw = cfg->head_place != MTA_OFF ? dw : nullptr;
+  a.B = cfg->B; a.H = cfg->H; a.L = cfg->L; a.d = cfg->d;
+  a.cq = cfg->c_q; a.ck = cfg->c_k; a.ch = cfg->c_h;
+  a.kq = cfg->kq_place; a.hp = cfg->head_place; a.dtype = cfg->dtype;
+  a.scale = cfg->scale > 0.f ? cfg->scale : 1.0f / sqrtf(static_cast<float>(cfg->d));
+  a.stream = static_cast<cudaStream_t>(cfg->stream);
+  return a;
+}
+
+bool bwd_supported(const BwdArgs &a) {
+  return (a.kqp ? attn_bwd_post_pick_rows(a) : attn_bwd_simt_pick_rows(a)) != 0;
+}
+
+// The layer backward's fixed scratch, in this order (each 256-byte aligned): the
+// error word; QKV, O, Y (bf16); dY (fp32); dO (bf16); the attention core's fp32
+// gradients dq, dk, dv; dQKV (bf16).  All of them hold their values after the call.
+size_t layer_bwd_fixed_bytes(const mta_cfg *cfg) {
+  if (check_cfg(cfg) != MTA_OK) return 0;
+  const size_t T = static_cast<size_t>(cfg->B) * cfg->L, D = static_cast<size_t>(cfg->H) * cfg->d;
+  return kStatusBytes + 2 * align_up(T * 3 * D * 2) + 3 * align_up(T * D * 2) + 4 * align_up(T * D * 4);
+}
+
 }  // namespace
 
 bool encode_tmap_bf16(void *map_out, const void *base, int rank, const unsigned long long *dims,
@@ -363,29 +400,117 @@ mta_status mta_attn_bwd(const void *q, const void *k, const void *v, const float
   }
   if ((dtheta && !aligned(dtheta, 4)) || (dw && !aligned(dw, 4))) return MTA_ERR_INVALID;
   if ((s = check_workspace(cfg, kStatusBytes)) != MTA_OK) return s;
-  BwdArgs a;
-  a.q = q; a.k = k; a.v = v; a.dout = dout;
-  a.rs = cfg->qkv_row_stride ? cfg->qkv_row_stride : static_cast<long long>(cfg->H) * cfg->d;
-  a.theta = theta_kq; a.w = w_head;
-  a.dq = dq; a.dk = dk; a.dv = dv;
-  // theta_kq (and dtheta) hold the pre-softmax kernels when on, then the post-softmax ones
-  const size_t nth = static_cast<size_t>(cfg->H) * cfg->c_q * cfg->c_k;
-  a.dtheta = cfg->kq_place != MTA_OFF ? dtheta : nullptr;
-  a.kqp = cfg->kq_post;
-  a.theta_post = cfg->kq_post ? theta_kq + (cfg->kq_place != MTA_OFF ? nth : 0) : nullptr;
-  a.dtheta_post = (cfg->kq_post && dtheta) ? dtheta + (cfg->kq_place != MTA_OFF ? nth : 0) : nullptr;
-  a.dw = cfg->head_place != MTA_OFF ? dw : nullptr;
-  a.B = cfg->B; a.H = cfg->H; a.L = cfg->L; a.d = cfg->d;
-  a.cq = cfg->c_q; a.ck = cfg->c_k; a.ch = cfg->c_h;
-  a.kq = cfg->kq_place; a.hp = cfg->head_place; a.dtype = cfg->dtype;
-  a.scale = cfg->scale > 0.f ? cfg->scale : 1.0f / sqrtf(static_cast<float>(cfg->d));
-  a.stream = static_cast<cudaStream_t>(cfg->stream);
-  if ((a.kqp ? attn_bwd_post_pick_rows(a) : attn_bwd_simt_pick_rows(a)) == 0) return MTA_ERR_UNSUPPORTED;
+  BwdArgs a = make_bwd_args(q, k, v, theta_kq, w_head, dout, cfg, dq, dk, dv, dtheta, dw);
+  if (!bwd_supported(a)) return MTA_ERR_UNSUPPORTED;
   if ((s = clear_status(cfg)) != MTA_OK) return s;
   Marks m = make_marks(cfg);
   if (m.next() != cudaSuccess) return MTA_ERR_CUDA;
   if ((a.kqp ? launch_attn_bwd_post(a) : launch_attn_bwd_simt(a)) != cudaSuccess) return MTA_ERR_CUDA;
   return m.next() == cudaSuccess ? MTA_OK : MTA_ERR_CUDA;
+}
+
+size_t mta_layer_bwd_workspace_bytes(const mta_cfg *cfg) {
+  const size_t fixed = layer_bwd_fixed_bytes(cfg);
+  return fixed ? fixed + kq_bytes(cfg) : 0;
+}
+
+mta_status mta_layer_bwd(const void *x, const void *Wqkv, const float *theta, const float *w_head,
+                         const mta_gn *gn, const void *Wo, const void *dout, const mta_cfg *cfg, float *dx,
+                         float *dWqkv, float *dWo, float *dtheta, float *dw, float *dgamma, float *dbeta,
+                         float *dgate) {
+  mta_status s = check_cfg(cfg);
+  if (s != MTA_OK) return s;
+  if (cfg->dtype != MTA_BF16) return MTA_ERR_UNSUPPORTED;
+  if (!x || !Wqkv || !Wo || !dout || !gn || !gn->gamma || !gn->beta) return MTA_ERR_INVALID;
+  if (!dx || !dWqkv || !dWo || !dgamma || !dbeta || (gn->gate && !dgate)) return MTA_ERR_INVALID;
+  if ((cfg->kq_place != MTA_OFF || cfg->kq_post) && !theta) return MTA_ERR_INVALID;
+  if (cfg->head_place != MTA_OFF && !w_head) return MTA_ERR_INVALID;
+  if (!aligned(x, 16) || !aligned(Wqkv, 16) || !aligned(Wo, 16) || !aligned(dout, 16)) return MTA_ERR_INVALID;
+  if (!aligned(dx, 16) || !aligned(dWqkv, 16) || !aligned(dWo, 16) || !aligned(dgamma, 4) ||
+      !aligned(dbeta, 4) || (dgate && !aligned(dgate, 4)) || (dtheta && !aligned(dtheta, 4)) ||
+      (dw && !aligned(dw, 4)) || (theta && !aligned(theta, 4)) || !aligned(gn->gamma, 4) || !aligned(gn->beta, 4))
+    return MTA_ERR_INVALID;
+  const size_t T = layer_tokens(cfg), D = static_cast<size_t>(cfg->H) * cfg->d;
+  if (T > static_cast<size_t>(65535) * 64 || 3 * D > static_cast<size_t>(1) << 30) return MTA_ERR_UNSUPPORTED;
+  if (cfg->d != 32 && cfg->d != 64 && cfg->d != 96 && cfg->d != 128) return MTA_ERR_UNSUPPORTED;
+  {
+    // no output may share memory with an input or with another output
+    const void *in[4] = {x, Wqkv, Wo, dout};
+    const size_t nin[4] = {T * D * 2, 3 * D * D * 2, D * D * 2, T * D * 2};
+    const void *outp[3] = {dx, dWqkv, dWo};
+    const size_t nout[3] = {T * D * 4, 3 * D * D * 4, D * D * 4};
+    for (int i = 0; i < 3; ++i) {
+      for (int j = 0; j < 4; ++j)
+        if (overlaps(outp[i], nout[i], in[j], nin[j])) return MTA_ERR_INVALID;
+      for (int j = 0; j < i; ++j)
+        if (overlaps(outp[i], nout[i], outp[j], nout[j])) return MTA_ERR_INVALID;
+    }
+  }
+  if ((s = check_workspace(cfg, layer_bwd_fixed_bytes(cfg))) != MTA_OK) return s;
+
+  char *ws = static_cast<char *>(cfg->workspace);
+  char *qkv = ws + kStatusBytes;
+  char *obuf = qkv + align_up(T * 3 * D * 2);
+  char *ybuf = obuf + align_up(T * D * 2);
+  char *dybuf = ybuf + align_up(T * D * 2);
+  char *dobuf = dybuf + align_up(T * D * 4);
+  float *dq = reinterpret_cast<float *>(dobuf + align_up(T * D * 2));
+  float *dk = reinterpret_cast<float *>(reinterpret_cast<char *>(dq) + align_up(T * D * 4));
+  float *dv = reinterpret_cast<float *>(reinterpret_cast<char *>(dk) + align_up(T * D * 4));
+  char *dqkv = reinterpret_cast<char *>(dv) + align_up(T * D * 4);
+  char *kq_ws = dqkv + align_up(T * 3 * D * 2);
+  const size_t kq_room = cfg->workspace_bytes - (kq_ws - ws);
+  const uint16_t *qkvb = reinterpret_cast<const uint16_t *>(qkv);
+
+  // the forward's attention (recomputed) and the attention backward, both on QKV
+  mta_cfg acfg = *cfg;
+  acfg.qkv_row_stride = static_cast<long long>(3 * D);
+  AttnArgs a = make_args(qkvb, qkvb + D, qkvb + 2 * D, theta, w_head, &acfg, obuf);
+  Kernel kern = K_SIMT;
+  if ((s = select_kernel(a, cfg->path, kq_room, &kern)) != MTA_OK) return s;
+  mta_cfg bcfg = acfg;
+  bcfg.path = 0;
+  BwdArgs ba = make_bwd_args(qkvb, qkvb + D, qkvb + 2 * D, theta, w_head, dobuf, &bcfg, dq, dk, dv, dtheta, dw);
+  if (!bwd_supported(ba)) return MTA_ERR_UNSUPPORTED;
+
+  const GnArgs g = make_gn(gn);
+  cudaStream_t st = static_cast<cudaStream_t>(cfg->stream);
+  unsigned *err = static_cast<unsigned *>(cfg->workspace);
+  if ((s = clear_status(cfg)) != MTA_OK) return s;
+  if (cudaMemsetAsync(dgamma, 0, D * 4, st) != cudaSuccess || cudaMemsetAsync(dbeta, 0, D * 4, st) != cudaSuccess ||
+      (gn->gate && cudaMemsetAsync(dgate, 0, cfg->H * 4, st) != cudaSuccess))
+    return MTA_ERR_CUDA;
+  Marks m = make_marks(cfg);
+  a.marks = &m;
+  const int iT = static_cast<int>(T), iD = static_cast<int>(D), i3D = static_cast<int>(3 * D);
+  if (m.next() != cudaSuccess) return MTA_ERR_CUDA;
+  // forward: QKV = x Wqkv^T, O = attention(QKV)
+  if (launch_gemm(x, Wqkv, qkv, iT, i3D, iD, false, false, false, err, st) != cudaSuccess || m.next() != cudaSuccess)
+    return MTA_ERR_CUDA;
+  if (launch_kernel(kern, a, nullptr, kq_ws) != cudaSuccess) return MTA_ERR_CUDA;
+  // dY = dOut Wo (Wo read as the MN-major operand)
+  if (launch_gemm(dout, Wo, dybuf, iT, iD, iD, false, true, true, err, st) != cudaSuccess || m.next() != cudaSuccess)
+    return MTA_ERR_CUDA;
+  // group norm: Y, dO, dgamma, dbeta, dgate
+  if (launch_group_norm_bwd(obuf, reinterpret_cast<const float *>(dybuf), g, iT, cfg->H, cfg->d, ybuf, dobuf, dgamma,
+                            dbeta, dgate, st) != cudaSuccess ||
+      m.next() != cudaSuccess)
+    return MTA_ERR_CUDA;
+  // dWo = dOut^T Y (both operands MN-major, K = tokens)
+  if (launch_gemm(dout, ybuf, dWo, iD, iD, iT, true, true, true, err, st) != cudaSuccess || m.next() != cudaSuccess)
+    return MTA_ERR_CUDA;
+  // attention core: dq, dk, dv (fp32), dtheta, dw
+  if ((ba.kqp ? launch_attn_bwd_post(ba) : launch_attn_bwd_simt(ba)) != cudaSuccess || m.next() != cudaSuccess)
+    return MTA_ERR_CUDA;
+  if (launch_pack_qkv_grad(dq, dk, dv, static_cast<long long>(T), iD, dqkv, st) != cudaSuccess ||
+      m.next() != cudaSuccess)
+    return MTA_ERR_CUDA;
+  // dx = dQKV Wqkv, dWqkv = dQKV^T x
+  if (launch_gemm(dqkv, Wqkv, dx, iT, iD, i3D, false, true, true, err, st) != cudaSuccess || m.next() != cudaSuccess)
+    return MTA_ERR_CUDA;
+  if (launch_gemm(dqkv, x, dWqkv, i3D, iD, iT, true, true, true, err, st) != cudaSuccess || m.next() != cudaSuccess)
+    return MTA_ERR_CUDA;
+  return MTA_OK;
 }
 
 mta_status mta_gemm_bf16_nt(const void *A, const void *Bm, void *C, int M, int N, int K, void *stream) {
@@ -406,6 +531,44 @@ mta_status mta_group_norm_scale(const void *o, const mta_gn *gn, int tokens, int
     return MTA_ERR_INVALID;
   return launch_group_norm(o, make_gn(gn), tokens, H, d, y, static_cast<cudaStream_t>(stream)) ==
                  cudaSuccess
+             ? MTA_OK
+             : MTA_ERR_CUDA;
+}
+
+mta_status mta_gemm_bf16(const void *A, const void *Bm, void *C, int M, int N, int K, int a_mn, int b_mn,
+                         int f32_out, void *stream) {
+  if (!A || !Bm || !C || M < 1 || N < 1 || K < 1) return MTA_ERR_INVALID;
+  if ((a_mn != 0 && a_mn != 1) || (b_mn != 0 && b_mn != 1) || (f32_out != 0 && f32_out != 1))
+    return MTA_ERR_INVALID;
+  if ((a_mn ? M : K) % 8 != 0 || (b_mn ? N : K) % 8 != 0) return MTA_ERR_INVALID;
+  if (!aligned(A, 16) || !aligned(Bm, 16) || !aligned(C, 16)) return MTA_ERR_INVALID;
+  const size_t es = f32_out ? 4 : 2;
+  if (overlaps(C, static_cast<size_t>(M) * N * es, A, static_cast<size_t>(M) * K * 2) ||
+      overlaps(C, static_cast<size_t>(M) * N * es, Bm, static_cast<size_t>(N) * K * 2))
+    return MTA_ERR_INVALID;
+  return launch_gemm(A, Bm, C, M, N, K, a_mn != 0, b_mn != 0, f32_out != 0, nullptr,
+                     static_cast<cudaStream_t>(stream)) == cudaSuccess
+             ? MTA_OK
+             : MTA_ERR_CUDA;
+}
+
+mta_status mta_group_norm_scale_bwd(const void *o, const float *dy, const mta_gn *gn, int tokens, int H, int d,
+                                    void *y, void *dout, float *dgamma, float *dbeta, float *dgate,
+                                    void *stream) {
+  if (!o || !dy || !gn || !gn->gamma || !gn->beta || !y || !dout || !dgamma || !dbeta || tokens < 0 || H < 1)
+    return MTA_ERR_INVALID;
+  if (gn->gate && !dgate) return MTA_ERR_INVALID;
+  if (d != 32 && d != 64 && d != 96 && d != 128) return MTA_ERR_UNSUPPORTED;
+  if (tokens > 65535 * 64) return MTA_ERR_UNSUPPORTED;
+  if (!aligned(o, 2) || !aligned(y, 2) || !aligned(dout, 2) || !aligned(dy, 4) || !aligned(dgamma, 4) ||
+      !aligned(dbeta, 4) || (dgate && !aligned(dgate, 4)) || !aligned(gn->gamma, 4) || !aligned(gn->beta, 4))
+    return MTA_ERR_INVALID;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const size_t hd = static_cast<size_t>(H) * d;
+  if (cudaMemsetAsync(dgamma, 0, hd * 4, st) != cudaSuccess || cudaMemsetAsync(dbeta, 0, hd * 4, st) != cudaSuccess ||
+      (gn->gate && cudaMemsetAsync(dgate, 0, static_cast<size_t>(H) * 4, st) != cudaSuccess))
+    return MTA_ERR_CUDA;
+  return launch_group_norm_bwd(o, dy, make_gn(gn), tokens, H, d, y, dout, dgamma, dbeta, dgate, st) == cudaSuccess
              ? MTA_OK
              : MTA_ERR_CUDA;
 }

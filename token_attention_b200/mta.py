@@ -27,7 +27,8 @@ EXPORTS = ["mta_attn_workspace_bytes", "mta_attn_fwd", "mta_layer_workspace_byte
            "mta_layer_fwd", "mta_gemm_bf16_nt", "mta_group_norm_scale", "mta_sync_status",
            "mta_status_string", "mta_abi_version", "mta_layer_fwd_static",
            "mta_attn_bwd_workspace_bytes", "mta_attn_bwd", "mta_attn_kernel",
-           "mta_selftest_wait_timeout"]
+           "mta_selftest_wait_timeout", "mta_layer_bwd_workspace_bytes", "mta_layer_bwd",
+           "mta_gemm_bf16", "mta_group_norm_scale_bwd"]
 
 
 class MtaCfg(ctypes.Structure):
@@ -80,6 +81,14 @@ def lib() -> ctypes.CDLL:
         L.mta_attn_bwd_workspace_bytes.restype = S
         L.mta_attn_bwd.argtypes = [P, P, P, P, P, P, cfgp, P, P, P, P, P]
         L.mta_attn_bwd.restype = I
+        L.mta_layer_bwd_workspace_bytes.argtypes = [cfgp]
+        L.mta_layer_bwd_workspace_bytes.restype = S
+        L.mta_layer_bwd.argtypes = [P, P, P, P, ctypes.POINTER(MtaGn), P, P, cfgp] + [P] * 8
+        L.mta_layer_bwd.restype = I
+        L.mta_gemm_bf16.argtypes = [P, P, P, I, I, I, I, I, I, P]
+        L.mta_gemm_bf16.restype = I
+        L.mta_group_norm_scale_bwd.argtypes = [P, P, ctypes.POINTER(MtaGn), I, I, I, P, P, P, P, P, P]
+        L.mta_group_norm_scale_bwd.restype = I
         L.mta_attn_kernel.argtypes = [cfgp]
         L.mta_attn_kernel.restype = I
         L.mta_selftest_wait_timeout.argtypes = [cfgp, ctypes.c_uint]
@@ -385,6 +394,60 @@ def layer_fwd(x, wqkv, theta, w, gamma, beta, wo, H, c_q, c_k, c_h, kq_place=PRE
     return out
 
 
+def layer_bwd(x, wqkv, theta, w, gamma, beta, wo, dout, H, c_q, c_k, c_h, kq_place=PRE,
+              head_place=POST, *, eps=1e-5, layer=12, lam=-1.0, gate=None, ws=None,
+              path=PATH_AUTO, stream=None, check=False, theta_post=None, events=None):
+    """Gradients of layer_fwd for dout [B, L, D] bf16.  Returns a dict of fp32
+    tensors: dx [B, L, D], dwqkv [3D, D], dwo [D, D], dgamma, dbeta [D], dgate [H]
+    (with a gate), dtheta / dtheta_post [H, c_q, c_k] (views of dtheta_all, laid
+    out as the kernel array) and dw [H/c_h, c_h, c_h] as for attn_bwd."""
+    import torch
+    B, L, D = x.shape
+    if D % H:
+        raise ValueError(f"D = {D} is not a multiple of H = {H}")
+    d = D // H
+    dv = x.device
+    _need("x", x, dv)
+    _need("wqkv", wqkv, dv, x.dtype, (3 * D, D))
+    _need("wo", wo, dv, x.dtype, (D, D))
+    _need("dout", dout, dv, x.dtype, (B, L, D))
+    for name, t in (("theta", theta), ("w", w), ("theta_post", theta_post)):
+        _need(name, t, dv, torch.float32)
+    _need("gamma", gamma, dv, torch.float32, (D,))
+    _need("beta", beta, dv, torch.float32, (D,))
+    _need("gate", gate, dv, torch.float32, (H,))
+    _need("ws", ws, dv)
+    theta, kq_post = _kernels(theta, theta_post, kq_place)
+    n_th = (1 if kq_place != OFF else 0) + kq_post
+    z = lambda *shape: torch.empty(shape, dtype=torch.float32, device=dv)
+    dth = z(n_th, H, c_q, c_k) if n_th else None
+    g = {"dx": z(B, L, D), "dwqkv": z(3 * D, D), "dwo": z(D, D), "dgamma": z(D), "dbeta": z(D),
+         "dgate": z(H) if gate is not None else None, "dtheta_all": dth,
+         "dtheta": dth[0] if kq_place != OFF else None,
+         "dtheta_post": dth[n_th - 1] if kq_post else None,
+         "dw": z(H // c_h, c_h, c_h) if head_place != OFF else None}
+    cfg = make_cfg(B, H, L, d, c_q, c_k, c_h, kq_place, head_place, _dtype_code(x), path, 0.0, 0,
+                   _stream_handle(stream), kq_post=kq_post, events=events)
+    if ws is None:
+        ws = workspace(lib().mta_layer_bwd_workspace_bytes(ctypes.byref(cfg)), x.device)
+    cfg.workspace, cfg.workspace_bytes = ws.data_ptr(), _nbytes(ws)
+    gn = MtaGn(gamma.data_ptr(), beta.data_ptr(), eps, layer, lam,
+               gate.data_ptr() if gate is not None else None)
+    _check("mta_layer_bwd", lib().mta_layer_bwd(
+        _ptr(x), _ptr(wqkv), _ptr(theta), _ptr(w), ctypes.byref(gn), _ptr(wo), _ptr(dout),
+        ctypes.byref(cfg), _ptr(g["dx"]), _ptr(g["dwqkv"]), _ptr(g["dwo"]), _ptr(g["dtheta_all"]),
+        _ptr(g["dw"]), _ptr(g["dgamma"]), _ptr(g["dbeta"]), _ptr(g["dgate"])))
+    if check:
+        _check("mta_sync_status", lib().mta_sync_status(ctypes.byref(cfg)))
+    return g
+
+
+def layer_bwd_workspace_bytes(B, L, H, d, c_q, c_k, c_h, kq_place=PRE, head_place=POST,
+                              kq_post=0) -> int:
+    cfg = make_cfg(B, H, L, d, c_q, c_k, c_h, kq_place, head_place, BF16, kq_post=kq_post)
+    return lib().mta_layer_bwd_workspace_bytes(ctypes.byref(cfg))
+
+
 def layer_workspace_bytes(B, L, H, d, c_q, c_k, c_h, kq_place=PRE, head_place=POST,
                           kq_post=0) -> int:
     cfg = make_cfg(B, H, L, d, c_q, c_k, c_h, kq_place, head_place, BF16, kq_post=kq_post)
@@ -404,6 +467,45 @@ def gemm_bf16_nt(a, b, out=None, stream=None):
     _check("mta_gemm_bf16_nt", lib().mta_gemm_bf16_nt(_ptr(a), _ptr(b), _ptr(out), M, N, K,
                                                      _stream_handle(stream)))
     return out
+
+
+def gemm_bf16(a, b, M, N, K, a_mn=False, b_mn=False, f32_out=False, out=None, stream=None):
+    """C [M, N] = A B^T with A given as a [M, K] (a_mn: as [K, M]) and B as b [N, K]
+    (b_mn: as [K, N]), bf16 contiguous; C bf16, or fp32 with f32_out."""
+    import torch
+    _need("a", a, a.device, torch.bfloat16, (K, M) if a_mn else (M, K))
+    _need("b", b, a.device, torch.bfloat16, (K, N) if b_mn else (N, K))
+    odt = torch.float32 if f32_out else torch.bfloat16
+    _need("out", out, a.device, odt, (M, N))
+    if out is None:
+        out = torch.empty((M, N), dtype=odt, device=a.device)
+    _check("mta_gemm_bf16", lib().mta_gemm_bf16(_ptr(a), _ptr(b), _ptr(out), M, N, K, int(a_mn), int(b_mn),
+                                               int(f32_out), _stream_handle(stream)))
+    return out
+
+
+def group_norm_scale_bwd(o, dy, gamma, beta, eps=1e-5, lam=1.0, gate=None, stream=None):
+    """Backward of group_norm_scale: o [..., H, d] bf16, dy the same shape fp32.
+    Returns (y bf16, do bf16, dgamma, dbeta [H*d] fp32, dgate [H] fp32 or None)."""
+    import torch
+    H, d = o.shape[-2], o.shape[-1]
+    tokens = o.numel() // (H * d)
+    dv = o.device
+    _need("o", o, dv, torch.bfloat16)
+    _need("dy", dy, dv, torch.float32, tuple(o.shape))
+    _need("gamma", gamma, dv, torch.float32, (H * d,))
+    _need("beta", beta, dv, torch.float32, (H * d,))
+    _need("gate", gate, dv, torch.float32, (H,))
+    y = torch.empty_like(o)
+    do = torch.empty_like(o)
+    z = lambda *shape: torch.empty(shape, dtype=torch.float32, device=dv)
+    dgamma, dbeta = z(H * d), z(H * d)
+    dgate = z(H) if gate is not None else None
+    gn = MtaGn(gamma.data_ptr(), beta.data_ptr(), eps, 0, lam, gate.data_ptr() if gate is not None else None)
+    _check("mta_group_norm_scale_bwd", lib().mta_group_norm_scale_bwd(
+        _ptr(o), _ptr(dy), ctypes.byref(gn), tokens, H, d, _ptr(y), _ptr(do), _ptr(dgamma), _ptr(dbeta),
+        _ptr(dgate), _stream_handle(stream)))
+    return y, do, dgamma, dbeta, dgate
 
 
 def group_norm_scale(o, gamma, beta, eps=1e-5, lam=1.0, out=None, stream=None, gate=None):
