@@ -262,11 +262,28 @@ mta_status mta_group_norm_scale_bwd(const void *o, const float *dy, const mta_gn
  *                  NULL; n = 0 leaves it unused)
  *   dw           : [H/c_h][c_h][c_h] fp32, overwritten (may be NULL; ignored when
  *                  head_place == MTA_OFF)
- * Runs on the CUDA cores in fp32 arithmetic for every forward configuration
- * (attn_bwd_simt.cu; attn_bwd_post_simt.cu with the post-softmax convolution).
- * cfg->path must be 0 or 1.  dk, dv, dtheta and dw are summed with atomic additions, so their
- * last bits may differ between runs.  The workspace holds the error word only
- * (mta_attn_bwd_workspace_bytes).  No L x L map is stored. */
+ * Two implementations (cfg->path):
+ *   3: the contractions on the tensor cores (attn_bwd_tc.cu): bf16, d = 64 or
+ *      128, c_q = 6, c_k = 11, kq_place = MTA_PRE, no post-softmax convolution,
+ *      c_h = 2 with head mixing; query blocks of 118 rows, every head at once,
+ *      their maps in strips of the workspace (S = s Q K^T, dA'' = dO V^T, dQ,
+ *      dK, dV as batched tcgen05 GEMMs; the convolution, its adjoint and the
+ *      softmax on the CUDA cores).  MTA_ERR_UNSUPPORTED for other
+ *      configurations, MTA_ERR_WORKSPACE when the strips do not fit.
+ *   1: the CUDA cores in fp32 arithmetic, every forward configuration
+ *      (attn_bwd_simt.cu; attn_bwd_post_simt.cu with the post-softmax
+ *      convolution).
+ *   0: 3 where it applies and the workspace holds its strips, else 1.
+ *   2 returns MTA_ERR_UNSUPPORTED.
+ * Both agree with fp64 to a relative error of about 1e-5: path 3 feeds its
+ * computed MMA operands (dS, A'') as two bf16 halves.  dtheta and dw (both
+ * paths) and dk, dv (path 1) are summed with atomic additions, so their last
+ * bits may differ between runs.  The workspace (mta_attn_bwd_workspace_bytes)
+ * holds the error word and, where path 3 applies, its strips: for one query
+ * block of every head, a 128-row S strip and two (three with pre-softmax
+ * mixing) fp32 strips of 123 rows over the keys, and two bf16 strips of 256 rows
+ * (B*H*pitch*(128*4 + 2*123*4 + 2*256*2) bytes, pitch = L rounded up to 64).  No
+ * L x L map is stored. */
 size_t mta_attn_bwd_workspace_bytes(const mta_cfg *cfg);
 mta_status mta_attn_bwd(const void *q, const void *k, const void *v, const float *theta_kq,
                         const float *w_head, const void *dout, const mta_cfg *cfg, float *dq,

@@ -49,7 +49,9 @@ int main(void) {
   ws = mta_attn_workspace_bytes(&c);
   EXPECT(ws >= (size_t)6 * 4 * 16 * 2048 * 128 * 2);
   EXPECT(mta_layer_workspace_bytes(&c) > ws);
-  EXPECT(mta_attn_bwd_workspace_bytes(&c) == 256);
+  /* the backward: the status word and its tensor-core strips (one query block of
+   * every head, several 128-row strips spanning the keys) */
+  EXPECT(mta_attn_bwd_workspace_bytes(&c) > (size_t)256 + (size_t)4 * 16 * 128 * 2048 * 4);
 
   /* kernel choice on the host: the contraction kernel once its operands fit */
   EXPECT(mta_attn_kernel(&c) == -MTA_ERR_WORKSPACE);
@@ -90,9 +92,12 @@ int main(void) {
   EXPECT(mta_layer_fwd(fake(1), fake(2), th, w, &gn, fake(3), &bad, fake(6)) == MTA_ERR_UNSUPPORTED);
   EXPECT(mta_attn_bwd(fake(1), fake(2), fake(3), th, w, fake(10), &c, NULL, (float *)fake(12),
                       (float *)fake(13), NULL, NULL) == MTA_ERR_INVALID);
-  bad = c; bad.path = 3;
+  bad = c; bad.path = 2;  /* no direct tensor-core backward */
   EXPECT(mta_attn_bwd(fake(1), fake(2), fake(3), th, w, fake(10), &bad, (float *)fake(11),
                       (float *)fake(12), (float *)fake(13), NULL, NULL) == MTA_ERR_UNSUPPORTED);
+  bad = c; bad.path = 3;  /* the tensor-core backward: its strips do not fit the workspace */
+  EXPECT(mta_attn_bwd(fake(1), fake(2), fake(3), th, w, fake(10), &bad, (float *)fake(11),
+                      (float *)fake(12), (float *)fake(13), NULL, NULL) == MTA_ERR_WORKSPACE);
   EXPECT(mta_gemm_bf16_nt(fake(1), fake(2), fake(3), 128, 256, 60, NULL) == MTA_ERR_INVALID);
 
   /* an output that overlaps an input is refused before anything is enqueued */

@@ -220,13 +220,28 @@ def test_backward_argument_errors(L):
     assert f(cfg, dout=None) == 1
     assert f(cfg, theta=None) == 1                      # kq_place PRE needs the kernels
     assert f(cfg, dq=ctypes.c_void_p(fake(11).value + 2)) == 1   # fp32 gradients, 4-byte aligned
-    forced = good_cfg(path=mta.PATH_TC)                 # only the CUDA-core backward exists
+    forced = good_cfg(path=mta.PATH_TC)                 # no direct tensor-core backward
     forced.workspace, forced.workspace_bytes = 0x100000, 1 << 20
     assert f(forced) == 2
+    kq = good_cfg(path=mta.PATH_KQ)                     # the tensor-core backward, strips too small
+    kq.workspace, kq.workspace_bytes = 0x100000, 1 << 20
+    assert f(kq) == 3
+    other = good_cfg(path=mta.PATH_KQ, c_q=3)           # a shape it does not serve
+    other.workspace, other.workspace_bytes = 0x100000, 1 << 20
+    assert f(other) == 2
     small = good_cfg()
     small.workspace, small.workspace_bytes = 0x100000, 16
     assert f(small) == 3
-    assert L.mta_attn_bwd_workspace_bytes(ctypes.byref(good_cfg())) == 256
+    # the status word, then the tensor-core backward's strips for one query block of
+    # every head (B H = 8, pitch 64): S [128 rows] and A, dA/dC [123 rows] fp32, the
+    # dS and A'' halves [256 rows] bf16
+    Z, P, rc = 2 * 4, 64, 128 - 5
+    strips = up(Z * 128 * P * 4) + 2 * up(Z * rc * P * 4) + 2 * up(Z * 256 * P * 2)
+    assert L.mta_attn_bwd_workspace_bytes(ctypes.byref(good_cfg())) == 256 + strips
+    # pre-softmax mixing keeps the unmixed C as well
+    assert L.mta_attn_bwd_workspace_bytes(ctypes.byref(good_cfg(head_place=mta.PRE))) == \
+        256 + strips + up(Z * rc * P * 4)
+    assert L.mta_attn_bwd_workspace_bytes(ctypes.byref(good_cfg(c_q=3))) == 256   # CUDA cores only
     assert L.mta_attn_bwd_workspace_bytes(ctypes.byref(good_cfg(c_k=4))) == 0
 
 

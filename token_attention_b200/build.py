@@ -23,7 +23,7 @@ LIB = os.path.join(HERE, "libmta.so")
 
 SOURCES = ["mta_api.cu", "attn_simt.cu", "attn_tc.cu", "attn_kq.cu", "attn_kq_pair.cu", "kq_prep.cu", "gemm_tc.cu",
            "group_norm.cu", "layer_static.cu", "attn_bwd_simt.cu", "attn_bwd_post_simt.cu",
-           "selftest.cu", "layer_bwd.cu"]
+           "selftest.cu", "layer_bwd.cu", "gemm_batched.cu", "attn_bwd_tc.cu"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 FLAGS = ["-O3", "-lineinfo", "-std=c++17", "-Xcompiler", "-fPIC", "--expt-relaxed-constexpr",
          "-I", INCLUDE, "-I", CSRC]

@@ -1,0 +1,540 @@
+// attn_bwd_tc.cu -- the MTA attention backward with its contractions on the
+// tensor cores ("Multi-Token Attention | Summary" (greeksharifa), sections 2,
+// 3.1 and 3.2, each forward step taken in reverse; the pages train with this
+// forward, section 4 and appendix F).
+//
+// The forward per head group: logits S = s Q K^T, Mask_0, the key-query
+// convolution C = Conv2d_theta(Mask_0 S), optional pre-softmax mixing
+// C'_h = sum_s w[h][s] C_s, Mask_-inf and the softmax A, optional post-softmax
+// mixing A''_h = sum_s w[h][s] A_s, O_h = A''_h V_h.  Its adjoints:
+//   dA''_h = dO_h V_h^T                      (tensor cores)
+//   dV_h   = A''_h^T dO_h                    (tensor cores)
+//   dA_s   = sum_h w[h][s] dA''_h, dw[h][s] = sum dA''_h . A_s   (post mixing)
+//   dC_s   = A_s (dA_s - D_s), D_s = rowsum(dA_s . A_s)          (softmax)
+//   dC_s   = sum_h w[h][s] dC'_h, dw[h][s] = sum dC'_h . C_s     (pre mixing)
+//   dS[i][j] = [j <= i] sum_{a,t} theta[a][t] dC[i+a][j+t-c]     (the convolution's adjoint)
+//   dtheta[a][t] = sum dC[i][j] Mask_0 S[i-a][j-(t-c)]
+//   dQ = s dS K, dK = s dS^T Q               (tensor cores)
+//
+// Query blocks of NO = 128 - 2 (c_q - 1) rows are processed one after another,
+// all heads at once.  For block rows r0 .. r0+NO-1 the maps are held in strips
+// of the workspace that span every key up to the block's last row: S for rows
+// r0-(c_q-1) .. r0+NO+c_q-2 (128 rows: the convolution reads c_q-1 earlier query
+// rows, its adjoint c_q-1 later ones), A, dA'' then dC for rows r0 .. r0+NO+c_q-2,
+// dS and A'' for the block's own rows.  A strip holds whole rows, so the softmax
+// statistics and D come from the strip itself (no statistics pass).  The strips
+// are O(B H 128 L): never an L x L map.  Per block:
+//   1. S strip      = s Q K^T                      batched GEMM (fp32 out)
+//   2. C, softmax   -> A strip                     bwd_scores_kernel (CUDA cores)
+//   3. dA'' strip   = dO V^T                       batched GEMM
+//   4. dC, D, dw, A''                              bwd_softmax_grad_kernel
+//   5. dS, dtheta                                  bwd_adjoint_kernel
+//   6. dQ rows (=), dK, dV (+=)                    batched GEMMs
+// dS and A'' enter the GEMMs of step 6 as two bf16 halves, hi = bf16(x) and
+// lo = bf16(x - hi), summed by two GEMMs into the same fp32 output: the operands
+// then carry about 16 significant bits and the gradients stay within fp32
+// tolerance of the CUDA-core backward.  The other GEMM operands (q, k, v, dO) are
+// the bf16 inputs themselves.
+#include <cuda_bf16.h>
+#include <stdint.h>
+
+#include <algorithm>
+
+#include "internal.h"
+#include "ptx.cuh"
+
+namespace mta {
+namespace {
+
+constexpr int kRowsT = 128;  // rows of the S strip (and of the halves of the dS / A'' strips)
+constexpr int kKeyTile = 128;
+constexpr int kThreadsB = 256;
+constexpr int kRowsPerCta = 4;  // rows of a CTA in the CUDA-core kernels: 4 x 64 threads
+
+struct Geo {
+  int halo, c, no, rc, pitch;  // c_q - 1, c_k / 2, own rows, C rows, strip pitch (elements)
+};
+
+struct StripArgs {
+  int B, H, L, ch, hp;        // hp: 0 off, 1 pre, 2 post
+  int r0, W, Wp;              // block's first row, keys 0 .. W-1 (Wp = W rounded up to 64)
+  Geo g;
+  const float *theta;         // [H][c_q][c_k]
+  const float *w;             // [H/c_h][c_h][c_h]
+  float *S;                   // [B][H][128][pitch]
+  float *Cpre;                // [B][H][rc][pitch] pre-mixing C (pre mixing only)
+  float *A;                   // [B][H][rc][pitch]
+  float *D;                   // [B][H][rc][pitch]: dA'' from the GEMM, then dC
+  __nv_bfloat16 *dS;          // [B][H][256][pitch]: hi rows 0..127, lo rows 128..255
+  __nv_bfloat16 *Ap;          // [B][H][256][pitch]: A'' hi / lo
+  float *dtheta, *dw;
+};
+
+__device__ __forceinline__ float blocksum64(float v, float *red, int row, int sub) {
+  // sum over the 64 threads (two warps) of one row
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  if ((sub & 31) == 0) red[2 * row + (sub >> 5)] = v;
+  __syncthreads();
+  const float s = red[2 * row] + red[2 * row + 1];
+  __syncthreads();
+  return s;
+}
+
+__device__ __forceinline__ void split_bf16(float x, __nv_bfloat16 &hi, __nv_bfloat16 &lo) {
+  hi = __float2bfloat16_rn(x);
+  lo = __float2bfloat16_rn(x - __bfloat162float(hi));
+}
+
+// Step 2: C = Conv2d_theta(Mask_0 S) for the block's C rows (and pre mixing),
+// Mask_-inf, softmax over the row -> A strip.  CTA: one head group, 4 rows; thread
+// (row, sub): keys sub, sub + 64 of every 128-key tile.
+template <int CQ, int CK, int CH>
+__global__ void __launch_bounds__(kThreadsB) bwd_scores_kernel(StripArgs p) {
+  constexpr int HALO = CQ - 1, C = CK / 2, TR = kRowsPerCta + HALO, TC = kKeyTile + 2 * C;
+  __shared__ float tile[CH][TR][TC];
+  __shared__ float th[CH][CQ * CK], wm[CH * CH];
+  __shared__ float red[2 * kRowsPerCta];
+  const int G = p.H / CH, bg = blockIdx.y, b = bg / G, g = bg % G;
+  const int u0 = blockIdx.x * kRowsPerCta, row = threadIdx.x >> 6, sub = threadIdx.x & 63;
+  const int u = u0 + row, i = p.r0 + u;
+  const bool valid = u < p.g.rc && i < p.L;
+  const int P = p.g.pitch;
+  for (int x = threadIdx.x; x < CH * CQ * CK; x += kThreadsB)
+    th[x / (CQ * CK)][x % (CQ * CK)] = p.theta[(g * CH + x / (CQ * CK)) * CQ * CK + x % (CQ * CK)];
+  for (int x = threadIdx.x; x < CH * CH; x += kThreadsB) wm[x] = p.w ? p.w[g * CH * CH + x] : (x % (CH + 1) == 0);
+  auto strip = [&](float *base, int hl, int rows) {
+    return base + ((static_cast<long long>(b) * p.H + g * CH + hl) * rows) * P;
+  };
+  float m[CH], l[CH];
+#pragma unroll
+  for (int h = 0; h < CH; ++h) { m[h] = -INFINITY; l[h] = 0.f; }
+  const int jend = p.W;
+  for (int j0 = 0; j0 < jend; j0 += kKeyTile) {
+    __syncthreads();
+    // stage Mask_0 S: strip rows u0 .. u0+TR-1 (queries r0 - HALO + su), keys j0-C .. j0+128+C-1
+    for (int x = threadIdx.x; x < CH * TR * TC; x += kThreadsB) {
+      const int hl = x / (TR * TC), r = (x / TC) % TR, cc = x % TC;
+      const int su = u0 + r, iq = p.r0 - HALO + su, jk = j0 - C + cc;
+      float v = 0.f;
+      if (su < kRowsT && iq >= 0 && iq < p.L && jk >= 0 && jk <= iq) v = strip(p.S, hl, kRowsT)[su * P + jk];
+      tile[hl][r][cc] = v;
+    }
+    __syncthreads();
+    if (!valid) continue;
+#pragma unroll
+    for (int kk = 0; kk < 2; ++kk) {
+      const int jl = sub + 64 * kk, j = j0 + jl;
+      if (j >= p.Wp) continue;
+      float cv[CH];
+#pragma unroll
+      for (int h = 0; h < CH; ++h) {
+        float acc = 0.f;
+#pragma unroll
+        for (int a = 0; a < CQ; ++a)
+#pragma unroll
+          for (int t = 0; t < CK; ++t) acc = fmaf(th[h][a * CK + t], tile[h][row + HALO - a][jl + 2 * C - t], acc);
+        cv[h] = acc;
+      }
+      if (p.hp == 1 && p.Cpre) {
+#pragma unroll
+        for (int h = 0; h < CH; ++h) strip(p.Cpre, h, p.g.rc)[u * P + j] = j <= i ? cv[h] : 0.f;
+      }
+#pragma unroll
+      for (int h = 0; h < CH; ++h) {
+        float x = cv[h];
+        if (p.hp == 1) {
+          x = 0.f;
+#pragma unroll
+          for (int s = 0; s < CH; ++s) x = fmaf(wm[h * CH + s], cv[s], x);
+        }
+        // Mask_-inf: keys after the query
+        x = j <= i ? x : -INFINITY;
+        strip(p.A, h, p.g.rc)[u * P + j] = x;  // logits for now
+        if (x > m[h]) {
+          l[h] = l[h] * __expf(m[h] - x) + 1.f;
+          m[h] = x;
+        } else if (x != -INFINITY) {
+          l[h] += __expf(x - m[h]);
+        }
+      }
+    }
+  }
+  // row statistics over the 64 threads of the row
+  float mr[CH], lr[CH];
+#pragma unroll
+  for (int h = 0; h < CH; ++h) {
+    float mx = m[h];
+    for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+    __syncthreads();
+    if ((sub & 31) == 0) red[2 * row + (sub >> 5)] = mx;
+    __syncthreads();
+    mr[h] = fmaxf(red[2 * row], red[2 * row + 1]);
+    const float part = m[h] == -INFINITY ? 0.f : l[h] * __expf(m[h] - mr[h]);
+    lr[h] = blocksum64(part, red, row, sub);
+  }
+  if (!valid) return;
+  for (int j = sub; j < p.Wp; j += 64) {
+#pragma unroll
+    for (int h = 0; h < CH; ++h) {
+      float *a = strip(p.A, h, p.g.rc) + u * P + j;
+      const float x = *a;
+      *a = j <= i ? __expf(x - mr[h]) / lr[h] : 0.f;
+    }
+  }
+}
+
+// Step 4: dA (post mixing: mixed back to the sources), D, dC = A (dA - D) (pre
+// mixing: then mixed back), dw, and A'' (hi / lo) of the block's own rows.  Rows
+// u = 0 .. 127: rows past the C rows only clear their A'' halves.
+template <int CH>
+__global__ void __launch_bounds__(kThreadsB) bwd_softmax_grad_kernel(StripArgs p) {
+  __shared__ float wm[CH * CH];
+  __shared__ float red[2 * kRowsPerCta];
+  __shared__ float dwr[CH * CH];
+  const int G = p.H / CH, bg = blockIdx.y, b = bg / G, g = bg % G;
+  const int u = blockIdx.x * kRowsPerCta + (threadIdx.x >> 6), row = threadIdx.x >> 6, sub = threadIdx.x & 63;
+  const int i = p.r0 + u;
+  const bool valid = u < p.g.rc && i < p.L;
+  const bool own = u < p.g.no && i < p.L;
+  const int P = p.g.pitch;
+  for (int x = threadIdx.x; x < CH * CH; x += kThreadsB) {
+    wm[x] = p.w ? p.w[g * CH * CH + x] : (x % (CH + 1) == 0);
+    dwr[x] = 0.f;
+  }
+  __syncthreads();
+  auto strip = [&](auto *base, int hl, int rows) {
+    return base + ((static_cast<long long>(b) * p.H + g * CH + hl) * rows) * P;
+  };
+  // pass 1: D_s (post / none: dA_s = sum_h w[h][s] dA''_h; pre: dA'_h = dA''_h)
+  float Dp[CH], dwp[CH * CH];
+#pragma unroll
+  for (int h = 0; h < CH; ++h) Dp[h] = 0.f;
+#pragma unroll
+  for (int x = 0; x < CH * CH; ++x) dwp[x] = 0.f;
+  if (valid) {
+    for (int j = sub; j <= i && j < p.W; j += 64) {
+      float a[CH], da[CH];
+#pragma unroll
+      for (int h = 0; h < CH; ++h) {
+        a[h] = strip(p.A, h, p.g.rc)[u * P + j];
+        da[h] = strip(p.D, h, p.g.rc)[u * P + j];
+      }
+#pragma unroll
+      for (int s = 0; s < CH; ++s) {
+        float d = da[s];
+        if (p.hp == 2) {
+          d = 0.f;
+#pragma unroll
+          for (int h = 0; h < CH; ++h) d = fmaf(wm[h * CH + s], da[h], d);
+        }
+        Dp[s] = fmaf(d, a[s], Dp[s]);
+      }
+      if (p.hp == 2 && own) {
+#pragma unroll
+        for (int h = 0; h < CH; ++h)
+#pragma unroll
+          for (int s = 0; s < CH; ++s) dwp[h * CH + s] = fmaf(da[h], a[s], dwp[h * CH + s]);
+      }
+    }
+  }
+  float Dr[CH];
+#pragma unroll
+  for (int h = 0; h < CH; ++h) Dr[h] = blocksum64(Dp[h], red, row, sub);
+  // pass 2: dC (into the dA'' strip), pre-mixing dw, A'' halves
+  for (int j = sub; j < p.Wp; j += 64) {
+    const bool in = valid && j <= i;
+    float a[CH], da[CH], dc[CH];
+#pragma unroll
+    for (int h = 0; h < CH; ++h) {
+      a[h] = in ? strip(p.A, h, p.g.rc)[u * P + j] : 0.f;
+      da[h] = in ? strip(p.D, h, p.g.rc)[u * P + j] : 0.f;
+    }
+    if (p.hp == 1) {
+      float dcp[CH];  // dC'_h = A_h (dA''_h - D_h), then mixed back to the sources
+#pragma unroll
+      for (int h = 0; h < CH; ++h) dcp[h] = a[h] * (da[h] - Dr[h]);
+#pragma unroll
+      for (int s = 0; s < CH; ++s) {
+        float x = 0.f;
+#pragma unroll
+        for (int h = 0; h < CH; ++h) x = fmaf(wm[h * CH + s], dcp[h], x);
+        dc[s] = x;
+      }
+      if (in && own) {
+        float cs[CH];
+#pragma unroll
+        for (int s = 0; s < CH; ++s) cs[s] = strip(p.Cpre, s, p.g.rc)[u * P + j];
+#pragma unroll
+        for (int h = 0; h < CH; ++h)
+#pragma unroll
+          for (int s = 0; s < CH; ++s) dwp[h * CH + s] = fmaf(dcp[h], cs[s], dwp[h * CH + s]);
+      }
+    } else {
+#pragma unroll
+      for (int s = 0; s < CH; ++s) {
+        float d = da[s];
+        if (p.hp == 2) {
+          d = 0.f;
+#pragma unroll
+          for (int h = 0; h < CH; ++h) d = fmaf(wm[h * CH + s], da[h], d);
+        }
+        dc[s] = a[s] * (d - Dr[s]);
+      }
+    }
+    if (u < p.g.rc) {
+#pragma unroll
+      for (int s = 0; s < CH; ++s) strip(p.D, s, p.g.rc)[u * P + j] = in ? dc[s] : 0.f;
+    }
+    // A''_h = sum_s w[h][s] A_s (post mixing), else A_h; own rows only
+#pragma unroll
+    for (int h = 0; h < CH; ++h) {
+      float x = a[h];
+      if (p.hp == 2) {
+        x = 0.f;
+#pragma unroll
+        for (int s = 0; s < CH; ++s) x = fmaf(wm[h * CH + s], a[s], x);
+      }
+      __nv_bfloat16 hi, lo;
+      split_bf16(own && in ? x : 0.f, hi, lo);
+      __nv_bfloat16 *ap = strip(p.Ap, h, 2 * kRowsT);
+      ap[u * P + j] = hi;
+      ap[(kRowsT + u) * P + j] = lo;
+    }
+  }
+  if (p.hp != 0 && p.dw) {
+#pragma unroll
+    for (int x = 0; x < CH * CH; ++x) {
+      float v = dwp[x];
+      for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+      if ((threadIdx.x & 31) == 0) atomicAdd(&dwr[x], v);
+    }
+    __syncthreads();
+    if (threadIdx.x < CH * CH) atomicAdd(p.dw + g * CH * CH + threadIdx.x, dwr[threadIdx.x]);
+  }
+}
+
+// Step 5: dS = [j <= i] sum theta[a][t] dC[i+a][j+t-c] (hi / lo halves) for the
+// block's own rows, zeros elsewhere, and dtheta over the own rows.  CTA: one
+// head, 4 rows u = 0 .. 127.
+template <int CQ, int CK>
+__global__ void __launch_bounds__(kThreadsB) bwd_adjoint_kernel(StripArgs p) {
+  constexpr int HALO = CQ - 1, C = CK / 2, TR = kRowsPerCta + HALO, TC = kKeyTile + 2 * C, NT = CQ * CK;
+  __shared__ float dct[TR][TC], st[TR][TC];
+  __shared__ float th[NT];
+  const int z = blockIdx.y, h = z % p.H;
+  const int u0 = blockIdx.x * kRowsPerCta, row = threadIdx.x >> 6, sub = threadIdx.x & 63;
+  const int u = u0 + row, i = p.r0 + u;
+  const bool own = u < p.g.no && i < p.L;
+  const int P = p.g.pitch;
+  const float *Dz = p.D + static_cast<long long>(z) * p.g.rc * P;
+  const float *Sz = p.S + static_cast<long long>(z) * kRowsT * P;
+  __nv_bfloat16 *dSz = p.dS + static_cast<long long>(z) * 2 * kRowsT * P;
+  for (int x = threadIdx.x; x < NT; x += kThreadsB) th[x] = p.theta[h * NT + x];
+  float dth[NT];
+#pragma unroll
+  for (int x = 0; x < NT; ++x) dth[x] = 0.f;
+  for (int j0 = 0; j0 < p.Wp; j0 += kKeyTile) {
+    __syncthreads();
+    for (int x = threadIdx.x; x < TR * TC; x += kThreadsB) {
+      const int r = x / TC, cc = x % TC, jk = j0 - C + cc;
+      // dC rows u0 .. u0+TR-1 (queries r0 + u'), zero past the C rows, the sequence and the diagonal
+      const int uc = u0 + r, ic = p.r0 + uc;
+      dct[r][cc] = (uc < p.g.rc && ic < p.L && jk >= 0 && jk <= ic) ? Dz[uc * P + jk] : 0.f;
+      // Mask_0 S rows u0 .. u0+TR-1 of the S strip (queries r0 - HALO + su)
+      const int su = u0 + r, is = p.r0 - HALO + su;
+      st[r][cc] = (su < kRowsT && is >= 0 && is < p.L && jk >= 0 && jk <= is) ? Sz[su * P + jk] : 0.f;
+    }
+    __syncthreads();
+#pragma unroll
+    for (int kk = 0; kk < 2; ++kk) {
+      const int jl = sub + 64 * kk, j = j0 + jl;
+      if (j >= p.Wp) continue;
+      float ds = 0.f;
+      if (own && j <= i) {
+#pragma unroll
+        for (int a = 0; a < CQ; ++a)
+#pragma unroll
+          for (int t = 0; t < CK; ++t) ds = fmaf(th[a * CK + t], dct[row + a][jl + t], ds);
+        // dtheta[a][t] += dC[i][j] Mask_0 S[i-a][j-(t-c)]
+        const float g = dct[row][jl + C];
+#pragma unroll
+        for (int a = 0; a < CQ; ++a)
+#pragma unroll
+          for (int t = 0; t < CK; ++t) dth[a * CK + t] = fmaf(g, st[row + HALO - a][jl + 2 * C - t], dth[a * CK + t]);
+      }
+      __nv_bfloat16 hi, lo;
+      split_bf16(ds, hi, lo);
+      dSz[u * P + j] = hi;
+      dSz[(kRowsT + u) * P + j] = lo;
+    }
+  }
+  if (p.dtheta) {
+#pragma unroll
+    for (int x = 0; x < NT; ++x) {
+      float v = dth[x];
+      for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+      if ((threadIdx.x & 31) == 0 && v != 0.f) atomicAdd(p.dtheta + h * NT + x, v);
+    }
+  }
+}
+
+Geo geometry(const BwdArgs &a) {
+  Geo g;
+  g.halo = a.cq - 1;
+  g.c = a.ck / 2;
+  g.no = kRowsT - 2 * g.halo;
+  g.rc = g.no + g.halo;
+  g.pitch = (a.L + 63) / 64 * 64;
+  return g;
+}
+
+size_t up256(size_t x) { return (x + 255) / 256 * 256; }
+
+// [B][L][H][d] bf16 with token stride rs: dims (d, H, L, B), the row index at position 2
+BgTensor qkv_tensor(const void *base, const BwdArgs &a, long long rs) {
+  BgTensor t;
+  t.base = base;
+  t.dims[0] = a.d; t.dims[1] = a.H; t.dims[2] = a.L; t.dims[3] = a.B;
+  t.strides[0] = static_cast<unsigned long long>(a.d) * 2;
+  t.strides[1] = static_cast<unsigned long long>(rs) * 2;
+  t.strides[2] = static_cast<unsigned long long>(rs) * a.L * 2;
+  t.pos_row = 2;
+  return t;
+}
+// a bf16 strip [B][H][rows][pitch]: dims (pitch, rows, H, B), the row index at position 1
+BgTensor strip_tensor(const void *base, const BwdArgs &a, int rows, int pitch) {
+  BgTensor t;
+  t.base = base;
+  t.dims[0] = pitch; t.dims[1] = rows; t.dims[2] = a.H; t.dims[3] = a.B;
+  t.strides[0] = static_cast<unsigned long long>(pitch) * 2;
+  t.strides[1] = static_cast<unsigned long long>(pitch) * rows * 2;
+  t.strides[2] = static_cast<unsigned long long>(pitch) * rows * a.H * 2;
+  t.pos_row = 1;
+  return t;
+}
+
+}  // namespace
+
+bool attn_bwd_tc_supported(const BwdArgs &a) {
+  return a.dtype == 1 && (a.d == 64 || a.d == 128) && a.cq == 6 && a.ck == 11 && a.kq == 1 && !a.kqp &&
+         (a.hp == 0 || a.ch == 2) && a.rs % 8 == 0 &&
+         (reinterpret_cast<uintptr_t>(a.q) | reinterpret_cast<uintptr_t>(a.k) | reinterpret_cast<uintptr_t>(a.v) |
+          reinterpret_cast<uintptr_t>(a.dout)) % 16 == 0 &&
+         (reinterpret_cast<uintptr_t>(a.dq) | reinterpret_cast<uintptr_t>(a.dk) | reinterpret_cast<uintptr_t>(a.dv)) %
+                 16 == 0;
+}
+
+size_t attn_bwd_tc_workspace_bytes(int B, int H, int L, int cq, int hp) {
+  const size_t Z = static_cast<size_t>(B) * H, P = (static_cast<size_t>(L) + 63) / 64 * 64;
+  const size_t rc = kRowsT - (cq - 1);
+  return up256(Z * kRowsT * P * 4) + 2 * up256(Z * rc * P * 4) + (hp == 1 ? up256(Z * rc * P * 4) : 0) +
+         2 * up256(Z * 2 * kRowsT * P * 2);
+}
+
+cudaError_t launch_attn_bwd_tc(const BwdArgs &a, void *ws) {
+  const Geo g = geometry(a);
+  const size_t Z = static_cast<size_t>(a.B) * a.H, P = g.pitch;
+  char *w = static_cast<char *>(ws);
+  float *S = reinterpret_cast<float *>(w);
+  w += up256(Z * kRowsT * P * 4);
+  float *A = reinterpret_cast<float *>(w);
+  w += up256(Z * g.rc * P * 4);
+  float *D = reinterpret_cast<float *>(w);
+  w += up256(Z * g.rc * P * 4);
+  float *Cpre = nullptr;
+  if (a.hp == 1) {
+    Cpre = reinterpret_cast<float *>(w);
+    w += up256(Z * g.rc * P * 4);
+  }
+  __nv_bfloat16 *dS = reinterpret_cast<__nv_bfloat16 *>(w);
+  w += up256(Z * 2 * kRowsT * P * 2);
+  __nv_bfloat16 *Ap = reinterpret_cast<__nv_bfloat16 *>(w);
+
+  cudaStream_t st = a.stream;
+  const size_t n = static_cast<size_t>(a.B) * a.L * a.H * a.d;
+  cudaError_t e;
+  if ((e = cudaMemsetAsync(a.dk, 0, n * 4, st)) != cudaSuccess) return e;
+  if ((e = cudaMemsetAsync(a.dv, 0, n * 4, st)) != cudaSuccess) return e;
+  if (a.dtheta && (e = cudaMemsetAsync(a.dtheta, 0, static_cast<size_t>(a.H) * a.cq * a.ck * 4, st)) != cudaSuccess)
+    return e;
+  if (a.hp && a.dw && (e = cudaMemsetAsync(a.dw, 0, static_cast<size_t>(a.H) * a.ch * 4, st)) != cudaSuccess)
+    return e;
+
+  const BgTensor tq = qkv_tensor(a.q, a, a.rs), tk = qkv_tensor(a.k, a, a.rs), tv = qkv_tensor(a.v, a, a.rs);
+  const BgTensor tdo = qkv_tensor(a.dout, a, static_cast<long long>(a.H) * a.d);
+  const BgTensor tdS = strip_tensor(dS, a, 2 * kRowsT, g.pitch), tAp = strip_tensor(Ap, a, 2 * kRowsT, g.pitch);
+  const long long HD = static_cast<long long>(a.H) * a.d, LHD = HD * a.L;
+  const int ch = a.hp ? a.ch : 1, G = a.H / ch;
+  unsigned *err = a.err;
+
+  StripArgs sp;
+  sp.B = a.B; sp.H = a.H; sp.L = a.L; sp.ch = ch; sp.hp = a.hp;
+  sp.g = g;
+  sp.theta = a.theta; sp.w = a.hp ? a.w : nullptr;
+  sp.S = S; sp.Cpre = Cpre; sp.A = A; sp.D = D; sp.dS = dS; sp.Ap = Ap;
+  sp.dtheta = a.dtheta; sp.dw = a.hp ? a.dw : nullptr;
+
+  auto K_major = [](int pos_row, int off_mn, int off_k) { return BgOperand{0, pos_row, off_mn, off_k}; };
+  auto MN_major = [](int pos_row, int off_mn, int off_k) { return BgOperand{1, pos_row, off_mn, off_k}; };
+  for (int r0 = 0; r0 < a.L; r0 += g.no) {
+    const int W = std::min(a.L, r0 + g.rc), Wp = (W + 63) / 64 * 64;
+    sp.r0 = r0; sp.W = W; sp.Wp = Wp;
+    // 1. S strip = s Q K^T: rows r0 - halo .. r0 - halo + 127, keys 0 .. W-1
+    BgArgs ga = {};
+    ga.Z = static_cast<int>(Z); ga.H = a.H; ga.err = err;
+    ga.M = kRowsT; ga.N = W; ga.K = a.d; ga.alpha = a.scale; ga.accumulate = 0;
+    ga.C = S; ga.sm = g.pitch; ga.sh = static_cast<long long>(kRowsT) * g.pitch; ga.sb = ga.sh * a.H;
+    ga.a = K_major(2, r0 - g.halo, 0); ga.b = K_major(2, 0, 0);
+    if ((e = launch_gemm_batched(tq, tk, ga, st)) != cudaSuccess) return e;
+    // 2. convolution, mixing, softmax -> A
+    const dim3 grid2((g.rc + kRowsPerCta - 1) / kRowsPerCta, a.B * G);
+    if (ch == 2)
+      bwd_scores_kernel<6, 11, 2><<<grid2, kThreadsB, 0, st>>>(sp);
+    else
+      bwd_scores_kernel<6, 11, 1><<<grid2, kThreadsB, 0, st>>>(sp);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    // 3. dA'' strip = dO V^T: rows r0 .. r0 + rc - 1
+    ga.M = g.rc; ga.alpha = 1.f;
+    ga.C = D; ga.sh = static_cast<long long>(g.rc) * g.pitch; ga.sb = ga.sh * a.H;
+    ga.a = K_major(2, r0, 0); ga.b = K_major(2, 0, 0);
+    if ((e = launch_gemm_batched(tdo, tv, ga, st)) != cudaSuccess) return e;
+    // 4. dC, D, dw, A''
+    const dim3 grid4(kRowsT / kRowsPerCta, a.B * G);
+    if (ch == 2)
+      bwd_softmax_grad_kernel<2><<<grid4, kThreadsB, 0, st>>>(sp);
+    else
+      bwd_softmax_grad_kernel<1><<<grid4, kThreadsB, 0, st>>>(sp);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    // 5. dS (hi / lo), dtheta
+    bwd_adjoint_kernel<6, 11><<<dim3(kRowsT / kRowsPerCta, static_cast<unsigned>(Z)), kThreadsB, 0, st>>>(sp);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    // 6. dQ rows r0 .. r0 + no - 1 = s dS K (hi, then lo added)
+    const int own = std::min(g.no, a.L - r0);
+    BgArgs gq = {};
+    gq.Z = static_cast<int>(Z); gq.H = a.H; gq.err = err;
+    gq.M = own; gq.N = a.d; gq.K = W; gq.alpha = a.scale;
+    gq.C = a.dq + static_cast<long long>(r0) * HD; gq.sm = HD; gq.sh = a.d; gq.sb = LHD;
+    gq.b = MN_major(2, 0, 0);
+    for (int half = 0; half < 2; ++half) {
+      gq.a = K_major(1, half * kRowsT, 0);
+      gq.accumulate = half;
+      if ((e = launch_gemm_batched(tdS, tk, gq, st)) != cudaSuccess) return e;
+    }
+    //    dK += s dS^T Q and dV += A''^T dO over the block's rows (keys 0 .. W-1)
+    BgArgs gk = {};
+    gk.Z = static_cast<int>(Z); gk.H = a.H; gk.err = err;
+    gk.M = W; gk.N = a.d; gk.K = kRowsT; gk.accumulate = 1;
+    gk.sm = HD; gk.sh = a.d; gk.sb = LHD;
+    gk.b = MN_major(2, 0, r0);
+    for (int half = 0; half < 2; ++half) {
+      gk.a = MN_major(1, 0, half * kRowsT);
+      gk.alpha = a.scale; gk.C = a.dk;
+      if ((e = launch_gemm_batched(tdS, tq, gk, st)) != cudaSuccess) return e;
+      gk.alpha = 1.f; gk.C = a.dv;
+      if ((e = launch_gemm_batched(tAp, tdo, gk, st)) != cudaSuccess) return e;
+    }
+  }
+  return cudaSuccess;
+}
+
+}  // namespace mta

@@ -67,8 +67,15 @@ struct BwdArgs {
   int kqp;                // 1: the convolution also acts after the softmax
   float scale;
   cudaStream_t stream;
+  unsigned *err;          // status word (bounded waits of the tensor-core path)
 };
 int attn_bwd_simt_pick_rows(const BwdArgs &a);  // 0 if nothing fits
+// The backward with its contractions on the tensor cores (attn_bwd_tc.cu): the
+// configurations it serves, its workspace (strips of every head for one query
+// block), and the launch.
+bool attn_bwd_tc_supported(const BwdArgs &a);
+size_t attn_bwd_tc_workspace_bytes(int B, int H, int L, int cq, int hp);
+cudaError_t launch_attn_bwd_tc(const BwdArgs &a, void *ws);
 cudaError_t launch_attn_bwd_simt(const BwdArgs &a);
 // With the post-softmax convolution (kqp == 1).
 int attn_bwd_post_pick_rows(const BwdArgs &a);
@@ -119,6 +126,34 @@ size_t attn_kq_pair_scratch_bytes(int B, int H, int L, int d, int hp);
 cudaError_t launch_attn_kq_pair(const AttnArgs &a, const GnArgs *gn, const KqPrepArgs &pa, void *scratch);
 
 // tcgen05 GEMM: C[M][N] = A[M][K] * B[N][K]^T (bf16 -> fp32 -> bf16).
+// Batched GEMM of the attention backward (gemm_batched.cu).  An operand tensor is
+// a bf16 array seen through a four-dimensional TMA map: dims[0] contiguous, then
+// three more with byte strides; one of positions 1 and 2 holds the row index and
+// the other the head, position 3 the batch.
+struct BgTensor {
+  const void *base;
+  unsigned long long dims[4];
+  unsigned long long strides[3];  // bytes, of dims 1..3
+  int pos_row;                    // 1 or 2
+};
+struct BgOperand {
+  int mn;      // 1: MN-major (contiguous index = M or N, row index = K); 0: K-major
+  int pos_row; // as the tensor's
+  int off_mn;  // added to the M (or N) index
+  int off_k;   // added to the K index
+};
+struct BgArgs {
+  int Z, H;         // batches z = b * H + h
+  int M, N, K;
+  float alpha;
+  int accumulate;   // C += alpha A B^T instead of C = alpha A B^T
+  float *C;         // element (b, h, m, n) at C + b*sb + h*sh + m*sm + n
+  long long sb, sh, sm;
+  BgOperand a, b;
+  unsigned *err;
+};
+cudaError_t launch_gemm_batched(const BgTensor &A, const BgTensor &B, const BgArgs &args, cudaStream_t stream);
+
 // C[M][N] = A B^T with A [M][K] (a_mn: stored [K][M]) and B [N][K] (b_mn: stored
 // [K][N]), bf16 in, fp32 accumulate, bf16 or (f32_out) fp32 out.
 cudaError_t launch_gemm(const void *A, const void *B, void *C, int M, int N, int K, bool a_mn, bool b_mn,

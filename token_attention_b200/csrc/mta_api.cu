@@ -7,6 +7,8 @@
 #include <math.h>
 #include <stdint.h>
 
+#include <algorithm>
+
 #include "internal.h"
 #include "mta.h"
 
@@ -202,11 +204,38 @@ BwdArgs make_bwd_args(const void *q, const void *k, const void *v, const float *
   a.kq = cfg->kq_place; a.hp = cfg->head_place; a.dtype = cfg->dtype;
   a.scale = cfg->scale > 0.f ? cfg->scale : 1.0f / sqrtf(static_cast<float>(cfg->d));
   a.stream = static_cast<cudaStream_t>(cfg->stream);
+  a.err = static_cast<unsigned *>(cfg->workspace);
   return a;
 }
 
 bool bwd_supported(const BwdArgs &a) {
   return (a.kqp ? attn_bwd_post_pick_rows(a) : attn_bwd_simt_pick_rows(a)) != 0;
+}
+
+// The tensor-core backward's strips for cfg, or 0 where its shape does not apply
+// (pointer alignment aside).
+size_t bwd_tc_bytes(const mta_cfg *c) {
+  const bool shape = c->dtype == MTA_BF16 && (c->d == 64 || c->d == 128) && c->c_q == 6 && c->c_k == 11 &&
+                     c->kq_place == MTA_PRE && !c->kq_post && (c->head_place == MTA_OFF || c->c_h == 2);
+  return shape ? attn_bwd_tc_workspace_bytes(c->B, c->H, c->L, c->c_q, c->head_place) : 0;
+}
+
+// Which backward serves `a`: path 0 the tensor-core one where it applies and
+// `room` bytes hold its strips, else the CUDA-core one; 1 the CUDA-core one; 3
+// the tensor-core one.  Returns the status of the choice; *tc says which.
+mta_status select_bwd(const BwdArgs &a, const mta_cfg *cfg, int path, size_t room, bool *tc) {
+  const bool tc_shape = attn_bwd_tc_supported(a);
+  const size_t need = bwd_tc_bytes(cfg);
+  if (path == 3) {
+    if (!tc_shape || need == 0) return MTA_ERR_UNSUPPORTED;
+    if (room < need) return MTA_ERR_WORKSPACE;
+    *tc = true;
+    return MTA_OK;
+  }
+  if (path == 2) return MTA_ERR_UNSUPPORTED;
+  *tc = path == 0 && tc_shape && need != 0 && room >= need;
+  if (!*tc && !bwd_supported(a)) return MTA_ERR_UNSUPPORTED;
+  return MTA_OK;
 }
 
 // The layer backward's fixed scratch, in this order (each 256-byte aligned): the
@@ -380,7 +409,7 @@ mta_status mta_layer_fwd(const void *x, const void *Wqkv, const float *theta, co
 }
 
 size_t mta_attn_bwd_workspace_bytes(const mta_cfg *cfg) {
-  return check_cfg(cfg) == MTA_OK ? kStatusBytes : 0;
+  return check_cfg(cfg) == MTA_OK ? kStatusBytes + bwd_tc_bytes(cfg) : 0;
 }
 
 mta_status mta_attn_bwd(const void *q, const void *k, const void *v, const float *theta_kq,
@@ -388,7 +417,7 @@ mta_status mta_attn_bwd(const void *q, const void *k, const void *v, const float
                         float *dk, float *dv, float *dtheta, float *dw) {
   mta_status s = check_cfg(cfg);
   if (s != MTA_OK) return s;
-  if (cfg->path > 1) return MTA_ERR_UNSUPPORTED;
+  if (cfg->path == 2) return MTA_ERR_UNSUPPORTED;
   if ((s = check_attn_pointers(q, k, v, theta_kq, w_head, cfg, dout)) != MTA_OK) return s;
   if (!dq || !dk || !dv || !aligned(dq, 4) || !aligned(dk, 4) || !aligned(dv, 4)) return MTA_ERR_INVALID;
   {
@@ -401,17 +430,22 @@ mta_status mta_attn_bwd(const void *q, const void *k, const void *v, const float
   if ((dtheta && !aligned(dtheta, 4)) || (dw && !aligned(dw, 4))) return MTA_ERR_INVALID;
   if ((s = check_workspace(cfg, kStatusBytes)) != MTA_OK) return s;
   BwdArgs a = make_bwd_args(q, k, v, theta_kq, w_head, dout, cfg, dq, dk, dv, dtheta, dw);
-  if (!bwd_supported(a)) return MTA_ERR_UNSUPPORTED;
+  bool tc = false;
+  if ((s = select_bwd(a, cfg, cfg->path, cfg->workspace_bytes - kStatusBytes, &tc)) != MTA_OK) return s;
   if ((s = clear_status(cfg)) != MTA_OK) return s;
   Marks m = make_marks(cfg);
   if (m.next() != cudaSuccess) return MTA_ERR_CUDA;
-  if ((a.kqp ? launch_attn_bwd_post(a) : launch_attn_bwd_simt(a)) != cudaSuccess) return MTA_ERR_CUDA;
+  const cudaError_t e = tc ? launch_attn_bwd_tc(a, static_cast<char *>(cfg->workspace) + kStatusBytes)
+                           : (a.kqp ? launch_attn_bwd_post(a) : launch_attn_bwd_simt(a));
+  if (e != cudaSuccess) return MTA_ERR_CUDA;
   return m.next() == cudaSuccess ? MTA_OK : MTA_ERR_CUDA;
 }
 
 size_t mta_layer_bwd_workspace_bytes(const mta_cfg *cfg) {
   const size_t fixed = layer_bwd_fixed_bytes(cfg);
-  return fixed ? fixed + kq_bytes(cfg) : 0;
+  // the forward recompute's contraction operands and the backward's strips are
+  // live at different times and share the space after the fixed part
+  return fixed ? fixed + std::max(kq_bytes(cfg), bwd_tc_bytes(cfg)) : 0;
 }
 
 mta_status mta_layer_bwd(const void *x, const void *Wqkv, const float *theta, const float *w_head,
@@ -471,7 +505,8 @@ mta_status mta_layer_bwd(const void *x, const void *Wqkv, const float *theta, co
   mta_cfg bcfg = acfg;
   bcfg.path = 0;
   BwdArgs ba = make_bwd_args(qkvb, qkvb + D, qkvb + 2 * D, theta, w_head, dobuf, &bcfg, dq, dk, dv, dtheta, dw);
-  if (!bwd_supported(ba)) return MTA_ERR_UNSUPPORTED;
+  bool bwd_tc = false;
+  if ((s = select_bwd(ba, &bcfg, 0, kq_room, &bwd_tc)) != MTA_OK) return s;
 
   const GnArgs g = make_gn(gn);
   cudaStream_t st = static_cast<cudaStream_t>(cfg->stream);
@@ -500,7 +535,9 @@ mta_status mta_layer_bwd(const void *x, const void *Wqkv, const float *theta, co
   if (launch_gemm(dout, ybuf, dWo, iD, iD, iT, true, true, true, err, st) != cudaSuccess || m.next() != cudaSuccess)
     return MTA_ERR_CUDA;
   // attention core: dq, dk, dv (fp32), dtheta, dw
-  if ((ba.kqp ? launch_attn_bwd_post(ba) : launch_attn_bwd_simt(ba)) != cudaSuccess || m.next() != cudaSuccess)
+  if ((bwd_tc ? launch_attn_bwd_tc(ba, kq_ws) : ba.kqp ? launch_attn_bwd_post(ba) : launch_attn_bwd_simt(ba)) !=
+          cudaSuccess ||
+      m.next() != cudaSuccess)
     return MTA_ERR_CUDA;
   if (launch_pack_qkv_grad(dq, dk, dv, static_cast<long long>(T), iD, dqkv, st) != cudaSuccess ||
       m.next() != cudaSuccess)
