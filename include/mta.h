@@ -120,8 +120,9 @@ typedef struct mta_cfg {
                             mta_layer_fwd: the QKV GEMM, the attention kernels
                             as above (with the norm fused), or, on the CUDA-core
                             path, the attention kernel and then the stand-alone
-                            group norm; the output GEMM.  mta_attn_bwd: its one
-                            kernel.                                              */
+                            group norm; the output GEMM.  mta_attn_bwd: the
+                            whole backward (one mark after its last kernel).
+                            mta_layer_bwd: see there.                            */
   int n_events;          /* number of handles in events, 0 .. 64                 */
 } mta_cfg;
 
