@@ -49,7 +49,7 @@ namespace {
 constexpr int kRowsT = 128;  // rows of the S strip (and of the halves of the dS / A'' strips)
 constexpr int kKeyTile = 128;
 constexpr int kThreadsB = 256;
-constexpr int kRowsPerCta = 4;  // rows of a CTA in the CUDA-core kernels: 4 x 64 threads
+constexpr int kRowsPerCta = 4;  // rows of a CTA in the softmax-gradient kernel: 4 x 64 threads
 
 struct Geo {
   int halo, c, no, rc, pitch;  // c_q - 1, c_k / 2, own rows, C rows, strip pitch (elements)
@@ -86,16 +86,23 @@ __device__ __forceinline__ void split_bf16(float x, __nv_bfloat16 &hi, __nv_bflo
 }
 
 // Step 2: C = Conv2d_theta(Mask_0 S) for the block's C rows (and pre mixing),
-// Mask_-inf, softmax over the row -> A strip.  CTA: one head group, 4 rows; thread
-// (row, sub): keys sub, sub + 64 of every 128-key tile.
+// Mask_-inf, softmax over the row -> A strip.  CTA: one head group, 16 rows;
+// thread (row, seg): 8 consecutive keys 8 seg .. 8 seg + 7 of every 128-key tile.
+// For each tap row a the thread loads the 8 + 2c values of the staged S row it
+// needs once and forms its 8 outputs x c_k taps from registers.  Key tiles past
+// the CTA's last row are skipped (their weights are zero and nothing reads them).
+constexpr int kRows = 16;               // rows of a CTA in the convolution kernels
+constexpr int kSeg = 8;                 // consecutive keys of a thread
+constexpr int kTilePitch = kKeyTile + 16;  // staged row: 128 + 2c keys, padded to 16 bytes
+
 template <int CQ, int CK, int CH>
 __global__ void __launch_bounds__(kThreadsB) bwd_scores_kernel(StripArgs p) {
-  constexpr int HALO = CQ - 1, C = CK / 2, TR = kRowsPerCta + HALO, TC = kKeyTile + 2 * C;
-  __shared__ float tile[CH][TR][TC];
+  constexpr int HALO = CQ - 1, C = CK / 2, TR = kRows + HALO, WIN = kSeg + 2 * C;
+  static_assert(kKeyTile + 2 * C <= kTilePitch, "tile pitch");
+  __shared__ __align__(16) float tile[CH][TR][kTilePitch];
   __shared__ float th[CH][CQ * CK], wm[CH * CH];
-  __shared__ float red[2 * kRowsPerCta];
   const int G = p.H / CH, bg = blockIdx.y, b = bg / G, g = bg % G;
-  const int u0 = blockIdx.x * kRowsPerCta, row = threadIdx.x >> 6, sub = threadIdx.x & 63;
+  const int u0 = blockIdx.x * kRows, row = threadIdx.x >> 4, seg = threadIdx.x & 15;
   const int u = u0 + row, i = p.r0 + u;
   const bool valid = u < p.g.rc && i < p.L;
   const int P = p.g.pitch;
@@ -108,77 +115,106 @@ __global__ void __launch_bounds__(kThreadsB) bwd_scores_kernel(StripArgs p) {
   float m[CH], l[CH];
 #pragma unroll
   for (int h = 0; h < CH; ++h) { m[h] = -INFINITY; l[h] = 0.f; }
-  const int jend = p.W;
-  for (int j0 = 0; j0 < jend; j0 += kKeyTile) {
+  const int i_last = min(p.L - 1, p.r0 + u0 + kRows - 1);  // the CTA's last query
+  for (int j0 = 0; j0 <= i_last; j0 += kKeyTile) {
     __syncthreads();
-    // stage Mask_0 S: strip rows u0 .. u0+TR-1 (queries r0 - HALO + su), keys j0-C .. j0+128+C-1
-    for (int x = threadIdx.x; x < CH * TR * TC; x += kThreadsB) {
-      const int hl = x / (TR * TC), r = (x / TC) % TR, cc = x % TC;
+    // stage Mask_0 S: strip rows u0 .. u0+TR-1 (queries r0 - HALO + su), keys j0-C ..
+    for (int x = threadIdx.x; x < CH * TR * kTilePitch; x += kThreadsB) {
+      const int hl = x / (TR * kTilePitch), r = (x / kTilePitch) % TR, cc = x % kTilePitch;
       const int su = u0 + r, iq = p.r0 - HALO + su, jk = j0 - C + cc;
       float v = 0.f;
       if (su < kRowsT && iq >= 0 && iq < p.L && jk >= 0 && jk <= iq) v = strip(p.S, hl, kRowsT)[su * P + jk];
       tile[hl][r][cc] = v;
     }
     __syncthreads();
-    if (!valid) continue;
+    const int jb = j0 + kSeg * seg;  // first key of the thread
+    if (!valid || jb > i) continue;
+    float cv[CH][kSeg];
 #pragma unroll
-    for (int kk = 0; kk < 2; ++kk) {
-      const int jl = sub + 64 * kk, j = j0 + jl;
-      if (j >= p.Wp) continue;
-      float cv[CH];
+    for (int h = 0; h < CH; ++h) {
 #pragma unroll
-      for (int h = 0; h < CH; ++h) {
-        float acc = 0.f;
+      for (int x = 0; x < kSeg; ++x) cv[h][x] = 0.f;
 #pragma unroll
-        for (int a = 0; a < CQ; ++a)
+      for (int a = 0; a < CQ; ++a) {
+        // keys jb - c .. jb + 7 + c of query i - a: tile columns 8 seg .. 8 seg + 7 + 2c
+        float w[WIN];
+        const float4 *src = reinterpret_cast<const float4 *>(&tile[h][row + HALO - a][kSeg * seg]);
 #pragma unroll
-          for (int t = 0; t < CK; ++t) acc = fmaf(th[h][a * CK + t], tile[h][row + HALO - a][jl + 2 * C - t], acc);
-        cv[h] = acc;
-      }
-      if (p.hp == 1 && p.Cpre) {
-#pragma unroll
-        for (int h = 0; h < CH; ++h) strip(p.Cpre, h, p.g.rc)[u * P + j] = j <= i ? cv[h] : 0.f;
-      }
-#pragma unroll
-      for (int h = 0; h < CH; ++h) {
-        float x = cv[h];
-        if (p.hp == 1) {
-          x = 0.f;
-#pragma unroll
-          for (int s = 0; s < CH; ++s) x = fmaf(wm[h * CH + s], cv[s], x);
+        for (int v4 = 0; v4 < (WIN + 3) / 4; ++v4) {
+          const float4 q4 = src[v4];
+          if (4 * v4 + 0 < WIN) w[4 * v4 + 0] = q4.x;
+          if (4 * v4 + 1 < WIN) w[4 * v4 + 1] = q4.y;
+          if (4 * v4 + 2 < WIN) w[4 * v4 + 2] = q4.z;
+          if (4 * v4 + 3 < WIN) w[4 * v4 + 3] = q4.w;
         }
-        // Mask_-inf: keys after the query
-        x = j <= i ? x : -INFINITY;
-        strip(p.A, h, p.g.rc)[u * P + j] = x;  // logits for now
-        if (x > m[h]) {
-          l[h] = l[h] * __expf(m[h] - x) + 1.f;
-          m[h] = x;
-        } else if (x != -INFINITY) {
-          l[h] += __expf(x - m[h]);
-        }
+        // C[i][j] += theta[a][t] S[i-a][j-(t-c)]: key j - t + c = column x + 2c - t
+#pragma unroll
+        for (int t = 0; t < CK; ++t)
+#pragma unroll
+          for (int x = 0; x < kSeg; ++x) cv[h][x] = fmaf(th[h][a * CK + t], w[x + 2 * C - t], cv[h][x]);
       }
     }
+    if (p.hp == 1 && p.Cpre) {
+#pragma unroll
+      for (int h = 0; h < CH; ++h) {
+        float *dst = strip(p.Cpre, h, p.g.rc) + u * P + jb;
+#pragma unroll
+        for (int x = 0; x < kSeg; x += 4)
+          *reinterpret_cast<float4 *>(dst + x) = make_float4(cv[h][x], cv[h][x + 1], cv[h][x + 2], cv[h][x + 3]);
+      }
+    }
+#pragma unroll
+    for (int h = 0; h < CH; ++h) {
+      float lg[kSeg];
+#pragma unroll
+      for (int x = 0; x < kSeg; ++x) {
+        float z = cv[h][x];
+        if (p.hp == 1) {
+          z = 0.f;
+#pragma unroll
+          for (int s2 = 0; s2 < CH; ++s2) z = fmaf(wm[h * CH + s2], cv[s2][x], z);
+        }
+        z = jb + x <= i ? z : -INFINITY;  // Mask_-inf
+        lg[x] = z;
+        if (z > m[h]) {
+          l[h] = l[h] * __expf(m[h] - z) + 1.f;
+          m[h] = z;
+        } else if (z != -INFINITY) {
+          l[h] += __expf(z - m[h]);
+        }
+      }
+      float *dst = strip(p.A, h, p.g.rc) + u * P + jb;  // logits for now
+#pragma unroll
+      for (int x = 0; x < kSeg; x += 4)
+        *reinterpret_cast<float4 *>(dst + x) = make_float4(lg[x], lg[x + 1], lg[x + 2], lg[x + 3]);
+    }
   }
-  // row statistics over the 64 threads of the row
+  // row statistics over the 16 threads of the row (16 consecutive lanes)
   float mr[CH], lr[CH];
 #pragma unroll
   for (int h = 0; h < CH; ++h) {
     float mx = m[h];
-    for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
-    __syncthreads();
-    if ((sub & 31) == 0) red[2 * row + (sub >> 5)] = mx;
-    __syncthreads();
-    mr[h] = fmaxf(red[2 * row], red[2 * row + 1]);
-    const float part = m[h] == -INFINITY ? 0.f : l[h] * __expf(m[h] - mr[h]);
-    lr[h] = blocksum64(part, red, row, sub);
+    for (int o = 8; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+    float part = m[h] == -INFINITY ? 0.f : l[h] * __expf(m[h] - mx);
+    for (int o = 8; o > 0; o >>= 1) part += __shfl_xor_sync(0xffffffffu, part, o);
+    mr[h] = mx;
+    lr[h] = part;
   }
   if (!valid) return;
-  for (int j = sub; j < p.Wp; j += 64) {
+  for (int jb = kSeg * seg; jb <= i; jb += kKeyTile) {
 #pragma unroll
     for (int h = 0; h < CH; ++h) {
-      float *a = strip(p.A, h, p.g.rc) + u * P + j;
-      const float x = *a;
-      *a = j <= i ? __expf(x - mr[h]) / lr[h] : 0.f;
+      float *a = strip(p.A, h, p.g.rc) + u * P + jb;
+      const float inv = 1.f / lr[h];
+#pragma unroll
+      for (int x = 0; x < kSeg; x += 4) {
+        float4 v = *reinterpret_cast<float4 *>(a + x);
+        v.x = jb + x + 0 <= i ? __expf(v.x - mr[h]) * inv : 0.f;
+        v.y = jb + x + 1 <= i ? __expf(v.y - mr[h]) * inv : 0.f;
+        v.z = jb + x + 2 <= i ? __expf(v.z - mr[h]) * inv : 0.f;
+        v.w = jb + x + 3 <= i ? __expf(v.w - mr[h]) * inv : 0.f;
+        *reinterpret_cast<float4 *>(a + x) = v;
+      }
     }
   }
 }
@@ -315,14 +351,17 @@ __global__ void __launch_bounds__(kThreadsB) bwd_softmax_grad_kernel(StripArgs p
 
 // Step 5: dS = [j <= i] sum theta[a][t] dC[i+a][j+t-c] (hi / lo halves) for the
 // block's own rows, zeros elsewhere, and dtheta over the own rows.  CTA: one
-// head, 4 rows u = 0 .. 127.
+// head, 16 rows u = 0 .. 127; thread (row, seg): 8 consecutive keys, register
+// windows of 8 + 2c staged values per tap row as in the scores kernel.  Key tiles
+// past the CTA's last row only write zeros.
 template <int CQ, int CK>
 __global__ void __launch_bounds__(kThreadsB) bwd_adjoint_kernel(StripArgs p) {
-  constexpr int HALO = CQ - 1, C = CK / 2, TR = kRowsPerCta + HALO, TC = kKeyTile + 2 * C, NT = CQ * CK;
-  __shared__ float dct[TR][TC], st[TR][TC];
+  constexpr int HALO = CQ - 1, C = CK / 2, TR = kRows + HALO, NT = CQ * CK, WIN = kSeg + 2 * C;
+  __shared__ __align__(16) float dct[TR][kTilePitch];
+  __shared__ __align__(16) float st[TR][kTilePitch];
   __shared__ float th[NT];
   const int z = blockIdx.y, h = z % p.H;
-  const int u0 = blockIdx.x * kRowsPerCta, row = threadIdx.x >> 6, sub = threadIdx.x & 63;
+  const int u0 = blockIdx.x * kRows, row = threadIdx.x >> 4, seg = threadIdx.x & 15;
   const int u = u0 + row, i = p.r0 + u;
   const bool own = u < p.g.no && i < p.L;
   const int P = p.g.pitch;
@@ -333,39 +372,74 @@ __global__ void __launch_bounds__(kThreadsB) bwd_adjoint_kernel(StripArgs p) {
   float dth[NT];
 #pragma unroll
   for (int x = 0; x < NT; ++x) dth[x] = 0.f;
+  const int i_last = min(p.L - 1, p.r0 + min(u0 + kRows - 1, p.g.no - 1));  // last own query of the CTA
   for (int j0 = 0; j0 < p.Wp; j0 += kKeyTile) {
-    __syncthreads();
-    for (int x = threadIdx.x; x < TR * TC; x += kThreadsB) {
-      const int r = x / TC, cc = x % TC, jk = j0 - C + cc;
-      // dC rows u0 .. u0+TR-1 (queries r0 + u'), zero past the C rows, the sequence and the diagonal
-      const int uc = u0 + r, ic = p.r0 + uc;
-      dct[r][cc] = (uc < p.g.rc && ic < p.L && jk >= 0 && jk <= ic) ? Dz[uc * P + jk] : 0.f;
-      // Mask_0 S rows u0 .. u0+TR-1 of the S strip (queries r0 - HALO + su)
-      const int su = u0 + r, is = p.r0 - HALO + su;
-      st[r][cc] = (su < kRowsT && is >= 0 && is < p.L && jk >= 0 && jk <= is) ? Sz[su * P + jk] : 0.f;
-    }
-    __syncthreads();
-#pragma unroll
-    for (int kk = 0; kk < 2; ++kk) {
-      const int jl = sub + 64 * kk, j = j0 + jl;
-      if (j >= p.Wp) continue;
-      float ds = 0.f;
-      if (own && j <= i) {
-#pragma unroll
-        for (int a = 0; a < CQ; ++a)
-#pragma unroll
-          for (int t = 0; t < CK; ++t) ds = fmaf(th[a * CK + t], dct[row + a][jl + t], ds);
-        // dtheta[a][t] += dC[i][j] Mask_0 S[i-a][j-(t-c)]
-        const float g = dct[row][jl + C];
-#pragma unroll
-        for (int a = 0; a < CQ; ++a)
-#pragma unroll
-          for (int t = 0; t < CK; ++t) dth[a * CK + t] = fmaf(g, st[row + HALO - a][jl + 2 * C - t], dth[a * CK + t]);
+    const int jb = j0 + kSeg * seg;
+    const bool work = j0 <= i_last && u0 < p.g.no;  // uniform over the CTA
+    if (work) {
+      __syncthreads();
+      for (int x = threadIdx.x; x < TR * kTilePitch; x += kThreadsB) {
+        const int r = x / kTilePitch, cc = x % kTilePitch, jk = j0 - C + cc;
+        // dC rows u0 .. u0+TR-1 (queries r0 + u'), zero past the C rows, the sequence and the diagonal
+        const int uc = u0 + r, ic = p.r0 + uc;
+        dct[r][cc] = (uc < p.g.rc && ic < p.L && jk >= 0 && jk <= ic) ? Dz[uc * P + jk] : 0.f;
+        // Mask_0 S rows u0 .. u0+TR-1 of the S strip (queries r0 - HALO + su)
+        const int su = u0 + r, is = p.r0 - HALO + su;
+        st[r][cc] = (su < kRowsT && is >= 0 && is < p.L && jk >= 0 && jk <= is) ? Sz[su * P + jk] : 0.f;
       }
-      __nv_bfloat16 hi, lo;
-      split_bf16(ds, hi, lo);
-      dSz[u * P + j] = hi;
-      dSz[(kRowsT + u) * P + j] = lo;
+      __syncthreads();
+    }
+    float ds[kSeg];
+#pragma unroll
+    for (int x = 0; x < kSeg; ++x) ds[x] = 0.f;
+    if (work && own && jb <= i && jb < p.Wp) {
+      // dC[i][j] of the thread's keys (zero past the diagonal) for dtheta
+      float gk[kSeg];
+#pragma unroll
+      for (int x = 0; x < kSeg; ++x) gk[x] = dct[row][kSeg * seg + C + x];
+#pragma unroll
+      for (int a = 0; a < CQ; ++a) {
+        float w[WIN], v[WIN];
+        const float4 *sd = reinterpret_cast<const float4 *>(&dct[row + a][kSeg * seg]);
+        const float4 *ss = reinterpret_cast<const float4 *>(&st[row + HALO - a][kSeg * seg]);
+#pragma unroll
+        for (int v4 = 0; v4 < (WIN + 3) / 4; ++v4) {
+          const float4 q4 = sd[v4], s4 = ss[v4];
+          if (4 * v4 + 0 < WIN) { w[4 * v4 + 0] = q4.x; v[4 * v4 + 0] = s4.x; }
+          if (4 * v4 + 1 < WIN) { w[4 * v4 + 1] = q4.y; v[4 * v4 + 1] = s4.y; }
+          if (4 * v4 + 2 < WIN) { w[4 * v4 + 2] = q4.z; v[4 * v4 + 2] = s4.z; }
+          if (4 * v4 + 3 < WIN) { w[4 * v4 + 3] = q4.w; v[4 * v4 + 3] = s4.w; }
+        }
+#pragma unroll
+        for (int t = 0; t < CK; ++t) {
+          const float tt = th[a * CK + t];
+          float acc = dth[a * CK + t];
+#pragma unroll
+          for (int x = 0; x < kSeg; ++x) {
+            // dS[i][j] += theta[a][t] dC[i+a][j+t-c]: column x + t
+            ds[x] = fmaf(tt, w[x + t], ds[x]);
+            // dtheta[a][t] += dC[i][j] Mask_0 S[i-a][j-(t-c)]: column x + 2c - t
+            acc = fmaf(gk[x], v[x + 2 * C - t], acc);
+          }
+          dth[a * CK + t] = acc;
+        }
+      }
+#pragma unroll
+      for (int x = 0; x < kSeg; ++x) ds[x] = jb + x <= i ? ds[x] : 0.f;
+    }
+    if (jb < p.Wp) {
+      uint32_t hi[kSeg / 2], lo[kSeg / 2];
+#pragma unroll
+      for (int x = 0; x < kSeg; x += 2) {
+        __nv_bfloat16 h0, l0, h1, l1;
+        split_bf16(ds[x], h0, l0);
+        split_bf16(ds[x + 1], h1, l1);
+        hi[x / 2] = static_cast<uint32_t>(__bfloat16_as_ushort(h0)) | (static_cast<uint32_t>(__bfloat16_as_ushort(h1)) << 16);
+        lo[x / 2] = static_cast<uint32_t>(__bfloat16_as_ushort(l0)) | (static_cast<uint32_t>(__bfloat16_as_ushort(l1)) << 16);
+      }
+      *reinterpret_cast<uint4 *>(dSz + static_cast<long long>(u) * P + jb) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
+      *reinterpret_cast<uint4 *>(dSz + static_cast<long long>(kRowsT + u) * P + jb) =
+          make_uint4(lo[0], lo[1], lo[2], lo[3]);
     }
   }
   if (p.dtheta) {
@@ -474,8 +548,13 @@ cudaError_t launch_attn_bwd_tc(const BwdArgs &a, void *ws) {
   sp.S = S; sp.Cpre = Cpre; sp.A = A; sp.D = D; sp.dS = dS; sp.Ap = Ap;
   sp.dtheta = a.dtheta; sp.dw = a.hp ? a.dw : nullptr;
 
-  auto K_major = [](int pos_row, int off_mn, int off_k) { return BgOperand{0, pos_row, off_mn, off_k}; };
-  auto MN_major = [](int pos_row, int off_mn, int off_k) { return BgOperand{1, pos_row, off_mn, off_k}; };
+  auto K_major = [](int pos_row, int off_mn, int off_k) { return BgOperand{0, pos_row, off_mn, off_k, 0, 0}; };
+  auto MN_major = [](int pos_row, int off_mn, int off_k) { return BgOperand{1, pos_row, off_mn, off_k, 0, 0}; };
+  auto periodic = [](BgOperand o, int period, int shift) {
+    o.k_period = period;
+    o.period_shift = shift;
+    return o;
+  };
   for (int r0 = 0; r0 < a.L; r0 += g.no) {
     const int W = std::min(a.L, r0 + g.rc), Wp = (W + 63) / 64 * 64;
     sp.r0 = r0; sp.W = W; sp.Wp = Wp;
@@ -487,7 +566,7 @@ cudaError_t launch_attn_bwd_tc(const BwdArgs &a, void *ws) {
     ga.a = K_major(2, r0 - g.halo, 0); ga.b = K_major(2, 0, 0);
     if ((e = launch_gemm_batched(tq, tk, ga, st)) != cudaSuccess) return e;
     // 2. convolution, mixing, softmax -> A
-    const dim3 grid2((g.rc + kRowsPerCta - 1) / kRowsPerCta, a.B * G);
+    const dim3 grid2((g.rc + kRows - 1) / kRows, a.B * G);
     if (ch == 2)
       bwd_scores_kernel<6, 11, 2><<<grid2, kThreadsB, 0, st>>>(sp);
     else
@@ -506,33 +585,30 @@ cudaError_t launch_attn_bwd_tc(const BwdArgs &a, void *ws) {
       bwd_softmax_grad_kernel<1><<<grid4, kThreadsB, 0, st>>>(sp);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     // 5. dS (hi / lo), dtheta
-    bwd_adjoint_kernel<6, 11><<<dim3(kRowsT / kRowsPerCta, static_cast<unsigned>(Z)), kThreadsB, 0, st>>>(sp);
+    bwd_adjoint_kernel<6, 11><<<dim3(kRowsT / kRows, static_cast<unsigned>(Z)), kThreadsB, 0, st>>>(sp);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
-    // 6. dQ rows r0 .. r0 + no - 1 = s dS K (hi, then lo added)
+    // 6. dQ rows r0 .. r0 + no - 1 = s dS K: K runs over the keys twice, the hi
+    //    rows of dS against K, then its lo rows (128 further) against K again
     const int own = std::min(g.no, a.L - r0);
     BgArgs gq = {};
     gq.Z = static_cast<int>(Z); gq.H = a.H; gq.err = err;
-    gq.M = own; gq.N = a.d; gq.K = W; gq.alpha = a.scale;
+    gq.M = own; gq.N = a.d; gq.K = 2 * Wp; gq.alpha = a.scale; gq.accumulate = 0;
     gq.C = a.dq + static_cast<long long>(r0) * HD; gq.sm = HD; gq.sh = a.d; gq.sb = LHD;
-    gq.b = MN_major(2, 0, 0);
-    for (int half = 0; half < 2; ++half) {
-      gq.a = K_major(1, half * kRowsT, 0);
-      gq.accumulate = half;
-      if ((e = launch_gemm_batched(tdS, tk, gq, st)) != cudaSuccess) return e;
-    }
-    //    dK += s dS^T Q and dV += A''^T dO over the block's rows (keys 0 .. W-1)
+    gq.a = periodic(K_major(1, 0, 0), Wp, kRowsT);
+    gq.b = periodic(MN_major(2, 0, 0), Wp, 0);
+    if ((e = launch_gemm_batched(tdS, tk, gq, st)) != cudaSuccess) return e;
+    //    dK += s dS^T Q and dV += A''^T dO over the block's rows (keys 0 .. W-1): K runs
+    //    over the 256 rows of the hi and lo halves, the block's 128 query rows twice
     BgArgs gk = {};
     gk.Z = static_cast<int>(Z); gk.H = a.H; gk.err = err;
-    gk.M = W; gk.N = a.d; gk.K = kRowsT; gk.accumulate = 1;
+    gk.M = W; gk.N = a.d; gk.K = 2 * kRowsT; gk.accumulate = 1;
     gk.sm = HD; gk.sh = a.d; gk.sb = LHD;
-    gk.b = MN_major(2, 0, r0);
-    for (int half = 0; half < 2; ++half) {
-      gk.a = MN_major(1, 0, half * kRowsT);
-      gk.alpha = a.scale; gk.C = a.dk;
-      if ((e = launch_gemm_batched(tdS, tq, gk, st)) != cudaSuccess) return e;
-      gk.alpha = 1.f; gk.C = a.dv;
-      if ((e = launch_gemm_batched(tAp, tdo, gk, st)) != cudaSuccess) return e;
-    }
+    gk.a = MN_major(1, 0, 0);
+    gk.b = periodic(MN_major(2, 0, r0), kRowsT, 0);
+    gk.alpha = a.scale; gk.C = a.dk;
+    if ((e = launch_gemm_batched(tdS, tq, gk, st)) != cudaSuccess) return e;
+    gk.alpha = 1.f; gk.C = a.dv;
+    if ((e = launch_gemm_batched(tAp, tdo, gk, st)) != cudaSuccess) return e;
   }
   return cudaSuccess;
 }

@@ -53,6 +53,10 @@ __device__ __forceinline__ void load_op(uint8_t *dst, const CUtensorMap *map, co
     else
       tma_load_4d(d, map, bar, c0, h, row, b);
   };
+  if (o.k_period) {
+    r += (k / o.k_period) * o.period_shift;
+    k %= o.k_period;
+  }
   if (!o.mn) {
     load(dst, k + o.off_k, r + o.off_mn);
   } else {
@@ -228,6 +232,9 @@ cudaError_t launch_gemm_batched(const BgTensor &A, const BgTensor &B, const BgAr
     return cudaGetLastError();
   };
   if (args.N > 128) return run(gemm_batched_kernel<256>, 256, BG<256>::SMEM);
+  // narrow outputs: 64-column tiles when 128-column ones would leave SMs idle
+  const long long t128 = static_cast<long long>(args.Z) * ((args.M + BM - 1) / BM) * ((args.N + 127) / 128);
+  if (args.N <= 64 || t128 < sms) return run(gemm_batched_kernel<64>, 64, BG<64>::SMEM);
   return run(gemm_batched_kernel<128>, 128, BG<128>::SMEM);
 }
 

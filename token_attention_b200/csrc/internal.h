@@ -141,6 +141,11 @@ struct BgOperand {
   int pos_row; // as the tensor's
   int off_mn;  // added to the M (or N) index
   int off_k;   // added to the K index
+  // K index k reads the operand at k mod k_period (a multiple of 64; 0 = no
+  // period), its M (N) index shifted by (k / k_period) * period_shift: two halves
+  // of one operand summed in one GEMM against the same other operand
+  int k_period;
+  int period_shift;
 };
 struct BgArgs {
   int Z, H;         // batches z = b * H + h
