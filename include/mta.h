@@ -266,7 +266,7 @@ mta_status mta_group_norm_scale_bwd(const void *o, const float *dy, const mta_gn
  * Two implementations (cfg->path):
  *   3: the contractions on the tensor cores (attn_bwd_tc.cu): bf16, d = 64 or
  *      128, c_q = 6, c_k = 11, kq_place = MTA_PRE, no post-softmax convolution,
- *      c_h = 2 with head mixing; query blocks of 118 rows, every head at once,
+ *      c_h = 2 with head mixing; query blocks of 246 rows, every head at once,
  *      their maps in strips of the workspace (S = s Q K^T, dA'' = dO V^T, dQ,
  *      dK, dV as batched tcgen05 GEMMs; the convolution, its adjoint and the
  *      softmax on the CUDA cores).  MTA_ERR_UNSUPPORTED for other
@@ -281,9 +281,9 @@ mta_status mta_group_norm_scale_bwd(const void *o, const float *dy, const mta_gn
  * paths) and dk, dv (path 1) are summed with atomic additions, so their last
  * bits may differ between runs.  The workspace (mta_attn_bwd_workspace_bytes)
  * holds the error word and, where path 3 applies, its strips: for one query
- * block of every head, a 128-row S strip and two (three with pre-softmax
- * mixing) fp32 strips of 123 rows over the keys, and two bf16 strips of 256 rows
- * (B*H*pitch*(128*4 + 2*123*4 + 2*256*2) bytes, pitch = L rounded up to 64).  No
+ * block of every head, a 256-row S strip and two (three with pre-softmax
+ * mixing) fp32 strips of 251 rows over the keys, and two bf16 strips of 512 rows
+ * (B*H*pitch*(256*4 + 2*251*4 + 2*512*2) bytes, pitch = L rounded up to 64).  No
  * L x L map is stored. */
 size_t mta_attn_bwd_workspace_bytes(const mta_cfg *cfg);
 mta_status mta_attn_bwd(const void *q, const void *k, const void *v, const float *theta_kq,

@@ -233,10 +233,10 @@ def test_backward_argument_errors(L):
     small.workspace, small.workspace_bytes = 0x100000, 16
     assert f(small) == 3
     # the status word, then the tensor-core backward's strips for one query block of
-    # every head (B H = 8, pitch 64): S [128 rows] and A, dA/dC [123 rows] fp32, the
-    # dS and A'' halves [256 rows] bf16
-    Z, P, rc = 2 * 4, 64, 128 - 5
-    strips = up(Z * 128 * P * 4) + 2 * up(Z * rc * P * 4) + 2 * up(Z * 256 * P * 2)
+    # every head (B H = 8, pitch 64): S [256 rows] and A, dA/dC [251 rows] fp32, the
+    # dS and A'' halves [512 rows] bf16
+    Z, P, rc = 2 * 4, 64, 256 - 5
+    strips = up(Z * 256 * P * 4) + 2 * up(Z * rc * P * 4) + 2 * up(Z * 512 * P * 2)
     assert L.mta_attn_bwd_workspace_bytes(ctypes.byref(good_cfg())) == 256 + strips
     # pre-softmax mixing keeps the unmixed C as well
     assert L.mta_attn_bwd_workspace_bytes(ctypes.byref(good_cfg(head_place=mta.PRE))) == \

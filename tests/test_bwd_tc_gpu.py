@@ -5,7 +5,7 @@ Every gradient (q, k, v, theta, w) at the CUDA-core backward's fp32 tolerance
 (relative L2 error 1e-4): the tensor-core path takes the bf16 inputs themselves as
 MMA operands and splits its computed operands (dS, A'') into two bf16 halves, so
 its products carry about 16 significant bits and its sums fp32 accumulation.
-Lengths span one query block (L <= 118), several blocks and a ragged tail; the
+Lengths span one query block (L <= 246), several blocks and a ragged tail; the
 pretraining recipe runs at its full length for one head group.
 """
 import numpy as np
@@ -62,8 +62,8 @@ def check(wl, inp, dout, path=mta.PATH_KQ):
     return got, out
 
 
-CASES = [(128, synth.POST, 9), (128, synth.POST, 130), (128, synth.PRE, 130), (128, synth.OFF, 70),
-         (64, synth.POST, 300), (64, synth.PRE, 250), (64, synth.OFF, 119), (128, synth.POST, 237)]
+CASES = [(128, synth.POST, 9), (128, synth.POST, 247), (128, synth.PRE, 300), (128, synth.OFF, 70),
+         (64, synth.POST, 600), (64, synth.PRE, 250), (64, synth.OFF, 119), (128, synth.POST, 237)]
 
 
 @pytest.mark.parametrize("d,hp,L", CASES)
@@ -76,7 +76,7 @@ def test_bwd_tc_small(d, hp, L):
 
 
 def test_bwd_tc_matches_cuda_core_path():
-    """Both backward paths on the same inputs (L = 512, four query blocks and a tail)."""
+    """Both backward paths on the same inputs (L = 512, two query blocks and a tail)."""
     wl = synth.shrink(synth.WORKLOADS["pretrain_d128_L2048"], B=1, H=4, L=512, seed=951)
     inp = synth.make_attn_inputs(wl)
     dout = synth.round_bf16(synth.normal(wl.seed, 20, (wl.B, wl.L, wl.H, wl.d)))
@@ -88,7 +88,7 @@ def test_bwd_tc_matches_cuda_core_path():
 
 
 def test_bwd_tc_full_length_one_group():
-    """The pretraining recipe at its full length L = 2048 (18 query blocks), one batch
+    """The pretraining recipe at its full length L = 2048 (9 query blocks), one batch
     and one head group, against the oracle's full L x L backward of that group."""
     wl = synth.shrink(synth.WORKLOADS["pretrain_d128_L2048"], B=1, H=2, seed=952)
     inp = synth.make_attn_inputs(wl)

@@ -16,14 +16,14 @@
 //   dtheta[a][t] = sum dC[i][j] Mask_0 S[i-a][j-(t-c)]
 //   dQ = s dS K, dK = s dS^T Q               (tensor cores)
 //
-// Query blocks of NO = 128 - 2 (c_q - 1) rows are processed one after another,
+// Query blocks of NO = 256 - 2 (c_q - 1) rows are processed one after another,
 // all heads at once.  For block rows r0 .. r0+NO-1 the maps are held in strips
 // of the workspace that span every key up to the block's last row: S for rows
-// r0-(c_q-1) .. r0+NO+c_q-2 (128 rows: the convolution reads c_q-1 earlier query
+// r0-(c_q-1) .. r0+NO+c_q-2 (256 rows: the convolution reads c_q-1 earlier query
 // rows, its adjoint c_q-1 later ones), A, dA'' then dC for rows r0 .. r0+NO+c_q-2,
 // dS and A'' for the block's own rows.  A strip holds whole rows, so the softmax
 // statistics and D come from the strip itself (no statistics pass).  The strips
-// are O(B H 128 L): never an L x L map.  Per block:
+// are O(B H 256 L): never an L x L map.  Per block:
 //   1. S strip      = s Q K^T                      batched GEMM (fp32 out)
 //   2. C, softmax   -> A strip                     bwd_scores_kernel (CUDA cores)
 //   3. dA'' strip   = dO V^T                       batched GEMM
@@ -46,7 +46,7 @@
 namespace mta {
 namespace {
 
-constexpr int kRowsT = 128;  // rows of the S strip (and of the halves of the dS / A'' strips)
+constexpr int kRowsT = 256;  // rows of the S strip (and of the halves of the dS / A'' strips)
 constexpr int kKeyTile = 128;
 constexpr int kThreadsB = 256;
 constexpr int kRowsPerCta = 4;  // rows of a CTA in the softmax-gradient kernel: 4 x 64 threads
@@ -61,12 +61,12 @@ struct StripArgs {
   Geo g;
   const float *theta;         // [H][c_q][c_k]
   const float *w;             // [H/c_h][c_h][c_h]
-  float *S;                   // [B][H][128][pitch]
+  float *S;                   // [B][H][256][pitch]
   float *Cpre;                // [B][H][rc][pitch] pre-mixing C (pre mixing only)
   float *A;                   // [B][H][rc][pitch]
   float *D;                   // [B][H][rc][pitch]: dA'' from the GEMM, then dC
-  __nv_bfloat16 *dS;          // [B][H][256][pitch]: hi rows 0..127, lo rows 128..255
-  __nv_bfloat16 *Ap;          // [B][H][256][pitch]: A'' hi / lo
+  __nv_bfloat16 *dS;          // [B][H][512][pitch]: hi rows 0..255, lo rows 256..511
+  __nv_bfloat16 *Ap;          // [B][H][512][pitch]: A'' hi / lo
   float *dtheta, *dw;
 };
 
@@ -95,6 +95,43 @@ constexpr int kRows = 16;               // rows of a CTA in the convolution kern
 constexpr int kSeg = 8;                 // consecutive keys of a thread
 constexpr int kTilePitch = kKeyTile + 16;  // staged row: 128 + 2c keys, padded to 16 bytes
 
+// Stages TR rows of a strip into tile[TR][kTilePitch]: tile row r holds strip row
+// row0 + r (its query q0 + r; zeros once the strip row reaches nrows or the
+// query reaches L), tile column cc key j0 - C + cc, zero for a key below 0 or
+// past the row's query (Mask_0 and the causal mask of the gradients).  A warp per
+// row, 16-byte loads of keys j0 - 8 + 4 v (aligned, the strip pitch being a
+// multiple of 64), each stored to its four columns.
+template <int TR, int C>
+__device__ __forceinline__ void stage_rows(float (*tile)[kTilePitch], const float *strip0, int P, int row0,
+                                           int nrows, int q0, int L, int j0) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  constexpr int NV = (kTilePitch + 8 - C + 3) / 4;  // float4 groups reaching the tile
+  for (int r = warp; r < TR; r += kThreadsB / 32) {
+    const int sr = row0 + r, q = q0 + r;
+    const bool rv = sr < nrows && q >= 0 && q < L;
+    const float *src = strip0 + static_cast<long long>(sr) * P;
+    for (int v = lane; v < NV; v += 32) {
+      const int k0 = j0 - 8 + 4 * v;
+      float x[4] = {0.f, 0.f, 0.f, 0.f};
+      if (rv && k0 + 3 >= 0 && k0 <= q) {
+        if (k0 >= 0 && k0 + 3 <= q) {
+          const float4 f = *reinterpret_cast<const float4 *>(src + k0);
+          x[0] = f.x; x[1] = f.y; x[2] = f.z; x[3] = f.w;
+        } else {
+#pragma unroll
+          for (int e = 0; e < 4; ++e)
+            if (k0 + e >= 0 && k0 + e <= q) x[e] = src[k0 + e];
+        }
+      }
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const int cc = 4 * v - 8 + C + e;
+        if (cc >= 0 && cc < kTilePitch) tile[r][cc] = x[e];
+      }
+    }
+  }
+}
+
 template <int CQ, int CK, int CH>
 __global__ void __launch_bounds__(kThreadsB) bwd_scores_kernel(StripArgs p) {
   constexpr int HALO = CQ - 1, C = CK / 2, TR = kRows + HALO, WIN = kSeg + 2 * C;
@@ -119,13 +156,9 @@ __global__ void __launch_bounds__(kThreadsB) bwd_scores_kernel(StripArgs p) {
   for (int j0 = 0; j0 <= i_last; j0 += kKeyTile) {
     __syncthreads();
     // stage Mask_0 S: strip rows u0 .. u0+TR-1 (queries r0 - HALO + su), keys j0-C ..
-    for (int x = threadIdx.x; x < CH * TR * kTilePitch; x += kThreadsB) {
-      const int hl = x / (TR * kTilePitch), r = (x / kTilePitch) % TR, cc = x % kTilePitch;
-      const int su = u0 + r, iq = p.r0 - HALO + su, jk = j0 - C + cc;
-      float v = 0.f;
-      if (su < kRowsT && iq >= 0 && iq < p.L && jk >= 0 && jk <= iq) v = strip(p.S, hl, kRowsT)[su * P + jk];
-      tile[hl][r][cc] = v;
-    }
+#pragma unroll
+    for (int hl = 0; hl < CH; ++hl)
+      stage_rows<TR, C>(tile[hl], strip(p.S, hl, kRowsT), P, u0, kRowsT, p.r0 - HALO + u0, p.L, j0);
     __syncthreads();
     const int jb = j0 + kSeg * seg;  // first key of the thread
     if (!valid || jb > i) continue;
@@ -378,15 +411,10 @@ __global__ void __launch_bounds__(kThreadsB) bwd_adjoint_kernel(StripArgs p) {
     const bool work = j0 <= i_last && u0 < p.g.no;  // uniform over the CTA
     if (work) {
       __syncthreads();
-      for (int x = threadIdx.x; x < TR * kTilePitch; x += kThreadsB) {
-        const int r = x / kTilePitch, cc = x % kTilePitch, jk = j0 - C + cc;
-        // dC rows u0 .. u0+TR-1 (queries r0 + u'), zero past the C rows, the sequence and the diagonal
-        const int uc = u0 + r, ic = p.r0 + uc;
-        dct[r][cc] = (uc < p.g.rc && ic < p.L && jk >= 0 && jk <= ic) ? Dz[uc * P + jk] : 0.f;
-        // Mask_0 S rows u0 .. u0+TR-1 of the S strip (queries r0 - HALO + su)
-        const int su = u0 + r, is = p.r0 - HALO + su;
-        st[r][cc] = (su < kRowsT && is >= 0 && is < p.L && jk >= 0 && jk <= is) ? Sz[su * P + jk] : 0.f;
-      }
+      // dC rows u0 .. u0+TR-1 (queries r0 + u'), zero past the C rows, the sequence and the diagonal
+      stage_rows<TR, C>(dct, Dz, P, u0, p.g.rc, p.r0 + u0, p.L, j0);
+      // Mask_0 S rows u0 .. u0+TR-1 of the S strip (queries r0 - HALO + su)
+      stage_rows<TR, C>(st, Sz, P, u0, kRowsT, p.r0 - HALO + u0, p.L, j0);
       __syncthreads();
     }
     float ds[kSeg];
@@ -588,7 +616,7 @@ cudaError_t launch_attn_bwd_tc(const BwdArgs &a, void *ws) {
     bwd_adjoint_kernel<6, 11><<<dim3(kRowsT / kRows, static_cast<unsigned>(Z)), kThreadsB, 0, st>>>(sp);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     // 6. dQ rows r0 .. r0 + no - 1 = s dS K: K runs over the keys twice, the hi
-    //    rows of dS against K, then its lo rows (128 further) against K again
+    //    rows of dS against K, then its lo rows (256 further) against K again
     const int own = std::min(g.no, a.L - r0);
     BgArgs gq = {};
     gq.Z = static_cast<int>(Z); gq.H = a.H; gq.err = err;
@@ -598,7 +626,7 @@ cudaError_t launch_attn_bwd_tc(const BwdArgs &a, void *ws) {
     gq.b = periodic(MN_major(2, 0, 0), Wp, 0);
     if ((e = launch_gemm_batched(tdS, tk, gq, st)) != cudaSuccess) return e;
     //    dK += s dS^T Q and dV += A''^T dO over the block's rows (keys 0 .. W-1): K runs
-    //    over the 256 rows of the hi and lo halves, the block's 128 query rows twice
+    //    over the rows of the hi and lo halves, the block's query rows twice
     BgArgs gk = {};
     gk.Z = static_cast<int>(Z); gk.H = a.H; gk.err = err;
     gk.M = W; gk.N = a.d; gk.K = 2 * kRowsT; gk.accumulate = 1;
