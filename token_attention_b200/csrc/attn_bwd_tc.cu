@@ -93,7 +93,16 @@ __device__ __forceinline__ void split_bf16(float x, __nv_bfloat16 &hi, __nv_bflo
 // the CTA's last row are skipped (their weights are zero and nothing reads them).
 constexpr int kRows = 16;               // rows of a CTA in the convolution kernels
 constexpr int kSeg = 8;                 // consecutive keys of a thread
-constexpr int kTilePitch = kKeyTile + 16;  // staged row: 128 + 2c keys, padded to 16 bytes
+// Staged rows are 164 floats (128 + 2c keys, padded): 656 bytes, 16 modulo 128, so
+// that the 16-byte window loads of a quarter warp -- four threads of one row and
+// four of the next, 32 bytes apart along a row -- fall on eight different bank
+// groups.
+constexpr int kTilePitch = 164;
+constexpr int kTileCols = kKeyTile + 16;  // columns staged (128 + 2c used)
+// thread -> (row, seg): a warp holds rows 2 warp, 2 warp + 1; lane bit 2 picks
+// the row, the other bits the 8-key segment
+__device__ __forceinline__ int tile_row(int tid) { return 2 * (tid >> 5) + ((tid >> 2) & 1); }
+__device__ __forceinline__ int tile_seg(int tid) { return (tid & 3) | (((tid & 31) >> 3) << 2); }
 
 // Stages TR rows of a strip into tile[TR][kTilePitch]: tile row r holds strip row
 // row0 + r (its query q0 + r; zeros once the strip row reaches nrows or the
@@ -105,7 +114,7 @@ template <int TR, int C>
 __device__ __forceinline__ void stage_rows(float (*tile)[kTilePitch], const float *strip0, int P, int row0,
                                            int nrows, int q0, int L, int j0) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  constexpr int NV = (kTilePitch + 8 - C + 3) / 4;  // float4 groups reaching the tile
+  constexpr int NV = (kTileCols + 8 - C + 3) / 4;  // float4 groups reaching the staged columns
   for (int r = warp; r < TR; r += kThreadsB / 32) {
     const int sr = row0 + r, q = q0 + r;
     const bool rv = sr < nrows && q >= 0 && q < L;
@@ -126,7 +135,7 @@ __device__ __forceinline__ void stage_rows(float (*tile)[kTilePitch], const floa
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
         const int cc = 4 * v - 8 + C + e;
-        if (cc >= 0 && cc < kTilePitch) tile[r][cc] = x[e];
+        if (cc >= 0 && cc < kTileCols) tile[r][cc] = x[e];
       }
     }
   }
@@ -135,11 +144,11 @@ __device__ __forceinline__ void stage_rows(float (*tile)[kTilePitch], const floa
 template <int CQ, int CK, int CH>
 __global__ void __launch_bounds__(kThreadsB) bwd_scores_kernel(StripArgs p) {
   constexpr int HALO = CQ - 1, C = CK / 2, TR = kRows + HALO, WIN = kSeg + 2 * C;
-  static_assert(kKeyTile + 2 * C <= kTilePitch, "tile pitch");
+  static_assert(kKeyTile + 2 * C + 4 <= kTileCols && kTileCols <= kTilePitch, "tile columns");
   __shared__ __align__(16) float tile[CH][TR][kTilePitch];
   __shared__ float th[CH][CQ * CK], wm[CH * CH];
   const int G = p.H / CH, bg = blockIdx.y, b = bg / G, g = bg % G;
-  const int u0 = blockIdx.x * kRows, row = threadIdx.x >> 4, seg = threadIdx.x & 15;
+  const int u0 = blockIdx.x * kRows, row = tile_row(threadIdx.x), seg = tile_seg(threadIdx.x);
   const int u = u0 + row, i = p.r0 + u;
   const bool valid = u < p.g.rc && i < p.L;
   const int P = p.g.pitch;
@@ -222,14 +231,16 @@ __global__ void __launch_bounds__(kThreadsB) bwd_scores_kernel(StripArgs p) {
         *reinterpret_cast<float4 *>(dst + x) = make_float4(lg[x], lg[x + 1], lg[x + 2], lg[x + 3]);
     }
   }
-  // row statistics over the 16 threads of the row (16 consecutive lanes)
+  // row statistics over the 16 threads of the row (the lanes with the same bit 2)
   float mr[CH], lr[CH];
 #pragma unroll
   for (int h = 0; h < CH; ++h) {
     float mx = m[h];
-    for (int o = 8; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+#pragma unroll
+    for (int o : {1, 2, 8, 16}) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
     float part = m[h] == -INFINITY ? 0.f : l[h] * __expf(m[h] - mx);
-    for (int o = 8; o > 0; o >>= 1) part += __shfl_xor_sync(0xffffffffu, part, o);
+#pragma unroll
+    for (int o : {1, 2, 8, 16}) part += __shfl_xor_sync(0xffffffffu, part, o);
     mr[h] = mx;
     lr[h] = part;
   }
@@ -394,7 +405,7 @@ __global__ void __launch_bounds__(kThreadsB) bwd_adjoint_kernel(StripArgs p) {
   __shared__ __align__(16) float st[TR][kTilePitch];
   __shared__ float th[NT];
   const int z = blockIdx.y, h = z % p.H;
-  const int u0 = blockIdx.x * kRows, row = threadIdx.x >> 4, seg = threadIdx.x & 15;
+  const int u0 = blockIdx.x * kRows, row = tile_row(threadIdx.x), seg = tile_seg(threadIdx.x);
   const int u = u0 + row, i = p.r0 + u;
   const bool own = u < p.g.no && i < p.L;
   const int P = p.g.pitch;
