@@ -98,54 +98,54 @@ constexpr int kSeg = 8;                 // consecutive keys of a thread
 // four of the next, 32 bytes apart along a row -- fall on eight different bank
 // groups.
 constexpr int kTilePitch = 164;
-constexpr int kTileCols = kKeyTile + 16;  // columns staged (128 + 2c used)
+constexpr int kTileCols = kKeyTile + 16;  // columns staged: keys j0 - 8 .. j0 + 135
+constexpr int kStagedRows = kRows + 5;     // rows staged for c_q = 6 (dynamic shared memory)
 // thread -> (row, seg): a warp holds rows 2 warp, 2 warp + 1; lane bit 2 picks
 // the row, the other bits the 8-key segment
 __device__ __forceinline__ int tile_row(int tid) { return 2 * (tid >> 5) + ((tid >> 2) & 1); }
 __device__ __forceinline__ int tile_seg(int tid) { return (tid & 3) | (((tid & 31) >> 3) << 2); }
 
-// Stages TR rows of a strip into tile[TR][kTilePitch]: tile row r holds strip row
-// row0 + r (its query q0 + r; zeros once the strip row reaches nrows or the
-// query reaches L), tile column cc key j0 - C + cc, zero for a key below 0 or
+// Asynchronous 16-byte copy global -> shared of the first src_bytes bytes (0 ..
+// 16), the rest of the 16 zero-filled; src must be a valid address even when
+// src_bytes is 0.
+__device__ __forceinline__ void cp_async16(void *dst, const void *src, int src_bytes) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(smem_u32(dst)), "l"(src), "r"(src_bytes)
+               : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+__device__ __forceinline__ void cp_async_wait_prev() { asm volatile("cp.async.wait_group 1;" ::: "memory"); }
+
+// Starts staging TR rows of a strip into tile[TR][kTilePitch]: tile row r gets
+// strip row row0 + r (its query q0 + r; zeros once the strip row reaches nrows or
+// the query reaches L), tile column cc key j0 - 8 + cc, zero for a key below 0 or
 // past the row's query (Mask_0 and the causal mask of the gradients).  A warp per
-// row, 16-byte loads of keys j0 - 8 + 4 v (aligned, the strip pitch being a
-// multiple of 64), each stored to its four columns.
-template <int TR, int C>
+// row, one 16-byte copy per four keys (aligned: the strip pitch is a multiple of
+// 64); the copy of a group that straddles the row's query takes only its valid
+// leading keys and zero-fills the rest.
+template <int TR>
 __device__ __forceinline__ void stage_rows(float (*tile)[kTilePitch], const float *strip0, int P, int row0,
                                            int nrows, int q0, int L, int j0) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  constexpr int NV = (kTileCols + 8 - C + 3) / 4;  // float4 groups reaching the staged columns
+  constexpr int NV = kTileCols / 4;
   for (int r = warp; r < TR; r += kThreadsB / 32) {
     const int sr = row0 + r, q = q0 + r;
     const bool rv = sr < nrows && q >= 0 && q < L;
-    const float *src = strip0 + static_cast<long long>(sr) * P;
+    const float *src = strip0 + static_cast<long long>(rv ? sr : 0) * P;
     for (int v = lane; v < NV; v += 32) {
       const int k0 = j0 - 8 + 4 * v;
-      float x[4] = {0.f, 0.f, 0.f, 0.f};
-      if (rv && k0 + 3 >= 0 && k0 <= q) {
-        if (k0 >= 0 && k0 + 3 <= q) {
-          const float4 f = *reinterpret_cast<const float4 *>(src + k0);
-          x[0] = f.x; x[1] = f.y; x[2] = f.z; x[3] = f.w;
-        } else {
-#pragma unroll
-          for (int e = 0; e < 4; ++e)
-            if (k0 + e >= 0 && k0 + e <= q) x[e] = src[k0 + e];
-        }
-      }
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const int cc = 4 * v - 8 + C + e;
-        if (cc >= 0 && cc < kTileCols) tile[r][cc] = x[e];
-      }
+      const int n = (rv && k0 >= 0) ? min(4, max(0, q - k0 + 1)) : 0;
+      cp_async16(&tile[r][4 * v], n ? src + k0 : strip0, 4 * n);
     }
   }
 }
 
 template <int CQ, int CK, int CH>
 __global__ void __launch_bounds__(kThreadsB) bwd_scores_kernel(StripArgs p) {
-  constexpr int HALO = CQ - 1, C = CK / 2, TR = kRows + HALO, WIN = kSeg + 2 * C;
-  static_assert(kKeyTile + 2 * C + 4 <= kTileCols && kTileCols <= kTilePitch, "tile columns");
-  __shared__ __align__(16) float tile[CH][TR][kTilePitch];
+  constexpr int HALO = CQ - 1, C = CK / 2, TR = kRows + HALO, WIN = kSeg + 16;
+  static_assert(C <= 8 && kKeyTile + 16 <= kTileCols && kTileCols <= kTilePitch, "tile columns");
+  static_assert(TR == kStagedRows, "dynamic shared memory sized for c_q = 6");
+  extern __shared__ __align__(16) float dyn[];
+  float(*tile)[CH][TR][kTilePitch] = reinterpret_cast<float(*)[CH][TR][kTilePitch]>(dyn);  // [2 stages]
   __shared__ float th[CH][CQ * CK], wm[CH * CH];
   const int G = p.H / CH, bg = blockIdx.y, b = bg / G, g = bg % G;
   const int u0 = blockIdx.x * kRows, row = tile_row(threadIdx.x), seg = tile_seg(threadIdx.x);
@@ -162,15 +162,23 @@ __global__ void __launch_bounds__(kThreadsB) bwd_scores_kernel(StripArgs p) {
 #pragma unroll
   for (int h = 0; h < CH; ++h) { m[h] = -INFINITY; l[h] = 0.f; }
   const int i_last = min(p.L - 1, p.r0 + u0 + kRows - 1);  // the CTA's last query
-  for (int j0 = 0; j0 <= i_last; j0 += kKeyTile) {
-    __syncthreads();
-    // stage Mask_0 S: strip rows u0 .. u0+TR-1 (queries r0 - HALO + su), keys j0-C ..
+  const int ntiles = i_last / kKeyTile + 1;
+  // Mask_0 S: strip rows u0 .. u0+TR-1 (queries r0 - HALO + su), keys j0 - 8 ..
+  auto stage = [&](int tt) {
 #pragma unroll
     for (int hl = 0; hl < CH; ++hl)
-      stage_rows<TR, C>(tile[hl], strip(p.S, hl, kRowsT), P, u0, kRowsT, p.r0 - HALO + u0, p.L, j0);
+      stage_rows<TR>(tile[tt & 1][hl], strip(p.S, hl, kRowsT), P, u0, kRowsT, p.r0 - HALO + u0, p.L, tt * kKeyTile);
+  };
+  stage(0);
+  cp_async_commit();
+  for (int tt = 0; tt < ntiles; ++tt) {
+    const int j0 = tt * kKeyTile;
+    if (tt + 1 < ntiles) stage(tt + 1);  // the next tile's copies run under this tile's arithmetic
+    cp_async_commit();
+    cp_async_wait_prev();
     __syncthreads();
     const int jb = j0 + kSeg * seg;  // first key of the thread
-    if (!valid || jb > i) continue;
+    if (valid && jb <= i) {
     float cv[CH][kSeg];
 #pragma unroll
     for (int h = 0; h < CH; ++h) {
@@ -178,22 +186,19 @@ __global__ void __launch_bounds__(kThreadsB) bwd_scores_kernel(StripArgs p) {
       for (int x = 0; x < kSeg; ++x) cv[h][x] = 0.f;
 #pragma unroll
       for (int a = 0; a < CQ; ++a) {
-        // keys jb - c .. jb + 7 + c of query i - a: tile columns 8 seg .. 8 seg + 7 + 2c
+        // keys jb - 8 .. jb + 15 of query i - a: tile columns 8 seg .. 8 seg + 23
         float w[WIN];
-        const float4 *src = reinterpret_cast<const float4 *>(&tile[h][row + HALO - a][kSeg * seg]);
+        const float4 *src = reinterpret_cast<const float4 *>(&tile[tt & 1][h][row + HALO - a][kSeg * seg]);
 #pragma unroll
-        for (int v4 = 0; v4 < (WIN + 3) / 4; ++v4) {
+        for (int v4 = 0; v4 < WIN / 4; ++v4) {
           const float4 q4 = src[v4];
-          if (4 * v4 + 0 < WIN) w[4 * v4 + 0] = q4.x;
-          if (4 * v4 + 1 < WIN) w[4 * v4 + 1] = q4.y;
-          if (4 * v4 + 2 < WIN) w[4 * v4 + 2] = q4.z;
-          if (4 * v4 + 3 < WIN) w[4 * v4 + 3] = q4.w;
+          w[4 * v4 + 0] = q4.x; w[4 * v4 + 1] = q4.y; w[4 * v4 + 2] = q4.z; w[4 * v4 + 3] = q4.w;
         }
-        // C[i][j] += theta[a][t] S[i-a][j-(t-c)]: key j - t + c = column x + 2c - t
+        // C[i][j] += theta[a][t] S[i-a][j-(t-c)]: key jb + x - t + c = window x + 8 + c - t
 #pragma unroll
         for (int t = 0; t < CK; ++t)
 #pragma unroll
-          for (int x = 0; x < kSeg; ++x) cv[h][x] = fmaf(th[h][a * CK + t], w[x + 2 * C - t], cv[h][x]);
+          for (int x = 0; x < kSeg; ++x) cv[h][x] = fmaf(th[h][a * CK + t], w[x + 8 + C - t], cv[h][x]);
       }
     }
     if (p.hp == 1 && p.Cpre) {
@@ -230,6 +235,8 @@ __global__ void __launch_bounds__(kThreadsB) bwd_scores_kernel(StripArgs p) {
       for (int x = 0; x < kSeg; x += 4)
         *reinterpret_cast<float4 *>(dst + x) = make_float4(lg[x], lg[x + 1], lg[x + 2], lg[x + 3]);
     }
+    }
+    __syncthreads();  // the buffer is restaged two tiles on
   }
   // row statistics over the 16 threads of the row (the lanes with the same bit 2)
   float mr[CH], lr[CH];
@@ -400,9 +407,12 @@ __global__ void __launch_bounds__(kThreadsB) bwd_softmax_grad_kernel(StripArgs p
 // past the CTA's last row only write zeros.
 template <int CQ, int CK>
 __global__ void __launch_bounds__(kThreadsB) bwd_adjoint_kernel(StripArgs p) {
-  constexpr int HALO = CQ - 1, C = CK / 2, TR = kRows + HALO, NT = CQ * CK, WIN = kSeg + 2 * C;
-  __shared__ __align__(16) float dct[TR][kTilePitch];
-  __shared__ __align__(16) float st[TR][kTilePitch];
+  constexpr int HALO = CQ - 1, C = CK / 2, TR = kRows + HALO, NT = CQ * CK, WIN = kSeg + 16;
+  static_assert(C <= 8 && TR == kStagedRows, "window; dynamic shared memory sized for c_q = 6");
+  extern __shared__ __align__(16) float dyn[];
+  // [2 stages]: dC rows and Mask_0 S rows, tile column cc = key j0 - 8 + cc
+  float(*dct)[TR][kTilePitch] = reinterpret_cast<float(*)[TR][kTilePitch]>(dyn);
+  float(*st)[TR][kTilePitch] = reinterpret_cast<float(*)[TR][kTilePitch]>(dyn + 2 * TR * kTilePitch);
   __shared__ float th[NT];
   const int z = blockIdx.y, h = z % p.H;
   const int u0 = blockIdx.x * kRows, row = tile_row(threadIdx.x), seg = tile_seg(threadIdx.x);
@@ -417,15 +427,23 @@ __global__ void __launch_bounds__(kThreadsB) bwd_adjoint_kernel(StripArgs p) {
 #pragma unroll
   for (int x = 0; x < NT; ++x) dth[x] = 0.f;
   const int i_last = min(p.L - 1, p.r0 + min(u0 + kRows - 1, p.g.no - 1));  // last own query of the CTA
-  for (int j0 = 0; j0 < p.Wp; j0 += kKeyTile) {
+  // key tiles with work (uniform over the CTA); the later ones only write zeros
+  const int nwork = u0 < p.g.no ? i_last / kKeyTile + 1 : 0;
+  auto stage = [&](int tt) {
+    // dC rows u0 .. u0+TR-1 (queries r0 + u'), zero past the C rows, the sequence and the diagonal
+    stage_rows<TR>(dct[tt & 1], Dz, P, u0, p.g.rc, p.r0 + u0, p.L, tt * kKeyTile);
+    // Mask_0 S rows u0 .. u0+TR-1 of the S strip (queries r0 - HALO + su)
+    stage_rows<TR>(st[tt & 1], Sz, P, u0, kRowsT, p.r0 - HALO + u0, p.L, tt * kKeyTile);
+  };
+  if (nwork) stage(0);
+  cp_async_commit();
+  for (int j0 = 0, tt = 0; j0 < p.Wp; j0 += kKeyTile, ++tt) {
     const int jb = j0 + kSeg * seg;
-    const bool work = j0 <= i_last && u0 < p.g.no;  // uniform over the CTA
+    const bool work = tt < nwork;
     if (work) {
-      __syncthreads();
-      // dC rows u0 .. u0+TR-1 (queries r0 + u'), zero past the C rows, the sequence and the diagonal
-      stage_rows<TR, C>(dct, Dz, P, u0, p.g.rc, p.r0 + u0, p.L, j0);
-      // Mask_0 S rows u0 .. u0+TR-1 of the S strip (queries r0 - HALO + su)
-      stage_rows<TR, C>(st, Sz, P, u0, kRowsT, p.r0 - HALO + u0, p.L, j0);
+      if (tt + 1 < nwork) stage(tt + 1);
+      cp_async_commit();
+      cp_async_wait_prev();
       __syncthreads();
     }
     float ds[kSeg];
@@ -433,32 +451,32 @@ __global__ void __launch_bounds__(kThreadsB) bwd_adjoint_kernel(StripArgs p) {
     for (int x = 0; x < kSeg; ++x) ds[x] = 0.f;
     if (work && own && jb <= i && jb < p.Wp) {
       // dC[i][j] of the thread's keys (zero past the diagonal) for dtheta
+      const int bf = tt & 1;
       float gk[kSeg];
 #pragma unroll
-      for (int x = 0; x < kSeg; ++x) gk[x] = dct[row][kSeg * seg + C + x];
+      for (int x = 0; x < kSeg; ++x) gk[x] = dct[bf][row][kSeg * seg + 8 + x];
 #pragma unroll
       for (int a = 0; a < CQ; ++a) {
+        // tile columns 8 seg .. 8 seg + 23: keys jb - 8 .. jb + 15
         float w[WIN], v[WIN];
-        const float4 *sd = reinterpret_cast<const float4 *>(&dct[row + a][kSeg * seg]);
-        const float4 *ss = reinterpret_cast<const float4 *>(&st[row + HALO - a][kSeg * seg]);
+        const float4 *sd = reinterpret_cast<const float4 *>(&dct[bf][row + a][kSeg * seg]);
+        const float4 *ss = reinterpret_cast<const float4 *>(&st[bf][row + HALO - a][kSeg * seg]);
 #pragma unroll
-        for (int v4 = 0; v4 < (WIN + 3) / 4; ++v4) {
+        for (int v4 = 0; v4 < WIN / 4; ++v4) {
           const float4 q4 = sd[v4], s4 = ss[v4];
-          if (4 * v4 + 0 < WIN) { w[4 * v4 + 0] = q4.x; v[4 * v4 + 0] = s4.x; }
-          if (4 * v4 + 1 < WIN) { w[4 * v4 + 1] = q4.y; v[4 * v4 + 1] = s4.y; }
-          if (4 * v4 + 2 < WIN) { w[4 * v4 + 2] = q4.z; v[4 * v4 + 2] = s4.z; }
-          if (4 * v4 + 3 < WIN) { w[4 * v4 + 3] = q4.w; v[4 * v4 + 3] = s4.w; }
+          w[4 * v4 + 0] = q4.x; w[4 * v4 + 1] = q4.y; w[4 * v4 + 2] = q4.z; w[4 * v4 + 3] = q4.w;
+          v[4 * v4 + 0] = s4.x; v[4 * v4 + 1] = s4.y; v[4 * v4 + 2] = s4.z; v[4 * v4 + 3] = s4.w;
         }
 #pragma unroll
         for (int t = 0; t < CK; ++t) {
-          const float tt = th[a * CK + t];
+          const float th_at = th[a * CK + t];
           float acc = dth[a * CK + t];
 #pragma unroll
           for (int x = 0; x < kSeg; ++x) {
-            // dS[i][j] += theta[a][t] dC[i+a][j+t-c]: column x + t
-            ds[x] = fmaf(tt, w[x + t], ds[x]);
-            // dtheta[a][t] += dC[i][j] Mask_0 S[i-a][j-(t-c)]: column x + 2c - t
-            acc = fmaf(gk[x], v[x + 2 * C - t], acc);
+            // dS[i][j] += theta[a][t] dC[i+a][j+t-c]: key jb + x + t - c = window x + 8 + t - c
+            ds[x] = fmaf(th_at, w[x + 8 + t - C], ds[x]);
+            // dtheta[a][t] += dC[i][j] Mask_0 S[i-a][j-(t-c)]: window x + 8 + c - t
+            acc = fmaf(gk[x], v[x + 8 + C - t], acc);
           }
           dth[a * CK + t] = acc;
         }
@@ -480,6 +498,7 @@ __global__ void __launch_bounds__(kThreadsB) bwd_adjoint_kernel(StripArgs p) {
       *reinterpret_cast<uint4 *>(dSz + static_cast<long long>(kRowsT + u) * P + jb) =
           make_uint4(lo[0], lo[1], lo[2], lo[3]);
     }
+    if (work) __syncthreads();  // the buffer is restaged two tiles on
   }
   if (p.dtheta) {
 #pragma unroll
@@ -490,6 +509,9 @@ __global__ void __launch_bounds__(kThreadsB) bwd_adjoint_kernel(StripArgs p) {
     }
   }
 }
+
+int scores_smem(int ch) { return 2 * ch * kStagedRows * kTilePitch * 4; }
+int adjoint_smem() { return 2 * 2 * kStagedRows * kTilePitch * 4; }
 
 Geo geometry(const BwdArgs &a) {
   Geo g;
@@ -566,6 +588,13 @@ cudaError_t launch_attn_bwd_tc(const BwdArgs &a, void *ws) {
   cudaStream_t st = a.stream;
   const size_t n = static_cast<size_t>(a.B) * a.L * a.H * a.d;
   cudaError_t e;
+  if ((e = cudaFuncSetAttribute(bwd_scores_kernel<6, 11, 2>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                scores_smem(2))) != cudaSuccess ||
+      (e = cudaFuncSetAttribute(bwd_scores_kernel<6, 11, 1>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                scores_smem(1))) != cudaSuccess ||
+      (e = cudaFuncSetAttribute(bwd_adjoint_kernel<6, 11>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                adjoint_smem())) != cudaSuccess)
+    return e;
   if ((e = cudaMemsetAsync(a.dk, 0, n * 4, st)) != cudaSuccess) return e;
   if ((e = cudaMemsetAsync(a.dv, 0, n * 4, st)) != cudaSuccess) return e;
   if (a.dtheta && (e = cudaMemsetAsync(a.dtheta, 0, static_cast<size_t>(a.H) * a.cq * a.ck * 4, st)) != cudaSuccess)
@@ -607,9 +636,9 @@ cudaError_t launch_attn_bwd_tc(const BwdArgs &a, void *ws) {
     // 2. convolution, mixing, softmax -> A
     const dim3 grid2((g.rc + kRows - 1) / kRows, a.B * G);
     if (ch == 2)
-      bwd_scores_kernel<6, 11, 2><<<grid2, kThreadsB, 0, st>>>(sp);
+      bwd_scores_kernel<6, 11, 2><<<grid2, kThreadsB, scores_smem(2), st>>>(sp);
     else
-      bwd_scores_kernel<6, 11, 1><<<grid2, kThreadsB, 0, st>>>(sp);
+      bwd_scores_kernel<6, 11, 1><<<grid2, kThreadsB, scores_smem(1), st>>>(sp);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     // 3. dA'' strip = dO V^T: rows r0 .. r0 + rc - 1
     ga.M = g.rc; ga.alpha = 1.f;
@@ -624,7 +653,7 @@ cudaError_t launch_attn_bwd_tc(const BwdArgs &a, void *ws) {
       bwd_softmax_grad_kernel<1><<<grid4, kThreadsB, 0, st>>>(sp);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     // 5. dS (hi / lo), dtheta
-    bwd_adjoint_kernel<6, 11><<<dim3(kRowsT / kRows, static_cast<unsigned>(Z)), kThreadsB, 0, st>>>(sp);
+    bwd_adjoint_kernel<6, 11><<<dim3(kRowsT / kRows, static_cast<unsigned>(Z)), kThreadsB, adjoint_smem(), st>>>(sp);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     // 6. dQ rows r0 .. r0 + no - 1 = s dS K: K runs over the keys twice, the hi
     //    rows of dS against K, then its lo rows (256 further) against K again
