@@ -25,11 +25,10 @@
 // statistics and D come from the strip itself (no statistics pass).  The strips
 // are O(B H 256 L): never an L x L map.  Per block:
 //   1. S strip      = s Q K^T                      batched GEMM (fp32 out)
-//   2. C, softmax   -> A strip                     bwd_scores_kernel (CUDA cores)
-//   3. dA'' strip   = dO V^T                       batched GEMM
-//   4. dC, D, dw, A''                              bwd_softmax_grad_kernel
-//   5. dS, dtheta                                  bwd_adjoint_kernel
-//   6. dQ rows (=), dK, dV (+=)                    batched GEMMs
+//   2. dA'' strip   = dO V^T                       batched GEMM
+//   3. C, softmax, then dC, D, dw, A''             bwd_scores_kernel (CUDA cores)
+//   4. dS, dtheta                                  bwd_adjoint_kernel
+//   5. dQ rows (=), dK, dV (+=)                    batched GEMMs
 // dS and A'' enter the GEMMs of step 6 as two bf16 halves, hi = bf16(x) and
 // lo = bf16(x - hi), summed by two GEMMs into the same fp32 output: the operands
 // then carry about 16 significant bits and the gradients stay within fp32
@@ -49,7 +48,6 @@ namespace {
 constexpr int kRowsT = 256;  // rows of the S strip (and of the halves of the dS / A'' strips)
 constexpr int kKeyTile = 128;
 constexpr int kThreadsB = 256;
-constexpr int kRowsPerCta = 4;  // rows of a CTA in the softmax-gradient kernel: 4 x 64 threads
 
 struct Geo {
   int halo, c, no, rc, pitch;  // c_q - 1, c_k / 2, own rows, C rows, strip pitch (elements)
@@ -70,23 +68,16 @@ struct StripArgs {
   float *dtheta, *dw;
 };
 
-__device__ __forceinline__ float blocksum64(float v, float *red, int row, int sub) {
-  // sum over the 64 threads (two warps) of one row
-  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-  if ((sub & 31) == 0) red[2 * row + (sub >> 5)] = v;
-  __syncthreads();
-  const float s = red[2 * row] + red[2 * row + 1];
-  __syncthreads();
-  return s;
-}
-
 __device__ __forceinline__ void split_bf16(float x, __nv_bfloat16 &hi, __nv_bfloat16 &lo) {
   hi = __float2bfloat16_rn(x);
   lo = __float2bfloat16_rn(x - __bfloat162float(hi));
 }
 
-// Step 2: C = Conv2d_theta(Mask_0 S) for the block's C rows (and pre mixing),
-// Mask_-inf, softmax over the row -> A strip.  CTA: one head group, 16 rows;
+// Step 3: C = Conv2d_theta(Mask_0 S) for the block's C rows (and pre mixing),
+// Mask_-inf, the softmax statistics of each row (its logits kept in the A strip),
+// then the softmax's backward on the same rows: dA (post mixing: mixed back to
+// the sources), D, dC = A (dA - D) (pre mixing: then mixed back) into the dA''
+// strip, dw, and A'' (hi / lo) of the block's own rows.  CTA: one head group, 16 rows;
 // thread (row, seg): 8 consecutive keys 8 seg .. 8 seg + 7 of every 128-key tile.
 // For each tap row a the thread loads the 8 + 2c values of the staged S row it
 // needs once and forms its 8 outputs x c_k taps from registers.  Key tiles past
@@ -251,144 +242,165 @@ __global__ void __launch_bounds__(kThreadsB) bwd_scores_kernel(StripArgs p) {
     mr[h] = mx;
     lr[h] = part;
   }
-  if (!valid) return;
-  for (int jb = kSeg * seg; jb <= i; jb += kKeyTile) {
+  // ---- the softmax's backward on the same rows: the weights A_s = exp(C - m) / l
+  // are recomputed from the logits wherever they are needed, never stored
+  float inv[CH];
 #pragma unroll
-    for (int h = 0; h < CH; ++h) {
-      float *a = strip(p.A, h, p.g.rc) + u * P + jb;
-      const float inv = 1.f / lr[h];
+  for (int h = 0; h < CH; ++h) inv[h] = 1.f / lr[h];
+  auto weights = [&](int jb, int h, float (&a)[kSeg]) {
+    const float *lg = strip(p.A, h, p.g.rc) + u * P + jb;
 #pragma unroll
-      for (int x = 0; x < kSeg; x += 4) {
-        float4 v = *reinterpret_cast<float4 *>(a + x);
-        v.x = jb + x + 0 <= i ? __expf(v.x - mr[h]) * inv : 0.f;
-        v.y = jb + x + 1 <= i ? __expf(v.y - mr[h]) * inv : 0.f;
-        v.z = jb + x + 2 <= i ? __expf(v.z - mr[h]) * inv : 0.f;
-        v.w = jb + x + 3 <= i ? __expf(v.w - mr[h]) * inv : 0.f;
-        *reinterpret_cast<float4 *>(a + x) = v;
-      }
+    for (int x = 0; x < kSeg; x += 4) {
+      const float4 v = *reinterpret_cast<const float4 *>(lg + x);
+      a[x + 0] = jb + x + 0 <= i ? __expf(v.x - mr[h]) * inv[h] : 0.f;
+      a[x + 1] = jb + x + 1 <= i ? __expf(v.y - mr[h]) * inv[h] : 0.f;
+      a[x + 2] = jb + x + 2 <= i ? __expf(v.z - mr[h]) * inv[h] : 0.f;
+      a[x + 3] = jb + x + 3 <= i ? __expf(v.w - mr[h]) * inv[h] : 0.f;
     }
-  }
-}
-
-// Step 4: dA (post mixing: mixed back to the sources), D, dC = A (dA - D) (pre
-// mixing: then mixed back), dw, and A'' (hi / lo) of the block's own rows.  Rows
-// u = 0 .. 127: rows past the C rows only clear their A'' halves.
-template <int CH>
-__global__ void __launch_bounds__(kThreadsB) bwd_softmax_grad_kernel(StripArgs p) {
-  __shared__ float wm[CH * CH];
-  __shared__ float red[2 * kRowsPerCta];
-  __shared__ float dwr[CH * CH];
-  const int G = p.H / CH, bg = blockIdx.y, b = bg / G, g = bg % G;
-  const int u = blockIdx.x * kRowsPerCta + (threadIdx.x >> 6), row = threadIdx.x >> 6, sub = threadIdx.x & 63;
-  const int i = p.r0 + u;
-  const bool valid = u < p.g.rc && i < p.L;
-  const bool own = u < p.g.no && i < p.L;
-  const int P = p.g.pitch;
-  for (int x = threadIdx.x; x < CH * CH; x += kThreadsB) {
-    wm[x] = p.w ? p.w[g * CH * CH + x] : (x % (CH + 1) == 0);
-    dwr[x] = 0.f;
-  }
-  __syncthreads();
-  auto strip = [&](auto *base, int hl, int rows) {
-    return base + ((static_cast<long long>(b) * p.H + g * CH + hl) * rows) * P;
   };
-  // pass 1: D_s (post / none: dA_s = sum_h w[h][s] dA''_h; pre: dA'_h = dA''_h)
+  auto grads = [&](int jb, int h, float (&da)[kSeg]) {  // dA'' from the GEMM
+    const float *src = strip(p.D, h, p.g.rc) + u * P + jb;
+#pragma unroll
+    for (int x = 0; x < kSeg; x += 4) {
+      const float4 v = *reinterpret_cast<const float4 *>(src + x);
+      da[x + 0] = jb + x + 0 <= i ? v.x : 0.f;
+      da[x + 1] = jb + x + 1 <= i ? v.y : 0.f;
+      da[x + 2] = jb + x + 2 <= i ? v.z : 0.f;
+      da[x + 3] = jb + x + 3 <= i ? v.w : 0.f;
+    }
+  };
+  const bool own = valid && u < p.g.no;
   float Dp[CH], dwp[CH * CH];
 #pragma unroll
   for (int h = 0; h < CH; ++h) Dp[h] = 0.f;
 #pragma unroll
   for (int x = 0; x < CH * CH; ++x) dwp[x] = 0.f;
+  // pass 2: D_s = sum_j dA_s A_s (post mixing: dA_s = sum_h w[h][s] dA''_h; pre or
+  // none: dA'_h = dA''_h), and the post-mixing dw = sum dA''_h A_s
   if (valid) {
-    for (int j = sub; j <= i && j < p.W; j += 64) {
-      float a[CH], da[CH];
+    for (int jb = kSeg * seg; jb <= i; jb += kKeyTile) {
+      float a[CH][kSeg], da[CH][kSeg];
 #pragma unroll
-      for (int h = 0; h < CH; ++h) {
-        a[h] = strip(p.A, h, p.g.rc)[u * P + j];
-        da[h] = strip(p.D, h, p.g.rc)[u * P + j];
-      }
+      for (int h = 0; h < CH; ++h) { weights(jb, h, a[h]); grads(jb, h, da[h]); }
 #pragma unroll
-      for (int s = 0; s < CH; ++s) {
-        float d = da[s];
-        if (p.hp == 2) {
-          d = 0.f;
+      for (int s2 = 0; s2 < CH; ++s2)
 #pragma unroll
-          for (int h = 0; h < CH; ++h) d = fmaf(wm[h * CH + s], da[h], d);
+        for (int x = 0; x < kSeg; ++x) {
+          float d = da[s2][x];
+          if (p.hp == 2) {
+            d = 0.f;
+#pragma unroll
+            for (int h = 0; h < CH; ++h) d = fmaf(wm[h * CH + s2], da[h][x], d);
+          }
+          Dp[s2] = fmaf(d, a[s2][x], Dp[s2]);
         }
-        Dp[s] = fmaf(d, a[s], Dp[s]);
-      }
       if (p.hp == 2 && own) {
 #pragma unroll
         for (int h = 0; h < CH; ++h)
 #pragma unroll
-          for (int s = 0; s < CH; ++s) dwp[h * CH + s] = fmaf(da[h], a[s], dwp[h * CH + s]);
+          for (int s2 = 0; s2 < CH; ++s2)
+#pragma unroll
+            for (int x = 0; x < kSeg; ++x) dwp[h * CH + s2] = fmaf(da[h][x], a[s2][x], dwp[h * CH + s2]);
       }
     }
   }
   float Dr[CH];
 #pragma unroll
-  for (int h = 0; h < CH; ++h) Dr[h] = blocksum64(Dp[h], red, row, sub);
-  // pass 2: dC (into the dA'' strip), pre-mixing dw, A'' halves
-  for (int j = sub; j < p.Wp; j += 64) {
-    const bool in = valid && j <= i;
-    float a[CH], da[CH], dc[CH];
+  for (int h = 0; h < CH; ++h) {
+    float v = Dp[h];
 #pragma unroll
-    for (int h = 0; h < CH; ++h) {
-      a[h] = in ? strip(p.A, h, p.g.rc)[u * P + j] : 0.f;
-      da[h] = in ? strip(p.D, h, p.g.rc)[u * P + j] : 0.f;
-    }
-    if (p.hp == 1) {
-      float dcp[CH];  // dC'_h = A_h (dA''_h - D_h), then mixed back to the sources
+    for (int o : {1, 2, 8, 16}) v += __shfl_xor_sync(0xffffffffu, v, o);
+    Dr[h] = v;
+  }
+  // pass 3: dC = A (dA - D) into the dA'' strip (pre mixing: dC'_h, then mixed
+  // back, with dw = sum dC'_h C_s); A'' (hi / lo) of the own rows
+  if (valid) {
+    for (int jb = kSeg * seg; jb <= i; jb += kKeyTile) {
+      float a[CH][kSeg], da[CH][kSeg], dc[CH][kSeg];
 #pragma unroll
-      for (int h = 0; h < CH; ++h) dcp[h] = a[h] * (da[h] - Dr[h]);
+      for (int h = 0; h < CH; ++h) { weights(jb, h, a[h]); grads(jb, h, da[h]); }
+      if (p.hp == 1) {
 #pragma unroll
-      for (int s = 0; s < CH; ++s) {
-        float x = 0.f;
+        for (int x = 0; x < kSeg; ++x) {
+          float dcp[CH];
 #pragma unroll
-        for (int h = 0; h < CH; ++h) x = fmaf(wm[h * CH + s], dcp[h], x);
-        dc[s] = x;
-      }
-      if (in && own) {
-        float cs[CH];
+          for (int h = 0; h < CH; ++h) dcp[h] = a[h][x] * (da[h][x] - Dr[h]);
 #pragma unroll
-        for (int s = 0; s < CH; ++s) cs[s] = strip(p.Cpre, s, p.g.rc)[u * P + j];
+          for (int s2 = 0; s2 < CH; ++s2) {
+            float v = 0.f;
 #pragma unroll
-        for (int h = 0; h < CH; ++h)
+            for (int h = 0; h < CH; ++h) v = fmaf(wm[h * CH + s2], dcp[h], v);
+            dc[s2][x] = v;
+          }
+          if (own && jb + x <= i) {
 #pragma unroll
-          for (int s = 0; s < CH; ++s) dwp[h * CH + s] = fmaf(dcp[h], cs[s], dwp[h * CH + s]);
-      }
-    } else {
+            for (int s2 = 0; s2 < CH; ++s2) {
+              const float cs = strip(p.Cpre, s2, p.g.rc)[u * P + jb + x];
 #pragma unroll
-      for (int s = 0; s < CH; ++s) {
-        float d = da[s];
-        if (p.hp == 2) {
-          d = 0.f;
-#pragma unroll
-          for (int h = 0; h < CH; ++h) d = fmaf(wm[h * CH + s], da[h], d);
+              for (int h = 0; h < CH; ++h) dwp[h * CH + s2] = fmaf(dcp[h], cs, dwp[h * CH + s2]);
+            }
+          }
         }
-        dc[s] = a[s] * (d - Dr[s]);
+      } else {
+#pragma unroll
+        for (int s2 = 0; s2 < CH; ++s2)
+#pragma unroll
+          for (int x = 0; x < kSeg; ++x) {
+            float d = da[s2][x];
+            if (p.hp == 2) {
+              d = 0.f;
+#pragma unroll
+              for (int h = 0; h < CH; ++h) d = fmaf(wm[h * CH + s2], da[h][x], d);
+            }
+            dc[s2][x] = a[s2][x] * (d - Dr[s2]);
+          }
       }
-    }
-    if (u < p.g.rc) {
 #pragma unroll
-      for (int s = 0; s < CH; ++s) strip(p.D, s, p.g.rc)[u * P + j] = in ? dc[s] : 0.f;
-    }
-    // A''_h = sum_s w[h][s] A_s (post mixing), else A_h; own rows only
+      for (int s2 = 0; s2 < CH; ++s2) {
+        float *dst = strip(p.D, s2, p.g.rc) + u * P + jb;
 #pragma unroll
-    for (int h = 0; h < CH; ++h) {
-      float x = a[h];
-      if (p.hp == 2) {
-        x = 0.f;
-#pragma unroll
-        for (int s = 0; s < CH; ++s) x = fmaf(wm[h * CH + s], a[s], x);
+        for (int x = 0; x < kSeg; x += 4)
+          *reinterpret_cast<float4 *>(dst + x) = make_float4(dc[s2][x], dc[s2][x + 1], dc[s2][x + 2], dc[s2][x + 3]);
       }
-      __nv_bfloat16 hi, lo;
-      split_bf16(own && in ? x : 0.f, hi, lo);
-      __nv_bfloat16 *ap = strip(p.Ap, h, 2 * kRowsT);
-      ap[u * P + j] = hi;
-      ap[(kRowsT + u) * P + j] = lo;
+      if (own) {
+        // A''_h = sum_s w[h][s] A_s (post mixing), else A_h
+#pragma unroll
+        for (int h = 0; h < CH; ++h) {
+          uint32_t hi[kSeg / 2], lo[kSeg / 2];
+#pragma unroll
+          for (int x = 0; x < kSeg; x += 2) {
+            float y[2];
+#pragma unroll
+            for (int e = 0; e < 2; ++e) {
+              float v = a[h][x + e];
+              if (p.hp == 2) {
+                v = 0.f;
+#pragma unroll
+                for (int s2 = 0; s2 < CH; ++s2) v = fmaf(wm[h * CH + s2], a[s2][x + e], v);
+              }
+              y[e] = v;
+            }
+            __nv_bfloat16 h0, l0, h1, l1;
+            split_bf16(y[0], h0, l0);
+            split_bf16(y[1], h1, l1);
+            hi[x / 2] = static_cast<uint32_t>(__bfloat16_as_ushort(h0)) |
+                        (static_cast<uint32_t>(__bfloat16_as_ushort(h1)) << 16);
+            lo[x / 2] = static_cast<uint32_t>(__bfloat16_as_ushort(l0)) |
+                        (static_cast<uint32_t>(__bfloat16_as_ushort(l1)) << 16);
+          }
+          __nv_bfloat16 *ap = reinterpret_cast<__nv_bfloat16 *>(
+              p.Ap + ((static_cast<long long>(b) * p.H + g * CH + h) * 2 * kRowsT) * P);
+          *reinterpret_cast<uint4 *>(ap + static_cast<long long>(u) * P + jb) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
+          *reinterpret_cast<uint4 *>(ap + static_cast<long long>(kRowsT + u) * P + jb) =
+              make_uint4(lo[0], lo[1], lo[2], lo[3]);
+        }
+      }
     }
   }
   if (p.hp != 0 && p.dw) {
+    __shared__ float dwr[CH * CH];
+    if (threadIdx.x < CH * CH) dwr[threadIdx.x] = 0.f;
+    __syncthreads();
 #pragma unroll
     for (int x = 0; x < CH * CH; ++x) {
       float v = dwp[x];
@@ -400,7 +412,7 @@ __global__ void __launch_bounds__(kThreadsB) bwd_softmax_grad_kernel(StripArgs p
   }
 }
 
-// Step 5: dS = [j <= i] sum theta[a][t] dC[i+a][j+t-c] (hi / lo halves) for the
+// Step 4: dS = [j <= i] sum theta[a][t] dC[i+a][j+t-c] (hi / lo halves) for the
 // block's own rows, zeros elsewhere, and dtheta over the own rows.  CTA: one
 // head, 16 rows u = 0 .. 127; thread (row, seg): 8 consecutive keys, register
 // windows of 8 + 2c staged values per tap row as in the scores kernel.  Key tiles
@@ -601,6 +613,8 @@ cudaError_t launch_attn_bwd_tc(const BwdArgs &a, void *ws) {
     return e;
   if (a.hp && a.dw && (e = cudaMemsetAsync(a.dw, 0, static_cast<size_t>(a.H) * a.ch * 4, st)) != cudaSuccess)
     return e;
+  // A'' is written for the own rows up to each row's query only: the rest stays zero
+  if ((e = cudaMemsetAsync(Ap, 0, Z * 2 * kRowsT * P * 2, st)) != cudaSuccess) return e;
 
   const BgTensor tq = qkv_tensor(a.q, a, a.rs), tk = qkv_tensor(a.k, a, a.rs), tv = qkv_tensor(a.v, a, a.rs);
   const BgTensor tdo = qkv_tensor(a.dout, a, static_cast<long long>(a.H) * a.d);
@@ -626,36 +640,29 @@ cudaError_t launch_attn_bwd_tc(const BwdArgs &a, void *ws) {
   for (int r0 = 0; r0 < a.L; r0 += g.no) {
     const int W = std::min(a.L, r0 + g.rc), Wp = (W + 63) / 64 * 64;
     sp.r0 = r0; sp.W = W; sp.Wp = Wp;
-    // 1. S strip = s Q K^T: rows r0 - halo .. r0 - halo + 127, keys 0 .. W-1
+    // 1. S strip = s Q K^T: rows r0 - halo .. r0 - halo + 255, keys 0 .. W-1
     BgArgs ga = {};
     ga.Z = static_cast<int>(Z); ga.H = a.H; ga.err = err;
     ga.M = kRowsT; ga.N = W; ga.K = a.d; ga.alpha = a.scale; ga.accumulate = 0;
     ga.C = S; ga.sm = g.pitch; ga.sh = static_cast<long long>(kRowsT) * g.pitch; ga.sb = ga.sh * a.H;
     ga.a = K_major(2, r0 - g.halo, 0); ga.b = K_major(2, 0, 0);
     if ((e = launch_gemm_batched(tq, tk, ga, st)) != cudaSuccess) return e;
-    // 2. convolution, mixing, softmax -> A
+    // 2. dA'' strip = dO V^T: rows r0 .. r0 + rc - 1
+    ga.M = g.rc; ga.alpha = 1.f;
+    ga.C = D; ga.sh = static_cast<long long>(g.rc) * g.pitch; ga.sb = ga.sh * a.H;
+    ga.a = K_major(2, r0, 0); ga.b = K_major(2, 0, 0);
+    if ((e = launch_gemm_batched(tdo, tv, ga, st)) != cudaSuccess) return e;
+    // 3. convolution, mixing, softmax; dC, D, dw, A''
     const dim3 grid2((g.rc + kRows - 1) / kRows, a.B * G);
     if (ch == 2)
       bwd_scores_kernel<6, 11, 2><<<grid2, kThreadsB, scores_smem(2), st>>>(sp);
     else
       bwd_scores_kernel<6, 11, 1><<<grid2, kThreadsB, scores_smem(1), st>>>(sp);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
-    // 3. dA'' strip = dO V^T: rows r0 .. r0 + rc - 1
-    ga.M = g.rc; ga.alpha = 1.f;
-    ga.C = D; ga.sh = static_cast<long long>(g.rc) * g.pitch; ga.sb = ga.sh * a.H;
-    ga.a = K_major(2, r0, 0); ga.b = K_major(2, 0, 0);
-    if ((e = launch_gemm_batched(tdo, tv, ga, st)) != cudaSuccess) return e;
-    // 4. dC, D, dw, A''
-    const dim3 grid4(kRowsT / kRowsPerCta, a.B * G);
-    if (ch == 2)
-      bwd_softmax_grad_kernel<2><<<grid4, kThreadsB, 0, st>>>(sp);
-    else
-      bwd_softmax_grad_kernel<1><<<grid4, kThreadsB, 0, st>>>(sp);
-    if ((e = cudaGetLastError()) != cudaSuccess) return e;
-    // 5. dS (hi / lo), dtheta
+    // 4. dS (hi / lo), dtheta
     bwd_adjoint_kernel<6, 11><<<dim3(kRowsT / kRows, static_cast<unsigned>(Z)), kThreadsB, adjoint_smem(), st>>>(sp);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
-    // 6. dQ rows r0 .. r0 + no - 1 = s dS K: K runs over the keys twice, the hi
+    // 5. dQ rows r0 .. r0 + no - 1 = s dS K: K runs over the keys twice, the hi
     //    rows of dS against K, then its lo rows (256 further) against K again
     const int own = std::min(g.no, a.L - r0);
     BgArgs gq = {};
