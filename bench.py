@@ -100,6 +100,33 @@ def uses_direct_tc(wl: synth.Workload) -> bool:
             and (wl.kq_place == synth.OFF or (wl.c_q, wl.c_k) == (6, 11)))
 
 
+def uses_bwd_tc(wl: synth.Workload) -> bool:
+    """Whether the default backward runs on the tensor cores (attn_bwd_tc.cu)."""
+    return (wl.dtype == "bf16" and wl.d in (64, 128) and wl.kq_place == synth.PRE
+            and (wl.c_q, wl.c_k) == (6, 11) and not wl.kq_post
+            and (wl.head_place == synth.OFF or wl.c_h == 2))
+
+
+def bwd_tc_launches(wl: synth.Workload) -> int:
+    """Kernels of the tensor-core backward per call: per query block of 256 - 2 (c_q - 1)
+    rows the S and dA'' GEMMs, the convolution / softmax kernel, the adjoint kernel and
+    the dQ, dK and dV GEMMs."""
+    return 7 * -(-wl.L // (256 - 2 * (wl.c_q - 1)))
+
+
+def bwd_tc_gemm_flops(wl: synth.Workload) -> float:
+    """Tensor flops the tensor-core backward's GEMMs execute per call (bf16 MMAs):
+    per query block of NO rows (strips of 256 rows) and keys 0 .. W-1, for every
+    head: S (256 x W x d), dA'' (251 x W x d), dQ (NO x d x 2W: hi and lo halves),
+    dK and dV (W x d x 512)."""
+    no = 256 - 2 * (wl.c_q - 1)
+    f = 0.0
+    for r0 in range(0, wl.L, no):
+        W = min(wl.L, r0 + no + wl.c_q - 1)
+        f += 2 * (256 + (no + wl.c_q - 1)) * W * wl.d + 2 * no * wl.d * 2 * W + 2 * 2 * W * wl.d * 512
+    return f * wl.B * wl.H
+
+
 def launches_per_step(wl: synth.Workload) -> int:
     """Kernels of this library one step launches: the attention kernel (and the
     prepass of the contraction kernel); a layer adds the two projection GEMMs,
@@ -317,7 +344,8 @@ def step_fn(wl, mta, sets, ws, outs, stream, bwd=False):
 def step_kernels(wl: synth.Workload, bwd: bool) -> list[str]:
     """Names of the library's kernels one step launches, in launch order (the
     library records a timing event after each; see mta_cfg.events)."""
-    bwd_kernel = "attn_bwd_post_kernel" if wl.kq_post else "attn_bwd_simt_kernel"
+    bwd_kernel = ("attn_bwd_tc" if uses_bwd_tc(wl) else
+                  "attn_bwd_post_kernel" if wl.kq_post else "attn_bwd_simt_kernel")
     if bwd and wl.layer:
         return (["gemm_qkv"] + [k for k in step_kernels(wl, False)[1:-1] if k != "group_norm_kernel"] +
                 ["gemm_dy", "group_norm_bwd_kernel", "gemm_dwo", bwd_kernel, "pack_qkv_grad_kernel",
@@ -339,7 +367,7 @@ def dominant_kernel(wl: synth.Workload, bwd: bool) -> tuple[int, int, str]:
     k-th; see mta_cfg.events), and its name."""
     if bwd:
         names = step_kernels(wl, True)
-        i = names.index("attn_bwd_post_kernel" if wl.kq_post else "attn_bwd_simt_kernel")
+        i = next(k for k, n in enumerate(names) if n.startswith("attn_bwd"))
         return i, i + 1, names[i]
     n = launches_per_step(wl) + 1
     if uses_contraction(wl):
@@ -774,7 +802,23 @@ def main():
     fp32_src = "148 SMs x 128 FP32 lanes x 2 x 1965 MHz"
     timing = (f"achieved = per_unit x units / {kernel}'s mean duration over the {args.steps} timed "
               f"steps (CUDA events the library records around it on the launch stream)")
-    if args.bwd:
+    if args.bwd and uses_bwd_tc(wl):
+        # the tensor-core backward: its CUDA-core kernels take most of its time; their
+        # algorithmic work is the convolution recomputed, its adjoint and the kernel
+        # gradient, 3 x 2 c_q c_k fp32 flop per causal pair-head.  The time is the whole
+        # backward's (its GEMMs included), so the fraction is a lower bound.
+        f_cc = 6 * wl.c_q * wl.c_k * wl.causal_pairs
+        achieved = f_cc / ks / 1e12
+        roof = {"bound": "alu", "achieved": achieved, "peak": FP32_PEAK_TFLOPS, "unit": "TFLOP/s",
+                "frac": achieved / FP32_PEAK_TFLOPS, "traffic": None,
+                "kernel": kernel, "kernel_ms": ks * 1e3,
+                "per_unit": f"F_cc = 6 c_q c_k = {6 * wl.c_q * wl.c_k} fp32 flop per causal pair-head "
+                            f"(convolution, adjoint, kernel gradient on the CUDA cores), x {wl.causal_pairs} "
+                            f"pair-heads per call; the time is the whole backward's, its "
+                            f"{bwd_tc_launches(wl)} kernels (GEMMs included)",
+                "peak_source": fp32_src, "timing": timing,
+                "tensor_gemm_tflops": bwd_tc_gemm_flops(wl) / ks / 1e12}
+    elif args.bwd:
         # the backward on the CUDA cores: F_bwd = 8d + 4 c_q c_k + 4 c_h fp32 flop per causal
         # pair-head (dS, dQ, dK, dV products; the convolution's adjoint and kernel gradient;
         # the mixing adjoints)
@@ -841,7 +885,8 @@ def main():
         "pct_bf16_peak": {"std": fl["std"] / s / 1e12 / bf16_peak,
                           "mta": fl["mta"] / s / 1e12 / bf16_peak,
                           "peak_tflops": bf16_peak, "peak_source": f"{peak_src} bf16 {peak_kind}"},
-        "roofline": roof, "gpu_launches": args.steps * len(step_kernels(wl, args.bwd)),
+        "roofline": roof, "gpu_launches": args.steps * (len(step_kernels(wl, args.bwd))
+                                       + (bwd_tc_launches(wl) - 1 if args.bwd and uses_bwd_tc(wl) else 0)),
         "timed_region_ms": res["region_ms"], "per_kernel_ms": res["per_kernel_ms"],
         "clocks": res["clocks"], "e2e": res["e2e"], "epilogue_group_norm": epi,
     }
