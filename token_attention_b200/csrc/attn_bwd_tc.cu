@@ -149,9 +149,15 @@ __global__ void __launch_bounds__(kThreadsB) bwd_scores_kernel(StripArgs p) {
   auto strip = [&](float *base, int hl, int rows) {
     return base + ((static_cast<long long>(b) * p.H + g * CH + hl) * rows) * P;
   };
-  float m[CH], l[CH];
+  // online statistics of each softmax head s: max m, sum l = sum_j e_j, and, with
+  // e_j = exp(C_s[j] - m), Dt = sum_j dA_s[j] e_j (D_s = Dt / l) and, with post
+  // mixing on the own rows, Wt[h][s] = sum_j dA''_h[j] e_j (dw[h][s] += Wt / l)
+  float m[CH], l[CH], Dt[CH], Wt[CH * CH];
 #pragma unroll
-  for (int h = 0; h < CH; ++h) { m[h] = -INFINITY; l[h] = 0.f; }
+  for (int h = 0; h < CH; ++h) { m[h] = -INFINITY; l[h] = 0.f; Dt[h] = 0.f; }
+#pragma unroll
+  for (int x = 0; x < CH * CH; ++x) Wt[x] = 0.f;
+  const bool own = valid && u < p.g.no;
   const int i_last = min(p.L - 1, p.r0 + u0 + kRows - 1);  // the CTA's last query
   const int ntiles = i_last / kKeyTile + 1;
   // Mask_0 S: strip rows u0 .. u0+TR-1 (queries r0 - HALO + su), keys j0 - 8 ..
@@ -201,6 +207,17 @@ __global__ void __launch_bounds__(kThreadsB) bwd_scores_kernel(StripArgs p) {
           *reinterpret_cast<float4 *>(dst + x) = make_float4(cv[h][x], cv[h][x + 1], cv[h][x + 2], cv[h][x + 3]);
       }
     }
+    // dA'' of every head of the group at the thread's keys (the GEMM ran before)
+    float da2[CH][kSeg];
+#pragma unroll
+    for (int h = 0; h < CH; ++h) {
+      const float *src = strip(p.D, h, p.g.rc) + u * P + jb;
+#pragma unroll
+      for (int x = 0; x < kSeg; x += 4) {
+        const float4 v = *reinterpret_cast<const float4 *>(src + x);
+        da2[h][x] = v.x; da2[h][x + 1] = v.y; da2[h][x + 2] = v.z; da2[h][x + 3] = v.w;
+      }
+    }
 #pragma unroll
     for (int h = 0; h < CH; ++h) {
       float lg[kSeg];
@@ -214,11 +231,32 @@ __global__ void __launch_bounds__(kThreadsB) bwd_scores_kernel(StripArgs p) {
         }
         z = jb + x <= i ? z : -INFINITY;  // Mask_-inf
         lg[x] = z;
+        if (z == -INFINITY) continue;
+        // dA of softmax head h: post mixing mixes dA'' back to the source
+        float d = da2[h][x];
+        if (p.hp == 2) {
+          d = 0.f;
+#pragma unroll
+          for (int h2 = 0; h2 < CH; ++h2) d = fmaf(wm[h2 * CH + h], da2[h2][x], d);
+        }
+        float e = 1.f;
         if (z > m[h]) {
-          l[h] = l[h] * __expf(m[h] - z) + 1.f;
+          const float sc = __expf(m[h] - z);
+          l[h] *= sc;
+          Dt[h] *= sc;
+          if (p.hp == 2) {
+#pragma unroll
+            for (int h2 = 0; h2 < CH; ++h2) Wt[h2 * CH + h] *= sc;
+          }
           m[h] = z;
-        } else if (z != -INFINITY) {
-          l[h] += __expf(z - m[h]);
+        } else {
+          e = __expf(z - m[h]);
+        }
+        l[h] += e;
+        Dt[h] = fmaf(d, e, Dt[h]);
+        if (p.hp == 2 && own) {
+#pragma unroll
+          for (int h2 = 0; h2 < CH; ++h2) Wt[h2 * CH + h] = fmaf(da2[h2][x], e, Wt[h2 * CH + h]);
         }
       }
       float *dst = strip(p.A, h, p.g.rc) + u * P + jb;  // logits for now
@@ -230,17 +268,30 @@ __global__ void __launch_bounds__(kThreadsB) bwd_scores_kernel(StripArgs p) {
     __syncthreads();  // the buffer is restaged two tiles on
   }
   // row statistics over the 16 threads of the row (the lanes with the same bit 2)
-  float mr[CH], lr[CH];
+  float mr[CH], lr[CH], Dr[CH], dwp[CH * CH];
+#pragma unroll
+  for (int x = 0; x < CH * CH; ++x) dwp[x] = 0.f;
 #pragma unroll
   for (int h = 0; h < CH; ++h) {
     float mx = m[h];
 #pragma unroll
     for (int o : {1, 2, 8, 16}) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
-    float part = m[h] == -INFINITY ? 0.f : l[h] * __expf(m[h] - mx);
+    const float sc = m[h] == -INFINITY ? 0.f : __expf(m[h] - mx);
+    float part = l[h] * sc, dpart = Dt[h] * sc;
 #pragma unroll
-    for (int o : {1, 2, 8, 16}) part += __shfl_xor_sync(0xffffffffu, part, o);
+    for (int o : {1, 2, 8, 16}) {
+      part += __shfl_xor_sync(0xffffffffu, part, o);
+      dpart += __shfl_xor_sync(0xffffffffu, dpart, o);
+    }
     mr[h] = mx;
     lr[h] = part;
+    Dr[h] = part > 0.f ? dpart / part : 0.f;
+    if (p.hp == 2) {
+      // dw[h2][h] over this row: Wt / l, summed over the row's 16 threads (each
+      // thread's share taken once, by the block reduction below)
+#pragma unroll
+      for (int h2 = 0; h2 < CH; ++h2) dwp[h2 * CH + h] = part > 0.f ? Wt[h2 * CH + h] * sc / part : 0.f;
+    }
   }
   // ---- the softmax's backward on the same rows: the weights A_s = exp(C - m) / l
   // are recomputed from the logits wherever they are needed, never stored
@@ -269,50 +320,7 @@ __global__ void __launch_bounds__(kThreadsB) bwd_scores_kernel(StripArgs p) {
       da[x + 3] = jb + x + 3 <= i ? v.w : 0.f;
     }
   };
-  const bool own = valid && u < p.g.no;
-  float Dp[CH], dwp[CH * CH];
-#pragma unroll
-  for (int h = 0; h < CH; ++h) Dp[h] = 0.f;
-#pragma unroll
-  for (int x = 0; x < CH * CH; ++x) dwp[x] = 0.f;
-  // pass 2: D_s = sum_j dA_s A_s (post mixing: dA_s = sum_h w[h][s] dA''_h; pre or
-  // none: dA'_h = dA''_h), and the post-mixing dw = sum dA''_h A_s
-  if (valid) {
-    for (int jb = kSeg * seg; jb <= i; jb += kKeyTile) {
-      float a[CH][kSeg], da[CH][kSeg];
-#pragma unroll
-      for (int h = 0; h < CH; ++h) { weights(jb, h, a[h]); grads(jb, h, da[h]); }
-#pragma unroll
-      for (int s2 = 0; s2 < CH; ++s2)
-#pragma unroll
-        for (int x = 0; x < kSeg; ++x) {
-          float d = da[s2][x];
-          if (p.hp == 2) {
-            d = 0.f;
-#pragma unroll
-            for (int h = 0; h < CH; ++h) d = fmaf(wm[h * CH + s2], da[h][x], d);
-          }
-          Dp[s2] = fmaf(d, a[s2][x], Dp[s2]);
-        }
-      if (p.hp == 2 && own) {
-#pragma unroll
-        for (int h = 0; h < CH; ++h)
-#pragma unroll
-          for (int s2 = 0; s2 < CH; ++s2)
-#pragma unroll
-            for (int x = 0; x < kSeg; ++x) dwp[h * CH + s2] = fmaf(da[h][x], a[s2][x], dwp[h * CH + s2]);
-      }
-    }
-  }
-  float Dr[CH];
-#pragma unroll
-  for (int h = 0; h < CH; ++h) {
-    float v = Dp[h];
-#pragma unroll
-    for (int o : {1, 2, 8, 16}) v += __shfl_xor_sync(0xffffffffu, v, o);
-    Dr[h] = v;
-  }
-  // pass 3: dC = A (dA - D) into the dA'' strip (pre mixing: dC'_h, then mixed
+  // pass 2: dC = A (dA - D) into the dA'' strip (pre mixing: dC'_h, then mixed
   // back, with dw = sum dC'_h C_s); A'' (hi / lo) of the own rows
   if (valid) {
     for (int jb = kSeg * seg; jb <= i; jb += kKeyTile) {
