@@ -206,6 +206,64 @@ def test_building_block_argument_errors(L):
     gn = mta.MtaGn(0x20000, 0x20000, 1e-5, 12, -1.0)
     assert L.mta_group_norm_scale(FAKE, ctypes.byref(gn), 4, 2, 0, FAKE, None) == 1
     assert L.mta_group_norm_scale(FAKE, None, 4, 2, 64, FAKE, None) == 1
+    # the general GEMM: flags are 0 or 1; the contiguous extent of each operand a
+    # multiple of 8 (K for [rows][K], M or N for a transposed operand); C apart from A, B
+    g = lambda M, N, K, am=0, bm=0, f=0, c=fake(3): L.mta_gemm_bf16(fake(1), fake(2), c, M, N, K, am, bm, f, None)
+    assert g(16, 16, 16, am=2) == 1
+    assert g(16, 16, 16, f=3) == 1
+    assert g(12, 16, 16, am=1) == 1     # transposed A: M % 8
+    assert g(16, 12, 16, bm=1) == 1     # transposed B: N % 8
+    assert g(16, 16, 12) == 1           # K-major: K % 8
+    assert g(16, 16, 16, c=fake(1)) == 1   # C overlaps A
+    # the group norm's backward: d in {32, 64, 96, 128}; the gate's gradient when gated
+    gb = lambda d, g_=ctypes.byref(gn), dgate=None: L.mta_group_norm_scale_bwd(
+        fake(1), fake(2), g_, 4, 2, d, fake(3), fake(4), fake(5), fake(6), dgate, None)
+    assert gb(48) == 2
+    assert gb(64, g_=None) == 1
+    gated = mta.MtaGn(0x20000, 0x20000, 1e-5, 12, -1.0, 0x30000)
+    assert gb(64, g_=ctypes.byref(gated)) == 1   # no dgate
+
+
+def test_layer_backward_argument_errors(L):
+    """mta_layer_bwd checks its arguments on the host and enqueues nothing on error."""
+    cfg = good_cfg()
+    cfg.workspace, cfg.workspace_bytes = 0x100000, 1 << 40
+    gn = mta.MtaGn(0x20000, 0x20000, 1e-5, 12, -1.0)
+    f = lambda c, g=ctypes.byref(gn), dx=fake(11), dwq=fake(12), dwo=fake(13), dout=fake(4): L.mta_layer_bwd(
+        fake(1), fake(2), FAKE, FAKE, g, fake(3), dout, ctypes.byref(c) if c else None,
+        dx, dwq, dwo, None, None, fake(14), fake(15), None)
+    assert f(None) == 1
+    assert f(cfg, g=None) == 1
+    assert f(cfg, dx=None) == 1
+    assert f(cfg, dout=None) == 1
+    assert f(cfg, dx=fake(1)) == 1                      # dx overlaps x
+    assert f(cfg, dwo=fake(12)) == 1                    # two outputs overlap
+    bad = good_cfg(dtype=mta.F32)
+    bad.workspace, bad.workspace_bytes = 0x100000, 1 << 40
+    assert f(bad) == 2
+    odd = good_cfg(d=48)                                # d outside {32, 64, 96, 128}
+    odd.workspace, odd.workspace_bytes = 0x100000, 1 << 40
+    assert f(odd) == 2
+    small = good_cfg()
+    small.workspace, small.workspace_bytes = 0x100000, 1 << 10
+    assert f(small) == 3
+    gated = mta.MtaGn(0x20000, 0x20000, 1e-5, 12, -1.0, 0x30000)
+    assert f(cfg, g=ctypes.byref(gated)) == 1           # gated without dgate
+
+
+def test_layer_backward_workspace_query(L):
+    """The fixed part (status; QKV, O, Y bf16; dY fp32; dO bf16; dq, dk, dv fp32; dQKV
+    bf16), then the larger of the forward recompute's contraction operands and the
+    tensor-core backward's strips."""
+    B, H, Ls, d = 2, 4, 64, 64
+    T, D = B * Ls, H * d
+    fixed = 256 + 2 * up(T * 3 * D * 2) + 3 * up(T * D * 2) + 4 * up(T * D * 4)
+    cfg = good_cfg()
+    attn_bwd = L.mta_attn_bwd_workspace_bytes(ctypes.byref(cfg)) - 256
+    attn_fwd = L.mta_attn_workspace_bytes(ctypes.byref(cfg)) - 256
+    assert L.mta_layer_bwd_workspace_bytes(ctypes.byref(cfg)) == fixed + max(attn_bwd, attn_fwd)
+    other = good_cfg(c_q=3)   # neither the contraction kernel nor the tensor-core backward
+    assert L.mta_layer_bwd_workspace_bytes(ctypes.byref(other)) == fixed
 
 
 def test_backward_argument_errors(L):
