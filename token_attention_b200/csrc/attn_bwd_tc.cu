@@ -74,14 +74,17 @@ __device__ __forceinline__ void split_bf16(float x, __nv_bfloat16 &hi, __nv_bflo
 }
 
 // Step 3: C = Conv2d_theta(Mask_0 S) for the block's C rows (and pre mixing),
-// Mask_-inf, the softmax statistics of each row (its logits kept in the A strip),
-// then the softmax's backward on the same rows: dA (post mixing: mixed back to
-// the sources), D, dC = A (dA - D) (pre mixing: then mixed back) into the dA''
-// strip, dw, and A'' (hi / lo) of the block's own rows.  CTA: one head group, 16 rows;
-// thread (row, seg): 8 consecutive keys 8 seg .. 8 seg + 7 of every 128-key tile.
-// For each tap row a the thread loads the 8 + 2c values of the staged S row it
-// needs once and forms its 8 outputs x c_k taps from registers.  Key tiles past
-// the CTA's last row are skipped (their weights are zero and nothing reads them).
+// Mask_-inf, the softmax statistics of each row (its logits kept in the A strip)
+// and, in the same pass, D = sum_j dA A and the post-mixing dw online (rescaled
+// with the running maximum as the sum is); then the softmax's backward on the
+// same rows: dA (post mixing: mixed back to the sources), dC = A (dA - D) (pre
+// mixing: then mixed back) into the dA'' strip, the pre-mixing dw, and A'' (hi /
+// lo) of the block's own rows.  CTA: one head group, 16 rows; thread (row, seg):
+// 8 consecutive keys 8 seg .. 8 seg + 7 of every 128-key tile.  For each tap row
+// a the thread loads the 24 staged values around its keys (keys jb - 8 .. jb + 15,
+// 8 + 2c of them used) once and forms its 8 outputs x c_k taps from registers.
+// Key tiles past the CTA's last row are skipped (their weights are zero and
+// nothing reads them).
 constexpr int kRows = 16;               // rows of a CTA in the convolution kernels
 constexpr int kSeg = 8;                 // consecutive keys of a thread
 // Staged rows are 164 floats (128 + 2c keys, padded): 656 bytes, 16 modulo 128, so
