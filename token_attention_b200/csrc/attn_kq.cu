@@ -157,6 +157,12 @@ struct KGeo {
   static constexpr uint32_t TMEM_COLS = 512, C_COL = 0, P_COL = DB ? 0 : 128 * NSRC;
   static constexpr uint32_t Z_COL0 = DB ? 256 : POST ? P_COL : P_COL + 128;
   static_assert(Z_COL0 + 128 * (NV - 1) + D <= TMEM_COLS, "tensor memory");
+  // C double-buffered (tile T in buffer T & 1): DB, and the post-softmax variant when
+  // a second C fits after Z (its weights are in shared memory, not over C); buffer 1
+  // starts at column CB1
+  static constexpr bool CDB = DB || (POST && Z_COL0 + 128 * (NV - 1) + D + 128 * NSRC <= TMEM_COLS);
+  static constexpr uint32_t CB1 = DB ? 128 : TMEM_COLS - 128 * NSRC;
+  static_assert(5 + 2 * NS + 9 <= 32, "barriers before the item ring");
   static_assert(MIX != 1 || NV == 1, "pre-softmax mixing uses the destination head's V only");
   static_assert(OFF_K % 1024 == 0 && OFF_V % 1024 == 0, "swizzle alignment");
   static_assert(OFF_PS % 16 == 0 && OFF_DG % 16 == 0 && OFF_U % 16 == 0, "alignment");
@@ -253,6 +259,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   // DB: C complete and P written, per buffer (tile T uses buffer T & 1)
   uint64_t *const c_fullb[2] = {c_full, v_full + 6};
   uint64_t *const p_fullb[2] = {p_full, v_full + 7};
+  // CDB without DB (post-softmax variant): C of buffer b has been read by the softmax
+  uint64_t *const c_freeb[2] = {c_free, v_full + 8};
   uint32_t *tslot = reinterpret_cast<uint32_t *>(small + G::TSLOT_OFF);
   volatile int *abort_flag = reinterpret_cast<volatile int *>(small + G::ABORT_OFF);
   // item ring: it_full[s] completes when slot s holds the next item index (or -1 at
@@ -317,7 +325,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int s = 0; s < G::NS; ++s) { mbar_init(k_full + s, 1); mbar_init(k_empty + s, 1); }
     mbar_init(v_full, 1); mbar_init(v_empty, 1); mbar_init(c_full, 1); mbar_init(c_free, 8);
     mbar_init(p_full, 8); mbar_init(mma_done, 1);
-    mbar_init(c_fullb[1], 1); mbar_init(p_fullb[1], 8);
+    mbar_init(c_fullb[1], 1); mbar_init(p_fullb[1], 8); mbar_init(c_freeb[1], 8);
     // consumers per item: the V and query loaders, the MMA thread and the 8 softmax
     // warps of each CTA, and the second CTA's key loader (no V loader with POST)
     constexpr int per_cta = (POST ? 1 : 2) + 1 + 8;
@@ -470,8 +478,14 @@ __global__ void __launch_bounds__(kThreads, 1)
       // DB: into buffer T & 1 without waiting for the softmax (the buffer's previous
       // tile, T - 2, had its P V issued before, and MMAs run in issue order)
       auto issue_c = [&](bool last_of_item) -> bool {
-        if (!G::DB && T > 0 && !wwait(c_free, (T - 1) & 1)) return false;
-        const uint32_t c_dst = tmem + G::C_COL + (G::DB ? 128u * (T & 1) : 0u);
+        if constexpr (!G::DB) {
+          if constexpr (G::CDB) {  // the softmax has read the buffer's previous tile, T - 2
+            if (T >= 2 && !wwait(c_freeb[T & 1], ((T - 2) >> 1) & 1)) return false;
+          } else if (T > 0 && !wwait(c_free, (T - 1) & 1)) {
+            return false;
+          }
+        }
+        const uint32_t c_dst = tmem + G::C_COL + ((G::CDB && (T & 1)) ? G::CB1 : 0u);
         for (int ch = 0; ch < G::NSRC * G::NCH; ch += G::SB, ++cnt) {
           const int st = cnt % G::NS;
           // source head sc (its own accumulator and query rows); the 16 elements
@@ -511,7 +525,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           mma_commit_if(issuer, k_empty + st);
         }
-        mma_commit_if(issuer, G::DB ? c_fullb[T & 1] : c_full);
+        mma_commit_if(issuer, G::CDB ? c_fullb[T & 1] : c_full);
         if (last_of_item) mma_commit_if(issuer, q_free);  // the query buffer may take the next item
         return true;
       };
@@ -884,12 +898,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         float fnext[G::NSRC];
 #pragma unroll
         for (int sc = 0; sc < G::NSRC; ++sc) fnext[sc] = st_id < G::BN ? fac_next(sc, sl) : 0.f;
-        if constexpr (G::DB)
+        if constexpr (G::CDB)
           mbar_wait(c_fullb[T & 1], (T >> 1) & 1, abort_flag, p.err);
         else
           mbar_wait(c_full, T & 1, abort_flag, p.err);
         tc_fence_after();
-        const uint32_t cbuf = G::DB ? 128u * (T & 1) : 0u;  // this tile's C (and, with DB, P) buffer
+        const uint32_t cbuf = (G::CDB && (T & 1)) ? G::CB1 : 0u;  // this tile's C (and, with DB, P) buffer
         // C' = sum over source heads of w * (C_s x its column factors); one source without mixing
         float cv[G::HALF];
 #pragma unroll
@@ -920,7 +934,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc_fence_before();  // (with DB: orders the C reads before the barrier that precedes the P writes)
         if constexpr (!G::DB) {  // with DB the buffer is reused only after this tile's P V
           __syncwarp();
-          if (lane == 0) mbar_arrive(c_free);
+          if (lane == 0) mbar_arrive(G::CDB ? c_freeb[T & 1] : c_free);
         }
         if (eq != 0) {  // queries were scaled down (|q| > 2^14)
 #pragma unroll
