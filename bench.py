@@ -74,6 +74,16 @@ def uses_contraction(wl: synth.Workload) -> bool:
             and (wl.head_place == synth.OFF or wl.c_h == 2))
 
 
+def kq_kernel_name(wl: synth.Workload) -> str:
+    """The contraction kernel the library launches: the CTA-pair form for sequences of
+    8192 and more (d = 128, or d = 64 with post-softmax mixing; no post-softmax
+    convolution), else the one-CTA form."""
+    pair = (wl.L >= 8192 and not wl.kq_post and
+            ((wl.d == 128 and wl.head_place in (synth.OFF, synth.POST)) or
+             (wl.d == 64 and wl.head_place == synth.POST)))
+    return "attn_kq_pair_kernel" if pair else "attn_kq_kernel"
+
+
 def contraction_tensor_flops(wl: synth.Workload) -> float:
     """Tensor flops the contraction kernel executes per launch: per (batch, head,
     query tile, key tile at or below the diagonal) a 128x128 tile of the
@@ -102,7 +112,7 @@ def uses_direct_tc(wl: synth.Workload) -> bool:
 
 def uses_bwd_tc(wl: synth.Workload) -> bool:
     """Whether the default backward runs on the tensor cores (attn_bwd_tc.cu)."""
-    return (wl.dtype == "bf16" and wl.d in (64, 128) and wl.kq_place == synth.PRE
+    return (wl.dtype == "bf16" and wl.d in (64, 96, 128) and wl.kq_place == synth.PRE
             and (wl.c_q, wl.c_k) == (6, 11) and not wl.kq_post
             and (wl.head_place == synth.OFF or wl.c_h == 2))
 
@@ -172,6 +182,7 @@ def read_peaks() -> tuple[dict, str]:
 # while these files are unchanged since its capture)
 KERNEL_SOURCES = {
     "attn_kq_kernel": ("attn_kq.cu", "ptx.cuh"),
+    "attn_kq_pair_kernel": ("attn_kq_pair.cu", "ptx.cuh"),
     "kq_prep_kernel": ("kq_prep.cu",),
     "vt_prep_kernel": ("kq_prep.cu",),
     "attn_tc_kernel": ("attn_tc.cu", "ptx.cuh"),
@@ -353,7 +364,7 @@ def step_kernels(wl: synth.Workload, bwd: bool) -> list[str]:
     if bwd:
         return [bwd_kernel]
     if uses_contraction(wl):
-        attn = ["kq_prep_kernel"] + (["vt_prep_kernel"] if wl.kq_post else []) + ["attn_kq_kernel"]
+        attn = ["kq_prep_kernel"] + (["vt_prep_kernel"] if wl.kq_post else []) + [kq_kernel_name(wl)]
     elif uses_direct_tc(wl):
         attn = ["attn_tc_kernel"]
     else:
@@ -372,7 +383,8 @@ def dominant_kernel(wl: synth.Workload, bwd: bool) -> tuple[int, int, str]:
     n = launches_per_step(wl) + 1
     if uses_contraction(wl):
         # ... key prepass, (value prepass), attention kernel, (output GEMM)
-        return (n - 3, n - 2, "attn_kq_kernel") if wl.layer else (n - 2, n - 1, "attn_kq_kernel")
+        k = kq_kernel_name(wl)
+        return (n - 3, n - 2, k) if wl.layer else (n - 2, n - 1, k)
     name = "attn_tc_kernel" if uses_direct_tc(wl) else "attn_simt_kernel"
     return (1, 2, name) if wl.layer else (0, 1, name)
 

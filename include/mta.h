@@ -264,7 +264,7 @@ mta_status mta_group_norm_scale_bwd(const void *o, const float *dy, const mta_gn
  *   dw           : [H/c_h][c_h][c_h] fp32, overwritten (may be NULL; ignored when
  *                  head_place == MTA_OFF)
  * Two implementations (cfg->path):
- *   3: the contractions on the tensor cores (attn_bwd_tc.cu): bf16, d = 64 or
+ *   3: the contractions on the tensor cores (attn_bwd_tc.cu): bf16, d = 64, 96 or
  *      128, c_q = 6, c_k = 11, kq_place = MTA_PRE, no post-softmax convolution,
  *      c_h = 2 with head mixing; query blocks of 246 rows, every head at once,
  *      their maps in strips of the workspace (S = s Q K^T, dA'' = dO V^T, dQ,

@@ -2,7 +2,7 @@
 against the fp64 oracle's backward, through the C ABI.
 
 Every gradient (q, k, v, theta, w) at the CUDA-core backward's fp32 tolerance
-(relative L2 error 1e-4): the tensor-core path takes the bf16 inputs themselves as
+(relative L2 error 1e-4): the tensor-core path (d = 64, 96 or 128) takes the bf16 inputs themselves as
 MMA operands and splits its computed operands (dS, A'') into two bf16 halves, so
 its products carry about 16 significant bits and its sums fp32 accumulation.
 Lengths span one query block (L <= 246), several blocks and a ragged tail; the
@@ -63,7 +63,8 @@ def check(wl, inp, dout, path=mta.PATH_KQ):
 
 
 CASES = [(128, synth.POST, 9), (128, synth.POST, 247), (128, synth.PRE, 300), (128, synth.OFF, 70),
-         (64, synth.POST, 600), (64, synth.PRE, 250), (64, synth.OFF, 119), (128, synth.POST, 237)]
+         (64, synth.POST, 600), (64, synth.PRE, 250), (64, synth.OFF, 119), (128, synth.POST, 237),
+         (96, synth.POST, 300), (96, synth.PRE, 130)]
 
 
 @pytest.mark.parametrize("d,hp,L", CASES)
@@ -91,6 +92,16 @@ def test_bwd_tc_full_length_one_group():
     """The pretraining recipe at its full length L = 2048 (9 query blocks), one batch
     and one head group, against the oracle's full L x L backward of that group."""
     wl = synth.shrink(synth.WORKLOADS["pretrain_d128_L2048"], B=1, H=2, seed=952)
+    inp = synth.make_attn_inputs(wl)
+    dout = synth.round_bf16(synth.normal(wl.seed, 20, (wl.B, wl.L, wl.H, wl.d)))
+    check(wl, inp, dout)
+
+
+def test_bwd_tc_d96_full_length_one_group():
+    """The pages' 880M shape (d = 96: 1536 over 16 heads) at L = 2048, one head group:
+    the operands' 96 channels are read as two 64-channel TMA boxes, the second half
+    past d zero-filled."""
+    wl = synth.shrink(synth.WORKLOADS["pretrain_d96_L2048"], B=1, H=2, seed=954)
     inp = synth.make_attn_inputs(wl)
     dout = synth.round_bf16(synth.normal(wl.seed, 20, (wl.B, wl.L, wl.H, wl.d)))
     check(wl, inp, dout)

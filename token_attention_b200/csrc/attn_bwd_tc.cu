@@ -574,7 +574,7 @@ BgTensor strip_tensor(const void *base, const BwdArgs &a, int rows, int pitch) {
 }  // namespace
 
 bool attn_bwd_tc_supported(const BwdArgs &a) {
-  return a.dtype == 1 && (a.d == 64 || a.d == 128) && a.cq == 6 && a.ck == 11 && a.kq == 1 && !a.kqp &&
+  return a.dtype == 1 && (a.d == 64 || a.d == 96 || a.d == 128) && a.cq == 6 && a.ck == 11 && a.kq == 1 && !a.kqp &&
          (a.hp == 0 || a.ch == 2) && a.rs % 8 == 0 &&
          (reinterpret_cast<uintptr_t>(a.q) | reinterpret_cast<uintptr_t>(a.k) | reinterpret_cast<uintptr_t>(a.v) |
           reinterpret_cast<uintptr_t>(a.dout)) % 16 == 0 &&
