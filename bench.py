@@ -113,15 +113,21 @@ def uses_direct_tc(wl: synth.Workload) -> bool:
 def uses_bwd_tc(wl: synth.Workload) -> bool:
     """Whether the default backward runs on the tensor cores (attn_bwd_tc.cu)."""
     return (wl.dtype == "bf16" and wl.d in (64, 96, 128) and wl.kq_place == synth.PRE
-            and (wl.c_q, wl.c_k) == (6, 11) and not wl.kq_post
+            and (wl.c_q, wl.c_k) == (6, 11)
             and (wl.head_place == synth.OFF or wl.c_h == 2))
 
 
+def bwd_tc_no(wl: synth.Workload) -> int:
+    """Own rows of a query block of the tensor-core backward."""
+    return 256 - (3 if wl.kq_post else 2) * (wl.c_q - 1)
+
+
 def bwd_tc_launches(wl: synth.Workload) -> int:
-    """Kernels of the tensor-core backward per call: per query block of 256 - 2 (c_q - 1)
-    rows the S and dA'' GEMMs, the convolution / softmax kernel, the adjoint kernel and
-    the dQ, dK and dV GEMMs."""
-    return 7 * -(-wl.L // (256 - 2 * (wl.c_q - 1)))
+    """Kernels of the tensor-core backward per call: per query block the S and dA''
+    GEMMs, the convolution / softmax kernel, the adjoint kernel and the dQ, dK and dV
+    GEMMs; with the convolution after the softmax four more (its output gradient, its
+    adjoint, the mixed weights, the softmax's backward)."""
+    return (11 if wl.kq_post else 7) * -(-wl.L // bwd_tc_no(wl))
 
 
 def bwd_tc_gemm_flops(wl: synth.Workload) -> float:
@@ -129,11 +135,12 @@ def bwd_tc_gemm_flops(wl: synth.Workload) -> float:
     per query block of NO rows (strips of 256 rows) and keys 0 .. W-1, for every
     head: S (256 x W x d), dA'' (251 x W x d), dQ (NO x d x 2W: hi and lo halves),
     dK and dV (W x d x 512)."""
-    no = 256 - 2 * (wl.c_q - 1)
+    no = bwd_tc_no(wl)
+    rc = no + (2 if wl.kq_post else 1) * (wl.c_q - 1)
     f = 0.0
     for r0 in range(0, wl.L, no):
-        W = min(wl.L, r0 + no + wl.c_q - 1)
-        f += 2 * (256 + (no + wl.c_q - 1)) * W * wl.d + 2 * no * wl.d * 2 * W + 2 * 2 * W * wl.d * 512
+        W = min(wl.L, r0 + rc)
+        f += 2 * (256 + rc) * W * wl.d + 2 * no * wl.d * 2 * W + 2 * 2 * W * wl.d * 512
     return f * wl.B * wl.H
 
 
@@ -819,13 +826,15 @@ def main():
         # algorithmic work is the convolution recomputed, its adjoint and the kernel
         # gradient, 3 x 2 c_q c_k fp32 flop per causal pair-head.  The time is the whole
         # backward's (its GEMMs included), so the fraction is a lower bound.
-        f_cc = 6 * wl.c_q * wl.c_k * wl.causal_pairs
+        n_conv = 2 if wl.kq_post else 1
+        f_cc = 6 * wl.c_q * wl.c_k * n_conv * wl.causal_pairs
         achieved = f_cc / ks / 1e12
         roof = {"bound": "alu", "achieved": achieved, "peak": FP32_PEAK_TFLOPS, "unit": "TFLOP/s",
                 "frac": achieved / FP32_PEAK_TFLOPS, "traffic": None,
                 "kernel": kernel, "kernel_ms": ks * 1e3,
-                "per_unit": f"F_cc = 6 c_q c_k = {6 * wl.c_q * wl.c_k} fp32 flop per causal pair-head "
-                            f"(convolution, adjoint, kernel gradient on the CUDA cores), x {wl.causal_pairs} "
+                "per_unit": f"F_cc = 6 c_q c_k per convolution = {6 * wl.c_q * wl.c_k * n_conv} fp32 flop per "
+                            f"causal pair-head (each convolution recomputed, its adjoint and its kernel "
+                            f"gradient on the CUDA cores), x {wl.causal_pairs} "
                             f"pair-heads per call; the time is the whole backward's, its "
                             f"{bwd_tc_launches(wl)} kernels (GEMMs included)",
                 "peak_source": fp32_src, "timing": timing,

@@ -265,12 +265,13 @@ mta_status mta_group_norm_scale_bwd(const void *o, const float *dy, const mta_gn
  *                  head_place == MTA_OFF)
  * Two implementations (cfg->path):
  *   3: the contractions on the tensor cores (attn_bwd_tc.cu): bf16, d = 64, 96 or
- *      128, c_q = 6, c_k = 11, kq_place = MTA_PRE, no post-softmax convolution,
- *      c_h = 2 with head mixing; query blocks of 246 rows, every head at once,
- *      their maps in strips of the workspace (S = s Q K^T, dA'' = dO V^T, dQ,
- *      dK, dV as batched tcgen05 GEMMs; the convolution, its adjoint and the
- *      softmax on the CUDA cores).  MTA_ERR_UNSUPPORTED for other
- *      configurations, MTA_ERR_WORKSPACE when the strips do not fit.
+ *      128, c_q = 6, c_k = 11, kq_place = MTA_PRE (with or without the
+ *      post-softmax convolution, kq_post), c_h = 2 with head mixing; query
+ *      blocks of 246 rows (241 with kq_post), every head at once, their maps in
+ *      strips of the workspace (S = s Q K^T, dA'' = dO V^T, dQ, dK, dV as batched
+ *      tcgen05 GEMMs; the convolutions, their adjoints and the softmax on the
+ *      CUDA cores).  MTA_ERR_UNSUPPORTED for other configurations,
+ *      MTA_ERR_WORKSPACE when the strips do not fit.
  *   1: the CUDA cores in fp32 arithmetic, every forward configuration
  *      (attn_bwd_simt.cu; attn_bwd_post_simt.cu with the post-softmax
  *      convolution).
@@ -283,8 +284,9 @@ mta_status mta_group_norm_scale_bwd(const void *o, const float *dy, const mta_gn
  * holds the error word and, where path 3 applies, its strips: for one query
  * block of every head, a 256-row S strip and two (three with pre-softmax
  * mixing) fp32 strips of 251 rows over the keys, and two bf16 strips of 512 rows
- * (B*H*pitch*(256*4 + 2*251*4 + 2*512*2) bytes, pitch = L rounded up to 64).  No
- * L x L map is stored. */
+ * (B*H*pitch*(256*4 + 2*251*4 + 2*512*2) bytes, pitch = L rounded up to 64);
+ * with kq_post the fp32 strips have 251 rows and three more are added (251, 246
+ * and 241 rows).  No L x L map is stored. */
 size_t mta_attn_bwd_workspace_bytes(const mta_cfg *cfg);
 mta_status mta_attn_bwd(const void *q, const void *k, const void *v, const float *theta_kq,
                         const float *w_head, const void *dout, const mta_cfg *cfg, float *dq,

@@ -299,6 +299,10 @@ def test_backward_argument_errors(L):
     # pre-softmax mixing keeps the unmixed C as well
     assert L.mta_attn_bwd_workspace_bytes(ctypes.byref(good_cfg(head_place=mta.PRE))) == \
         256 + strips + up(Z * rc * P * 4)
+    # the convolution after the softmax: blocks of 256 - 3 (c_q - 1) = 241 own rows, the
+    # same 251-row strips, and its output gradient G [251], dA / dC [246] and A' [241]
+    assert L.mta_attn_bwd_workspace_bytes(ctypes.byref(good_cfg(kq_post=1))) == \
+        256 + strips + up(Z * 251 * P * 4) + up(Z * 246 * P * 4) + up(Z * 241 * P * 4)
     assert L.mta_attn_bwd_workspace_bytes(ctypes.byref(good_cfg(c_q=3))) == 256   # CUDA cores only
     assert L.mta_attn_bwd_workspace_bytes(ctypes.byref(good_cfg(c_k=4))) == 0
 

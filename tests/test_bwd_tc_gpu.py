@@ -5,8 +5,10 @@ Every gradient (q, k, v, theta, w) at the CUDA-core backward's fp32 tolerance
 (relative L2 error 1e-4): the tensor-core path (d = 64, 96 or 128) takes the bf16 inputs themselves as
 MMA operands and splits its computed operands (dS, A'') into two bf16 halves, so
 its products carry about 16 significant bits and its sums fp32 accumulation.
-Lengths span one query block (L <= 246), several blocks and a ragged tail; the
-pretraining recipe runs at its full length for one head group.
+Lengths span one query block (L <= 246; 241 with the convolution after the
+softmax), several blocks and a ragged tail; the pretraining recipe and the
+convolution on both sides of the softmax run at their full length for one head
+group.
 """
 import numpy as np
 import pytest
@@ -18,7 +20,7 @@ from token_attention_b200 import build, mta, synth
 pytestmark = pytest.mark.gpu
 
 TOL_F32 = 1e-4
-GRAD_NAMES = ("dq", "dk", "dv", "dtheta", "dw")
+GRAD_NAMES = ("dq", "dk", "dv", "dtheta", "dw", "dtheta_post")
 
 
 @pytest.fixture(scope="module", autouse=True)
@@ -42,8 +44,9 @@ def errs(gpu, ref):
 
 def run_bwd(wl, inp, dout, path):
     q, k, v = (dev(inp[n], wl.dtype) for n in ("q", "k", "v"))
+    tp = None if inp.get("theta_post") is None else dev(inp["theta_post"], "f32")
     g = mta.attn_bwd(q, k, v, dev(inp["theta"], "f32"), dev(inp["w"], "f32"), dev(dout, wl.dtype),
-                     wl.c_q, wl.c_k, wl.c_h, wl.kq_place, wl.head_place, check=True, path=path)
+                     wl.c_q, wl.c_k, wl.c_h, wl.kq_place, wl.head_place, check=True, path=path, theta_post=tp)
     torch.cuda.synchronize()
     return g
 
@@ -51,7 +54,7 @@ def run_bwd(wl, inp, dout, path):
 def check(wl, inp, dout, path=mta.PATH_KQ):
     got = run_bwd(wl, inp, dout, path)
     ref = O.mta_attention_bwd(inp["q"], inp["k"], inp["v"], inp["theta"], inp["w"], wl.c_h, dout,
-                              wl.kq_place, wl.head_place)
+                              wl.kq_place, wl.head_place, theta_post=inp.get("theta_post"))
     out = {}
     for n in GRAD_NAMES:
         if ref[n] is None:
@@ -76,6 +79,30 @@ def test_bwd_tc_small(d, hp, L):
     check(wl, inp, dout)
 
 
+POST_CASES = [(128, synth.POST, 9), (128, synth.POST, 300), (128, synth.PRE, 250), (128, synth.OFF, 242),
+              (64, synth.POST, 500), (96, synth.POST, 130)]
+
+
+@pytest.mark.parametrize("d,hp,L", POST_CASES)
+def test_bwd_tc_post_conv_small(d, hp, L):
+    """The convolution on both sides of the softmax (the pages' default): every
+    gradient, the post-softmax kernels' included, from one query block of 241 rows
+    to three."""
+    wl = synth.shrink(synth.WORKLOADS["both_d128_L2048"], B=2, H=4, L=L, d=d, head_place=hp,
+                      seed=931 + L + d + 3 * hp)
+    inp = synth.make_attn_inputs(wl)
+    dout = synth.round_bf16(synth.normal(wl.seed, 20, (wl.B, wl.L, wl.H, wl.d)))
+    check(wl, inp, dout)
+
+
+def test_bwd_tc_post_conv_full_length_one_group():
+    """The convolution on both sides at L = 2048 (9 query blocks), one head group."""
+    wl = synth.shrink(synth.WORKLOADS["both_d128_L2048"], B=1, H=2, seed=955)
+    inp = synth.make_attn_inputs(wl)
+    dout = synth.round_bf16(synth.normal(wl.seed, 20, (wl.B, wl.L, wl.H, wl.d)))
+    check(wl, inp, dout)
+
+
 def test_bwd_tc_matches_cuda_core_path():
     """Both backward paths on the same inputs (L = 512, two query blocks and a tail)."""
     wl = synth.shrink(synth.WORKLOADS["pretrain_d128_L2048"], B=1, H=4, L=512, seed=951)
@@ -84,6 +111,8 @@ def test_bwd_tc_matches_cuda_core_path():
     tc, _ = check(wl, inp, dout, mta.PATH_KQ)
     simt = run_bwd(wl, inp, dout, mta.PATH_SIMT)
     for n in GRAD_NAMES:
+        if tc[n] is None:
+            continue
         a, b = tc[n].double(), simt[n].double()
         assert float((a - b).norm() / b.norm()) <= 2 * TOL_F32, n
 

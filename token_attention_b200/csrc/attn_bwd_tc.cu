@@ -66,6 +66,8 @@ struct StripArgs {
   __nv_bfloat16 *dS;          // [B][H][512][pitch]: hi rows 0..255, lo rows 256..511
   __nv_bfloat16 *Ap;          // [B][H][512][pitch]: A'' hi / lo
   float *dtheta, *dw;
+  int post;                   // the convolution after the softmax: the scores kernel
+                              // only writes the normalised weights A
 };
 
 __device__ __forceinline__ void split_bf16(float x, __nv_bfloat16 &hi, __nv_bfloat16 &lo) {
@@ -210,14 +212,15 @@ __global__ void __launch_bounds__(kThreadsB) bwd_scores_kernel(StripArgs p) {
           *reinterpret_cast<float4 *>(dst + x) = make_float4(cv[h][x], cv[h][x + 1], cv[h][x + 2], cv[h][x + 3]);
       }
     }
-    // dA'' of every head of the group at the thread's keys (the GEMM ran before)
+    // dA'' of every head of the group at the thread's keys (the GEMM ran before;
+    // with the convolution after the softmax the D strip holds other rows: unused)
     float da2[CH][kSeg];
 #pragma unroll
     for (int h = 0; h < CH; ++h) {
       const float *src = strip(p.D, h, p.g.rc) + u * P + jb;
 #pragma unroll
       for (int x = 0; x < kSeg; x += 4) {
-        const float4 v = *reinterpret_cast<const float4 *>(src + x);
+        const float4 v = p.post ? make_float4(0.f, 0.f, 0.f, 0.f) : *reinterpret_cast<const float4 *>(src + x);
         da2[h][x] = v.x; da2[h][x + 1] = v.y; da2[h][x + 2] = v.z; da2[h][x + 3] = v.w;
       }
     }
@@ -296,11 +299,32 @@ __global__ void __launch_bounds__(kThreadsB) bwd_scores_kernel(StripArgs p) {
       for (int h2 = 0; h2 < CH; ++h2) dwp[h2 * CH + h] = part > 0.f ? Wt[h2 * CH + h] * sc / part : 0.f;
     }
   }
-  // ---- the softmax's backward on the same rows: the weights A_s = exp(C - m) / l
-  // are recomputed from the logits wherever they are needed, never stored
   float inv[CH];
 #pragma unroll
   for (int h = 0; h < CH; ++h) inv[h] = 1.f / lr[h];
+  if (p.post) {
+    // the convolution after the softmax comes between the weights and their
+    // gradient: store the normalised weights A (zero past the diagonal) and stop
+    if (!valid) return;
+    for (int jb = kSeg * seg; jb <= i; jb += kKeyTile) {
+#pragma unroll
+      for (int h = 0; h < CH; ++h) {
+        float *a = strip(p.A, h, p.g.rc) + u * P + jb;
+#pragma unroll
+        for (int x = 0; x < kSeg; x += 4) {
+          float4 v = *reinterpret_cast<float4 *>(a + x);
+          v.x = jb + x + 0 <= i ? __expf(v.x - mr[h]) * inv[h] : 0.f;
+          v.y = jb + x + 1 <= i ? __expf(v.y - mr[h]) * inv[h] : 0.f;
+          v.z = jb + x + 2 <= i ? __expf(v.z - mr[h]) * inv[h] : 0.f;
+          v.w = jb + x + 3 <= i ? __expf(v.w - mr[h]) * inv[h] : 0.f;
+          *reinterpret_cast<float4 *>(a + x) = v;
+        }
+      }
+    }
+    return;
+  }
+  // ---- the softmax's backward on the same rows: the weights A_s = exp(C - m) / l
+  // are recomputed from the logits wherever they are needed, never stored
   auto weights = [&](int jb, int h, float (&a)[kSeg]) {
     const float *lg = strip(p.A, h, p.g.rc) + u * P + jb;
 #pragma unroll
@@ -423,17 +447,37 @@ __global__ void __launch_bounds__(kThreadsB) bwd_scores_kernel(StripArgs p) {
   }
 }
 
-// Step 4: dS = [j <= i] sum theta[a][t] dC[i+a][j+t-c] (hi / lo halves) for the
-// block's own rows, zeros elsewhere, and dtheta over the own rows.  CTA: one
-// head, 16 rows u = 0 .. 127; thread (row, seg): 8 consecutive keys, register
-// windows of 8 + 2c staged values per tap row as in the scores kernel.  Key tiles
-// past the CTA's last row only write zeros.
-template <int CQ, int CK>
-__global__ void __launch_bounds__(kThreadsB) bwd_adjoint_kernel(StripArgs p) {
+// The adjoint of one key-query convolution, for the rows of one head:
+//   out[i][j] = [j <= i] sum_{a,t} theta[a][t] G[i+a][j+t-c]
+//   dtheta[a][t] += sum over the own rows of G[i][j] X[i-a][j-(t-c)]
+// where G is the gradient at the convolution's output (zero past the diagonal)
+// and X its input.  MODE 0, the convolution before the softmax: G = dC, X =
+// Mask_0 S, out = dS written as hi / lo bf16 halves for the own rows (zeros for
+// the others).  MODE 1, the convolution after the softmax: G = Mask_0 dA', X = A,
+// out = dA in fp32 for every row below out_rows; the kernel also forms the
+// convolution itself on the own rows, A' = Mask_0(Conv2d(A)), into a strip.
+struct AdjArgs {
+  const float *G;       // [B][H][g_rows][pitch], row u <-> query r0 + u
+  int g_rows;
+  const float *X;       // [B][H][x_rows][pitch], row u <-> query x_base + u
+  int x_rows, x_base;
+  const float *theta;   // [H][c_q][c_k]
+  float *dtheta;        // [H][c_q][c_k] (or null)
+  int out_rows;         // MODE 1: rows of dA
+  __nv_bfloat16 *dS;    // MODE 0: [B][H][512][pitch]
+  float *dA;            // MODE 1: [B][H][out_rows][pitch]
+  float *Ac;            // MODE 1: A' of the own rows, [B][H][no][pitch]
+};
+
+// Step 4: CTA = one head and 16 rows u = 0 .. 255; thread (row, seg): 8
+// consecutive keys, register windows of the staged rows as in the scores kernel.
+// Key tiles past the CTA's last row only write zeros (MODE 0).
+template <int CQ, int CK, int MODE>
+__global__ void __launch_bounds__(kThreadsB) bwd_adjoint_kernel(StripArgs p, AdjArgs q) {
   constexpr int HALO = CQ - 1, C = CK / 2, TR = kRows + HALO, NT = CQ * CK, WIN = kSeg + 16;
   static_assert(C <= 8 && TR == kStagedRows, "window; dynamic shared memory sized for c_q = 6");
   extern __shared__ __align__(16) float dyn[];
-  // [2 stages]: dC rows and Mask_0 S rows, tile column cc = key j0 - 8 + cc
+  // [2 stages]: G rows and X rows, tile column cc = key j0 - 8 + cc
   float(*dct)[TR][kTilePitch] = reinterpret_cast<float(*)[TR][kTilePitch]>(dyn);
   float(*st)[TR][kTilePitch] = reinterpret_cast<float(*)[TR][kTilePitch]>(dyn + 2 * TR * kTilePitch);
   __shared__ float th[NT];
@@ -441,26 +485,31 @@ __global__ void __launch_bounds__(kThreadsB) bwd_adjoint_kernel(StripArgs p) {
   const int u0 = blockIdx.x * kRows, row = tile_row(threadIdx.x), seg = tile_seg(threadIdx.x);
   const int u = u0 + row, i = p.r0 + u;
   const bool own = u < p.g.no && i < p.L;
+  // rows whose convolution adjoint is written
+  const int n_out = MODE == 0 ? p.g.no : q.out_rows;
+  const bool outr = u < n_out && i < p.L;
   const int P = p.g.pitch;
-  const float *Dz = p.D + static_cast<long long>(z) * p.g.rc * P;
-  const float *Sz = p.S + static_cast<long long>(z) * kRowsT * P;
-  __nv_bfloat16 *dSz = p.dS + static_cast<long long>(z) * 2 * kRowsT * P;
-  for (int x = threadIdx.x; x < NT; x += kThreadsB) th[x] = p.theta[h * NT + x];
+  const float *Gz = q.G + static_cast<long long>(z) * q.g_rows * P;
+  const float *Xz = q.X + static_cast<long long>(z) * q.x_rows * P;
+  // X row of query i - a for tile row row + HALO - a: X rows start at u0 + xoff
+  const int xoff = p.r0 - q.x_base - HALO;
+  for (int x = threadIdx.x; x < NT; x += kThreadsB) th[x] = q.theta[h * NT + x];
   float dth[NT];
 #pragma unroll
   for (int x = 0; x < NT; ++x) dth[x] = 0.f;
-  const int i_last = min(p.L - 1, p.r0 + min(u0 + kRows - 1, p.g.no - 1));  // last own query of the CTA
+  const int i_last = min(p.L - 1, p.r0 + min(u0 + kRows - 1, n_out - 1));  // last written query of the CTA
   // key tiles with work (uniform over the CTA); the later ones only write zeros
-  const int nwork = u0 < p.g.no ? i_last / kKeyTile + 1 : 0;
+  const int nwork = u0 < n_out ? i_last / kKeyTile + 1 : 0;
   auto stage = [&](int tt) {
-    // dC rows u0 .. u0+TR-1 (queries r0 + u'), zero past the C rows, the sequence and the diagonal
-    stage_rows<TR>(dct[tt & 1], Dz, P, u0, p.g.rc, p.r0 + u0, p.L, tt * kKeyTile);
-    // Mask_0 S rows u0 .. u0+TR-1 of the S strip (queries r0 - HALO + su)
-    stage_rows<TR>(st[tt & 1], Sz, P, u0, kRowsT, p.r0 - HALO + u0, p.L, tt * kKeyTile);
+    // G rows u0 .. u0+TR-1 (queries r0 + u'), zero past its rows, the sequence and the diagonal
+    stage_rows<TR>(dct[tt & 1], Gz, P, u0, q.g_rows, p.r0 + u0, p.L, tt * kKeyTile);
+    // X rows of queries r0 + u0 - HALO .. (Mask_0 S, or A: zero past the diagonal)
+    stage_rows<TR>(st[tt & 1], Xz, P, u0 + xoff, q.x_rows, q.x_base + u0 + xoff, p.L, tt * kKeyTile);
   };
   if (nwork) stage(0);
   cp_async_commit();
-  for (int j0 = 0, tt = 0; j0 < p.Wp; j0 += kKeyTile, ++tt) {
+  const int jend = MODE == 0 ? p.Wp : (nwork ? nwork * kKeyTile : 0);
+  for (int j0 = 0, tt = 0; j0 < jend; j0 += kKeyTile, ++tt) {
     const int jb = j0 + kSeg * seg;
     const bool work = tt < nwork;
     if (work) {
@@ -469,15 +518,15 @@ __global__ void __launch_bounds__(kThreadsB) bwd_adjoint_kernel(StripArgs p) {
       cp_async_wait_prev();
       __syncthreads();
     }
-    float ds[kSeg];
+    float ds[kSeg], ac[kSeg];
 #pragma unroll
-    for (int x = 0; x < kSeg; ++x) ds[x] = 0.f;
-    if (work && own && jb <= i && jb < p.Wp) {
-      // dC[i][j] of the thread's keys (zero past the diagonal) for dtheta
+    for (int x = 0; x < kSeg; ++x) { ds[x] = 0.f; ac[x] = 0.f; }
+    if (work && outr && jb <= i && jb < p.Wp) {
+      // G[i][j] of the thread's keys (zero past the diagonal) for dtheta, own rows only
       const int bf = tt & 1;
       float gk[kSeg];
 #pragma unroll
-      for (int x = 0; x < kSeg; ++x) gk[x] = dct[bf][row][kSeg * seg + 8 + x];
+      for (int x = 0; x < kSeg; ++x) gk[x] = own ? dct[bf][row][kSeg * seg + 8 + x] : 0.f;
 #pragma unroll
       for (int a = 0; a < CQ; ++a) {
         // tile columns 8 seg .. 8 seg + 23: keys jb - 8 .. jb + 15
@@ -496,18 +545,24 @@ __global__ void __launch_bounds__(kThreadsB) bwd_adjoint_kernel(StripArgs p) {
           float acc = dth[a * CK + t];
 #pragma unroll
           for (int x = 0; x < kSeg; ++x) {
-            // dS[i][j] += theta[a][t] dC[i+a][j+t-c]: key jb + x + t - c = window x + 8 + t - c
+            // out[i][j] += theta[a][t] G[i+a][j+t-c]: key jb + x + t - c = window x + 8 + t - c
             ds[x] = fmaf(th_at, w[x + 8 + t - C], ds[x]);
-            // dtheta[a][t] += dC[i][j] Mask_0 S[i-a][j-(t-c)]: window x + 8 + c - t
+            // dtheta[a][t] += G[i][j] X[i-a][j-(t-c)]: window x + 8 + c - t
             acc = fmaf(gk[x], v[x + 8 + C - t], acc);
+            // MODE 1: A'[i][j] += theta[a][t] A[i-a][j-(t-c)] (the convolution itself)
+            if (MODE == 1) ac[x] = fmaf(th_at, v[x + 8 + C - t], ac[x]);
           }
           dth[a * CK + t] = acc;
         }
       }
 #pragma unroll
-      for (int x = 0; x < kSeg; ++x) ds[x] = jb + x <= i ? ds[x] : 0.f;
+      for (int x = 0; x < kSeg; ++x) {
+        ds[x] = jb + x <= i ? ds[x] : 0.f;
+        ac[x] = jb + x <= i ? ac[x] : 0.f;
+      }
     }
-    if (jb < p.Wp) {
+    if (MODE == 0 && jb < p.Wp) {
+      __nv_bfloat16 *dSz = q.dS + static_cast<long long>(z) * 2 * kRowsT * P;
       uint32_t hi[kSeg / 2], lo[kSeg / 2];
 #pragma unroll
       for (int x = 0; x < kSeg; x += 2) {
@@ -521,27 +576,262 @@ __global__ void __launch_bounds__(kThreadsB) bwd_adjoint_kernel(StripArgs p) {
       *reinterpret_cast<uint4 *>(dSz + static_cast<long long>(kRowsT + u) * P + jb) =
           make_uint4(lo[0], lo[1], lo[2], lo[3]);
     }
+    if (MODE == 1 && work && outr && jb <= i && jb < p.Wp) {
+      float *dst = q.dA + (static_cast<long long>(z) * q.out_rows + u) * P + jb;
+      reinterpret_cast<float4 *>(dst)[0] = make_float4(ds[0], ds[1], ds[2], ds[3]);
+      reinterpret_cast<float4 *>(dst)[1] = make_float4(ds[4], ds[5], ds[6], ds[7]);
+      if (own) {
+        float *ad = q.Ac + (static_cast<long long>(z) * p.g.no + u) * P + jb;
+        reinterpret_cast<float4 *>(ad)[0] = make_float4(ac[0], ac[1], ac[2], ac[3]);
+        reinterpret_cast<float4 *>(ad)[1] = make_float4(ac[4], ac[5], ac[6], ac[7]);
+      }
+    }
     if (work) __syncthreads();  // the buffer is restaged two tiles on
   }
-  if (p.dtheta) {
+  if (q.dtheta) {
 #pragma unroll
     for (int x = 0; x < NT; ++x) {
       float v = dth[x];
       for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-      if ((threadIdx.x & 31) == 0 && v != 0.f) atomicAdd(p.dtheta + h * NT + x, v);
+      if ((threadIdx.x & 31) == 0 && v != 0.f) atomicAdd(q.dtheta + h * NT + x, v);
     }
+  }
+}
+
+// The convolution after the softmax: per head group, the gradient at its output
+// G_s = Mask_0(sum_h w[h][s] dA''_h) (post mixing; dA''_s otherwise), rows u <->
+// query r0 + u, keys up to each row's query (the rest is never read).
+template <int CH>
+__global__ void __launch_bounds__(kThreadsB) bwd_post_grad_kernel(StripArgs p, float *G) {
+  const int G_ = p.H / CH, bg = blockIdx.y, b = bg / G_, g = bg % G_;
+  const int u = blockIdx.x * kRows + tile_row(threadIdx.x), seg = tile_seg(threadIdx.x);
+  const int i = p.r0 + u, P = p.g.pitch;
+  if (u >= p.g.rc || i >= p.L) return;
+  float wm[CH * CH];
+#pragma unroll
+  for (int x = 0; x < CH * CH; ++x) wm[x] = (p.hp == 2 && p.w) ? p.w[g * CH * CH + x] : (x % (CH + 1) == 0);
+  const long long z0 = static_cast<long long>(b) * p.H + g * CH;
+  for (int jb = kSeg * seg; jb <= i; jb += kKeyTile) {
+    float da[CH][kSeg];
+#pragma unroll
+    for (int h = 0; h < CH; ++h) {
+      const float *src = p.D + ((z0 + h) * p.g.rc + u) * P + jb;
+      const float4 a = reinterpret_cast<const float4 *>(src)[0], c = reinterpret_cast<const float4 *>(src)[1];
+      da[h][0] = a.x; da[h][1] = a.y; da[h][2] = a.z; da[h][3] = a.w;
+      da[h][4] = c.x; da[h][5] = c.y; da[h][6] = c.z; da[h][7] = c.w;
+    }
+#pragma unroll
+    for (int s2 = 0; s2 < CH; ++s2) {
+      float o[kSeg];
+#pragma unroll
+      for (int x = 0; x < kSeg; ++x) {
+        float v = 0.f;
+#pragma unroll
+        for (int h = 0; h < CH; ++h) v = fmaf(wm[h * CH + s2], da[h][x], v);
+        o[x] = jb + x <= i ? v : 0.f;
+      }
+      float *dst = G + ((z0 + s2) * p.g.rc + u) * P + jb;
+      reinterpret_cast<float4 *>(dst)[0] = make_float4(o[0], o[1], o[2], o[3]);
+      reinterpret_cast<float4 *>(dst)[1] = make_float4(o[4], o[5], o[6], o[7]);
+    }
+  }
+}
+
+// The convolution after the softmax, own rows: A''_h = sum_s w[h][s] A'_s (post
+// mixing; A'_h otherwise) as hi / lo halves for dV, and the post-mixing dw[h][s] +=
+// sum dA''_h A'_s.
+template <int CH>
+__global__ void __launch_bounds__(kThreadsB) bwd_post_mix_kernel(StripArgs p, const float *Ac) {
+  __shared__ float dwr[CH * CH];
+  const int G_ = p.H / CH, bg = blockIdx.y, b = bg / G_, g = bg % G_;
+  const int u = blockIdx.x * kRows + tile_row(threadIdx.x), seg = tile_seg(threadIdx.x);
+  const int i = p.r0 + u, P = p.g.pitch;
+  const bool own = u < p.g.no && i < p.L;
+  if (threadIdx.x < CH * CH) dwr[threadIdx.x] = 0.f;
+  __syncthreads();
+  float wm[CH * CH], dwp[CH * CH];
+#pragma unroll
+  for (int x = 0; x < CH * CH; ++x) {
+    wm[x] = (p.hp == 2 && p.w) ? p.w[g * CH * CH + x] : (x % (CH + 1) == 0);
+    dwp[x] = 0.f;
+  }
+  const long long z0 = static_cast<long long>(b) * p.H + g * CH;
+  if (own) {
+    for (int jb = kSeg * seg; jb <= i; jb += kKeyTile) {
+      float ac[CH][kSeg], da[CH][kSeg];
+#pragma unroll
+      for (int h = 0; h < CH; ++h) {
+        const float *sa = Ac + ((z0 + h) * p.g.no + u) * P + jb;
+        const float *sd = p.D + ((z0 + h) * p.g.rc + u) * P + jb;
+#pragma unroll
+        for (int x = 0; x < kSeg; x += 4) {
+          const float4 a = *reinterpret_cast<const float4 *>(sa + x), d = *reinterpret_cast<const float4 *>(sd + x);
+          ac[h][x] = a.x; ac[h][x + 1] = a.y; ac[h][x + 2] = a.z; ac[h][x + 3] = a.w;
+          da[h][x] = d.x; da[h][x + 1] = d.y; da[h][x + 2] = d.z; da[h][x + 3] = d.w;
+        }
+      }
+#pragma unroll
+      for (int h = 0; h < CH; ++h) {
+        uint32_t hi[kSeg / 2], lo[kSeg / 2];
+#pragma unroll
+        for (int x = 0; x < kSeg; x += 2) {
+          float y[2];
+#pragma unroll
+          for (int e = 0; e < 2; ++e) {
+            float v = 0.f;
+#pragma unroll
+            for (int s2 = 0; s2 < CH; ++s2) v = fmaf(wm[h * CH + s2], ac[s2][x + e], v);
+            y[e] = jb + x + e <= i ? v : 0.f;
+          }
+          __nv_bfloat16 h0, l0, h1, l1;
+          split_bf16(y[0], h0, l0);
+          split_bf16(y[1], h1, l1);
+          hi[x / 2] = static_cast<uint32_t>(__bfloat16_as_ushort(h0)) | (static_cast<uint32_t>(__bfloat16_as_ushort(h1)) << 16);
+          lo[x / 2] = static_cast<uint32_t>(__bfloat16_as_ushort(l0)) | (static_cast<uint32_t>(__bfloat16_as_ushort(l1)) << 16);
+        }
+        __nv_bfloat16 *ap = p.Ap + ((z0 + h) * 2 * kRowsT) * P;
+        *reinterpret_cast<uint4 *>(ap + static_cast<long long>(u) * P + jb) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
+        *reinterpret_cast<uint4 *>(ap + static_cast<long long>(kRowsT + u) * P + jb) =
+            make_uint4(lo[0], lo[1], lo[2], lo[3]);
+      }
+      if (p.hp == 2) {
+#pragma unroll
+        for (int h = 0; h < CH; ++h)
+#pragma unroll
+          for (int s2 = 0; s2 < CH; ++s2)
+#pragma unroll
+            for (int x = 0; x < kSeg; ++x)
+              if (jb + x <= i) dwp[h * CH + s2] = fmaf(da[h][x], ac[s2][x], dwp[h * CH + s2]);
+      }
+    }
+  }
+  if (p.hp == 2 && p.dw) {
+#pragma unroll
+    for (int x = 0; x < CH * CH; ++x) {
+      float v = dwp[x];
+      for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+      if ((threadIdx.x & 31) == 0) atomicAdd(&dwr[x], v);
+    }
+    __syncthreads();
+    if (threadIdx.x < CH * CH) atomicAdd(p.dw + g * CH * CH + threadIdx.x, dwr[threadIdx.x]);
+  }
+}
+
+// The softmax's backward with the convolution after the softmax: dA from the
+// adjoint kernel (rows u <-> query r0 + u), A from the A strip (row u + a_off),
+// D = sum_j dA A, dC = A (dA - D) in place of dA (pre mixing: dC'_h = A_h (dA_h -
+// D_h) mixed back to the sources, and dw[h][s] += sum dC'_h C_s over the own rows).
+template <int CH>
+__global__ void __launch_bounds__(kThreadsB) bwd_post_softmax_kernel(StripArgs p, float *dA, int da_rows, int a_off) {
+  __shared__ float dwr[CH * CH];
+  const int G_ = p.H / CH, bg = blockIdx.y, b = bg / G_, g = bg % G_;
+  const int u = blockIdx.x * kRows + tile_row(threadIdx.x), seg = tile_seg(threadIdx.x);
+  const int i = p.r0 + u, P = p.g.pitch;
+  const bool valid = u < da_rows && i < p.L, own = valid && u < p.g.no;
+  if (threadIdx.x < CH * CH) dwr[threadIdx.x] = 0.f;
+  __syncthreads();
+  float wm[CH * CH], dwp[CH * CH], Dp[CH];
+#pragma unroll
+  for (int x = 0; x < CH * CH; ++x) {
+    wm[x] = (p.hp == 1 && p.w) ? p.w[g * CH * CH + x] : (x % (CH + 1) == 0);
+    dwp[x] = 0.f;
+  }
+#pragma unroll
+  for (int h = 0; h < CH; ++h) Dp[h] = 0.f;
+  const long long z0 = static_cast<long long>(b) * p.H + g * CH;
+  auto load8 = [&](const float *src, float (&o)[kSeg]) {
+    const float4 a = reinterpret_cast<const float4 *>(src)[0], c = reinterpret_cast<const float4 *>(src)[1];
+    o[0] = a.x; o[1] = a.y; o[2] = a.z; o[3] = a.w; o[4] = c.x; o[5] = c.y; o[6] = c.z; o[7] = c.w;
+  };
+  if (valid) {
+    for (int jb = kSeg * seg; jb <= i; jb += kKeyTile) {
+#pragma unroll
+      for (int h = 0; h < CH; ++h) {
+        float a[kSeg], d[kSeg];
+        load8(p.A + ((z0 + h) * p.g.rc + u + a_off) * P + jb, a);
+        load8(dA + ((z0 + h) * da_rows + u) * P + jb, d);
+#pragma unroll
+        for (int x = 0; x < kSeg; ++x)
+          if (jb + x <= i) Dp[h] = fmaf(d[x], a[x], Dp[h]);
+      }
+    }
+  }
+  float Dr[CH];
+#pragma unroll
+  for (int h = 0; h < CH; ++h) {
+    float v = Dp[h];
+#pragma unroll
+    for (int o : {1, 2, 8, 16}) v += __shfl_xor_sync(0xffffffffu, v, o);
+    Dr[h] = v;
+  }
+  if (valid) {
+    for (int jb = kSeg * seg; jb <= i; jb += kKeyTile) {
+      float a[CH][kSeg], d[CH][kSeg], dc[CH][kSeg];
+#pragma unroll
+      for (int h = 0; h < CH; ++h) {
+        load8(p.A + ((z0 + h) * p.g.rc + u + a_off) * P + jb, a[h]);
+        load8(dA + ((z0 + h) * da_rows + u) * P + jb, d[h]);
+      }
+      if (p.hp == 1) {
+#pragma unroll
+        for (int x = 0; x < kSeg; ++x) {
+          float dcp[CH];
+#pragma unroll
+          for (int h = 0; h < CH; ++h) dcp[h] = a[h][x] * (d[h][x] - Dr[h]);
+#pragma unroll
+          for (int s2 = 0; s2 < CH; ++s2) {
+            float v = 0.f;
+#pragma unroll
+            for (int h = 0; h < CH; ++h) v = fmaf(wm[h * CH + s2], dcp[h], v);
+            dc[s2][x] = jb + x <= i ? v : 0.f;
+          }
+          if (own && jb + x <= i) {
+#pragma unroll
+            for (int s2 = 0; s2 < CH; ++s2) {
+              const float cs = p.Cpre[((z0 + s2) * p.g.rc + u + a_off) * P + jb + x];
+#pragma unroll
+              for (int h = 0; h < CH; ++h) dwp[h * CH + s2] = fmaf(dcp[h], cs, dwp[h * CH + s2]);
+            }
+          }
+        }
+      } else {
+#pragma unroll
+        for (int h = 0; h < CH; ++h)
+#pragma unroll
+          for (int x = 0; x < kSeg; ++x) dc[h][x] = jb + x <= i ? a[h][x] * (d[h][x] - Dr[h]) : 0.f;
+      }
+#pragma unroll
+      for (int h = 0; h < CH; ++h) {
+        float *dst = dA + ((z0 + h) * da_rows + u) * P + jb;
+        reinterpret_cast<float4 *>(dst)[0] = make_float4(dc[h][0], dc[h][1], dc[h][2], dc[h][3]);
+        reinterpret_cast<float4 *>(dst)[1] = make_float4(dc[h][4], dc[h][5], dc[h][6], dc[h][7]);
+      }
+    }
+  }
+  if (p.hp == 1 && p.dw) {
+#pragma unroll
+    for (int x = 0; x < CH * CH; ++x) {
+      float v = dwp[x];
+      for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+      if ((threadIdx.x & 31) == 0) atomicAdd(&dwr[x], v);
+    }
+    __syncthreads();
+    if (threadIdx.x < CH * CH) atomicAdd(p.dw + g * CH * CH + threadIdx.x, dwr[threadIdx.x]);
   }
 }
 
 int scores_smem(int ch) { return 2 * ch * kStagedRows * kTilePitch * 4; }
 int adjoint_smem() { return 2 * 2 * kStagedRows * kTilePitch * 4; }
 
+// Rows of a block.  Without the convolution after the softmax: own rows NO = 256 -
+// 2 (c_q - 1), C / dC rows NO + c_q - 1.  With it, one more halo of c_q - 1 rows
+// on each side: own rows 256 - 3 (c_q - 1), A rows (and dA'' rows) NO + 2 (c_q - 1).
 Geo geometry(const BwdArgs &a) {
   Geo g;
   g.halo = a.cq - 1;
   g.c = a.ck / 2;
-  g.no = kRowsT - 2 * g.halo;
-  g.rc = g.no + g.halo;
+  g.no = kRowsT - (a.kqp ? 3 : 2) * g.halo;
+  g.rc = g.no + (a.kqp ? 2 : 1) * g.halo;
   g.pitch = (a.L + 63) / 64 * 64;
   return g;
 }
@@ -574,24 +864,29 @@ BgTensor strip_tensor(const void *base, const BwdArgs &a, int rows, int pitch) {
 }  // namespace
 
 bool attn_bwd_tc_supported(const BwdArgs &a) {
-  return a.dtype == 1 && (a.d == 64 || a.d == 96 || a.d == 128) && a.cq == 6 && a.ck == 11 && a.kq == 1 && !a.kqp &&
-         (a.hp == 0 || a.ch == 2) && a.rs % 8 == 0 &&
+  return a.dtype == 1 && (a.d == 64 || a.d == 96 || a.d == 128) && a.cq == 6 && a.ck == 11 && a.kq == 1 &&
+         (!a.kqp || a.theta_post) && (a.hp == 0 || a.ch == 2) && a.rs % 8 == 0 &&
          (reinterpret_cast<uintptr_t>(a.q) | reinterpret_cast<uintptr_t>(a.k) | reinterpret_cast<uintptr_t>(a.v) |
           reinterpret_cast<uintptr_t>(a.dout)) % 16 == 0 &&
          (reinterpret_cast<uintptr_t>(a.dq) | reinterpret_cast<uintptr_t>(a.dk) | reinterpret_cast<uintptr_t>(a.dv)) %
                  16 == 0;
 }
 
-size_t attn_bwd_tc_workspace_bytes(int B, int H, int L, int cq, int hp) {
+size_t attn_bwd_tc_workspace_bytes(int B, int H, int L, int cq, int hp, int kqp) {
   const size_t Z = static_cast<size_t>(B) * H, P = (static_cast<size_t>(L) + 63) / 64 * 64;
-  const size_t rc = kRowsT - (cq - 1);
-  return up256(Z * kRowsT * P * 4) + 2 * up256(Z * rc * P * 4) + (hp == 1 ? up256(Z * rc * P * 4) : 0) +
-         2 * up256(Z * 2 * kRowsT * P * 2);
+  const size_t halo = static_cast<size_t>(cq - 1);
+  const size_t no = kRowsT - (kqp ? 3 : 2) * halo, rc = no + (kqp ? 2 : 1) * halo;
+  size_t b = up256(Z * kRowsT * P * 4) + 2 * up256(Z * rc * P * 4) + (hp == 1 ? up256(Z * rc * P * 4) : 0) +
+             2 * up256(Z * 2 * kRowsT * P * 2);
+  // with the convolution after the softmax: its output gradient G, dA (then dC) and A'
+  if (kqp) b += up256(Z * rc * P * 4) + up256(Z * (no + halo) * P * 4) + up256(Z * no * P * 4);
+  return b;
 }
 
 cudaError_t launch_attn_bwd_tc(const BwdArgs &a, void *ws) {
   const Geo g = geometry(a);
   const size_t Z = static_cast<size_t>(a.B) * a.H, P = g.pitch;
+  const int post = a.kqp ? 1 : 0, ndc = g.no + g.halo;  // rows of dA / dC with post
   char *w = static_cast<char *>(ws);
   float *S = reinterpret_cast<float *>(w);
   w += up256(Z * kRowsT * P * 4);
@@ -607,6 +902,15 @@ cudaError_t launch_attn_bwd_tc(const BwdArgs &a, void *ws) {
   __nv_bfloat16 *dS = reinterpret_cast<__nv_bfloat16 *>(w);
   w += up256(Z * 2 * kRowsT * P * 2);
   __nv_bfloat16 *Ap = reinterpret_cast<__nv_bfloat16 *>(w);
+  w += up256(Z * 2 * kRowsT * P * 2);
+  float *Gp = nullptr, *dAp = nullptr, *Ac = nullptr;
+  if (post) {
+    Gp = reinterpret_cast<float *>(w);
+    w += up256(Z * g.rc * P * 4);
+    dAp = reinterpret_cast<float *>(w);
+    w += up256(Z * ndc * P * 4);
+    Ac = reinterpret_cast<float *>(w);
+  }
 
   cudaStream_t st = a.stream;
   const size_t n = static_cast<size_t>(a.B) * a.L * a.H * a.d;
@@ -615,13 +919,16 @@ cudaError_t launch_attn_bwd_tc(const BwdArgs &a, void *ws) {
                                 scores_smem(2))) != cudaSuccess ||
       (e = cudaFuncSetAttribute(bwd_scores_kernel<6, 11, 1>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                 scores_smem(1))) != cudaSuccess ||
-      (e = cudaFuncSetAttribute(bwd_adjoint_kernel<6, 11>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+      (e = cudaFuncSetAttribute(bwd_adjoint_kernel<6, 11, 0>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                adjoint_smem())) != cudaSuccess ||
+      (e = cudaFuncSetAttribute(bwd_adjoint_kernel<6, 11, 1>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                 adjoint_smem())) != cudaSuccess)
     return e;
   if ((e = cudaMemsetAsync(a.dk, 0, n * 4, st)) != cudaSuccess) return e;
   if ((e = cudaMemsetAsync(a.dv, 0, n * 4, st)) != cudaSuccess) return e;
-  if (a.dtheta && (e = cudaMemsetAsync(a.dtheta, 0, static_cast<size_t>(a.H) * a.cq * a.ck * 4, st)) != cudaSuccess)
-    return e;
+  const size_t nth = static_cast<size_t>(a.H) * a.cq * a.ck * 4;
+  if (a.dtheta && (e = cudaMemsetAsync(a.dtheta, 0, nth, st)) != cudaSuccess) return e;
+  if (post && a.dtheta_post && (e = cudaMemsetAsync(a.dtheta_post, 0, nth, st)) != cudaSuccess) return e;
   if (a.hp && a.dw && (e = cudaMemsetAsync(a.dw, 0, static_cast<size_t>(a.H) * a.ch * 4, st)) != cudaSuccess)
     return e;
   // A'' is written for the own rows up to each row's query only: the rest stays zero
@@ -640,6 +947,7 @@ cudaError_t launch_attn_bwd_tc(const BwdArgs &a, void *ws) {
   sp.theta = a.theta; sp.w = a.hp ? a.w : nullptr;
   sp.S = S; sp.Cpre = Cpre; sp.A = A; sp.D = D; sp.dS = dS; sp.Ap = Ap;
   sp.dtheta = a.dtheta; sp.dw = a.hp ? a.dw : nullptr;
+  sp.post = post;
 
   auto K_major = [](int pos_row, int off_mn, int off_k) { return BgOperand{0, pos_row, off_mn, off_k, 0, 0}; };
   auto MN_major = [](int pos_row, int off_mn, int off_k) { return BgOperand{1, pos_row, off_mn, off_k, 0, 0}; };
@@ -648,31 +956,70 @@ cudaError_t launch_attn_bwd_tc(const BwdArgs &a, void *ws) {
     o.period_shift = shift;
     return o;
   };
+  auto check = [&]() { return cudaGetLastError(); };
+  const int s_lead = (post ? 2 : 1) * g.halo;  // S strip row 0 is query r0 - s_lead
   for (int r0 = 0; r0 < a.L; r0 += g.no) {
+    // keys 0 .. W-1: up to the last row of the block's maps
     const int W = std::min(a.L, r0 + g.rc), Wp = (W + 63) / 64 * 64;
     sp.r0 = r0; sp.W = W; sp.Wp = Wp;
-    // 1. S strip = s Q K^T: rows r0 - halo .. r0 - halo + 255, keys 0 .. W-1
+    // 1. S strip = s Q K^T: rows r0 - s_lead .. r0 - s_lead + 255, keys 0 .. W-1
     BgArgs ga = {};
     ga.Z = static_cast<int>(Z); ga.H = a.H; ga.err = err;
     ga.M = kRowsT; ga.N = W; ga.K = a.d; ga.alpha = a.scale; ga.accumulate = 0;
     ga.C = S; ga.sm = g.pitch; ga.sh = static_cast<long long>(kRowsT) * g.pitch; ga.sb = ga.sh * a.H;
-    ga.a = K_major(2, r0 - g.halo, 0); ga.b = K_major(2, 0, 0);
+    ga.a = K_major(2, r0 - s_lead, 0); ga.b = K_major(2, 0, 0);
     if ((e = launch_gemm_batched(tq, tk, ga, st)) != cudaSuccess) return e;
     // 2. dA'' strip = dO V^T: rows r0 .. r0 + rc - 1
     ga.M = g.rc; ga.alpha = 1.f;
     ga.C = D; ga.sh = static_cast<long long>(g.rc) * g.pitch; ga.sb = ga.sh * a.H;
     ga.a = K_major(2, r0, 0); ga.b = K_major(2, 0, 0);
     if ((e = launch_gemm_batched(tdo, tv, ga, st)) != cudaSuccess) return e;
-    // 3. convolution, mixing, softmax; dC, D, dw, A''
-    const dim3 grid2((g.rc + kRows - 1) / kRows, a.B * G);
+    // 3. convolution, mixing, softmax (rows r0 .. without the convolution after the
+    //    softmax, with its backward fused; with it, rows r0 - halo .., the weights only)
+    const dim3 grid_g((g.rc + kRows - 1) / kRows, a.B * G);
+    StripArgs s3 = sp;
+    if (post) s3.r0 = r0 - g.halo;
     if (ch == 2)
-      bwd_scores_kernel<6, 11, 2><<<grid2, kThreadsB, scores_smem(2), st>>>(sp);
+      bwd_scores_kernel<6, 11, 2><<<grid_g, kThreadsB, scores_smem(2), st>>>(s3);
     else
-      bwd_scores_kernel<6, 11, 1><<<grid2, kThreadsB, scores_smem(1), st>>>(sp);
-    if ((e = cudaGetLastError()) != cudaSuccess) return e;
-    // 4. dS (hi / lo), dtheta
-    bwd_adjoint_kernel<6, 11><<<dim3(kRowsT / kRows, static_cast<unsigned>(Z)), kThreadsB, adjoint_smem(), st>>>(sp);
-    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+      bwd_scores_kernel<6, 11, 1><<<grid_g, kThreadsB, scores_smem(1), st>>>(s3);
+    if ((e = check()) != cudaSuccess) return e;
+    const dim3 grid_h(kRowsT / kRows, static_cast<unsigned>(Z));
+    if (post) {
+      // 3a. the gradient at the post-softmax convolution's output, G = Mask_0(mix back dA'')
+      if (ch == 2)
+        bwd_post_grad_kernel<2><<<grid_g, kThreadsB, 0, st>>>(sp, Gp);
+      else
+        bwd_post_grad_kernel<1><<<grid_g, kThreadsB, 0, st>>>(sp, Gp);
+      if ((e = check()) != cudaSuccess) return e;
+      // 3b. its adjoint dA (rows r0 .. r0 + no + halo - 1), dtheta_post, and A' of the own rows
+      AdjArgs q1 = {};
+      q1.G = Gp; q1.g_rows = g.rc;
+      q1.X = A; q1.x_rows = g.rc; q1.x_base = r0 - g.halo;
+      q1.theta = a.theta_post; q1.dtheta = a.dtheta_post;
+      q1.out_rows = ndc; q1.dA = dAp; q1.Ac = Ac;
+      bwd_adjoint_kernel<6, 11, 1><<<grid_h, kThreadsB, adjoint_smem(), st>>>(sp, q1);
+      if ((e = check()) != cudaSuccess) return e;
+      // 3c. A'' = mix(A') for dV, and the post-mixing dw
+      if (ch == 2)
+        bwd_post_mix_kernel<2><<<grid_g, kThreadsB, 0, st>>>(sp, Ac);
+      else
+        bwd_post_mix_kernel<1><<<grid_g, kThreadsB, 0, st>>>(sp, Ac);
+      if ((e = check()) != cudaSuccess) return e;
+      // 3d. the softmax's backward: dC in place of dA (pre mixing: mixed back, dw)
+      if (ch == 2)
+        bwd_post_softmax_kernel<2><<<grid_g, kThreadsB, 0, st>>>(sp, dAp, ndc, g.halo);
+      else
+        bwd_post_softmax_kernel<1><<<grid_g, kThreadsB, 0, st>>>(sp, dAp, ndc, g.halo);
+      if ((e = check()) != cudaSuccess) return e;
+    }
+    // 4. dS (hi / lo), dtheta: the adjoint of the convolution before the softmax
+    AdjArgs q0 = {};
+    q0.G = post ? dAp : D; q0.g_rows = post ? ndc : g.rc;
+    q0.X = S; q0.x_rows = kRowsT; q0.x_base = r0 - s_lead;
+    q0.theta = a.theta; q0.dtheta = a.dtheta; q0.dS = dS;
+    bwd_adjoint_kernel<6, 11, 0><<<grid_h, kThreadsB, adjoint_smem(), st>>>(sp, q0);
+    if ((e = check()) != cudaSuccess) return e;
     // 5. dQ rows r0 .. r0 + no - 1 = s dS K: K runs over the keys twice, the hi
     //    rows of dS against K, then its lo rows (256 further) against K again
     const int own = std::min(g.no, a.L - r0);

@@ -74,7 +74,7 @@ int attn_bwd_simt_pick_rows(const BwdArgs &a);  // 0 if nothing fits
 // configurations it serves, its workspace (strips of every head for one query
 // block), and the launch.
 bool attn_bwd_tc_supported(const BwdArgs &a);
-size_t attn_bwd_tc_workspace_bytes(int B, int H, int L, int cq, int hp);
+size_t attn_bwd_tc_workspace_bytes(int B, int H, int L, int cq, int hp, int kqp);
 cudaError_t launch_attn_bwd_tc(const BwdArgs &a, void *ws);
 cudaError_t launch_attn_bwd_simt(const BwdArgs &a);
 // With the post-softmax convolution (kqp == 1).

@@ -216,8 +216,8 @@ bool bwd_supported(const BwdArgs &a) {
 // (pointer alignment aside).
 size_t bwd_tc_bytes(const mta_cfg *c) {
   const bool shape = c->dtype == MTA_BF16 && (c->d == 64 || c->d == 96 || c->d == 128) && c->c_q == 6 && c->c_k == 11 &&
-                     c->kq_place == MTA_PRE && !c->kq_post && (c->head_place == MTA_OFF || c->c_h == 2);
-  return shape ? attn_bwd_tc_workspace_bytes(c->B, c->H, c->L, c->c_q, c->head_place) : 0;
+                     c->kq_place == MTA_PRE && (c->head_place == MTA_OFF || c->c_h == 2);
+  return shape ? attn_bwd_tc_workspace_bytes(c->B, c->H, c->L, c->c_q, c->head_place, c->kq_post) : 0;
 }
 
 // Which backward serves `a`: path 0 the tensor-core one where it applies and
