@@ -29,7 +29,15 @@
 //   3. C, softmax, then dC, D, dw, A''             bwd_scores_kernel (CUDA cores)
 //   4. dS, dtheta                                  bwd_adjoint_kernel
 //   5. dQ rows (=), dK, dV (+=)                    batched GEMMs
-// dS and A'' enter the GEMMs of step 6 as two bf16 halves, hi = bf16(x) and
+// With the convolution after the softmax, A' = Mask_0(Conv2d_theta_post A) sits
+// between the softmax and the post-softmax mixing; its adjoint reads G = dL/dA'
+// c_q-1 rows below each row and A' reads A c_q-1 rows above, so a block carries a
+// second halo: NO = 256 - 3 (c_q - 1), S from row r0 - 2 (c_q - 1), the weights A
+// from r0 - (c_q - 1).  Step 3 then writes the normalised weights only, and four
+// kernels follow it: G (bwd_post_grad_kernel), dA = its adjoint with dtheta_post
+// and A' of the own rows (bwd_adjoint_kernel, mode 1), A'' and the post-mixing dw
+// (bwd_post_mix_kernel), dC and D (bwd_post_softmax_kernel).
+// dS and A'' enter the GEMMs of step 5 as two bf16 halves, hi = bf16(x) and
 // lo = bf16(x - hi), summed by two GEMMs into the same fp32 output: the operands
 // then carry about 16 significant bits and the gradients stay within fp32
 // tolerance of the CUDA-core backward.  The other GEMM operands (q, k, v, dO) are
