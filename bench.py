@@ -76,9 +76,9 @@ def uses_contraction(wl: synth.Workload) -> bool:
 
 def kq_kernel_name(wl: synth.Workload) -> str:
     """The contraction kernel the library launches: the CTA-pair form for sequences of
-    8192 and more (d = 128, or d = 64 with post-softmax mixing; no post-softmax
+    4096 and more (d = 128, or d = 64 with post-softmax mixing; no post-softmax
     convolution), else the one-CTA form."""
-    pair = (wl.L >= 8192 and not wl.kq_post and
+    pair = (wl.L >= 4096 and not wl.kq_post and
             ((wl.d == 128 and wl.head_place in (synth.OFF, synth.POST)) or
              (wl.d == 64 and wl.head_place == synth.POST)))
     return "attn_kq_pair_kernel" if pair else "attn_kq_kernel"

@@ -97,15 +97,15 @@ def test_workspace_query(L):
     assert L.mta_attn_workspace_bytes(ctypes.byref(post_nomix)) == 256 + kq0 + up(B * H * Ls * cq * d * 2)
     post_off = good_cfg(kq_post=1, kq_place=mta.OFF)   # CUDA-core kernel only
     assert L.mta_attn_workspace_bytes(ctypes.byref(post_off)) == 256
-    # L >= 8192: the CTA-pair kernel serves d = 64 with post-softmax mixing; its
+    # L >= 4096: the CTA-pair kernel serves d = 64 with post-softmax mixing; its
     # mixing scratch is per (batch, head group, query tile): two heads x two parts
     # of d x 128 fp32, then a counter per slot
-    Ll = 8192
-    long_cfg = good_cfg(L=Ll)
-    slots = B * (H // 2) * (Ll // 128)
-    xg_pair = slots * 2 * 2 * d * 128 * 4 + up(slots * 4)
-    kq_long = up(B * H * cq * Ll * d * 2) + up(B * H * Ll * 4) + up(B * H * Ll * M * 4) + xg_pair
-    assert L.mta_attn_workspace_bytes(ctypes.byref(long_cfg)) == 256 + kq_long
+    for Ll in (4096, 8192):
+        long_cfg = good_cfg(L=Ll)
+        slots = B * (H // 2) * (Ll // 128)
+        xg_pair = slots * 2 * 2 * d * 128 * 4 + up(slots * 4)
+        kq_long = up(B * H * cq * Ll * d * 2) + up(B * H * Ll * 4) + up(B * H * Ll * M * 4) + xg_pair
+        assert L.mta_attn_workspace_bytes(ctypes.byref(long_cfg)) == 256 + kq_long
     assert L.mta_attn_workspace_bytes(ctypes.byref(good_cfg(c_k=4))) == 0
     assert L.mta_attn_workspace_bytes(None) == 0
 

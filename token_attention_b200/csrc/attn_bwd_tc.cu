@@ -109,16 +109,6 @@ constexpr int kStagedRows = kRows + 5;     // rows staged for c_q = 6 (dynamic s
 __device__ __forceinline__ int tile_row(int tid) { return 2 * (tid >> 5) + ((tid >> 2) & 1); }
 __device__ __forceinline__ int tile_seg(int tid) { return (tid & 3) | (((tid & 31) >> 3) << 2); }
 
-// Asynchronous 16-byte copy global -> shared of the first src_bytes bytes (0 ..
-// 16), the rest of the 16 zero-filled; src must be a valid address even when
-// src_bytes is 0.
-__device__ __forceinline__ void cp_async16(void *dst, const void *src, int src_bytes) {
-  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(smem_u32(dst)), "l"(src), "r"(src_bytes)
-               : "memory");
-}
-__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
-__device__ __forceinline__ void cp_async_wait_prev() { asm volatile("cp.async.wait_group 1;" ::: "memory"); }
-
 // Starts staging TR rows of a strip into tile[TR][kTilePitch]: tile row r gets
 // strip row row0 + r (its query q0 + r; zeros once the strip row reaches nrows or
 // the query reaches L), tile column cc key j0 - 8 + cc, zero for a key below 0 or

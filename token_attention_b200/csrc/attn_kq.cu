@@ -661,7 +661,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int zn = G::DH1 == G::DH ? G::DH : (wg ? G::DH1 : G::DH);  // a constant unless d = 96
     const uint32_t tl = tmem + (static_cast<uint32_t>(32 * q4) << 16);
     const float sc0 = p.qk_scale * kLog2e;
-    float *crow = Cs + (wg * G::BM + r_) * G::W;
+    float *brow = Cs + r_ * G::W;             // this row of the item's band table
 
     // Stage item r: its query rows in fp16 (scaled down by a power of 2 only if
     // |q| > 2^14), the past dot products of its staged rows and its kernel taps.
@@ -857,9 +857,13 @@ __global__ void __launch_bounds__(kThreads, 1)
       // tap over the kept taps, from the dot products (key (i-a) - m, m = dd - a + t - c):
       //   Mask_0: taps with m >= 0; exact indicator: taps with key <= i, i.e. t >= c - dd
       //   C[i][i-dd] = s * sum_{kept a,t} theta[a][t] q[i-a] . k[i-a-m]   (acc[dd] / s)
-      auto band_acc = [&](float (&acc)[G::W]) {
+      // Each warpgroup takes half of the W diagonals of its row, once per item, into
+      // the band table brow[dd] (log2 units; read by both warpgroups after a barrier).
+      auto band_part = [&](auto lo_c) {
+        constexpr int LO = decltype(lo_c)::value, NB = LO == 0 ? (G::W + 1) / 2 : G::W - (G::W + 1) / 2;
+        float acc[NB];
 #pragma unroll
-        for (int dd = 0; dd < G::W; ++dd) acc[dd] = 0.f;
+        for (int e = 0; e < NB; ++e) acc[e] = 0.f;
 #pragma unroll
         for (int sc = 0; sc < G::NSRC; ++sc)
 #pragma unroll
@@ -874,16 +878,22 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int tp = 0; tp < CK; ++tp) {
             const float thv = th[a * CK + tp] * wmix[sc];
 #pragma unroll
-            for (int dd = 0; dd < G::W; ++dd) {
-              const int m = dd - a + tp - G::C;
+            for (int e = 0; e < NB; ++e) {
+              const int dd = LO + e, m = dd - a + tp - G::C;
               const bool kept = EXACT ? tp >= G::C - dd : m >= 0;
-              if (kept && m + G::OFF >= 0 && m + G::OFF < G::M) acc[dd] = fmaf(thv, vr[m + G::OFF], acc[dd]);
+              if (kept && m + G::OFF >= 0 && m + G::OFF < G::M) acc[e] = fmaf(thv, vr[m + G::OFF], acc[e]);
             }
           }
         }
+#pragma unroll
+        for (int e = 0; e < NB; ++e) brow[LO + e] = acc[e] * sc0;
       };
       float m_run = -INFINITY, l_run = 0.f;
       float mm = INFINITY;  // POST: log2 of (row max x row sum), final after the first pass
+      // column factors two slots ahead: loaded a whole tile before they are stored
+      float fpre[G::NSRC];
+#pragma unroll
+      for (int sc = 0; sc < G::NSRC; ++sc) fpre[sc] = st_id < G::BN ? fac_next(sc, 0) : 0.f;
       for (int sl = 0; sl < nsl; ++sl, ++T) {
         const int t = POST ? sl % n_kv : sl;
         const bool pass2 = POST && sl >= n_kv;
@@ -894,10 +904,24 @@ __global__ void __launch_bounds__(kThreads, 1)
           const float l_tot = l_run + red[(4 + (wg ^ 1)) * G::BM + r_];
           mm = (row_ok && l_tot > 0.f) ? m_run + log2f(l_tot) : INFINITY;
         }
-        // next key tile's column factors (stored before this tile's barrier, read after it)
+        // the band table of the item, while the first C is computed
+        if (sl == 0) {
+          if (row_ok) {
+            if (wg == 0)
+              band_part(std::integral_constant<int, 0>());
+            else
+              band_part(std::integral_constant<int, (G::W + 1) / 2>());
+          }
+          named_bar_sync(kBarAll, kSmThreads);
+        }
+        // next key tile's column factors (stored before this tile's barrier, read after
+        // it), and the load of the one after
         float fnext[G::NSRC];
 #pragma unroll
-        for (int sc = 0; sc < G::NSRC; ++sc) fnext[sc] = st_id < G::BN ? fac_next(sc, sl) : 0.f;
+        for (int sc = 0; sc < G::NSRC; ++sc) {
+          fnext[sc] = fpre[sc];
+          fpre[sc] = st_id < G::BN ? fac_next(sc, sl + 1) : 0.f;
+        }
         if constexpr (G::CDB)
           mbar_wait(c_fullb[T & 1], (T >> 1) & 1, abort_flag, p.err);
         else
@@ -909,25 +933,20 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
         for (int sc = 0; sc < G::NSRC; ++sc) {
           const float4 *f4 = reinterpret_cast<const float4 *>(facs + (sc * 2 + (T & 1)) * G::BN + cb);
+          // both 32-column halves in flight before one wait
+          uint32_t u32[2][32];
+          tmem_ld32(tl + G::C_COL + cbuf + 128 * sc + cb, u32[0]);
+          tmem_ld32(tl + G::C_COL + cbuf + 128 * sc + cb + 32, u32[1]);
+          tmem_wait_ld();
 #pragma unroll
-          for (int c0 = 0; c0 < G::HALF; c0 += 32) {
-            uint32_t u32[32];
-            tmem_ld32(tl + G::C_COL + cbuf + 128 * sc + cb + c0, u32);
-            float4 f[8];
+          for (int i = 0; i < G::HALF / 4; ++i) {
+            float4 f = f4[i];
+            if (G::NSRC == 2) { f.x *= wmix[sc]; f.y *= wmix[sc]; f.z *= wmix[sc]; f.w *= wmix[sc]; }
 #pragma unroll
-            for (int i = 0; i < 8; ++i) {
-              f[i] = f4[c0 / 4 + i];
-              if (G::NSRC == 2) { f[i].x *= wmix[sc]; f[i].y *= wmix[sc]; f[i].z *= wmix[sc]; f[i].w *= wmix[sc]; }
-            }
-            tmem_wait_ld();
-#pragma unroll
-            for (int i = 0; i < 8; ++i) {
-#pragma unroll
-              for (int e = 0; e < 4; ++e) {
-                const float fe = e == 0 ? f[i].x : e == 1 ? f[i].y : e == 2 ? f[i].z : f[i].w;
-                const float x = __uint_as_float(u32[4 * i + e]) * fe;
-                cv[c0 + 4 * i + e] = sc == 0 ? x : cv[c0 + 4 * i + e] + x;
-              }
+            for (int e = 0; e < 4; ++e) {
+              const float fe = e == 0 ? f.x : e == 1 ? f.y : e == 2 ? f.z : f.w;
+              const float x = __uint_as_float(u32[i / 8][4 * (i % 8) + e]) * fe;
+              cv[4 * i + e] = sc == 0 ? x : cv[4 * i + e] + x;
             }
           }
         }
@@ -942,14 +961,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         const int dmax = qi - j0 - cb;  // i - j for this warpgroup's first column
         if (row_ok && dmax >= 0 && dmax - (G::W - 1) < G::HALF) {
-          float acc[G::W];
-          band_acc(acc);
-#pragma unroll
-          for (int dd = 0; dd < G::W; ++dd) crow[dd] = acc[dd] * sc0;
 #pragma unroll
           for (int jj = 0; jj < G::HALF; ++jj) {
             const int dd = dmax - jj;
-            if (static_cast<unsigned>(dd) < static_cast<unsigned>(G::W)) cv[jj] = crow[dd];
+            if (static_cast<unsigned>(dd) < static_cast<unsigned>(G::W)) cv[jj] = brow[dd];
           }
         }
         // Mask_-inf: keys after the query (only tiles reaching past the tile's first row)
@@ -1065,11 +1080,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       if constexpr (POST) {
         // normalised weights of the c keys ending at each row's diagonal, for the band
         if (wg == 0) {
-          float acc[G::W];
-          band_acc(acc);
 #pragma unroll
           for (int dl = 0; dl < G::C; ++dl)
-            Dg[r_ * G::C + dl] = (row_ok && qi - dl >= 0) ? ex2(acc[dl] * sc0 - mm) : 0.f;
+            Dg[r_ * G::C + dl] = (row_ok && qi - dl >= 0) ? ex2(brow[dl] - mm) : 0.f;
         }
       }
       // the next item's queries, dot products and taps, while this item's last P V runs

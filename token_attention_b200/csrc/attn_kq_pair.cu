@@ -35,6 +35,7 @@
 #include <cuda.h>
 
 #include <algorithm>
+#include <type_traits>
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 #include <math.h>
@@ -52,13 +53,15 @@ constexpr int kThreads = 352;
 constexpr int kSmThreads = 256;
 constexpr int kTmaWarp = 8, kMmaWarp = 9, kTma2Warp = 10;
 constexpr int kBarAll = 1;
+constexpr int kBarP = 2;   // the softmax warps of a CTA, before its one arrival on P
 constexpr int kItemSlots = 4;
 constexpr int kMaxPairs = 80;  // persistent grid: at most this many CTA pairs (>= SM count / 2)
 // Sequences at least this long use this kernel for the shapes below (measured on
-// B200, one call, d = 128, groups of 2: the one-CTA kernel is faster at L = 2048
-// (316 vs 336 us) and L = 4096 (491 vs 516 us), this one at L = 16384 (3.32 vs
-// 3.53 ms), where each item runs over many more key tiles)
-constexpr int kPairMinL = 8192;
+// B200, one call, d = 128, groups of 2 mixed after the softmax: the one-CTA kernel
+// is faster at L = 2048 (309 vs 326 us: this kernel's per-item exchange between
+// the two heads' pairs weighs more on short items), this one at L = 4096 (459 vs
+// 465 us) and L = 16384 (3.04 vs 3.53 ms))
+constexpr int kPairMinL = 4096;
 
 template <int D, int MIX, bool EXACT>
 struct PGeo {
@@ -235,7 +238,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     mbar_init(z_free, 16);
     mbar_init(v_full, 1);
     mbar_init(v_empty, 1);
-    for (int b = 0; b < 2; ++b) { mbar_init(c_full + b, 1); mbar_init(p_full + b, 16); }
+    for (int b = 0; b < 2; ++b) { mbar_init(c_full + b, 1); mbar_init(p_full + b, 2); }
     mbar_init(mma_done, 1);
     for (int s = 0; s < G::NS; ++s) { mbar_init(k_full + s, 1); mbar_init(k_empty + s, 1); }
     // consumers per item: both CTAs' V and query loaders and 8 softmax warps, the
@@ -398,7 +401,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int zc = G::DH * wg;       // output channels of this warpgroup
     const uint32_t tl = tmem + (static_cast<uint32_t>(32 * q4) << 16);
     const float sc0 = p.qk_scale * kLog2e;
-    float *crow = Cs + (wg * G::BM + r_) * G::W;
+    float *brow = Cs + r_ * G::W;             // this row of the item's band table
 
     auto arrive_all = [&](uint64_t *bar) {  // one arrival per warp on a barrier of the first CTA
       __syncwarp();
@@ -549,9 +552,13 @@ __global__ void __launch_bounds__(kThreads, 1)
       const long long fbase = (static_cast<long long>(it.b) * p.H + h) * p.lpad;
       const float qinv = exp2f(static_cast<float>(-eq));
       // the band 0 <= i-j < W, where the mask removes taps (see attn_kq.cu)
-      auto band_acc = [&](float (&acc)[G::W]) {
+      // (each warpgroup takes half of the W diagonals of its row, once per item, into
+      // the band table brow[dd], log2 units, read by both after a barrier)
+      auto band_part = [&](auto lo_c) {
+        constexpr int LO = decltype(lo_c)::value, NB = LO == 0 ? (G::W + 1) / 2 : G::W - (G::W + 1) / 2;
+        float acc[NB];
 #pragma unroll
-        for (int dd = 0; dd < G::W; ++dd) acc[dd] = 0.f;
+        for (int e = 0; e < NB; ++e) acc[e] = 0.f;
 #pragma unroll
         for (int a = 0; a < CQ; ++a) {
           const float *vrow = Us + (r_ + G::HALO - a) * G::M;
@@ -563,39 +570,50 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int tp = 0; tp < CK; ++tp) {
             const float thv = th[a * CK + tp];
 #pragma unroll
-            for (int dd = 0; dd < G::W; ++dd) {
-              const int m = dd - a + tp - G::C;
+            for (int e = 0; e < NB; ++e) {
+              const int dd = LO + e, m = dd - a + tp - G::C;
               const bool kept = EXACT ? tp >= G::C - dd : m >= 0;
-              if (kept && m + G::OFF >= 0 && m + G::OFF < G::M) acc[dd] = fmaf(thv, vr[m + G::OFF], acc[dd]);
+              if (kept && m + G::OFF >= 0 && m + G::OFF < G::M) acc[e] = fmaf(thv, vr[m + G::OFF], acc[e]);
             }
           }
         }
+#pragma unroll
+        for (int e = 0; e < NB; ++e) brow[LO + e] = acc[e] * sc0;
       };
       float m_run = -INFINITY, l_run = 0.f;
+      // column factors two tiles ahead: loaded a whole tile before they are stored
+      float fpre = (st_id < G::BN && 1 < nsl) ? p.fac[fbase + G::BN + st_id] : 0.f;
       for (int sl = 0; sl < nsl; ++sl, ++T) {
         const int j0 = sl * G::BN;
-        const float fnext = (st_id < G::BN && sl + 1 < nsl) ? p.fac[fbase + (sl + 1) * G::BN + st_id] : 0.f;
+        if (sl == 0) {  // the band table of the item, while the first C is computed
+          if (row_ok) {
+            if (wg == 0)
+              band_part(std::integral_constant<int, 0>());
+            else
+              band_part(std::integral_constant<int, (G::W + 1) / 2>());
+          }
+          named_bar_sync(kBarAll, kSmThreads);
+        }
+        const float fnext = fpre;
+        fpre = (st_id < G::BN && sl + 2 < nsl) ? p.fac[fbase + (sl + 2) * G::BN + st_id] : 0.f;
         mbar_wait_cluster(c_full + (T & 1), (T >> 1) & 1, abort_flag, p.err);
         tc_fence_after();
         const uint32_t cbuf = 128u * (T & 1);
         float cv[G::HALF];
         {
           const float4 *f4 = reinterpret_cast<const float4 *>(facs + (T & 1) * G::BN + cb);
+          // both 32-column halves in flight before one wait
+          uint32_t u32[2][32];
+          tmem_ld32(tl + cbuf + cb, u32[0]);
+          tmem_ld32(tl + cbuf + cb + 32, u32[1]);
+          tmem_wait_ld();
 #pragma unroll
-          for (int c0 = 0; c0 < G::HALF; c0 += 32) {
-            uint32_t u32[32];
-            tmem_ld32(tl + cbuf + cb + c0, u32);
-            float4 f[8];
-#pragma unroll
-            for (int i = 0; i < 8; ++i) f[i] = f4[c0 / 4 + i];
-            tmem_wait_ld();
-#pragma unroll
-            for (int i = 0; i < 8; ++i) {
-              cv[c0 + 4 * i] = __uint_as_float(u32[4 * i]) * f[i].x;
-              cv[c0 + 4 * i + 1] = __uint_as_float(u32[4 * i + 1]) * f[i].y;
-              cv[c0 + 4 * i + 2] = __uint_as_float(u32[4 * i + 2]) * f[i].z;
-              cv[c0 + 4 * i + 3] = __uint_as_float(u32[4 * i + 3]) * f[i].w;
-            }
+          for (int i = 0; i < G::HALF / 4; ++i) {
+            const float4 f = f4[i];
+            cv[4 * i] = __uint_as_float(u32[i / 8][4 * (i % 8)]) * f.x;
+            cv[4 * i + 1] = __uint_as_float(u32[i / 8][4 * (i % 8) + 1]) * f.y;
+            cv[4 * i + 2] = __uint_as_float(u32[i / 8][4 * (i % 8) + 2]) * f.z;
+            cv[4 * i + 3] = __uint_as_float(u32[i / 8][4 * (i % 8) + 3]) * f.w;
           }
         }
         tc_fence_before();  // orders the C reads before the barrier that precedes the P writes
@@ -605,14 +623,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         const int dmax = qi - j0 - cb;  // i - j for this warpgroup's first column
         if (row_ok && dmax >= 0 && dmax - (G::W - 1) < G::HALF) {
-          float acc[G::W];
-          band_acc(acc);
-#pragma unroll
-          for (int dd = 0; dd < G::W; ++dd) crow[dd] = acc[dd] * sc0;
 #pragma unroll
           for (int jj = 0; jj < G::HALF; ++jj) {
             const int dd = dmax - jj;
-            if (static_cast<unsigned>(dd) < static_cast<unsigned>(G::W)) cv[jj] = crow[dd];
+            if (static_cast<unsigned>(dd) < static_cast<unsigned>(G::W)) cv[jj] = brow[dd];
           }
         }
         if (j0 + G::BN - 1 > R0) {  // Mask_-inf: keys after the query
@@ -668,7 +682,14 @@ __global__ void __launch_bounds__(kThreads, 1)
         l_run += ls;
         tmem_wait_st();
         tc_fence_before();
-        arrive_all(p_full + (T & 1));
+        // one arrival per CTA: the TMEM stores of all eight warps are ordered before it
+        // by their fences and the barrier (a release at cluster scope per warp cost
+        // about as much as the tile's exponentials)
+        named_bar_sync(kBarP, kSmThreads);
+        if (st_id == 0) {
+          tc_fence_after();
+          arrive_first(p_full + (T & 1));
+        }
         if (pend && sl == 0) {  // the previous item's mixing, while this tile's P V and the next C run
           finish(pend_it);
           pend = false;

@@ -27,7 +27,8 @@
 // only, and Kt_a[j] is used only for queries i >= j + W > j + c: the path stays
 // exactly causal.  One CTA per (key tile, head, batch); the key rows with their
 // halo are staged in shared memory as bf16, and the convolution runs in packed
-// fp32 FMAs on channel pairs.
+// fp32 FMAs on channel pairs.  Four CTAs per SM (64 registers a thread): 78.9
+// against 83.8 us with three at B = 4, H = 16, L = 2048, d = 128.
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 #include <math.h>
@@ -88,7 +89,7 @@ __device__ __forceinline__ float2 fma2(float2 a, float2 b, float2 c) {
 }
 
 template <int D, int CQ, int CK, bool EXACT>
-__global__ void __launch_bounds__(kPrepThreads, 3) kq_prep_kernel(KqPrepArgs p) {
+__global__ void __launch_bounds__(kPrepThreads, 4) kq_prep_kernel(KqPrepArgs p) {
   using G = PrepGeo<D, CQ, CK, EXACT>;
   extern __shared__ uint32_t ks[];  // [ROWS][KSTR/2] bf16 pairs, row r = key j0 - LO + r
   __shared__ float rmax[G::ROWS];
