@@ -15,8 +15,11 @@
 // 4-stage ring; warp 1 runs the MMA loop in all lanes and issues tcgen05.mma
 // (M=128, N=BN, K=16) from one elected lane into one of two BN-column fp32
 // accumulators in tensor memory; warps 2..5 read a finished tile back with
-// tcgen05.ld and store (or add) it while the next tile's MMAs run.  Every
-// mbarrier wait is bounded.
+// tcgen05.ld while the next tile's MMAs run, 32 rows x 32 columns at a time, into
+// a 128-byte-swizzled shared-memory box that one lane writes out with a TMA store
+// (or, accumulating, a TMA add into the fp32 output).  A warp's 32 rows then
+// leave as whole 128-byte lines, not as 32 scattered 16-byte pieces per
+// instruction.  Every mbarrier wait is bounded.
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <stdint.h>
@@ -32,13 +35,17 @@ namespace {
 constexpr int BM = 128, BK = 64, STAGES = 4;
 constexpr int PANEL = 64 * BK * 2;  // an MN-major box: 64 rows x 64 K, 8 KB
 
+constexpr int EBOX = 32 * 32 * 4;  // an epilogue box: 32 rows x 32 fp32, 4 KB
+
 template <int BN>
 struct BG {
   static constexpr int A_BYTES = BM * BK * 2;
   static constexpr int B_BYTES = BN * BK * 2;
   static constexpr int STAGE = A_BYTES + B_BYTES;
-  static constexpr int SMEM = STAGES * STAGE + 1024 + 256;
+  static constexpr int EPI = 4 * 2 * EBOX;  // two boxes per epilogue warp
+  static constexpr int SMEM = STAGES * STAGE + EPI + 1024 + 256;
   static constexpr uint32_t TMEM_COLS = 2 * BN;
+  static_assert(SMEM <= 232448, "shared memory");
 };
 
 // Loads rows [r, r + R) x K slice [k, k + 64) of operand `o` for batch (b, h).
@@ -72,11 +79,12 @@ __device__ __forceinline__ uint64_t op_desc(bool mn, uint32_t base, int k) {
 template <int BN>
 __global__ void __launch_bounds__(192, 1)
     gemm_batched_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-                        const BgArgs p) {
+                        const __grid_constant__ CUtensorMap tmC, const BgArgs p) {
   using G = BG<BN>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint64_t *full = reinterpret_cast<uint64_t *>(smem + STAGES * G::STAGE);
+  uint8_t *epi = smem + STAGES * G::STAGE;  // 1024-aligned: STAGE is a multiple of 8 KB
+  uint64_t *full = reinterpret_cast<uint64_t *>(epi + G::EPI);
   uint64_t *empty = full + STAGES;
   uint64_t *acc_full = empty + STAGES;  // [2]
   uint64_t *acc_empty = acc_full + 2;   // [2]
@@ -101,6 +109,7 @@ __global__ void __launch_bounds__(192, 1)
     fence_mbar_init();
     prefetch_tmap(&tmA);
     prefetch_tmap(&tmB);
+    prefetch_tmap(&tmC);
   }
   if (warp == 1) { tmem_alloc(tslot, G::TMEM_COLS); tmem_relinquish(); }
   tc_fence_before();
@@ -156,8 +165,10 @@ __global__ void __launch_bounds__(192, 1)
       if (ok) mma_commit_if(issuer, &acc_full[ab]);
     }
   } else {
+    // warp 2 + q takes TMEM lanes (tile rows) 32 qd .. 32 qd + 31, qd = warp & 3
     const int qd = warp & 3;
-    int local = 0;
+    uint8_t *ebox = epi + qd * 2 * EBOX;
+    int local = 0, nbox = 0;
     for (int t = blockIdx.x; t < n_tiles; t += gridDim.x, ++local) {
       const int ab = local & 1;
       if (!mbar_wait(&acc_full[ab], (local >> 1) & 1, abort_flag, p.err)) break;
@@ -165,38 +176,41 @@ __global__ void __launch_bounds__(192, 1)
       int z, m0, n0;
       tile_of(t, z, m0, n0);
       const int b = z / p.H, h = z - b * p.H;
-      const int row = m0 + 32 * qd + lane;
-      float *crow = p.C + b * p.sb + h * p.sh + static_cast<long long>(row) * p.sm;
-      const bool vec = ((p.sm | p.sh | p.sb) & 3) == 0 && (reinterpret_cast<uintptr_t>(p.C) & 15) == 0;
+      const int r0 = m0 + 32 * qd;
 #pragma unroll 1
-      for (int c0 = 0; c0 < BN; c0 += 32) {
+      for (int c0 = 0; c0 < BN; c0 += 32, ++nbox) {
         uint32_t r[32];
         tmem_ld32(tmem + BN * ab + (static_cast<uint32_t>(32 * qd) << 16) + c0, r);
         tmem_wait_ld();
-        const int col = n0 + c0;
-        if (row >= p.M || col >= p.N) continue;
-        float *dst = crow + col;
-        if (vec && col + 32 <= p.N) {
+        // the box written two boxes ago has been read by its store
+        uint8_t *box = ebox + (nbox & 1) * EBOX;
+        if (lane == 0) bulk_wait_read<1>();
+        __syncwarp();
+        // row `lane` of the box; its 16-byte chunk i sits at i ^ (row & 7) (128-byte swizzle)
 #pragma unroll
-          for (int i = 0; i < 8; ++i) {
-            float4 v = make_float4(p.alpha * __uint_as_float(r[4 * i]), p.alpha * __uint_as_float(r[4 * i + 1]),
-                                   p.alpha * __uint_as_float(r[4 * i + 2]), p.alpha * __uint_as_float(r[4 * i + 3]));
-            if (p.accumulate) {
-              const float4 o = reinterpret_cast<const float4 *>(dst)[i];
-              v.x += o.x; v.y += o.y; v.z += o.z; v.w += o.w;
-            }
-            reinterpret_cast<float4 *>(dst)[i] = v;
+        for (int i = 0; i < 8; ++i)
+          *reinterpret_cast<float4 *>(box + lane * 128 + ((i ^ (lane & 7)) << 4)) =
+              make_float4(p.alpha * __uint_as_float(r[4 * i]), p.alpha * __uint_as_float(r[4 * i + 1]),
+                          p.alpha * __uint_as_float(r[4 * i + 2]), p.alpha * __uint_as_float(r[4 * i + 3]));
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) {
+          // rows past M and columns past N are clipped by the map
+          if (r0 < p.M && n0 + c0 < p.N) {
+            const int c1 = p.c_pos_row == 1 ? r0 : h, c2 = p.c_pos_row == 1 ? h : r0;
+            if (p.accumulate)
+              tma_reduce_add_4d(&tmC, box, n0 + c0, c1, c2, b);
+            else
+              tma_store_4d(&tmC, box, n0 + c0, c1, c2, b);
           }
-        } else {
-#pragma unroll
-          for (int i = 0; i < 32; ++i)
-            if (col + i < p.N) dst[i] = p.alpha * __uint_as_float(r[i]) + (p.accumulate ? dst[i] : 0.f);
+          bulk_commit();
         }
       }
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&acc_empty[ab]);
     }
+    if (lane == 0) bulk_wait_all();  // the output is written before the CTA exits
   }
   tc_fence_before();
   __syncthreads();
@@ -211,7 +225,26 @@ bool make_bg_map(void *map, const BgTensor &t, bool mn, int rows) {
   return encode_tmap_bf16(map, t.base, 4, t.dims, t.strides, box, true);
 }
 
-cudaError_t launch_gemm_batched(const BgTensor &A, const BgTensor &B, const BgArgs &args, cudaStream_t stream) {
+// The output as a 4-D fp32 map (n, m or h, h or m, b), the two middle dimensions in
+// increasing stride order; boxes of 32 columns x 32 rows, 128-byte swizzle.
+static bool make_c_map(CUtensorMap *map, BgArgs &a) {
+  if ((reinterpret_cast<uintptr_t>(a.C) & 15) || ((a.sm | a.sh | a.sb) & 3) || a.Z % a.H) return false;
+  const bool m_first = a.sm <= a.sh;
+  a.c_pos_row = m_first ? 1 : 2;
+  const unsigned long long B = static_cast<unsigned long long>(a.Z / a.H);
+  unsigned long long dims[4] = {static_cast<unsigned long long>(a.N), 0, 0, B};
+  unsigned long long str[3] = {0, 0, static_cast<unsigned long long>(a.sb) * 4};
+  dims[1] = m_first ? static_cast<unsigned long long>(a.M) : static_cast<unsigned long long>(a.H);
+  dims[2] = m_first ? static_cast<unsigned long long>(a.H) : static_cast<unsigned long long>(a.M);
+  str[0] = static_cast<unsigned long long>(m_first ? a.sm : a.sh) * 4;
+  str[1] = static_cast<unsigned long long>(m_first ? a.sh : a.sm) * 4;
+  unsigned box[4] = {32u, 1u, 1u, 1u};
+  box[a.c_pos_row] = 32u;
+  return encode_tmap_f32(map, a.C, 4, dims, str, box, true);
+}
+
+cudaError_t launch_gemm_batched(const BgTensor &A, const BgTensor &B, const BgArgs &args_in, cudaStream_t stream) {
+  BgArgs args = args_in;
   if (args.Z < 1 || args.M < 1 || args.N < 1 || args.K < 1) return cudaSuccess;
   // the contiguous coordinate of every TMA box must start on 16 bytes
   if ((args.a.mn ? args.a.off_mn : args.a.off_k) % 8 != 0 || (args.b.mn ? args.b.off_mn : args.b.off_k) % 8 != 0)
@@ -221,14 +254,15 @@ cudaError_t launch_gemm_batched(const BgTensor &A, const BgTensor &B, const BgAr
   cudaError_t e;
   if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
   if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return e;
-  alignas(64) CUtensorMap ta, tb;
+  alignas(64) CUtensorMap ta, tb, tc;
+  if (!make_c_map(&tc, args)) return cudaErrorInvalidValue;
   auto run = [&](auto kern, int bn, int smem) -> cudaError_t {
     if (!make_bg_map(&ta, A, args.a.mn, BM) || !make_bg_map(&tb, B, args.b.mn, bn)) return cudaErrorInvalidValue;
     cudaError_t e2 = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e2 != cudaSuccess) return e2;
     const long long tiles = static_cast<long long>(args.Z) * ((args.M + BM - 1) / BM) * ((args.N + bn - 1) / bn);
     const int grid = static_cast<int>(std::min<long long>(tiles, sms));
-    kern<<<grid, 192, smem, stream>>>(ta, tb, args);
+    kern<<<grid, 192, smem, stream>>>(ta, tb, tc, args);
     return cudaGetLastError();
   };
   if (args.N > 128) return run(gemm_batched_kernel<256>, 256, BG<256>::SMEM);

@@ -156,7 +156,10 @@ struct BgArgs {
   long long sb, sh, sm;
   BgOperand a, b;
   unsigned *err;
+  int c_pos_row;    // set by the launcher: position of m in the output map (1, or 2 when sh < sm)
 };
+// C is written through a TMA map: its base and the strides sm, sh, sb (in elements)
+// must be multiples of 16 bytes; cudaErrorInvalidValue otherwise.
 cudaError_t launch_gemm_batched(const BgTensor &A, const BgTensor &B, const BgArgs &args, cudaStream_t stream);
 
 // C[M][N] = A B^T with A [M][K] (a_mn: stored [K][M]) and B [N][K] (b_mn: stored
@@ -188,5 +191,8 @@ cudaError_t launch_wait_timeout_selftest(unsigned long long limit_ns, unsigned *
 bool encode_tmap_bf16(void *map_out, const void *base, int rank, const unsigned long long *dims,
                       const unsigned long long *strides_bytes, const unsigned *box,
                       bool swizzle128);
+// The same for fp32 elements.
+bool encode_tmap_f32(void *map_out, const void *base, int rank, const unsigned long long *dims,
+                     const unsigned long long *strides_bytes, const unsigned *box, bool swizzle128);
 
 }  // namespace mta

@@ -249,8 +249,10 @@ size_t layer_bwd_fixed_bytes(const mta_cfg *cfg) {
 
 }  // namespace
 
-bool encode_tmap_bf16(void *map_out, const void *base, int rank, const unsigned long long *dims,
-                      const unsigned long long *strides_bytes, const unsigned *box, bool swizzle128) {
+namespace {
+bool encode_tmap(CUtensorMapDataType dtype, void *map_out, const void *base, int rank,
+                 const unsigned long long *dims, const unsigned long long *strides_bytes, const unsigned *box,
+                 bool swizzle128) {
   static PFN_cuTensorMapEncodeTiled_v12000 fn = [] {
     void *p = nullptr;
     cudaDriverEntryPointQueryResult q;
@@ -268,12 +270,23 @@ bool encode_tmap_bf16(void *map_out, const void *base, int rank, const unsigned 
     estr[i] = 1;
     if (i > 0) gstr[i - 1] = strides_bytes[i - 1];
   }
-  CUresult r = fn(static_cast<CUtensorMap *>(map_out), CU_TENSOR_MAP_DATA_TYPE_BFLOAT16,
+  CUresult r = fn(static_cast<CUtensorMap *>(map_out), dtype,
                   static_cast<cuuint32_t>(rank), const_cast<void *>(base), gdim, gstr, bdim, estr,
                   CU_TENSOR_MAP_INTERLEAVE_NONE,
                   swizzle128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
+}
+}  // namespace
+
+bool encode_tmap_bf16(void *map_out, const void *base, int rank, const unsigned long long *dims,
+                      const unsigned long long *strides_bytes, const unsigned *box, bool swizzle128) {
+  return encode_tmap(CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, map_out, base, rank, dims, strides_bytes, box, swizzle128);
+}
+
+bool encode_tmap_f32(void *map_out, const void *base, int rank, const unsigned long long *dims,
+                     const unsigned long long *strides_bytes, const unsigned *box, bool swizzle128) {
+  return encode_tmap(CU_TENSOR_MAP_DATA_TYPE_FLOAT32, map_out, base, rank, dims, strides_bytes, box, swizzle128);
 }
 
 // The layer's fixed scratch: error word, QKV, attention output O, normalised Y
