@@ -922,6 +922,7 @@ cudaError_t launch_attn_bwd_tc(const BwdArgs &a, void *ws) {
       (e = cudaFuncSetAttribute(bwd_adjoint_kernel<6, 11, 1>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                 adjoint_smem())) != cudaSuccess)
     return e;
+  if ((e = cudaMemsetAsync(a.dq, 0, n * 4, st)) != cudaSuccess) return e;
   if ((e = cudaMemsetAsync(a.dk, 0, n * 4, st)) != cudaSuccess) return e;
   if ((e = cudaMemsetAsync(a.dv, 0, n * 4, st)) != cudaSuccess) return e;
   const size_t nth = static_cast<size_t>(a.H) * a.cq * a.ck * 4;
@@ -1023,7 +1024,8 @@ cudaError_t launch_attn_bwd_tc(const BwdArgs &a, void *ws) {
     const int own = std::min(g.no, a.L - r0);
     BgArgs gq = {};
     gq.Z = static_cast<int>(Z); gq.H = a.H; gq.err = err;
-    gq.M = own; gq.N = a.d; gq.K = 2 * Wp; gq.alpha = a.scale; gq.accumulate = 0;
+    // (added into the zeroed dq: the GEMM may split K in two)
+    gq.M = own; gq.N = a.d; gq.K = 2 * Wp; gq.alpha = a.scale; gq.accumulate = 1; gq.split_ok = 1;
     gq.C = a.dq + static_cast<long long>(r0) * HD; gq.sm = HD; gq.sh = a.d; gq.sb = LHD;
     gq.a = periodic(K_major(1, 0, 0), Wp, kRowsT);
     gq.b = periodic(MN_major(2, 0, 0), Wp, 0);

@@ -93,13 +93,18 @@ __global__ void __launch_bounds__(192, 1)
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int n_tm = (p.M + BM - 1) / BM, n_tn = (p.N + BN - 1) / BN;
-  const int per_z = n_tm * n_tn, n_tiles = p.Z * per_z;
-  const int nk = (p.K + BK - 1) / BK;
-  auto tile_of = [&](int t, int &z, int &m0, int &n0) {
+  const int per_z = n_tm * n_tn * p.ksplit, n_tiles = p.Z * per_z;
+  const int nk_all = (p.K + BK - 1) / BK, nkc = (nk_all + p.ksplit - 1) / p.ksplit;
+  // tile t: batch z, output block (m0, n0), K slices [k0, k1) (every range non-empty)
+  auto tile_of = [&](int t, int &z, int &m0, int &n0, int &k0, int &k1) {
     z = t / per_z;
-    const int r = t - z * per_z;
+    int r = t - z * per_z;
+    const int ks = r % p.ksplit;
+    r /= p.ksplit;
     m0 = (r / n_tn) * BM;
     n0 = (r % n_tn) * BN;
+    k0 = ks * nkc;
+    k1 = min(nk_all, k0 + nkc);
   };
 
   if (threadIdx.x == 0) {
@@ -121,10 +126,10 @@ __global__ void __launch_bounds__(192, 1)
     if (lane == 0) {
       int issued = 0;
       for (int t = blockIdx.x; t < n_tiles && !*abort_flag; t += gridDim.x) {
-        int z, m0, n0;
-        tile_of(t, z, m0, n0);
+        int z, m0, n0, k0, k1;
+        tile_of(t, z, m0, n0, k0, k1);
         const int b = z / p.H, h = z - b * p.H;
-        for (int kt = 0; kt < nk; ++kt, ++issued) {
+        for (int kt = k0; kt < k1; ++kt, ++issued) {
           const int s = issued % STAGES;
           if (!mbar_wait(&empty[s], ((issued / STAGES) & 1) ^ 1, abort_flag, p.err)) break;
           uint8_t *a_s = smem + s * G::STAGE;
@@ -150,7 +155,9 @@ __global__ void __launch_bounds__(192, 1)
       const int ab = local & 1;
       if (local >= 2 && !wwait(&acc_empty[ab], ((local >> 1) - 1) & 1)) break;
       tc_fence_after();
-      for (int kt = 0; kt < nk; ++kt, ++used) {
+      int z, m0, n0, k0, k1;
+      tile_of(t, z, m0, n0, k0, k1);
+      for (int kt = k0; kt < k1; ++kt, ++used) {
         const int s = used % STAGES;
         if (!wwait(&full[s], (used / STAGES) & 1)) { ok = false; break; }
         tc_fence_after();
@@ -159,7 +166,7 @@ __global__ void __launch_bounds__(192, 1)
 #pragma unroll
         for (int k = 0; k < BK / 16; ++k)
           mma_ss_if(issuer, tmem + BN * ab, op_desc(p.a.mn, a_base, k), op_desc(p.b.mn, b_base, k), idesc,
-                    (kt | k) != 0);
+                    (kt - k0) + k != 0);
         mma_commit_if(issuer, &empty[s]);
       }
       if (ok) mma_commit_if(issuer, &acc_full[ab]);
@@ -173,8 +180,8 @@ __global__ void __launch_bounds__(192, 1)
       const int ab = local & 1;
       if (!mbar_wait(&acc_full[ab], (local >> 1) & 1, abort_flag, p.err)) break;
       tc_fence_after();
-      int z, m0, n0;
-      tile_of(t, z, m0, n0);
+      int z, m0, n0, k0, k1;
+      tile_of(t, z, m0, n0, k0, k1);
       const int b = z / p.H, h = z - b * p.H;
       const int r0 = m0 + 32 * qd;
 #pragma unroll 1
@@ -256,18 +263,26 @@ cudaError_t launch_gemm_batched(const BgTensor &A, const BgTensor &B, const BgAr
   if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return e;
   alignas(64) CUtensorMap ta, tb, tc;
   if (!make_c_map(&tc, args)) return cudaErrorInvalidValue;
+  args.ksplit = 1;
   auto run = [&](auto kern, int bn, int smem) -> cudaError_t {
     if (!make_bg_map(&ta, A, args.a.mn, BM) || !make_bg_map(&tb, B, args.b.mn, bn)) return cudaErrorInvalidValue;
     cudaError_t e2 = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e2 != cudaSuccess) return e2;
-    const long long tiles = static_cast<long long>(args.Z) * ((args.M + BM - 1) / BM) * ((args.N + bn - 1) / bn);
+    const long long tiles =
+        static_cast<long long>(args.Z) * ((args.M + BM - 1) / BM) * ((args.N + bn - 1) / bn) * args.ksplit;
     const int grid = static_cast<int>(std::min<long long>(tiles, sms));
     kern<<<grid, 192, smem, stream>>>(ta, tb, tc, args);
     return cudaGetLastError();
   };
   if (args.N > 128) return run(gemm_batched_kernel<256>, 256, BG<256>::SMEM);
-  // narrow outputs: 64-column tiles when 128-column ones would leave SMs idle
+  // narrow outputs: when 128-column tiles would leave SMs idle, K in two halves
+  // (added into the zeroed output: with exactly two partial sums the result does not
+  // depend on their order) or else 64-column tiles
   const long long t128 = static_cast<long long>(args.Z) * ((args.M + BM - 1) / BM) * ((args.N + 127) / 128);
+  if (args.N > 64 && t128 < sms && args.split_ok && args.accumulate && (args.K + BK - 1) / BK >= 2) {
+    args.ksplit = 2;
+    return run(gemm_batched_kernel<128>, 128, BG<128>::SMEM);
+  }
   if (args.N <= 64 || t128 < sms) return run(gemm_batched_kernel<64>, 64, BG<64>::SMEM);
   return run(gemm_batched_kernel<128>, 128, BG<128>::SMEM);
 }

@@ -156,7 +156,9 @@ struct BgArgs {
   long long sb, sh, sm;
   BgOperand a, b;
   unsigned *err;
+  int split_ok;     // accumulating into a zeroed C: the launcher may split K in two
   int c_pos_row;    // set by the launcher: position of m in the output map (1, or 2 when sh < sm)
+  int ksplit;       // set by the launcher: K ranges per output tile (1 or 2)
 };
 // C is written through a TMA map: its base and the strides sm, sh, sb (in elements)
 // must be multiples of 16 bytes; cudaErrorInvalidValue otherwise.
