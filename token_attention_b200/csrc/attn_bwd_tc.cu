@@ -179,6 +179,10 @@ __global__ void __launch_bounds__(kThreadsB) bwd_scores_kernel(StripArgs p) {
     __syncthreads();
     const int jb = j0 + kSeg * seg;  // first key of the thread
     if (valid && jb <= i) {
+    if (!p.post) {  // dA'' of the thread's keys, read after the convolution: fetch it now
+#pragma unroll
+      for (int h = 0; h < CH; ++h) prefetch_l1(strip(p.D, h, p.g.rc) + u * P + jb);
+    }
     float cv[CH][kSeg];
 #pragma unroll
     for (int h = 0; h < CH; ++h) {
@@ -349,6 +353,13 @@ __global__ void __launch_bounds__(kThreadsB) bwd_scores_kernel(StripArgs p) {
   // back, with dw = sum dC'_h C_s); A'' (hi / lo) of the own rows
   if (valid) {
     for (int jb = kSeg * seg; jb <= i; jb += kKeyTile) {
+      if (jb + kKeyTile <= i) {  // the next chunk's logits and dA'', while this one is computed
+#pragma unroll
+        for (int h = 0; h < CH; ++h) {
+          prefetch_l1(strip(p.A, h, p.g.rc) + u * P + jb + kKeyTile);
+          prefetch_l1(strip(p.D, h, p.g.rc) + u * P + jb + kKeyTile);
+        }
+      }
       float a[CH][kSeg], da[CH][kSeg], dc[CH][kSeg];
 #pragma unroll
       for (int h = 0; h < CH; ++h) { weights(jb, h, a[h]); grads(jb, h, da[h]); }
