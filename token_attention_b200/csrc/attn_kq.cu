@@ -162,14 +162,14 @@ struct KGeo {
   // starts at column CB1
   static constexpr bool CDB = DB || (POST && Z_COL0 + 128 * (NV - 1) + D + 128 * NSRC <= TMEM_COLS);
   static constexpr uint32_t CB1 = DB ? 128 : TMEM_COLS - 128 * NSRC;
-  static_assert(5 + 2 * NS + 9 <= 32, "barriers before the item ring");
+  static_assert(5 + 2 * NS + 10 <= 32, "barriers before the item ring");
   static_assert(MIX != 1 || NV == 1, "pre-softmax mixing uses the destination head's V only");
   static_assert(OFF_K % 1024 == 0 && OFF_V % 1024 == 0, "swizzle alignment");
   static_assert(OFF_PS % 16 == 0 && OFF_DG % 16 == 0 && OFF_U % 16 == 0, "alignment");
   static_assert(OFF_SMALL % 16 == 0, "alignment");
   static_assert(NS >= 3, "Kt ring");
   static_assert(NCH % SB == 0 && NDC % SB == 0, "whole stages");
-  static_assert(13 + 2 * NS <= 32, "barrier slots (32 .. 39: the item ring)");
+  static_assert(15 + 2 * NS <= 32, "barrier slots (32 .. 39: the item ring)");
   static_assert(SMEM <= 232448, "shared memory");
   static_assert(CQ * CK <= 120, "kernel taps");
   static_assert(CQ * D % 64 == 0 && D % 16 == 0, "contraction chunks");
@@ -261,6 +261,13 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t *const p_fullb[2] = {p_full, v_full + 7};
   // CDB without DB (post-softmax variant): C of buffer b has been read by the softmax
   uint64_t *const c_freeb[2] = {c_free, v_full + 8};
+  // post-softmax mixing: the peer's exchange data of item r is in place, one barrier
+  // per item parity.  With one barrier the peer, one short item ahead, could complete
+  // a second phase before this CTA waited for the first, and the parity wait then
+  // waited for a phase that needs this CTA's own progress.  The peer cannot get two
+  // items ahead: its item r+2 needs this CTA's arrival for r+1, which follows the wait
+  // for r.
+  uint64_t *const x_readyb[2] = {x_ready, v_full + 9};
   uint32_t *tslot = reinterpret_cast<uint32_t *>(small + G::TSLOT_OFF);
   volatile int *abort_flag = reinterpret_cast<volatile int *>(small + G::ABORT_OFF);
   // item ring: it_full[s] completes when slot s holds the next item index (or -1 at
@@ -321,7 +328,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (threadIdx.x == 0) {
     mbar_init(q_full, 1); mbar_init(q_ready, 8); mbar_init(q_free, 1); mbar_init(z_free, 8);
-    mbar_init(x_ready, kSmThreads);
+    mbar_init(x_readyb[0], kSmThreads); mbar_init(x_readyb[1], kSmThreads);
     for (int s = 0; s < G::NS; ++s) { mbar_init(k_full + s, 1); mbar_init(k_empty + s, 1); }
     mbar_init(v_full, 1); mbar_init(v_empty, 1); mbar_init(c_full, 1); mbar_init(c_free, 8);
     mbar_init(p_full, 8); mbar_init(mma_done, 1);
@@ -747,7 +754,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int ph = pi.g * CL + hr, pg = pi.g;
       const int pq = row_start(pi) + r_;
       const bool pout = pq >= 0 && pq < L && r_ >= G::RSH;
-      mbar_wait_cluster(x_ready, pr & 1, abort_flag, p.err);
+      mbar_wait_cluster(x_readyb[pr & 1], (pr >> 1) & 1, abort_flag, p.err);
       const float4 *own = xslot(c, hr, pr & 1, 1);
       const float4 *theirs = xslot(c, hr ^ 1, pr & 1, 0);
       const float w_peer = p.w[pg * 4 + hr * 2 + (hr ^ 1)];
@@ -1183,7 +1190,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         __syncwarp();
         if (lane == 0) mbar_arrive(z_free);  // the next item's first P V may overwrite Z
         // every thread's stores are released to the peer by its own arrival
-        mbar_arrive_cluster(map_peer(smem_u32(x_ready), static_cast<uint32_t>(hr ^ 1)));
+        mbar_arrive_cluster(map_peer(smem_u32(x_readyb[r & 1]), static_cast<uint32_t>(hr ^ 1)));
         pend = true;
         pend_r = r;
         pend_it = it;
@@ -1216,8 +1223,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         __syncwarp();
         if (lane == 0) mbar_arrive(z_free);  // the next item's first P V may overwrite Z
         // every thread's stores are released to the peer by its own arrival
-        mbar_arrive_cluster(map_peer(smem_u32(x_ready), static_cast<uint32_t>(hr ^ 1)));
-        mbar_wait_cluster(x_ready, r & 1, abort_flag, p.err);
+        mbar_arrive_cluster(map_peer(smem_u32(x_readyb[r & 1]), static_cast<uint32_t>(hr ^ 1)));
+        mbar_wait_cluster(x_readyb[r & 1], (r >> 1) & 1, abort_flag, p.err);
 #pragma unroll
         for (int c4 = 0; c4 < G::DH / 4; ++c4) {
           if (4 * c4 >= zn) break;
