@@ -528,10 +528,11 @@ def run_mine(args, wl, rank, world, local_rank):
     if st != 0:
         raise RuntimeError(f"timed-region status {mta.STATUS.get(st, st)}")
     # every call clears the error word, so a wait that ran out in an earlier step shows
-    # only as that step's time: at least the 2 s wait bound (not checked under a
-    # profiler, whose replays make steps that long)
+    # only as that step's time: at least the 2 s wait bound, hidden in the mean of a
+    # long timed region (short profiling runs, whose profiled steps take that long
+    # too, are not checked)
     med = statistics.median(step_ms)
-    if max(step_ms) >= 1900.0 and not os.environ.get("CUDA_INJECTION64_PATH"):
+    if args.steps >= 20 and max(step_ms) >= 1900.0:
         raise RuntimeError(f"a step took {max(step_ms):.1f} ms against a median of {med:.3f} ms: "
                            "a bounded wait ran out during the timed region")
     clocks = sampler.stop() if sampler else None
