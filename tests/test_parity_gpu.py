@@ -272,30 +272,32 @@ def test_identity_workload_equals_causal_attention():
     assert_close(out, ref, "bf16")
 
 
-@pytest.mark.parametrize("name,calls", [("identity_d64_L2048", 2000), ("pretrain_d128_L2048", 500)])
+@pytest.mark.parametrize("name,calls", [("identity_d64_L2048", 2000), ("pretrain_d128_L2048", 500),
+                                        ("layer_pre_D2048_L4096", 200), ("layer_post_D2048_L4096", 300),
+                                        ("both_d128_L2048", 150)])
 def test_repeated_calls_never_time_out(name, calls):
-    """Back-to-back calls, the status word read after every one (each call clears it).
+    """Back-to-back calls, the status word read after every one (each call clears it):
+    the one-CTA kernel with and without pre- or post-softmax mixing, the CTA-pair
+    kernel (L = 4096) and the two-pass kernel of the convolution after the softmax.
     With post-softmax mixing the two CTAs of a cluster exchange their partial outputs
     once per work item; the last items of the queue span a single key tile, so one CTA
     can finish an item's exchange while its peer still waits for the previous one.  A
     single exchange barrier then completed two phases under the waiter and its bounded
-    wait ran out, about once per 250 calls at d = 64.  Every call's output is also
-    compared with the first call's: the same inputs give the same bits."""
+    wait ran out, about once per 250 calls at d = 64.  Every 100th call's output is
+    also compared with the first call's: the same inputs give the same bits."""
     wl = synth.WORKLOADS[name]
     inp = synth.make_attn_inputs(wl)
     q, k, v = (dev(inp[n]) for n in "qkv")
     th, w = dev(inp["theta"], "f32"), dev(inp["w"], "f32")
-    cfg = mta.make_cfg(wl.B, wl.H, wl.L, wl.d, wl.c_q, wl.c_k, wl.c_h, wl.kq_place, wl.head_place, mta.BF16)
-    lib = mta.lib()
-    ws = mta.workspace(lib.mta_attn_workspace_bytes(ctypes.byref(cfg)))
-    stream = torch.cuda.current_stream()
-    cfg.workspace, cfg.workspace_bytes, cfg.stream = ws.data_ptr(), ws.numel(), stream.cuda_stream
+    tp = dev(inp["theta_post"], "f32") if wl.kq_post else None
+    cfg = mta.make_cfg(wl.B, wl.H, wl.L, wl.d, wl.c_q, wl.c_k, wl.c_h, wl.kq_place, wl.head_place, mta.BF16,
+                       kq_post=int(wl.kq_post))
+    ws = mta.workspace(mta.lib().mta_attn_workspace_bytes(ctypes.byref(cfg)))
     first = None
     out = torch.empty_like(q)
     for i in range(calls):
-        mta.attn_fwd(q, k, v, th, w, wl.c_q, wl.c_k, wl.c_h, wl.kq_place, wl.head_place, out=out, ws=ws)
-        st = lib.mta_sync_status(ctypes.byref(cfg))
-        assert st == 0, f"call {i}: {mta.STATUS.get(st, st)}"
+        mta.attn_fwd(q, k, v, th, w, wl.c_q, wl.c_k, wl.c_h, wl.kq_place, wl.head_place, out=out, ws=ws,
+                     check=True, theta_post=tp)
         if first is None:
             first = out.clone()
         elif i % 100 == 0:
