@@ -117,9 +117,14 @@ def uses_bwd_tc(wl: synth.Workload) -> bool:
             and (wl.head_place == synth.OFF or wl.c_h == 2))
 
 
+def bwd_tc_rows(wl: synth.Workload) -> int:
+    """Rows of a query block's S strip in the tensor-core backward (its choice from L)."""
+    return 384 if wl.L <= 3072 else 512
+
+
 def bwd_tc_no(wl: synth.Workload) -> int:
     """Own rows of a query block of the tensor-core backward."""
-    return 256 - (3 if wl.kq_post else 2) * (wl.c_q - 1)
+    return bwd_tc_rows(wl) - (3 if wl.kq_post else 2) * (wl.c_q - 1)
 
 
 def bwd_tc_launches(wl: synth.Workload) -> int:
@@ -132,15 +137,15 @@ def bwd_tc_launches(wl: synth.Workload) -> int:
 
 def bwd_tc_gemm_flops(wl: synth.Workload) -> float:
     """Tensor flops the tensor-core backward's GEMMs execute per call (bf16 MMAs):
-    per query block of NO rows (strips of 256 rows) and keys 0 .. W-1, for every
-    head: S (256 x W x d), dA'' (251 x W x d), dQ (NO x d x 2W: hi and lo halves),
-    dK and dV (W x d x 512)."""
-    no = bwd_tc_no(wl)
+    per query block of NO rows (strips of R rows) and keys 0 .. W-1, for every
+    head: S (R x W x d), dA'' (RC x W x d), dQ (NO x d x 2W: hi and lo halves),
+    dK and dV (W x d x 2R)."""
+    R, no = bwd_tc_rows(wl), bwd_tc_no(wl)
     rc = no + (2 if wl.kq_post else 1) * (wl.c_q - 1)
     f = 0.0
     for r0 in range(0, wl.L, no):
         W = min(wl.L, r0 + rc)
-        f += 2 * (256 + rc) * W * wl.d + 2 * no * wl.d * 2 * W + 2 * 2 * W * wl.d * 512
+        f += 2 * (R + rc) * W * wl.d + 2 * no * wl.d * 2 * W + 2 * 2 * W * wl.d * 2 * R
     return f * wl.B * wl.H
 
 

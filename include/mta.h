@@ -267,8 +267,8 @@ mta_status mta_group_norm_scale_bwd(const void *o, const float *dy, const mta_gn
  *   3: the contractions on the tensor cores (attn_bwd_tc.cu): bf16, d = 64, 96 or
  *      128, c_q = 6, c_k = 11, kq_place = MTA_PRE (with or without the
  *      post-softmax convolution, kq_post), c_h = 2 with head mixing; query
- *      blocks of 246 rows (241 with kq_post), every head at once, their maps in
- *      strips of the workspace (S = s Q K^T, dA'' = dO V^T, dQ, dK, dV as batched
+ *      blocks of R - 10 rows (R - 15 with kq_post; R = 384 up to L = 3072, else
+ *      512), every head at once, their maps in strips of the workspace (S = s Q K^T, dA'' = dO V^T, dQ, dK, dV as batched
  *      tcgen05 GEMMs; the convolutions, their adjoints and the softmax on the
  *      CUDA cores).  MTA_ERR_UNSUPPORTED for other configurations,
  *      MTA_ERR_WORKSPACE when the strips do not fit.
@@ -282,11 +282,11 @@ mta_status mta_group_norm_scale_bwd(const void *o, const float *dy, const mta_gn
  * paths) and dk, dv (path 1) are summed with atomic additions, so their last
  * bits may differ between runs.  The workspace (mta_attn_bwd_workspace_bytes)
  * holds the error word and, where path 3 applies, its strips: for one query
- * block of every head, a 256-row S strip and two (three with pre-softmax
- * mixing) fp32 strips of 251 rows over the keys, and two bf16 strips of 512 rows
- * (B*H*pitch*(256*4 + 2*251*4 + 2*512*2) bytes, pitch = L rounded up to 64);
- * with kq_post the fp32 strips have 251 rows and three more are added (251, 246
- * and 241 rows).  No L x L map is stored. */
+ * block of every head, an R-row S strip and two (three with pre-softmax mixing)
+ * fp32 strips of R - 5 rows over the keys, and two bf16 strips of 2R rows
+ * (B*H*pitch*(R*4 + 2*(R-5)*4 + 2*2R*2) bytes, pitch = L rounded up to 64, each
+ * strip rounded up to 256 bytes; c_q = 6); with kq_post three more fp32 strips
+ * (R - 5, R - 10 and R - 15 rows).  No L x L map is stored. */
 size_t mta_attn_bwd_workspace_bytes(const mta_cfg *cfg);
 mta_status mta_attn_bwd(const void *q, const void *k, const void *v, const float *theta_kq,
                         const float *w_head, const void *dout, const mta_cfg *cfg, float *dq,

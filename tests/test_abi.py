@@ -291,18 +291,23 @@ def test_backward_argument_errors(L):
     small.workspace, small.workspace_bytes = 0x100000, 16
     assert f(small) == 3
     # the status word, then the tensor-core backward's strips for one query block of
-    # every head (B H = 8, pitch 64): S [256 rows] and A, dA/dC [251 rows] fp32, the
-    # dS and A'' halves [512 rows] bf16
-    Z, P, rc = 2 * 4, 64, 256 - 5
-    strips = up(Z * 256 * P * 4) + 2 * up(Z * rc * P * 4) + 2 * up(Z * 512 * P * 2)
+    # every head (B H = 8, pitch 64; blocks of R = 384 rows up to L = 3072): S [R rows]
+    # and A, dA/dC [R - 5 rows] fp32, the dS and A'' halves [2R rows] bf16
+    Z, P, R = 2 * 4, 64, 384
+    rc = R - 5
+    strips = up(Z * R * P * 4) + 2 * up(Z * rc * P * 4) + 2 * up(Z * 2 * R * P * 2)
     assert L.mta_attn_bwd_workspace_bytes(ctypes.byref(good_cfg())) == 256 + strips
     # pre-softmax mixing keeps the unmixed C as well
     assert L.mta_attn_bwd_workspace_bytes(ctypes.byref(good_cfg(head_place=mta.PRE))) == \
         256 + strips + up(Z * rc * P * 4)
-    # the convolution after the softmax: blocks of 256 - 3 (c_q - 1) = 241 own rows, the
-    # same 251-row strips, and its output gradient G [251], dA / dC [246] and A' [241]
+    # the convolution after the softmax: blocks of R - 3 (c_q - 1) own rows, the same
+    # R - 5 row strips, and its output gradient G [R - 5], dA / dC [R - 10] and A' [R - 15]
     assert L.mta_attn_bwd_workspace_bytes(ctypes.byref(good_cfg(kq_post=1))) == \
-        256 + strips + up(Z * 251 * P * 4) + up(Z * 246 * P * 4) + up(Z * 241 * P * 4)
+        256 + strips + up(Z * (R - 5) * P * 4) + up(Z * (R - 10) * P * 4) + up(Z * (R - 15) * P * 4)
+    # past L = 3072 the blocks have R = 512 rows
+    Ll, Rl = 4096, 512
+    long_strips = (up(Z * Rl * Ll * 4) + 2 * up(Z * (Rl - 5) * Ll * 4) + 2 * up(Z * 2 * Rl * Ll * 2))
+    assert L.mta_attn_bwd_workspace_bytes(ctypes.byref(good_cfg(L=Ll))) == 256 + long_strips
     assert L.mta_attn_bwd_workspace_bytes(ctypes.byref(good_cfg(c_q=3))) == 256   # CUDA cores only
     assert L.mta_attn_bwd_workspace_bytes(ctypes.byref(good_cfg(c_k=4))) == 0
 

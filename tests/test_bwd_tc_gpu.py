@@ -5,8 +5,8 @@ Every gradient (q, k, v, theta, w) at the CUDA-core backward's fp32 tolerance
 (relative L2 error 1e-4): the tensor-core path (d = 64, 96 or 128) takes the bf16 inputs themselves as
 MMA operands and splits its computed operands (dS, A'') into two bf16 halves, so
 its products carry about 16 significant bits and its sums fp32 accumulation.
-Lengths span one query block (L <= 246; 241 with the convolution after the
-softmax), several blocks and a ragged tail; the pretraining recipe and the
+Lengths span one query block (L <= 374 own rows, 369 with the convolution after the
+softmax: blocks of 384 rows up to L = 3072), several blocks and a ragged tail; the pretraining recipe and the
 convolution on both sides of the softmax run at their full length for one head
 group.
 """
@@ -65,9 +65,9 @@ def check(wl, inp, dout, path=mta.PATH_KQ):
     return got, out
 
 
-CASES = [(128, synth.POST, 9), (128, synth.POST, 247), (128, synth.PRE, 300), (128, synth.OFF, 70),
-         (64, synth.POST, 600), (64, synth.PRE, 250), (64, synth.OFF, 119), (128, synth.POST, 237),
-         (96, synth.POST, 300), (96, synth.PRE, 130)]
+CASES = [(128, synth.POST, 9), (128, synth.POST, 375), (128, synth.PRE, 300), (128, synth.OFF, 70),
+         (64, synth.POST, 800), (64, synth.PRE, 250), (64, synth.OFF, 119), (128, synth.POST, 374),
+         (96, synth.POST, 500), (96, synth.PRE, 130), (128, synth.PRE, 760)]
 
 
 @pytest.mark.parametrize("d,hp,L", CASES)
@@ -79,15 +79,15 @@ def test_bwd_tc_small(d, hp, L):
     check(wl, inp, dout)
 
 
-POST_CASES = [(128, synth.POST, 9), (128, synth.POST, 300), (128, synth.PRE, 250), (128, synth.OFF, 242),
-              (64, synth.POST, 500), (96, synth.POST, 130)]
+POST_CASES = [(128, synth.POST, 9), (128, synth.POST, 370), (128, synth.PRE, 250), (128, synth.OFF, 369),
+              (64, synth.POST, 500), (96, synth.POST, 130), (128, synth.POST, 760)]
 
 
 @pytest.mark.parametrize("d,hp,L", POST_CASES)
 def test_bwd_tc_post_conv_small(d, hp, L):
     """The convolution on both sides of the softmax (the pages' default): every
-    gradient, the post-softmax kernels' included, from one query block of 241 rows
-    to three."""
+    gradient, the post-softmax kernels' included, from one query block of 369 own
+    rows to three."""
     wl = synth.shrink(synth.WORKLOADS["both_d128_L2048"], B=2, H=4, L=L, d=d, head_place=hp,
                       seed=931 + L + d + 3 * hp)
     inp = synth.make_attn_inputs(wl)
@@ -96,7 +96,8 @@ def test_bwd_tc_post_conv_small(d, hp, L):
 
 
 def test_bwd_tc_post_conv_full_length_one_group():
-    """The convolution on both sides at L = 2048 (9 query blocks), one head group."""
+    """The convolution on both sides at L = 2048 (6 query blocks of 369 own rows), one head
+    group."""
     wl = synth.shrink(synth.WORKLOADS["both_d128_L2048"], B=1, H=2, seed=955)
     inp = synth.make_attn_inputs(wl)
     dout = synth.round_bf16(synth.normal(wl.seed, 20, (wl.B, wl.L, wl.H, wl.d)))
@@ -104,7 +105,7 @@ def test_bwd_tc_post_conv_full_length_one_group():
 
 
 def test_bwd_tc_matches_cuda_core_path():
-    """Both backward paths on the same inputs (L = 512, two query blocks and a tail)."""
+    """Both backward paths on the same inputs (L = 512: two query blocks, the second ragged)."""
     wl = synth.shrink(synth.WORKLOADS["pretrain_d128_L2048"], B=1, H=4, L=512, seed=951)
     inp = synth.make_attn_inputs(wl)
     dout = synth.round_bf16(synth.normal(wl.seed, 20, (wl.B, wl.L, wl.H, wl.d)))
@@ -118,7 +119,7 @@ def test_bwd_tc_matches_cuda_core_path():
 
 
 def test_bwd_tc_full_length_one_group():
-    """The pretraining recipe at its full length L = 2048 (9 query blocks), one batch
+    """The pretraining recipe at its full length L = 2048 (6 query blocks), one batch
     and one head group, against the oracle's full L x L backward of that group."""
     wl = synth.shrink(synth.WORKLOADS["pretrain_d128_L2048"], B=1, H=2, seed=952)
     inp = synth.make_attn_inputs(wl)

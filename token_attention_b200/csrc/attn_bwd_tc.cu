@@ -16,14 +16,15 @@
 //   dtheta[a][t] = sum dC[i][j] Mask_0 S[i-a][j-(t-c)]
 //   dQ = s dS K, dK = s dS^T Q               (tensor cores)
 //
-// Query blocks of NO = 256 - 2 (c_q - 1) rows are processed one after another,
-// all heads at once.  For block rows r0 .. r0+NO-1 the maps are held in strips
-// of the workspace that span every key up to the block's last row: S for rows
-// r0-(c_q-1) .. r0+NO+c_q-2 (256 rows: the convolution reads c_q-1 earlier query
+// Query blocks of NO = R - 2 (c_q - 1) rows (R = 384 or 512, block_rows below) are
+// processed one after another, all heads at once.  For block rows r0 .. r0+NO-1
+// the maps are held in strips of the workspace that span every key up to the
+// block's last row: S for rows r0-(c_q-1) .. r0+NO+c_q-2 (R rows: the convolution
+// reads c_q-1 earlier query
 // rows, its adjoint c_q-1 later ones), A, dA'' then dC for rows r0 .. r0+NO+c_q-2,
 // dS and A'' for the block's own rows.  A strip holds whole rows, so the softmax
 // statistics and D come from the strip itself (no statistics pass).  The strips
-// are O(B H 256 L): never an L x L map.  Per block:
+// are O(B H R L): never an L x L map.  Per block:
 //   1. S strip      = s Q K^T                      batched GEMM (fp32 out)
 //   2. dA'' strip   = dO V^T                       batched GEMM
 //   3. C, softmax, then dC, D, dw, A''             bwd_scores_kernel (CUDA cores)
@@ -32,7 +33,7 @@
 // With the convolution after the softmax, A' = Mask_0(Conv2d_theta_post A) sits
 // between the softmax and the post-softmax mixing; its adjoint reads G = dL/dA'
 // c_q-1 rows below each row and A' reads A c_q-1 rows above, so a block carries a
-// second halo: NO = 256 - 3 (c_q - 1), S from row r0 - 2 (c_q - 1), the weights A
+// second halo: NO = R - 3 (c_q - 1), S from row r0 - 2 (c_q - 1), the weights A
 // from r0 - (c_q - 1).  Step 3 then writes the normalised weights only, and four
 // kernels follow it: G (bwd_post_grad_kernel), dA = its adjoint with dtheta_post
 // and A' of the own rows (bwd_adjoint_kernel, mode 1), A'' and the post-mixing dw
@@ -53,12 +54,17 @@
 namespace mta {
 namespace {
 
-constexpr int kRowsT = 256;  // rows of the S strip (and of the halves of the dS / A'' strips)
+// Rows of a query block's S strip (and of each half of its dS / A'' strips): 384 up
+// to L = 3072, else 512.  Measured on one B200 (d = 128, groups of 2): at L = 2048,
+// 4.61 ms with 384 rows against 4.74 with 256 and 4.87 with 512 (four full blocks and
+// a 40-row one); at L = 4096, 9.68 ms with 512 against 9.92 with 384 and 9.97 with 256.
+int block_rows(int L) { return L <= 3072 ? 384 : 512; }
 constexpr int kKeyTile = 128;
 constexpr int kThreadsB = 256;
 
 struct Geo {
   int halo, c, no, rc, pitch;  // c_q - 1, c_k / 2, own rows, C rows, strip pitch (elements)
+  int rt;                      // rows of the S strip and of each dS / A'' half (block_rows)
 };
 
 struct StripArgs {
@@ -67,12 +73,12 @@ struct StripArgs {
   Geo g;
   const float *theta;         // [H][c_q][c_k]
   const float *w;             // [H/c_h][c_h][c_h]
-  float *S;                   // [B][H][256][pitch]
+  float *S;                   // [B][H][R][pitch]
   float *Cpre;                // [B][H][rc][pitch] pre-mixing C (pre mixing only)
   float *A;                   // [B][H][rc][pitch]
   float *D;                   // [B][H][rc][pitch]: dA'' from the GEMM, then dC
-  __nv_bfloat16 *dS;          // [B][H][512][pitch]: hi rows 0..255, lo rows 256..511
-  __nv_bfloat16 *Ap;          // [B][H][512][pitch]: A'' hi / lo
+  __nv_bfloat16 *dS;          // [B][H][2R][pitch]: hi rows 0..R-1, lo rows R..2R-1
+  __nv_bfloat16 *Ap;          // [B][H][2R][pitch]: A'' hi / lo
   float *dtheta, *dw;
   int post;                   // the convolution after the softmax: the scores kernel
                               // only writes the normalised weights A
@@ -167,7 +173,7 @@ __global__ void __launch_bounds__(kThreadsB) bwd_scores_kernel(StripArgs p) {
   auto stage = [&](int tt) {
 #pragma unroll
     for (int hl = 0; hl < CH; ++hl)
-      stage_rows<TR>(tile[tt & 1][hl], strip(p.S, hl, kRowsT), P, u0, kRowsT, p.r0 - HALO + u0, p.L, tt * kKeyTile);
+      stage_rows<TR>(tile[tt & 1][hl], strip(p.S, hl, p.g.rt), P, u0, p.g.rt, p.r0 - HALO + u0, p.L, tt * kKeyTile);
   };
   stage(0);
   cp_async_commit();
@@ -433,9 +439,9 @@ __global__ void __launch_bounds__(kThreadsB) bwd_scores_kernel(StripArgs p) {
                         (static_cast<uint32_t>(__bfloat16_as_ushort(l1)) << 16);
           }
           __nv_bfloat16 *ap = reinterpret_cast<__nv_bfloat16 *>(
-              p.Ap + ((static_cast<long long>(b) * p.H + g * CH + h) * 2 * kRowsT) * P);
+              p.Ap + ((static_cast<long long>(b) * p.H + g * CH + h) * 2 * p.g.rt) * P);
           *reinterpret_cast<uint4 *>(ap + static_cast<long long>(u) * P + jb) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
-          *reinterpret_cast<uint4 *>(ap + static_cast<long long>(kRowsT + u) * P + jb) =
+          *reinterpret_cast<uint4 *>(ap + static_cast<long long>(p.g.rt + u) * P + jb) =
               make_uint4(lo[0], lo[1], lo[2], lo[3]);
         }
       }
@@ -473,12 +479,12 @@ struct AdjArgs {
   const float *theta;   // [H][c_q][c_k]
   float *dtheta;        // [H][c_q][c_k] (or null)
   int out_rows;         // MODE 1: rows of dA
-  __nv_bfloat16 *dS;    // MODE 0: [B][H][512][pitch]
+  __nv_bfloat16 *dS;    // MODE 0: [B][H][2R][pitch]
   float *dA;            // MODE 1: [B][H][out_rows][pitch]
   float *Ac;            // MODE 1: A' of the own rows, [B][H][no][pitch]
 };
 
-// Step 4: CTA = one head and 16 rows u = 0 .. 255; thread (row, seg): 8
+// Step 4: CTA = one head and 16 rows u = 0 .. R-1; thread (row, seg): 8
 // consecutive keys, register windows of the staged rows as in the scores kernel.
 // Key tiles past the CTA's last row only write zeros (MODE 0).
 template <int CQ, int CK, int MODE>
@@ -571,7 +577,7 @@ __global__ void __launch_bounds__(kThreadsB) bwd_adjoint_kernel(StripArgs p, Adj
       }
     }
     if (MODE == 0 && jb < p.Wp) {
-      __nv_bfloat16 *dSz = q.dS + static_cast<long long>(z) * 2 * kRowsT * P;
+      __nv_bfloat16 *dSz = q.dS + static_cast<long long>(z) * 2 * p.g.rt * P;
       uint32_t hi[kSeg / 2], lo[kSeg / 2];
 #pragma unroll
       for (int x = 0; x < kSeg; x += 2) {
@@ -582,7 +588,7 @@ __global__ void __launch_bounds__(kThreadsB) bwd_adjoint_kernel(StripArgs p, Adj
         lo[x / 2] = static_cast<uint32_t>(__bfloat16_as_ushort(l0)) | (static_cast<uint32_t>(__bfloat16_as_ushort(l1)) << 16);
       }
       *reinterpret_cast<uint4 *>(dSz + static_cast<long long>(u) * P + jb) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
-      *reinterpret_cast<uint4 *>(dSz + static_cast<long long>(kRowsT + u) * P + jb) =
+      *reinterpret_cast<uint4 *>(dSz + static_cast<long long>(p.g.rt + u) * P + jb) =
           make_uint4(lo[0], lo[1], lo[2], lo[3]);
     }
     if (MODE == 1 && work && outr && jb <= i && jb < p.Wp) {
@@ -698,9 +704,9 @@ __global__ void __launch_bounds__(kThreadsB) bwd_post_mix_kernel(StripArgs p, co
           hi[x / 2] = static_cast<uint32_t>(__bfloat16_as_ushort(h0)) | (static_cast<uint32_t>(__bfloat16_as_ushort(h1)) << 16);
           lo[x / 2] = static_cast<uint32_t>(__bfloat16_as_ushort(l0)) | (static_cast<uint32_t>(__bfloat16_as_ushort(l1)) << 16);
         }
-        __nv_bfloat16 *ap = p.Ap + ((z0 + h) * 2 * kRowsT) * P;
+        __nv_bfloat16 *ap = p.Ap + ((z0 + h) * 2 * p.g.rt) * P;
         *reinterpret_cast<uint4 *>(ap + static_cast<long long>(u) * P + jb) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
-        *reinterpret_cast<uint4 *>(ap + static_cast<long long>(kRowsT + u) * P + jb) =
+        *reinterpret_cast<uint4 *>(ap + static_cast<long long>(p.g.rt + u) * P + jb) =
             make_uint4(lo[0], lo[1], lo[2], lo[3]);
       }
       if (p.hp == 2) {
@@ -832,14 +838,16 @@ __global__ void __launch_bounds__(kThreadsB) bwd_post_softmax_kernel(StripArgs p
 int scores_smem(int ch) { return 2 * ch * kStagedRows * kTilePitch * 4; }
 int adjoint_smem() { return 2 * 2 * kStagedRows * kTilePitch * 4; }
 
-// Rows of a block.  Without the convolution after the softmax: own rows NO = 256 -
-// 2 (c_q - 1), C / dC rows NO + c_q - 1.  With it, one more halo of c_q - 1 rows
-// on each side: own rows 256 - 3 (c_q - 1), A rows (and dA'' rows) NO + 2 (c_q - 1).
+// Rows of a block (R = block_rows(L)).  Without the convolution after the softmax:
+// own rows NO = R - 2 (c_q - 1), C / dC rows NO + c_q - 1.  With it, one more halo
+// of c_q - 1 rows on each side: own rows R - 3 (c_q - 1), A rows (and dA'' rows)
+// NO + 2 (c_q - 1).
 Geo geometry(const BwdArgs &a) {
   Geo g;
   g.halo = a.cq - 1;
   g.c = a.ck / 2;
-  g.no = kRowsT - (a.kqp ? 3 : 2) * g.halo;
+  g.rt = block_rows(a.L);
+  g.no = g.rt - (a.kqp ? 3 : 2) * g.halo;
   g.rc = g.no + (a.kqp ? 2 : 1) * g.halo;
   g.pitch = (a.L + 63) / 64 * 64;
   return g;
@@ -883,10 +891,10 @@ bool attn_bwd_tc_supported(const BwdArgs &a) {
 
 size_t attn_bwd_tc_workspace_bytes(int B, int H, int L, int cq, int hp, int kqp) {
   const size_t Z = static_cast<size_t>(B) * H, P = (static_cast<size_t>(L) + 63) / 64 * 64;
-  const size_t halo = static_cast<size_t>(cq - 1);
-  const size_t no = kRowsT - (kqp ? 3 : 2) * halo, rc = no + (kqp ? 2 : 1) * halo;
-  size_t b = up256(Z * kRowsT * P * 4) + 2 * up256(Z * rc * P * 4) + (hp == 1 ? up256(Z * rc * P * 4) : 0) +
-             2 * up256(Z * 2 * kRowsT * P * 2);
+  const size_t halo = static_cast<size_t>(cq - 1), RT = static_cast<size_t>(block_rows(L));
+  const size_t no = RT - (kqp ? 3 : 2) * halo, rc = no + (kqp ? 2 : 1) * halo;
+  size_t b = up256(Z * RT * P * 4) + 2 * up256(Z * rc * P * 4) + (hp == 1 ? up256(Z * rc * P * 4) : 0) +
+             2 * up256(Z * 2 * RT * P * 2);
   // with the convolution after the softmax: its output gradient G, dA (then dC) and A'
   if (kqp) b += up256(Z * rc * P * 4) + up256(Z * (no + halo) * P * 4) + up256(Z * no * P * 4);
   return b;
@@ -898,7 +906,7 @@ cudaError_t launch_attn_bwd_tc(const BwdArgs &a, void *ws) {
   const int post = a.kqp ? 1 : 0, ndc = g.no + g.halo;  // rows of dA / dC with post
   char *w = static_cast<char *>(ws);
   float *S = reinterpret_cast<float *>(w);
-  w += up256(Z * kRowsT * P * 4);
+  w += up256(Z * g.rt * P * 4);
   float *A = reinterpret_cast<float *>(w);
   w += up256(Z * g.rc * P * 4);
   float *D = reinterpret_cast<float *>(w);
@@ -909,9 +917,9 @@ cudaError_t launch_attn_bwd_tc(const BwdArgs &a, void *ws) {
     w += up256(Z * g.rc * P * 4);
   }
   __nv_bfloat16 *dS = reinterpret_cast<__nv_bfloat16 *>(w);
-  w += up256(Z * 2 * kRowsT * P * 2);
+  w += up256(Z * 2 * g.rt * P * 2);
   __nv_bfloat16 *Ap = reinterpret_cast<__nv_bfloat16 *>(w);
-  w += up256(Z * 2 * kRowsT * P * 2);
+  w += up256(Z * 2 * g.rt * P * 2);
   float *Gp = nullptr, *dAp = nullptr, *Ac = nullptr;
   if (post) {
     Gp = reinterpret_cast<float *>(w);
@@ -942,11 +950,11 @@ cudaError_t launch_attn_bwd_tc(const BwdArgs &a, void *ws) {
   if (a.hp && a.dw && (e = cudaMemsetAsync(a.dw, 0, static_cast<size_t>(a.H) * a.ch * 4, st)) != cudaSuccess)
     return e;
   // A'' is written for the own rows up to each row's query only: the rest stays zero
-  if ((e = cudaMemsetAsync(Ap, 0, Z * 2 * kRowsT * P * 2, st)) != cudaSuccess) return e;
+  if ((e = cudaMemsetAsync(Ap, 0, Z * 2 * g.rt * P * 2, st)) != cudaSuccess) return e;
 
   const BgTensor tq = qkv_tensor(a.q, a, a.rs), tk = qkv_tensor(a.k, a, a.rs), tv = qkv_tensor(a.v, a, a.rs);
   const BgTensor tdo = qkv_tensor(a.dout, a, static_cast<long long>(a.H) * a.d);
-  const BgTensor tdS = strip_tensor(dS, a, 2 * kRowsT, g.pitch), tAp = strip_tensor(Ap, a, 2 * kRowsT, g.pitch);
+  const BgTensor tdS = strip_tensor(dS, a, 2 * g.rt, g.pitch), tAp = strip_tensor(Ap, a, 2 * g.rt, g.pitch);
   const long long HD = static_cast<long long>(a.H) * a.d, LHD = HD * a.L;
   const int ch = a.hp ? a.ch : 1, G = a.H / ch;
   unsigned *err = a.err;
@@ -972,11 +980,11 @@ cudaError_t launch_attn_bwd_tc(const BwdArgs &a, void *ws) {
     // keys 0 .. W-1: up to the last row of the block's maps
     const int W = std::min(a.L, r0 + g.rc), Wp = (W + 63) / 64 * 64;
     sp.r0 = r0; sp.W = W; sp.Wp = Wp;
-    // 1. S strip = s Q K^T: rows r0 - s_lead .. r0 - s_lead + 255, keys 0 .. W-1
+    // 1. S strip = s Q K^T: rows r0 - s_lead .. r0 - s_lead + R - 1, keys 0 .. W-1
     BgArgs ga = {};
     ga.Z = static_cast<int>(Z); ga.H = a.H; ga.err = err;
-    ga.M = kRowsT; ga.N = W; ga.K = a.d; ga.alpha = a.scale; ga.accumulate = 0;
-    ga.C = S; ga.sm = g.pitch; ga.sh = static_cast<long long>(kRowsT) * g.pitch; ga.sb = ga.sh * a.H;
+    ga.M = g.rt; ga.N = W; ga.K = a.d; ga.alpha = a.scale; ga.accumulate = 0;
+    ga.C = S; ga.sm = g.pitch; ga.sh = static_cast<long long>(g.rt) * g.pitch; ga.sb = ga.sh * a.H;
     ga.a = K_major(2, r0 - s_lead, 0); ga.b = K_major(2, 0, 0);
     if ((e = launch_gemm_batched(tq, tk, ga, st)) != cudaSuccess) return e;
     // 2. dA'' strip = dO V^T: rows r0 .. r0 + rc - 1
@@ -994,7 +1002,7 @@ cudaError_t launch_attn_bwd_tc(const BwdArgs &a, void *ws) {
     else
       bwd_scores_kernel<6, 11, 1><<<grid_g, kThreadsB, scores_smem(1), st>>>(s3);
     if ((e = check()) != cudaSuccess) return e;
-    const dim3 grid_h(kRowsT / kRows, static_cast<unsigned>(Z));
+    const dim3 grid_h(g.rt / kRows, static_cast<unsigned>(Z));
     if (post) {
       // 3a. the gradient at the post-softmax convolution's output, G = Mask_0(mix back dA'')
       if (ch == 2)
@@ -1026,29 +1034,29 @@ cudaError_t launch_attn_bwd_tc(const BwdArgs &a, void *ws) {
     // 4. dS (hi / lo), dtheta: the adjoint of the convolution before the softmax
     AdjArgs q0 = {};
     q0.G = post ? dAp : D; q0.g_rows = post ? ndc : g.rc;
-    q0.X = S; q0.x_rows = kRowsT; q0.x_base = r0 - s_lead;
+    q0.X = S; q0.x_rows = g.rt; q0.x_base = r0 - s_lead;
     q0.theta = a.theta; q0.dtheta = a.dtheta; q0.dS = dS;
     bwd_adjoint_kernel<6, 11, 0><<<grid_h, kThreadsB, adjoint_smem(), st>>>(sp, q0);
     if ((e = check()) != cudaSuccess) return e;
     // 5. dQ rows r0 .. r0 + no - 1 = s dS K: K runs over the keys twice, the hi
-    //    rows of dS against K, then its lo rows (256 further) against K again
+    //    rows of dS against K, then its lo rows (R further) against K again
     const int own = std::min(g.no, a.L - r0);
     BgArgs gq = {};
     gq.Z = static_cast<int>(Z); gq.H = a.H; gq.err = err;
     // (added into the zeroed dq: the GEMM may split K in two)
     gq.M = own; gq.N = a.d; gq.K = 2 * Wp; gq.alpha = a.scale; gq.accumulate = 1; gq.split_ok = 1;
     gq.C = a.dq + static_cast<long long>(r0) * HD; gq.sm = HD; gq.sh = a.d; gq.sb = LHD;
-    gq.a = periodic(K_major(1, 0, 0), Wp, kRowsT);
+    gq.a = periodic(K_major(1, 0, 0), Wp, g.rt);
     gq.b = periodic(MN_major(2, 0, 0), Wp, 0);
     if ((e = launch_gemm_batched(tdS, tk, gq, st)) != cudaSuccess) return e;
     //    dK += s dS^T Q and dV += A''^T dO over the block's rows (keys 0 .. W-1): K runs
     //    over the rows of the hi and lo halves, the block's query rows twice
     BgArgs gk = {};
     gk.Z = static_cast<int>(Z); gk.H = a.H; gk.err = err;
-    gk.M = W; gk.N = a.d; gk.K = 2 * kRowsT; gk.accumulate = 1;
+    gk.M = W; gk.N = a.d; gk.K = 2 * g.rt; gk.accumulate = 1;
     gk.sm = HD; gk.sh = a.d; gk.sb = LHD;
     gk.a = MN_major(1, 0, 0);
-    gk.b = periodic(MN_major(2, 0, r0), kRowsT, 0);
+    gk.b = periodic(MN_major(2, 0, r0), g.rt, 0);
     gk.alpha = a.scale; gk.C = a.dk;
     if ((e = launch_gemm_batched(tdS, tq, gk, st)) != cudaSuccess) return e;
     gk.alpha = 1.f; gk.C = a.dv;
