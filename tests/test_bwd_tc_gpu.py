@@ -127,6 +127,15 @@ def test_bwd_tc_full_length_one_group():
     check(wl, inp, dout)
 
 
+def test_bwd_tc_taller_blocks_one_group():
+    """Past L = 3072 the blocks are 512 rows tall (502 own rows): L = 3100, six full
+    blocks and an 88-row tail, one head group, against the oracle's full backward."""
+    wl = synth.shrink(synth.WORKLOADS["pretrain_d128_L2048"], B=1, H=2, L=3100, seed=956)
+    inp = synth.make_attn_inputs(wl)
+    dout = synth.round_bf16(synth.normal(wl.seed, 20, (wl.B, wl.L, wl.H, wl.d)))
+    check(wl, inp, dout)
+
+
 def test_bwd_tc_d96_full_length_one_group():
     """The pages' 880M shape (d = 96: 1536 over 16 heads) at L = 2048, one head group:
     the operands' 96 channels are read as two 64-channel TMA boxes, the second half
